@@ -1,0 +1,234 @@
+"""fp64 CPU oracle for S²-Attn (shifted sparse attention), forward and backward.
+
+TEST INFRASTRUCTURE. This module exists to check the CUDA path. Only the test suite,
+the smoke check and the bench's CPU-baseline leg may import or run it; the library
+never calls it and has no CPU fallback.
+
+Source: "LongLoRA: Efficient Fine-tuning of Long-Context Large Language Models",
+paper-graph summary page, §3.4 "S2-Attn: Shifted Sparse Attention as a Training-Time
+Proxy for Full Attention", Algorithm 1 (key line 1, standard self-attention, key line 2)
+and the three-step description (split heads, shift one chunk, recombine).
+
+The forward is the algorithm written out literally, in the pages' notation:
+  1. split the H heads into two chunks; roll the second chunk by -G/2 along N
+     (``np.roll``, i.e. torch.roll semantics: rolled[r] = x[(r + G/2) mod N]);
+  2. view the sequence as B*N/G independent groups of G tokens;
+  3. run standard causal self-attention softmax(scale * q k^T) v inside each group;
+  4. reshape back to [B, N, H, d] and roll the second chunk back by +G/2.
+The backward differentiates those four steps directly: per group
+dP = dO V^T, dS = P o (dP - rowsum(P o dP)), dQ = scale dS K, dK = scale dS^T Q,
+dV = P^T dO; the derivative of a roll is the opposite roll and the derivative of the
+shared K/V view (grouped-query heads) is a sum over the query heads that share it.
+
+Readings where the page is silent (each also listed in the design notes):
+  * scale: the page writes softmax(q k^T); the caller's ``scale`` multiplies q k^T.
+  * causal mask: applied in rolled order within each group, so in the shifted heads the
+    wrap group (last G/2 tokens followed by the first G/2) lets the first G/2 tokens see
+    the last G/2 ones (the page's §3.4 "Information leakage considerations" accepts it).
+  * LSE: natural log of the row sum of exp(scale * q k^T) over the allowed keys, stored
+    per original token as [B, Hq, N].
+  * grouped-query heads: query head h reads key/value head h // (Hq / Hkv); the shift of
+    query head h is applied to that shared view.
+  * ``shift_head_begin`` (default Hq/2, the page's chunk(2)) and ``shift`` (default G/2)
+    generalise the split point and the roll amount for the ablation patterns; the roll
+    is always rolled[r] = x[(r + shift) mod N].
+
+Everything is float64; inputs are the bf16 values widened exactly.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "chunk_roll",
+    "expand_kv",
+    "causal_self_attn",
+    "causal_self_attn_backward",
+    "s2attn_forward",
+    "s2attn_backward",
+    "rolled_token_index",
+    "head_group_rows",
+]
+
+
+def chunk_roll(x: np.ndarray, amount: int, shift_head_begin: int) -> np.ndarray:
+    """Roll heads [shift_head_begin, H) of x [B, N, H, ...] by ``amount`` along N.
+
+    Key line 1 of Algorithm 1 is chunk_roll(qkv, -G/2, H/2); key line 2 is
+    chunk_roll(out, +G/2, H/2). np.roll has torch.roll's semantics:
+    np.roll(x, a)[r] = x[(r - a) mod N].
+    """
+    out = x.copy()
+    out[:, :, shift_head_begin:] = np.roll(x[:, :, shift_head_begin:], amount, axis=1)
+    return out
+
+
+def expand_kv(x: np.ndarray, Hq: int) -> np.ndarray:
+    """Per-query-head view of grouped key/value heads: head h reads kv head h // (Hq/Hkv)."""
+    rep = Hq // x.shape[2]
+    return np.repeat(x, rep, axis=2)
+
+
+def _group_probs(q: np.ndarray, k: np.ndarray, scale: float):
+    """Causal softmax of scale * q k^T for one group and head; q, k are [G, d].
+
+    Returns (P, lse) with P [G, G] (zero above the diagonal) and lse [G].
+    """
+    G = q.shape[0]
+    s = scale * (q @ k.T)
+    s = np.where(np.tril(np.ones((G, G), dtype=bool)), s, -np.inf)
+    m = s.max(axis=1, keepdims=True)
+    e = np.exp(s - m)
+    l = e.sum(axis=1, keepdims=True)
+    return e / l, (m + np.log(l))[:, 0]
+
+
+def causal_self_attn(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float):
+    """Standard causal self-attention on every batch element: q, k, v [Bg, G, H, d].
+
+    This is the ``self_attn(qkv)`` call of Algorithm 1 after the view into groups.
+    Returns o [Bg, G, H, d] and lse [Bg, G, H].
+    """
+    Bg, G, H, d = q.shape
+    o = np.empty((Bg, G, H, v.shape[3]))
+    lse = np.empty((Bg, G, H))
+    for b in range(Bg):
+        for h in range(H):
+            p, lse[b, :, h] = _group_probs(q[b, :, h], k[b, :, h], scale)
+            o[b, :, h] = p @ v[b, :, h]
+    return o, lse
+
+
+def causal_self_attn_backward(q, k, v, do, scale):
+    """Gradients of causal_self_attn for upstream do [Bg, G, H, d] (direct differentiation).
+
+    Returns dq, dk, dv, each [Bg, G, H, d]; dk and dv are per query head (not yet summed
+    over heads that share a kv head).
+    """
+    Bg, G, H, d = q.shape
+    dq = np.empty_like(q)
+    dk = np.empty_like(k)
+    dv = np.empty_like(v)
+    for b in range(Bg):
+        for h in range(H):
+            p, _ = _group_probs(q[b, :, h], k[b, :, h], scale)
+            dp = do[b, :, h] @ v[b, :, h].T
+            ds = p * (dp - (p * dp).sum(axis=1, keepdims=True))
+            dq[b, :, h] = scale * (ds @ k[b, :, h])
+            dk[b, :, h] = scale * (ds.T @ q[b, :, h])
+            dv[b, :, h] = p.T @ do[b, :, h]
+    return dq, dk, dv
+
+
+def _defaults(Hq, G, shift_head_begin, shift):
+    if shift_head_begin is None:
+        shift_head_begin = Hq // 2
+    if shift is None:
+        shift = G // 2
+    return shift_head_begin, shift
+
+
+def s2attn_forward(q, k, v, G, scale, shift_head_begin=None, shift=None):
+    """S²-Attn forward. q [B,N,Hq,d], k, v [B,N,Hkv,d] float64.
+
+    Returns o [B,N,Hq,d] and lse [B,Hq,N], both in original token order.
+    """
+    B, N, Hq, d = q.shape
+    if N % G != 0:
+        raise ValueError("the view into groups needs G to divide N")
+    shb, shift = _defaults(Hq, G, shift_head_begin, shift)
+    ke, ve = expand_kv(k, Hq), expand_kv(v, Hq)
+    # Key line 1: roll the second chunk of heads by -shift, then view as groups.
+    qr = chunk_roll(q, -shift, shb).reshape(B * N // G, G, Hq, d)
+    kr = chunk_roll(ke, -shift, shb).reshape(B * N // G, G, Hq, d)
+    vr = chunk_roll(ve, -shift, shb).reshape(B * N // G, G, Hq, v.shape[3])
+    o, lse = causal_self_attn(qr, kr, vr, scale)
+    # Key line 2: back to [B, N, H, d], roll the second chunk back by +shift.
+    o = chunk_roll(o.reshape(B, N, Hq, v.shape[3]), shift, shb)
+    lse = chunk_roll(lse.reshape(B, N, Hq), shift, shb)
+    return o, np.ascontiguousarray(lse.transpose(0, 2, 1))
+
+
+def s2attn_backward(q, k, v, do, G, scale, shift_head_begin=None, shift=None):
+    """Gradients of s2attn_forward's o with respect to q, k, v for upstream do [B,N,Hq,d].
+
+    Returns dq [B,N,Hq,d], dk [B,N,Hkv,d], dv [B,N,Hkv,d] in original token order.
+    """
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    shb, shift = _defaults(Hq, G, shift_head_begin, shift)
+    ke, ve = expand_kv(k, Hq), expand_kv(v, Hq)
+    qr = chunk_roll(q, -shift, shb).reshape(B * N // G, G, Hq, d)
+    kr = chunk_roll(ke, -shift, shb).reshape(B * N // G, G, Hq, d)
+    vr = chunk_roll(ve, -shift, shb).reshape(B * N // G, G, Hq, d)
+    dor = chunk_roll(do, -shift, shb).reshape(B * N // G, G, Hq, d)
+    dq, dk, dv = causal_self_attn_backward(qr, kr, vr, dor, scale)
+    # The derivative of a roll is the opposite roll ...
+    dq = chunk_roll(dq.reshape(B, N, Hq, d), shift, shb)
+    dk = chunk_roll(dk.reshape(B, N, Hq, d), shift, shb)
+    dv = chunk_roll(dv.reshape(B, N, Hq, d), shift, shb)
+    # ... and that of the shared K/V view is the sum over the query heads sharing it.
+    rep = Hq // Hkv
+    dk = dk.reshape(B, N, Hkv, rep, d).sum(axis=3)
+    dv = dv.reshape(B, N, Hkv, rep, d).sum(axis=3)
+    return dq, dk, dv
+
+
+def rolled_token_index(N: int, G: int, shift: int) -> np.ndarray:
+    """Original token of every (group, in-group row) of a shifted head, as [N/G, G].
+
+    Obtained by applying key line 1 to the token index itself: np.roll(arange(N), -shift).
+    """
+    return np.roll(np.arange(N), -shift).reshape(N // G, G)
+
+
+def head_group_rows(qh, kh, vh, doh, G, scale, shift, g, q_rows, kv_rows=None):
+    """The S²-Attn definition for one (batch, query head) restricted to group g.
+
+    qh, doh [N, d] and kh, vh [N, d] are that query head's sequences (kh, vh being the
+    kv head it reads) in original order; ``shift`` is the head's roll (0 when unshifted).
+    ``q_rows`` are in-group rows i (rolled order) whose o, lse and dq are wanted;
+    ``kv_rows`` are in-group rows j whose dk, dv contributions from this head are wanted.
+
+    Each requested row is the definition evaluated at that row: row i attends to rows
+    0..i of its group, and the gradient of kv row j gathers rows i >= j (rows i < j have
+    P[i, j] = 0 under the causal mask). Rows are given back with their original tokens.
+    Returns a dict with 'q_tok', 'o', 'lse', 'dq' and, if kv_rows, 'kv_tok', 'dk', 'dv'.
+    """
+    N = qh.shape[0]
+    tok = rolled_token_index(N, G, shift)[g]
+    q_g = np.roll(qh, -shift, axis=0).reshape(N // G, G, -1)[g]
+    k_g = np.roll(kh, -shift, axis=0).reshape(N // G, G, -1)[g]
+    v_g = np.roll(vh, -shift, axis=0).reshape(N // G, G, -1)[g]
+    do_g = np.roll(doh, -shift, axis=0).reshape(N // G, G, -1)[g]
+
+    def rows_softmax(rows):
+        s = scale * (q_g[rows] @ k_g.T)
+        allowed = np.arange(G)[None, :] <= np.asarray(rows)[:, None]
+        s = np.where(allowed, s, -np.inf)
+        m = s.max(axis=1, keepdims=True)
+        e = np.exp(s - m)
+        l = e.sum(axis=1, keepdims=True)
+        return e / l, (m + np.log(l))[:, 0]
+
+    def rows_ds(rows, p):
+        dp = do_g[rows] @ v_g.T
+        return p * (dp - (p * dp).sum(axis=1, keepdims=True))
+
+    q_rows = np.asarray(q_rows)
+    p, lse = rows_softmax(q_rows)
+    out = {
+        "q_tok": tok[q_rows],
+        "o": p @ v_g,
+        "lse": lse,
+        "dq": scale * (rows_ds(q_rows, p) @ k_g),
+    }
+    if kv_rows is not None:
+        kv_rows = np.asarray(kv_rows)
+        rows = np.arange(int(kv_rows.min()), G)
+        p2, _ = rows_softmax(rows)
+        ds2 = rows_ds(rows, p2)
+        out["kv_tok"] = tok[kv_rows]
+        out["dv"] = p2[:, kv_rows].T @ do_g[rows]
+        out["dk"] = scale * (ds2[:, kv_rows].T @ q_g[rows])
+    return out
