@@ -1,0 +1,414 @@
+"""Throughput of S²-Attn forward + backward on B200 (TFLOP/s, fraction of dense-BF16 peak).
+
+One step = one pass of the whole hot path over one batch: forward (O, LSE), backward
+preprocess (D), dK/dV and dQ kernels, all through the C ABI. FLOPs are algorithmic:
+7 * B * Hq * N * G * d per fwd+bwd (causal half of each G x G group; fwd 2, bwd 5).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--workload NAME]
+
+N > 1 runs under torchrun, one process per GPU, each on its own batch of the same workload
+(weak scaling, no data-path collective); timing is the max over ranks of device time.
+`--impl reference` times the fp64 CPU oracle (the reference arm) on a bounded sample.
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from shifted_sparse_attention_fwd_b200.inputs import METRIC_WORKLOAD, WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "S²-Attn fwd+bwd TFLOP/s (N=8192,G=2048,bf16); % of B200 dense BF16 peak"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+def fwd_bwd_flops(w) -> float:
+    return 7.0 * w.B * w.Hq * w.N * w.G * w.d
+
+
+def kernel_flops(w):
+    unit = float(w.B) * w.Hq * w.N * w.G * w.d   # one causal in-group GEMM over all heads
+    return {"s2_fwd": 2 * unit, "s2_bwd_dkdv": 4 * unit, "s2_bwd_dq": 1 * unit}
+
+
+def pre_bytes(w) -> float:
+    # O and dO read once (bf16), LSE read, D and LSE*log2(e) written (fp32)
+    return 2.0 * (2 * w.B * w.N * w.Hq * w.d) + 3.0 * 4 * w.B * w.Hq * w.N
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------------------------------
+# Clock sampling during the timed region (NVML).
+# ------------------------------------------------------------------------------------------
+REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    def __init__(self, device_index: int, period_s: float = 0.02):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: report that, never guess
+            self.nv, self.err = None, str(e)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                mask = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in REASON_BITS.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def summary(self):
+        if self.nv is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": self.err}
+        med = statistics.median(self.samples) if self.samples else None
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons - {"gpu_idle"}),
+                "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------------------------------
+# CPU baseline: the oracle as it stands, on a bounded sample of the workload.
+# ------------------------------------------------------------------------------------------
+def oracle_sample(w, target_s: float = 12.0):
+    """Time the fp64 oracle's fwd+bwd over whole heads of the workload (all groups of each),
+    alternating unrolled and rolled heads, until about target_s seconds have passed."""
+    import numpy as np
+    from oracle import s2attn_oracle as orc
+    from shifted_sparse_attention_fwd_b200.inputs import to_f64
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:
+        cores = os.cpu_count() or 1
+    q, k, v, do = make_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, w.seed)
+    rep = w.Hq // w.Hkv
+    order = []
+    for i in range(w.Hq // 2):   # 0, Hq/2, 1, Hq/2+1, ...
+        order += [i, w.Hq // 2 + i]
+    done, elapsed = 0, 0.0
+    for h in order:
+        kvh = h // rep
+        sl = lambda x, j: to_f64(x[:, :, j:j + 1])  # noqa: E731
+        shb = 0 if h >= w.Hq // 2 else 1
+        qh, kh, vh, doh = sl(q, h), sl(k, kvh), sl(v, kvh), sl(do, h)
+        t0 = time.perf_counter()
+        orc.s2attn_forward(qh, kh, vh, w.G, w.scale, shift_head_begin=shb)
+        orc.s2attn_backward(qh, kh, vh, doh, w.G, w.scale, shift_head_begin=shb)
+        elapsed += time.perf_counter() - t0
+        done += 1
+        if elapsed >= target_s:
+            break
+    flops = 7.0 * w.B * done * w.N * w.G * w.d
+    return {"value": flops / elapsed / 1e12, "unit": UNIT, "cores": int(cores), "kind": "oracle",
+            "sample": f"{done} of {w.Hq} heads (all {w.N // w.G} groups, B={w.B}) fwd+bwd, "
+                      f"{elapsed:.1f} s, numpy fp64", "seconds": round(elapsed, 2)}
+
+
+# ------------------------------------------------------------------------------------------
+# GPU arm
+# ------------------------------------------------------------------------------------------
+def run_gpu(args, rank, world, local_rank):
+    import shifted_sparse_attention_fwd_b200 as s2
+    dist = torch.distributed if world > 1 else None
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = WORKLOADS[args.workload]
+    stream = torch.cuda.current_stream()
+
+    # Each rank: its own batch of the workload (weak scaling).
+    q, k, v, do = make_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, w.seed + 7919 * rank)
+    qd, kd, vd, dod = (x.to(dev) for x in (q, k, v, do))
+    o = torch.empty_like(qd)
+    lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
+    ws = torch.empty(s2.s2attn_bwd_workspace_size(w.B, w.Hq, w.N), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step(ev=None):
+        if ev: ev[0].record(stream)
+        s2.s2attn_fwd(qd, kd, vd, o, lse, w.G, w.scale)
+        if ev: ev[1].record(stream)
+        s2.s2attn_bwd_preprocess(o, lse, dod, ws)
+        if ev: ev[2].record(stream)
+        s2.s2attn_bwd_dkdv(qd, kd, vd, dod, dk, dv, w.G, ws, w.scale)
+        if ev: ev[3].record(stream)
+        s2.s2attn_bwd_dq(qd, kd, vd, dod, dq, w.G, ws, w.scale)
+        if ev: ev[4].record(stream)
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+    st, code = s2.s2attn_get_device_error()
+    if st != s2.S2ATTN_OK:
+        raise RuntimeError(f"device error {st} code {code:#x} during warm-up")
+
+    # Timed region: K steps, L2 flushed (untimed) before each, per-kernel CUDA events.
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    if dist: dist.barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(dev.index)
+    with sampler:
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            step(evs[i])
+        torch.cuda.synchronize()
+    if dist: dist.barrier()
+    st, code = s2.s2attn_get_device_error()
+    if st != s2.S2ATTN_OK:
+        raise RuntimeError(f"device error {st} code {code:#x} in the timed region")
+    names = ["s2_fwd", "s2_bwd_pre", "s2_bwd_dkdv", "s2_bwd_dq"]
+    per_k = {n: [e[j].elapsed_time(e[j + 1]) for e in evs] for j, n in enumerate(names)}
+    step_ms = [e[0].elapsed_time(e[4]) for e in evs]
+    total_ms = sum(step_ms)
+
+    # End to end through the public API with host buffers: pinned H2D of the step's inputs,
+    # fwd + bwd, D2H of the step's results, all inside the timed region.
+    hq_, hk_, hv_, hdo_ = (x.pin_memory() for x in (q, k, v, do))
+    ho, hdq = torch.empty_like(hq_).pin_memory(), torch.empty_like(hq_).pin_memory()
+    hdk, hdv = torch.empty_like(hk_).pin_memory(), torch.empty_like(hv_).pin_memory()
+    hlse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        for dst, src in ((qd, hq_), (kd, hk_), (vd, hv_), (dod, hdo_)):
+            dst.copy_(src, non_blocking=True)
+        step()
+        for dst, src in ((ho, o), (hlse, lse), (hdq, dq), (hdk, dk), (hdv, dv)):
+            dst.copy_(src, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    if dist: dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    h2d = sum(x.numel() * x.element_size() for x in (hq_, hk_, hv_, hdo_))
+    d2h = sum(x.numel() * x.element_size() for x in (ho, hlse, hdq, hdk, hdv))
+
+    if dist:
+        t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms, e2e_ms = float(t[0]), float(t[1])
+    if rank != 0:
+        return None
+
+    flops_step = fwd_bwd_flops(w)
+    value = world * flops_step * args.steps / (total_ms * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    peak_tf = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    avg = {n: sum(v_) / len(v_) for n, v_ in per_k.items()}
+    kflops = kernel_flops(w)
+    dominant = max(avg, key=avg.get)
+    traffic = load_traffic(dominant, args.workload)
+    if dominant in kflops:
+        achieved = kflops[dominant] / (avg[dominant] * 1e-3) / 1e12
+        roof = {"bound": "tensor", "kernel": dominant, "achieved": round(achieved, 1),
+                "peak": peak_tf, "unit": "TFLOP/s", "frac": round(achieved / peak_tf, 4),
+                "traffic": traffic, "peak_source": f"{peak_src} (burst bf16)",
+                "algorithmic_per_launch": kflops[dominant]}
+    else:
+        hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        achieved = pre_bytes(w) / (avg[dominant] * 1e-3) / 1e9
+        roof = {"bound": "hbm", "kernel": dominant, "achieved": round(achieved, 1), "peak": hbm,
+                "unit": "GB/s", "frac": round(achieved / hbm, 4), "traffic": traffic,
+                "peak_source": peak_src}
+    kern = {}
+    for n in names:
+        entry = {"ms": round(avg[n], 4)}
+        if n in kflops:
+            tf = kflops[n] / (avg[n] * 1e-3) / 1e12
+            entry.update(tflops_algorithmic=round(tf, 1), frac=round(tf / peak_tf, 4))
+        else:
+            gbs = pre_bytes(w) / (avg[n] * 1e-3) / 1e9
+            entry.update(gbs=round(gbs, 1))
+        kern[n] = entry
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16 Q/K/V/dO, Llama2-7B attention layer shape)",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "G": w.G,
+                   "d": w.d, "shift_heads": f"{w.Hq // 2}-{w.Hq - 1}", "batch_per_gpu": w.B,
+                   "l2": f"flushed before every step ({L2_FLUSH_BYTES >> 20} MiB write, untimed)",
+                   "parallelism": f"{world} independent replicas (weak scaling)"},
+        "pct_of_peak": round(100 * value / peak_tf, 2),
+        "peak": {"bf16_tflops": peak_tf, "source": peak_src},
+        "kernels": kern,
+        "roofline": roof,
+        "e2e": {"value": round(world * flops_step * e2e_steps / (e2e_ms * 1e-3) / 1e12, 2),
+                "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": e2e_steps, "ms_per_step": round(e2e_ms / e2e_steps, 4)},
+        "clocks": sampler.summary(),
+        "gpu_launches": 4 * args.steps,
+    }
+    return line
+
+
+def load_traffic(kernel, workload):
+    """DRAM bytes per launch for `kernel` from the committed ncu summary, if it is current."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+        e = t.get(workload, {}).get(kernel)
+        return None if e is None else e.get("bytes_per_launch")
+    except (OSError, ValueError):
+        return None
+
+
+# ------------------------------------------------------------------------------------------
+# Reference arm: the CPU oracle, as it stands.
+# ------------------------------------------------------------------------------------------
+def oracle_group_step(w, units, q, k, v, do):
+    """One reference step: the oracle's row-restricted evaluation of whole (head, group)
+    units (every row of the group, o/lse/dq and dk/dv), cycling over heads and groups."""
+    from oracle import s2attn_oracle as orc
+    from shifted_sparse_attention_fwd_b200.inputs import to_f64
+    rep = w.Hq // w.Hkv
+    t0 = time.perf_counter()
+    for (b, h, g) in units:
+        shift = w.G // 2 if h >= w.Hq // 2 else 0
+        rows = list(range(w.G))
+        orc.head_group_rows(to_f64(q[b, :, h]), to_f64(k[b, :, h // rep]), to_f64(v[b, :, h // rep]),
+                            to_f64(do[b, :, h]), w.G, w.scale, shift, g, rows, kv_rows=rows)
+    dt = time.perf_counter() - t0
+    return 7.0 * len(units) * w.G * w.G * w.d / dt / 1e12, dt
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return None
+    w = WORKLOADS[args.workload]
+    q, k, v, do = make_inputs(w.B, w.Hq, w.Hkv, w.N, w.d, w.seed)
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:
+        cores = os.cpu_count() or 1
+    ng = w.N // w.G
+    seq = [(b, h, g) for b in range(w.B) for g in range(ng)
+           for i in range(w.Hq // 2) for h in (i, w.Hq // 2 + i)]
+    pos = 0
+
+    def next_unit():
+        nonlocal pos
+        u = seq[pos % len(seq)]
+        pos += 1
+        return [u]
+
+    for _ in range(args.warmup):
+        oracle_group_step(w, next_unit(), q, k, v, do)
+    vals, secs = [], 0.0
+    for _ in range(args.steps):
+        tf, dt = oracle_group_step(w, next_unit(), q, k, v, do)
+        vals.append(tf)
+        secs += dt
+    value = statistics.mean(vals)
+    cb = {"value": round(value, 6), "unit": UNIT, "cores": int(cores), "kind": "oracle",
+          "sample": f"each step: one (batch, head, group) unit of G={w.G} rows, fwd+bwd, all "
+                    f"rows; heads alternate unrolled/rolled; {secs:.1f} s over {args.steps} steps"}
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT,
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "ms_per_step": round(1e3 * secs / max(1, args.steps), 3),
+            "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N,
+                       "G": w.G, "d": w.d},
+            "cpu_baseline": cb,
+            "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="s2attn", choices=["s2attn", "reference"])
+    ap.add_argument("--workload", default=METRIC_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+
+    if args.impl == "reference":
+        line = run_reference(args, rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_gpu(args, rank, world, local_rank)
+        if line is not None:
+            if not args.no_cpu_baseline and world == 1:
+                line["cpu_baseline"] = oracle_sample(WORKLOADS[args.workload])
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,164 @@
+/*
+ * s2attn.h — C ABI of the sm_100a S²-Attn (shifted sparse attention) library.
+ *
+ * The operation is LongLoRA's S²-Attn ("LongLoRA: Efficient Fine-tuning of Long-Context
+ * Large Language Models", paper-graph summary page, §3.4 "S2-Attn: Shifted Sparse
+ * Attention as a Training-Time Proxy for Full Attention", Algorithm 1):
+ *   1. split the Hq query heads into two chunks; in the second chunk (heads
+ *      [Hq/2, Hq)) roll every sequence by -G/2 along the token axis, with wrap-around
+ *      (key line 1, torch.roll semantics: rolled[r] = x[(r + G/2) mod N]);
+ *   2. view the N tokens as N/G independent groups of G consecutive (rolled) tokens;
+ *   3. inside each group apply standard causal self-attention
+ *      o = softmax(scale * q k^T) v, the causal mask taken in rolled order;
+ *   4. roll the second chunk's output back by +G/2 (key line 2).
+ * The backward is the gradient of those steps (the page uses S²-Attn only during
+ * fine-tuning, §3.2, so gradients flow through it).
+ * Grouped-query heads: query head h reads key/value head h / (Hq / Hkv); its roll is
+ * applied to that shared key/value view.
+ *
+ * Layouts (all row-major, contiguous, every token axis in ORIGINAL order):
+ *   q, o, dO, dq : bf16 [B, N, Hq,  d]
+ *   k, v, dk, dv : bf16 [B, N, Hkv, d]
+ *   lse          : fp32 [B, Hq, N]   natural-log row log-sum-exp of scale * q k^T over
+ *                                    the keys the row attends to
+ * Pointers are device pointers (the caller's CUDA device must be current), 16-byte
+ * aligned. `stream` is a cudaStream_t (NULL = legacy default stream).
+ *
+ * Ownership and behaviour: the caller owns every buffer. The library allocates no memory,
+ * keeps no per-call state, never synchronises the stream (except
+ * s2attn_get_device_error), and launches asynchronously on `stream`. Outputs are
+ * overwritten, never accumulated.
+ *
+ * Errors: arguments are validated on the host before any launch;
+ *   S2ATTN_ERR_INVALID_ARG  null / misaligned pointer, a size <= 0, Hq % Hkv != 0,
+ *                           N % G != 0, odd G, odd Hq (default split), scale not a
+ *                           positive finite number, shift_head_begin outside [0, Hq],
+ *                           workspace too small;
+ *   S2ATTN_ERR_UNSUPPORTED  d not in {64, 128}; G or the roll not a multiple of 8 tokens
+ *                           (for the default roll G/2: G % 16 != 0); N >= 2^30;
+ *   S2ATTN_ERR_CUDA         a CUDA call or a launch failed (see s2attn_last_error);
+ *   S2ATTN_ERR_TIMEOUT      reported by s2attn_get_device_error: a kernel's pipeline wait
+ *                           exceeded its limit; the kernel stopped early and returned
+ *                           (its outputs are undefined), the context stays usable.
+ */
+#ifndef S2ATTN_H_
+#define S2ATTN_H_
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define S2ATTN_API __attribute__((visibility("default")))
+#else
+#define S2ATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  S2ATTN_OK = 0,
+  S2ATTN_ERR_INVALID_ARG = 1,
+  S2ATTN_ERR_UNSUPPORTED = 2,
+  S2ATTN_ERR_CUDA = 3,
+  S2ATTN_ERR_TIMEOUT = 4
+} s2attn_status;
+
+/* Version of this ABI (bumped on any signature change). */
+S2ATTN_API int s2attn_abi_version(void);
+
+/* Static description of a status code. */
+S2ATTN_API const char* s2attn_status_string(int status);
+
+/* Text of the last CUDA error seen by the calling host thread ("" if none). */
+S2ATTN_API const char* s2attn_last_error(void);
+
+/*
+ * Forward: o and lse from q, k, v (Algorithm 1, key line 1 -> self_attn -> key line 2).
+ * Heads [Hq/2, Hq) are rolled by G/2. scale multiplies q k^T (1/sqrt(d) for Llama2).
+ */
+S2ATTN_API s2attn_status s2attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                         int B, int Hq, int Hkv, int N, int d, int G, float scale,
+                         void* stream);
+
+/*
+ * Forward with the head split and the roll made explicit: heads
+ * [shift_head_begin, Hq) are rolled so that rolled[r] = x[(r + shift) mod N].
+ * s2attn_fwd == s2attn_fwd_ex(..., Hq/2, G/2, ...). shift_head_begin = Hq gives plain
+ * grouped causal attention (the page's "short attention", Pattern 1 only); 0 rolls every
+ * head (Pattern 2 only); shift = N - G/2 is the page's "shift up" variant (Table 8);
+ * G = N with shift_head_begin = Hq is full causal attention. shift may be any integer; it
+ * is taken mod N and must then be a multiple of 8.
+ */
+S2ATTN_API s2attn_status s2attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse,
+                            int B, int Hq, int Hkv, int N, int d, int G, float scale,
+                            int shift_head_begin, int shift, void* stream);
+
+/* Bytes of device workspace s2attn_bwd needs: two fp32 [B, Hq, N] arrays (D and LSE in
+ * base 2), each rounded up to 256 bytes. */
+S2ATTN_API size_t s2attn_bwd_workspace_size(int B, int Hq, int N);
+
+/*
+ * Backward: dq, dk, dv from q, k, v, the forward's o and lse, and the upstream dO.
+ * Runs, in order on `stream`: the preprocess D = rowsum(dO o O), the dK/dV kernel and the
+ * dQ kernel. `workspace` (device, 256-byte aligned, >= s2attn_bwd_workspace_size bytes)
+ * is scratch owned by the caller; its contents on entry do not matter.
+ * dk and dv are the sums over the query heads sharing each kv head.
+ */
+S2ATTN_API s2attn_status s2attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                         const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                         int B, int Hq, int Hkv, int N, int d, int G, float scale,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/* Backward with explicit head split and roll (same meaning as s2attn_fwd_ex). */
+S2ATTN_API s2attn_status s2attn_bwd_ex(const void* q, const void* k, const void* v, const void* o,
+                            const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                            int B, int Hq, int Hkv, int N, int d, int G, float scale,
+                            int shift_head_begin, int shift, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
+/*
+ * The three stages of s2attn_bwd, callable one at a time (same arguments; the workspace
+ * must carry the preprocess results into the two gradient stages):
+ *   s2attn_bwd_preprocess  workspace <- D = rowsum(dO o O) and LSE * log2(e)
+ *   s2attn_bwd_dkdv        dk, dv    <- from q, k, v, dO and the workspace
+ *   s2attn_bwd_dq          dq        <- from q, k, v, dO and the workspace
+ * Arguments a stage does not use may be NULL.
+ */
+S2ATTN_API s2attn_status s2attn_bwd_preprocess(const void* o, const float* lse, const void* dO,
+                                    int B, int Hq, int N, int d, void* workspace,
+                                    size_t workspace_bytes, void* stream);
+S2ATTN_API s2attn_status s2attn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO,
+                              void* dk, void* dv, int B, int Hq, int Hkv, int N, int d, int G,
+                              float scale, int shift_head_begin, int shift,
+                              const void* workspace, size_t workspace_bytes, void* stream);
+S2ATTN_API s2attn_status s2attn_bwd_dq(const void* q, const void* k, const void* v, const void* dO,
+                            void* dq, int B, int Hq, int Hkv, int N, int d, int G, float scale,
+                            int shift_head_begin, int shift, const void* workspace,
+                            size_t workspace_bytes, void* stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the current device's error word.
+ * Returns S2ATTN_ERR_TIMEOUT if a kernel gave up on a pipeline wait since the last call
+ * (code_out, if not NULL, receives (kernel << 8) | wait site; 0 if none), S2ATTN_ERR_CUDA
+ * if the synchronisation failed, S2ATTN_OK otherwise.
+ */
+S2ATTN_API s2attn_status s2attn_get_device_error(void* stream, unsigned int* code_out);
+
+/* Limit on every pipeline wait inside the kernels, in nanoseconds (default 1e9). Applies
+ * to launches made after the call, from any thread. 0 restores the default. */
+S2ATTN_API void s2attn_set_wait_timeout_ns(unsigned long long ns);
+
+/*
+ * Failure-detection self test: launches one CTA that waits, with the same bounded wait the
+ * attention kernels use, on a barrier nothing ever arrives on. After `timeout_ns` the wait
+ * gives up and records an error, so the following s2attn_get_device_error returns
+ * S2ATTN_ERR_TIMEOUT. No fault, trap or hang is involved.
+ */
+S2ATTN_API s2attn_status s2attn_selftest_wait_timeout(unsigned long long timeout_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* S2ATTN_H_ */

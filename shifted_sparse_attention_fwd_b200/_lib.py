@@ -1,0 +1,208 @@
+"""ctypes binding of libs2attn.so (the C ABI declared in include/s2attn.h).
+
+Argument marshalling only: every step of S²-Attn runs in the library's CUDA kernels.
+Functions carry the C names; tensors are torch CUDA tensors (device memory and streams are
+torch's), passed as raw pointers. There is no CPU fallback: if the library cannot be
+loaded, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libs2attn.so")
+
+S2ATTN_OK = 0
+S2ATTN_ERR_INVALID_ARG = 1
+S2ATTN_ERR_UNSUPPORTED = 2
+S2ATTN_ERR_CUDA = 3
+S2ATTN_ERR_TIMEOUT = 4
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_F = ctypes.c_float
+_Z = ctypes.c_size_t
+
+# name -> (restype, argtypes); mirrors include/s2attn.h
+SIGNATURES = {
+    "s2attn_abi_version": (_I, []),
+    "s2attn_status_string": (ctypes.c_char_p, [_I]),
+    "s2attn_last_error": (ctypes.c_char_p, []),
+    "s2attn_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
+    "s2attn_fwd_ex": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
+    "s2attn_bwd_workspace_size": (_Z, [_I, _I, _I]),
+    "s2attn_bwd": (_I, [_P] * 9 + [_I] * 6 + [_F, _P, _Z, _P]),
+    "s2attn_bwd_ex": (_I, [_P] * 9 + [_I] * 6 + [_F, _I, _I, _P, _Z, _P]),
+    "s2attn_bwd_preprocess": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _Z, _P]),
+    "s2attn_bwd_dkdv": (_I, [_P] * 6 + [_I] * 6 + [_F, _I, _I, _P, _Z, _P]),
+    "s2attn_bwd_dq": (_I, [_P] * 5 + [_I] * 6 + [_F, _I, _I, _P, _Z, _P]),
+    "s2attn_get_device_error": (_I, [_P, ctypes.POINTER(ctypes.c_uint)]),
+    "s2attn_set_wait_timeout_ns": (None, [ctypes.c_ulonglong]),
+    "s2attn_selftest_wait_timeout": (_I, [ctypes.c_ulonglong, _P]),
+}
+
+_lib = None
+
+
+class S2AttnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = f"{where}: {status_string(status)}"
+        if status == S2ATTN_ERR_CUDA:
+            msg += f" ({lib().s2attn_last_error().decode()})"
+        super().__init__(msg)
+
+
+def lib():
+    """Load libs2attn.so once; raise if it is missing (no fallback exists)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with "
+                "`python -m shifted_sparse_attention_fwd_b200.build` (nvcc, sm_100a)")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().s2attn_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str):
+    if status != S2ATTN_OK:
+        raise S2AttnError(status, where)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        return t  # raw integer address
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _dims(q, k, G):
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    return B, Hq, Hkv, N, d, G
+
+
+def _check_bf16(*ts):
+    for t in ts:
+        if t is not None and isinstance(t, torch.Tensor) and t.dtype != torch.bfloat16:
+            raise ValueError(f"expected bf16, got {t.dtype}")
+
+
+def s2attn_fwd(q, k, v, o, lse, G, scale=None, shift_head_begin=None, shift=None, stream=None):
+    """O and LSE of S²-Attn. q [B,N,Hq,d], k/v [B,N,Hkv,d] bf16; o like q; lse fp32 [B,Hq,N]."""
+    _check_bf16(q, k, v, o)
+    B, Hq, Hkv, N, d, G = _dims(q, k, G)
+    scale = d ** -0.5 if scale is None else scale
+    shb = Hq // 2 if shift_head_begin is None else shift_head_begin
+    sh = G // 2 if shift is None else shift
+    _check(lib().s2attn_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, N, d,
+                               G, scale, shb, sh, _stream(stream)), "s2attn_fwd")
+
+
+def s2attn_bwd_workspace_size(B, Hq, N) -> int:
+    return int(lib().s2attn_bwd_workspace_size(B, Hq, N))
+
+
+def s2attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, G, scale=None, shift_head_begin=None,
+               shift=None, workspace=None, stream=None):
+    """dQ, dK, dV of S²-Attn (overwritten). workspace: a uint8 CUDA tensor, or None to let
+    torch allocate one of s2attn_bwd_workspace_size bytes."""
+    _check_bf16(q, k, v, o, dO, dq, dk, dv)
+    B, Hq, Hkv, N, d, G = _dims(q, k, G)
+    scale = d ** -0.5 if scale is None else scale
+    shb = Hq // 2 if shift_head_begin is None else shift_head_begin
+    sh = G // 2 if shift is None else shift
+    ws_bytes = s2attn_bwd_workspace_size(B, Hq, N)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    _check(lib().s2attn_bwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO),
+                               _ptr(dq), _ptr(dk), _ptr(dv), B, Hq, Hkv, N, d, G, scale, shb, sh,
+                               _ptr(workspace), workspace.numel(), _stream(stream)),
+           "s2attn_bwd")
+
+
+def s2attn_bwd_preprocess(o, lse, dO, workspace, stream=None):
+    B, N, Hq, d = o.shape
+    _check(lib().s2attn_bwd_preprocess(_ptr(o), _ptr(lse), _ptr(dO), B, Hq, N, d,
+                                       _ptr(workspace), workspace.numel(), _stream(stream)),
+           "s2attn_bwd_preprocess")
+
+
+def s2attn_bwd_dkdv(q, k, v, dO, dk, dv, G, workspace, scale=None, shift_head_begin=None,
+                    shift=None, stream=None):
+    B, Hq, Hkv, N, d, G = _dims(q, k, G)
+    scale = d ** -0.5 if scale is None else scale
+    shb = Hq // 2 if shift_head_begin is None else shift_head_begin
+    sh = G // 2 if shift is None else shift
+    _check(lib().s2attn_bwd_dkdv(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(dk), _ptr(dv), B, Hq,
+                                 Hkv, N, d, G, scale, shb, sh, _ptr(workspace), workspace.numel(),
+                                 _stream(stream)), "s2attn_bwd_dkdv")
+
+
+def s2attn_bwd_dq(q, k, v, dO, dq, G, workspace, scale=None, shift_head_begin=None, shift=None,
+                  stream=None):
+    B, Hq, Hkv, N, d, G = _dims(q, k, G)
+    scale = d ** -0.5 if scale is None else scale
+    shb = Hq // 2 if shift_head_begin is None else shift_head_begin
+    sh = G // 2 if shift is None else shift
+    _check(lib().s2attn_bwd_dq(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(dq), B, Hq, Hkv, N, d,
+                               G, scale, shb, sh, _ptr(workspace), workspace.numel(),
+                               _stream(stream)), "s2attn_bwd_dq")
+
+
+def s2attn_get_device_error(stream=None):
+    """(status, code): S2ATTN_ERR_TIMEOUT with a nonzero code if a kernel gave up a wait."""
+    code = ctypes.c_uint(0)
+    st = lib().s2attn_get_device_error(_stream(stream), ctypes.byref(code))
+    return int(st), int(code.value)
+
+
+def s2attn_set_wait_timeout_ns(ns: int):
+    lib().s2attn_set_wait_timeout_ns(int(ns))
+
+
+def s2attn_selftest_wait_timeout(timeout_ns: int, stream=None):
+    _check(lib().s2attn_selftest_wait_timeout(int(timeout_ns), _stream(stream)),
+           "s2attn_selftest_wait_timeout")
+
+
+# ------------------------------------------------------------------------------------------
+# Allocating conveniences (torch provides the memory; the library does the work).
+# ------------------------------------------------------------------------------------------
+def fwd(q, k, v, G, scale=None, shift_head_begin=None, shift=None, stream=None):
+    o = torch.empty_like(q)
+    lse = torch.empty((q.shape[0], q.shape[2], q.shape[1]), dtype=torch.float32, device=q.device)
+    s2attn_fwd(q, k, v, o, lse, G, scale, shift_head_begin, shift, stream)
+    return o, lse
+
+
+def bwd(q, k, v, o, lse, dO, G, scale=None, shift_head_begin=None, shift=None, stream=None):
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    s2attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, G, scale, shift_head_begin, shift, None, stream)
+    return dq, dk, dv

@@ -1,0 +1,308 @@
+// S²-Attn backward, dK and dV, on sm_100a tensor cores.
+//
+// Gradient of the per-group causal self-attention of LongLoRA's Algorithm 1 (summary page
+// §3.4), taken through the roll: a key/value row t of kv head j receives, from every query
+// head h that reads it (grouped-query heads h with h / (Hq/Hkv) == j), the contributions of
+// the query rows that follow it in h's rolled order inside the same group:
+//   P^T  = exp(scale * K Q^T - LSE)             (recomputed, per column = query row)
+//   dV  += P^T dO
+//   dP^T = V dO^T
+//   dS^T = P^T o (dP^T - D)
+//   dK  += scale * dS^T Q
+// One CTA owns 128 ORIGINAL key/value rows of one (batch, kv head), so the tile is shared
+// by all its query heads whatever their roll, and dK/dV are written once, without atomics.
+// For each query head the rows map to at most two runs of rolled rows; the query tiles
+// visited are those covering [rolled row, end of its group) for every row of the tile.
+//
+// Warp roles (192 threads): warps 0-3 elementwise (thread i owns kv row i = TMEM lane i),
+// warp 4 TMA producer (K, V once; Q, dO, LSE2, D per query tile, 2 stages), warp 5 TMEM
+// allocator + MMA issuer. TMEM: S^T/P^T [0,128), dP^T/dS^T [128,256), dV [256,256+D),
+// dK [256+D, 256+2D).
+#pragma once
+
+#include "s2_common.cuh"
+
+namespace s2 {
+
+struct BwdParams {
+  const float* lse2;   // [B, Hq, N]  LSE * log2(e)
+  const float* dvec;   // [B, Hq, N]  D = rowsum(dO o O)
+  __nv_bfloat16* dq;
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+  int B, Hq, Hkv, N, G, shift_head_begin, shift;
+  float scale_log2;   // scale * log2(e)
+  float scale;
+  unsigned int* err;
+  unsigned long long timeout_ns;
+};
+
+template <int D>
+struct DkdvLayout {
+  static constexpr uint32_t kTile = Tile<D>::kBytes;
+  static constexpr uint32_t kK = 0;
+  static constexpr uint32_t kV = kK + kTile;
+  static constexpr uint32_t kQ = kV + kTile;          // 2 stages
+  static constexpr uint32_t kDO = kQ + 2 * kTile;     // 2 stages
+  static constexpr uint32_t kLse = kDO + 2 * kTile;   // 2 stages x 128 floats
+  static constexpr uint32_t kDv = kLse + 1024;        // 2 stages x 128 floats
+  static constexpr uint32_t kBar = kDv + 1024;
+  enum { B_KV = 0, B_QF = 1, B_QE = 3, B_S = 5, B_DP = 6, B_P = 7, B_DS = 8, B_ACC = 9,
+         B_DRAIN = 10, B_COUNT = 11 };
+  static constexpr uint32_t kTmemSlot = kBar + B_COUNT * 8;
+  static constexpr uint32_t kAbort = kTmemSlot + 4;
+  static constexpr uint32_t kBytes = kAbort + 4;
+  static constexpr uint32_t kLaunchBytes =
+      (kBytes + 1024 > 116 * 1024) ? kBytes + 1024 : 116 * 1024;
+};
+
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+    s2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQ8,
+                       const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmK8,
+                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmV8,
+                       const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmO8,
+                       const BwdParams p) {
+  using L = DkdvLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = aligned_smem(smem_raw);
+  const uint32_t sbase = smem_u32(smem);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  auto bar = [&](int i) { return sbase + L::kBar + 8u * i; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kTmemSlot);
+  const WaitCtx ctx{abort_flag, p.err, p.timeout_ns, KID_DKDV};
+
+  int b, kvh, t0;
+  kv_tile_coords(blockIdx.x, p.B, p.Hq, p.Hkv, p.N, p.G, p.shift_head_begin, p.shift, b, kvh, t0);
+  const int rep = p.Hq / p.Hkv;
+  const int h_begin = kvh * rep;
+  auto head_shift = [&](int hq) { return hq >= p.shift_head_begin ? p.shift : 0; };
+
+  if (warp == 4 && lane == 0) {
+    mbar_init(bar(L::B_KV), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(L::B_QF + s), 1);
+      mbar_init(bar(L::B_QE + s), 1);
+    }
+    mbar_init(bar(L::B_S), 1);
+    mbar_init(bar(L::B_DP), 1);
+    mbar_init(bar(L::B_P), 128);
+    mbar_init(bar(L::B_DS), 128);
+    mbar_init(bar(L::B_ACC), 1);
+    mbar_init(bar(L::B_DRAIN), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_map(&tmQ);
+    tma_prefetch_map(&tmK);
+    tma_prefetch_map(&tmV);
+    tma_prefetch_map(&tmO);
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tm_s = tmem, tm_dp = tmem + 128, tm_dv = tmem + 256, tm_dk = tmem + 256 + D;
+
+  if (warp == 4) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      int last_parity[2] = {-1, -1};
+      mbar_expect_tx(bar(L::B_KV), 2 * L::kTile);
+      const TileRuns kv_runs = rolled_tile_runs(t0, 0, p.N);
+      load_tile<D>(sbase + L::kK, &tmK, &tmK8, bar(L::B_KV), b, kvh, kv_runs, p.N);
+      load_tile<D>(sbase + L::kV, &tmV, &tmV8, bar(L::B_KV), b, kvh, kv_runs, p.N);
+      int n = 0;
+      bool ok = true;
+      for (int hq = h_begin; ok && hq < h_begin + rep; ++hq) {
+        const int sh = head_shift(hq);
+        const QTileRanges qr = kv_tile_qtiles(t0, sh, p.N, p.G);
+        const float* lse_row = p.lse2 + (static_cast<size_t>(b) * p.Hq + hq) * p.N;
+        const float* d_row = p.dvec + (static_cast<size_t>(b) * p.Hq + hq) * p.N;
+        for (int i = 0; i < qr.count(); ++i, ++n) {
+          const int st = n & 1;
+          if (n >= 2 && !wait_bar(bar(L::B_QE + st), ((n >> 1) - 1) & 1, ctx, 1)) { ok = false; break; }
+          const TileRuns tr = rolled_tile_runs(qr.at(i) * kTileRows, sh, p.N);
+          const uint32_t fb = bar(L::B_QF + st);
+          mbar_expect_tx(fb, 2 * L::kTile + 8u * tr.valid);
+          load_tile<D>(sbase + L::kQ + st * L::kTile, &tmQ, &tmQ8, fb, b, hq, tr, p.N);
+          load_tile<D>(sbase + L::kDO + st * L::kTile, &tmO, &tmO8, fb, b, hq, tr, p.N);
+          const uint32_t sl = sbase + L::kLse + st * 512, sd = sbase + L::kDv + st * 512;
+          bulk_load(sl, lse_row + tr.start, 4u * tr.first, fb);
+          bulk_load(sd, d_row + tr.start, 4u * tr.first, fb);
+          if (tr.valid > tr.first) {
+            bulk_load(sl + 4u * tr.first, lse_row, 4u * (tr.valid - tr.first), fb);
+            bulk_load(sd + 4u * tr.first, d_row, 4u * (tr.valid - tr.first), fb);
+          }
+          last_parity[st] = (n >> 1) & 1;
+        }
+      }
+      drain_wait(bar(L::B_KV), 0, p.timeout_ns);
+      for (int s = 0; s < 2; ++s)
+        if (last_parity[s] >= 0) drain_wait(bar(L::B_QF + s), last_parity[s], p.timeout_ns);
+    }
+  } else if (warp == 5) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16(128, 128, false, false);  // K Q^T, V dO^T
+      constexpr uint32_t idesc_acc = idesc_bf16(128, D, false, true);   // P^T dO, dS^T Q
+      int total = 0;
+      for (int hq = h_begin; hq < h_begin + rep; ++hq)
+        total += kv_tile_qtiles(t0, head_shift(hq), p.N, p.G).count();
+      auto issue_nt = [&](uint32_t d_tmem, uint32_t a_base, uint32_t b_base) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * Tile<D>::kHalfBytes + (kk % 4) * 32;
+          mma_ss(d_tmem, sdesc_sw128(a_base + off, 16, 1024), sdesc_sw128(b_base + off, 16, 1024),
+                 idesc_s, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_acc = [&](uint32_t d_tmem, uint32_t a_tmem, uint32_t b_base, int n) {
+#pragma unroll
+        for (int kk = 0; kk < kTileRows / 16; ++kk)
+          mma_ts(d_tmem, a_tmem + kk * 8, sdesc_sw128(b_base + kk * 2048, Tile<D>::kHalfBytes, 1024),
+                 idesc_acc, (n > 0 || kk > 0) ? 1u : 0u);
+      };
+      bool ok = wait_bar(bar(L::B_KV), 0, ctx, 2);
+      if (ok && total > 0) ok = wait_bar(bar(L::B_QF + 0), 0, ctx, 3);
+      if (ok && total > 0) {
+        tc_fence_after();
+        issue_nt(tm_s, sbase + L::kK, sbase + L::kQ);
+        mma_commit(bar(L::B_S));
+      }
+      for (int n = 0; ok && n < total; ++n) {
+        const int st = n & 1;
+        const uint32_t q_s = sbase + L::kQ + st * L::kTile, do_s = sbase + L::kDO + st * L::kTile;
+        issue_nt(tm_dp, sbase + L::kV, do_s);
+        mma_commit(bar(L::B_DP));
+        if (!wait_bar(bar(L::B_P), n & 1, ctx, 4)) { ok = false; break; }
+        tc_fence_after();
+        issue_acc(tm_dv, tm_s, do_s, n);
+        if (n + 1 < total) {
+          const int st1 = (n + 1) & 1;
+          if (!wait_bar(bar(L::B_QF + st1), ((n + 1) >> 1) & 1, ctx, 5)) { ok = false; break; }
+          tc_fence_after();
+          issue_nt(tm_s, sbase + L::kK, sbase + L::kQ + st1 * L::kTile);
+          mma_commit(bar(L::B_S));
+        }
+        if (!wait_bar(bar(L::B_DS), n & 1, ctx, 6)) { ok = false; break; }
+        tc_fence_after();
+        issue_acc(tm_dk, tm_dp, q_s, n);
+        mma_commit(bar(L::B_QE + st));
+      }
+      if (ok) mma_commit(bar(L::B_ACC));
+    }
+  } else {
+    // ---------------- elementwise warps 0-3 ----------------
+    const int row = threadIdx.x;
+    const int t = t0 + row;
+    const bool kv_valid = t < p.N;
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const float c = p.scale_log2;
+    const float* s_lse = reinterpret_cast<const float*>(smem + L::kLse);
+    const float* s_dv = reinterpret_cast<const float*>(smem + L::kDv);
+    int n = 0;
+    bool ok = true;
+    for (int hq = h_begin; ok && hq < h_begin + rep; ++hq) {
+      const int sh = head_shift(hq);
+      const QTileRanges qr = kv_tile_qtiles(t0, sh, p.N, p.G);
+      const int r_k = kv_valid ? (t - sh < 0 ? t - sh + p.N : t - sh) : 0;
+      const int ge_k = group_end(r_k, p.G);
+      for (int i = 0; i < qr.count(); ++i, ++n) {
+        const int st = n & 1;
+        const int q0 = qr.at(i) * kTileRows;
+        const int cl = kv_valid ? r_k - q0 : 1;
+        const int ch = kv_valid ? ge_k - 1 - q0 : 0;
+        if (!warp_wait(bar(L::B_QF + st), (n >> 1) & 1, ctx, 7)) { ok = false; break; }
+        if (!warp_wait(bar(L::B_S), n & 1, ctx, 8)) { ok = false; break; }
+        tc_fence_after();
+        const float* lse_t = s_lse + st * 128;
+        const float* d_t = s_dv + st * 128;
+        float pv[128];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint32_t rr[32];
+          tmem_ld32(t_lane + 32 * j, rr);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int col = 32 * j + e;
+            const float x = fast_exp2(fmaf(__uint_as_float(rr[e]), c, -lse_t[col]));
+            pv[col] = (col >= cl && col <= ch) ? x : 0.f;
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(pv[32 * j + 2 * e], pv[32 * j + 2 * e + 1]);
+          tmem_st16(t_lane + 16 * j, pk);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar(L::B_P));
+        if (!warp_wait(bar(L::B_DP), n & 1, ctx, 9)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint32_t rr[32];
+          tmem_ld32(t_lane + 128 + 32 * j, rr);
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int col = 32 * j + 2 * e;
+            const float d0 = pv[col] * (__uint_as_float(rr[2 * e]) - d_t[col]);
+            const float d1 = pv[col + 1] * (__uint_as_float(rr[2 * e + 1]) - d_t[col + 1]);
+            pk[e] = pack_bf16(d0, d1);
+          }
+          tmem_st16(t_lane + 128 + 16 * j, pk);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar(L::B_DS));
+      }
+    }
+    if (ok && warp_wait(bar(L::B_ACC), 0, ctx, 10)) {
+      tc_fence_after();
+      const size_t orow = ((static_cast<size_t>(b) * p.N + (kv_valid ? t : 0)) * p.Hkv + kvh) * D;
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t src = which == 0 ? tm_dv : tm_dk;
+        const float mul = which == 0 ? 1.f : p.scale;
+        __nv_bfloat16* dst_row = (which == 0 ? p.dv : p.dk) + orow;
+#pragma unroll
+        for (int j = 0; j < D / 32; ++j) {
+          uint32_t rr[32];
+          tmem_ld32(src + (static_cast<uint32_t>(warp * 32) << 16) + 32 * j, rr);
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pk[e] = pack_bf16(__uint_as_float(rr[2 * e]) * mul, __uint_as_float(rr[2 * e + 1]) * mul);
+          if (kv_valid) {
+            uint4* dst = reinterpret_cast<uint4*>(dst_row + 32 * j);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    if (lane == 0) {
+      mma_commit(bar(L::B_DRAIN));
+      drain_wait(bar(L::B_DRAIN), 0, p.timeout_ns);
+    }
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace s2

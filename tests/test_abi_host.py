@@ -1,0 +1,232 @@
+"""CPU-side checks of the C ABI and of the host/index logic (no kernel is launched).
+
+* libs2attn.so loads and exports every function include/s2attn.h declares;
+* argument validation rejects bad calls before any CUDA call (fake device addresses);
+* the remap and tile-order functions the kernels use (s2_tiles.cuh), compiled here with g++,
+  agree with the oracle's literal roll (LongLoRA summary page, §3.4 Algorithm 1 key line 1)
+  and with a brute-force enumeration of which query rows see which key rows.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+from oracle import s2attn_oracle as orc
+import shifted_sparse_attention_fwd_b200 as s2
+from shifted_sparse_attention_fwd_b200 import build as s2build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "s2attn.h")
+CSRC = os.path.join(ROOT, "shifted_sparse_attention_fwd_b200", "csrc")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    s2build.build()
+    return s2.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(s2attn_\w+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert len(names) >= 14
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(s2.SIGNATURES), set(names) ^ set(s2.SIGNATURES)
+    out = subprocess.run(["nm", "-D", "--defined-only", s2.LIB_PATH], capture_output=True,
+                         text=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    assert set(names) <= exported
+    # Nothing else leaks out of the library (hidden visibility by default).
+    assert {e for e in exported if e.startswith("s2attn_")} == set(names)
+
+
+def test_version_and_status_strings(lib):
+    assert lib.s2attn_abi_version() == 1
+    for st in range(5):
+        assert s2.status_string(st)
+    assert s2.status_string(99) == "unknown status"
+    assert lib.s2attn_bwd_workspace_size(1, 32, 8192) == 2 * 32 * 8192 * 4
+    assert lib.s2attn_bwd_workspace_size(1, 1, 8) == 2 * 256
+    assert lib.s2attn_bwd_workspace_size(0, 1, 8) == 0
+
+
+A = 0x10000  # fake, 16-byte aligned device addresses: validation must reject before use
+
+
+def fwd_call(lib, **kw):
+    a = dict(q=A, k=A, v=A, o=A, lse=A, B=1, Hq=4, Hkv=4, N=256, d=64, G=64, scale=0.125)
+    a.update(kw)
+    return lib.s2attn_fwd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["Hq"], a["Hkv"],
+                          a["N"], a["d"], a["G"], a["scale"], None)
+
+
+def fwd_ex_call(lib, shb, shift, **kw):
+    a = dict(B=1, Hq=4, Hkv=4, N=256, d=64, G=64, scale=0.125)
+    a.update(kw)
+    return lib.s2attn_fwd_ex(A, A, A, A, A, a["B"], a["Hq"], a["Hkv"], a["N"], a["d"], a["G"],
+                             a["scale"], shb, shift, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), 1), (dict(lse=None), 1), (dict(k=A + 8), 1), (dict(o=A + 2), 1),
+    (dict(B=0), 1), (dict(N=-8), 1), (dict(Hq=3, Hkv=3), 1), (dict(Hkv=3), 1),
+    (dict(N=200), 1), (dict(G=63, N=63 * 4), 1), (dict(scale=0.0), 1),
+    (dict(scale=float("nan")), 1), (dict(scale=float("inf")), 1), (dict(scale=-1.0), 1),
+    (dict(d=96), 2), (dict(d=256), 2), (dict(G=24, N=240), 2), (dict(G=8, N=64), 2),
+    (dict(N=1 << 30, G=1 << 29), 2),
+])
+def test_fwd_rejects(lib, kw, status):
+    assert fwd_call(lib, **kw) == status
+
+
+@pytest.mark.parametrize("shb,shift,kw,status", [
+    (-1, 32, {}, 1), (5, 32, {}, 1), (2, 4, {}, 2), (2, 36, {}, 2),
+    # G=24: G/2 = 12 is not a multiple of 8, but a roll of 8 (or none) is fine -> reaches
+    # CUDA set-up, which is not available here; we only check it is not rejected as bad shape
+])
+def test_fwd_ex_rejects(lib, shb, shift, kw, status):
+    assert fwd_ex_call(lib, shb, shift, **kw) == status
+
+
+def test_bwd_rejects(lib):
+    ws = 0x100000
+    need = lib.s2attn_bwd_workspace_size(1, 4, 256)
+    args = [A] * 9 + [1, 4, 4, 256, 64, 64, ctypes.c_float(0.125)]
+    assert lib.s2attn_bwd(*args, None, need, None) == 1                  # null workspace
+    assert lib.s2attn_bwd(*args, ws + 16, need, None) == 1               # misaligned
+    assert lib.s2attn_bwd(*args, ws, need - 4, None) == 1                # too small
+    bad = [A] * 8 + [None] + [1, 4, 4, 256, 64, 64, ctypes.c_float(0.125)]
+    assert lib.s2attn_bwd(*bad, ws, need, None) == 1                     # null dv
+    odd = [A] * 9 + [1, 3, 3, 256, 64, 64, ctypes.c_float(0.125)]
+    assert lib.s2attn_bwd(*odd, ws, need, None) == 1                     # odd Hq
+    d96 = [A] * 9 + [1, 4, 4, 256, 96, 64, ctypes.c_float(0.125)]
+    assert lib.s2attn_bwd(*d96, ws, need, None) == 2
+    assert lib.s2attn_bwd_preprocess(A, A, A, 1, 4, 256, 64, ws, 8, None) == 1
+    assert lib.s2attn_bwd_preprocess(A, A, A, 1, 4, 256, 80, ws, need, None) == 2
+    assert lib.s2attn_bwd_dq(A, A, A, A, None, 1, 4, 4, 256, 64, 64, ctypes.c_float(0.1), 2,
+                             32, ws, need, None) == 1
+    assert lib.s2attn_bwd_dkdv(A, A, A, A, A, A, 1, 4, 4, 256, 64, 64, ctypes.c_float(0.1), 2,
+                               36, ws, need, None) == 2
+
+
+# --------------------------------------------------------------------------------------
+# Index logic of the kernels, compiled for the host.
+# --------------------------------------------------------------------------------------
+SHIM = r"""
+#include "s2_tiles.cuh"
+extern "C" {
+void rolled_runs(int r0, int shift, int N, int* o) {
+  s2::TileRuns t = s2::rolled_tile_runs(r0, shift, N); o[0]=t.valid; o[1]=t.first; o[2]=t.start; }
+void original_runs(int t0, int shift, int N, int* o) {
+  s2::TileRuns t = s2::original_tile_runs(t0, shift, N); o[0]=t.valid; o[1]=t.first; o[2]=t.start; }
+int qtiles(int t0, int sh, int N, int G, int* o) {
+  s2::QTileRanges q = s2::kv_tile_qtiles(t0, sh, N, G);
+  int n = q.count(); for (int i = 0; i < n; ++i) o[i] = q.at(i); return n; }
+void qcoords(int bid, int B, int Hq, int N, int G, int* o) {
+  s2::query_tile_coords(bid, B, Hq, N, G, o[0], o[1], o[2]); }
+void kvcoords(int bid, int B, int Hq, int Hkv, int N, int G, int shb, int sh, int* o) {
+  s2::kv_tile_coords(bid, B, Hq, Hkv, N, G, shb, sh, o[0], o[1], o[2]); }
+}
+"""
+
+
+@pytest.fixture(scope="module")
+def shim(tmp_path_factory):
+    d = tmp_path_factory.mktemp("shim")
+    src = d / "shim.cpp"
+    src.write_text(SHIM)
+    so = d / "shim.so"
+    subprocess.run(["g++", "-O1", "-shared", "-fPIC", "-std=c++17", "-I", CSRC, str(src), "-o",
+                    str(so)], check=True)
+    return ctypes.CDLL(str(so))
+
+
+def call4(fn, *args):
+    out = (ctypes.c_int * 4)()
+    fn(*args, out)
+    return list(out)
+
+
+CASES = [(256, 64, 32), (8192, 2048, 1024), (320, 64, 32), (384, 192, 96), (200, 200, 0),
+         (96, 32, 16), (1024, 1024, 512), (640, 128, 64), (2048, 512, 256), (448, 64, 8),
+         (96, 96, 88), (768, 256, 640)]
+
+
+@pytest.mark.parametrize("N,G,shift", CASES)
+def test_rolled_runs_match_literal_roll(shim, N, G, shift):
+    tok = orc.rolled_token_index(N, G, shift).reshape(-1)   # rolled row -> original token
+    for r0 in range(0, N, 128):
+        valid, first, start = call4(shim.rolled_runs, r0, shift, N)[:3]
+        assert valid == min(128, N - r0)
+        got = [start + i for i in range(first)] + [i - first for i in range(first, valid)]
+        assert got == list(tok[r0:r0 + valid])
+        assert first % 8 == 0 and valid % 8 == 0 and start % 8 == 0
+
+
+@pytest.mark.parametrize("N,G,shift", CASES)
+def test_original_runs_invert_the_roll(shim, N, G, shift):
+    tok = orc.rolled_token_index(N, G, shift).reshape(-1)
+    rolled_of = np.empty(N, dtype=np.int64)
+    rolled_of[tok] = np.arange(N)
+    for t0 in range(0, N, 128):
+        valid, first, start = call4(shim.original_runs, t0, shift, N)[:3]
+        got = [start + i for i in range(first)] + [i - first for i in range(first, valid)]
+        assert got == list(rolled_of[t0:t0 + valid])
+
+
+@pytest.mark.parametrize("N,G,shift", CASES)
+def test_kv_tile_query_tiles_exact(shim, N, G, shift):
+    """Brute force: q tile Qt is visited for kv tile t0 iff some rolled query row in Qt attends
+    some kv row of the tile (same rolled group, query not before key)."""
+    tok = orc.rolled_token_index(N, G, shift).reshape(-1)
+    rolled_of = np.empty(N, dtype=np.int64)
+    rolled_of[tok] = np.arange(N)
+    out = (ctypes.c_int * 4096)()
+    for t0 in range(0, N, 128):
+        n = shim.qtiles(t0, shift, N, G, out)
+        got = list(out[:n])
+        assert len(set(got)) == len(got)
+        want = set()
+        for t in range(t0, min(t0 + 128, N)):
+            rk = rolled_of[t]
+            ge = (rk // G + 1) * G
+            want.update(range(rk // 128, (ge - 1) // 128 + 1))
+        assert set(got) == want
+
+
+@pytest.mark.parametrize("B,Hq,N,G", [(1, 4, 256, 64), (2, 3, 8192, 2048), (1, 2, 384, 192),
+                                      (3, 2, 320, 64), (1, 1, 1024, 1024)])
+def test_query_tile_order_is_a_permutation(shim, B, Hq, N, G):
+    nt = (N + 127) // 128
+    seen = set()
+    for bid in range(B * Hq * nt):
+        seen.add(tuple(call4(shim.qcoords, bid, B, Hq, N, G)[:3]))
+    assert seen == {(b, h, q) for b in range(B) for h in range(Hq) for q in range(nt)}
+    if G % 128 == 0 and G > 128:
+        # the first wave holds the tiles with the most key tiles (last tile of each group)
+        b, h, qt = call4(shim.qcoords, 0, B, Hq, N, G)[:3]
+        assert qt % (G // 128) == G // 128 - 1
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,G,shb,sh", [(1, 4, 4, 256, 64, 2, 32),
+                                                  (2, 8, 2, 8192, 2048, 4, 1024),
+                                                  (1, 8, 1, 1024, 256, 4, 128),
+                                                  (1, 4, 2, 384, 192, 2, 96),
+                                                  (1, 64, 8, 32768, 8192, 32, 4096)])
+def test_kv_tile_order_is_a_permutation(shim, B, Hq, Hkv, N, G, shb, sh):
+    nt = (N + 127) // 128
+    seen = set()
+    for bid in range(B * Hkv * nt):
+        b, kvh, t0 = call4(shim.kvcoords, bid, B, Hq, Hkv, N, G, shb, sh)[:3]
+        assert t0 % 128 == 0
+        seen.add((b, kvh, t0 // 128))
+    assert seen == {(b, k, t) for b in range(B) for k in range(Hkv) for t in range(nt)}

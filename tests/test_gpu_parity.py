@@ -1,0 +1,95 @@
+"""CUDA path vs the fp64 oracle, element by element, on seeded inputs (small and edge cases).
+
+Every call goes through the C ABI (libs2attn.so); nothing here computes attention in torch.
+"""
+import zlib
+
+import pytest
+import torch
+
+import shifted_sparse_attention_fwd_b200 as s2
+from shifted_sparse_attention_fwd_b200.inputs import WORKLOADS, make_inputs
+
+from gpu_helpers import check_case, gpu_run
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    s2.lib()
+
+
+def test_small_workload():
+    w = WORKLOADS["small_h4_n256_g64_d64"]
+    check_case(w.B, w.Hq, w.Hkv, w.N, w.G, w.d, w.seed)
+
+
+@pytest.mark.parametrize("name,B,Hq,Hkv,N,G,d,shb,shift,q_gain", [
+    # ragged tail: N is not a multiple of the 128-row tile; GQA; batch 2
+    ("ragged_gqa", 2, 4, 2, 320, 64, 64, None, None, 1.0),
+    # groups straddle tiles and the roll splits tiles (G/2 = 96)
+    ("straddle", 1, 4, 4, 384, 192, 128, None, None, 1.0),
+    # one group, no roll: full causal attention
+    ("full_causal", 1, 2, 2, 256, 256, 128, 2, 0, 1.0),
+    # MQA: one kv head read by rolled and unrolled query heads
+    ("mqa_mixed", 1, 8, 1, 512, 128, 128, None, None, 1.0),
+    # every head rolled, and rolled the other way ("shift up")
+    ("pattern2_up", 1, 4, 2, 512, 256, 64, 0, 512 - 128, 1.0),
+    # no head rolled ("short attention")
+    ("pattern1", 1, 4, 4, 512, 128, 128, 4, 0, 1.0),
+    # peaky logits stress the running-max rescale
+    ("peaky", 1, 4, 4, 1024, 256, 128, None, None, 4.0),
+    # 8 groups per tile
+    ("tiny_groups", 1, 2, 2, 256, 16, 64, None, None, 1.0),
+    # a single short tile
+    ("one_tile", 1, 2, 2, 16, 16, 128, None, None, 1.0),
+    # several full tiles per group, rolled by a whole number of tiles
+    ("aligned", 1, 2, 2, 2048, 512, 128, None, None, 1.0),
+])
+def test_edge_cases(name, B, Hq, Hkv, N, G, d, shb, shift, q_gain):
+    check_case(B, Hq, Hkv, N, G, d, seed=zlib.crc32(name.encode()) % 10000, shb=shb, shift=shift, q_gain=q_gain)
+
+
+def test_shifted_head_equals_unshifted_on_rolled_input():
+    """A rolled head equals an unrolled run on torch.roll-ed inputs, rolled back (bitwise)."""
+    B, Hq, N, G, d = 1, 2, 1024, 256, 128
+    q, k, v, do = make_inputs(B, Hq, Hq, N, d, 77)
+    scale = d ** -0.5
+    a = gpu_run(q, k, v, do, G, scale, shb=1, shift=G // 2)
+    rq, rk, rv, rdo = (torch.roll(x, -G // 2, dims=1) for x in (q, k, v, do))
+    b = gpu_run(rq, rk, rv, rdo, G, scale, shb=2, shift=0)
+    for name in ("o", "dq", "dk", "dv"):
+        back = torch.roll(b[name], G // 2, dims=1)
+        assert torch.equal(a[name][:, :, 1], back[:, :, 1]), name
+    assert torch.equal(a["lse"][:, 1], torch.roll(b["lse"], G // 2, dims=2)[:, 1])
+
+
+def test_deterministic():
+    w = WORKLOADS["small_h4_n256_g64_d64"]
+    q, k, v, do = make_inputs(w.B, w.Hq, w.Hkv, 1024, 128, 5)
+    a = gpu_run(q, k, v, do, 256, 0.1)
+    b = gpu_run(q, k, v, do, 256, 0.1)
+    for name in a:
+        assert torch.equal(a[name], b[name]), name
+
+
+def test_wait_timeout_is_reported_and_context_survives():
+    s2.s2attn_selftest_wait_timeout(50_000_000)    # 50 ms
+    st, code = s2.s2attn_get_device_error()
+    assert st == s2.S2ATTN_ERR_TIMEOUT
+    assert code == (4 << 8) | 1
+    st, code = s2.s2attn_get_device_error()
+    assert st == s2.S2ATTN_OK and code == 0
+    check_case(1, 2, 2, 256, 64, 64, seed=3, backward=False)
+
+
+def test_invalid_args_raise():
+    q = torch.zeros(1, 256, 3, 64, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(s2.S2AttnError):
+        s2.fwd(q, q, q, 64)                         # odd head count with the default split
+    q = torch.zeros(1, 256, 4, 96, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(s2.S2AttnError):
+        s2.fwd(q, q, q, 64)                         # unsupported head dim
