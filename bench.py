@@ -297,16 +297,30 @@ def run_gpu(args, rank, world, local_rank):
     return line
 
 
+def kernel_source_hash() -> str:
+    """Hash of the kernel sources; DRAM counters recorded under another hash are stale."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "shifted_sparse_attention_fwd_b200", "csrc", "*"))):
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
 def load_traffic(kernel, workload):
-    """DRAM bytes per launch for `kernel` from the committed ncu summary, if it is current."""
+    """DRAM bytes per launch of `kernel` from the committed ncu summary (profiles/traffic.json),
+    or None when there is none or the kernels changed since it was captured."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             t = json.load(f)
-        e = t.get(workload, {}).get(kernel)
-        return None if e is None else e.get("bytes_per_launch")
     except (OSError, ValueError):
         return None
+    e = t.get(workload, {}).get(kernel)
+    if e is None or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("bytes_per_launch")
 
 
 # ------------------------------------------------------------------------------------------

@@ -119,10 +119,14 @@ def s2attn_fwd(q, k, v, o, lse, G, scale=None, shift_head_begin=None, shift=None
     _check_bf16(q, k, v, o)
     B, Hq, Hkv, N, d, G = _dims(q, k, G)
     scale = d ** -0.5 if scale is None else scale
+    if shift_head_begin is None and shift is None:
+        _check(lib().s2attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, N, d,
+                                G, scale, _stream(stream)), "s2attn_fwd")
+        return
     shb = Hq // 2 if shift_head_begin is None else shift_head_begin
     sh = G // 2 if shift is None else shift
     _check(lib().s2attn_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, N, d,
-                               G, scale, shb, sh, _stream(stream)), "s2attn_fwd")
+                               G, scale, shb, sh, _stream(stream)), "s2attn_fwd_ex")
 
 
 def s2attn_bwd_workspace_size(B, Hq, N) -> int:
@@ -136,15 +140,21 @@ def s2attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, G, scale=None, shift_head_begin=
     _check_bf16(q, k, v, o, dO, dq, dk, dv)
     B, Hq, Hkv, N, d, G = _dims(q, k, G)
     scale = d ** -0.5 if scale is None else scale
-    shb = Hq // 2 if shift_head_begin is None else shift_head_begin
-    sh = G // 2 if shift is None else shift
     ws_bytes = s2attn_bwd_workspace_size(B, Hq, N)
     if workspace is None:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    if shift_head_begin is None and shift is None:
+        _check(lib().s2attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO),
+                                _ptr(dq), _ptr(dk), _ptr(dv), B, Hq, Hkv, N, d, G, scale,
+                                _ptr(workspace), workspace.numel(), _stream(stream)),
+               "s2attn_bwd")
+        return
+    shb = Hq // 2 if shift_head_begin is None else shift_head_begin
+    sh = G // 2 if shift is None else shift
     _check(lib().s2attn_bwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO),
                                _ptr(dq), _ptr(dk), _ptr(dv), B, Hq, Hkv, N, d, G, scale, shb, sh,
                                _ptr(workspace), workspace.numel(), _stream(stream)),
-           "s2attn_bwd")
+           "s2attn_bwd_ex")
 
 
 def s2attn_bwd_preprocess(o, lse, dO, workspace, stream=None):
