@@ -138,6 +138,29 @@ S2ATTN_API s2attn_status s2attn_bwd_dq(const void* q, const void* k, const void*
                             size_t workspace_bytes, void* stream);
 
 /*
+ * Backward without a caller-provided workspace, for callers that cannot allocate device
+ * memory: plugin hosts whose fixed call signature carries no scratch buffer, or code on a
+ * latency-critical path that must not call cudaMalloc (which can synchronise the device and
+ * can fail under memory pressure at an arbitrary point). The pages have no counterpart to
+ * this entry point; it exists only for such callers.
+ *
+ * Same arguments and results as s2attn_bwd, minus the workspace. The scratch (D and
+ * LSE * log2(e), 8 bytes per (batch, head, token) row) lives in a 16 MiB array compiled into
+ * the library: B * Hq * N may be at most 2,097,152, larger shapes are rejected with
+ * S2ATTN_ERR_UNSUPPORTED (message in s2attn_last_error) before anything is launched. Every
+ * device that loads the library holds that array until the process exits. The first call on
+ * a device, with that device current, looks up the array's device address; make that first
+ * call before any stream capture. Nothing is allocated, by the library or by anything it
+ * calls. All calls share the one array, so two calls whose kernels overlap on the GPU (other
+ * streams, other host threads) race on it and give wrong results: serialise them. Nothing in
+ * the array needs to start at zero: each call overwrites what it reads.
+ */
+S2ATTN_API s2attn_status s2attn_bwd_noalloc(const void* q, const void* k, const void* v,
+                                            const void* o, const float* lse, const void* dO,
+                                            void* dq, void* dk, void* dv, int B, int Hq, int Hkv,
+                                            int N, int d, int G, float scale, void* stream);
+
+/*
  * Synchronises `stream`, then reads and clears the current device's error word.
  * Returns S2ATTN_ERR_TIMEOUT if a kernel gave up on a pipeline wait since the last call
  * (code_out, if not NULL, receives (kernel << 8) | wait site; 0 if none), S2ATTN_ERR_CUDA

@@ -21,6 +21,7 @@ from ._lib import (  # noqa: F401
     s2attn_bwd_preprocess,
     s2attn_bwd_dkdv,
     s2attn_bwd_dq,
+    s2attn_bwd_noalloc,
     s2attn_get_device_error,
     s2attn_set_wait_timeout_ns,
     s2attn_selftest_wait_timeout,

@@ -39,6 +39,7 @@ SIGNATURES = {
     "s2attn_bwd_preprocess": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _Z, _P]),
     "s2attn_bwd_dkdv": (_I, [_P] * 6 + [_I] * 6 + [_F, _I, _I, _P, _Z, _P]),
     "s2attn_bwd_dq": (_I, [_P] * 5 + [_I] * 6 + [_F, _I, _I, _P, _Z, _P]),
+    "s2attn_bwd_noalloc": (_I, [_P] * 9 + [_I] * 6 + [_F, _P]),
     "s2attn_get_device_error": (_I, [_P, ctypes.POINTER(ctypes.c_uint)]),
     "s2attn_set_wait_timeout_ns": (None, [ctypes.c_ulonglong]),
     "s2attn_selftest_wait_timeout": (_I, [ctypes.c_ulonglong, _P]),
@@ -184,6 +185,18 @@ def s2attn_bwd_dq(q, k, v, dO, dq, G, workspace, scale=None, shift_head_begin=No
     _check(lib().s2attn_bwd_dq(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(dq), B, Hq, Hkv, N, d,
                                G, scale, shb, sh, _ptr(workspace), workspace.numel(),
                                _stream(stream)), "s2attn_bwd_dq")
+
+
+def s2attn_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, G, scale=None, stream=None):
+    """s2attn_bwd without a workspace argument: the library's own static scratch is used
+    (for callers that cannot allocate; see include/s2attn.h for the size limit and the rule
+    that calls must not overlap on the GPU)."""
+    _check_bf16(q, k, v, o, dO, dq, dk, dv)
+    B, Hq, Hkv, N, d, G = _dims(q, k, G)
+    scale = d ** -0.5 if scale is None else scale
+    _check(lib().s2attn_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO),
+                                    _ptr(dq), _ptr(dk), _ptr(dv), B, Hq, Hkv, N, d, G, scale,
+                                    _stream(stream)), "s2attn_bwd_noalloc")
 
 
 def s2attn_get_device_error(stream=None):

@@ -437,3 +437,62 @@ s2attn_status s2attn_selftest_wait_timeout(unsigned long long timeout_ns, void* 
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------------------------
+// Allocation-free backward: the workspace is a static device array of this file.
+// ------------------------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;   // 16 MiB: 2^21 rows of D + LSE2
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+struct NoAllocScratch {
+  std::once_flag once;
+  cudaError_t err = cudaSuccess;
+  void* ptr = nullptr;   // device address of g_noalloc_scratch on this device
+};
+NoAllocScratch g_noalloc[kMaxDevices];
+
+// Device address of the static scratch for the current device. In host code the array's name
+// only stands in for the symbol; the address the kernels need comes from the runtime, looked
+// up once per device with that device current.
+s2attn_status noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) {
+    std::snprintf(g_last_error, sizeof(g_last_error), "device ordinal %d out of range", dev);
+    return S2ATTN_ERR_CUDA;
+  }
+  NoAllocScratch& s = g_noalloc[dev];
+  std::call_once(s.once, [&] {
+    void* p = nullptr;
+    s.err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    s.ptr = p;
+  });
+  if (s.err != cudaSuccess) return cuda_fail(s.err, "cudaGetSymbolAddress(static scratch)");
+  *out = s.ptr;
+  return S2ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" s2attn_status s2attn_bwd_noalloc(const void* q, const void* k, const void* v,
+                                            const void* o, const float* lse, const void* dO,
+                                            void* dq, void* dk, void* dv, int B, int Hq, int Hkv,
+                                            int N, int d, int G, float scale, void* stream) {
+  if (B > 0 && Hq > 0 && N > 0 &&
+      2 * ws_half(B, Hq, N) > kNoAllocScratchBytes) {
+    std::snprintf(g_last_error, sizeof(g_last_error),
+                  "s2attn_bwd_noalloc: B*Hq*N = %lld rows need %zu scratch bytes; the static "
+                  "scratch holds %zu (at most 2097152 rows)",
+                  static_cast<long long>(B) * Hq * N, 2 * ws_half(B, Hq, N), kNoAllocScratchBytes);
+    return S2ATTN_ERR_UNSUPPORTED;
+  }
+  if (Hq <= 0 || Hq % 2 != 0) return S2ATTN_ERR_INVALID_ARG;
+  void* scratch = nullptr;
+  s2attn_status s = noalloc_scratch(&scratch);
+  if (s != S2ATTN_OK) return s;
+  return s2attn_bwd_ex(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, N, d, G, scale, Hq / 2, G / 2,
+                       scratch, kNoAllocScratchBytes, stream);
+}
