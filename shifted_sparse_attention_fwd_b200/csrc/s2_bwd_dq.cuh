@@ -10,7 +10,9 @@
 // tiles as the forward (group start to diagonal); dQ is written once, without atomics.
 //
 // Warp roles (192 threads): warps 0-3 elementwise (thread i owns query row i), warp 4 TMA
-// producer (Q, dO once; K/V 2-stage ring), warp 5 TMEM allocator + MMA issuer.
+// producer (Q, dO once; K through a 3-stage ring one tile ahead of V's 2-stage ring, each slot
+// released by a commit right after its last reader: dP for V, dQ for K), warp 5 TMEM
+// allocator + MMA issuer.
 // TMEM: S/dS double buffer [0,128) and [128,256); dP [256,384); dQ [384, 384+D).
 #pragma once
 
@@ -21,13 +23,14 @@ namespace s2 {
 template <int D>
 struct DqLayout {
   static constexpr uint32_t kTile = Tile<D>::kBytes;
+  static constexpr int kKStages = 3, kVStages = 2;
   static constexpr uint32_t kQ = 0;
   static constexpr uint32_t kDO = kQ + kTile;
-  static constexpr uint32_t kK = kDO + kTile;       // 2 stages
-  static constexpr uint32_t kV = kK + 2 * kTile;    // 2 stages
-  static constexpr uint32_t kBar = kV + 2 * kTile;
-  enum { B_QDO = 0, B_K = 1, B_V = 3, B_EMPTY = 5, B_S = 7, B_DP = 9, B_DS = 10, B_ACC = 12,
-         B_DRAIN = 13, B_COUNT = 14 };
+  static constexpr uint32_t kK = kDO + kTile;                 // K ring
+  static constexpr uint32_t kV = kK + kKStages * kTile;       // V ring
+  static constexpr uint32_t kBar = kV + kVStages * kTile;
+  enum { B_QDO = 0, B_K = 1, B_KE = 4, B_V = 7, B_VE = 9, B_S = 11, B_DP = 13, B_DS = 14,
+         B_ACC = 16, B_DRAIN = 17, B_COUNT = 18 };
   static constexpr uint32_t kTmemSlot = kBar + B_COUNT * 8;
   static constexpr uint32_t kAbort = kTmemSlot + 4;
   static constexpr uint32_t kBytes = kAbort + 4;
@@ -64,11 +67,14 @@ __global__ void __launch_bounds__(192, 1)
   if (warp == 4 && lane == 0) {
     mbar_init(bar(L::B_QDO), 1);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(bar(L::B_K + s), 1);
       mbar_init(bar(L::B_V + s), 1);
-      mbar_init(bar(L::B_EMPTY + s), 1);
+      mbar_init(bar(L::B_VE + s), 1);
       mbar_init(bar(L::B_S + s), 1);
       mbar_init(bar(L::B_DS + s), 128);
+    }
+    for (int s = 0; s < L::kKStages; ++s) {
+      mbar_init(bar(L::B_K + s), 1);
+      mbar_init(bar(L::B_KE + s), 1);
     }
     mbar_init(bar(L::B_DP), 1);
     mbar_init(bar(L::B_ACC), 1);
@@ -92,28 +98,43 @@ __global__ void __launch_bounds__(192, 1)
 
   if (warp == 4) {
     if (lane == 0) {
-      int last_parity[2] = {-1, -1};
       const TileRuns q_runs = rolled_tile_runs(R0, shift_h, p.N);
       mbar_expect_tx(bar(L::B_QDO), 2 * L::kTile);
       load_tile<D>(sbase + L::kQ, &tmQ, &tmQ8, bar(L::B_QDO), b, h, q_runs, p.N);
       load_tile<D>(sbase + L::kDO, &tmO, &tmO8, bar(L::B_QDO), b, h, q_runs, p.N);
-      for (int it = 0; it < n_kv; ++it) {
-        const int st = it & 1;
-        if (it >= 2 && !wait_bar(bar(L::B_EMPTY + st), ((it >> 1) - 1) & 1, ctx, 1)) break;
-        const TileRuns tr = rolled_tile_runs((kt_begin + it) * kTileRows, shift_h, p.N);
+      int k_issued = 0, v_issued = 0;
+      auto issue_k = [&]() -> bool {
+        const int i = k_issued, st = i % L::kKStages;
+        if (i >= L::kKStages &&
+            !wait_bar(bar(L::B_KE + st), ((i / L::kKStages) - 1) & 1, ctx, 1))
+          return false;
         mbar_expect_tx(bar(L::B_K + st), L::kTile);
-        load_tile<D>(sbase + L::kK + st * L::kTile, &tmK, &tmK8, bar(L::B_K + st), b, kvh, tr, p.N);
+        load_tile<D>(sbase + L::kK + st * L::kTile, &tmK, &tmK8, bar(L::B_K + st), b, kvh,
+                     rolled_tile_runs((kt_begin + i) * kTileRows, shift_h, p.N), p.N);
+        ++k_issued;
+        return true;
+      };
+      auto issue_v = [&]() -> bool {
+        const int i = v_issued, st = i % L::kVStages;
+        if (i >= L::kVStages &&
+            !wait_bar(bar(L::B_VE + st), ((i / L::kVStages) - 1) & 1, ctx, 10))
+          return false;
         mbar_expect_tx(bar(L::B_V + st), L::kTile);
-        load_tile<D>(sbase + L::kV + st * L::kTile, &tmV, &tmV8, bar(L::B_V + st), b, kvh, tr, p.N);
-        last_parity[st] = (it >> 1) & 1;
+        load_tile<D>(sbase + L::kV + st * L::kTile, &tmV, &tmV8, bar(L::B_V + st), b, kvh,
+                     rolled_tile_runs((kt_begin + i) * kTileRows, shift_h, p.N), p.N);
+        ++v_issued;
+        return true;
+      };
+      bool ok = issue_k();
+      for (int j = 0; ok && j < n_kv; ++j) {
+        if (j + 1 < n_kv) ok = issue_k();
+        if (ok) ok = issue_v();
       }
       drain_wait(bar(L::B_QDO), 0, p.timeout_ns);
-      for (int s = 0; s < 2; ++s) {
-        if (last_parity[s] >= 0) {
-          drain_wait(bar(L::B_K + s), last_parity[s], p.timeout_ns);
-          drain_wait(bar(L::B_V + s), last_parity[s], p.timeout_ns);
-        }
-      }
+      for (int i = k_issued - L::kKStages; i < k_issued; ++i)
+        if (i >= 0) drain_wait(bar(L::B_K + i % L::kKStages), (i / L::kKStages) & 1, p.timeout_ns);
+      for (int i = v_issued - L::kVStages; i < v_issued; ++i)
+        if (i >= 0) drain_wait(bar(L::B_V + i % L::kVStages), (i / L::kVStages) & 1, p.timeout_ns);
     }
   } else if (warp == 5) {
     if (lane == 0) {
@@ -127,36 +148,39 @@ __global__ void __launch_bounds__(192, 1)
                  idesc_s, kk > 0 ? 1u : 0u);
         }
       };
+      auto wait_k = [&](int j) {
+        return wait_bar(bar(L::B_K + j % L::kKStages), (j / L::kKStages) & 1, ctx, 3);
+      };
       bool ok = wait_bar(bar(L::B_QDO), 0, ctx, 2);
-      if (ok) ok = wait_bar(bar(L::B_K + 0), 0, ctx, 3);
+      if (ok) ok = wait_k(0);
       if (ok) {
         tc_fence_after();
         issue_nt(tmem, sbase + L::kQ, sbase + L::kK);
         mma_commit(bar(L::B_S + 0));
       }
       for (int n = 0; ok && n < n_kv; ++n) {
-        const int st = n & 1;
-        const uint32_t ph = (n >> 1) & 1;
-        if (!wait_bar(bar(L::B_V + st), ph, ctx, 4)) { ok = false; break; }
+        const int st = n & 1, kst = n % L::kKStages, vst = n % L::kVStages;
+        if (!wait_bar(bar(L::B_V + vst), (n / L::kVStages) & 1, ctx, 4)) { ok = false; break; }
         tc_fence_after();
-        issue_nt(tm_dp, sbase + L::kDO, sbase + L::kV + st * L::kTile);
+        issue_nt(tm_dp, sbase + L::kDO, sbase + L::kV + vst * L::kTile);
         mma_commit(bar(L::B_DP));
+        mma_commit(bar(L::B_VE + vst));   // V(n) has no reader left
         if (n + 1 < n_kv) {
-          const int st1 = (n + 1) & 1;
-          if (!wait_bar(bar(L::B_K + st1), ((n + 1) >> 1) & 1, ctx, 5)) { ok = false; break; }
+          if (!wait_k(n + 1)) { ok = false; break; }
           tc_fence_after();
-          issue_nt(tmem + st1 * 128, sbase + L::kQ, sbase + L::kK + st1 * L::kTile);
-          mma_commit(bar(L::B_S + st1));
+          issue_nt(tmem + ((n + 1) & 1) * 128, sbase + L::kQ,
+                   sbase + L::kK + ((n + 1) % L::kKStages) * L::kTile);
+          mma_commit(bar(L::B_S + ((n + 1) & 1)));
         }
-        if (!wait_bar(bar(L::B_DS + st), ph, ctx, 6)) { ok = false; break; }
+        if (!wait_bar(bar(L::B_DS + st), (n >> 1) & 1, ctx, 6)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t k_base = sbase + L::kK + st * L::kTile;
+        const uint32_t k_base = sbase + L::kK + kst * L::kTile;
 #pragma unroll
         for (int kk = 0; kk < kTileRows / 16; ++kk)
           mma_ts(tm_dq, tmem + st * 128 + kk * 8,
                  sdesc_sw128(k_base + kk * 2048, Tile<D>::kHalfBytes, 1024), idesc_dq,
                  (n > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(bar(L::B_EMPTY + st));
+        mma_commit(bar(L::B_KE + kst));   // K(n): read by S(n) and dQ(n)
       }
       if (ok) mma_commit(bar(L::B_ACC));
     }

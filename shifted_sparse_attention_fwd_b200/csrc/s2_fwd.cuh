@@ -1,22 +1,31 @@
 // S²-Attn forward (O and row log-sum-exp) on sm_100a tensor cores.
 //
 // LongLoRA summary page, §3.4 Algorithm 1: per head, roll (second chunk of heads), view as
-// groups of G, causal softmax(scale * q k^T) v inside each group, roll back. One CTA owns a
-// 128-row tile of rolled query rows of one (batch, head); it walks the 128-row key/value
-// tiles of the same rolled frame from the start of the group of its first row up to its
-// own diagonal tile, so work is proportional to N*G rather than N^2. The roll never moves
-// data: TMA reads the original rows (see s2_tiles.cuh) and the epilogue stores O and LSE at
-// the original rows.
+// groups of G, causal softmax(scale * q k^T) v inside each group, roll back. One CTA owns two
+// consecutive 128-row tiles of rolled query rows of one (batch, head) and walks the 128-row
+// key/value tiles of the same rolled frame, from the start of the group of its first row to
+// its last diagonal tile: work is proportional to N*G rather than N^2. The roll never moves
+// data: TMA reads the original rows (s2_tiles.cuh) and the epilogue stores O and LSE at the
+// original rows.
 //
-// Warp roles (192 threads):
-//   warps 0-3  softmax: thread i owns query row i (TMEM lane i); online softmax in fp32,
-//              P written back to TMEM as bf16, O rescaled in TMEM, epilogue.
-//   warp 4     TMA producer: Q once, then K/V tiles through a 2-stage ring.
-//   warp 5     TMEM allocator and MMA issuer (one lane): S = Q K^T (SS), O += P V (TS).
-// TMEM columns: S/P double buffer at [0,128) and [128,256); O at [256, 256+D).
+// Warp roles (320 threads):
+//   warps 0-3, 4-7  softmax warpgroup of query tile 0 / 1: thread i owns query row i (TMEM
+//                   lane i); online softmax in fp32, P written back to TMEM as bf16 over S,
+//                   O rescaled in TMEM when the running max grows, epilogue.
+//   warp 8          TMA producer: both Q tiles once, then K tiles (3-stage ring) running one
+//                   tile ahead of V tiles (2-stage ring); each ring slot is released by a
+//                   commit right after the last MMA that reads it.
+//   warp 9          TMEM allocator and MMA issuer (one lane).
+// TMEM columns: S0/P0 [0,128), S1/P1 [128,256), O0 [256,256+D), O1 [256+D, 256+2D).
+//
+// MMA issue order S0(0) S1(0) PV0(0) S0(1) PV1(0) S1(1) PV0(1) ... lets each warpgroup's
+// softmax run while the tensor core works on the other tile. tcgen05 MMAs from one thread
+// complete in issue order, so when S_t(j+1) is signalled, PV_t(j) — which read P_t(j) from
+// the same columns and accumulated into O_t — is complete: the softmax may rescale O_t at once.
 #pragma once
 
 #include "s2_common.cuh"
+#include "s2_tmem_wide.cuh"
 
 namespace s2 {
 
@@ -29,15 +38,20 @@ struct FwdParams {
   unsigned long long timeout_ns;
 };
 
+// Rescale O only when the running max (log2 units) grows by more than this: until then
+// exp2(s - stale max) <= 2^8, harmless in fp32 and bf16, and the final 1/l uses the same max.
+constexpr float kRescaleThreshold = 8.0f;
+
 template <int D>
 struct FwdLayout {
   static constexpr uint32_t kTile = Tile<D>::kBytes;
-  static constexpr uint32_t kQ = 0;
-  static constexpr uint32_t kK = kQ + kTile;        // 2 stages
-  static constexpr uint32_t kV = kK + 2 * kTile;    // 2 stages
-  static constexpr uint32_t kBar = kV + 2 * kTile;
-  enum { B_Q = 0, B_K = 1, B_V = 3, B_EMPTY = 5, B_S = 7, B_P = 9, B_O = 11, B_DRAIN = 12,
-         B_COUNT = 13 };
+  static constexpr int kKStages = 3, kVStages = 2;
+  static constexpr uint32_t kQ = 0;                         // 2 query tiles
+  static constexpr uint32_t kK = kQ + 2 * kTile;            // K ring
+  static constexpr uint32_t kV = kK + kKStages * kTile;     // V ring
+  static constexpr uint32_t kBar = kV + kVStages * kTile;
+  enum { B_Q = 0, B_K = 2, B_KE = 5, B_V = 8, B_VE = 10, B_S = 12, B_P = 14, B_ODONE = 16,
+         B_DRAIN = 18, B_COUNT = 19 };
   static constexpr uint32_t kTmemSlot = kBar + B_COUNT * 8;
   static constexpr uint32_t kAbort = kTmemSlot + 4;
   static constexpr uint32_t kBytes = kAbort + 4;
@@ -45,10 +59,26 @@ struct FwdLayout {
   // CTA is resident per SM (each CTA takes all 512 TMEM columns).
   static constexpr uint32_t kLaunchBytes =
       (kBytes + 1024 > 116 * 1024) ? kBytes + 1024 : 116 * 1024;
+  static constexpr int kThreads = 320;
 };
 
+__device__ __forceinline__ float max_tree128(const float (&s)[128]) {
+  float m[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m[i] = s[i];
+#pragma unroll
+  for (int j = 1; j < 16; ++j)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m[i] = fmaxf(m[i], s[8 * j + i]);
+#pragma unroll
+  for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+    for (int i = 0; i < w; ++i) m[i] = fmaxf(m[i], m[i + w]);
+  return m[0];
+}
+
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     s2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQ8,
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmK8,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmV8,
@@ -63,24 +93,39 @@ __global__ void __launch_bounds__(192, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kTmemSlot);
   const WaitCtx ctx{abort_flag, p.err, p.timeout_ns, KID_FWD};
 
-  int b, h, qt;
-  query_tile_coords(blockIdx.x, p.B, p.Hq, p.N, p.G, b, h, qt);
-  const int R0 = qt * kTileRows;
+  int b, h, pair;
+  query_pair_coords(blockIdx.x, p.B, p.Hq, p.N, p.G, b, h, pair);
+  const int nqt = (p.N + kTileRows - 1) / kTileRows;
   const int shift_h = h >= p.shift_head_begin ? p.shift : 0;
   const int kvh = h / (p.Hq / p.Hkv);
-  const int kt_begin = group_begin(R0, p.G) / kTileRows;
-  const int n_kv = qt - kt_begin + 1;
+  // Tile t = 2*pair + t sees key tiles [kb[t], ke[t]]; tile 0 always exists, tile 1 may not.
+  int qt[2], kb[2], ke[2];
+  bool tv[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    qt[t] = 2 * pair + t;
+    tv[t] = qt[t] < nqt;
+    kb[t] = tv[t] ? group_begin(qt[t] * kTileRows, p.G) / kTileRows : 0;
+    ke[t] = qt[t];
+  }
+  const int kv_lo = kb[0];
+  const int kv_hi = tv[1] ? ke[1] : ke[0];
+  const int n_kv = kv_hi - kv_lo + 1;
+  auto part = [&](int t, int kt) { return tv[t] && kb[t] <= kt && kt <= ke[t]; };
 
-  if (warp == 4 && lane == 0) {
-    mbar_init(bar(L::B_Q), 1);
+  if (warp == 8 && lane == 0) {
     for (int s = 0; s < 2; ++s) {
-      mbar_init(bar(L::B_K + s), 1);
+      mbar_init(bar(L::B_Q + s), 1);
       mbar_init(bar(L::B_V + s), 1);
-      mbar_init(bar(L::B_EMPTY + s), 1);
+      mbar_init(bar(L::B_VE + s), 1);
       mbar_init(bar(L::B_S + s), 1);
       mbar_init(bar(L::B_P + s), 128);
+      mbar_init(bar(L::B_ODONE + s), 1);
     }
-    mbar_init(bar(L::B_O), 1);
+    for (int s = 0; s < L::kKStages; ++s) {
+      mbar_init(bar(L::B_K + s), 1);
+      mbar_init(bar(L::B_KE + s), 1);
+    }
     mbar_init(bar(L::B_DRAIN), 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -88,7 +133,7 @@ __global__ void __launch_bounds__(192, 1)
     tma_prefetch_map(&tmK);
     tma_prefetch_map(&tmV);
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
@@ -97,171 +142,223 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
-      int last_parity[2] = {-1, -1};
-      mbar_expect_tx(bar(L::B_Q), L::kTile);
-      load_tile<D>(sbase + L::kQ, &tmQ, &tmQ8, bar(L::B_Q), b, h,
-                   rolled_tile_runs(R0, shift_h, p.N), p.N);
-      for (int it = 0; it < n_kv; ++it) {
-        const int st = it & 1;
-        if (it >= 2 && !wait_bar(bar(L::B_EMPTY + st), ((it >> 1) - 1) & 1, ctx, 1)) break;
-        const TileRuns tr = rolled_tile_runs((kt_begin + it) * kTileRows, shift_h, p.N);
+      for (int t = 0; t < 2; ++t) {
+        if (!tv[t]) continue;
+        mbar_expect_tx(bar(L::B_Q + t), L::kTile);
+        load_tile<D>(sbase + L::kQ + t * L::kTile, &tmQ, &tmQ8, bar(L::B_Q + t), b, h,
+                     rolled_tile_runs(qt[t] * kTileRows, shift_h, p.N), p.N);
+      }
+      // K(j) is loaded into slot j % 3 once K(j - 3) has been released, V(j) into slot j % 2
+      // once V(j - 2) has; K runs one tile ahead of V.
+      int k_issued = 0, v_issued = 0;
+      auto issue_k = [&]() -> bool {
+        const int i = k_issued, st = i % L::kKStages;
+        if (i >= L::kKStages &&
+            !wait_bar(bar(L::B_KE + st), ((i / L::kKStages) - 1) & 1, ctx, 1))
+          return false;
         mbar_expect_tx(bar(L::B_K + st), L::kTile);
-        load_tile<D>(sbase + L::kK + st * L::kTile, &tmK, &tmK8, bar(L::B_K + st), b, kvh, tr, p.N);
+        load_tile<D>(sbase + L::kK + st * L::kTile, &tmK, &tmK8, bar(L::B_K + st), b, kvh,
+                     rolled_tile_runs((kv_lo + i) * kTileRows, shift_h, p.N), p.N);
+        ++k_issued;
+        return true;
+      };
+      auto issue_v = [&]() -> bool {
+        const int i = v_issued, st = i % L::kVStages;
+        if (i >= L::kVStages &&
+            !wait_bar(bar(L::B_VE + st), ((i / L::kVStages) - 1) & 1, ctx, 9))
+          return false;
         mbar_expect_tx(bar(L::B_V + st), L::kTile);
-        load_tile<D>(sbase + L::kV + st * L::kTile, &tmV, &tmV8, bar(L::B_V + st), b, kvh, tr, p.N);
-        last_parity[st] = (it >> 1) & 1;
+        load_tile<D>(sbase + L::kV + st * L::kTile, &tmV, &tmV8, bar(L::B_V + st), b, kvh,
+                     rolled_tile_runs((kv_lo + i) * kTileRows, shift_h, p.N), p.N);
+        ++v_issued;
+        return true;
+      };
+      bool ok = issue_k();
+      for (int j = 0; ok && j < n_kv; ++j) {
+        if (j + 1 < n_kv) ok = issue_k();
+        if (ok) ok = issue_v();
       }
       // Every issued copy lands before the CTA can exit.
-      drain_wait(bar(L::B_Q), 0, p.timeout_ns);
-      for (int s = 0; s < 2; ++s) {
-        if (last_parity[s] >= 0) {
-          drain_wait(bar(L::B_K + s), last_parity[s], p.timeout_ns);
-          drain_wait(bar(L::B_V + s), last_parity[s], p.timeout_ns);
-        }
-      }
+      for (int t = 0; t < 2; ++t)
+        if (tv[t]) drain_wait(bar(L::B_Q + t), 0, p.timeout_ns);
+      for (int i = k_issued - L::kKStages; i < k_issued; ++i)
+        if (i >= 0) drain_wait(bar(L::B_K + i % L::kKStages), (i / L::kKStages) & 1, p.timeout_ns);
+      for (int i = v_issued - L::kVStages; i < v_issued; ++i)
+        if (i >= 0) drain_wait(bar(L::B_V + i % L::kVStages), (i / L::kVStages) & 1, p.timeout_ns);
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16(128, 128, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16(128, D, false, true);
-      const uint32_t tm_o = tmem + 256;
-      auto issue_pv = [&](int j) -> bool {
-        const int st = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
-        if (!wait_bar(bar(L::B_P + st), ph, ctx, 2)) return false;
-        if (!wait_bar(bar(L::B_V + st), ph, ctx, 3)) return false;
-        tc_fence_after();
-        const uint32_t v_base = sbase + L::kV + st * L::kTile;
-#pragma unroll
-        for (int kk = 0; kk < kTileRows / 16; ++kk) {
-          const uint64_t bdesc = sdesc_sw128(v_base + kk * 2048, Tile<D>::kHalfBytes, 1024);
-          mma_ts(tm_o, tmem + st * 128 + kk * 8, bdesc, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+      bool q_ready[2] = {false, false};
+      int pcount[2] = {0, 0};
+      bool ok = true;
+      auto issue_s = [&](int t, int j) -> bool {
+        if (!q_ready[t]) {
+          if (!wait_bar(bar(L::B_Q + t), 0, ctx, 2)) return false;
+          q_ready[t] = true;
         }
-        mma_commit(bar(L::B_EMPTY + st));
-        mma_commit(bar(L::B_O));
-        return true;
-      };
-      bool ok = wait_bar(bar(L::B_Q), 0, ctx, 4);
-      for (int it = 0; ok && it < n_kv; ++it) {
-        const int st = it & 1;
-        if (!wait_bar(bar(L::B_K + st), (it >> 1) & 1, ctx, 5)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t q_base = sbase + L::kQ;
-        const uint32_t k_base = sbase + L::kK + st * L::kTile;
+        const uint32_t q_base = sbase + L::kQ + t * L::kTile;
+        const uint32_t k_base = sbase + L::kK + (j % L::kKStages) * L::kTile;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * Tile<D>::kHalfBytes + (kk % 4) * 32;
-          mma_ss(tmem + st * 128, sdesc_sw128(q_base + off, 16, 1024),
+          mma_ss(tmem + t * 128, sdesc_sw128(q_base + off, 16, 1024),
                  sdesc_sw128(k_base + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
         }
-        mma_commit(bar(L::B_S + st));
-        if (it > 0) ok = issue_pv(it - 1);
-      }
-      if (ok) issue_pv(n_kv - 1);
-    }
-  } else {
-    // ---------------- softmax warps 0-3 ----------------
-    const int row = threadIdx.x;
-    const int r = R0 + row;
-    const bool row_valid = r < p.N;
-    const int lo = row_valid ? group_begin(r, p.G) : kt_begin * kTileRows;
-    const int hi = row_valid ? r : kt_begin * kTileRows;
-    const uint32_t t_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    const float c = p.scale_log2;
-    float m_run = -INFINITY, l_run = 0.f;
-    bool ok = true;
-    for (int it = 0; it < n_kv; ++it) {
-      const int st = it & 1;
-      if (!warp_wait(bar(L::B_S + st), (it >> 1) & 1, ctx, 6)) { ok = false; break; }
-      tc_fence_after();
-      float s[128];
+        mma_commit(bar(L::B_S + t));
+        return true;
+      };
+      auto wait_k = [&](int j) {
+        return wait_bar(bar(L::B_K + j % L::kKStages), (j / L::kKStages) & 1, ctx, 3);
+      };
+      // S for key tile 0, then release of its K slot once both S MMAs are done.
+      if (!wait_k(0)) ok = false;
+      for (int t = 0; ok && t < 2; ++t)
+        if (part(t, kv_lo)) ok = issue_s(t, 0);
+      if (ok) mma_commit(bar(L::B_KE + 0));
+      for (int j = 0; ok && j < n_kv; ++j) {
+        const int kt = kv_lo + j, vst = j % L::kVStages;
+        const bool next = j + 1 < n_kv;
+        bool v_ready = false, k_next_ready = false;
+        for (int t = 0; ok && t < 2; ++t) {
+          if (part(t, kt)) {
+            if (!wait_bar(bar(L::B_P + t), pcount[t] & 1, ctx, 4)) { ok = false; break; }
+            if (!v_ready) {
+              if (!wait_bar(bar(L::B_V + vst), (j / L::kVStages) & 1, ctx, 5)) { ok = false; break; }
+              v_ready = true;
+            }
+            tc_fence_after();
+            const uint32_t v_base = sbase + L::kV + vst * L::kTile;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        uint32_t rr[32];
-        tmem_ld32(t_lane + st * 128 + 32 * j, rr);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) s[32 * j + i] = __uint_as_float(rr[i]);
-      }
-      const int c0 = (kt_begin + it) * kTileRows;
-      const int cl = lo - c0, ch = hi - c0;
-      if (cl > 0 || ch < kTileRows - 1) {
-#pragma unroll
-        for (int i = 0; i < 128; ++i) s[i] = (i < cl || i > ch) ? -INFINITY : s[i];
-      }
-      float mx = s[0];
-#pragma unroll
-      for (int i = 1; i < 128; ++i) mx = fmaxf(mx, s[i]);
-      const float m_new = fmaxf(m_run, mx * c);
-      const float m_use = m_new == -INFINITY ? 0.f : m_new;
-      float sum = 0.f;
-#pragma unroll
-      for (int i = 0; i < 128; ++i) {
-        s[i] = fast_exp2(fmaf(s[i], c, -m_use));
-        sum += s[i];
-      }
-      const float alpha = fast_exp2(m_run - m_use);
-      if (it > 0) {
-        if (!warp_wait(bar(L::B_O), (it - 1) & 1, ctx, 7)) { ok = false; break; }
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll
-          for (int j = 0; j < D / 32; ++j) {
-            uint32_t rr[32];
-            tmem_ld32(t_lane + 256 + 32 * j, rr);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * alpha);
-            tmem_st32(t_lane + 256 + 32 * j, rr);
+            for (int kk = 0; kk < kTileRows / 16; ++kk)
+              mma_ts(tmem + 256 + t * D, tmem + t * 128 + kk * 8,
+                     sdesc_sw128(v_base + kk * 2048, Tile<D>::kHalfBytes, 1024), idesc_pv,
+                     (pcount[t] > 0 || kk > 0) ? 1u : 0u);
+            ++pcount[t];
+            if (kt == ke[t]) mma_commit(bar(L::B_ODONE + t));
+          }
+          if (t == 1) mma_commit(bar(L::B_VE + vst));   // V(j) has no reader left
+          if (next && part(t, kt + 1)) {
+            if (!k_next_ready) {
+              if (!wait_k(j + 1)) { ok = false; break; }
+              k_next_ready = true;
+            }
+            if (!issue_s(t, j + 1)) { ok = false; break; }
           }
         }
+        if (ok && next) mma_commit(bar(L::B_KE + (j + 1) % L::kKStages));   // K(j+1) likewise
       }
-      l_run = l_run * alpha + sum;
-      m_run = m_new;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(s[32 * j + 2 * i], s[32 * j + 2 * i + 1]);
-        tmem_st16(t_lane + st * 128 + 16 * j, pk);
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(bar(L::B_P + st));
     }
-    if (ok && warp_wait(bar(L::B_O), (n_kv - 1) & 1, ctx, 8)) {
-      tc_fence_after();
-      const float inv_l = 1.f / l_run;
-      long long tt = static_cast<long long>(r) + shift_h;
-      const int t = static_cast<int>(tt >= p.N ? tt - p.N : tt);
-      __nv_bfloat16* orow =
-          p.o + ((static_cast<size_t>(b) * p.N + (row_valid ? t : 0)) * p.Hq + h) * D;
+  } else {
+    // ---------------- softmax warpgroups ----------------
+    const int wg = warp / 4;
+    if (tv[wg]) {
+      const int row = threadIdx.x % 128;
+      const int r = qt[wg] * kTileRows + row;
+      const bool row_valid = r < p.N;
+      const int lo = row_valid ? group_begin(r, p.G) : kb[wg] * kTileRows;
+      const int hi = row_valid ? r : kb[wg] * kTileRows;
+      const uint32_t t_lane = tmem + (static_cast<uint32_t>((warp % 4) * 32) << 16);
+      const uint32_t s_col = t_lane + wg * 128;
+      const uint32_t o_col = t_lane + 256 + wg * D;
+      const float c = p.scale_log2;
+      float m_run = -INFINITY, l_run = 0.f;
+      bool ok = true;
+      int cnt = 0;
+      for (int kt = kb[wg]; kt <= ke[wg]; ++kt, ++cnt) {
+        if (!warp_wait(bar(L::B_S + wg), cnt & 1, ctx, 7)) { ok = false; break; }
+        tc_fence_after();
+        float s[128];
+        {
+          uint32_t raw[128];
+          tmem_ld128(s_col, raw);
 #pragma unroll
-      for (int j = 0; j < D / 32; ++j) {
-        uint32_t rr[32];
-        tmem_ld32(t_lane + 256 + 32 * j, rr);
-        uint32_t pk[16];
+          for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(raw[i]);
+        }
+        const int cl = lo - kt * kTileRows, ch = hi - kt * kTileRows;
+        if (__any_sync(0xffffffffu, cl > 0 || ch < kTileRows - 1)) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          pk[i] = pack_bf16(__uint_as_float(rr[2 * i]) * inv_l, __uint_as_float(rr[2 * i + 1]) * inv_l);
+          for (int i = 0; i < 128; ++i) s[i] = (i < cl || i > ch) ? -INFINITY : s[i];
+        }
+        const float m_cand = fmaxf(m_run, max_tree128(s) * c);
+        const bool need = m_cand > m_run + kRescaleThreshold;
+        if (__any_sync(0xffffffffu, need)) {
+          const float alpha = fast_exp2(m_run - m_cand);   // 0 when m_run = -inf
+          if (cnt > 0) {
+#pragma unroll 1
+            for (int j = 0; j < D / 32; ++j) {
+              uint32_t ov[32];
+              tmem_ld32(o_col + 32 * j, ov);
+#pragma unroll
+              for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+              tmem_st32(o_col + 32 * j, ov);
+            }
+          }
+          l_run *= alpha;
+          m_run = m_cand;
+        }
+        const float m_use = m_run == -INFINITY ? 0.f : m_run;
+        float part_sum[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) part_sum[i] = 0.f;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float e0 = fast_exp2(fmaf(s[32 * j + 2 * i], c, -m_use));
+            const float e1 = fast_exp2(fmaf(s[32 * j + 2 * i + 1], c, -m_use));
+            part_sum[(2 * i) & 7] += e0;
+            part_sum[(2 * i + 1) & 7] += e1;
+            pk[i] = pack_bf16(e0, e1);
+          }
+          tmem_st16(s_col + 16 * j, pk);
+        }
+#pragma unroll
+        for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+          for (int i = 0; i < w; ++i) part_sum[i] += part_sum[i + w];
+        l_run += part_sum[0];
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar(L::B_P + wg));
+      }
+      if (ok && warp_wait(bar(L::B_ODONE + wg), 0, ctx, 8)) {
+        tc_fence_after();
+        const float inv_l = 1.f / l_run;
+        const long long tt = static_cast<long long>(r) + shift_h;
+        const int t = static_cast<int>(tt >= p.N ? tt - p.N : tt);
+        __nv_bfloat16* orow =
+            p.o + ((static_cast<size_t>(b) * p.N + (row_valid ? t : 0)) * p.Hq + h) * D;
+        uint32_t ov[D];
+        if constexpr (D == 128) tmem_ld128(o_col, ov); else tmem_ld64(o_col, ov);
         if (row_valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * j);
 #pragma unroll
-          for (int v = 0; v < 4; ++v)
-            dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          for (int v = 0; v < D / 8; ++v) {
+            uint4 w4;
+            w4.x = pack_bf16(__uint_as_float(ov[8 * v + 0]) * inv_l, __uint_as_float(ov[8 * v + 1]) * inv_l);
+            w4.y = pack_bf16(__uint_as_float(ov[8 * v + 2]) * inv_l, __uint_as_float(ov[8 * v + 3]) * inv_l);
+            w4.z = pack_bf16(__uint_as_float(ov[8 * v + 4]) * inv_l, __uint_as_float(ov[8 * v + 5]) * inv_l);
+            w4.w = pack_bf16(__uint_as_float(ov[8 * v + 6]) * inv_l, __uint_as_float(ov[8 * v + 7]) * inv_l);
+            reinterpret_cast<uint4*>(orow)[v] = w4;
+          }
+          p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.N + t] =
+              (m_run + __log2f(l_run)) * 0.6931471805599453f;
         }
       }
-      if (row_valid)
-        p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.N + t] = (m_run + __log2f(l_run)) * 0.6931471805599453f;
     }
   }
 
   // ---------------- teardown ----------------
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     if (lane == 0) {
       mma_commit(bar(L::B_DRAIN));
       drain_wait(bar(L::B_DRAIN), 0, p.timeout_ns);

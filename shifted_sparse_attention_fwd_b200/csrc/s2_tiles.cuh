@@ -109,6 +109,32 @@ __host__ __device__ inline void query_tile_coords(int bid, int B, int Hq, int N,
   }
 }
 
+// Block index -> (b, h, pair) for kernels whose CTA owns the two rolled query tiles 2*pair
+// and 2*pair + 1 of one (b, h). When G is a multiple of two tiles, pairs late in their group
+// (more key tiles to visit) come first.
+__host__ __device__ inline int query_pairs_per_head(int N) {
+  return ((N + kTileRows - 1) / kTileRows + 1) / 2;
+}
+__host__ __device__ inline void query_pair_coords(int bid, int B, int Hq, int N, int G, int& b,
+                                                  int& h, int& pair) {
+  if (G % (2 * kTileRows) == 0) {
+    const int ppg = G / (2 * kTileRows), ng = N / G;
+    const int per = B * Hq * ng;
+    const int pl = ppg - 1 - bid / per;
+    const int rest = bid % per;
+    const int g = rest % ng;
+    const int bh = rest / ng;
+    h = bh % Hq;
+    b = bh / Hq;
+    pair = g * ppg + pl;
+  } else {
+    const int bh = bid % (B * Hq);
+    pair = bid / (B * Hq);
+    h = bh % Hq;
+    b = bh / Hq;
+  }
+}
+
 // Block index -> (b, kv head, first original row t0 of the kv tile) for the dK/dV kernel.
 // When groups and roll are tile-aligned, kv tiles early in their (rolled) group, which see
 // the most query tiles, come first.

@@ -170,8 +170,8 @@ s2attn_status launch_fwd(const Shape& sh, const void* q, const void* k, const vo
   p.scale_log2 = scale * 1.4426950408889634f;
   p.err = err;
   p.timeout_ns = g_timeout_ns.load();
-  const unsigned grid = static_cast<unsigned>(sh.B) * sh.Hq * ((sh.N + 127) / 128);
-  s2::s2_fwd_kernel<D><<<grid, 192, s2::FwdLayout<D>::kLaunchBytes, stream>>>(
+  const unsigned grid = static_cast<unsigned>(sh.B) * sh.Hq * s2::query_pairs_per_head(sh.N);
+  s2::s2_fwd_kernel<D><<<grid, s2::FwdLayout<D>::kThreads, s2::FwdLayout<D>::kLaunchBytes, stream>>>(
       mq.m128, mq.m8, mk.m128, mk.m8, mv.m128, mv.m8, p);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? S2ATTN_OK : cuda_fail(e, "s2_fwd_kernel launch");

@@ -133,6 +133,8 @@ int qtiles(int t0, int sh, int N, int G, int* o) {
   int n = q.count(); for (int i = 0; i < n; ++i) o[i] = q.at(i); return n; }
 void qcoords(int bid, int B, int Hq, int N, int G, int* o) {
   s2::query_tile_coords(bid, B, Hq, N, G, o[0], o[1], o[2]); }
+void paircoords(int bid, int B, int Hq, int N, int G, int* o) {
+  s2::query_pair_coords(bid, B, Hq, N, G, o[0], o[1], o[2]); o[3] = s2::query_pairs_per_head(N); }
 void kvcoords(int bid, int B, int Hq, int Hkv, int N, int G, int shb, int sh, int* o) {
   s2::kv_tile_coords(bid, B, Hq, Hkv, N, G, shb, sh, o[0], o[1], o[2]); }
 }
@@ -230,3 +232,19 @@ def test_kv_tile_order_is_a_permutation(shim, B, Hq, Hkv, N, G, shb, sh):
         assert t0 % 128 == 0
         seen.add((b, kvh, t0 // 128))
     assert seen == {(b, k, t) for b in range(B) for k in range(Hkv) for t in range(nt)}
+
+
+@pytest.mark.parametrize("B,Hq,N,G", [(1, 4, 256, 64), (2, 3, 8192, 2048), (1, 2, 384, 192),
+                                      (3, 2, 320, 64), (1, 1, 1024, 1024), (1, 2, 640, 128),
+                                      (1, 2, 16, 16)])
+def test_query_pair_order_is_a_permutation(shim, B, Hq, N, G):
+    nt = (N + 127) // 128
+    npair = call4(shim.paircoords, 0, B, Hq, N, G)[3]
+    assert npair == (nt + 1) // 2
+    seen = set()
+    for bid in range(B * Hq * npair):
+        seen.add(tuple(call4(shim.paircoords, bid, B, Hq, N, G)[:3]))
+    assert seen == {(b, h, p) for b in range(B) for h in range(Hq) for p in range(npair)}
+    if G % 256 == 0 and G > 256:
+        b, h, p = call4(shim.paircoords, 0, B, Hq, N, G)[:3]
+        assert p % (G // 256) == G // 256 - 1
