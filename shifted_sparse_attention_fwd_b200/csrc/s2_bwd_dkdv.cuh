@@ -14,13 +14,18 @@
 // For each query head the rows map to at most two runs of rolled rows; the query tiles
 // visited are those covering [rolled row, end of its group) for every row of the tile.
 //
-// Warp roles (192 threads): warps 0-3 elementwise (thread i owns kv row i = TMEM lane i),
-// warp 4 TMA producer (K, V once; Q, dO, LSE2, D per query tile, 2 stages), warp 5 TMEM
-// allocator + MMA issuer. TMEM: S^T/P^T [0,128), dP^T/dS^T [128,256), dV [256,256+D),
-// dK [256+D, 256+2D).
+// Warp roles (320 threads): warps 0-7 elementwise — kv row i (TMEM lane i) is shared by warp
+// i/32 (query columns 0-63) and warp i/32 + 4 (columns 64-127), so two warps per SM
+// sub-partition work on every tile; warp 8 TMA producer (K, V once; Q, dO, LSE2, D per query
+// tile, 2 stages); warp 9 TMEM allocator + MMA issuer.
+// TMEM: S^T [0,128) with P^T (bf16) written to [32,96); dP^T [128,256) with dS^T (bf16) to
+// [160,224) — each column half packs its bf16 output inside its own fp32 input columns, so the
+// two warps of a row never overwrite each other's unread data; dV [256,256+D), dK
+// [256+D, 256+2D).
 #pragma once
 
 #include "s2_common.cuh"
+#include "s2_tmem_wide.cuh"
 
 namespace s2 {
 
@@ -54,10 +59,11 @@ struct DkdvLayout {
   static constexpr uint32_t kBytes = kAbort + 4;
   static constexpr uint32_t kLaunchBytes =
       (kBytes + 1024 > 116 * 1024) ? kBytes + 1024 : 116 * 1024;
+  static constexpr int kThreads = 320;
 };
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     s2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQ8,
                        const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmK8,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmV8,
@@ -79,7 +85,7 @@ __global__ void __launch_bounds__(192, 1)
   const int h_begin = kvh * rep;
   auto head_shift = [&](int hq) { return hq >= p.shift_head_begin ? p.shift : 0; };
 
-  if (warp == 4 && lane == 0) {
+  if (warp == 8 && lane == 0) {
     mbar_init(bar(L::B_KV), 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(L::B_QF + s), 1);
@@ -87,8 +93,8 @@ __global__ void __launch_bounds__(192, 1)
     }
     mbar_init(bar(L::B_S), 1);
     mbar_init(bar(L::B_DP), 1);
-    mbar_init(bar(L::B_P), 128);
-    mbar_init(bar(L::B_DS), 128);
+    mbar_init(bar(L::B_P), 256);
+    mbar_init(bar(L::B_DS), 256);
     mbar_init(bar(L::B_ACC), 1);
     mbar_init(bar(L::B_DRAIN), 1);
     *abort_flag = 0;
@@ -98,7 +104,7 @@ __global__ void __launch_bounds__(192, 1)
     tma_prefetch_map(&tmV);
     tma_prefetch_map(&tmO);
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
@@ -107,8 +113,9 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tm_s = tmem, tm_dp = tmem + 128, tm_dv = tmem + 256, tm_dk = tmem + 256 + D;
+  const uint32_t tm_p = tmem + 32, tm_ds = tmem + 160;   // bf16 P^T and dS^T (MMA A operands)
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
       int last_parity[2] = {-1, -1};
@@ -145,7 +152,7 @@ __global__ void __launch_bounds__(192, 1)
       for (int s = 0; s < 2; ++s)
         if (last_parity[s] >= 0) drain_wait(bar(L::B_QF + s), last_parity[s], p.timeout_ns);
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16(128, 128, false, false);  // K Q^T, V dO^T
@@ -181,7 +188,7 @@ __global__ void __launch_bounds__(192, 1)
         mma_commit(bar(L::B_DP));
         if (!wait_bar(bar(L::B_P), n & 1, ctx, 4)) { ok = false; break; }
         tc_fence_after();
-        issue_acc(tm_dv, tm_s, do_s, n);
+        issue_acc(tm_dv, tm_p, do_s, n);
         if (n + 1 < total) {
           const int st1 = (n + 1) & 1;
           if (!wait_bar(bar(L::B_QF + st1), ((n + 1) >> 1) & 1, ctx, 5)) { ok = false; break; }
@@ -191,17 +198,18 @@ __global__ void __launch_bounds__(192, 1)
         }
         if (!wait_bar(bar(L::B_DS), n & 1, ctx, 6)) { ok = false; break; }
         tc_fence_after();
-        issue_acc(tm_dk, tm_dp, q_s, n);
+        issue_acc(tm_dk, tm_ds, q_s, n);
         mma_commit(bar(L::B_QE + st));
       }
       if (ok) mma_commit(bar(L::B_ACC));
     }
   } else {
-    // ---------------- elementwise warps 0-3 ----------------
-    const int row = threadIdx.x;
+    // ---------------- elementwise warps 0-7 ----------------
+    const int half = warp / 4;                     // query columns [64 half, 64 half + 64)
+    const int row = (warp % 4) * 32 + lane;
     const int t = t0 + row;
     const bool kv_valid = t < p.N;
-    const uint32_t t_lane = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>((warp % 4) * 32) << 16);
     const float c = p.scale_log2;
     const float* s_lse = reinterpret_cast<const float*>(smem + L::kLse);
     const float* s_dv = reinterpret_cast<const float*>(smem + L::kDv);
@@ -214,51 +222,51 @@ __global__ void __launch_bounds__(192, 1)
       const int ge_k = group_end(r_k, p.G);
       for (int i = 0; i < qr.count(); ++i, ++n) {
         const int st = n & 1;
-        const int q0 = qr.at(i) * kTileRows;
+        const int q0 = qr.at(i) * kTileRows + 64 * half;
         const int cl = kv_valid ? r_k - q0 : 1;
         const int ch = kv_valid ? ge_k - 1 - q0 : 0;
         if (!warp_wait(bar(L::B_QF + st), (n >> 1) & 1, ctx, 7)) { ok = false; break; }
         if (!warp_wait(bar(L::B_S), n & 1, ctx, 8)) { ok = false; break; }
         tc_fence_after();
-        const float* lse_t = s_lse + st * 128;
-        const float* d_t = s_dv + st * 128;
-        float pv[128];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          uint32_t rr[32];
-          tmem_ld32(t_lane + 32 * j, rr);
+        const float* lse_t = s_lse + st * 128 + 64 * half;
+        const float* d_t = s_dv + st * 128 + 64 * half;
+        // P^T phase: 64 columns of S^T -> P^T (bf16), kept in registers for the dS phase.
+        uint32_t pk[32];
+        {
+          uint32_t raw[64];
+          tmem_ld64(t_lane + 64 * half, raw);
+          const bool mask = __any_sync(0xffffffffu, cl > 0 || ch < 63);
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
-            const int col = 32 * j + e;
-            const float x = fast_exp2(fmaf(__uint_as_float(rr[e]), c, -lse_t[col]));
-            pv[col] = (col >= cl && col <= ch) ? x : 0.f;
+            const int col = 2 * e;
+            float x0 = fast_exp2(fmaf(__uint_as_float(raw[col]), c, -lse_t[col]));
+            float x1 = fast_exp2(fmaf(__uint_as_float(raw[col + 1]), c, -lse_t[col + 1]));
+            if (mask) {
+              x0 = (col >= cl && col <= ch) ? x0 : 0.f;
+              x1 = (col + 1 >= cl && col + 1 <= ch) ? x1 : 0.f;
+            }
+            pk[e] = pack_bf16(x0, x1);
           }
         }
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(pv[32 * j + 2 * e], pv[32 * j + 2 * e + 1]);
-          tmem_st16(t_lane + 16 * j, pk);
-        }
+        tmem_st32(t_lane + 32 + 32 * half, pk);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(bar(L::B_P));
+        // dS^T phase: dS^T = P^T o (dP^T - D).
         if (!warp_wait(bar(L::B_DP), n & 1, ctx, 9)) { ok = false; break; }
         tc_fence_after();
+        {
+          uint32_t raw[64];
+          tmem_ld64(t_lane + 128 + 64 * half, raw);
+          uint32_t ds[32];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          uint32_t rr[32];
-          tmem_ld32(t_lane + 128 + 32 * j, rr);
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int col = 32 * j + 2 * e;
-            const float d0 = pv[col] * (__uint_as_float(rr[2 * e]) - d_t[col]);
-            const float d1 = pv[col + 1] * (__uint_as_float(rr[2 * e + 1]) - d_t[col + 1]);
-            pk[e] = pack_bf16(d0, d1);
+          for (int e = 0; e < 32; ++e) {
+            const int col = 2 * e;
+            const float2 pf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[e]));
+            ds[e] = pack_bf16(pf.x * (__uint_as_float(raw[col]) - d_t[col]),
+                              pf.y * (__uint_as_float(raw[col + 1]) - d_t[col + 1]));
           }
-          tmem_st16(t_lane + 128 + 16 * j, pk);
+          tmem_st32(t_lane + 160 + 32 * half, ds);
         }
         tmem_st_wait();
         tc_fence_before();
@@ -270,13 +278,13 @@ __global__ void __launch_bounds__(192, 1)
       const size_t orow = ((static_cast<size_t>(b) * p.N + (kv_valid ? t : 0)) * p.Hkv + kvh) * D;
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
-        const uint32_t src = which == 0 ? tm_dv : tm_dk;
+        const uint32_t src = (which == 0 ? tm_dv : tm_dk) - tmem + t_lane;
         const float mul = which == 0 ? 1.f : p.scale;
         __nv_bfloat16* dst_row = (which == 0 ? p.dv : p.dk) + orow;
 #pragma unroll
-        for (int j = 0; j < D / 32; ++j) {
+        for (int j = half * (D / 64); j < (half + 1) * (D / 64); ++j) {
           uint32_t rr[32];
-          tmem_ld32(src + (static_cast<uint32_t>(warp * 32) << 16) + 32 * j, rr);
+          tmem_ld32(src + 32 * j, rr);
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e)
@@ -294,7 +302,7 @@ __global__ void __launch_bounds__(192, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     if (lane == 0) {
       mma_commit(bar(L::B_DRAIN));
       drain_wait(bar(L::B_DRAIN), 0, p.timeout_ns);

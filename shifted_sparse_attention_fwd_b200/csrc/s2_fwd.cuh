@@ -1,12 +1,16 @@
 // S²-Attn forward (O and row log-sum-exp) on sm_100a tensor cores.
 //
 // LongLoRA summary page, §3.4 Algorithm 1: per head, roll (second chunk of heads), view as
-// groups of G, causal softmax(scale * q k^T) v inside each group, roll back. One CTA owns two
-// consecutive 128-row tiles of rolled query rows of one (batch, head) and walks the 128-row
-// key/value tiles of the same rolled frame, from the start of the group of its first row to
-// its last diagonal tile: work is proportional to N*G rather than N^2. The roll never moves
-// data: TMA reads the original rows (s2_tiles.cuh) and the epilogue stores O and LSE at the
-// original rows.
+// groups of G, causal softmax(scale * q k^T) v inside each group, roll back. A work unit is
+// two consecutive 128-row tiles of rolled query rows of one (batch, head); it walks the
+// 128-row key/value tiles of the same rolled frame, from the start of the group of its first
+// row to its last diagonal tile: work is proportional to N*G rather than N^2. The roll never
+// moves data: TMA reads the original rows (s2_tiles.cuh) and the epilogue stores O and LSE at
+// the original rows.
+//
+// The kernel is persistent: one CTA per SM sets up its barriers and TMEM once and takes work
+// units blockIdx.x, blockIdx.x + gridDim.x, ... (units are numbered heaviest first), so one
+// unit's epilogue and the next unit's loads overlap the tensor-core work.
 //
 // Warp roles (320 threads):
 //   warps 0-3, 4-7  softmax warpgroup of query tile 0 / 1: thread i owns query row i (TMEM
@@ -50,8 +54,8 @@ struct FwdLayout {
   static constexpr uint32_t kK = kQ + 2 * kTile;            // K ring
   static constexpr uint32_t kV = kK + kKStages * kTile;     // V ring
   static constexpr uint32_t kBar = kV + kVStages * kTile;
-  enum { B_Q = 0, B_K = 2, B_KE = 5, B_V = 8, B_VE = 10, B_S = 12, B_P = 14, B_ODONE = 16,
-         B_DRAIN = 18, B_COUNT = 19 };
+  enum { B_Q = 0, B_QE = 2, B_K = 4, B_KE = 7, B_V = 10, B_VE = 12, B_S = 14, B_P = 16,
+         B_ODONE = 18, B_DRAIN = 20, B_COUNT = 21 };
   static constexpr uint32_t kTmemSlot = kBar + B_COUNT * 8;
   static constexpr uint32_t kAbort = kTmemSlot + 4;
   static constexpr uint32_t kBytes = kAbort + 4;
@@ -77,6 +81,37 @@ __device__ __forceinline__ float max_tree128(const float (&s)[128]) {
   return m[0];
 }
 
+// One work unit: query tiles 2*pair and 2*pair + 1 of (b, h) and the key tiles they see.
+struct FwdUnit {
+  int b, h, kvh, shift_h;
+  int qt[2], kb[2], ke[2];
+  bool tv[2];
+  int kv_lo, n_kv;
+  __device__ __forceinline__ bool part(int t, int kt) const {
+    return tv[t] && kb[t] <= kt && kt <= ke[t];
+  }
+};
+
+__device__ __forceinline__ FwdUnit fwd_unit(const FwdParams& p, int unit) {
+  FwdUnit u;
+  int pair;
+  query_pair_coords(unit, p.B, p.Hq, p.N, p.G, u.b, u.h, pair);
+  const int nqt = (p.N + kTileRows - 1) / kTileRows;
+  u.shift_h = u.h >= p.shift_head_begin ? p.shift : 0;
+  u.kvh = u.h / (p.Hq / p.Hkv);
+  // Tile t = 2*pair + t sees key tiles [kb[t], ke[t]]; tile 0 always exists, tile 1 may not.
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    u.qt[t] = 2 * pair + t;
+    u.tv[t] = u.qt[t] < nqt;
+    u.kb[t] = u.tv[t] ? group_begin(u.qt[t] * kTileRows, p.G) / kTileRows : 0;
+    u.ke[t] = u.qt[t];
+  }
+  u.kv_lo = u.kb[0];
+  u.n_kv = (u.tv[1] ? u.ke[1] : u.ke[0]) - u.kv_lo + 1;
+  return u;
+}
+
 template <int D>
 __global__ void __launch_bounds__(320, 1)
     s2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQ8,
@@ -92,30 +127,12 @@ __global__ void __launch_bounds__(320, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kTmemSlot);
   const WaitCtx ctx{abort_flag, p.err, p.timeout_ns, KID_FWD};
-
-  int b, h, pair;
-  query_pair_coords(blockIdx.x, p.B, p.Hq, p.N, p.G, b, h, pair);
-  const int nqt = (p.N + kTileRows - 1) / kTileRows;
-  const int shift_h = h >= p.shift_head_begin ? p.shift : 0;
-  const int kvh = h / (p.Hq / p.Hkv);
-  // Tile t = 2*pair + t sees key tiles [kb[t], ke[t]]; tile 0 always exists, tile 1 may not.
-  int qt[2], kb[2], ke[2];
-  bool tv[2];
-#pragma unroll
-  for (int t = 0; t < 2; ++t) {
-    qt[t] = 2 * pair + t;
-    tv[t] = qt[t] < nqt;
-    kb[t] = tv[t] ? group_begin(qt[t] * kTileRows, p.G) / kTileRows : 0;
-    ke[t] = qt[t];
-  }
-  const int kv_lo = kb[0];
-  const int kv_hi = tv[1] ? ke[1] : ke[0];
-  const int n_kv = kv_hi - kv_lo + 1;
-  auto part = [&](int t, int kt) { return tv[t] && kb[t] <= kt && kt <= ke[t]; };
+  const int n_units = p.B * p.Hq * query_pairs_per_head(p.N);
 
   if (warp == 8 && lane == 0) {
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(L::B_Q + s), 1);
+      mbar_init(bar(L::B_QE + s), 1);
       mbar_init(bar(L::B_V + s), 1);
       mbar_init(bar(L::B_VE + s), 1);
       mbar_init(bar(L::B_S + s), 1);
@@ -144,46 +161,56 @@ __global__ void __launch_bounds__(320, 1)
 
   if (warp == 8) {
     // ---------------- TMA producer ----------------
+    // K(i) (i counts every key tile this CTA loads) goes to slot i % 3 once K(i - 3) has been
+    // released, V(i) to slot i % 2 once V(i - 2) has; within a unit K runs one tile ahead of
+    // V. Q tile t of a unit is loaded once the previous unit's last S MMA on it is done.
     if (lane == 0) {
-      for (int t = 0; t < 2; ++t) {
-        if (!tv[t]) continue;
-        mbar_expect_tx(bar(L::B_Q + t), L::kTile);
-        load_tile<D>(sbase + L::kQ + t * L::kTile, &tmQ, &tmQ8, bar(L::B_Q + t), b, h,
-                     rolled_tile_runs(qt[t] * kTileRows, shift_h, p.N), p.N);
-      }
-      // K(j) is loaded into slot j % 3 once K(j - 3) has been released, V(j) into slot j % 2
-      // once V(j - 2) has; K runs one tile ahead of V.
-      int k_issued = 0, v_issued = 0;
-      auto issue_k = [&]() -> bool {
+      int k_issued = 0, v_issued = 0, q_loads[2] = {0, 0};
+      bool ok = true;
+      auto issue_k = [&](const FwdUnit& u, int j) -> bool {
         const int i = k_issued, st = i % L::kKStages;
         if (i >= L::kKStages &&
             !wait_bar(bar(L::B_KE + st), ((i / L::kKStages) - 1) & 1, ctx, 1))
           return false;
         mbar_expect_tx(bar(L::B_K + st), L::kTile);
-        load_tile<D>(sbase + L::kK + st * L::kTile, &tmK, &tmK8, bar(L::B_K + st), b, kvh,
-                     rolled_tile_runs((kv_lo + i) * kTileRows, shift_h, p.N), p.N);
+        load_tile<D>(sbase + L::kK + st * L::kTile, &tmK, &tmK8, bar(L::B_K + st), u.b, u.kvh,
+                     rolled_tile_runs((u.kv_lo + j) * kTileRows, u.shift_h, p.N), p.N);
         ++k_issued;
         return true;
       };
-      auto issue_v = [&]() -> bool {
+      auto issue_v = [&](const FwdUnit& u, int j) -> bool {
         const int i = v_issued, st = i % L::kVStages;
         if (i >= L::kVStages &&
             !wait_bar(bar(L::B_VE + st), ((i / L::kVStages) - 1) & 1, ctx, 9))
           return false;
         mbar_expect_tx(bar(L::B_V + st), L::kTile);
-        load_tile<D>(sbase + L::kV + st * L::kTile, &tmV, &tmV8, bar(L::B_V + st), b, kvh,
-                     rolled_tile_runs((kv_lo + i) * kTileRows, shift_h, p.N), p.N);
+        load_tile<D>(sbase + L::kV + st * L::kTile, &tmV, &tmV8, bar(L::B_V + st), u.b, u.kvh,
+                     rolled_tile_runs((u.kv_lo + j) * kTileRows, u.shift_h, p.N), p.N);
         ++v_issued;
         return true;
       };
-      bool ok = issue_k();
-      for (int j = 0; ok && j < n_kv; ++j) {
-        if (j + 1 < n_kv) ok = issue_k();
-        if (ok) ok = issue_v();
+      for (int unit = blockIdx.x; ok && unit < n_units; unit += gridDim.x) {
+        const FwdUnit u = fwd_unit(p, unit);
+        ok = issue_k(u, 0);   // the first key tile can stream while the last unit finishes
+        for (int t = 0; ok && t < 2; ++t) {
+          if (!u.tv[t]) continue;
+          if (q_loads[t] > 0 && !wait_bar(bar(L::B_QE + t), (q_loads[t] - 1) & 1, ctx, 10)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(bar(L::B_Q + t), L::kTile);
+          load_tile<D>(sbase + L::kQ + t * L::kTile, &tmQ, &tmQ8, bar(L::B_Q + t), u.b, u.h,
+                       rolled_tile_runs(u.qt[t] * kTileRows, u.shift_h, p.N), p.N);
+          ++q_loads[t];
+        }
+        for (int j = 0; ok && j < u.n_kv; ++j) {
+          if (j + 1 < u.n_kv) ok = issue_k(u, j + 1);
+          if (ok) ok = issue_v(u, j);
+        }
       }
       // Every issued copy lands before the CTA can exit.
       for (int t = 0; t < 2; ++t)
-        if (tv[t]) drain_wait(bar(L::B_Q + t), 0, p.timeout_ns);
+        if (q_loads[t] > 0) drain_wait(bar(L::B_Q + t), (q_loads[t] - 1) & 1, p.timeout_ns);
       for (int i = k_issued - L::kKStages; i < k_issued; ++i)
         if (i >= 0) drain_wait(bar(L::B_K + i % L::kKStages), (i / L::kKStages) & 1, p.timeout_ns);
       for (int i = v_issued - L::kVStages; i < v_issued; ++i)
@@ -194,85 +221,100 @@ __global__ void __launch_bounds__(320, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16(128, 128, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16(128, D, false, true);
-      bool q_ready[2] = {false, false};
-      int pcount[2] = {0, 0};
+      int k_used = 0, v_used = 0, q_used[2] = {0, 0}, pcount[2] = {0, 0};
       bool ok = true;
-      auto issue_s = [&](int t, int j) -> bool {
-        if (!q_ready[t]) {
-          if (!wait_bar(bar(L::B_Q + t), 0, ctx, 2)) return false;
-          q_ready[t] = true;
-        }
-        tc_fence_after();
-        const uint32_t q_base = sbase + L::kQ + t * L::kTile;
-        const uint32_t k_base = sbase + L::kK + (j % L::kKStages) * L::kTile;
+      auto wait_k = [&](int i) {
+        return wait_bar(bar(L::B_K + i % L::kKStages), (i / L::kKStages) & 1, ctx, 3);
+      };
+      for (int unit = blockIdx.x; ok && unit < n_units; unit += gridDim.x) {
+        const FwdUnit u = fwd_unit(p, unit);
+        bool q_ready[2] = {false, false}, first_pv[2] = {true, true};
+        // S_t(j) = Q_t K(j)^T into TMEM columns [128 t, 128 t + 128).
+        auto issue_s = [&](int t, int kidx) -> bool {
+          if (!q_ready[t]) {
+            if (!wait_bar(bar(L::B_Q + t), q_used[t] & 1, ctx, 2)) return false;
+            q_ready[t] = true;
+            ++q_used[t];
+          }
+          tc_fence_after();
+          const uint32_t q_base = sbase + L::kQ + t * L::kTile;
+          const uint32_t k_base = sbase + L::kK + (kidx % L::kKStages) * L::kTile;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk / 4) * Tile<D>::kHalfBytes + (kk % 4) * 32;
-          mma_ss(tmem + t * 128, sdesc_sw128(q_base + off, 16, 1024),
-                 sdesc_sw128(k_base + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
-        }
-        mma_commit(bar(L::B_S + t));
-        return true;
-      };
-      auto wait_k = [&](int j) {
-        return wait_bar(bar(L::B_K + j % L::kKStages), (j / L::kKStages) & 1, ctx, 3);
-      };
-      // S for key tile 0, then release of its K slot once both S MMAs are done.
-      if (!wait_k(0)) ok = false;
-      for (int t = 0; ok && t < 2; ++t)
-        if (part(t, kv_lo)) ok = issue_s(t, 0);
-      if (ok) mma_commit(bar(L::B_KE + 0));
-      for (int j = 0; ok && j < n_kv; ++j) {
-        const int kt = kv_lo + j, vst = j % L::kVStages;
-        const bool next = j + 1 < n_kv;
-        bool v_ready = false, k_next_ready = false;
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk / 4) * Tile<D>::kHalfBytes + (kk % 4) * 32;
+            mma_ss(tmem + t * 128, sdesc_sw128(q_base + off, 16, 1024),
+                   sdesc_sw128(k_base + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(bar(L::B_S + t));
+          return true;
+        };
+        const int k0 = k_used, v0 = v_used;
+        if (!wait_k(k0)) { ok = false; break; }
         for (int t = 0; ok && t < 2; ++t) {
-          if (part(t, kt)) {
-            if (!wait_bar(bar(L::B_P + t), pcount[t] & 1, ctx, 4)) { ok = false; break; }
-            if (!v_ready) {
-              if (!wait_bar(bar(L::B_V + vst), (j / L::kVStages) & 1, ctx, 5)) { ok = false; break; }
-              v_ready = true;
-            }
-            tc_fence_after();
-            const uint32_t v_base = sbase + L::kV + vst * L::kTile;
-#pragma unroll
-            for (int kk = 0; kk < kTileRows / 16; ++kk)
-              mma_ts(tmem + 256 + t * D, tmem + t * 128 + kk * 8,
-                     sdesc_sw128(v_base + kk * 2048, Tile<D>::kHalfBytes, 1024), idesc_pv,
-                     (pcount[t] > 0 || kk > 0) ? 1u : 0u);
-            ++pcount[t];
-            if (kt == ke[t]) mma_commit(bar(L::B_ODONE + t));
-          }
-          if (t == 1) mma_commit(bar(L::B_VE + vst));   // V(j) has no reader left
-          if (next && part(t, kt + 1)) {
-            if (!k_next_ready) {
-              if (!wait_k(j + 1)) { ok = false; break; }
-              k_next_ready = true;
-            }
-            if (!issue_s(t, j + 1)) { ok = false; break; }
-          }
+          if (!u.part(t, u.kv_lo)) continue;
+          ok = issue_s(t, k0);
+          if (ok && u.kv_lo == u.ke[t]) mma_commit(bar(L::B_QE + t));   // last S on Q_t
         }
-        if (ok && next) mma_commit(bar(L::B_KE + (j + 1) % L::kKStages));   // K(j+1) likewise
+        if (!ok) break;
+        mma_commit(bar(L::B_KE + k0 % L::kKStages));
+        for (int j = 0; ok && j < u.n_kv; ++j) {
+          const int kt = u.kv_lo + j, vi = v0 + j, vst = vi % L::kVStages;
+          const bool next = j + 1 < u.n_kv;
+          bool v_ready = false, k_next_ready = false;
+          for (int t = 0; ok && t < 2; ++t) {
+            if (u.part(t, kt)) {
+              if (!wait_bar(bar(L::B_P + t), pcount[t] & 1, ctx, 4)) { ok = false; break; }
+              if (!v_ready) {
+                if (!wait_bar(bar(L::B_V + vst), (vi / L::kVStages) & 1, ctx, 5)) { ok = false; break; }
+                v_ready = true;
+              }
+              tc_fence_after();
+              const uint32_t v_base = sbase + L::kV + vst * L::kTile;
+#pragma unroll
+              for (int kk = 0; kk < kTileRows / 16; ++kk)
+                mma_ts(tmem + 256 + t * D, tmem + t * 128 + kk * 8,
+                       sdesc_sw128(v_base + kk * 2048, Tile<D>::kHalfBytes, 1024), idesc_pv,
+                       (!first_pv[t] || kk > 0) ? 1u : 0u);
+              first_pv[t] = false;
+              ++pcount[t];
+              if (kt == u.ke[t]) mma_commit(bar(L::B_ODONE + t));
+            }
+            if (t == 1) mma_commit(bar(L::B_VE + vst));   // V(j) has no reader left
+            if (next && u.part(t, kt + 1)) {
+              if (!k_next_ready) {
+                if (!wait_k(k0 + j + 1)) { ok = false; break; }
+                k_next_ready = true;
+              }
+              if (!issue_s(t, k0 + j + 1)) { ok = false; break; }
+              if (kt + 1 == u.ke[t]) mma_commit(bar(L::B_QE + t));   // last S on Q_t
+            }
+          }
+          if (ok && next) mma_commit(bar(L::B_KE + (k0 + j + 1) % L::kKStages));
+        }
+        k_used = k0 + u.n_kv;
+        v_used = v0 + u.n_kv;
       }
     }
   } else {
     // ---------------- softmax warpgroups ----------------
     const int wg = warp / 4;
-    if (tv[wg]) {
-      const int row = threadIdx.x % 128;
-      const int r = qt[wg] * kTileRows + row;
+    const int row = threadIdx.x % 128;
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>((warp % 4) * 32) << 16);
+    const uint32_t s_col = t_lane + wg * 128;
+    const uint32_t o_col = t_lane + 256 + wg * D;
+    const float c = p.scale_log2;
+    int s_cnt = 0, o_cnt = 0;
+    bool ok = true;
+    for (int unit = blockIdx.x; ok && unit < n_units; unit += gridDim.x) {
+      const FwdUnit u = fwd_unit(p, unit);
+      if (!u.tv[wg]) continue;
+      const int r = u.qt[wg] * kTileRows + row;
       const bool row_valid = r < p.N;
-      const int lo = row_valid ? group_begin(r, p.G) : kb[wg] * kTileRows;
-      const int hi = row_valid ? r : kb[wg] * kTileRows;
-      const uint32_t t_lane = tmem + (static_cast<uint32_t>((warp % 4) * 32) << 16);
-      const uint32_t s_col = t_lane + wg * 128;
-      const uint32_t o_col = t_lane + 256 + wg * D;
-      const float c = p.scale_log2;
+      const int lo = row_valid ? group_begin(r, p.G) : u.kb[wg] * kTileRows;
+      const int hi = row_valid ? r : u.kb[wg] * kTileRows;
       float m_run = -INFINITY, l_run = 0.f;
-      bool ok = true;
-      int cnt = 0;
-      for (int kt = kb[wg]; kt <= ke[wg]; ++kt, ++cnt) {
-        if (!warp_wait(bar(L::B_S + wg), cnt & 1, ctx, 7)) { ok = false; break; }
+      for (int kt = u.kb[wg], cnt = 0; kt <= u.ke[wg]; ++kt, ++cnt, ++s_cnt) {
+        if (!warp_wait(bar(L::B_S + wg), s_cnt & 1, ctx, 7)) { ok = false; break; }
         tc_fence_after();
         float s[128];
         {
@@ -329,29 +371,35 @@ __global__ void __launch_bounds__(320, 1)
         tc_fence_before();
         mbar_arrive(bar(L::B_P + wg));
       }
-      if (ok && warp_wait(bar(L::B_ODONE + wg), 0, ctx, 8)) {
-        tc_fence_after();
-        const float inv_l = 1.f / l_run;
-        const long long tt = static_cast<long long>(r) + shift_h;
-        const int t = static_cast<int>(tt >= p.N ? tt - p.N : tt);
-        __nv_bfloat16* orow =
-            p.o + ((static_cast<size_t>(b) * p.N + (row_valid ? t : 0)) * p.Hq + h) * D;
-        uint32_t ov[D];
-        if constexpr (D == 128) tmem_ld128(o_col, ov); else tmem_ld64(o_col, ov);
+      if (!ok || !warp_wait(bar(L::B_ODONE + wg), o_cnt & 1, ctx, 8)) { ok = false; break; }
+      ++o_cnt;
+      tc_fence_after();
+      const float inv_l = 1.f / l_run;
+      const long long tt = static_cast<long long>(r) + u.shift_h;
+      const int t = static_cast<int>(tt >= p.N ? tt - p.N : tt);
+      __nv_bfloat16* orow =
+          p.o + ((static_cast<size_t>(u.b) * p.N + (row_valid ? t : 0)) * p.Hq + u.h) * D;
+#pragma unroll
+      for (int j = 0; j < D / 32; ++j) {
+        uint32_t ov[32];
+        tmem_ld32(o_col + 32 * j, ov);
         if (row_valid) {
 #pragma unroll
-          for (int v = 0; v < D / 8; ++v) {
+          for (int v = 0; v < 4; ++v) {
             uint4 w4;
             w4.x = pack_bf16(__uint_as_float(ov[8 * v + 0]) * inv_l, __uint_as_float(ov[8 * v + 1]) * inv_l);
             w4.y = pack_bf16(__uint_as_float(ov[8 * v + 2]) * inv_l, __uint_as_float(ov[8 * v + 3]) * inv_l);
             w4.z = pack_bf16(__uint_as_float(ov[8 * v + 4]) * inv_l, __uint_as_float(ov[8 * v + 5]) * inv_l);
             w4.w = pack_bf16(__uint_as_float(ov[8 * v + 6]) * inv_l, __uint_as_float(ov[8 * v + 7]) * inv_l);
-            reinterpret_cast<uint4*>(orow)[v] = w4;
+            reinterpret_cast<uint4*>(orow + 32 * j)[v] = w4;
           }
-          p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.N + t] =
-              (m_run + __log2f(l_run)) * 0.6931471805599453f;
         }
       }
+      if (row_valid)
+        p.lse[(static_cast<size_t>(u.b) * p.Hq + u.h) * p.N + t] =
+            (m_run + __log2f(l_run)) * 0.6931471805599453f;
+      // O_t is read: the next unit's first PV on it waits for this warpgroup's P anyway.
+      tc_fence_before();
     }
   }
 

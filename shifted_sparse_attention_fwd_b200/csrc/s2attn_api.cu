@@ -36,6 +36,7 @@ struct DeviceState {
   std::once_flag once;
   cudaError_t init_err = cudaSuccess;
   unsigned int* err_word = nullptr;
+  int num_sms = 0;
 };
 DeviceState g_dev[kMaxDevices];
 
@@ -57,7 +58,7 @@ cudaError_t set_smem_attrs() {
 
 // Per-device one-time set-up (with that device current): the device address of the error
 // word, and the kernels' shared-memory limits.
-s2attn_status device_state(unsigned int** err_word) {
+s2attn_status device_state(unsigned int** err_word, int* num_sms = nullptr) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
@@ -72,10 +73,13 @@ s2attn_status device_state(unsigned int** err_word) {
     if (s.init_err == cudaSuccess) s.init_err = cudaMemset(p, 0, sizeof(unsigned int));
     if (s.init_err == cudaSuccess) s.init_err = set_smem_attrs<64>();
     if (s.init_err == cudaSuccess) s.init_err = set_smem_attrs<128>();
+    if (s.init_err == cudaSuccess)
+      s.init_err = cudaDeviceGetAttribute(&s.num_sms, cudaDevAttrMultiProcessorCount, dev);
     s.err_word = static_cast<unsigned int*>(p);
   });
   if (s.init_err != cudaSuccess) return cuda_fail(s.init_err, "device set-up");
   *err_word = s.err_word;
+  if (num_sms) *num_sms = s.num_sms;
   return S2ATTN_OK;
 }
 
@@ -156,7 +160,8 @@ s2attn_status check_shape(int B, int Hq, int Hkv, int N, int d, int G, float sca
 
 template <int D>
 s2attn_status launch_fwd(const Shape& sh, const void* q, const void* k, const void* v, void* o,
-                         float* lse, float scale, cudaStream_t stream, unsigned int* err) {
+                         float* lse, float scale, cudaStream_t stream, unsigned int* err,
+                         int num_sms) {
   MapPair mq, mk, mv;
   s2attn_status s;
   if ((s = encode_pair(mq, q, sh.B, sh.Hq, sh.N, D)) != S2ATTN_OK) return s;
@@ -170,7 +175,8 @@ s2attn_status launch_fwd(const Shape& sh, const void* q, const void* k, const vo
   p.scale_log2 = scale * 1.4426950408889634f;
   p.err = err;
   p.timeout_ns = g_timeout_ns.load();
-  const unsigned grid = static_cast<unsigned>(sh.B) * sh.Hq * s2::query_pairs_per_head(sh.N);
+  const unsigned units = static_cast<unsigned>(sh.B) * sh.Hq * s2::query_pairs_per_head(sh.N);
+  const unsigned grid = units < static_cast<unsigned>(num_sms) ? units : static_cast<unsigned>(num_sms);
   s2::s2_fwd_kernel<D><<<grid, s2::FwdLayout<D>::kThreads, s2::FwdLayout<D>::kLaunchBytes, stream>>>(
       mq.m128, mq.m8, mk.m128, mk.m8, mv.m128, mv.m8, p);
   cudaError_t e = cudaGetLastError();
@@ -223,11 +229,11 @@ s2attn_status launch_grad(const Shape& sh, const void* q, const void* k, const v
   const unsigned tiles = (sh.N + 127) / 128;
   if (kDkdv) {
     const unsigned grid = static_cast<unsigned>(sh.B) * sh.Hkv * tiles;
-    s2::s2_bwd_dkdv_kernel<D><<<grid, 192, s2::DkdvLayout<D>::kLaunchBytes, stream>>>(
+    s2::s2_bwd_dkdv_kernel<D><<<grid, s2::DkdvLayout<D>::kThreads, s2::DkdvLayout<D>::kLaunchBytes, stream>>>(
         mq.m128, mq.m8, mk.m128, mk.m8, mv.m128, mv.m8, mo.m128, mo.m8, p);
   } else {
-    const unsigned grid = static_cast<unsigned>(sh.B) * sh.Hq * tiles;
-    s2::s2_bwd_dq_kernel<D><<<grid, 192, s2::DqLayout<D>::kLaunchBytes, stream>>>(
+    const unsigned grid = static_cast<unsigned>(sh.B) * sh.Hq * s2::query_pairs_per_head(sh.N);
+    s2::s2_bwd_dq_kernel<D><<<grid, s2::DqLayout<D>::kThreads, s2::DqLayout<D>::kLaunchBytes, stream>>>(
         mq.m128, mq.m8, mk.m128, mk.m8, mv.m128, mv.m8, mo.m128, mo.m8, p);
   }
   cudaError_t e = cudaGetLastError();
@@ -308,10 +314,11 @@ s2attn_status s2attn_fwd_ex(const void* q, const void* k, const void* v, void* o
   if (s != S2ATTN_OK) return s;
   if ((s = get_encoder()) != S2ATTN_OK) return s;
   unsigned int* err = nullptr;
-  if ((s = device_state(&err)) != S2ATTN_OK) return s;
+  int num_sms = 0;
+  if ((s = device_state(&err, &num_sms)) != S2ATTN_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return d == 64 ? launch_fwd<64>(sh, q, k, v, o, lse, scale, st, err)
-                 : launch_fwd<128>(sh, q, k, v, o, lse, scale, st, err);
+  return d == 64 ? launch_fwd<64>(sh, q, k, v, o, lse, scale, st, err, num_sms)
+                 : launch_fwd<128>(sh, q, k, v, o, lse, scale, st, err, num_sms);
 }
 
 s2attn_status s2attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
