@@ -161,18 +161,10 @@ __global__ void __launch_bounds__(320, 1)
       for (int hq = h_begin; hq < h_begin + rep; ++hq)
         total += kv_tile_qtiles(t0, head_shift(hq), p.N, p.G).count();
       auto issue_nt = [&](uint32_t d_tmem, uint32_t a_base, uint32_t b_base) {
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk / 4) * Tile<D>::kHalfBytes + (kk % 4) * 32;
-          mma_ss(d_tmem, sdesc_sw128(a_base + off, 16, 1024), sdesc_sw128(b_base + off, 16, 1024),
-                 idesc_s, kk > 0 ? 1u : 0u);
-        }
+        gemm_ss_k<D>(d_tmem, a_base, b_base, idesc_s);
       };
       auto issue_acc = [&](uint32_t d_tmem, uint32_t a_tmem, uint32_t b_base, int n) {
-#pragma unroll
-        for (int kk = 0; kk < kTileRows / 16; ++kk)
-          mma_ts(d_tmem, a_tmem + kk * 8, sdesc_sw128(b_base + kk * 2048, Tile<D>::kHalfBytes, 1024),
-                 idesc_acc, (n > 0 || kk > 0) ? 1u : 0u);
+        gemm_ts_mn<D>(d_tmem, a_tmem, b_base, idesc_acc, n > 0);
       };
       bool ok = wait_bar(bar(L::B_KV), 0, ctx, 2);
       if (ok && total > 0) ok = wait_bar(bar(L::B_QF + 0), 0, ctx, 3);

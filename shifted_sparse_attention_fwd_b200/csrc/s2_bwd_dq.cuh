@@ -6,18 +6,20 @@
 //   dP = dO V^T
 //   dS = P o (dP - D)
 //   dQ = scale * dS K
-// One CTA owns two consecutive 128-row rolled query tiles of one (batch, head) and walks the
-// key tiles the forward walks (group start to diagonal); dQ is written once, without atomics.
+// One CTA owns a 128-row rolled query tile of one (batch, head) and walks the key tiles the
+// forward walks (group start to diagonal); dQ is written once, without atomics.
 //
-// Warp roles (320 threads): warps 0-3 and 4-7 elementwise for query tile 0 and 1 (thread i
-// owns query row i), warp 8 TMA producer (Q and dO of both tiles once; K through a 2-slot
-// ring, V through a 1-slot ring, each slot released right after its last reader), warp 9
+// Warp roles (320 threads): warps 0-7 elementwise — query row i (TMEM lane i) is shared by
+// warp i/32 (key columns 0-63) and warp i/32 + 4 (columns 64-127), so two warps per SM
+// sub-partition work on every tile; warp 8 TMA producer (Q, dO once; K through a 3-slot ring
+// one tile ahead of V's 2-slot ring, each slot released right after its last reader); warp 9
 // TMEM allocator + MMA issuer.
 //
-// TMEM: tile t uses columns R_t = [128 t, 128 t + 128) in turn for S, then dP, then dS (bf16),
-// and dQ_t = [256 + 128 t, 384 + 128 t). P is kept in registers (bf16) between the S and dP
-// phases, which is what frees R_t for dP. The MMA issuer interleaves the tiles
-// (dP0 dP1 dQ0 S0' dQ1 S1' ...) so one tile's elementwise phase overlaps the other's MMAs.
+// TMEM: S double buffer [0,128) and [128,256); dP [256,384); dQ [384,384+D). dS (bf16) is
+// written into the S buffer it came from, at columns [32,96): each column half packs its
+// output inside its own, already consumed, fp32 columns. P stays in registers (bf16) between
+// the S and dS phases. Per key tile the MMA issuer runs dP(n), S(n+1), dQ(n): the P phase
+// overlaps dP(n) and the dS phase overlaps S(n+1).
 #pragma once
 
 #include "s2_bwd_dkdv.cuh"
@@ -28,14 +30,14 @@ namespace s2 {
 template <int D>
 struct DqLayout {
   static constexpr uint32_t kTile = Tile<D>::kBytes;
-  static constexpr int kKStages = 2, kVStages = 1;
-  static constexpr uint32_t kQ = 0;                          // Q0, Q1
-  static constexpr uint32_t kDO = kQ + 2 * kTile;            // dO0, dO1
-  static constexpr uint32_t kK = kDO + 2 * kTile;            // K ring
-  static constexpr uint32_t kV = kK + kKStages * kTile;      // V ring
+  static constexpr int kKStages = 3, kVStages = 2;
+  static constexpr uint32_t kQ = 0;
+  static constexpr uint32_t kDO = kQ + kTile;
+  static constexpr uint32_t kK = kDO + kTile;                 // K ring
+  static constexpr uint32_t kV = kK + kKStages * kTile;       // V ring
   static constexpr uint32_t kBar = kV + kVStages * kTile;
-  enum { B_QD = 0, B_K = 2, B_KE = 4, B_V = 6, B_VE = 7, B_S = 8, B_PF = 10, B_DP = 12,
-         B_DS = 14, B_ACC = 16, B_DRAIN = 18, B_COUNT = 19 };
+  enum { B_QDO = 0, B_K = 1, B_KE = 4, B_V = 7, B_VE = 9, B_S = 11, B_DP = 13, B_DS = 14,
+         B_ACC = 15, B_DRAIN = 16, B_COUNT = 17 };
   static constexpr uint32_t kTmemSlot = kBar + B_COUNT * 8;
   static constexpr uint32_t kAbort = kTmemSlot + 4;
   static constexpr uint32_t kBytes = kAbort + 4;
@@ -61,38 +63,28 @@ __global__ void __launch_bounds__(320, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kTmemSlot);
   const WaitCtx ctx{abort_flag, p.err, p.timeout_ns, KID_DQ};
 
-  // Same work decomposition as the forward: tiles 2*pair and 2*pair + 1 of (b, h).
-  int b, h, pair;
-  query_pair_coords(blockIdx.x, p.B, p.Hq, p.N, p.G, b, h, pair);
-  const int nqt = (p.N + kTileRows - 1) / kTileRows;
+  int b, h, qt;
+  query_tile_coords(blockIdx.x, p.B, p.Hq, p.N, p.G, b, h, qt);
+  const int R0 = qt * kTileRows;
   const int shift_h = h >= p.shift_head_begin ? p.shift : 0;
   const int kvh = h / (p.Hq / p.Hkv);
-  int qt[2], kb[2], ke[2];
-  bool tv[2];
-#pragma unroll
-  for (int t = 0; t < 2; ++t) {
-    qt[t] = 2 * pair + t;
-    tv[t] = qt[t] < nqt;
-    kb[t] = tv[t] ? group_begin(qt[t] * kTileRows, p.G) / kTileRows : 0;
-    ke[t] = qt[t];
-  }
-  const int kv_lo = kb[0];
-  const int n_kv = (tv[1] ? ke[1] : ke[0]) - kv_lo + 1;
-  auto part = [&](int t, int kt) { return tv[t] && kb[t] <= kt && kt <= ke[t]; };
+  const int kt_begin = group_begin(R0, p.G) / kTileRows;
+  const int n_kv = qt - kt_begin + 1;
 
   if (warp == 8 && lane == 0) {
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(bar(L::B_QD + s), 1);
+    mbar_init(bar(L::B_QDO), 1);
+    for (int s = 0; s < L::kKStages; ++s) {
       mbar_init(bar(L::B_K + s), 1);
       mbar_init(bar(L::B_KE + s), 1);
-      mbar_init(bar(L::B_S + s), 1);
-      mbar_init(bar(L::B_PF + s), 128);
-      mbar_init(bar(L::B_DP + s), 1);
-      mbar_init(bar(L::B_DS + s), 128);
-      mbar_init(bar(L::B_ACC + s), 1);
     }
-    mbar_init(bar(L::B_V), 1);
-    mbar_init(bar(L::B_VE), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(L::B_V + s), 1);
+      mbar_init(bar(L::B_VE + s), 1);
+      mbar_init(bar(L::B_S + s), 1);
+    }
+    mbar_init(bar(L::B_DP), 1);
+    mbar_init(bar(L::B_DS), 256);
+    mbar_init(bar(L::B_ACC), 1);
     mbar_init(bar(L::B_DRAIN), 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -109,17 +101,15 @@ __global__ void __launch_bounds__(320, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  const uint32_t tm_dp = tmem + 256, tm_dq = tmem + 384;
 
   if (warp == 8) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
-      for (int t = 0; t < 2; ++t) {
-        if (!tv[t]) continue;
-        const TileRuns q_runs = rolled_tile_runs(qt[t] * kTileRows, shift_h, p.N);
-        mbar_expect_tx(bar(L::B_QD + t), 2 * L::kTile);
-        load_tile<D>(sbase + L::kQ + t * L::kTile, &tmQ, &tmQ8, bar(L::B_QD + t), b, h, q_runs, p.N);
-        load_tile<D>(sbase + L::kDO + t * L::kTile, &tmO, &tmO8, bar(L::B_QD + t), b, h, q_runs, p.N);
-      }
+      const TileRuns q_runs = rolled_tile_runs(R0, shift_h, p.N);
+      mbar_expect_tx(bar(L::B_QDO), 2 * L::kTile);
+      load_tile<D>(sbase + L::kQ, &tmQ, &tmQ8, bar(L::B_QDO), b, h, q_runs, p.N);
+      load_tile<D>(sbase + L::kDO, &tmO, &tmO8, bar(L::B_QDO), b, h, q_runs, p.N);
       int k_issued = 0, v_issued = 0;
       auto issue_k = [&]() -> bool {
         const int i = k_issued, st = i % L::kKStages;
@@ -128,196 +118,143 @@ __global__ void __launch_bounds__(320, 1)
           return false;
         mbar_expect_tx(bar(L::B_K + st), L::kTile);
         load_tile<D>(sbase + L::kK + st * L::kTile, &tmK, &tmK8, bar(L::B_K + st), b, kvh,
-                     rolled_tile_runs((kv_lo + i) * kTileRows, shift_h, p.N), p.N);
+                     rolled_tile_runs((kt_begin + i) * kTileRows, shift_h, p.N), p.N);
         ++k_issued;
         return true;
       };
       auto issue_v = [&]() -> bool {
-        const int i = v_issued;
-        if (i >= L::kVStages && !wait_bar(bar(L::B_VE), (i - 1) & 1, ctx, 11)) return false;
-        mbar_expect_tx(bar(L::B_V), L::kTile);
-        load_tile<D>(sbase + L::kV, &tmV, &tmV8, bar(L::B_V), b, kvh,
-                     rolled_tile_runs((kv_lo + i) * kTileRows, shift_h, p.N), p.N);
+        const int i = v_issued, st = i % L::kVStages;
+        if (i >= L::kVStages &&
+            !wait_bar(bar(L::B_VE + st), ((i / L::kVStages) - 1) & 1, ctx, 10))
+          return false;
+        mbar_expect_tx(bar(L::B_V + st), L::kTile);
+        load_tile<D>(sbase + L::kV + st * L::kTile, &tmV, &tmV8, bar(L::B_V + st), b, kvh,
+                     rolled_tile_runs((kt_begin + i) * kTileRows, shift_h, p.N), p.N);
         ++v_issued;
         return true;
       };
       bool ok = issue_k();
       for (int j = 0; ok && j < n_kv; ++j) {
+        if (j + 1 < n_kv) ok = issue_k();
         if (ok) ok = issue_v();
-        if (ok && j + 1 < n_kv) ok = issue_k();
       }
-      for (int t = 0; t < 2; ++t)
-        if (tv[t]) drain_wait(bar(L::B_QD + t), 0, p.timeout_ns);
+      drain_wait(bar(L::B_QDO), 0, p.timeout_ns);
       for (int i = k_issued - L::kKStages; i < k_issued; ++i)
         if (i >= 0) drain_wait(bar(L::B_K + i % L::kKStages), (i / L::kKStages) & 1, p.timeout_ns);
-      if (v_issued > 0) drain_wait(bar(L::B_V), (v_issued - 1) & 1, p.timeout_ns);
+      for (int i = v_issued - L::kVStages; i < v_issued; ++i)
+        if (i >= 0) drain_wait(bar(L::B_V + i % L::kVStages), (i / L::kVStages) & 1, p.timeout_ns);
     }
   } else if (warp == 9) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16(128, 128, false, false);   // Q K^T, dO V^T
       constexpr uint32_t idesc_dq = idesc_bf16(128, D, false, true);     // dS K
-      bool qd_ready[2] = {false, false}, first_dq[2] = {true, true};
-      int pf_cnt[2] = {0, 0}, ds_cnt[2] = {0, 0};
-      bool ok = true;
-      auto issue_nt = [&](uint32_t d_tmem, uint32_t a_base, uint32_t b_base) {
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk / 4) * Tile<D>::kHalfBytes + (kk % 4) * 32;
-          mma_ss(d_tmem, sdesc_sw128(a_base + off, 16, 1024), sdesc_sw128(b_base + off, 16, 1024),
-                 idesc_s, kk > 0 ? 1u : 0u);
-        }
+      auto wait_k = [&](int j) {
+        return wait_bar(bar(L::B_K + j % L::kKStages), (j / L::kKStages) & 1, ctx, 3);
       };
-      auto ensure_qd = [&](int t) -> bool {
-        if (qd_ready[t]) return true;
-        if (!wait_bar(bar(L::B_QD + t), 0, ctx, 2)) return false;
-        qd_ready[t] = true;
-        return true;
-      };
-      auto wait_k = [&](int i) {
-        return wait_bar(bar(L::B_K + i % L::kKStages), (i / L::kKStages) & 1, ctx, 3);
-      };
-      auto issue_s = [&](int t, int kidx) -> bool {
-        if (!ensure_qd(t)) return false;
+      bool ok = wait_bar(bar(L::B_QDO), 0, ctx, 2);
+      if (ok) ok = wait_k(0);
+      if (ok) {
         tc_fence_after();
-        issue_nt(tmem + t * 128, sbase + L::kQ + t * L::kTile,
-                 sbase + L::kK + (kidx % L::kKStages) * L::kTile);
-        mma_commit(bar(L::B_S + t));
-        return true;
-      };
-      if (!wait_k(0)) ok = false;
-      for (int t = 0; ok && t < 2; ++t)
-        if (part(t, kv_lo)) ok = issue_s(t, 0);
-      for (int j = 0; ok && j < n_kv; ++j) {
-        const int kt = kv_lo + j, kst = j % L::kKStages;
-        const bool next = j + 1 < n_kv;
-        // dP_t(j) = dO_t V(j)^T into R_t once the elementwise warps hold P_t(j) in registers.
-        bool v_ready = false;
-        for (int t = 0; ok && t < 2; ++t) {
-          if (!part(t, kt)) continue;
-          if (!wait_bar(bar(L::B_PF + t), pf_cnt[t] & 1, ctx, 4)) { ok = false; break; }
-          ++pf_cnt[t];
-          if (!v_ready) {
-            if (!wait_bar(bar(L::B_V), j & 1, ctx, 5)) { ok = false; break; }
-            v_ready = true;
-          }
-          tc_fence_after();
-          issue_nt(tmem + t * 128, sbase + L::kDO + t * L::kTile, sbase + L::kV);
-          mma_commit(bar(L::B_DP + t));
-        }
-        if (!ok) break;
-        mma_commit(bar(L::B_VE));   // V(j) has no reader left
-        // dQ_t += dS_t(j) K(j), then S_t(j+1) into R_t.
-        bool k_next_ready = false;
-        for (int t = 0; ok && t < 2; ++t) {
-          if (part(t, kt)) {
-            if (!wait_bar(bar(L::B_DS + t), ds_cnt[t] & 1, ctx, 6)) { ok = false; break; }
-            ++ds_cnt[t];
-            tc_fence_after();
-            const uint32_t k_base = sbase + L::kK + kst * L::kTile;
-#pragma unroll
-            for (int kk = 0; kk < kTileRows / 16; ++kk)
-              mma_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8,
-                     sdesc_sw128(k_base + kk * 2048, Tile<D>::kHalfBytes, 1024), idesc_dq,
-                     (!first_dq[t] || kk > 0) ? 1u : 0u);
-            first_dq[t] = false;
-            if (kt == ke[t]) mma_commit(bar(L::B_ACC + t));
-          }
-          if (next && part(t, kt + 1)) {
-            if (!k_next_ready) {
-              if (!wait_k(j + 1)) { ok = false; break; }
-              k_next_ready = true;
-            }
-            if (!issue_s(t, j + 1)) { ok = false; break; }
-          }
-        }
-        if (ok) mma_commit(bar(L::B_KE + kst));   // K(j): read by S(j) and dQ(j)
+        gemm_ss_k<D>(tmem, sbase + L::kQ, sbase + L::kK, idesc_s);
+        mma_commit(bar(L::B_S + 0));
       }
+      for (int n = 0; ok && n < n_kv; ++n) {
+        const int st = n & 1, kst = n % L::kKStages, vst = n % L::kVStages;
+        if (!wait_bar(bar(L::B_V + vst), (n / L::kVStages) & 1, ctx, 4)) { ok = false; break; }
+        tc_fence_after();
+        gemm_ss_k<D>(tm_dp, sbase + L::kDO, sbase + L::kV + vst * L::kTile, idesc_s);
+        mma_commit(bar(L::B_DP));
+        mma_commit(bar(L::B_VE + vst));   // V(n) has no reader left
+        if (n + 1 < n_kv) {
+          if (!wait_k(n + 1)) { ok = false; break; }
+          tc_fence_after();
+          gemm_ss_k<D>(tmem + ((n + 1) & 1) * 128, sbase + L::kQ,
+                       sbase + L::kK + ((n + 1) % L::kKStages) * L::kTile, idesc_s);
+          mma_commit(bar(L::B_S + ((n + 1) & 1)));
+        }
+        if (!wait_bar(bar(L::B_DS), n & 1, ctx, 6)) { ok = false; break; }
+        tc_fence_after();
+        gemm_ts_mn<D>(tm_dq, tmem + st * 128 + 32, sbase + L::kK + kst * L::kTile, idesc_dq, n > 0);
+        mma_commit(bar(L::B_KE + kst));   // K(n): read by S(n) and dQ(n)
+      }
+      if (ok) mma_commit(bar(L::B_ACC));
     }
   } else {
-    // ---------------- elementwise warpgroups ----------------
-    const int wg = warp / 4;
-    if (tv[wg]) {
-      const int row = threadIdx.x % 128;
-      const int r = qt[wg] * kTileRows + row;
-      const bool row_valid = r < p.N;
-      const int lo = row_valid ? group_begin(r, p.G) : kb[wg] * kTileRows;
-      const int hi = row_valid ? r : kb[wg] * kTileRows;
-      const long long tt = static_cast<long long>(r) + shift_h;
-      const int t = row_valid ? static_cast<int>(tt >= p.N ? tt - p.N : tt) : 0;
-      const size_t lrow = (static_cast<size_t>(b) * p.Hq + h) * p.N + t;
-      const float lse2 = row_valid ? p.lse2[lrow] : 0.f;
-      const float dd = row_valid ? p.dvec[lrow] : 0.f;
-      const uint32_t t_lane = tmem + (static_cast<uint32_t>((warp % 4) * 32) << 16);
-      const uint32_t r_col = t_lane + wg * 128;
-      const uint32_t dq_col = t_lane + 256 + wg * 128;
-      const float c = p.scale_log2;
-      bool ok = true;
-      int cnt = 0;
-      for (int kt = kb[wg]; kt <= ke[wg]; ++kt, ++cnt) {
-        // P phase: S_t(j) -> P (bf16, registers); R_t is then free for dP.
-        if (!warp_wait(bar(L::B_S + wg), cnt & 1, ctx, 7)) { ok = false; break; }
-        tc_fence_after();
-        uint32_t pk[64];
-        {
-          const int cl = lo - kt * kTileRows, ch = hi - kt * kTileRows;
-          const bool mask = __any_sync(0xffffffffu, cl > 0 || ch < kTileRows - 1);
+    // ---------------- elementwise warps 0-7 ----------------
+    const int half = warp / 4;                     // key columns [64 half, 64 half + 64)
+    const int row = (warp % 4) * 32 + lane;
+    const int r = R0 + row;
+    const bool row_valid = r < p.N;
+    const int lo = row_valid ? group_begin(r, p.G) : kt_begin * kTileRows;
+    const int hi = row_valid ? r : kt_begin * kTileRows;
+    const long long tt = static_cast<long long>(r) + shift_h;
+    const int t = row_valid ? static_cast<int>(tt >= p.N ? tt - p.N : tt) : 0;
+    const size_t lrow = (static_cast<size_t>(b) * p.Hq + h) * p.N + t;
+    const float lse2 = row_valid ? p.lse2[lrow] : 0.f;
+    const float dd = row_valid ? p.dvec[lrow] : 0.f;
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>((warp % 4) * 32) << 16);
+    const float c = p.scale_log2;
+    bool ok = true;
+    for (int n = 0; n < n_kv; ++n) {
+      const int st = n & 1;
+      // P phase: 64 columns of S -> P (bf16, registers).
+      if (!warp_wait(bar(L::B_S + st), (n >> 1) & 1, ctx, 7)) { ok = false; break; }
+      tc_fence_after();
+      const int c0 = (kt_begin + n) * kTileRows + 64 * half;
+      const int cl = lo - c0, ch = hi - c0;
+      uint32_t pk[32];
+      {
+        uint32_t raw[64];
+        tmem_ld64(t_lane + st * 128 + 64 * half, raw);
+        const bool mask = __any_sync(0xffffffffu, cl > 0 || ch < 63);
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            uint32_t raw[64];
-            tmem_ld64(r_col + 64 * half, raw);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int col = 64 * half + 2 * i;
-              float e0 = fast_exp2(fmaf(__uint_as_float(raw[2 * i]), c, -lse2));
-              float e1 = fast_exp2(fmaf(__uint_as_float(raw[2 * i + 1]), c, -lse2));
-              if (mask) {
-                e0 = (col < cl || col > ch) ? 0.f : e0;
-                e1 = (col + 1 < cl || col + 1 > ch) ? 0.f : e1;
-              }
-              pk[32 * half + i] = pack_bf16(e0, e1);
-            }
+        for (int e = 0; e < 32; ++e) {
+          const int col = 2 * e;
+          float x0 = fast_exp2(fmaf(__uint_as_float(raw[col]), c, -lse2));
+          float x1 = fast_exp2(fmaf(__uint_as_float(raw[col + 1]), c, -lse2));
+          if (mask) {
+            x0 = (col < cl || col > ch) ? 0.f : x0;
+            x1 = (col + 1 < cl || col + 1 > ch) ? 0.f : x1;
           }
+          pk[e] = pack_bf16(x0, x1);
         }
-        tc_fence_before();
-        mbar_arrive(bar(L::B_PF + wg));
-        // dS phase: dS = P o (dP - D) into R_t (bf16).
-        if (!warp_wait(bar(L::B_DP + wg), cnt & 1, ctx, 8)) { ok = false; break; }
-        tc_fence_after();
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          uint32_t dp[16];
-          tmem_ld16(r_col + 16 * j, dp);
-          uint32_t ds[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float2 pf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[8 * j + e]));
-            ds[e] = pack_bf16(pf.x * (__uint_as_float(dp[2 * e]) - dd),
-                              pf.y * (__uint_as_float(dp[2 * e + 1]) - dd));
-          }
-          tmem_st8(r_col + 8 * j, ds);
-        }
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(bar(L::B_DS + wg));
       }
-      if (ok && warp_wait(bar(L::B_ACC + wg), 0, ctx, 9)) {
-        tc_fence_after();
-        __nv_bfloat16* qrow = p.dq + ((static_cast<size_t>(b) * p.N + t) * p.Hq + h) * D;
+      // dS phase: dS = P o (dP - D), packed into this half's own consumed S columns.
+      if (!warp_wait(bar(L::B_DP), n & 1, ctx, 8)) { ok = false; break; }
+      tc_fence_after();
+      {
+        uint32_t raw[64];
+        tmem_ld64(tm_dp - tmem + t_lane + 64 * half, raw);
+        uint32_t ds[32];
 #pragma unroll
-        for (int j = 0; j < D / 32; ++j) {
-          uint32_t rr[32];
-          tmem_ld32(dq_col + 32 * j, rr);
-          if (row_valid) {
+        for (int e = 0; e < 32; ++e) {
+          const float2 pf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[e]));
+          ds[e] = pack_bf16(pf.x * (__uint_as_float(raw[2 * e]) - dd),
+                            pf.y * (__uint_as_float(raw[2 * e + 1]) - dd));
+        }
+        tmem_st32(t_lane + st * 128 + 32 + 32 * half, ds);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar(L::B_DS));
+    }
+    if (ok && warp_wait(bar(L::B_ACC), 0, ctx, 9)) {
+      tc_fence_after();
+      __nv_bfloat16* qrow = p.dq + ((static_cast<size_t>(b) * p.N + t) * p.Hq + h) * D;
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              uint4 w4;
-              w4.x = pack_bf16(__uint_as_float(rr[8 * v + 0]) * p.scale, __uint_as_float(rr[8 * v + 1]) * p.scale);
-              w4.y = pack_bf16(__uint_as_float(rr[8 * v + 2]) * p.scale, __uint_as_float(rr[8 * v + 3]) * p.scale);
-              w4.z = pack_bf16(__uint_as_float(rr[8 * v + 4]) * p.scale, __uint_as_float(rr[8 * v + 5]) * p.scale);
-              w4.w = pack_bf16(__uint_as_float(rr[8 * v + 6]) * p.scale, __uint_as_float(rr[8 * v + 7]) * p.scale);
-              reinterpret_cast<uint4*>(qrow + 32 * j)[v] = w4;
-            }
+      for (int j = half * (D / 64); j < (half + 1) * (D / 64); ++j) {
+        uint32_t rr[32];
+        tmem_ld32(tm_dq - tmem + t_lane + 32 * j, rr);
+        if (row_valid) {
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            uint4 w4;
+            w4.x = pack_bf16(__uint_as_float(rr[8 * v + 0]) * p.scale, __uint_as_float(rr[8 * v + 1]) * p.scale);
+            w4.y = pack_bf16(__uint_as_float(rr[8 * v + 2]) * p.scale, __uint_as_float(rr[8 * v + 3]) * p.scale);
+            w4.z = pack_bf16(__uint_as_float(rr[8 * v + 4]) * p.scale, __uint_as_float(rr[8 * v + 5]) * p.scale);
+            w4.w = pack_bf16(__uint_as_float(rr[8 * v + 6]) * p.scale, __uint_as_float(rr[8 * v + 7]) * p.scale);
+            reinterpret_cast<uint4*>(qrow + 32 * j)[v] = w4;
           }
         }
       }

@@ -38,6 +38,32 @@ __device__ __forceinline__ void load_tile(uint32_t dst, const CUtensorMap* m128,
   }
 }
 
+// Whole-tile GEMMs issued by the MMA thread. Operand descriptors are built once per call and
+// advanced by constant offsets: the tensor core's issue queue is only a few instructions
+// deep, so per-instruction scalar work in the issuing thread shows up as tensor-core idle time.
+//
+// D[128 x 128] (+)= A[128 x D] * B[128 x D]^T, both operands 128-row K-major tiles (SW128).
+template <int D>
+__device__ __forceinline__ void gemm_ss_k(uint32_t d_tmem, uint32_t a_base, uint32_t b_base,
+                                          uint32_t idesc) {
+  const uint64_t a0 = sdesc_sw128(a_base, 16, 1024), b0 = sdesc_sw128(b_base, 16, 1024);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint64_t off = static_cast<uint64_t>(((kk / 4) * Tile<D>::kHalfBytes + (kk % 4) * 32) >> 4);
+    mma_ss(d_tmem, a0 + off, b0 + off, idesc, kk > 0 ? 1u : 0u);
+  }
+}
+// D[128 x D] (+)= A[128 x 128 bf16, in TMEM] * B[128 (K) x D], B an MN-major tile (SW128).
+template <int D>
+__device__ __forceinline__ void gemm_ts_mn(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_base,
+                                           uint32_t idesc, bool accumulate) {
+  const uint64_t b0 = sdesc_sw128(b_base, Tile<D>::kHalfBytes, 1024);
+#pragma unroll
+  for (int kk = 0; kk < kTileRows / 16; ++kk)
+    mma_ts(d_tmem, a_tmem + kk * 8, b0 + static_cast<uint64_t>((kk * 2048) >> 4), idesc,
+           (accumulate || kk > 0) ? 1u : 0u);
+}
+
 // Wait used only while tearing down: ignores the abort flag, bounded by the timeout.
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity,
                                            unsigned long long timeout_ns) {

@@ -237,14 +237,8 @@ __global__ void __launch_bounds__(320, 1)
             ++q_used[t];
           }
           tc_fence_after();
-          const uint32_t q_base = sbase + L::kQ + t * L::kTile;
-          const uint32_t k_base = sbase + L::kK + (kidx % L::kKStages) * L::kTile;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk / 4) * Tile<D>::kHalfBytes + (kk % 4) * 32;
-            mma_ss(tmem + t * 128, sdesc_sw128(q_base + off, 16, 1024),
-                   sdesc_sw128(k_base + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
-          }
+          gemm_ss_k<D>(tmem + t * 128, sbase + L::kQ + t * L::kTile,
+                       sbase + L::kK + (kidx % L::kKStages) * L::kTile, idesc_qk);
           mma_commit(bar(L::B_S + t));
           return true;
         };
@@ -269,12 +263,8 @@ __global__ void __launch_bounds__(320, 1)
                 v_ready = true;
               }
               tc_fence_after();
-              const uint32_t v_base = sbase + L::kV + vst * L::kTile;
-#pragma unroll
-              for (int kk = 0; kk < kTileRows / 16; ++kk)
-                mma_ts(tmem + 256 + t * D, tmem + t * 128 + kk * 8,
-                       sdesc_sw128(v_base + kk * 2048, Tile<D>::kHalfBytes, 1024), idesc_pv,
-                       (!first_pv[t] || kk > 0) ? 1u : 0u);
+              gemm_ts_mn<D>(tmem + 256 + t * D, tmem + t * 128, sbase + L::kV + vst * L::kTile,
+                            idesc_pv, !first_pv[t]);
               first_pv[t] = false;
               ++pcount[t];
               if (kt == u.ke[t]) mma_commit(bar(L::B_ODONE + t));

@@ -232,7 +232,7 @@ s2attn_status launch_grad(const Shape& sh, const void* q, const void* k, const v
     s2::s2_bwd_dkdv_kernel<D><<<grid, s2::DkdvLayout<D>::kThreads, s2::DkdvLayout<D>::kLaunchBytes, stream>>>(
         mq.m128, mq.m8, mk.m128, mk.m8, mv.m128, mv.m8, mo.m128, mo.m8, p);
   } else {
-    const unsigned grid = static_cast<unsigned>(sh.B) * sh.Hq * s2::query_pairs_per_head(sh.N);
+    const unsigned grid = static_cast<unsigned>(sh.B) * sh.Hq * tiles;
     s2::s2_bwd_dq_kernel<D><<<grid, s2::DqLayout<D>::kThreads, s2::DqLayout<D>::kLaunchBytes, stream>>>(
         mq.m128, mq.m8, mk.m128, mk.m8, mv.m128, mv.m8, mo.m128, mo.m8, p);
   }
