@@ -1,7 +1,8 @@
 """Throughput of S²-Attn forward + backward on B200 (TFLOP/s, fraction of dense-BF16 peak).
 
 One step = one pass of the whole hot path over one batch: forward (O, LSE), backward
-preprocess (D), dK/dV and dQ kernels, all through the C ABI. FLOPs are algorithmic:
+preprocess (D), the dK/dV kernel (which also hands its bf16 dS tiles to the dQ pass) and the
+dQ kernel (dQ = scale * dS K over those tiles), all through the C ABI. FLOPs are algorithmic:
 7 * B * Hq * N * G * d per fwd+bwd (causal half of each G x G group; fwd 2, bwd 5).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--workload NAME]
@@ -40,7 +41,12 @@ def fwd_bwd_flops(w) -> float:
 
 def kernel_flops(w):
     unit = float(w.B) * w.Hq * w.N * w.G * w.d   # one causal in-group GEMM over all heads
-    return {"s2_fwd": 2 * unit, "s2_bwd_dkdv": 4 * unit, "s2_bwd_dq": 1 * unit}
+    return {"s2_fwd": 2 * unit, "s2_bwd_dkdv": 4 * unit, "s2_bwd_dq_ds": 1 * unit}
+
+
+def dq_ds_bytes(w, ds_tiles) -> float:
+    # dS tiles read once (32 KB each), K read once, dQ written once (bf16)
+    return ds_tiles * 32768.0 + 2.0 * w.B * w.N * w.Hkv * w.d + 2.0 * w.B * w.N * w.Hq * w.d
 
 
 def pre_bytes(w) -> float:
@@ -168,7 +174,10 @@ def run_gpu(args, rank, world, local_rank):
     o = torch.empty_like(qd)
     lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=dev)
     dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
-    ws = torch.empty(s2.s2attn_bwd_workspace_size(w.B, w.Hq, w.N), dtype=torch.uint8, device=dev)
+    ws_min = s2.s2attn_bwd_workspace_size(w.B, w.Hq, w.N)
+    ws_bytes = s2.s2attn_bwd_workspace_size_ex(w.B, w.Hq, w.Hkv, w.N, w.d, w.G)
+    ds_tiles = (ws_bytes - ws_min) // 32768
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
     def step(ev=None):
@@ -177,9 +186,9 @@ def run_gpu(args, rank, world, local_rank):
         if ev: ev[1].record(stream)
         s2.s2attn_bwd_preprocess(o, lse, dod, ws)
         if ev: ev[2].record(stream)
-        s2.s2attn_bwd_dkdv(qd, kd, vd, dod, dk, dv, w.G, ws, w.scale)
+        s2.s2attn_bwd_dkdv_ds(qd, kd, vd, dod, dk, dv, w.G, ws, w.scale)
         if ev: ev[3].record(stream)
-        s2.s2attn_bwd_dq(qd, kd, vd, dod, dq, w.G, ws, w.scale)
+        s2.s2attn_bwd_dq_ds(kd, dq, w.G, ws, w.scale)
         if ev: ev[4].record(stream)
 
     for _ in range(args.warmup):
@@ -204,7 +213,7 @@ def run_gpu(args, rank, world, local_rank):
     st, code = s2.s2attn_get_device_error()
     if st != s2.S2ATTN_OK:
         raise RuntimeError(f"device error {st} code {code:#x} in the timed region")
-    names = ["s2_fwd", "s2_bwd_pre", "s2_bwd_dkdv", "s2_bwd_dq"]
+    names = ["s2_fwd", "s2_bwd_pre", "s2_bwd_dkdv", "s2_bwd_dq_ds"]
     per_k = {n: [e[j].elapsed_time(e[j + 1]) for e in evs] for j, n in enumerate(names)}
     step_ms = [e[0].elapsed_time(e[4]) for e in evs]
     total_ms = sum(step_ms)
@@ -219,7 +228,8 @@ def run_gpu(args, rank, world, local_rank):
     def e2e_step():
         for dst, src in ((qd, hq_), (kd, hk_), (vd, hv_), (dod, hdo_)):
             dst.copy_(src, non_blocking=True)
-        step()
+        s2.s2attn_fwd(qd, kd, vd, o, lse, w.G, w.scale)
+        s2.s2attn_bwd(qd, kd, vd, o, lse, dod, dq, dk, dv, w.G, w.scale, workspace=ws)
         for dst, src in ((ho, o), (hlse, lse), (hdq, dq), (hdk, dk), (hdv, dv)):
             dst.copy_(src, non_blocking=True)
 
@@ -271,9 +281,11 @@ def run_gpu(args, rank, world, local_rank):
         if n in kflops:
             tf = kflops[n] / (avg[n] * 1e-3) / 1e12
             entry.update(tflops_algorithmic=round(tf, 1), frac=round(tf / peak_tf, 4))
-        else:
-            gbs = pre_bytes(w) / (avg[n] * 1e-3) / 1e9
-            entry.update(gbs=round(gbs, 1))
+        if n == "s2_bwd_pre":
+            entry.update(gbs=round(pre_bytes(w) / (avg[n] * 1e-3) / 1e9, 1))
+        if n == "s2_bwd_dq_ds":
+            entry.update(gbs=round(dq_ds_bytes(w, ds_tiles) / (avg[n] * 1e-3) / 1e9, 1),
+                         ds_tiles=int(ds_tiles))
         kern[n] = entry
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,

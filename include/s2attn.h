@@ -94,15 +94,34 @@ S2ATTN_API s2attn_status s2attn_fwd_ex(const void* q, const void* k, const void*
                             int B, int Hq, int Hkv, int N, int d, int G, float scale,
                             int shift_head_begin, int shift, void* stream);
 
-/* Bytes of device workspace s2attn_bwd needs: two fp32 [B, Hq, N] arrays (D and LSE in
- * base 2), each rounded up to 256 bytes. */
+/* Smallest device workspace s2attn_bwd accepts: two fp32 [B, Hq, N] arrays (D and LSE in
+ * base 2), each rounded up to 256 bytes. With only this much the dQ kernel recomputes S and
+ * dP (three GEMMs for one gradient). */
 S2ATTN_API size_t s2attn_bwd_workspace_size(int B, int Hq, int N);
 
 /*
+ * Workspace that lets s2attn_bwd skip that recomputation: the minimum above plus room for
+ * the bf16 dS tiles (128 x 128, 32 KB each) that the dK/dV kernel hands to the dQ kernel,
+ * one per (batch, query head, rolled query tile, original kv tile it reads) — about
+ * B * Hq * (N/128) * (G/128 + 1) / 2 tiles when G and the roll are multiples of 128, and
+ * B * Hq * (N/128) * (largest such count) otherwise. cap_bytes = 0 returns the size for all
+ * kv heads in one pass; otherwise the largest size <= cap_bytes that holds a whole number of
+ * kv heads (at least one, even if that exceeds the cap): s2attn_bwd then runs the dK/dV and
+ * dQ kernels once per group of that many kv heads. Returns 0 for arguments s2attn_bwd_ex
+ * would reject.
+ */
+S2ATTN_API size_t s2attn_bwd_workspace_size_ex(int B, int Hq, int Hkv, int N, int d, int G,
+                                               int shift_head_begin, int shift, size_t cap_bytes);
+
+/*
  * Backward: dq, dk, dv from q, k, v, the forward's o and lse, and the upstream dO.
- * Runs, in order on `stream`: the preprocess D = rowsum(dO o O), the dK/dV kernel and the
- * dQ kernel. `workspace` (device, 256-byte aligned, >= s2attn_bwd_workspace_size bytes)
- * is scratch owned by the caller; its contents on entry do not matter.
+ * Runs, in order on `stream`: the preprocess D = rowsum(dO o O), then the dK/dV kernel and
+ * a dQ kernel. `workspace` (device, 256-byte aligned, >= s2attn_bwd_workspace_size bytes)
+ * is scratch owned by the caller; its contents on entry do not matter. If it also holds the
+ * dS tiles of at least one kv head (s2attn_bwd_workspace_size_ex), the dK/dV kernel stores
+ * dS there and the dQ kernel is a plain GEMM over them, repeated per group of kv heads that
+ * fits; otherwise the dQ kernel recomputes S and dP. Both give the same gradients up to
+ * fp32 summation order.
  * dk and dv are the sums over the query heads sharing each kv head.
  */
 S2ATTN_API s2attn_status s2attn_bwd(const void* q, const void* k, const void* v, const void* o,
@@ -138,6 +157,24 @@ S2ATTN_API s2attn_status s2attn_bwd_dq(const void* q, const void* k, const void*
                             size_t workspace_bytes, void* stream);
 
 /*
+ * The two gradient stages of the dS hand-off, one kv-head group covering all kv heads: the
+ * workspace must be at least s2attn_bwd_workspace_size_ex(..., cap_bytes = 0) bytes, else
+ * S2ATTN_ERR_INVALID_ARG. Run s2attn_bwd_preprocess, then, on the same stream and with the
+ * same workspace:
+ *   s2attn_bwd_dkdv_ds  dk, dv and the dS tiles <- from q, k, v, dO and D, LSE2
+ *   s2attn_bwd_dq_ds    dq                      <- from k and the dS tiles
+ */
+S2ATTN_API s2attn_status s2attn_bwd_dkdv_ds(const void* q, const void* k, const void* v,
+                                            const void* dO, void* dk, void* dv, int B, int Hq,
+                                            int Hkv, int N, int d, int G, float scale,
+                                            int shift_head_begin, int shift, void* workspace,
+                                            size_t workspace_bytes, void* stream);
+S2ATTN_API s2attn_status s2attn_bwd_dq_ds(const void* k, void* dq, int B, int Hq, int Hkv, int N,
+                                          int d, int G, float scale, int shift_head_begin,
+                                          int shift, const void* workspace,
+                                          size_t workspace_bytes, void* stream);
+
+/*
  * Backward without a caller-provided workspace, for callers that cannot allocate device
  * memory: plugin hosts whose fixed call signature carries no scratch buffer, or code on a
  * latency-critical path that must not call cudaMalloc (which can synchronise the device and
@@ -145,8 +182,8 @@ S2ATTN_API s2attn_status s2attn_bwd_dq(const void* q, const void* k, const void*
  * this entry point; it exists only for such callers.
  *
  * Same arguments and results as s2attn_bwd, minus the workspace. The scratch (D and
- * LSE * log2(e), 8 bytes per (batch, head, token) row) lives in a 16 MiB array compiled into
- * the library: B * Hq * N may be at most 2,097,152, larger shapes are rejected with
+ * LSE * log2(e), 8 bytes per (batch, head, token) row, and the dS tiles of the dQ pass when
+ * one kv head's fit in the rest) lives in a 16 MiB array compiled into the library: B * Hq * N may be at most 2,097,152, larger shapes are rejected with
  * S2ATTN_ERR_UNSUPPORTED (message in s2attn_last_error) before anything is launched. Every
  * device that loads the library holds that array until the process exits. The first call on
  * a device, with that device current, looks up the array's device address; make that first

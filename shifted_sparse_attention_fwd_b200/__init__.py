@@ -18,9 +18,13 @@ from ._lib import (  # noqa: F401
     s2attn_fwd,
     s2attn_bwd,
     s2attn_bwd_workspace_size,
+    s2attn_bwd_workspace_size_ex,
+    DEFAULT_WORKSPACE_CAP,
     s2attn_bwd_preprocess,
     s2attn_bwd_dkdv,
     s2attn_bwd_dq,
+    s2attn_bwd_dkdv_ds,
+    s2attn_bwd_dq_ds,
     s2attn_bwd_noalloc,
     s2attn_get_device_error,
     s2attn_set_wait_timeout_ns,

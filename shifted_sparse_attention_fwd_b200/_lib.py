@@ -40,6 +40,9 @@ SIGNATURES = {
     "s2attn_bwd_dkdv": (_I, [_P] * 6 + [_I] * 6 + [_F, _I, _I, _P, _Z, _P]),
     "s2attn_bwd_dq": (_I, [_P] * 5 + [_I] * 6 + [_F, _I, _I, _P, _Z, _P]),
     "s2attn_bwd_noalloc": (_I, [_P] * 9 + [_I] * 6 + [_F, _P]),
+    "s2attn_bwd_workspace_size_ex": (_Z, [_I] * 8 + [_Z]),
+    "s2attn_bwd_dkdv_ds": (_I, [_P] * 6 + [_I] * 6 + [_F, _I, _I, _P, _Z, _P]),
+    "s2attn_bwd_dq_ds": (_I, [_P] * 2 + [_I] * 6 + [_F, _I, _I, _P, _Z, _P]),
     "s2attn_get_device_error": (_I, [_P, ctypes.POINTER(ctypes.c_uint)]),
     "s2attn_set_wait_timeout_ns": (None, [ctypes.c_ulonglong]),
     "s2attn_selftest_wait_timeout": (_I, [ctypes.c_ulonglong, _P]),
@@ -134,15 +137,31 @@ def s2attn_bwd_workspace_size(B, Hq, N) -> int:
     return int(lib().s2attn_bwd_workspace_size(B, Hq, N))
 
 
+# Default cap on the workspace the allocating paths request for the dS hand-off.
+DEFAULT_WORKSPACE_CAP = 8 << 30
+
+
+def s2attn_bwd_workspace_size_ex(B, Hq, Hkv, N, d, G, shift_head_begin=None, shift=None,
+                                 cap_bytes=0) -> int:
+    """Workspace for the backward without dQ recomputation (see include/s2attn.h)."""
+    shb = Hq // 2 if shift_head_begin is None else shift_head_begin
+    sh = G // 2 if shift is None else shift
+    n = int(lib().s2attn_bwd_workspace_size_ex(B, Hq, Hkv, N, d, G, shb, sh, int(cap_bytes)))
+    if n == 0:
+        raise S2AttnError(S2ATTN_ERR_INVALID_ARG, "s2attn_bwd_workspace_size_ex")
+    return n
+
+
 def s2attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, G, scale=None, shift_head_begin=None,
                shift=None, workspace=None, stream=None):
     """dQ, dK, dV of S²-Attn (overwritten). workspace: a uint8 CUDA tensor, or None to let
-    torch allocate one of s2attn_bwd_workspace_size bytes."""
+    torch allocate s2attn_bwd_workspace_size_ex(..., DEFAULT_WORKSPACE_CAP) bytes."""
     _check_bf16(q, k, v, o, dO, dq, dk, dv)
     B, Hq, Hkv, N, d, G = _dims(q, k, G)
     scale = d ** -0.5 if scale is None else scale
-    ws_bytes = s2attn_bwd_workspace_size(B, Hq, N)
     if workspace is None:
+        ws_bytes = s2attn_bwd_workspace_size_ex(B, Hq, Hkv, N, d, G, shift_head_begin, shift,
+                                                DEFAULT_WORKSPACE_CAP)
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
     if shift_head_begin is None and shift is None:
         _check(lib().s2attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO),
@@ -185,6 +204,29 @@ def s2attn_bwd_dq(q, k, v, dO, dq, G, workspace, scale=None, shift_head_begin=No
     _check(lib().s2attn_bwd_dq(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(dq), B, Hq, Hkv, N, d,
                                G, scale, shb, sh, _ptr(workspace), workspace.numel(),
                                _stream(stream)), "s2attn_bwd_dq")
+
+
+def s2attn_bwd_dkdv_ds(q, k, v, dO, dk, dv, G, workspace, scale=None, shift_head_begin=None,
+                       shift=None, stream=None):
+    B, Hq, Hkv, N, d, G = _dims(q, k, G)
+    scale = d ** -0.5 if scale is None else scale
+    shb = Hq // 2 if shift_head_begin is None else shift_head_begin
+    sh = G // 2 if shift is None else shift
+    _check(lib().s2attn_bwd_dkdv_ds(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(dk), _ptr(dv), B,
+                                    Hq, Hkv, N, d, G, scale, shb, sh, _ptr(workspace),
+                                    workspace.numel(), _stream(stream)), "s2attn_bwd_dkdv_ds")
+
+
+def s2attn_bwd_dq_ds(k, dq, G, workspace, scale=None, shift_head_begin=None, shift=None,
+                     stream=None):
+    B, N, Hq, d = dq.shape
+    Hkv = k.shape[2]
+    scale = d ** -0.5 if scale is None else scale
+    shb = Hq // 2 if shift_head_begin is None else shift_head_begin
+    sh = G // 2 if shift is None else shift
+    _check(lib().s2attn_bwd_dq_ds(_ptr(k), _ptr(dq), B, Hq, Hkv, N, d, G, scale, shb, sh,
+                                  _ptr(workspace), workspace.numel(), _stream(stream)),
+           "s2attn_bwd_dq_ds")
 
 
 def s2attn_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, G, scale=None, stream=None):

@@ -40,7 +40,22 @@ struct BwdParams {
   float scale;
   unsigned int* err;
   unsigned long long timeout_ns;
+  // kv heads [kvh_begin, kvh_begin + kvh_count) are processed by this pass (with all their
+  // query heads); dS tiles, when `ds` is set, are numbered within the pass.
+  int kvh_begin, kvh_count;
+  __nv_bfloat16* ds;   // bf16 dS tiles for the dQ pass (DsSlots layout), or null
+  DsSlots slots;
 };
+
+constexpr uint32_t kDsTileBytes = kTileRows * kTileRows * 2;   // one bf16 dS tile, 32 KB
+
+// First element of dS slot `slot` of (batch b, query head hq of this pass).
+__device__ __forceinline__ __nv_bfloat16* ds_slot_ptr(const BwdParams& p, int b, int hq,
+                                                      long long slot) {
+  const int rep = p.Hq / p.Hkv;
+  const long long hl = static_cast<long long>(b) * (p.kvh_count * rep) + (hq - p.kvh_begin * rep);
+  return p.ds + (hl * p.slots.per_head + slot) * (kDsTileBytes / 2);
+}
 
 template <int D>
 struct DkdvLayout {
@@ -79,9 +94,15 @@ __global__ void __launch_bounds__(320, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kTmemSlot);
   const WaitCtx ctx{abort_flag, p.err, p.timeout_ns, KID_DKDV};
 
-  int b, kvh, t0;
-  kv_tile_coords(blockIdx.x, p.B, p.Hq, p.Hkv, p.N, p.G, p.shift_head_begin, p.shift, b, kvh, t0);
   const int rep = p.Hq / p.Hkv;
+  int b, kvh, t0;
+  {
+    int shb = p.shift_head_begin - p.kvh_begin * rep;
+    shb = shb < 0 ? 0 : (shb > p.kvh_count * rep ? p.kvh_count * rep : shb);
+    kv_tile_coords(blockIdx.x, p.B, p.kvh_count * rep, p.kvh_count, p.N, p.G, shb, p.shift, b,
+                   kvh, t0);
+    kvh += p.kvh_begin;
+  }
   const int h_begin = kvh * rep;
   auto head_shift = [&](int hq) { return hq >= p.shift_head_begin ? p.shift : 0; };
 
@@ -214,9 +235,11 @@ __global__ void __launch_bounds__(320, 1)
       const int ge_k = group_end(r_k, p.G);
       for (int i = 0; i < qr.count(); ++i, ++n) {
         const int st = n & 1;
-        const int q0 = qr.at(i) * kTileRows + 64 * half;
+        const int qt = qr.at(i);
+        const int q0 = qt * kTileRows + 64 * half;
         const int cl = kv_valid ? r_k - q0 : 1;
         const int ch = kv_valid ? ge_k - 1 - q0 : 0;
+        const bool mask = __any_sync(0xffffffffu, cl > 0 || ch < 63);
         if (!warp_wait(bar(L::B_QF + st), (n >> 1) & 1, ctx, 7)) { ok = false; break; }
         if (!warp_wait(bar(L::B_S), n & 1, ctx, 8)) { ok = false; break; }
         tc_fence_after();
@@ -227,7 +250,6 @@ __global__ void __launch_bounds__(320, 1)
         {
           uint32_t raw[64];
           tmem_ld64(t_lane + 64 * half, raw);
-          const bool mask = __any_sync(0xffffffffu, cl > 0 || ch < 63);
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             const int col = 2 * e;
@@ -247,22 +269,45 @@ __global__ void __launch_bounds__(320, 1)
         // dS^T phase: dS^T = P^T o (dP^T - D).
         if (!warp_wait(bar(L::B_DP), n & 1, ctx, 9)) { ok = false; break; }
         tc_fence_after();
+        uint32_t ds[32];
         {
           uint32_t raw[64];
           tmem_ld64(t_lane + 128 + 64 * half, raw);
-          uint32_t ds[32];
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             const int col = 2 * e;
             const float2 pf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[e]));
-            ds[e] = pack_bf16(pf.x * (__uint_as_float(raw[col]) - d_t[col]),
-                              pf.y * (__uint_as_float(raw[col + 1]) - d_t[col + 1]));
+            float y0 = pf.x * (__uint_as_float(raw[col]) - d_t[col]);
+            float y1 = pf.y * (__uint_as_float(raw[col + 1]) - d_t[col + 1]);
+            if (mask) {   // exact zeros where P is masked, whatever D holds for padding rows
+              y0 = (col >= cl && col <= ch) ? y0 : 0.f;
+              y1 = (col + 1 >= cl && col + 1 <= ch) ? y1 : 0.f;
+            }
+            ds[e] = pack_bf16(y0, y1);
           }
           tmem_st32(t_lane + 160 + 32 * half, ds);
         }
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(bar(L::B_DS));
+        if (p.ds) {
+          // Hand the tile to the dQ pass, after the arrive so the stores stay off the tensor
+          // core's critical path. Layout (DsSlots): 16 blocks of 2 KB, block c holding query
+          // columns [8c, 8c + 8) of all 128 kv rows, 16 bytes per row — so each store below
+          // writes 512 contiguous bytes per warp. Streaming stores: the tile is read once,
+          // by another kernel, and should not evict this kernel's operands from L2.
+          const KvSpan sp = qtile_kv_span(qt, sh, p.N, p.G);
+          int idx = t0 / kTileRows - sp.first;
+          if (idx < 0) idx += (p.N + kTileRows - 1) / kTileRows;
+          if (idx < sp.count) {
+            uint4* dst = reinterpret_cast<uint4*>(ds_slot_ptr(p, b, hq, p.slots.base(qt) + idx)) +
+                         half * 8 * kTileRows + row;
+#pragma unroll
+            for (int c8 = 0; c8 < 8; ++c8)
+              __stcs(dst + c8 * kTileRows,
+                     make_uint4(ds[4 * c8], ds[4 * c8 + 1], ds[4 * c8 + 2], ds[4 * c8 + 3]));
+          }
+        }
       }
     }
     if (ok && warp_wait(bar(L::B_ACC), 0, ctx, 10)) {

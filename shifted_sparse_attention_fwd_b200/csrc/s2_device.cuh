@@ -13,7 +13,7 @@ namespace s2 {
 // Error reporting shared by every kernel (read back by s2attn_get_device_error).
 // code = (kernel id << 8) | wait site; the first failing wait wins.
 // ----------------------------------------------------------------------------------------
-enum KernelId : uint32_t { KID_FWD = 1, KID_DKDV = 2, KID_DQ = 3, KID_SELFTEST = 4 };
+enum KernelId : uint32_t { KID_FWD = 1, KID_DKDV = 2, KID_DQ = 3, KID_SELFTEST = 4, KID_DQDS = 5 };
 
 struct WaitCtx {
   volatile int* abort_flag;   // CTA-shared; set by the first waiter that gives up
@@ -178,6 +178,19 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
   d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
   d |= static_cast<uint64_t>(1) << 46;   // descriptor version for sm_100
   d |= static_cast<uint64_t>(2) << 61;   // SWIZZLE_128B
+  return d;
+}
+
+// Shared-memory matrix descriptor for an unswizzled operand built from 8 x 16-byte core
+// matrices (128 contiguous bytes each). For an MN-major operand: SBO = byte distance between
+// core matrices adjacent along M/N, LBO = between core matrices adjacent along K.
+__device__ __forceinline__ uint64_t sdesc_noswz(uint32_t saddr, uint32_t lbo_bytes,
+                                                uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1) << 46;   // descriptor version for sm_100; layout 0 = none
   return d;
 }
 

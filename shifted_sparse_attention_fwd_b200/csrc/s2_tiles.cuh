@@ -87,6 +87,71 @@ __host__ __device__ inline QTileRanges kv_tile_qtiles(int t0, int sh, int N, int
   return q;
 }
 
+// Original kv tiles that rolled query tile qt (head roll sh) reads. Its rows see the rolled
+// kv rows [start of the group of its first row, its last row]; under the roll these are a
+// contiguous range of original rows modulo N, covered by `count` consecutive original tiles
+// (indices taken modulo the tile count T) starting at `first`.
+struct KvSpan {
+  int first, count;
+};
+__host__ __device__ inline KvSpan qtile_kv_span(int qt, int sh, int N, int G) {
+  const int T = (N + kTileRows - 1) / kTileRows;
+  const int r0 = qt * kTileRows;
+  const int last = r0 + kTileRows - 1 < N - 1 ? r0 + kTileRows - 1 : N - 1;
+  const int gb = group_begin(r0, G);
+  const int len = last - gb + 1;
+  const long long o = static_cast<long long>(gb) + sh;
+  const int o0 = static_cast<int>(o >= N ? o - N : o);
+  int count;
+  if (o0 + len <= N)
+    count = (o0 + len - 1) / kTileRows - o0 / kTileRows + 1;
+  else
+    count = (T - o0 / kTileRows) + (o0 + len - N - 1) / kTileRows + 1;
+  KvSpan s;
+  s.first = o0 / kTileRows;
+  s.count = count < T ? count : T;
+  return s;
+}
+
+// Slots of the bf16 dS tiles that the dK/dV kernel hands to the dQ pass: one 128 x 128 tile
+// (32 KB) per (query tile qt, original kv tile first + i), i < count, at slot base(qt) + i of
+// its (batch, query head). When groups and roll are tile-aligned, count = qt mod (G/128) + 1
+// and the slots are packed (a triangle per group); otherwise every query tile gets `stride`
+// slots, the largest count of any query tile.
+struct DsSlots {
+  int aligned;          // G and every head's roll are multiples of the tile
+  int gt;               // G / 128 (aligned case)
+  int stride;           // slots per query tile (unaligned case)
+  long long per_head;   // slots of one (batch, query head)
+  __host__ __device__ __forceinline__ long long base(int qt) const {
+    if (aligned) {
+      const long long g = qt / gt, i = qt % gt;
+      return g * gt * (gt + 1) / 2 + i * (i + 1) / 2;
+    }
+    return static_cast<long long>(qt) * stride;
+  }
+};
+inline DsSlots ds_slots(int N, int G, int shifted_heads, int shift) {
+  DsSlots d;
+  const int T = (N + kTileRows - 1) / kTileRows;
+  const int sh = shifted_heads ? shift : 0;
+  d.aligned = (G % kTileRows == 0 && sh % kTileRows == 0) ? 1 : 0;
+  d.gt = G / kTileRows;
+  d.stride = 0;
+  if (d.aligned) {
+    d.per_head = static_cast<long long>(N / G) * d.gt * (d.gt + 1) / 2;
+  } else {
+    for (int qt = 0; qt < T; ++qt) {
+      const int c0 = qtile_kv_span(qt, 0, N, G).count;
+      const int c1 = qtile_kv_span(qt, sh, N, G).count;
+      const int c = c0 > c1 ? c0 : c1;
+      d.stride = c > d.stride ? c : d.stride;
+    }
+    d.per_head = static_cast<long long>(T) * d.stride;
+  }
+  return d;
+}
+
 // Block index -> (b, h, rolled query tile) for the forward and dQ kernels. When G is a
 // multiple of the tile, tiles late in their group (more key tiles to visit) come first.
 __host__ __device__ inline void query_tile_coords(int bid, int B, int Hq, int N, int G, int& b,

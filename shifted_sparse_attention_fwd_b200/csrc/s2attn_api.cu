@@ -13,6 +13,7 @@
 #include "../../include/s2attn.h"
 #include "s2_bwd_dkdv.cuh"
 #include "s2_bwd_dq.cuh"
+#include "s2_bwd_dq_ds.cuh"
 #include "s2_bwd_pre.cuh"
 #include "s2_fwd.cuh"
 
@@ -52,8 +53,12 @@ cudaError_t set_smem_attrs() {
   e = cudaFuncSetAttribute(s2::s2_bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            s2::DkdvLayout<D>::kLaunchBytes);
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(s2::s2_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              s2::DqLayout<D>::kLaunchBytes);
+  e = cudaFuncSetAttribute(s2::s2_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           s2::DqLayout<D>::kLaunchBytes);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(s2::s2_bwd_dq_ds_kernel<D>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              s2::DqDsLayout<D>::kLaunchBytes);
 }
 
 // Per-device one-time set-up (with that device current): the device address of the error
@@ -138,6 +143,24 @@ struct Shape {
   int B, Hq, Hkv, N, d, G, shb, shift;
 };
 
+// dS hand-off (backward without recomputation in the dQ pass): the slot layout, and the bytes
+// one kv head (all its query heads, all batches) needs. The dS tiles follow D and LSE2 in the
+// workspace.
+s2::DsSlots ds_layout(const Shape& sh) { return s2::ds_slots(sh.N, sh.G, sh.shb < sh.Hq, sh.shift); }
+size_t ds_bytes_per_kv_head(const Shape& sh) {
+  const s2::DsSlots sl = ds_layout(sh);
+  return static_cast<size_t>(sh.B) * (sh.Hq / sh.Hkv) * static_cast<size_t>(sl.per_head) *
+         s2::kDsTileBytes;
+}
+// kv heads per pass that a workspace of `bytes` allows (0: too small, recompute dQ instead).
+int ds_heads_per_pass(const Shape& sh, size_t bytes) {
+  const size_t base = 2 * ws_half(sh.B, sh.Hq, sh.N);
+  if (bytes <= base) return 0;
+  const size_t per = ds_bytes_per_kv_head(sh);
+  const size_t k = (bytes - base) / per;
+  return k >= static_cast<size_t>(sh.Hkv) ? sh.Hkv : static_cast<int>(k);
+}
+
 // Validation shared by every attention entry point (see s2attn.h, "Errors").
 s2attn_status check_shape(int B, int Hq, int Hkv, int N, int d, int G, float scale,
                           int shift_head_begin, long long shift, Shape& out) {
@@ -198,7 +221,21 @@ s2::BwdParams bwd_params(const Shape& sh, float scale, const void* workspace, vo
   p.scale_log2 = scale * 1.4426950408889634f;
   p.err = err;
   p.timeout_ns = g_timeout_ns.load();
+  p.kvh_begin = 0;
+  p.kvh_count = sh.Hkv;
+  p.ds = nullptr;
+  p.slots = s2::DsSlots{};
   return p;
+}
+
+// Point the parameters at the dS region of the workspace for kv heads [kvh_begin, +count).
+void set_ds_pass(s2::BwdParams& p, const Shape& sh, const void* workspace, int kvh_begin,
+                 int kvh_count) {
+  p.kvh_begin = kvh_begin;
+  p.kvh_count = kvh_count;
+  p.slots = ds_layout(sh);
+  p.ds = reinterpret_cast<__nv_bfloat16*>(const_cast<char*>(static_cast<const char*>(workspace)) +
+                                          2 * ws_half(sh.B, sh.Hq, sh.N));
 }
 
 template <int D>
@@ -218,17 +255,19 @@ s2attn_status launch_pre(const Shape& sh, const void* o, const float* lse, const
 template <int D, bool kDkdv>
 s2attn_status launch_grad(const Shape& sh, const void* q, const void* k, const void* v,
                           const void* dO, void* dq, void* dk, void* dv, float scale,
-                          const void* workspace, cudaStream_t stream, unsigned int* err) {
+                          const void* workspace, cudaStream_t stream, unsigned int* err,
+                          int ds_kvh_begin = -1, int ds_kvh_count = 0) {
   MapPair mq, mk, mv, mo;
   s2attn_status s;
   if ((s = encode_pair(mq, q, sh.B, sh.Hq, sh.N, D)) != S2ATTN_OK) return s;
   if ((s = encode_pair(mk, k, sh.B, sh.Hkv, sh.N, D)) != S2ATTN_OK) return s;
   if ((s = encode_pair(mv, v, sh.B, sh.Hkv, sh.N, D)) != S2ATTN_OK) return s;
   if ((s = encode_pair(mo, dO, sh.B, sh.Hq, sh.N, D)) != S2ATTN_OK) return s;
-  const s2::BwdParams p = bwd_params(sh, scale, workspace, dq, dk, dv, err);
+  s2::BwdParams p = bwd_params(sh, scale, workspace, dq, dk, dv, err);
+  if (ds_kvh_begin >= 0) set_ds_pass(p, sh, workspace, ds_kvh_begin, ds_kvh_count);
   const unsigned tiles = (sh.N + 127) / 128;
   if (kDkdv) {
-    const unsigned grid = static_cast<unsigned>(sh.B) * sh.Hkv * tiles;
+    const unsigned grid = static_cast<unsigned>(sh.B) * p.kvh_count * tiles;
     s2::s2_bwd_dkdv_kernel<D><<<grid, s2::DkdvLayout<D>::kThreads, s2::DkdvLayout<D>::kLaunchBytes, stream>>>(
         mq.m128, mq.m8, mk.m128, mk.m8, mv.m128, mv.m8, mo.m128, mo.m8, p);
   } else {
@@ -239,6 +278,24 @@ s2attn_status launch_grad(const Shape& sh, const void* q, const void* k, const v
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? S2ATTN_OK
                           : cuda_fail(e, kDkdv ? "s2_bwd_dkdv_kernel launch" : "s2_bwd_dq_kernel launch");
+}
+
+template <int D>
+s2attn_status launch_dq_ds(const Shape& sh, const void* k, void* dq, float scale,
+                           const void* workspace, int kvh_begin, int kvh_count,
+                           cudaStream_t stream, unsigned int* err, int num_sms) {
+  MapPair mk;
+  s2attn_status s;
+  if ((s = encode_pair(mk, k, sh.B, sh.Hkv, sh.N, D)) != S2ATTN_OK) return s;
+  s2::BwdParams p = bwd_params(sh, scale, workspace, dq, nullptr, nullptr, err);
+  set_ds_pass(p, sh, workspace, kvh_begin, kvh_count);
+  const unsigned units = static_cast<unsigned>(sh.B) * kvh_count * (sh.Hq / sh.Hkv) *
+                         ((sh.N + 127) / 128);
+  const unsigned grid = units < static_cast<unsigned>(num_sms) ? units : static_cast<unsigned>(num_sms);
+  s2::s2_bwd_dq_ds_kernel<D><<<grid, s2::DqDsLayout<D>::kThreads, s2::DqDsLayout<D>::kLaunchBytes,
+                               stream>>>(mk.m128, mk.m8, p);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? S2ATTN_OK : cuda_fail(e, "s2_bwd_dq_ds_kernel launch");
 }
 
 s2attn_status check_workspace(const Shape& sh, const void* ws, size_t bytes) {
@@ -258,6 +315,21 @@ s2attn_status dq_impl(const Shape& sh, const void* q, const void* k, const void*
                       unsigned int* err) {
   return sh.d == 64 ? launch_grad<64, false>(sh, q, k, v, dO, dq, nullptr, nullptr, scale, ws, stream, err)
                     : launch_grad<128, false>(sh, q, k, v, dO, dq, nullptr, nullptr, scale, ws, stream, err);
+}
+s2attn_status dkdv_ds_impl(const Shape& sh, const void* q, const void* k, const void* v,
+                           const void* dO, void* dk, void* dv, float scale, const void* ws,
+                           int kvh_begin, int kvh_count, cudaStream_t stream, unsigned int* err) {
+  return sh.d == 64
+             ? launch_grad<64, true>(sh, q, k, v, dO, nullptr, dk, dv, scale, ws, stream, err,
+                                     kvh_begin, kvh_count)
+             : launch_grad<128, true>(sh, q, k, v, dO, nullptr, dk, dv, scale, ws, stream, err,
+                                      kvh_begin, kvh_count);
+}
+s2attn_status dq_ds_impl(const Shape& sh, const void* k, void* dq, float scale, const void* ws,
+                         int kvh_begin, int kvh_count, cudaStream_t stream, unsigned int* err,
+                         int num_sms) {
+  return sh.d == 64 ? launch_dq_ds<64>(sh, k, dq, scale, ws, kvh_begin, kvh_count, stream, err, num_sms)
+                    : launch_dq_ds<128>(sh, k, dq, scale, ws, kvh_begin, kvh_count, stream, err, num_sms);
 }
 s2attn_status pre_impl(const Shape& sh, const void* o, const float* lse, const void* dO, void* ws,
                        cudaStream_t stream) {
@@ -333,6 +405,21 @@ size_t s2attn_bwd_workspace_size(int B, int Hq, int N) {
   return 2 * ws_half(B, Hq, N);
 }
 
+size_t s2attn_bwd_workspace_size_ex(int B, int Hq, int Hkv, int N, int d, int G,
+                                    int shift_head_begin, int shift, size_t cap_bytes) {
+  Shape sh;
+  if (check_shape(B, Hq, Hkv, N, d, G, 1.0f, shift_head_begin, shift, sh) != S2ATTN_OK) return 0;
+  const size_t base = 2 * ws_half(B, Hq, N);
+  const size_t per = ds_bytes_per_kv_head(sh);
+  size_t k = static_cast<size_t>(Hkv);
+  if (cap_bytes != 0) {
+    const size_t fit = cap_bytes > base ? (cap_bytes - base) / per : 0;
+    k = fit < k ? fit : k;
+    if (k == 0) k = 1;
+  }
+  return base + k * per;
+}
+
 s2attn_status s2attn_bwd_preprocess(const void* o, const float* lse, const void* dO, int B,
                                     int Hq, int N, int d, void* workspace,
                                     size_t workspace_bytes, void* stream) {
@@ -383,6 +470,53 @@ s2attn_status s2attn_bwd_dq(const void* q, const void* k, const void* v, const v
   return dq_impl(sh, q, k, v, dO, dq, scale, workspace, static_cast<cudaStream_t>(stream), err);
 }
 
+s2attn_status s2attn_bwd_dkdv_ds(const void* q, const void* k, const void* v, const void* dO,
+                                 void* dk, void* dv, int B, int Hq, int Hkv, int N, int d, int G,
+                                 float scale, int shift_head_begin, int shift, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !dO || !dk || !dv) return S2ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dO) || !aligned16(dk) ||
+      !aligned16(dv))
+    return S2ATTN_ERR_INVALID_ARG;
+  Shape sh;
+  s2attn_status s = check_shape(B, Hq, Hkv, N, d, G, scale, shift_head_begin, shift, sh);
+  if (s != S2ATTN_OK) return s;
+  if ((s = check_workspace(sh, workspace, workspace_bytes)) != S2ATTN_OK) return s;
+  if (ds_heads_per_pass(sh, workspace_bytes) < Hkv) {
+    std::snprintf(g_last_error, sizeof(g_last_error),
+                  "s2attn_bwd_dkdv_ds: workspace of %zu bytes holds the dS tiles of fewer than "
+                  "all %d kv heads", workspace_bytes, Hkv);
+    return S2ATTN_ERR_INVALID_ARG;
+  }
+  if ((s = get_encoder()) != S2ATTN_OK) return s;
+  unsigned int* err = nullptr;
+  if ((s = device_state(&err)) != S2ATTN_OK) return s;
+  return dkdv_ds_impl(sh, q, k, v, dO, dk, dv, scale, workspace, 0, Hkv,
+                      static_cast<cudaStream_t>(stream), err);
+}
+
+s2attn_status s2attn_bwd_dq_ds(const void* k, void* dq, int B, int Hq, int Hkv, int N, int d,
+                               int G, float scale, int shift_head_begin, int shift,
+                               const void* workspace, size_t workspace_bytes, void* stream) {
+  if (!k || !dq || !aligned16(k) || !aligned16(dq)) return S2ATTN_ERR_INVALID_ARG;
+  Shape sh;
+  s2attn_status s = check_shape(B, Hq, Hkv, N, d, G, scale, shift_head_begin, shift, sh);
+  if (s != S2ATTN_OK) return s;
+  if ((s = check_workspace(sh, workspace, workspace_bytes)) != S2ATTN_OK) return s;
+  if (ds_heads_per_pass(sh, workspace_bytes) < Hkv) {
+    std::snprintf(g_last_error, sizeof(g_last_error),
+                  "s2attn_bwd_dq_ds: workspace of %zu bytes holds the dS tiles of fewer than "
+                  "all %d kv heads", workspace_bytes, Hkv);
+    return S2ATTN_ERR_INVALID_ARG;
+  }
+  if ((s = get_encoder()) != S2ATTN_OK) return s;
+  unsigned int* err = nullptr;
+  int num_sms = 0;
+  if ((s = device_state(&err, &num_sms)) != S2ATTN_OK) return s;
+  return dq_ds_impl(sh, k, dq, scale, workspace, 0, Hkv, static_cast<cudaStream_t>(stream), err,
+                    num_sms);
+}
+
 s2attn_status s2attn_bwd_ex(const void* q, const void* k, const void* v, const void* o,
                             const float* lse, const void* dO, void* dq, void* dk, void* dv,
                             int B, int Hq, int Hkv, int N, int d, int G, float scale,
@@ -398,11 +532,24 @@ s2attn_status s2attn_bwd_ex(const void* q, const void* k, const void* v, const v
   if ((s = check_workspace(sh, workspace, workspace_bytes)) != S2ATTN_OK) return s;
   if ((s = get_encoder()) != S2ATTN_OK) return s;
   unsigned int* err = nullptr;
-  if ((s = device_state(&err)) != S2ATTN_OK) return s;
+  int num_sms = 0;
+  if ((s = device_state(&err, &num_sms)) != S2ATTN_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if ((s = pre_impl(sh, o, lse, dO, workspace, st)) != S2ATTN_OK) return s;
-  if ((s = dkdv_impl(sh, q, k, v, dO, dk, dv, scale, workspace, st, err)) != S2ATTN_OK) return s;
-  return dq_impl(sh, q, k, v, dO, dq, scale, workspace, st, err);
+  const int per_pass = ds_heads_per_pass(sh, workspace_bytes);
+  if (per_pass == 0) {
+    // Workspace too small for one kv head's dS tiles: the dQ kernel recomputes S and dP.
+    if ((s = dkdv_impl(sh, q, k, v, dO, dk, dv, scale, workspace, st, err)) != S2ATTN_OK) return s;
+    return dq_impl(sh, q, k, v, dO, dq, scale, workspace, st, err);
+  }
+  for (int h0 = 0; h0 < sh.Hkv; h0 += per_pass) {
+    const int cnt = sh.Hkv - h0 < per_pass ? sh.Hkv - h0 : per_pass;
+    if ((s = dkdv_ds_impl(sh, q, k, v, dO, dk, dv, scale, workspace, h0, cnt, st, err)) != S2ATTN_OK)
+      return s;
+    if ((s = dq_ds_impl(sh, k, dq, scale, workspace, h0, cnt, st, err, num_sms)) != S2ATTN_OK)
+      return s;
+  }
+  return S2ATTN_OK;
 }
 
 s2attn_status s2attn_bwd(const void* q, const void* k, const void* v, const void* o,

@@ -23,14 +23,43 @@ BF16_MEAN_ABS = 2e-3
 LSE_MAX_ABS = 1e-4
 
 
-def gpu_run(q, k, v, do, G, scale, shb=None, shift=None, backward=True):
+def _bwd(qd, kd, vd, o, lse, dod, G, scale, shb, shift, mode):
+    """Backward through one of the library's paths:
+    auto        the allocating convenience (dS hand-off, all kv heads in one pass when the
+                default cap allows);
+    recompute   the minimum workspace: the dQ kernel recomputes S and dP;
+    per_kv_head room for one kv head's dS tiles: one dK/dV + dQ pass per kv head;
+    phases      preprocess, s2attn_bwd_dkdv_ds and s2attn_bwd_dq_ds called one by one."""
+    if mode == "auto":
+        return s2.bwd(qd, kd, vd, o, lse, dod, G, scale, shb, shift)
+    B, N, Hq, d = qd.shape
+    Hkv = kd.shape[2]
+    shb_ = Hq // 2 if shb is None else shb
+    sh_ = G // 2 if shift is None else shift
+    if mode == "recompute":
+        n = s2.s2attn_bwd_workspace_size(B, Hq, N)
+    else:
+        n = s2.s2attn_bwd_workspace_size_ex(B, Hq, Hkv, N, d, G, shb_, sh_,
+                                            1 if mode == "per_kv_head" else 0)
+    ws = torch.empty(n, dtype=torch.uint8, device=qd.device)
+    dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
+    if mode == "phases":
+        s2.s2attn_bwd_preprocess(o, lse, dod, ws)
+        s2.s2attn_bwd_dkdv_ds(qd, kd, vd, dod, dk, dv, G, ws, scale, shb_, sh_)
+        s2.s2attn_bwd_dq_ds(kd, dq, G, ws, scale, shb_, sh_)
+    else:
+        s2.s2attn_bwd(qd, kd, vd, o, lse, dod, dq, dk, dv, G, scale, shb_, sh_, ws)
+    return dq, dk, dv
+
+
+def gpu_run(q, k, v, do, G, scale, shb=None, shift=None, backward=True, mode="auto"):
     """Forward (+ backward) of the CUDA path on bf16 CPU inputs; returns CPU tensors."""
     dev = torch.device("cuda")
     qd, kd, vd, dod = (x.to(dev) for x in (q, k, v, do))
     o, lse = s2.fwd(qd, kd, vd, G, scale, shb, shift)
     out = {"o": o, "lse": lse}
     if backward:
-        dq, dk, dv = s2.bwd(qd, kd, vd, o, lse, dod, G, scale, shb, shift)
+        dq, dk, dv = _bwd(qd, kd, vd, o, lse, dod, G, scale, shb, shift, mode)
         out.update(dq=dq, dk=dk, dv=dv)
     torch.cuda.synchronize()
     st, code = s2.s2attn_get_device_error()
@@ -74,10 +103,10 @@ def assert_close(name, gpu, ref):
 
 
 def check_case(B, Hq, Hkv, N, G, d, seed, shb=None, shift=None, q_gain=1.0, scale=None,
-               backward=True):
+               backward=True, mode="auto"):
     q, k, v, do = make_inputs(B, Hq, Hkv, N, d, seed, q_gain)
     scale = d ** -0.5 if scale is None else scale
-    g = gpu_run(q, k, v, do, G, scale, shb, shift, backward)
+    g = gpu_run(q, k, v, do, G, scale, shb, shift, backward, mode)
     r = oracle_run(q, k, v, do, G, scale, shb, shift, backward)
     report = {}
     for name in g:

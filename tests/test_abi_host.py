@@ -137,6 +137,11 @@ void paircoords(int bid, int B, int Hq, int N, int G, int* o) {
   s2::query_pair_coords(bid, B, Hq, N, G, o[0], o[1], o[2]); o[3] = s2::query_pairs_per_head(N); }
 void kvcoords(int bid, int B, int Hq, int Hkv, int N, int G, int shb, int sh, int* o) {
   s2::kv_tile_coords(bid, B, Hq, Hkv, N, G, shb, sh, o[0], o[1], o[2]); }
+void kvspan(int qt, int sh, int N, int G, int* o) {
+  s2::KvSpan s = s2::qtile_kv_span(qt, sh, N, G); o[0] = s.first; o[1] = s.count; }
+long long dsslots(int N, int G, int shifted, int shift, int qt) {
+  s2::DsSlots d = s2::ds_slots(N, G, shifted, shift);
+  return qt < 0 ? d.per_head : d.base(qt); }
 }
 """
 
@@ -248,3 +253,75 @@ def test_query_pair_order_is_a_permutation(shim, B, Hq, N, G):
     if G % 256 == 0 and G > 256:
         b, h, p = call4(shim.paircoords, 0, B, Hq, N, G)[:3]
         assert p % (G // 256) == G // 256 - 1
+
+
+@pytest.mark.parametrize("N,G,shift", CASES + [(102400, 25600, 12800), (32768, 8192, 4096)])
+def test_qtile_kv_span_exact(shim, N, G, shift):
+    """Brute force: the original kv tiles a rolled query tile reads are exactly the tiles
+    holding some kv row that one of its rows attends (same rolled group, key not after query),
+    listed once each from `first` on (indices modulo the tile count)."""
+    nt = (N + 127) // 128
+    for sh in {0, shift}:
+        for qt in range(nt) if N <= 8192 else list(range(0, nt, 37)) + [nt - 1]:
+            first, count = call4(shim.kvspan, qt, sh, N, G)[:2]
+            got = [(first + i) % nt for i in range(count)]
+            assert len(set(got)) == count
+            r0, last = qt * 128, min(qt * 128 + 127, N - 1)
+            gb = (r0 // G) * G
+            want = {((r + sh) % N) // 128 for r in range(gb, last + 1)}
+            assert set(got) == want
+
+
+@pytest.mark.parametrize("N,G,shift", CASES)
+def test_ds_slots_match_the_dkdv_pairs(shim, N, G, shift):
+    """Every (query tile, kv tile) pair the dQ pass reads is one the dK/dV kernel visits, and
+    the slots of one head are distinct and inside per_head."""
+    nt = (N + 127) // 128
+    shim.dsslots.restype = ctypes.c_longlong
+    per_head = shim.dsslots(N, G, 1, shift, -1)
+    out = (ctypes.c_int * 4096)()
+    for sh in {0, shift}:
+        visited = set()
+        for t in range(nt):
+            n = shim.qtiles(t * 128, sh, N, G, out)
+            visited.update((qt, t) for qt in out[:n])
+        slots = set()
+        for qt in range(nt):
+            first, count = call4(shim.kvspan, qt, sh, N, G)[:2]
+            base = shim.dsslots(N, G, 1, shift, qt)
+            for i in range(count):
+                assert (qt, (first + i) % nt) in visited
+                slots.add(base + i)
+            assert base + count <= per_head
+        assert len(slots) == sum(call4(shim.kvspan, qt, sh, N, G)[1] for qt in range(nt))
+    if G % 128 == 0 and shift % 128 == 0:
+        gt = G // 128
+        assert per_head == (N // G) * gt * (gt + 1) // 2
+
+
+def test_workspace_size_ex(lib):
+    base = lib.s2attn_bwd_workspace_size(1, 32, 8192)
+    full = lib.s2attn_bwd_workspace_size_ex(1, 32, 32, 8192, 128, 2048, 16, 1024, 0)
+    assert full == base + 32 * (4 * 16 * 17 // 2) * 32768           # 544 tiles per head
+    one = lib.s2attn_bwd_workspace_size_ex(1, 32, 32, 8192, 128, 2048, 16, 1024, 1)
+    assert one == base + 544 * 32768                                  # at least one kv head
+    capped = lib.s2attn_bwd_workspace_size_ex(1, 32, 32, 8192, 128, 2048, 16, 1024, base + 5 * 544 * 32768 + 7)
+    assert capped == base + 5 * 544 * 32768
+    gqa = lib.s2attn_bwd_workspace_size_ex(1, 64, 8, 32768, 128, 8192, 32, 4096, 0)
+    assert gqa == lib.s2attn_bwd_workspace_size(1, 64, 32768) + 64 * (4 * 64 * 65 // 2) * 32768
+    assert lib.s2attn_bwd_workspace_size_ex(1, 3, 3, 256, 64, 64, 1, 32, 0) > 0
+    assert lib.s2attn_bwd_workspace_size_ex(1, 4, 4, 256, 96, 64, 2, 32, 0) == 0   # d = 96
+    assert lib.s2attn_bwd_workspace_size_ex(1, 4, 3, 256, 64, 64, 2, 32, 0) == 0   # Hq % Hkv
+
+
+def test_ds_entries_reject(lib):
+    ws = 0x100000
+    small = lib.s2attn_bwd_workspace_size(1, 4, 256)
+    full = lib.s2attn_bwd_workspace_size_ex(1, 4, 4, 256, 64, 64, 2, 32, 0)
+    f = ctypes.c_float(0.125)
+    assert lib.s2attn_bwd_dkdv_ds(A, A, A, A, A, A, 1, 4, 4, 256, 64, 64, f, 2, 32, ws, small,
+                                  None) == 1                          # no room for dS
+    assert lib.s2attn_bwd_dq_ds(A, A, 1, 4, 4, 256, 64, 64, f, 2, 32, ws, full - 16,
+                                None) == 1
+    assert lib.s2attn_bwd_dq_ds(A, None, 1, 4, 4, 256, 64, 64, f, 2, 32, ws, full, None) == 1
+    assert lib.s2attn_bwd_dq_ds(A, A, 1, 4, 4, 256, 96, 64, f, 2, 32, ws, full, None) == 2

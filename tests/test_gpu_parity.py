@@ -53,6 +53,20 @@ def test_edge_cases(name, B, Hq, Hkv, N, G, d, shb, shift, q_gain):
     check_case(B, Hq, Hkv, N, G, d, seed=zlib.crc32(name.encode()) % 10000, shb=shb, shift=shift, q_gain=q_gain)
 
 
+@pytest.mark.parametrize("mode", ["recompute", "per_kv_head", "phases"])
+@pytest.mark.parametrize("name,B,Hq,Hkv,N,G,d,shb,shift", [
+    ("ragged_gqa", 2, 4, 2, 320, 64, 64, None, None),       # unaligned slots, 2 kv heads
+    ("straddle", 1, 4, 4, 384, 192, 128, None, None),       # roll splits tiles
+    ("mqa_mixed", 1, 8, 1, 512, 128, 128, None, None),      # 8 query heads on one kv head
+    ("aligned_gqa", 1, 8, 4, 2048, 512, 128, None, None),   # packed (triangular) slots
+])
+def test_backward_paths(mode, name, B, Hq, Hkv, N, G, d, shb, shift):
+    """Each backward path — dQ recomputed, dS handed off one kv head per pass, and the dS
+    stages called one at a time — against the oracle."""
+    check_case(B, Hq, Hkv, N, G, d, seed=zlib.crc32((name + mode).encode()) % 10000, shb=shb,
+               shift=shift, mode=mode)
+
+
 def test_shifted_head_equals_unshifted_on_rolled_input():
     """A rolled head equals an unrolled run on torch.roll-ed inputs, rolled back (bitwise)."""
     B, Hq, N, G, d = 1, 2, 1024, 256, 128
