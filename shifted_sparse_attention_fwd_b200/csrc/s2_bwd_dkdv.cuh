@@ -9,15 +9,20 @@
 //   dP^T = V dO^T
 //   dS^T = P^T o (dP^T - D)
 //   dK  += scale * dS^T Q
-// One CTA owns 128 ORIGINAL key/value rows of one (batch, kv head), so the tile is shared
+// A work tile is 128 ORIGINAL key/value rows of one (batch, kv head), so the tile is shared
 // by all its query heads whatever their roll, and dK/dV are written once, without atomics.
 // For each query head the rows map to at most two runs of rolled rows; the query tiles
 // visited are those covering [rolled row, end of its group) for every row of the tile.
+// The kernel is persistent: each CTA takes tiles blockIdx.x, blockIdx.x + gridDim.x, ...
+// (heaviest first), so one tile's epilogue overlaps the next tile's loads and first MMAs.
 //
-// Warp roles (320 threads): warps 0-7 elementwise — kv row i (TMEM lane i) is shared by warp
+// Warp roles (352 threads): warps 0-7 elementwise — kv row i (TMEM lane i) is shared by warp
 // i/32 (query columns 0-63) and warp i/32 + 4 (columns 64-127), so two warps per SM
-// sub-partition work on every tile; warp 8 TMA producer (K, V once; Q, dO, LSE2, D per query
-// tile, 2 stages); warp 9 TMEM allocator + MMA issuer.
+// sub-partition work on every tile; warp 8 TMA producer (K, V per tile; Q, dO, LSE2, D per
+// query tile, 2 stages); warp 9 TMEM allocator + MMA issuer; warp 10 store issuer: the
+// elementwise warps leave each dS tile (for the dQ pass) and the finished dV and dK tiles in
+// a shared-memory staging buffer, and warp 10 hands them to the TMA unit, so no elementwise
+// warp waits on global stores.
 // TMEM: S^T [0,128) with P^T (bf16) written to [32,96); dP^T [128,256) with dS^T (bf16) to
 // [160,224) — each column half packs its bf16 output inside its own fp32 input columns, so the
 // two warps of a row never overwrite each other's unread data; dV [256,256+D), dK
@@ -64,30 +69,45 @@ struct DkdvLayout {
   static constexpr uint32_t kV = kK + kTile;
   static constexpr uint32_t kQ = kV + kTile;          // 2 stages
   static constexpr uint32_t kDO = kQ + 2 * kTile;     // 2 stages
-  static constexpr uint32_t kLse = kDO + 2 * kTile;   // 2 stages x 128 floats
-  static constexpr uint32_t kDv = kLse + 1024;        // 2 stages x 128 floats
+  static constexpr uint32_t kStage = kDO + 2 * kTile; // dS tile, or the dV / dK tile, 32 KB
+  static constexpr uint32_t kLse = kStage + kDsTileBytes;   // 2 stages x 128 floats
+  static constexpr uint32_t kDv = kLse + 1024;               // 2 stages x 128 floats
   static constexpr uint32_t kBar = kDv + 1024;
-  enum { B_KV = 0, B_QF = 1, B_QE = 3, B_S = 5, B_DP = 6, B_P = 7, B_DS = 8, B_ACC = 9,
-         B_DRAIN = 10, B_COUNT = 11 };
+  enum { B_KV = 0, B_KVE = 1, B_QF = 2, B_QE = 4, B_S = 6, B_DP = 7, B_P = 8, B_DS = 9,
+         B_ACC = 10, B_ACCE = 11, B_STF = 12, B_STE = 13, B_DRAIN = 14, B_COUNT = 15 };
   static constexpr uint32_t kTmemSlot = kBar + B_COUNT * 8;
   static constexpr uint32_t kAbort = kTmemSlot + 4;
   static constexpr uint32_t kBytes = kAbort + 4;
-  static constexpr uint32_t kLaunchBytes =
-      (kBytes + 1024 > 116 * 1024) ? kBytes + 1024 : 116 * 1024;
-  static constexpr int kThreads = 320;
+  // No alignment slack: the kernel checks that the window starts on a 1024-byte boundary.
+  static constexpr uint32_t kLaunchBytes = kBytes > 116 * 1024 ? kBytes : 116 * 1024;
+  static constexpr int kThreads = 352;
 };
 
+// Work tile u (heaviest first) of this pass -> (b, kv head, first original row).
+__device__ __forceinline__ void dkdv_tile(const BwdParams& p, int u, int& b, int& kvh, int& t0) {
+  const int rep = p.Hq / p.Hkv;
+  int shb = p.shift_head_begin - p.kvh_begin * rep;
+  shb = shb < 0 ? 0 : (shb > p.kvh_count * rep ? p.kvh_count * rep : shb);
+  kv_tile_coords(u, p.B, p.kvh_count * rep, p.kvh_count, p.N, p.G, shb, p.shift, b, kvh, t0);
+  kvh += p.kvh_begin;
+}
+
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
     s2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQ8,
                        const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmK8,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmV8,
                        const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmO8,
+                       const __grid_constant__ CUtensorMap tmDK, const __grid_constant__ CUtensorMap tmDV,
                        const BwdParams p) {
   using L = DkdvLayout<D>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = aligned_smem(smem_raw);
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw;
   const uint32_t sbase = smem_u32(smem);
+  if (sbase & 1023u) {   // the layout has no slack for realignment: report, do nothing
+    if (threadIdx.x == 0) atomicCAS(p.err, 0u, (static_cast<uint32_t>(KID_DKDV) << 8) | 0xFFu);
+    return;
+  }
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   auto bar = [&](int i) { return sbase + L::kBar + 8u * i; };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
@@ -95,19 +115,19 @@ __global__ void __launch_bounds__(320, 1)
   const WaitCtx ctx{abort_flag, p.err, p.timeout_ns, KID_DKDV};
 
   const int rep = p.Hq / p.Hkv;
-  int b, kvh, t0;
-  {
-    int shb = p.shift_head_begin - p.kvh_begin * rep;
-    shb = shb < 0 ? 0 : (shb > p.kvh_count * rep ? p.kvh_count * rep : shb);
-    kv_tile_coords(blockIdx.x, p.B, p.kvh_count * rep, p.kvh_count, p.N, p.G, shb, p.shift, b,
-                   kvh, t0);
-    kvh += p.kvh_begin;
-  }
-  const int h_begin = kvh * rep;
+  const int T = (p.N + kTileRows - 1) / kTileRows;
+  const int n_tiles = p.B * p.kvh_count * T;
   auto head_shift = [&](int hq) { return hq >= p.shift_head_begin ? p.shift : 0; };
+  auto pairs_of = [&](int kvh, int t0) {
+    int total = 0;
+    for (int hq = kvh * rep; hq < (kvh + 1) * rep; ++hq)
+      total += kv_tile_qtiles(t0, head_shift(hq), p.N, p.G).count();
+    return total;
+  };
 
   if (warp == 8 && lane == 0) {
     mbar_init(bar(L::B_KV), 1);
+    mbar_init(bar(L::B_KVE), 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(L::B_QF + s), 1);
       mbar_init(bar(L::B_QE + s), 1);
@@ -117,6 +137,9 @@ __global__ void __launch_bounds__(320, 1)
     mbar_init(bar(L::B_P), 256);
     mbar_init(bar(L::B_DS), 256);
     mbar_init(bar(L::B_ACC), 1);
+    mbar_init(bar(L::B_ACCE), 256);
+    mbar_init(bar(L::B_STF), 256);
+    mbar_init(bar(L::B_STE), 1);
     mbar_init(bar(L::B_DRAIN), 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -140,36 +163,43 @@ __global__ void __launch_bounds__(320, 1)
     // ---------------- TMA producer ----------------
     if (lane == 0) {
       int last_parity[2] = {-1, -1};
-      mbar_expect_tx(bar(L::B_KV), 2 * L::kTile);
-      const TileRuns kv_runs = rolled_tile_runs(t0, 0, p.N);
-      load_tile<D>(sbase + L::kK, &tmK, &tmK8, bar(L::B_KV), b, kvh, kv_runs, p.N);
-      load_tile<D>(sbase + L::kV, &tmV, &tmV8, bar(L::B_KV), b, kvh, kv_runs, p.N);
-      int n = 0;
+      int n = 0, tc = 0, kv_loads = 0;
       bool ok = true;
-      for (int hq = h_begin; ok && hq < h_begin + rep; ++hq) {
-        const int sh = head_shift(hq);
-        const QTileRanges qr = kv_tile_qtiles(t0, sh, p.N, p.G);
-        const float* lse_row = p.lse2 + (static_cast<size_t>(b) * p.Hq + hq) * p.N;
-        const float* d_row = p.dvec + (static_cast<size_t>(b) * p.Hq + hq) * p.N;
-        for (int i = 0; i < qr.count(); ++i, ++n) {
-          const int st = n & 1;
-          if (n >= 2 && !wait_bar(bar(L::B_QE + st), ((n >> 1) - 1) & 1, ctx, 1)) { ok = false; break; }
-          const TileRuns tr = rolled_tile_runs(qr.at(i) * kTileRows, sh, p.N);
-          const uint32_t fb = bar(L::B_QF + st);
-          mbar_expect_tx(fb, 2 * L::kTile + 8u * tr.valid);
-          load_tile<D>(sbase + L::kQ + st * L::kTile, &tmQ, &tmQ8, fb, b, hq, tr, p.N);
-          load_tile<D>(sbase + L::kDO + st * L::kTile, &tmO, &tmO8, fb, b, hq, tr, p.N);
-          const uint32_t sl = sbase + L::kLse + st * 512, sd = sbase + L::kDv + st * 512;
-          bulk_load(sl, lse_row + tr.start, 4u * tr.first, fb);
-          bulk_load(sd, d_row + tr.start, 4u * tr.first, fb);
-          if (tr.valid > tr.first) {
-            bulk_load(sl + 4u * tr.first, lse_row, 4u * (tr.valid - tr.first), fb);
-            bulk_load(sd + 4u * tr.first, d_row, 4u * (tr.valid - tr.first), fb);
+      for (int u = blockIdx.x; ok && u < n_tiles; u += gridDim.x, ++tc) {
+        int b, kvh, t0;
+        dkdv_tile(p, u, b, kvh, t0);
+        // K and V of the previous tile are free once its last S and dP MMAs are done.
+        if (tc > 0 && !wait_bar(bar(L::B_KVE), (tc - 1) & 1, ctx, 11)) { ok = false; break; }
+        mbar_expect_tx(bar(L::B_KV), 2 * L::kTile);
+        const TileRuns kv_runs = rolled_tile_runs(t0, 0, p.N);
+        load_tile<D>(sbase + L::kK, &tmK, &tmK8, bar(L::B_KV), b, kvh, kv_runs, p.N);
+        load_tile<D>(sbase + L::kV, &tmV, &tmV8, bar(L::B_KV), b, kvh, kv_runs, p.N);
+        ++kv_loads;
+        for (int hq = kvh * rep; ok && hq < (kvh + 1) * rep; ++hq) {
+          const int sh = head_shift(hq);
+          const QTileRanges qr = kv_tile_qtiles(t0, sh, p.N, p.G);
+          const float* lse_row = p.lse2 + (static_cast<size_t>(b) * p.Hq + hq) * p.N;
+          const float* d_row = p.dvec + (static_cast<size_t>(b) * p.Hq + hq) * p.N;
+          for (int i = 0; i < qr.count(); ++i, ++n) {
+            const int st = n & 1;
+            if (n >= 2 && !wait_bar(bar(L::B_QE + st), ((n >> 1) - 1) & 1, ctx, 1)) { ok = false; break; }
+            const TileRuns tr = rolled_tile_runs(qr.at(i) * kTileRows, sh, p.N);
+            const uint32_t fb = bar(L::B_QF + st);
+            mbar_expect_tx(fb, 2 * L::kTile + 8u * tr.valid);
+            load_tile<D>(sbase + L::kQ + st * L::kTile, &tmQ, &tmQ8, fb, b, hq, tr, p.N);
+            load_tile<D>(sbase + L::kDO + st * L::kTile, &tmO, &tmO8, fb, b, hq, tr, p.N);
+            const uint32_t sl = sbase + L::kLse + st * 512, sd = sbase + L::kDv + st * 512;
+            bulk_load(sl, lse_row + tr.start, 4u * tr.first, fb);
+            bulk_load(sd, d_row + tr.start, 4u * tr.first, fb);
+            if (tr.valid > tr.first) {
+              bulk_load(sl + 4u * tr.first, lse_row, 4u * (tr.valid - tr.first), fb);
+              bulk_load(sd + 4u * tr.first, d_row, 4u * (tr.valid - tr.first), fb);
+            }
+            last_parity[st] = (n >> 1) & 1;
           }
-          last_parity[st] = (n >> 1) & 1;
         }
       }
-      drain_wait(bar(L::B_KV), 0, p.timeout_ns);
+      if (kv_loads > 0) drain_wait(bar(L::B_KV), (kv_loads - 1) & 1, p.timeout_ns);
       for (int s = 0; s < 2; ++s)
         if (last_parity[s] >= 0) drain_wait(bar(L::B_QF + s), last_parity[s], p.timeout_ns);
     }
@@ -178,161 +208,221 @@ __global__ void __launch_bounds__(320, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16(128, 128, false, false);  // K Q^T, V dO^T
       constexpr uint32_t idesc_acc = idesc_bf16(128, D, false, true);   // P^T dO, dS^T Q
-      int total = 0;
-      for (int hq = h_begin; hq < h_begin + rep; ++hq)
-        total += kv_tile_qtiles(t0, head_shift(hq), p.N, p.G).count();
-      auto issue_nt = [&](uint32_t d_tmem, uint32_t a_base, uint32_t b_base) {
-        gemm_ss_k<D>(d_tmem, a_base, b_base, idesc_s);
-      };
-      auto issue_acc = [&](uint32_t d_tmem, uint32_t a_tmem, uint32_t b_base, int n) {
-        gemm_ts_mn<D>(d_tmem, a_tmem, b_base, idesc_acc, n > 0);
-      };
-      bool ok = wait_bar(bar(L::B_KV), 0, ctx, 2);
-      if (ok && total > 0) ok = wait_bar(bar(L::B_QF + 0), 0, ctx, 3);
-      if (ok && total > 0) {
+      int n = 0, tc = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < n_tiles; u += gridDim.x, ++tc) {
+        int b, kvh, t0;
+        dkdv_tile(p, u, b, kvh, t0);
+        const int total = pairs_of(kvh, t0);
+        ok = wait_bar(bar(L::B_KV), tc & 1, ctx, 2) &&
+             wait_bar(bar(L::B_QF + (n & 1)), (n >> 1) & 1, ctx, 3);
+        if (!ok) break;
         tc_fence_after();
-        issue_nt(tm_s, sbase + L::kK, sbase + L::kQ);
+        gemm_ss_k<D>(tm_s, sbase + L::kK, sbase + L::kQ + (n & 1) * L::kTile, idesc_s);
         mma_commit(bar(L::B_S));
-      }
-      for (int n = 0; ok && n < total; ++n) {
-        const int st = n & 1;
-        const uint32_t q_s = sbase + L::kQ + st * L::kTile, do_s = sbase + L::kDO + st * L::kTile;
-        issue_nt(tm_dp, sbase + L::kV, do_s);
-        mma_commit(bar(L::B_DP));
-        if (!wait_bar(bar(L::B_P), n & 1, ctx, 4)) { ok = false; break; }
-        tc_fence_after();
-        issue_acc(tm_dv, tm_p, do_s, n);
-        if (n + 1 < total) {
-          const int st1 = (n + 1) & 1;
-          if (!wait_bar(bar(L::B_QF + st1), ((n + 1) >> 1) & 1, ctx, 5)) { ok = false; break; }
+        for (int i = 0; i < total; ++i, ++n) {
+          const int st = n & 1;
+          const uint32_t q_s = sbase + L::kQ + st * L::kTile, do_s = sbase + L::kDO + st * L::kTile;
+          gemm_ss_k<D>(tm_dp, sbase + L::kV, do_s, idesc_s);
+          mma_commit(bar(L::B_DP));
+          if (i + 1 == total) mma_commit(bar(L::B_KVE));   // last reader of K and V issued
+          if (!wait_bar(bar(L::B_P), n & 1, ctx, 4)) { ok = false; break; }
+          // The previous tile's dV and dK must have been read out before they restart.
+          if (i == 0 && tc > 0 && !wait_bar(bar(L::B_ACCE), (tc - 1) & 1, ctx, 12)) { ok = false; break; }
           tc_fence_after();
-          issue_nt(tm_s, sbase + L::kK, sbase + L::kQ + st1 * L::kTile);
-          mma_commit(bar(L::B_S));
+          gemm_ts_mn<D>(tm_dv, tm_p, do_s, idesc_acc, i > 0);
+          if (i + 1 < total) {
+            const int st1 = (n + 1) & 1;
+            if (!wait_bar(bar(L::B_QF + st1), ((n + 1) >> 1) & 1, ctx, 5)) { ok = false; break; }
+            tc_fence_after();
+            gemm_ss_k<D>(tm_s, sbase + L::kK, sbase + L::kQ + st1 * L::kTile, idesc_s);
+            mma_commit(bar(L::B_S));
+          }
+          if (!wait_bar(bar(L::B_DS), n & 1, ctx, 6)) { ok = false; break; }
+          tc_fence_after();
+          gemm_ts_mn<D>(tm_dk, tm_ds, q_s, idesc_acc, i > 0);
+          mma_commit(bar(L::B_QE + st));
         }
-        if (!wait_bar(bar(L::B_DS), n & 1, ctx, 6)) { ok = false; break; }
-        tc_fence_after();
-        issue_acc(tm_dk, tm_ds, q_s, n);
-        mma_commit(bar(L::B_QE + st));
+        if (ok) mma_commit(bar(L::B_ACC));
       }
-      if (ok) mma_commit(bar(L::B_ACC));
+    }
+  } else if (warp == 10) {
+    // ---------------- store issuer ----------------
+    // Mirrors the elementwise warps' use of the staging buffer: per query tile a dS tile
+    // (when handing off to the dQ pass), per work tile dV then dK.
+    if (lane == 0) {
+      int use = 0;
+      bool ok = true;
+      mbar_arrive(bar(L::B_STE));   // the buffer starts out free
+      auto hand_over = [&](auto&& issue) -> bool {
+        if (!wait_bar(bar(L::B_STF), use & 1, ctx, 13)) return false;
+        issue();
+        bulk_commit();
+        bulk_wait_read_all();
+        mbar_arrive(bar(L::B_STE));
+        ++use;
+        return true;
+      };
+      for (int u = blockIdx.x; ok && u < n_tiles; u += gridDim.x) {
+        int b, kvh, t0;
+        dkdv_tile(p, u, b, kvh, t0);
+        if (p.ds) {
+          for (int hq = kvh * rep; ok && hq < (kvh + 1) * rep; ++hq) {
+            const int sh = head_shift(hq);
+            const QTileRanges qr = kv_tile_qtiles(t0, sh, p.N, p.G);
+            for (int i = 0; ok && i < qr.count(); ++i) {
+              const int qt = qr.at(i);
+              const KvSpan sp = qtile_kv_span(qt, sh, p.N, p.G);
+              int idx = t0 / kTileRows - sp.first;
+              if (idx < 0) idx += T;
+              ok = hand_over([&] {
+                if (idx < sp.count)
+                  bulk_store(ds_slot_ptr(p, b, hq, p.slots.base(qt) + idx), sbase + L::kStage,
+                             kDsTileBytes);
+              });
+            }
+          }
+        }
+        for (int which = 0; ok && which < 2; ++which)
+          ok = hand_over([&] {
+#pragma unroll
+            for (int h = 0; h < D / 64; ++h)
+              tma_store_4d(which == 0 ? &tmDV : &tmDK, sbase + L::kStage + h * Tile<D>::kHalfBytes,
+                           64 * h, kvh, t0, b);
+          });
+      }
+      bulk_wait_all();
     }
   } else {
     // ---------------- elementwise warps 0-7 ----------------
     const int half = warp / 4;                     // query columns [64 half, 64 half + 64)
     const int row = (warp % 4) * 32 + lane;
-    const int t = t0 + row;
-    const bool kv_valid = t < p.N;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>((warp % 4) * 32) << 16);
     const float c = p.scale_log2;
     const float* s_lse = reinterpret_cast<const float*>(smem + L::kLse);
     const float* s_dv = reinterpret_cast<const float*>(smem + L::kDv);
-    int n = 0;
+    uint8_t* stage = smem + L::kStage;
+    int n = 0, tc = 0, use = 0;
     bool ok = true;
-    for (int hq = h_begin; ok && hq < h_begin + rep; ++hq) {
-      const int sh = head_shift(hq);
-      const QTileRanges qr = kv_tile_qtiles(t0, sh, p.N, p.G);
-      const int r_k = kv_valid ? (t - sh < 0 ? t - sh + p.N : t - sh) : 0;
-      const int ge_k = group_end(r_k, p.G);
-      for (int i = 0; i < qr.count(); ++i, ++n) {
-        const int st = n & 1;
-        const int qt = qr.at(i);
-        const int q0 = qt * kTileRows + 64 * half;
-        const int cl = kv_valid ? r_k - q0 : 1;
-        const int ch = kv_valid ? ge_k - 1 - q0 : 0;
-        const bool mask = __any_sync(0xffffffffu, cl > 0 || ch < 63);
-        if (!warp_wait(bar(L::B_QF + st), (n >> 1) & 1, ctx, 7)) { ok = false; break; }
-        if (!warp_wait(bar(L::B_S), n & 1, ctx, 8)) { ok = false; break; }
-        tc_fence_after();
-        const float* lse_t = s_lse + st * 128 + 64 * half;
-        const float* d_t = s_dv + st * 128 + 64 * half;
-        // P^T phase: 64 columns of S^T -> P^T (bf16), kept in registers for the dS phase.
-        uint32_t pk[32];
-        {
-          uint32_t raw[64];
-          tmem_ld64(t_lane + 64 * half, raw);
+    // Wait for the staging buffer, fill it with `fill`, hand it to the store issuer.
+    auto stage_out = [&](auto&& fill) -> bool {
+      if (!warp_wait(bar(L::B_STE), use & 1, ctx, 14)) return false;
+      fill();
+      fence_async_smem();
+      mbar_arrive(bar(L::B_STF));
+      ++use;
+      return true;
+    };
+    for (int u = blockIdx.x; ok && u < n_tiles; u += gridDim.x, ++tc) {
+      int b, kvh, t0;
+      dkdv_tile(p, u, b, kvh, t0);
+      const int t = t0 + row;
+      const bool kv_valid = t < p.N;
+      for (int hq = kvh * rep; ok && hq < (kvh + 1) * rep; ++hq) {
+        const int sh = head_shift(hq);
+        const QTileRanges qr = kv_tile_qtiles(t0, sh, p.N, p.G);
+        const int r_k = kv_valid ? (t - sh < 0 ? t - sh + p.N : t - sh) : 0;
+        const int ge_k = group_end(r_k, p.G);
+        for (int i = 0; i < qr.count(); ++i, ++n) {
+          const int st = n & 1;
+          const int q0 = qr.at(i) * kTileRows + 64 * half;
+          const int cl = kv_valid ? r_k - q0 : 1;
+          const int ch = kv_valid ? ge_k - 1 - q0 : 0;
+          const bool mask = __any_sync(0xffffffffu, cl > 0 || ch < 63);
+          if (!warp_wait(bar(L::B_QF + st), (n >> 1) & 1, ctx, 7)) { ok = false; break; }
+          if (!warp_wait(bar(L::B_S), n & 1, ctx, 8)) { ok = false; break; }
+          tc_fence_after();
+          const float* lse_t = s_lse + st * 128 + 64 * half;
+          const float* d_t = s_dv + st * 128 + 64 * half;
+          // P^T phase: 64 columns of S^T -> P^T (bf16), kept in registers for the dS phase.
+          uint32_t pk[32];
+          {
+            uint32_t raw[64];
+            tmem_ld64(t_lane + 64 * half, raw);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int col = 2 * e;
-            float x0 = fast_exp2(fmaf(__uint_as_float(raw[col]), c, -lse_t[col]));
-            float x1 = fast_exp2(fmaf(__uint_as_float(raw[col + 1]), c, -lse_t[col + 1]));
-            if (mask) {
-              x0 = (col >= cl && col <= ch) ? x0 : 0.f;
-              x1 = (col + 1 >= cl && col + 1 <= ch) ? x1 : 0.f;
+            for (int e = 0; e < 32; ++e) {
+              const int col = 2 * e;
+              float x0 = fast_exp2(fmaf(__uint_as_float(raw[col]), c, -lse_t[col]));
+              float x1 = fast_exp2(fmaf(__uint_as_float(raw[col + 1]), c, -lse_t[col + 1]));
+              if (mask) {
+                x0 = (col >= cl && col <= ch) ? x0 : 0.f;
+                x1 = (col + 1 >= cl && col + 1 <= ch) ? x1 : 0.f;
+              }
+              pk[e] = pack_bf16(x0, x1);
             }
-            pk[e] = pack_bf16(x0, x1);
           }
-        }
-        tmem_st32(t_lane + 32 + 32 * half, pk);
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(bar(L::B_P));
-        // dS^T phase: dS^T = P^T o (dP^T - D).
-        if (!warp_wait(bar(L::B_DP), n & 1, ctx, 9)) { ok = false; break; }
-        tc_fence_after();
-        uint32_t ds[32];
-        {
-          uint32_t raw[64];
-          tmem_ld64(t_lane + 128 + 64 * half, raw);
+          tmem_st32(t_lane + 32 + 32 * half, pk);
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(bar(L::B_P));
+          // dS^T phase: dS^T = P^T o (dP^T - D).
+          if (!warp_wait(bar(L::B_DP), n & 1, ctx, 9)) { ok = false; break; }
+          tc_fence_after();
+          uint32_t ds[32];
+          {
+            uint32_t raw[64];
+            tmem_ld64(t_lane + 128 + 64 * half, raw);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int col = 2 * e;
-            const float2 pf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[e]));
-            float y0 = pf.x * (__uint_as_float(raw[col]) - d_t[col]);
-            float y1 = pf.y * (__uint_as_float(raw[col + 1]) - d_t[col + 1]);
-            if (mask) {   // exact zeros where P is masked, whatever D holds for padding rows
-              y0 = (col >= cl && col <= ch) ? y0 : 0.f;
-              y1 = (col + 1 >= cl && col + 1 <= ch) ? y1 : 0.f;
+            for (int e = 0; e < 32; ++e) {
+              const int col = 2 * e;
+              const float2 pf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[e]));
+              float y0 = pf.x * (__uint_as_float(raw[col]) - d_t[col]);
+              float y1 = pf.y * (__uint_as_float(raw[col + 1]) - d_t[col + 1]);
+              if (mask) {   // exact zeros where P is masked, whatever D holds for padding rows
+                y0 = (col >= cl && col <= ch) ? y0 : 0.f;
+                y1 = (col + 1 >= cl && col + 1 <= ch) ? y1 : 0.f;
+              }
+              ds[e] = pack_bf16(y0, y1);
             }
-            ds[e] = pack_bf16(y0, y1);
+            tmem_st32(t_lane + 160 + 32 * half, ds);
           }
-          tmem_st32(t_lane + 160 + 32 * half, ds);
-        }
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(bar(L::B_DS));
-        if (p.ds) {
-          // Hand the tile to the dQ pass, after the arrive so the stores stay off the tensor
-          // core's critical path. Layout (DsSlots): 16 blocks of 2 KB, block c holding query
-          // columns [8c, 8c + 8) of all 128 kv rows, 16 bytes per row — so each store below
-          // writes 512 contiguous bytes per warp. Streaming stores: the tile is read once,
-          // by another kernel, and should not evict this kernel's operands from L2.
-          const KvSpan sp = qtile_kv_span(qt, sh, p.N, p.G);
-          int idx = t0 / kTileRows - sp.first;
-          if (idx < 0) idx += (p.N + kTileRows - 1) / kTileRows;
-          if (idx < sp.count) {
-            uint4* dst = reinterpret_cast<uint4*>(ds_slot_ptr(p, b, hq, p.slots.base(qt) + idx)) +
-                         half * 8 * kTileRows + row;
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(bar(L::B_DS));
+          if (p.ds) {
+            // The dS tile for the dQ pass, in its global layout (DsSlots): 16 blocks of 2 KB,
+            // block c holding query columns [8c, 8c + 8) of all 128 kv rows, 16 bytes per row.
+            ok = stage_out([&] {
 #pragma unroll
-            for (int c8 = 0; c8 < 8; ++c8)
-              __stcs(dst + c8 * kTileRows,
-                     make_uint4(ds[4 * c8], ds[4 * c8 + 1], ds[4 * c8 + 2], ds[4 * c8 + 3]));
+              for (int c8 = 0; c8 < 8; ++c8)
+                *reinterpret_cast<uint4*>(stage + (half * 8 + c8) * 2048 + row * 16) =
+                    make_uint4(ds[4 * c8], ds[4 * c8 + 1], ds[4 * c8 + 2], ds[4 * c8 + 3]);
+            });
+            if (!ok) break;
           }
         }
       }
-    }
-    if (ok && warp_wait(bar(L::B_ACC), 0, ctx, 10)) {
+      if (!ok || !warp_wait(bar(L::B_ACC), tc & 1, ctx, 10)) { ok = false; break; }
       tc_fence_after();
-      const size_t orow = ((static_cast<size_t>(b) * p.N + (kv_valid ? t : 0)) * p.Hkv + kvh) * D;
-#pragma unroll
-      for (int which = 0; which < 2; ++which) {
+      // dV, then scale * dK: this thread's D/2 columns of its row, in bf16, into the staging
+      // buffer in the 128-byte-swizzled layout of the TMA tile (64-column boxes of 128 rows).
+#pragma unroll 1
+      for (int which = 0; ok && which < 2; ++which) {
         const uint32_t src = (which == 0 ? tm_dv : tm_dk) - tmem + t_lane;
         const float mul = which == 0 ? 1.f : p.scale;
-        __nv_bfloat16* dst_row = (which == 0 ? p.dv : p.dk) + orow;
+        uint32_t pkd[D / 4];
 #pragma unroll
-        for (int j = half * (D / 64); j < (half + 1) * (D / 64); ++j) {
+        for (int j = 0; j < D / 64; ++j) {
           uint32_t rr[32];
-          tmem_ld32(src + 32 * j, rr);
-          uint32_t pk[16];
+          tmem_ld32(src + (D / 2) * half + 32 * j, rr);
 #pragma unroll
           for (int e = 0; e < 16; ++e)
-            pk[e] = pack_bf16(__uint_as_float(rr[2 * e]) * mul, __uint_as_float(rr[2 * e + 1]) * mul);
-          if (kv_valid) {
-            uint4* dst = reinterpret_cast<uint4*>(dst_row + 32 * j);
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-              dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-          }
+            pkd[16 * j + e] = pack_bf16(__uint_as_float(rr[2 * e]) * mul, __uint_as_float(rr[2 * e + 1]) * mul);
         }
+        if (which == 1) {   // both accumulators are in registers: the MMA may reuse them
+          tc_fence_before();
+          mbar_arrive(bar(L::B_ACCE));
+        }
+        ok = stage_out([&] {
+#pragma unroll
+          for (int v = 0; v < D / 16; ++v) {
+            const int col = (D / 2) * half + 8 * v;   // first of the 8 columns of chunk v
+            const int box = col / 64, chunk = (col % 64) / 8;
+            *reinterpret_cast<uint4*>(stage + box * Tile<D>::kHalfBytes + row * 128 +
+                                      ((chunk ^ (row & 7)) * 16)) =
+                make_uint4(pkd[4 * v], pkd[4 * v + 1], pkd[4 * v + 2], pkd[4 * v + 3]);
+          }
+        });
       }
     }
   }

@@ -16,9 +16,9 @@
 //   warps 0-3, 4-7  softmax warpgroup of query tile 0 / 1: thread i owns query row i (TMEM
 //                   lane i); online softmax in fp32, P written back to TMEM as bf16 over S,
 //                   O rescaled in TMEM when the running max grows, epilogue.
-//   warp 8          TMA producer: both Q tiles once, then K tiles (3-stage ring) running one
-//                   tile ahead of V tiles (2-stage ring); each ring slot is released by a
-//                   commit right after the last MMA that reads it.
+//   warp 8          TMA producer: both Q tiles once, then K tiles running one tile ahead of
+//                   V tiles (2-slot rings); each ring slot is released by a commit right
+//                   after the last MMA that reads it.
 //   warp 9          TMEM allocator and MMA issuer (one lane).
 // TMEM columns: S0/P0 [0,128), S1/P1 [128,256), O0 [256,256+D), O1 [256+D, 256+2D).
 //
@@ -26,6 +26,9 @@
 // softmax run while the tensor core works on the other tile. tcgen05 MMAs from one thread
 // complete in issue order, so when S_t(j+1) is signalled, PV_t(j) — which read P_t(j) from
 // the same columns and accumulated into O_t — is complete: the softmax may rescale O_t at once.
+//
+// The epilogue stages each warp's 32 rows of O (64 columns at a time) in shared memory and
+// writes whole 128-byte row segments, four rows per store instruction.
 #pragma once
 
 #include "s2_common.cuh"
@@ -49,13 +52,16 @@ constexpr float kRescaleThreshold = 8.0f;
 template <int D>
 struct FwdLayout {
   static constexpr uint32_t kTile = Tile<D>::kBytes;
-  static constexpr int kKStages = 3, kVStages = 2;
+  static constexpr int kKStages = 2, kVStages = 2;
   static constexpr uint32_t kQ = 0;                         // 2 query tiles
   static constexpr uint32_t kK = kQ + 2 * kTile;            // K ring
   static constexpr uint32_t kV = kK + kKStages * kTile;     // V ring
-  static constexpr uint32_t kBar = kV + kVStages * kTile;
-  enum { B_Q = 0, B_QE = 2, B_K = 4, B_KE = 7, B_V = 10, B_VE = 12, B_S = 14, B_P = 16,
-         B_ODONE = 18, B_DRAIN = 20, B_COUNT = 21 };
+  static constexpr uint32_t kStageWarp = 32 * 128;          // O staging: 32 rows x 64 columns
+  static constexpr uint32_t kStage = kV + kVStages * kTile; // ... for each softmax warp
+  static constexpr uint32_t kBar = kStage + 8 * kStageWarp;
+  enum { B_Q = 0, B_QE = 2, B_K = 4, B_KE = B_K + kKStages, B_V = B_KE + kKStages,
+         B_VE = B_V + kVStages, B_S = B_VE + kVStages, B_P = B_S + 2, B_ODONE = B_P + 2,
+         B_DRAIN = B_ODONE + 2, B_COUNT = B_DRAIN + 1 };
   static constexpr uint32_t kTmemSlot = kBar + B_COUNT * 8;
   static constexpr uint32_t kAbort = kTmemSlot + 4;
   static constexpr uint32_t kBytes = kAbort + 4;
@@ -364,16 +370,19 @@ __global__ void __launch_bounds__(320, 1)
       if (!ok || !warp_wait(bar(L::B_ODONE + wg), o_cnt & 1, ctx, 8)) { ok = false; break; }
       ++o_cnt;
       tc_fence_after();
+      // Epilogue: O / l in bf16 through this warp's staging area (row `lane` of the warp at
+      // 128 bytes per 64 columns, 16-byte chunks XOR-swizzled by row), then stored four rows
+      // at a time: lane l writes chunk l % 8 of row 4 i + l / 8 — whole 128-byte segments
+      // instead of 16-byte pieces of 32 different rows.
       const float inv_l = 1.f / l_run;
-      const long long tt = static_cast<long long>(r) + u.shift_h;
-      const int t = static_cast<int>(tt >= p.N ? tt - p.N : tt);
-      __nv_bfloat16* orow =
-          p.o + ((static_cast<size_t>(u.b) * p.N + (row_valid ? t : 0)) * p.Hq + u.h) * D;
+      uint8_t* stage = smem + L::kStage + warp * L::kStageWarp;
+      const int r_warp = u.qt[wg] * kTileRows + (warp % 4) * 32;
+#pragma unroll 1
+      for (int half = 0; half < D / 64; ++half) {
 #pragma unroll
-      for (int j = 0; j < D / 32; ++j) {
-        uint32_t ov[32];
-        tmem_ld32(o_col + 32 * j, ov);
-        if (row_valid) {
+        for (int q2 = 0; q2 < 2; ++q2) {
+          uint32_t ov[32];
+          tmem_ld32(o_col + 64 * half + 32 * q2, ov);
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
             uint4 w4;
@@ -381,13 +390,32 @@ __global__ void __launch_bounds__(320, 1)
             w4.y = pack_bf16(__uint_as_float(ov[8 * v + 2]) * inv_l, __uint_as_float(ov[8 * v + 3]) * inv_l);
             w4.z = pack_bf16(__uint_as_float(ov[8 * v + 4]) * inv_l, __uint_as_float(ov[8 * v + 5]) * inv_l);
             w4.w = pack_bf16(__uint_as_float(ov[8 * v + 6]) * inv_l, __uint_as_float(ov[8 * v + 7]) * inv_l);
-            reinterpret_cast<uint4*>(orow + 32 * j)[v] = w4;
+            const int chunk = 4 * q2 + v;
+            *reinterpret_cast<uint4*>(stage + lane * 128 + ((chunk ^ (lane & 7)) * 16)) = w4;
           }
         }
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int rr = 4 * i + (lane >> 3), chunk = lane & 7;
+          const uint4 w4 = *reinterpret_cast<const uint4*>(stage + rr * 128 + ((chunk ^ (rr & 7)) * 16));
+          const int rq = r_warp + rr;
+          if (rq < p.N) {
+            const long long tq = static_cast<long long>(rq) + u.shift_h;
+            const int tok = static_cast<int>(tq >= p.N ? tq - p.N : tq);
+            __nv_bfloat16* dst = p.o + ((static_cast<size_t>(u.b) * p.N + tok) * p.Hq + u.h) * D +
+                                 64 * half + 8 * chunk;
+            *reinterpret_cast<uint4*>(dst) = w4;
+          }
+        }
+        __syncwarp();
       }
-      if (row_valid)
-        p.lse[(static_cast<size_t>(u.b) * p.Hq + u.h) * p.N + t] =
+      if (row_valid) {
+        const long long tq = static_cast<long long>(r) + u.shift_h;
+        const int tok = static_cast<int>(tq >= p.N ? tq - p.N : tq);
+        p.lse[(static_cast<size_t>(u.b) * p.Hq + u.h) * p.N + tok] =
             (m_run + __log2f(l_run)) * 0.6931471805599453f;
+      }
       // O_t is read: the next unit's first PV on it waits for this warpgroup's P anyway.
       tc_fence_before();
     }

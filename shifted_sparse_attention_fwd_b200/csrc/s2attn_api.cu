@@ -256,7 +256,7 @@ template <int D, bool kDkdv>
 s2attn_status launch_grad(const Shape& sh, const void* q, const void* k, const void* v,
                           const void* dO, void* dq, void* dk, void* dv, float scale,
                           const void* workspace, cudaStream_t stream, unsigned int* err,
-                          int ds_kvh_begin = -1, int ds_kvh_count = 0) {
+                          int num_sms, int ds_kvh_begin = -1, int ds_kvh_count = 0) {
   MapPair mq, mk, mv, mo;
   s2attn_status s;
   if ((s = encode_pair(mq, q, sh.B, sh.Hq, sh.N, D)) != S2ATTN_OK) return s;
@@ -267,9 +267,13 @@ s2attn_status launch_grad(const Shape& sh, const void* q, const void* k, const v
   if (ds_kvh_begin >= 0) set_ds_pass(p, sh, workspace, ds_kvh_begin, ds_kvh_count);
   const unsigned tiles = (sh.N + 127) / 128;
   if (kDkdv) {
-    const unsigned grid = static_cast<unsigned>(sh.B) * p.kvh_count * tiles;
+    MapPair mdk, mdv;
+    if ((s = encode_pair(mdk, dk, sh.B, sh.Hkv, sh.N, D)) != S2ATTN_OK) return s;
+    if ((s = encode_pair(mdv, dv, sh.B, sh.Hkv, sh.N, D)) != S2ATTN_OK) return s;
+    const unsigned units = static_cast<unsigned>(sh.B) * p.kvh_count * tiles;
+    const unsigned grid = units < static_cast<unsigned>(num_sms) ? units : static_cast<unsigned>(num_sms);
     s2::s2_bwd_dkdv_kernel<D><<<grid, s2::DkdvLayout<D>::kThreads, s2::DkdvLayout<D>::kLaunchBytes, stream>>>(
-        mq.m128, mq.m8, mk.m128, mk.m8, mv.m128, mv.m8, mo.m128, mo.m8, p);
+        mq.m128, mq.m8, mk.m128, mk.m8, mv.m128, mv.m8, mo.m128, mo.m8, mdk.m128, mdv.m128, p);
   } else {
     const unsigned grid = static_cast<unsigned>(sh.B) * sh.Hq * tiles;
     s2::s2_bwd_dq_kernel<D><<<grid, s2::DqLayout<D>::kThreads, s2::DqLayout<D>::kLaunchBytes, stream>>>(
@@ -306,24 +310,25 @@ s2attn_status check_workspace(const Shape& sh, const void* ws, size_t bytes) {
 
 s2attn_status dkdv_impl(const Shape& sh, const void* q, const void* k, const void* v,
                         const void* dO, void* dk, void* dv, float scale, const void* ws,
-                        cudaStream_t stream, unsigned int* err) {
-  return sh.d == 64 ? launch_grad<64, true>(sh, q, k, v, dO, nullptr, dk, dv, scale, ws, stream, err)
-                    : launch_grad<128, true>(sh, q, k, v, dO, nullptr, dk, dv, scale, ws, stream, err);
+                        cudaStream_t stream, unsigned int* err, int num_sms) {
+  return sh.d == 64 ? launch_grad<64, true>(sh, q, k, v, dO, nullptr, dk, dv, scale, ws, stream, err, num_sms)
+                    : launch_grad<128, true>(sh, q, k, v, dO, nullptr, dk, dv, scale, ws, stream, err, num_sms);
 }
 s2attn_status dq_impl(const Shape& sh, const void* q, const void* k, const void* v,
                       const void* dO, void* dq, float scale, const void* ws, cudaStream_t stream,
                       unsigned int* err) {
-  return sh.d == 64 ? launch_grad<64, false>(sh, q, k, v, dO, dq, nullptr, nullptr, scale, ws, stream, err)
-                    : launch_grad<128, false>(sh, q, k, v, dO, dq, nullptr, nullptr, scale, ws, stream, err);
+  return sh.d == 64 ? launch_grad<64, false>(sh, q, k, v, dO, dq, nullptr, nullptr, scale, ws, stream, err, 0)
+                    : launch_grad<128, false>(sh, q, k, v, dO, dq, nullptr, nullptr, scale, ws, stream, err, 0);
 }
 s2attn_status dkdv_ds_impl(const Shape& sh, const void* q, const void* k, const void* v,
                            const void* dO, void* dk, void* dv, float scale, const void* ws,
-                           int kvh_begin, int kvh_count, cudaStream_t stream, unsigned int* err) {
+                           int kvh_begin, int kvh_count, cudaStream_t stream, unsigned int* err,
+                           int num_sms) {
   return sh.d == 64
              ? launch_grad<64, true>(sh, q, k, v, dO, nullptr, dk, dv, scale, ws, stream, err,
-                                     kvh_begin, kvh_count)
+                                     num_sms, kvh_begin, kvh_count)
              : launch_grad<128, true>(sh, q, k, v, dO, nullptr, dk, dv, scale, ws, stream, err,
-                                      kvh_begin, kvh_count);
+                                      num_sms, kvh_begin, kvh_count);
 }
 s2attn_status dq_ds_impl(const Shape& sh, const void* k, void* dq, float scale, const void* ws,
                          int kvh_begin, int kvh_count, cudaStream_t stream, unsigned int* err,
@@ -449,8 +454,10 @@ s2attn_status s2attn_bwd_dkdv(const void* q, const void* k, const void* v, const
   if ((s = check_workspace(sh, workspace, workspace_bytes)) != S2ATTN_OK) return s;
   if ((s = get_encoder()) != S2ATTN_OK) return s;
   unsigned int* err = nullptr;
-  if ((s = device_state(&err)) != S2ATTN_OK) return s;
-  return dkdv_impl(sh, q, k, v, dO, dk, dv, scale, workspace, static_cast<cudaStream_t>(stream), err);
+  int num_sms = 0;
+  if ((s = device_state(&err, &num_sms)) != S2ATTN_OK) return s;
+  return dkdv_impl(sh, q, k, v, dO, dk, dv, scale, workspace, static_cast<cudaStream_t>(stream), err,
+                   num_sms);
 }
 
 s2attn_status s2attn_bwd_dq(const void* q, const void* k, const void* v, const void* dO,
@@ -490,9 +497,10 @@ s2attn_status s2attn_bwd_dkdv_ds(const void* q, const void* k, const void* v, co
   }
   if ((s = get_encoder()) != S2ATTN_OK) return s;
   unsigned int* err = nullptr;
-  if ((s = device_state(&err)) != S2ATTN_OK) return s;
+  int num_sms = 0;
+  if ((s = device_state(&err, &num_sms)) != S2ATTN_OK) return s;
   return dkdv_ds_impl(sh, q, k, v, dO, dk, dv, scale, workspace, 0, Hkv,
-                      static_cast<cudaStream_t>(stream), err);
+                      static_cast<cudaStream_t>(stream), err, num_sms);
 }
 
 s2attn_status s2attn_bwd_dq_ds(const void* k, void* dq, int B, int Hq, int Hkv, int N, int d,
@@ -539,12 +547,14 @@ s2attn_status s2attn_bwd_ex(const void* q, const void* k, const void* v, const v
   const int per_pass = ds_heads_per_pass(sh, workspace_bytes);
   if (per_pass == 0) {
     // Workspace too small for one kv head's dS tiles: the dQ kernel recomputes S and dP.
-    if ((s = dkdv_impl(sh, q, k, v, dO, dk, dv, scale, workspace, st, err)) != S2ATTN_OK) return s;
+    if ((s = dkdv_impl(sh, q, k, v, dO, dk, dv, scale, workspace, st, err, num_sms)) != S2ATTN_OK)
+      return s;
     return dq_impl(sh, q, k, v, dO, dq, scale, workspace, st, err);
   }
   for (int h0 = 0; h0 < sh.Hkv; h0 += per_pass) {
     const int cnt = sh.Hkv - h0 < per_pass ? sh.Hkv - h0 : per_pass;
-    if ((s = dkdv_ds_impl(sh, q, k, v, dO, dk, dv, scale, workspace, h0, cnt, st, err)) != S2ATTN_OK)
+    if ((s = dkdv_ds_impl(sh, q, k, v, dO, dk, dv, scale, workspace, h0, cnt, st, err, num_sms)) !=
+        S2ATTN_OK)
       return s;
     if ((s = dq_ds_impl(sh, k, dq, scale, workspace, h0, cnt, st, err, num_sms)) != S2ATTN_OK)
       return s;
