@@ -137,6 +137,8 @@ void paircoords(int bid, int B, int Hq, int N, int G, int* o) {
   s2::query_pair_coords(bid, B, Hq, N, G, o[0], o[1], o[2]); o[3] = s2::query_pairs_per_head(N); }
 void kvcoords(int bid, int B, int Hq, int Hkv, int N, int G, int shb, int sh, int* o) {
   s2::kv_tile_coords(bid, B, Hq, Hkv, N, G, shb, sh, o[0], o[1], o[2]); }
+void qcoords_chunked(int bid, int B, int Hq, int N, int G, int chunk, int* o) {
+  s2::query_tile_coords_chunked(bid, B, Hq, N, G, chunk, o[0], o[1], o[2]); }
 void kvspan(int qt, int sh, int N, int G, int* o) {
   s2::KvSpan s = s2::qtile_kv_span(qt, sh, N, G); o[0] = s.first; o[1] = s.count; }
 long long dsslots(int N, int G, int shifted, int shift, int qt) {
@@ -325,3 +327,19 @@ def test_ds_entries_reject(lib):
                                 None) == 1
     assert lib.s2attn_bwd_dq_ds(A, None, 1, 4, 4, 256, 64, 64, f, 2, 32, ws, full, None) == 1
     assert lib.s2attn_bwd_dq_ds(A, A, 1, 4, 4, 256, 96, 64, f, 2, 32, ws, full, None) == 2
+
+
+@pytest.mark.parametrize("B,Hq,N,G,chunk", [(1, 32, 8192, 2048, 10), (2, 3, 8192, 2048, 4),
+                                            (1, 4, 256, 64, 10), (1, 2, 384, 192, 3),
+                                            (3, 2, 1024, 256, 5), (1, 1, 1024, 1024, 7)])
+def test_chunked_query_tile_order_is_a_permutation(shim, B, Hq, N, G, chunk):
+    """The L2-grouped order visits every (b, h, tile) once; within a chunk, tiles of equal
+    position in their group are adjacent and the heaviest (last in group) come first."""
+    nt = (N + 127) // 128
+    order = [tuple(call4(shim.qcoords_chunked, bid, B, Hq, N, G, chunk)[:3])
+             for bid in range(B * Hq * nt)]
+    assert set(order) == {(b, h, q) for b in range(B) for h in range(Hq) for q in range(nt)}
+    if G % 128 == 0:
+        tpg = G // 128
+        first = order[:min(chunk, B * Hq * (N // G))]
+        assert all(q % tpg == tpg - 1 for _, _, q in first)
