@@ -88,7 +88,8 @@ __device__ __forceinline__ void dkdv_tile(const BwdParams& p, int u, int& b, int
   const int rep = p.Hq / p.Hkv;
   int shb = p.shift_head_begin - p.kvh_begin * rep;
   shb = shb < 0 ? 0 : (shb > p.kvh_count * rep ? p.kvh_count * rep : shb);
-  kv_tile_coords(u, p.B, p.kvh_count * rep, p.kvh_count, p.N, p.G, shb, p.shift, b, kvh, t0);
+  kv_tile_coords_chunked(u, p.B, p.kvh_count * rep, p.kvh_count, p.N, p.G, shb, p.shift,
+                         kL2Chunk, b, kvh, t0);
   kvh += p.kvh_begin;
 }
 

@@ -45,7 +45,7 @@ struct DqDsLayout {
 __device__ __forceinline__ void dq_ds_tile(const BwdParams& p, int u, int& b, int& hq, int& qt) {
   const int rep = p.Hq / p.Hkv;
   int hl;
-  query_tile_coords(u, p.B, p.kvh_count * rep, p.N, p.G, b, hl, qt);
+  query_tile_coords_chunked(u, p.B, p.kvh_count * rep, p.N, p.G, kL2Chunk, b, hl, qt);
   hq = p.kvh_begin * rep + hl;
 }
 

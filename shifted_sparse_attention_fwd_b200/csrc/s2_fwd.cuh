@@ -101,7 +101,7 @@ struct FwdUnit {
 __device__ __forceinline__ FwdUnit fwd_unit(const FwdParams& p, int unit) {
   FwdUnit u;
   int pair;
-  query_pair_coords(unit, p.B, p.Hq, p.N, p.G, u.b, u.h, pair);
+  query_pair_coords_chunked(unit, p.B, p.Hq, p.N, p.G, kL2Chunk, u.b, u.h, pair);
   const int nqt = (p.N + kTileRows - 1) / kTileRows;
   u.shift_h = u.h >= p.shift_head_begin ? p.shift : 0;
   u.kvh = u.h / (p.Hq / p.Hkv);

@@ -21,6 +21,10 @@ namespace s2 {
 
 constexpr int kTileRows = 128;
 
+// (b, head, group) instances whose tiles the persistent kernels take together: the K/V (or
+// Q/dO) tiles of about this many groups stay resident in L2 while their work runs.
+constexpr int kL2Chunk = 10;
+
 struct TileRuns {
   int valid;   // rows of the tile inside the sequence (rows [valid, 128) are padding)
   int first;   // rows [0, first) come from original rows [start, start + first)
@@ -174,6 +178,30 @@ __host__ __device__ inline void query_tile_coords(int bid, int B, int Hq, int N,
   }
 }
 
+// Block index -> (b, h, rolled query tile), grouped for L2 reuse: the (b, h, group) instances
+// are taken `chunk` at a time, and within a chunk the tiles go heaviest first (last tile of
+// each group first). Work that runs concurrently then reads the key tiles of only `chunk`
+// groups. Falls back to query_tile_coords when G is not a multiple of the tile.
+__host__ __device__ inline void query_tile_coords_chunked(int bid, int B, int Hq, int N, int G,
+                                                          int chunk, int& b, int& h, int& qt) {
+  if (G % kTileRows != 0) {
+    query_tile_coords(bid, B, Hq, N, G, b, h, qt);
+    return;
+  }
+  const int tpg = G / kTileRows, ng = N / G;
+  const int instances = B * Hq * ng;
+  const int per_chunk = chunk * tpg;
+  const int ck = bid / per_chunk, within = bid % per_chunk;
+  const int rest = instances - ck * chunk;
+  const int cl = rest < chunk ? rest : chunk;
+  const int il = tpg - 1 - within / cl;
+  const int inst = ck * chunk + within % cl;
+  const int g = inst % ng, bh = inst / ng;
+  h = bh % Hq;
+  b = bh / Hq;
+  qt = g * tpg + il;
+}
+
 // Block index -> (b, h, pair) for kernels whose CTA owns the two rolled query tiles 2*pair
 // and 2*pair + 1 of one (b, h). When G is a multiple of two tiles, pairs late in their group
 // (more key tiles to visit) come first.
@@ -198,6 +226,29 @@ __host__ __device__ inline void query_pair_coords(int bid, int B, int Hq, int N,
     h = bh % Hq;
     b = bh / Hq;
   }
+}
+
+// Block index -> (b, h, pair) with the same L2 grouping as query_tile_coords_chunked: the
+// (b, h, group) instances `chunk` at a time, heaviest pairs (last in group) first within a
+// chunk. Falls back to query_pair_coords when G is not a multiple of two tiles.
+__host__ __device__ inline void query_pair_coords_chunked(int bid, int B, int Hq, int N, int G,
+                                                          int chunk, int& b, int& h, int& pair) {
+  if (G % (2 * kTileRows) != 0) {
+    query_pair_coords(bid, B, Hq, N, G, b, h, pair);
+    return;
+  }
+  const int ppg = G / (2 * kTileRows), ng = N / G;
+  const int instances = B * Hq * ng;
+  const int per_chunk = chunk * ppg;
+  const int ck = bid / per_chunk, within = bid % per_chunk;
+  const int rest = instances - ck * chunk;
+  const int cl = rest < chunk ? rest : chunk;
+  const int pl = ppg - 1 - within / cl;
+  const int inst = ck * chunk + within % cl;
+  const int g = inst % ng, bh = inst / ng;
+  h = bh % Hq;
+  b = bh / Hq;
+  pair = g * ppg + pl;
 }
 
 // Block index -> (b, kv head, first original row t0 of the kv tile) for the dK/dV kernel.
@@ -225,6 +276,34 @@ __host__ __device__ inline void kv_tile_coords(int bid, int B, int Hq, int Hkv, 
     kvh = bk % Hkv;
     b = bk / Hkv;
   }
+}
+
+// Block index -> (b, kv head, t0) with the L2 grouping of query_tile_coords_chunked: the
+// (b, kv head, rolled group) instances `chunk` at a time, kv tiles early in their group (most
+// query tiles) first within a chunk. Falls back to kv_tile_coords when groups or roll are not
+// tile-aligned.
+__host__ __device__ inline void kv_tile_coords_chunked(int bid, int B, int Hq, int Hkv, int N,
+                                                       int G, int shift_head_begin, int shift,
+                                                       int chunk, int& b, int& kvh, int& t0) {
+  if (!(G % kTileRows == 0 && shift % kTileRows == 0)) {
+    kv_tile_coords(bid, B, Hq, Hkv, N, G, shift_head_begin, shift, b, kvh, t0);
+    return;
+  }
+  const int rep = Hq / Hkv;
+  const int tpg = G / kTileRows, ng = N / G;
+  const int instances = B * Hkv * ng;
+  const int per_chunk = chunk * tpg;
+  const int ck = bid / per_chunk, within = bid % per_chunk;
+  const int rest = instances - ck * chunk;
+  const int cl = rest < chunk ? rest : chunk;
+  const int jl = within / cl;
+  const int inst = ck * chunk + within % cl;
+  const int g = inst % ng, bk = inst / ng;
+  kvh = bk % Hkv;
+  b = bk / Hkv;
+  const int sh = (kvh * rep >= shift_head_begin) ? shift : 0;
+  const int rs = g * G + jl * kTileRows;
+  t0 = rs + sh >= N ? rs + sh - N : rs + sh;
 }
 
 }  // namespace s2

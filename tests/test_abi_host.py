@@ -139,6 +139,11 @@ void kvcoords(int bid, int B, int Hq, int Hkv, int N, int G, int shb, int sh, in
   s2::kv_tile_coords(bid, B, Hq, Hkv, N, G, shb, sh, o[0], o[1], o[2]); }
 void qcoords_chunked(int bid, int B, int Hq, int N, int G, int chunk, int* o) {
   s2::query_tile_coords_chunked(bid, B, Hq, N, G, chunk, o[0], o[1], o[2]); }
+void paircoords_chunked(int bid, int B, int Hq, int N, int G, int chunk, int* o) {
+  s2::query_pair_coords_chunked(bid, B, Hq, N, G, chunk, o[0], o[1], o[2]); }
+void kvcoords_chunked(int bid, int B, int Hq, int Hkv, int N, int G, int shb, int sh, int chunk,
+                      int* o) {
+  s2::kv_tile_coords_chunked(bid, B, Hq, Hkv, N, G, shb, sh, chunk, o[0], o[1], o[2]); }
 void kvspan(int qt, int sh, int N, int G, int* o) {
   s2::KvSpan s = s2::qtile_kv_span(qt, sh, N, G); o[0] = s.first; o[1] = s.count; }
 long long dsslots(int N, int G, int shifted, int shift, int qt) {
@@ -343,3 +348,29 @@ def test_chunked_query_tile_order_is_a_permutation(shim, B, Hq, N, G, chunk):
         tpg = G // 128
         first = order[:min(chunk, B * Hq * (N // G))]
         assert all(q % tpg == tpg - 1 for _, _, q in first)
+
+
+@pytest.mark.parametrize("B,Hq,N,G,chunk", [(1, 32, 8192, 2048, 10), (2, 3, 8192, 2048, 4),
+                                            (1, 4, 256, 64, 10), (1, 2, 640, 128, 3),
+                                            (3, 2, 1024, 256, 5), (1, 1, 1024, 1024, 7)])
+def test_chunked_pair_order_is_a_permutation(shim, B, Hq, N, G, chunk):
+    nt = (N + 127) // 128
+    npair = (nt + 1) // 2
+    order = [tuple(call4(shim.paircoords_chunked, bid, B, Hq, N, G, chunk)[:3])
+             for bid in range(B * Hq * npair)]
+    assert set(order) == {(b, h, q) for b in range(B) for h in range(Hq) for q in range(npair)}
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,G,shb,sh,chunk", [(1, 32, 32, 8192, 2048, 16, 1024, 10),
+                                                        (2, 8, 2, 8192, 2048, 4, 1024, 3),
+                                                        (1, 64, 8, 32768, 8192, 32, 4096, 10),
+                                                        (1, 4, 4, 256, 64, 2, 32, 10),
+                                                        (1, 4, 2, 384, 192, 2, 96, 2)])
+def test_chunked_kv_tile_order_is_a_permutation(shim, B, Hq, Hkv, N, G, shb, sh, chunk):
+    nt = (N + 127) // 128
+    order = []
+    for bid in range(B * Hkv * nt):
+        b, kvh, t0 = call4(shim.kvcoords_chunked, bid, B, Hq, Hkv, N, G, shb, sh, chunk)[:3]
+        assert t0 % 128 == 0
+        order.append((b, kvh, t0 // 128))
+    assert set(order) == {(b, k, t) for b in range(B) for k in range(Hkv) for t in range(nt)}
