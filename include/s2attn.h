@@ -64,7 +64,8 @@ typedef enum {
   S2ATTN_ERR_TIMEOUT = 4
 } s2attn_status;
 
-/* Version of this ABI (bumped on any signature change). */
+/* Version of this ABI (bumped on any signature change or workspace-size change); 2 adds the
+ * dS hand-off entries and the work counters in the backward workspace. */
 S2ATTN_API int s2attn_abi_version(void);
 
 /* Static description of a status code. */
@@ -95,7 +96,8 @@ S2ATTN_API s2attn_status s2attn_fwd_ex(const void* q, const void* k, const void*
                             int shift_head_begin, int shift, void* stream);
 
 /* Smallest device workspace s2attn_bwd accepts: two fp32 [B, Hq, N] arrays (D and LSE in
- * base 2), each rounded up to 256 bytes. With only this much the dQ kernel recomputes S and
+ * base 2), each rounded up to 256 bytes, and 256 bytes of work counters for the gradient
+ * kernels (cleared by the preprocess). With only this much the dQ kernel recomputes S and
  * dP (three GEMMs for one gradient). */
 S2ATTN_API size_t s2attn_bwd_workspace_size(int B, int Hq, int N);
 
@@ -182,8 +184,9 @@ S2ATTN_API s2attn_status s2attn_bwd_dq_ds(const void* k, void* dq, int B, int Hq
  * this entry point; it exists only for such callers.
  *
  * Same arguments and results as s2attn_bwd, minus the workspace. The scratch (D and
- * LSE * log2(e), 8 bytes per (batch, head, token) row, and the dS tiles of the dQ pass when
- * one kv head's fit in the rest) lives in a 16 MiB array compiled into the library: B * Hq * N may be at most 2,097,152, larger shapes are rejected with
+ * LSE * log2(e), 8 bytes per (batch, head, token) row, the work counters, and the dS tiles
+ * of the dQ pass when one kv head's fit in the rest) lives in an array of 16 MiB + 256 bytes
+ * compiled into the library: B * Hq * N may be at most 2,097,152, larger shapes are rejected with
  * S2ATTN_ERR_UNSUPPORTED (message in s2attn_last_error) before anything is launched. Every
  * device that loads the library holds that array until the process exits. The first call on
  * a device, with that device current, looks up the array's device address; make that first

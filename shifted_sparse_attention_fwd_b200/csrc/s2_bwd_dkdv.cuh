@@ -13,8 +13,9 @@
 // by all its query heads whatever their roll, and dK/dV are written once, without atomics.
 // For each query head the rows map to at most two runs of rolled rows; the query tiles
 // visited are those covering [rolled row, end of its group) for every row of the tile.
-// The kernel is persistent: each CTA takes tiles blockIdx.x, blockIdx.x + gridDim.x, ...
-// (heaviest first), so one tile's epilogue overlaps the next tile's loads and first MMAs.
+// The kernel is persistent: each CTA claims work tiles from a global counter (heaviest first,
+// grouped for L2 reuse), so one tile's epilogue overlaps the next tile's loads and first MMAs
+// and the load stays balanced.
 //
 // Warp roles (352 threads): warps 0-7 elementwise — kv row i (TMEM lane i) is shared by warp
 // i/32 (query columns 0-63) and warp i/32 + 4 (columns 64-127), so two warps per SM
@@ -50,6 +51,7 @@ struct BwdParams {
   int kvh_begin, kvh_count;
   __nv_bfloat16* ds;   // bf16 dS tiles for the dQ pass (DsSlots layout), or null
   DsSlots slots;
+  unsigned int* sched;   // {next, done} work counter of this launch (claim_unit)
 };
 
 constexpr uint32_t kDsTileBytes = kTileRows * kTileRows * 2;   // one bf16 dS tile, 32 KB
@@ -72,9 +74,11 @@ struct DkdvLayout {
   static constexpr uint32_t kStage = kDO + 2 * kTile; // dS tile, or the dV / dK tile, 32 KB
   static constexpr uint32_t kLse = kStage + kDsTileBytes;   // 2 stages x 128 floats
   static constexpr uint32_t kDv = kLse + 1024;               // 2 stages x 128 floats
-  static constexpr uint32_t kBar = kDv + 1024;
+  static constexpr uint32_t kRing = kDv + 1024;             // claimed work units
+  static constexpr uint32_t kBar = kRing + 4 * kUnitRing;
   enum { B_KV = 0, B_KVE = 1, B_QF = 2, B_QE = 4, B_S = 6, B_DP = 7, B_P = 8, B_DS = 9,
-         B_ACC = 10, B_ACCE = 11, B_STF = 12, B_STE = 13, B_DRAIN = 14, B_COUNT = 15 };
+         B_ACC = 10, B_ACCE = 11, B_STF = 12, B_STE = 13, B_DRAIN = 14, B_UF = 15,
+         B_UE = B_UF + kUnitRing, B_COUNT = B_UE + kUnitRing };
   static constexpr uint32_t kTmemSlot = kBar + B_COUNT * 8;
   static constexpr uint32_t kAbort = kTmemSlot + 4;
   static constexpr uint32_t kBytes = kAbort + 4;
@@ -142,6 +146,10 @@ __global__ void __launch_bounds__(352, 1)
     mbar_init(bar(L::B_STF), 256);
     mbar_init(bar(L::B_STE), 1);
     mbar_init(bar(L::B_DRAIN), 1);
+    for (int i = 0; i < kUnitRing; ++i) {
+      mbar_init(bar(L::B_UF + i), 1);
+      mbar_init(bar(L::B_UE + i), 10);   // MMA thread, 8 elementwise warps, store thread
+    }
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_map(&tmQ);
@@ -159,6 +167,11 @@ __global__ void __launch_bounds__(352, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t tm_s = tmem, tm_dp = tmem + 128, tm_dv = tmem + 256, tm_dk = tmem + 256 + D;
   const uint32_t tm_p = tmem + 32, tm_ds = tmem + 160;   // bf16 P^T and dS^T (MMA A operands)
+  volatile int* ring = reinterpret_cast<volatile int*>(smem + L::kRing);
+  // Every role walks the same sequence of work tiles, claimed by the producer.
+  auto next_unit = [&](int k, int& u, bool whole_warp, uint32_t site) {
+    return read_unit(k, u, ring, bar(L::B_UF), bar(L::B_UE), ctx, site, whole_warp);
+  };
 
   if (warp == 8) {
     // ---------------- TMA producer ----------------
@@ -166,7 +179,10 @@ __global__ void __launch_bounds__(352, 1)
       int last_parity[2] = {-1, -1};
       int n = 0, tc = 0, kv_loads = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < n_tiles; u += gridDim.x, ++tc) {
+      for (int k = 0; ok; ++k, ++tc) {
+        int u;
+        if (!publish_unit(k, u, p.sched, n_tiles, ring, bar(L::B_UF), bar(L::B_UE), ctx, 15)) break;
+        if (u < 0) break;
         int b, kvh, t0;
         dkdv_tile(p, u, b, kvh, t0);
         // K and V of the previous tile are free once its last S and dP MMAs are done.
@@ -211,7 +227,10 @@ __global__ void __launch_bounds__(352, 1)
       constexpr uint32_t idesc_acc = idesc_bf16(128, D, false, true);   // P^T dO, dS^T Q
       int n = 0, tc = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < n_tiles; u += gridDim.x, ++tc) {
+      for (int k = 0; ok; ++k, ++tc) {
+        int u;
+        if (!next_unit(k, u, false, 16)) break;
+        if (u < 0) break;
         int b, kvh, t0;
         dkdv_tile(p, u, b, kvh, t0);
         const int total = pairs_of(kvh, t0);
@@ -264,7 +283,10 @@ __global__ void __launch_bounds__(352, 1)
         ++use;
         return true;
       };
-      for (int u = blockIdx.x; ok && u < n_tiles; u += gridDim.x) {
+      for (int k = 0; ok; ++k) {
+        int u;
+        if (!next_unit(k, u, false, 17)) break;
+        if (u < 0) break;
         int b, kvh, t0;
         dkdv_tile(p, u, b, kvh, t0);
         if (p.ds) {
@@ -314,7 +336,10 @@ __global__ void __launch_bounds__(352, 1)
       ++use;
       return true;
     };
-    for (int u = blockIdx.x; ok && u < n_tiles; u += gridDim.x, ++tc) {
+    for (int k = 0; ok; ++k, ++tc) {
+      int u;
+      if (!next_unit(k, u, true, 18)) break;
+      if (u < 0) break;
       int b, kvh, t0;
       dkdv_tile(p, u, b, kvh, t0);
       const int t = t0 + row;

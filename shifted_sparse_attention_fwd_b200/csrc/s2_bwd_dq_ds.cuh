@@ -8,8 +8,8 @@
 // layout of an MN-major A operand (DsSlots in s2_tiles.cuh), so this pass is a plain
 // streaming GEMM: no recomputation of S, P or dP, no softmax.
 //
-// Persistent: one CTA per SM takes rolled query tiles (heaviest first) blockIdx.x,
-// blockIdx.x + gridDim.x, ...; for each it accumulates, over the original kv tiles the query
+// Persistent: one CTA per SM claims rolled query tiles (heaviest first, grouped for L2 reuse)
+// from a global counter; for each it accumulates, over the original kv tiles the query
 // tile reads (qtile_kv_span), dQ += dS(qt, t) K(t) in TMEM, then scales, rounds to bf16 and
 // stores the rows at their original positions. The sum over kv rows is split by ORIGINAL kv
 // tile, which is the tiling the dK/dV kernel works in; kv rows a query row cannot see carry
@@ -30,9 +30,11 @@ struct DqDsLayout {
   static constexpr uint32_t kKBytes = Tile<D>::kBytes;
   static constexpr int kStages = 3;
   static constexpr uint32_t kStageBytes = kDsTileBytes + kKBytes;
-  static constexpr uint32_t kBar = kStages * kStageBytes;
+  static constexpr uint32_t kRing = kStages * kStageBytes;   // claimed work units
+  static constexpr uint32_t kBar = kRing + 4 * kUnitRing;
   enum { B_FULL = 0, B_EMPTY = kStages, B_ACC = 2 * kStages, B_ACCE = 2 * kStages + 2,
-         B_DRAIN = 2 * kStages + 4, B_COUNT = 2 * kStages + 5 };
+         B_DRAIN = 2 * kStages + 4, B_UF = 2 * kStages + 5, B_UE = B_UF + kUnitRing,
+         B_COUNT = B_UE + kUnitRing };
   static constexpr uint32_t kTmemSlot = kBar + B_COUNT * 8;
   static constexpr uint32_t kAbort = kTmemSlot + 4;
   static constexpr uint32_t kBytes = kAbort + 4;
@@ -78,6 +80,10 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(bar(L::B_ACCE + a), 4);
     }
     mbar_init(bar(L::B_DRAIN), 1);
+    for (int i = 0; i < kUnitRing; ++i) {
+      mbar_init(bar(L::B_UF + i), 1);
+      mbar_init(bar(L::B_UE + i), 5);   // MMA thread and the 4 epilogue warps
+    }
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_map(&tmK);
@@ -90,13 +96,17 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  volatile int* ring = reinterpret_cast<volatile int*>(smem + L::kRing);
 
   if (warp == 0) {
     // ---------------- loader ----------------
     if (lane == 0) {
       int it = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < units; u += gridDim.x) {
+      for (int k = 0; ok; ++k) {
+        int u;
+        if (!publish_unit(k, u, p.sched, units, ring, bar(L::B_UF), bar(L::B_UE), ctx, 5)) break;
+        if (u < 0) break;
         int b, hq, qt;
         dq_ds_tile(p, u, b, hq, qt);
         const KvSpan sp = qtile_kv_span(qt, head_shift(hq), p.N, p.G);
@@ -131,7 +141,10 @@ __global__ void __launch_bounds__(192, 1)
       constexpr uint32_t idesc = idesc_bf16(128, D, true, true);
       int it = 0, n = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < units; u += gridDim.x, ++n) {
+      for (int k = 0; ok; ++k, ++n) {
+        int u;
+        if (!read_unit(k, u, ring, bar(L::B_UF), bar(L::B_UE), ctx, 6, false)) break;
+        if (u < 0) break;
         int b, hq, qt;
         dq_ds_tile(p, u, b, hq, qt);
         const int count = qtile_kv_span(qt, head_shift(hq), p.N, p.G).count;
@@ -164,7 +177,10 @@ __global__ void __launch_bounds__(192, 1)
     const int row = quad * 32 + lane;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     int n = 0;
-    for (int u = blockIdx.x; u < units; u += gridDim.x, ++n) {
+    for (int k = 0;; ++k, ++n) {
+      int u;
+      if (!read_unit(k, u, ring, bar(L::B_UF), bar(L::B_UE), ctx, 7, true)) break;
+      if (u < 0) break;
       int b, hq, qt;
       dq_ds_tile(p, u, b, hq, qt);
       const int a = n & 1;

@@ -5,7 +5,8 @@
 // D_i = sum_j P_ij dP_ij = dO_i . O_i (the backward of the causal self-attention that
 // LongLoRA's Algorithm 1 applies per group, §3.4). Memory bound: every byte of O and dO is
 // read once with 16-byte loads; each block covers 128 consecutive tokens of one (b, h) so
-// that the [B, Hq, N] outputs are written as coalesced 512-byte rows.
+// that the [B, Hq, N] outputs are written as coalesced 512-byte rows. Block 0 also clears the
+// work counters the persistent gradient kernels claim their units from.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -18,12 +19,16 @@ __global__ void __launch_bounds__(256) s2_bwd_pre_kernel(const __nv_bfloat16* __
                                                          const __nv_bfloat16* __restrict__ dO,
                                                          const float* __restrict__ lse,
                                                          float* __restrict__ dvec,
-                                                         float* __restrict__ lse2, int Hq,
-                                                         int N) {
+                                                         float* __restrict__ lse2,
+                                                         unsigned int* __restrict__ sched,
+                                                         int sched_words, int Hq, int N) {
   constexpr int kLanesPerRow = D / 8;            // 16-byte chunks per row
   constexpr int kRowsPerPass = 32 / kLanesPerRow;
   constexpr int kPasses = 16 / kRowsPerPass;     // 16 rows per warp, 8 warps per block
   __shared__ float s_d[128];
+  // The work counters of the gradient kernels that follow start from zero.
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < sched_words; i += blockDim.x) sched[i] = 0u;
 
   const int tiles = (N + 127) / 128;
   const int tile = blockIdx.x % tiles;

@@ -64,6 +64,49 @@ __device__ __forceinline__ void gemm_ts_mn(uint32_t d_tmem, uint32_t a_tmem, uin
            (accumulate || kk > 0) ? 1u : 0u);
 }
 
+// Dynamic work distribution for the persistent kernels. One thread of the CTA claims units
+// from a global counter {next, done} (heaviest units have the lowest indices, so claiming in
+// counter order is longest-first and balances the load) and publishes each claimed unit, or
+// -1 when none is left, to the CTA's other roles through a 4-slot ring in shared memory:
+// ring slot k % 4 is filled after the slot's previous unit was acknowledged by every consumer.
+// The last CTA to run out of units resets the counter, so the next launch starts from zero.
+constexpr int kUnitRing = 4;
+__device__ __forceinline__ int claim_unit(unsigned int* sched, int n_units) {
+  const unsigned int u = atomicAdd(sched, 1u);
+  if (u < static_cast<unsigned int>(n_units)) return static_cast<int>(u);
+  __threadfence();
+  if (atomicAdd(sched + 1, 1u) == gridDim.x - 1) {
+    atomicExch(sched, 0u);
+    atomicExch(sched + 1, 0u);
+  }
+  return -1;
+}
+// Producer side: claim the k-th unit of this CTA and publish it (slot k % 4).
+__device__ __forceinline__ bool publish_unit(int k, int& u, unsigned int* sched, int n_units,
+                                             volatile int* ring, uint32_t full0, uint32_t empty0,
+                                             const WaitCtx& ctx, uint32_t site) {
+  const int slot = k % kUnitRing;
+  if (k >= kUnitRing &&
+      !wait_bar(empty0 + 8u * slot, ((k / kUnitRing) - 1) & 1, ctx, site)) return false;
+  u = claim_unit(sched, n_units);
+  ring[slot] = u;
+  mbar_arrive(full0 + 8u * slot);
+  return true;
+}
+// Consumer side (a whole warp, or one thread with lanes == 1): read the k-th unit.
+__device__ __forceinline__ bool read_unit(int k, int& u, volatile const int* ring, uint32_t full0,
+                                          uint32_t empty0, const WaitCtx& ctx, uint32_t site,
+                                          bool whole_warp) {
+  const int slot = k % kUnitRing;
+  bool ok = wait_bar(full0 + 8u * slot, (k / kUnitRing) & 1, ctx, site);
+  if (whole_warp) ok = __all_sync(0xffffffffu, ok);
+  if (!ok) return false;
+  u = ring[slot];
+  if (whole_warp) __syncwarp();
+  if (!whole_warp || (threadIdx.x % 32) == 0) mbar_arrive(empty0 + 8u * slot);
+  return true;
+}
+
 // Wait used only while tearing down: ignores the abort flag, bounded by the timeout.
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity,
                                            unsigned long long timeout_ns) {

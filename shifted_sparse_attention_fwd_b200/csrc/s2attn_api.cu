@@ -21,7 +21,7 @@ namespace {
 
 __device__ unsigned int g_err_word;   // first pipeline-wait failure since the last read
 
-constexpr int kAbiVersion = 1;
+constexpr int kAbiVersion = 2;
 constexpr int kMaxDevices = 64;
 constexpr unsigned long long kDefaultTimeoutNs = 1000000000ull;
 
@@ -134,6 +134,11 @@ s2attn_status encode_pair(MapPair& mp, const void* base, int B, int H, int N, in
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Workspace layout: D [B, Hq, N] fp32 | LSE2 [B, Hq, N] fp32 | scheduling words | dS tiles.
+// Each array is rounded up to 256 bytes; the scheduling words hold the work counters of the
+// persistent gradient kernels ({next, done} for dK/dV, then for dQ).
+constexpr size_t kSchedBytes = 256;
+constexpr int kSchedWords = static_cast<int>(kSchedBytes / 4);
 size_t ws_half(int B, int Hq, int N) {
   const size_t bytes = static_cast<size_t>(B) * Hq * N * sizeof(float);
   return (bytes + 255) & ~static_cast<size_t>(255);
@@ -146,6 +151,12 @@ struct Shape {
 // dS hand-off (backward without recomputation in the dQ pass): the slot layout, and the bytes
 // one kv head (all its query heads, all batches) needs. The dS tiles follow D and LSE2 in the
 // workspace.
+size_t ws_min_bytes(int B, int Hq, int N) { return 2 * ws_half(B, Hq, N) + kSchedBytes; }
+unsigned int* ws_sched(const void* workspace, const Shape& sh) {
+  return reinterpret_cast<unsigned int*>(const_cast<char*>(static_cast<const char*>(workspace)) +
+                                         2 * ws_half(sh.B, sh.Hq, sh.N));
+}
+
 s2::DsSlots ds_layout(const Shape& sh) { return s2::ds_slots(sh.N, sh.G, sh.shb < sh.Hq, sh.shift); }
 size_t ds_bytes_per_kv_head(const Shape& sh) {
   const s2::DsSlots sl = ds_layout(sh);
@@ -154,7 +165,7 @@ size_t ds_bytes_per_kv_head(const Shape& sh) {
 }
 // kv heads per pass that a workspace of `bytes` allows (0: too small, recompute dQ instead).
 int ds_heads_per_pass(const Shape& sh, size_t bytes) {
-  const size_t base = 2 * ws_half(sh.B, sh.Hq, sh.N);
+  const size_t base = ws_min_bytes(sh.B, sh.Hq, sh.N);
   if (bytes <= base) return 0;
   const size_t per = ds_bytes_per_kv_head(sh);
   const size_t k = (bytes - base) / per;
@@ -225,6 +236,7 @@ s2::BwdParams bwd_params(const Shape& sh, float scale, const void* workspace, vo
   p.kvh_count = sh.Hkv;
   p.ds = nullptr;
   p.slots = s2::DsSlots{};
+  p.sched = ws_sched(workspace, sh);
   return p;
 }
 
@@ -235,7 +247,7 @@ void set_ds_pass(s2::BwdParams& p, const Shape& sh, const void* workspace, int k
   p.kvh_count = kvh_count;
   p.slots = ds_layout(sh);
   p.ds = reinterpret_cast<__nv_bfloat16*>(const_cast<char*>(static_cast<const char*>(workspace)) +
-                                          2 * ws_half(sh.B, sh.Hq, sh.N));
+                                          ws_min_bytes(sh.B, sh.Hq, sh.N));
 }
 
 template <int D>
@@ -247,7 +259,7 @@ s2attn_status launch_pre(const Shape& sh, const void* o, const float* lse, const
   const unsigned grid = static_cast<unsigned>(sh.B) * sh.Hq * ((sh.N + 127) / 128);
   s2::s2_bwd_pre_kernel<D><<<grid, 256, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, dvec,
-      lse2, sh.Hq, sh.N);
+      lse2, ws_sched(workspace, sh), kSchedWords, sh.Hq, sh.N);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? S2ATTN_OK : cuda_fail(e, "s2_bwd_pre_kernel launch");
 }
@@ -293,6 +305,7 @@ s2attn_status launch_dq_ds(const Shape& sh, const void* k, void* dq, float scale
   if ((s = encode_pair(mk, k, sh.B, sh.Hkv, sh.N, D)) != S2ATTN_OK) return s;
   s2::BwdParams p = bwd_params(sh, scale, workspace, dq, nullptr, nullptr, err);
   set_ds_pass(p, sh, workspace, kvh_begin, kvh_count);
+  p.sched = ws_sched(workspace, sh) + 2;
   const unsigned units = static_cast<unsigned>(sh.B) * kvh_count * (sh.Hq / sh.Hkv) *
                          ((sh.N + 127) / 128);
   const unsigned grid = units < static_cast<unsigned>(num_sms) ? units : static_cast<unsigned>(num_sms);
@@ -304,7 +317,7 @@ s2attn_status launch_dq_ds(const Shape& sh, const void* k, void* dq, float scale
 
 s2attn_status check_workspace(const Shape& sh, const void* ws, size_t bytes) {
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return S2ATTN_ERR_INVALID_ARG;
-  if (bytes < 2 * ws_half(sh.B, sh.Hq, sh.N)) return S2ATTN_ERR_INVALID_ARG;
+  if (bytes < ws_min_bytes(sh.B, sh.Hq, sh.N)) return S2ATTN_ERR_INVALID_ARG;
   return S2ATTN_OK;
 }
 
@@ -407,14 +420,14 @@ s2attn_status s2attn_fwd(const void* q, const void* k, const void* v, void* o, f
 
 size_t s2attn_bwd_workspace_size(int B, int Hq, int N) {
   if (B <= 0 || Hq <= 0 || N <= 0) return 0;
-  return 2 * ws_half(B, Hq, N);
+  return ws_min_bytes(B, Hq, N);
 }
 
 size_t s2attn_bwd_workspace_size_ex(int B, int Hq, int Hkv, int N, int d, int G,
                                     int shift_head_begin, int shift, size_t cap_bytes) {
   Shape sh;
   if (check_shape(B, Hq, Hkv, N, d, G, 1.0f, shift_head_begin, shift, sh) != S2ATTN_OK) return 0;
-  const size_t base = 2 * ws_half(B, Hq, N);
+  const size_t base = ws_min_bytes(B, Hq, N);
   const size_t per = ds_bytes_per_kv_head(sh);
   size_t k = static_cast<size_t>(Hkv);
   if (cap_bytes != 0) {
@@ -607,7 +620,8 @@ s2attn_status s2attn_selftest_wait_timeout(unsigned long long timeout_ns, void* 
 // ------------------------------------------------------------------------------------------
 namespace {
 
-constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;   // 16 MiB: 2^21 rows of D + LSE2
+constexpr size_t kNoAllocRowBytes = size_t(16) << 20;        // 16 MiB: 2^21 rows of D + LSE2
+constexpr size_t kNoAllocScratchBytes = kNoAllocRowBytes + kSchedBytes;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 struct NoAllocScratch {
@@ -646,11 +660,11 @@ extern "C" s2attn_status s2attn_bwd_noalloc(const void* q, const void* k, const 
                                             void* dq, void* dk, void* dv, int B, int Hq, int Hkv,
                                             int N, int d, int G, float scale, void* stream) {
   if (B > 0 && Hq > 0 && N > 0 &&
-      2 * ws_half(B, Hq, N) > kNoAllocScratchBytes) {
+      2 * ws_half(B, Hq, N) > kNoAllocRowBytes) {
     std::snprintf(g_last_error, sizeof(g_last_error),
                   "s2attn_bwd_noalloc: B*Hq*N = %lld rows need %zu scratch bytes; the static "
                   "scratch holds %zu (at most 2097152 rows)",
-                  static_cast<long long>(B) * Hq * N, 2 * ws_half(B, Hq, N), kNoAllocScratchBytes);
+                  static_cast<long long>(B) * Hq * N, 2 * ws_half(B, Hq, N), kNoAllocRowBytes);
     return S2ATTN_ERR_UNSUPPORTED;
   }
   if (Hq <= 0 || Hq % 2 != 0) return S2ATTN_ERR_INVALID_ARG;

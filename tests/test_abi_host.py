@@ -50,12 +50,13 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.s2attn_abi_version() == 1
+    assert lib.s2attn_abi_version() == 2
     for st in range(5):
         assert s2.status_string(st)
     assert s2.status_string(99) == "unknown status"
-    assert lib.s2attn_bwd_workspace_size(1, 32, 8192) == 2 * 32 * 8192 * 4
-    assert lib.s2attn_bwd_workspace_size(1, 1, 8) == 2 * 256
+    # D and LSE2 (each rounded up to 256 bytes), then 256 bytes of work counters
+    assert lib.s2attn_bwd_workspace_size(1, 32, 8192) == 2 * 32 * 8192 * 4 + 256
+    assert lib.s2attn_bwd_workspace_size(1, 1, 8) == 3 * 256
     assert lib.s2attn_bwd_workspace_size(0, 1, 8) == 0
 
 
