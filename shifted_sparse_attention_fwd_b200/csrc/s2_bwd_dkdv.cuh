@@ -17,17 +17,18 @@
 // grouped for L2 reuse), so one tile's epilogue overlaps the next tile's loads and first MMAs
 // and the load stays balanced.
 //
-// Warp roles (352 threads): warps 0-7 elementwise — kv row i (TMEM lane i) is shared by warp
-// i/32 (query columns 0-63) and warp i/32 + 4 (columns 64-127), so two warps per SM
-// sub-partition work on every tile; warp 8 TMA producer (K, V per tile; Q, dO, LSE2, D per
-// query tile, 2 stages); warp 9 TMEM allocator + MMA issuer; warp 10 store issuer: the
+// Warp roles (608 threads): warps 0-15 elementwise — kv row i (TMEM lane i) is shared by the
+// four warps i/32 + 4 g, g = 0..3, warp group g taking query columns [32 g, 32 g + 32), so
+// four warps per SM sub-partition hide each other's TMEM and special-function latency;
+// warp 16 TMA producer (K, V per tile; Q, dO, LSE2, D per query tile, 2 stages); warp 17
+// TMEM allocator + MMA issuer; warp 18 store issuer: the
 // elementwise warps leave each dS tile (for the dQ pass) and the finished dV and dK tiles in
 // a shared-memory staging buffer, and warp 10 hands them to the TMA unit, so no elementwise
 // warp waits on global stores.
-// TMEM: S^T [0,128) with P^T (bf16) written to [32,96); dP^T [128,256) with dS^T (bf16) to
-// [160,224) — each column half packs its bf16 output inside its own fp32 input columns, so the
-// two warps of a row never overwrite each other's unread data; dV [256,256+D), dK
-// [256+D, 256+2D).
+// TMEM: S^T [0,128) and dP^T [128,256); each column group packs its bf16 P^T (dS^T) into the
+// first 16 of its own 32 fp32 input columns, so the warps of a row never overwrite each
+// other's unread data, and the dV (dK) MMA reads the A operand group by group
+// (gemm_ts_mn_grouped); dV [256,256+D), dK [256+D, 256+2D).
 #pragma once
 
 #include "s2_common.cuh"
@@ -64,6 +65,13 @@ __device__ __forceinline__ __nv_bfloat16* ds_slot_ptr(const BwdParams& p, int b,
   return p.ds + (hl * p.slots.per_head + slot) * (kDsTileBytes / 2);
 }
 
+// Elementwise column groups per kv row (warps per TMEM lane quadrant) and their width.
+constexpr int kDkdvGroups = 4;
+constexpr int kDkdvCols = kTileRows / kDkdvGroups;
+constexpr int kDkdvEwWarps = 4 * kDkdvGroups;
+constexpr int kDkdvEwThreads = 32 * kDkdvEwWarps;
+static_assert(kDkdvCols == 32, "the elementwise code moves 32 columns per TMEM access");
+
 template <int D>
 struct DkdvLayout {
   static constexpr uint32_t kTile = Tile<D>::kBytes;
@@ -84,7 +92,7 @@ struct DkdvLayout {
   static constexpr uint32_t kBytes = kAbort + 4;
   // No alignment slack: the kernel checks that the window starts on a 1024-byte boundary.
   static constexpr uint32_t kLaunchBytes = kBytes > 116 * 1024 ? kBytes : 116 * 1024;
-  static constexpr int kThreads = 352;
+  static constexpr int kThreads = 32 * (kDkdvEwWarps + 3);
 };
 
 // Work tile u (heaviest first) of this pass -> (b, kv head, first original row).
@@ -98,7 +106,7 @@ __device__ __forceinline__ void dkdv_tile(const BwdParams& p, int u, int& b, int
 }
 
 template <int D>
-__global__ void __launch_bounds__(352, 1)
+__global__ void __launch_bounds__(32 * (kDkdvEwWarps + 3), 1)
     s2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQ8,
                        const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmK8,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmV8,
@@ -130,7 +138,8 @@ __global__ void __launch_bounds__(352, 1)
     return total;
   };
 
-  if (warp == 8 && lane == 0) {
+  constexpr int kProducer = kDkdvEwWarps, kMma = kDkdvEwWarps + 1, kStore = kDkdvEwWarps + 2;
+  if (warp == kProducer && lane == 0) {
     mbar_init(bar(L::B_KV), 1);
     mbar_init(bar(L::B_KVE), 1);
     for (int s = 0; s < 2; ++s) {
@@ -139,16 +148,16 @@ __global__ void __launch_bounds__(352, 1)
     }
     mbar_init(bar(L::B_S), 1);
     mbar_init(bar(L::B_DP), 1);
-    mbar_init(bar(L::B_P), 256);
-    mbar_init(bar(L::B_DS), 256);
+    mbar_init(bar(L::B_P), kDkdvEwThreads);
+    mbar_init(bar(L::B_DS), kDkdvEwThreads);
     mbar_init(bar(L::B_ACC), 1);
-    mbar_init(bar(L::B_ACCE), 256);
-    mbar_init(bar(L::B_STF), 256);
+    mbar_init(bar(L::B_ACCE), kDkdvEwThreads);
+    mbar_init(bar(L::B_STF), kDkdvEwThreads);
     mbar_init(bar(L::B_STE), 1);
     mbar_init(bar(L::B_DRAIN), 1);
     for (int i = 0; i < kUnitRing; ++i) {
       mbar_init(bar(L::B_UF + i), 1);
-      mbar_init(bar(L::B_UE + i), 10);   // MMA thread, 8 elementwise warps, store thread
+      mbar_init(bar(L::B_UE + i), kDkdvEwWarps + 2);   // MMA, elementwise warps, store
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -157,7 +166,7 @@ __global__ void __launch_bounds__(352, 1)
     tma_prefetch_map(&tmV);
     tma_prefetch_map(&tmO);
   }
-  if (warp == 9) {
+  if (warp == kMma) {
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
@@ -166,14 +175,14 @@ __global__ void __launch_bounds__(352, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tm_s = tmem, tm_dp = tmem + 128, tm_dv = tmem + 256, tm_dk = tmem + 256 + D;
-  const uint32_t tm_p = tmem + 32, tm_ds = tmem + 160;   // bf16 P^T and dS^T (MMA A operands)
+  const uint32_t tm_p = tmem, tm_ds = tmem + 128;   // bf16 P^T and dS^T, grouped A operands
   volatile int* ring = reinterpret_cast<volatile int*>(smem + L::kRing);
   // Every role walks the same sequence of work tiles, claimed by the producer.
   auto next_unit = [&](int k, int& u, bool whole_warp, uint32_t site) {
     return read_unit(k, u, ring, bar(L::B_UF), bar(L::B_UE), ctx, site, whole_warp);
   };
 
-  if (warp == 8) {
+  if (warp == kProducer) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
       int last_parity[2] = {-1, -1};
@@ -220,7 +229,7 @@ __global__ void __launch_bounds__(352, 1)
       for (int s = 0; s < 2; ++s)
         if (last_parity[s] >= 0) drain_wait(bar(L::B_QF + s), last_parity[s], p.timeout_ns);
     }
-  } else if (warp == 9) {
+  } else if (warp == kMma) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16(128, 128, false, false);  // K Q^T, V dO^T
@@ -250,7 +259,7 @@ __global__ void __launch_bounds__(352, 1)
           // The previous tile's dV and dK must have been read out before they restart.
           if (i == 0 && tc > 0 && !wait_bar(bar(L::B_ACCE), (tc - 1) & 1, ctx, 12)) { ok = false; break; }
           tc_fence_after();
-          gemm_ts_mn<D>(tm_dv, tm_p, do_s, idesc_acc, i > 0);
+          gemm_ts_mn_grouped<D, kDkdvCols>(tm_dv, tm_p, do_s, idesc_acc, i > 0);
           if (i + 1 < total) {
             const int st1 = (n + 1) & 1;
             if (!wait_bar(bar(L::B_QF + st1), ((n + 1) >> 1) & 1, ctx, 5)) { ok = false; break; }
@@ -260,13 +269,13 @@ __global__ void __launch_bounds__(352, 1)
           }
           if (!wait_bar(bar(L::B_DS), n & 1, ctx, 6)) { ok = false; break; }
           tc_fence_after();
-          gemm_ts_mn<D>(tm_dk, tm_ds, q_s, idesc_acc, i > 0);
+          gemm_ts_mn_grouped<D, kDkdvCols>(tm_dk, tm_ds, q_s, idesc_acc, i > 0);
           mma_commit(bar(L::B_QE + st));
         }
         if (ok) mma_commit(bar(L::B_ACC));
       }
     }
-  } else if (warp == 10) {
+  } else if (warp == kStore) {
     // ---------------- store issuer ----------------
     // Mirrors the elementwise warps' use of the staging buffer: per query tile a dS tile
     // (when handing off to the dQ pass), per work tile dV then dK.
@@ -317,8 +326,10 @@ __global__ void __launch_bounds__(352, 1)
       bulk_wait_all();
     }
   } else {
-    // ---------------- elementwise warps 0-7 ----------------
-    const int half = warp / 4;                     // query columns [64 half, 64 half + 64)
+    // ---------------- elementwise warps ----------------
+    constexpr int W = kDkdvCols;                   // query columns per thread
+    constexpr int CPT = D / kDkdvGroups;           // dV / dK columns per thread in the epilogue
+    const int grp = warp / 4;                      // query columns [W grp, W grp + W)
     const int row = (warp % 4) * 32 + lane;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>((warp % 4) * 32) << 16);
     const float c = p.scale_log2;
@@ -351,22 +362,22 @@ __global__ void __launch_bounds__(352, 1)
         const int ge_k = group_end(r_k, p.G);
         for (int i = 0; i < qr.count(); ++i, ++n) {
           const int st = n & 1;
-          const int q0 = qr.at(i) * kTileRows + 64 * half;
+          const int q0 = qr.at(i) * kTileRows + W * grp;
           const int cl = kv_valid ? r_k - q0 : 1;
           const int ch = kv_valid ? ge_k - 1 - q0 : 0;
-          const bool mask = __any_sync(0xffffffffu, cl > 0 || ch < 63);
+          const bool mask = __any_sync(0xffffffffu, cl > 0 || ch < W - 1);
           if (!warp_wait(bar(L::B_QF + st), (n >> 1) & 1, ctx, 7)) { ok = false; break; }
           if (!warp_wait(bar(L::B_S), n & 1, ctx, 8)) { ok = false; break; }
           tc_fence_after();
-          const float* lse_t = s_lse + st * 128 + 64 * half;
-          const float* d_t = s_dv + st * 128 + 64 * half;
-          // P^T phase: 64 columns of S^T -> P^T (bf16), kept in registers for the dS phase.
-          uint32_t pk[32];
+          const float* lse_t = s_lse + st * 128 + W * grp;
+          const float* d_t = s_dv + st * 128 + W * grp;
+          // P^T phase: W columns of S^T -> P^T (bf16), kept in registers for the dS phase.
+          uint32_t pk[W / 2];
           {
-            uint32_t raw[64];
-            tmem_ld64(t_lane + 64 * half, raw);
+            uint32_t raw[W];
+            tmem_ld32(t_lane + W * grp, raw);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
+            for (int e = 0; e < W / 2; ++e) {
               const int col = 2 * e;
               float x0 = fast_exp2(fmaf(__uint_as_float(raw[col]), c, -lse_t[col]));
               float x1 = fast_exp2(fmaf(__uint_as_float(raw[col + 1]), c, -lse_t[col + 1]));
@@ -377,19 +388,19 @@ __global__ void __launch_bounds__(352, 1)
               pk[e] = pack_bf16(x0, x1);
             }
           }
-          tmem_st32(t_lane + 32 + 32 * half, pk);
+          tmem_st16(t_lane + W * grp, pk);
           tmem_st_wait();
           tc_fence_before();
           mbar_arrive(bar(L::B_P));
           // dS^T phase: dS^T = P^T o (dP^T - D).
           if (!warp_wait(bar(L::B_DP), n & 1, ctx, 9)) { ok = false; break; }
           tc_fence_after();
-          uint32_t ds[32];
+          uint32_t ds[W / 2];
           {
-            uint32_t raw[64];
-            tmem_ld64(t_lane + 128 + 64 * half, raw);
+            uint32_t raw[W];
+            tmem_ld32(t_lane + 128 + W * grp, raw);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
+            for (int e = 0; e < W / 2; ++e) {
               const int col = 2 * e;
               const float2 pf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[e]));
               float y0 = pf.x * (__uint_as_float(raw[col]) - d_t[col]);
@@ -400,7 +411,7 @@ __global__ void __launch_bounds__(352, 1)
               }
               ds[e] = pack_bf16(y0, y1);
             }
-            tmem_st32(t_lane + 160 + 32 * half, ds);
+            tmem_st16(t_lane + 128 + W * grp, ds);
           }
           tmem_st_wait();
           tc_fence_before();
@@ -410,8 +421,8 @@ __global__ void __launch_bounds__(352, 1)
             // block c holding query columns [8c, 8c + 8) of all 128 kv rows, 16 bytes per row.
             ok = stage_out([&] {
 #pragma unroll
-              for (int c8 = 0; c8 < 8; ++c8)
-                *reinterpret_cast<uint4*>(stage + (half * 8 + c8) * 2048 + row * 16) =
+              for (int c8 = 0; c8 < W / 8; ++c8)
+                *reinterpret_cast<uint4*>(stage + ((W / 8) * grp + c8) * 2048 + row * 16) =
                     make_uint4(ds[4 * c8], ds[4 * c8 + 1], ds[4 * c8 + 2], ds[4 * c8 + 3]);
             });
             if (!ok) break;
@@ -420,20 +431,20 @@ __global__ void __launch_bounds__(352, 1)
       }
       if (!ok || !warp_wait(bar(L::B_ACC), tc & 1, ctx, 10)) { ok = false; break; }
       tc_fence_after();
-      // dV, then scale * dK: this thread's D/2 columns of its row, in bf16, into the staging
+      // dV, then scale * dK: this thread's CPT columns of its row, in bf16, into the staging
       // buffer in the 128-byte-swizzled layout of the TMA tile (64-column boxes of 128 rows).
 #pragma unroll 1
       for (int which = 0; ok && which < 2; ++which) {
         const uint32_t src = (which == 0 ? tm_dv : tm_dk) - tmem + t_lane;
         const float mul = which == 0 ? 1.f : p.scale;
-        uint32_t pkd[D / 4];
+        uint32_t pkd[CPT / 2];
 #pragma unroll
-        for (int j = 0; j < D / 64; ++j) {
-          uint32_t rr[32];
-          tmem_ld32(src + (D / 2) * half + 32 * j, rr);
+        for (int j = 0; j < CPT / 16; ++j) {
+          uint32_t rr[16];
+          tmem_ld16(src + CPT * grp + 16 * j, rr);
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            pkd[16 * j + e] = pack_bf16(__uint_as_float(rr[2 * e]) * mul, __uint_as_float(rr[2 * e + 1]) * mul);
+          for (int e = 0; e < 8; ++e)
+            pkd[8 * j + e] = pack_bf16(__uint_as_float(rr[2 * e]) * mul, __uint_as_float(rr[2 * e + 1]) * mul);
         }
         if (which == 1) {   // both accumulators are in registers: the MMA may reuse them
           tc_fence_before();
@@ -441,8 +452,8 @@ __global__ void __launch_bounds__(352, 1)
         }
         ok = stage_out([&] {
 #pragma unroll
-          for (int v = 0; v < D / 16; ++v) {
-            const int col = (D / 2) * half + 8 * v;   // first of the 8 columns of chunk v
+          for (int v = 0; v < CPT / 8; ++v) {
+            const int col = CPT * grp + 8 * v;   // first of the 8 columns of chunk v
             const int box = col / 64, chunk = (col % 64) / 8;
             *reinterpret_cast<uint4*>(stage + box * Tile<D>::kHalfBytes + row * 128 +
                                       ((chunk ^ (row & 7)) * 16)) =
@@ -455,7 +466,7 @@ __global__ void __launch_bounds__(352, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kMma) {
     if (lane == 0) {
       mma_commit(bar(L::B_DRAIN));
       drain_wait(bar(L::B_DRAIN), 0, p.timeout_ns);

@@ -107,6 +107,19 @@ __device__ __forceinline__ bool read_unit(int k, int& u, volatile const int* rin
   return true;
 }
 
+// As gemm_ts_mn, with the bf16 A operand written by kGroups column groups of W = 128 / kGroups
+// columns, each packed into the first W/2 TMEM columns of its own range: the 16 K-values of
+// step kk sit at a_tmem + W * (16 kk / W) + (16 kk % W) / 2.
+template <int D, int W>
+__device__ __forceinline__ void gemm_ts_mn_grouped(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_base,
+                                                   uint32_t idesc, bool accumulate) {
+  const uint64_t b0 = sdesc_sw128(b_base, Tile<D>::kHalfBytes, 1024);
+#pragma unroll
+  for (int kk = 0; kk < kTileRows / 16; ++kk)
+    mma_ts(d_tmem, a_tmem + W * ((16 * kk) / W) + ((16 * kk) % W) / 2,
+           b0 + static_cast<uint64_t>((kk * 2048) >> 4), idesc, (accumulate || kk > 0) ? 1u : 0u);
+}
+
 // Wait used only while tearing down: ignores the abort flag, bounded by the timeout.
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity,
                                            unsigned long long timeout_ns) {
