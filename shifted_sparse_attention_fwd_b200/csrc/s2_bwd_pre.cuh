@@ -4,15 +4,19 @@
 // D is the row term of the softmax derivative, dS = P o (dP - D) with
 // D_i = sum_j P_ij dP_ij = dO_i . O_i (the backward of the causal self-attention that
 // LongLoRA's Algorithm 1 applies per group, §3.4). Memory bound: every byte of O and dO is
-// read once with 16-byte loads; each block covers 128 consecutive tokens of one (b, h) so
-// that the [B, Hq, N] outputs are written as coalesced 512-byte rows. Block 0 also clears the
-// work counters the persistent gradient kernels claim their units from.
+// read once with 16-byte loads, each block streaming one contiguous range of memory (a few
+// tokens, all heads); the small [B, Hq, N] outputs are written as 32-byte pieces. Block 0
+// also clears the work counters the persistent gradient kernels claim their units from.
 #pragma once
 
 #include <cuda_bf16.h>
 #include <cstdint>
 
 namespace s2 {
+
+// A block covers kPreTokens consecutive tokens of one batch and every head: the rows of O and
+// dO it reads (token-major, head-minor) are one contiguous range of memory.
+constexpr int kPreTokens = 8;
 
 template <int D>
 __global__ void __launch_bounds__(256) s2_bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
@@ -22,59 +26,56 @@ __global__ void __launch_bounds__(256) s2_bwd_pre_kernel(const __nv_bfloat16* __
                                                          float* __restrict__ lse2,
                                                          unsigned int* __restrict__ sched,
                                                          int sched_words, int Hq, int N) {
-  constexpr int kLanesPerRow = D / 8;            // 16-byte chunks per row
-  constexpr int kRowsPerPass = 32 / kLanesPerRow;
-  constexpr int kPasses = 16 / kRowsPerPass;     // 16 rows per warp, 8 warps per block
-  __shared__ float s_d[128];
+  constexpr int kLanesPerRow = D / 8;            // 16-byte chunks per (token, head) row
+  constexpr int kRowsPerWarp = 32 / kLanesPerRow;
   // The work counters of the gradient kernels that follow start from zero.
   if (blockIdx.x == 0)
     for (int i = threadIdx.x; i < sched_words; i += blockDim.x) sched[i] = 0u;
 
-  const int tiles = (N + 127) / 128;
-  const int tile = blockIdx.x % tiles;
-  const int bh = blockIdx.x / tiles;
-  const int h = bh % Hq, b = bh / Hq;
-  const int t0 = tile * 128;
+  const int tblocks = (N + kPreTokens - 1) / kPreTokens;
+  const int b = blockIdx.x / tblocks;
+  const int t0 = (blockIdx.x % tblocks) * kPreTokens;
+  const int nt = N - t0 < kPreTokens ? N - t0 : kPreTokens;
+  const int rows = nt * Hq;                      // rows r = (t - t0) * Hq + h
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int sub = lane / kLanesPerRow, li = lane % kLanesPerRow;
-
-  uint4 ov[kPasses], gv[kPasses];
+  const size_t base = (static_cast<size_t>(b) * N + t0) * Hq;   // first row of the block
+  constexpr int kUnroll = 4;                     // row pairs in flight per thread
+  for (int r0 = warp * kRowsPerWarp; r0 < rows; r0 += kUnroll * 8 * kRowsPerWarp) {
+    uint4 ov[kUnroll], gv[kUnroll];
 #pragma unroll
-  for (int i = 0; i < kPasses; ++i) {
-    const int t = t0 + warp * 16 + i * kRowsPerPass + sub;
-    if (t < N) {
-      const size_t off = ((static_cast<size_t>(b) * N + t) * Hq + h) * D + li * 8;
-      ov[i] = __ldg(reinterpret_cast<const uint4*>(o + off));
-      gv[i] = __ldg(reinterpret_cast<const uint4*>(dO + off));
-    } else {
-      ov[i] = make_uint4(0, 0, 0, 0);
-      gv[i] = make_uint4(0, 0, 0, 0);
-    }
-  }
-#pragma unroll
-  for (int i = 0; i < kPasses; ++i) {
-    const __nv_bfloat162* a = reinterpret_cast<const __nv_bfloat162*>(&ov[i]);
-    const __nv_bfloat162* g = reinterpret_cast<const __nv_bfloat162*>(&gv[i]);
-    float acc = 0.f;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 fa = __bfloat1622float2(a[e]);
-      const float2 fg = __bfloat1622float2(g[e]);
-      acc = fmaf(fa.x, fg.x, acc);
-      acc = fmaf(fa.y, fg.y, acc);
+    for (int k = 0; k < kUnroll; ++k) {
+      const int rr = r0 + k * 8 * kRowsPerWarp + sub;
+      if (rr < rows) {
+        const size_t off = (base + rr) * D + li * 8;
+        ov[k] = __ldg(reinterpret_cast<const uint4*>(o + off));
+        gv[k] = __ldg(reinterpret_cast<const uint4*>(dO + off));
+      } else {
+        ov[k] = make_uint4(0, 0, 0, 0);
+        gv[k] = make_uint4(0, 0, 0, 0);
+      }
     }
 #pragma unroll
-    for (int off = kLanesPerRow / 2; off > 0; off >>= 1)
-      acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (li == 0) s_d[warp * 16 + i * kRowsPerPass + sub] = acc;
-  }
-  __syncthreads();
-  if (threadIdx.x < 128) {
-    const int t = t0 + threadIdx.x;
-    if (t < N) {
-      const size_t idx = (static_cast<size_t>(b) * Hq + h) * N + t;
-      dvec[idx] = s_d[threadIdx.x];
-      lse2[idx] = lse[idx] * 1.4426950408889634f;
+    for (int k = 0; k < kUnroll; ++k) {
+      const int rr = r0 + k * 8 * kRowsPerWarp + sub;
+      const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&ov[k]);
+      const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv[k]);
+      float acc = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 fa = __bfloat1622float2(a2[e]);
+        const float2 fg = __bfloat1622float2(g2[e]);
+        acc = fmaf(fa.x, fg.x, acc);
+        acc = fmaf(fa.y, fg.y, acc);
+      }
+#pragma unroll
+      for (int sh = kLanesPerRow / 2; sh > 0; sh >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, sh);
+      if (li == 0 && rr < rows) {
+        const int h = rr % Hq, t = t0 + rr / Hq;
+        const size_t idx = (static_cast<size_t>(b) * Hq + h) * N + t;
+        dvec[idx] = acc;
+        lse2[idx] = lse[idx] * 1.4426950408889634f;
+      }
     }
   }
 }

@@ -256,7 +256,7 @@ s2attn_status launch_pre(const Shape& sh, const void* o, const float* lse, const
   const size_t half = ws_half(sh.B, sh.Hq, sh.N);
   float* dvec = static_cast<float*>(workspace);
   float* lse2 = reinterpret_cast<float*>(static_cast<char*>(workspace) + half);
-  const unsigned grid = static_cast<unsigned>(sh.B) * sh.Hq * ((sh.N + 127) / 128);
+  const unsigned grid = static_cast<unsigned>(sh.B) * ((sh.N + s2::kPreTokens - 1) / s2::kPreTokens);
   s2::s2_bwd_pre_kernel<D><<<grid, 256, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, dvec,
       lse2, ws_sched(workspace, sh), kSchedWords, sh.Hq, sh.N);
