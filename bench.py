@@ -297,6 +297,12 @@ def run_gpu(args, rank, world, local_rank):
                    "l2": f"flushed before every step ({L2_FLUSH_BYTES >> 20} MiB write, untimed)",
                    "parallelism": f"{world} independent replicas (weak scaling)"},
         "pct_of_peak": round(100 * value / peak_tf, 2),
+        "fwd": {"ms": round(avg["s2_fwd"], 4),
+                "tflops": round(kflops["s2_fwd"] / (avg["s2_fwd"] * 1e-3) / 1e12, 1)},
+        "bwd": {"ms": round(avg["s2_bwd_pre"] + avg["s2_bwd_dkdv"] + avg["s2_bwd_dq_ds"], 4),
+                "tflops": round(5.0 * float(w.B) * w.Hq * w.N * w.G * w.d /
+                                ((avg["s2_bwd_pre"] + avg["s2_bwd_dkdv"] + avg["s2_bwd_dq_ds"]) * 1e-3)
+                                / 1e12, 1)},
         "peak": {"bf16_tflops": peak_tf, "source": peak_src},
         "kernels": kern,
         "roofline": roof,
