@@ -188,9 +188,13 @@ __global__ void __launch_bounds__(32 * (kDkdvEwWarps + 3), 1)
       int last_parity[2] = {-1, -1};
       int n = 0, tc = 0, kv_loads = 0;
       bool ok = true;
+      // Units are claimed one ahead: unit k + 1 is published as soon as unit k's K and V
+      // loads are issued, so the other roles never wait for the producer to finish issuing
+      // unit k's query tiles before they can start on the next unit.
+      int u_next;
+      ok = publish_unit(0, u_next, p.sched, n_tiles, ring, bar(L::B_UF), bar(L::B_UE), ctx, 15);
       for (int k = 0; ok; ++k, ++tc) {
-        int u;
-        if (!publish_unit(k, u, p.sched, n_tiles, ring, bar(L::B_UF), bar(L::B_UE), ctx, 15)) break;
+        const int u = u_next;
         if (u < 0) break;
         int b, kvh, t0;
         dkdv_tile(p, u, b, kvh, t0);
@@ -201,6 +205,10 @@ __global__ void __launch_bounds__(32 * (kDkdvEwWarps + 3), 1)
         load_tile<D>(sbase + L::kK, &tmK, &tmK8, bar(L::B_KV), b, kvh, kv_runs, p.N);
         load_tile<D>(sbase + L::kV, &tmV, &tmV8, bar(L::B_KV), b, kvh, kv_runs, p.N);
         ++kv_loads;
+        if (!publish_unit(k + 1, u_next, p.sched, n_tiles, ring, bar(L::B_UF), bar(L::B_UE), ctx, 15)) {
+          ok = false;
+          break;
+        }
         for (int hq = kvh * rep; ok && hq < (kvh + 1) * rep; ++hq) {
           const int sh = head_shift(hq);
           const QTileRanges qr = kv_tile_qtiles(t0, sh, p.N, p.G);

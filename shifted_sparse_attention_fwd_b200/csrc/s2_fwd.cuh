@@ -72,19 +72,18 @@ struct FwdLayout {
   static constexpr int kThreads = 320;
 };
 
+// Row maximum of 128 values: eight independent chains of three-input max instructions.
 __device__ __forceinline__ float max_tree128(const float (&s)[128]) {
   float m[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) m[i] = s[i];
+  for (int i = 0; i < 8; ++i) m[i] = max3f(s[i], s[8 + i], s[16 + i]);
 #pragma unroll
-  for (int j = 1; j < 16; ++j)
+  for (int j = 3; j + 1 < 16; j += 2)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) m[i] = fmaxf(m[i], s[8 * j + i]);
+    for (int i = 0; i < 8; ++i) m[i] = max3f(m[i], s[8 * j + i], s[8 * (j + 1) + i]);
 #pragma unroll
-  for (int w = 4; w > 0; w >>= 1)
-#pragma unroll
-    for (int i = 0; i < w; ++i) m[i] = fmaxf(m[i], m[i + w]);
-  return m[0];
+  for (int i = 0; i < 8; ++i) m[i] = fmaxf(m[i], s[120 + i]);
+  return max3f(max3f(m[0], m[1], m[2]), max3f(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
 }
 
 // One work unit: query tiles 2*pair and 2*pair + 1 of (b, h) and the key tiles they see.
@@ -341,28 +340,24 @@ __global__ void __launch_bounds__(320, 1)
           l_run *= alpha;
           m_run = m_cand;
         }
+        // P = exp2(c s - m), two columns per packed f32x2 multiply-add and sum.
         const float m_use = m_run == -INFINITY ? 0.f : m_run;
-        float part_sum[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) part_sum[i] = 0.f;
+        const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(-m_use, -m_use);
+        uint64_t acc[4] = {0, 0, 0, 0};
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float e0 = fast_exp2(fmaf(s[32 * j + 2 * i], c, -m_use));
-            const float e1 = fast_exp2(fmaf(s[32 * j + 2 * i + 1], c, -m_use));
-            part_sum[(2 * i) & 7] += e0;
-            part_sum[(2 * i + 1) & 7] += e1;
+            const uint64_t a = f2_fma(f2_pack(s[32 * j + 2 * i], s[32 * j + 2 * i + 1]), c2, nm2);
+            const float e0 = fast_exp2(f2_lo(a)), e1 = fast_exp2(f2_hi(a));
+            acc[i & 3] = f2_add(acc[i & 3], f2_pack(e0, e1));
             pk[i] = pack_bf16(e0, e1);
           }
           tmem_st16(s_col + 16 * j, pk);
         }
-#pragma unroll
-        for (int w = 4; w > 0; w >>= 1)
-#pragma unroll
-          for (int i = 0; i < w; ++i) part_sum[i] += part_sum[i + w];
-        l_run += part_sum[0];
+        acc[0] = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
+        l_run += f2_lo(acc[0]) + f2_hi(acc[0]);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(bar(L::B_P + wg));
