@@ -300,26 +300,4 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   return d;
 }
 
-// 2^x for two arguments on the FMA and integer pipes only, to take load off the special
-// function unit that ex2.approx uses. Cody-Waite style reduction: x is clamped to >= -125,
-// n = round(x) is read from the low mantissa bits of x + 1.5 * 2^23, f = x - n lies in
-// [-0.5, 0.5], 2^f is a cubic in f, and n is added to the exponent field. The cubic is a
-// relative-error-weighted least-squares fit on Chebyshev nodes of [-0.5, 0.5] (fit_exp2_poly.py);
-// its maximum relative error is 7.8e-5, far below the bf16 rounding P receives afterwards.
-constexpr float kExp2C0 = 0.99992895f, kExp2C1 = 0.6932763f, kExp2C2 = 0.24260436f,
-                kExp2C3 = 0.05508872f;
-__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
-  constexpr float kRound = 12582912.0f;   // 1.5 * 2^23
-  const uint64_t x = f2_pack(fmaxf(f2_lo(x2), -125.f), fmaxf(f2_hi(x2), -125.f));
-  const uint64_t t = f2_add(x, f2_pack(kRound, kRound));
-  const uint64_t n = f2_add(t, f2_pack(-kRound, -kRound));
-  const uint64_t f = f2_fma(n, f2_pack(-1.f, -1.f), x);
-  uint64_t p = f2_fma(f, f2_pack(kExp2C3, kExp2C3), f2_pack(kExp2C2, kExp2C2));
-  p = f2_fma(p, f, f2_pack(kExp2C1, kExp2C1));
-  p = f2_fma(p, f, f2_pack(kExp2C0, kExp2C0));
-  const uint32_t lo = static_cast<uint32_t>(p) + (static_cast<uint32_t>(t) << 23);
-  const uint32_t hi = static_cast<uint32_t>(p >> 32) + (static_cast<uint32_t>(t >> 32) << 23);
-  return (static_cast<uint64_t>(hi) << 32) | lo;
-}
-
 }  // namespace s2
