@@ -315,13 +315,22 @@ def run_gpu(args, rank, world, local_rank):
     return line
 
 
-def kernel_source_hash() -> str:
-    """Hash of the kernel sources; DRAM counters recorded under another hash are stale."""
-    import glob
+KERNEL_SOURCES = {
+    "s2_fwd": ["s2_fwd.cuh"],
+    "s2_bwd_pre": ["s2_bwd_pre.cuh"],
+    "s2_bwd_dkdv": ["s2_bwd_dkdv.cuh"],
+    "s2_bwd_dq_ds": ["s2_bwd_dq_ds.cuh", "s2_bwd_dkdv.cuh"],
+}
+COMMON_SOURCES = ["s2_common.cuh", "s2_device.cuh", "s2_tiles.cuh", "s2_tmem_wide.cuh"]
+
+
+def kernel_source_hash(kernel: str) -> str:
+    """Hash of the sources a kernel is built from; DRAM counters recorded under another hash
+    are stale."""
     import hashlib
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "shifted_sparse_attention_fwd_b200", "csrc", "*"))):
-        with open(f, "rb") as fh:
+    for name in KERNEL_SOURCES.get(kernel, []) + COMMON_SOURCES:
+        with open(os.path.join(ROOT, "shifted_sparse_attention_fwd_b200", "csrc", name), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
@@ -336,7 +345,7 @@ def load_traffic(kernel, workload):
     except (OSError, ValueError):
         return None
     e = t.get(workload, {}).get(kernel)
-    if e is None or e.get("source_hash") != kernel_source_hash():
+    if e is None or e.get("source_hash") != kernel_source_hash(kernel):
         return None
     return e.get("bytes_per_launch")
 
