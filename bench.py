@@ -39,6 +39,21 @@ def fwd_bwd_flops(w) -> float:
     return 7.0 * w.B * w.Hq * w.N * w.G * w.d
 
 
+def max_over_ranks(values, dist=None, device=None):
+    """Elementwise maximum over all ranks (identity on one process): multi-GPU times are the
+    slowest rank's."""
+    if dist is None:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def weak_scaling_value(world, flops_per_step, steps, total_ms):
+    """Whole-job throughput in TFLOP/s: every rank ran `steps` steps of its own batch."""
+    return world * flops_per_step * steps / (total_ms * 1e-3) / 1e12
+
+
 def kernel_flops(w):
     unit = float(w.B) * w.Hq * w.N * w.G * w.d   # one causal in-group GEMM over all heads
     return {"s2_fwd": 2 * unit, "s2_bwd_dkdv": 4 * unit, "s2_bwd_dq_ds": 1 * unit}
@@ -248,15 +263,12 @@ def run_gpu(args, rank, world, local_rank):
     h2d = sum(x.numel() * x.element_size() for x in (hq_, hk_, hv_, hdo_))
     d2h = sum(x.numel() * x.element_size() for x in (ho, hlse, hdq, hdk, hdv))
 
-    if dist:
-        t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, e2e_ms = float(t[0]), float(t[1])
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dist, dev)
     if rank != 0:
         return None
 
     flops_step = fwd_bwd_flops(w)
-    value = world * flops_step * args.steps / (total_ms * 1e-3) / 1e12
+    value = weak_scaling_value(world, flops_step, args.steps, total_ms)
     peaks, peak_src = load_peaks()
     peak_tf = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     avg = {n: sum(v_) / len(v_) for n, v_ in per_k.items()}
@@ -306,7 +318,7 @@ def run_gpu(args, rank, world, local_rank):
         "peak": {"bf16_tflops": peak_tf, "source": peak_src},
         "kernels": kern,
         "roofline": roof,
-        "e2e": {"value": round(world * flops_step * e2e_steps / (e2e_ms * 1e-3) / 1e12, 2),
+        "e2e": {"value": round(weak_scaling_value(world, flops_step, e2e_steps, e2e_ms), 2),
                 "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps, "ms_per_step": round(e2e_ms / e2e_steps, 4)},
         "clocks": sampler.summary(),
