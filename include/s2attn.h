@@ -95,6 +95,22 @@ S2ATTN_API s2attn_status s2attn_fwd_ex(const void* q, const void* k, const void*
                             int B, int Hq, int Hkv, int N, int d, int G, float scale,
                             int shift_head_begin, int shift, void* stream);
 
+/*
+ * Strided forms. Each [B, N, H, d] tensor X is read or written at X + b*sb + t*st + h*d + c
+ * (elements): the (H, d) block of a token is contiguous, tokens and batches may be spaced
+ * freely. This takes q, k and v as views of one packed qkv [B, N, 3, H, d] buffer, the layout
+ * LongLoRA's Algorithm 1 (summary page, §3.4) feeds its attention: q = qkv, k = qkv + H*d,
+ * v = qkv + 2*H*d, st = 3*H*d, sb = N*st (and likewise dq, dk, dv into a packed dqkv).
+ * `strides` holds {sb, st} pairs: q, k, v, o for the forward; q, k, v, o, dO, dq, dk, dv for
+ * the backward; NULL means contiguous (the _ex forms). Every stride must be a multiple of 8
+ * elements, st >= H*d and, when B > 1, sb >= N*st; otherwise S2ATTN_ERR_INVALID_ARG. lse stays
+ * a contiguous [B, Hq, N] array. Outputs must not overlap each other or the inputs.
+ */
+S2ATTN_API s2attn_status s2attn_fwd_strided(const void* q, const void* k, const void* v, void* o,
+                                            float* lse, int B, int Hq, int Hkv, int N, int d,
+                                            int G, float scale, int shift_head_begin, int shift,
+                                            const long long* strides, void* stream);
+
 /* Smallest device workspace s2attn_bwd accepts: two fp32 [B, Hq, N] arrays (D and LSE in
  * base 2), each rounded up to 256 bytes, and 256 bytes of work counters for the gradient
  * kernels (cleared by the preprocess). With only this much the dQ kernel recomputes S and
@@ -137,6 +153,15 @@ S2ATTN_API s2attn_status s2attn_bwd_ex(const void* q, const void* k, const void*
                             int B, int Hq, int Hkv, int N, int d, int G, float scale,
                             int shift_head_begin, int shift, void* workspace,
                             size_t workspace_bytes, void* stream);
+
+/* Backward with strided tensors (see s2attn_fwd_strided; 8 {sb, st} pairs). */
+S2ATTN_API s2attn_status s2attn_bwd_strided(const void* q, const void* k, const void* v,
+                                            const void* o, const float* lse, const void* dO,
+                                            void* dq, void* dk, void* dv, int B, int Hq, int Hkv,
+                                            int N, int d, int G, float scale,
+                                            int shift_head_begin, int shift,
+                                            const long long* strides, void* workspace,
+                                            size_t workspace_bytes, void* stream);
 
 /*
  * The three stages of s2attn_bwd, callable one at a time (same arguments; the workspace

@@ -41,6 +41,8 @@ SIGNATURES = {
     "s2attn_bwd_dq": (_I, [_P] * 5 + [_I] * 6 + [_F, _I, _I, _P, _Z, _P]),
     "s2attn_bwd_noalloc": (_I, [_P] * 9 + [_I] * 6 + [_F, _P]),
     "s2attn_bwd_workspace_size_ex": (_Z, [_I] * 8 + [_Z]),
+    "s2attn_fwd_strided": (_I, [_P] * 5 + [_I] * 6 + [_F, _I, _I, _P, _P]),
+    "s2attn_bwd_strided": (_I, [_P] * 9 + [_I] * 6 + [_F, _I, _I, _P, _P, _Z, _P]),
     "s2attn_bwd_dkdv_ds": (_I, [_P] * 6 + [_I] * 6 + [_F, _I, _I, _P, _Z, _P]),
     "s2attn_bwd_dq_ds": (_I, [_P] * 2 + [_I] * 6 + [_F, _I, _I, _P, _Z, _P]),
     "s2attn_get_device_error": (_I, [_P, ctypes.POINTER(ctypes.c_uint)]),
@@ -86,16 +88,34 @@ def _check(status: int, where: str):
         raise S2AttnError(status, where)
 
 
-def _ptr(t):
+def _ptr(t, strided=False):
     if t is None:
         return None
     if not isinstance(t, torch.Tensor):
         return t  # raw integer address
     if not t.is_cuda:
         raise ValueError("expected a CUDA tensor")
-    if not t.is_contiguous():
+    if not strided and not t.is_contiguous():
         raise ValueError("expected a contiguous tensor")
     return t.data_ptr()
+
+
+def _bn_strides(t):
+    """(batch, token) element strides of a [B, N, H, d] tensor whose (H, d) block is contiguous."""
+    if t.dim() != 4 or t.stride(3) != 1 or t.stride(2) != t.shape[3]:
+        raise ValueError("expected a [B, N, H, d] tensor with contiguous (H, d) blocks")
+    return [t.stride(0), t.stride(1)]
+
+
+def _strides_array(*ts):
+    vals = []
+    for t in ts:
+        vals += _bn_strides(t)
+    return (ctypes.c_longlong * len(vals))(*vals)
+
+
+def _all_contiguous(*ts):
+    return all(t.is_contiguous() for t in ts if isinstance(t, torch.Tensor))
 
 
 def _stream(stream):
@@ -123,6 +143,15 @@ def s2attn_fwd(q, k, v, o, lse, G, scale=None, shift_head_begin=None, shift=None
     _check_bf16(q, k, v, o)
     B, Hq, Hkv, N, d, G = _dims(q, k, G)
     scale = d ** -0.5 if scale is None else scale
+    if not _all_contiguous(q, k, v, o):
+        # views (e.g. of a packed qkv buffer): the strided entry point
+        shb = Hq // 2 if shift_head_begin is None else shift_head_begin
+        sh = G // 2 if shift is None else shift
+        _check(lib().s2attn_fwd_strided(_ptr(q, True), _ptr(k, True), _ptr(v, True), _ptr(o, True),
+                                        _ptr(lse), B, Hq, Hkv, N, d, G, scale, shb, sh,
+                                        _strides_array(q, k, v, o), _stream(stream)),
+               "s2attn_fwd_strided")
+        return
     if shift_head_begin is None and shift is None:
         _check(lib().s2attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, N, d,
                                 G, scale, _stream(stream)), "s2attn_fwd")
@@ -163,6 +192,15 @@ def s2attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, G, scale=None, shift_head_begin=
         ws_bytes = s2attn_bwd_workspace_size_ex(B, Hq, Hkv, N, d, G, shift_head_begin, shift,
                                                 DEFAULT_WORKSPACE_CAP)
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    if not _all_contiguous(q, k, v, o, dO, dq, dk, dv):
+        shb = Hq // 2 if shift_head_begin is None else shift_head_begin
+        sh = G // 2 if shift is None else shift
+        _check(lib().s2attn_bwd_strided(
+            _ptr(q, True), _ptr(k, True), _ptr(v, True), _ptr(o, True), _ptr(lse),
+            _ptr(dO, True), _ptr(dq, True), _ptr(dk, True), _ptr(dv, True), B, Hq, Hkv, N, d, G,
+            scale, shb, sh, _strides_array(q, k, v, o, dO, dq, dk, dv), _ptr(workspace),
+            workspace.numel(), _stream(stream)), "s2attn_bwd_strided")
+        return
     if shift_head_begin is None and shift is None:
         _check(lib().s2attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO),
                                 _ptr(dq), _ptr(dk), _ptr(dv), B, Hq, Hkv, N, d, G, scale,

@@ -40,6 +40,7 @@ struct BwdParams {
   const float* lse2;   // [B, Hq, N]  LSE * log2(e)
   const float* dvec;   // [B, Hq, N]  D = rowsum(dO o O)
   __nv_bfloat16* dq;
+  long long dq_sb, dq_st;   // element strides of dQ's batch and token axes
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
   int B, Hq, Hkv, N, G, shift_head_begin, shift;

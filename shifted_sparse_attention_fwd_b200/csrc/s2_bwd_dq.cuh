@@ -241,7 +241,7 @@ __global__ void __launch_bounds__(320, 1)
     }
     if (ok && warp_wait(bar(L::B_ACC), 0, ctx, 9)) {
       tc_fence_after();
-      __nv_bfloat16* qrow = p.dq + ((static_cast<size_t>(b) * p.N + t) * p.Hq + h) * D;
+      __nv_bfloat16* qrow = p.dq + b * p.dq_sb + t * p.dq_st + static_cast<long long>(h) * D;
 #pragma unroll
       for (int j = half * (D / 64); j < (half + 1) * (D / 64); ++j) {
         uint32_t rr[32];

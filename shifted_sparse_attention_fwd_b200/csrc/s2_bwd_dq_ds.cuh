@@ -191,7 +191,7 @@ __global__ void __launch_bounds__(192, 1)
       int t = r + head_shift(hq);
       if (t >= p.N) t -= p.N;
       __nv_bfloat16* dst_row =
-          p.dq + ((static_cast<size_t>(b) * p.N + (valid ? t : 0)) * p.Hq + hq) * D;
+          p.dq + b * p.dq_sb + (valid ? t : 0) * p.dq_st + static_cast<long long>(hq) * D;
 #pragma unroll
       for (int j = 0; j < D / 32; ++j) {
         uint32_t rr[32];

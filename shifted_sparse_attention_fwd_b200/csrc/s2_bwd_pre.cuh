@@ -14,8 +14,9 @@
 
 namespace s2 {
 
-// A block covers kPreTokens consecutive tokens of one batch and every head: the rows of O and
-// dO it reads (token-major, head-minor) are one contiguous range of memory.
+// A block covers kPreTokens consecutive tokens of one batch and every head: for contiguous O
+// and dO the rows it reads (token-major, head-minor) are one contiguous range of memory.
+// O and dO are addressed through their batch and token strides (elements).
 constexpr int kPreTokens = 8;
 
 template <int D>
@@ -25,7 +26,9 @@ __global__ void __launch_bounds__(256) s2_bwd_pre_kernel(const __nv_bfloat16* __
                                                          float* __restrict__ dvec,
                                                          float* __restrict__ lse2,
                                                          unsigned int* __restrict__ sched,
-                                                         int sched_words, int Hq, int N) {
+                                                         int sched_words, int Hq, int N,
+                                                         long long o_sb, long long o_st,
+                                                         long long do_sb, long long do_st) {
   constexpr int kLanesPerRow = D / 8;            // 16-byte chunks per (token, head) row
   constexpr int kRowsPerWarp = 32 / kLanesPerRow;
   // The work counters of the gradient kernels that follow start from zero.
@@ -39,7 +42,7 @@ __global__ void __launch_bounds__(256) s2_bwd_pre_kernel(const __nv_bfloat16* __
   const int rows = nt * Hq;                      // rows r = (t - t0) * Hq + h
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int sub = lane / kLanesPerRow, li = lane % kLanesPerRow;
-  const size_t base = (static_cast<size_t>(b) * N + t0) * Hq;   // first row of the block
+
   constexpr int kUnroll = 4;                     // row pairs in flight per thread
   for (int r0 = warp * kRowsPerWarp; r0 < rows; r0 += kUnroll * 8 * kRowsPerWarp) {
     uint4 ov[kUnroll], gv[kUnroll];
@@ -47,9 +50,9 @@ __global__ void __launch_bounds__(256) s2_bwd_pre_kernel(const __nv_bfloat16* __
     for (int k = 0; k < kUnroll; ++k) {
       const int rr = r0 + k * 8 * kRowsPerWarp + sub;
       if (rr < rows) {
-        const size_t off = (base + rr) * D + li * 8;
-        ov[k] = __ldg(reinterpret_cast<const uint4*>(o + off));
-        gv[k] = __ldg(reinterpret_cast<const uint4*>(dO + off));
+        const long long t = t0 + rr / Hq, hd = static_cast<long long>(rr % Hq) * D + li * 8;
+        ov[k] = __ldg(reinterpret_cast<const uint4*>(o + b * o_sb + t * o_st + hd));
+        gv[k] = __ldg(reinterpret_cast<const uint4*>(dO + b * do_sb + t * do_st + hd));
       } else {
         ov[k] = make_uint4(0, 0, 0, 0);
         gv[k] = make_uint4(0, 0, 0, 0);

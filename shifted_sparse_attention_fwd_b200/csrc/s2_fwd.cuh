@@ -38,6 +38,7 @@ namespace s2 {
 
 struct FwdParams {
   __nv_bfloat16* o;
+  long long o_sb, o_st;   // element strides of O's batch and token axes
   float* lse;
   int B, Hq, Hkv, N, G, shift_head_begin, shift;
   float scale_log2;   // scale * log2(e)
@@ -398,7 +399,7 @@ __global__ void __launch_bounds__(320, 1)
           if (rq < p.N) {
             const long long tq = static_cast<long long>(rq) + u.shift_h;
             const int tok = static_cast<int>(tq >= p.N ? tq - p.N : tq);
-            __nv_bfloat16* dst = p.o + ((static_cast<size_t>(u.b) * p.N + tok) * p.Hq + u.h) * D +
+            __nv_bfloat16* dst = p.o + u.b * p.o_sb + tok * p.o_st + static_cast<long long>(u.h) * D +
                                  64 * half + 8 * chunk;
             *reinterpret_cast<uint4*>(dst) = w4;
           }

@@ -107,9 +107,9 @@ s2attn_status get_encoder() {
 // Tensor map over a bf16 [B, N, H, d] tensor: dims (d, H, N, B), box (64, 1, rows, 1),
 // 128-byte swizzle, zero fill out of bounds.
 s2attn_status encode_map(CUtensorMap* m, const void* base, int B, int H, int N, int d,
-                         int box_rows) {
+                         int box_rows, long long sb, long long st) {
   cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)B};
-  cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2, (cuuint64_t)N * H * d * 2};
+  cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)st * 2, (cuuint64_t)sb * 2};
   cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
@@ -126,10 +126,11 @@ s2attn_status encode_map(CUtensorMap* m, const void* base, int B, int H, int N, 
 struct MapPair {
   CUtensorMap m128, m8;
 };
-s2attn_status encode_pair(MapPair& mp, const void* base, int B, int H, int N, int d) {
-  s2attn_status s = encode_map(&mp.m128, base, B, H, N, d, s2::kTileRows);
+s2attn_status encode_pair(MapPair& mp, const void* base, int B, int H, int N, int d, long long sb,
+                          long long st) {
+  s2attn_status s = encode_map(&mp.m128, base, B, H, N, d, s2::kTileRows, sb, st);
   if (s != S2ATTN_OK) return s;
-  return encode_map(&mp.m8, base, B, H, N, d, 8);
+  return encode_map(&mp.m8, base, B, H, N, d, 8, sb, st);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -144,8 +145,20 @@ size_t ws_half(int B, int Hq, int N) {
   return (bytes + 255) & ~static_cast<size_t>(255);
 }
 
+// Element strides of each [B, N, H, d] tensor: X[b, t, h, c] is at X + b sb + t st + h d + c
+// (the (H, d) block of a token is contiguous). Contiguous tensors have st = H d, sb = N st.
+enum TensorId { T_Q = 0, T_K, T_V, T_O, T_DO, T_DQ, T_DK, T_DV, T_COUNT };
+
 struct Shape {
   int B, Hq, Hkv, N, d, G, shb, shift;
+  long long sb[T_COUNT], st[T_COUNT];
+  int heads(int t) const { return (t == T_K || t == T_V || t == T_DK || t == T_DV) ? Hkv : Hq; }
+  void set_contiguous() {
+    for (int t = 0; t < T_COUNT; ++t) {
+      st[t] = static_cast<long long>(heads(t)) * d;
+      sb[t] = st[t] * N;
+    }
+  }
 };
 
 // dS hand-off (backward without recomputation in the dQ pass): the slot layout, and the bytes
@@ -188,7 +201,8 @@ s2attn_status check_shape(int B, int Hq, int Hkv, int N, int d, int G, float sca
   if (s % 8 != 0) return S2ATTN_ERR_UNSUPPORTED;
   const long long rows = static_cast<long long>(B) * (Hq > Hkv ? Hq : Hkv) * ((N + 127) / 128);
   if (rows >= (1ll << 31)) return S2ATTN_ERR_UNSUPPORTED;
-  out = Shape{B, Hq, Hkv, N, d, G, shift_head_begin, static_cast<int>(s)};
+  out = Shape{B, Hq, Hkv, N, d, G, shift_head_begin, static_cast<int>(s), {}, {}};
+  out.set_contiguous();
   return S2ATTN_OK;
 }
 
@@ -198,11 +212,13 @@ s2attn_status launch_fwd(const Shape& sh, const void* q, const void* k, const vo
                          int num_sms) {
   MapPair mq, mk, mv;
   s2attn_status s;
-  if ((s = encode_pair(mq, q, sh.B, sh.Hq, sh.N, D)) != S2ATTN_OK) return s;
-  if ((s = encode_pair(mk, k, sh.B, sh.Hkv, sh.N, D)) != S2ATTN_OK) return s;
-  if ((s = encode_pair(mv, v, sh.B, sh.Hkv, sh.N, D)) != S2ATTN_OK) return s;
+  if ((s = encode_pair(mq, q, sh.B, sh.Hq, sh.N, D, sh.sb[T_Q], sh.st[T_Q])) != S2ATTN_OK) return s;
+  if ((s = encode_pair(mk, k, sh.B, sh.Hkv, sh.N, D, sh.sb[T_K], sh.st[T_K])) != S2ATTN_OK) return s;
+  if ((s = encode_pair(mv, v, sh.B, sh.Hkv, sh.N, D, sh.sb[T_V], sh.st[T_V])) != S2ATTN_OK) return s;
   s2::FwdParams p{};
   p.o = static_cast<__nv_bfloat16*>(o);
+  p.o_sb = sh.sb[T_O];
+  p.o_st = sh.st[T_O];
   p.lse = lse;
   p.B = sh.B; p.Hq = sh.Hq; p.Hkv = sh.Hkv; p.N = sh.N; p.G = sh.G;
   p.shift_head_begin = sh.shb; p.shift = sh.shift;
@@ -232,6 +248,8 @@ s2::BwdParams bwd_params(const Shape& sh, float scale, const void* workspace, vo
   p.scale_log2 = scale * 1.4426950408889634f;
   p.err = err;
   p.timeout_ns = g_timeout_ns.load();
+  p.dq_sb = sh.sb[T_DQ];
+  p.dq_st = sh.st[T_DQ];
   p.kvh_begin = 0;
   p.kvh_count = sh.Hkv;
   p.ds = nullptr;
@@ -259,7 +277,8 @@ s2attn_status launch_pre(const Shape& sh, const void* o, const float* lse, const
   const unsigned grid = static_cast<unsigned>(sh.B) * ((sh.N + s2::kPreTokens - 1) / s2::kPreTokens);
   s2::s2_bwd_pre_kernel<D><<<grid, 256, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, dvec,
-      lse2, ws_sched(workspace, sh), kSchedWords, sh.Hq, sh.N);
+      lse2, ws_sched(workspace, sh), kSchedWords, sh.Hq, sh.N, sh.sb[T_O], sh.st[T_O],
+      sh.sb[T_DO], sh.st[T_DO]);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? S2ATTN_OK : cuda_fail(e, "s2_bwd_pre_kernel launch");
 }
@@ -271,17 +290,19 @@ s2attn_status launch_grad(const Shape& sh, const void* q, const void* k, const v
                           int num_sms, int ds_kvh_begin = -1, int ds_kvh_count = 0) {
   MapPair mq, mk, mv, mo;
   s2attn_status s;
-  if ((s = encode_pair(mq, q, sh.B, sh.Hq, sh.N, D)) != S2ATTN_OK) return s;
-  if ((s = encode_pair(mk, k, sh.B, sh.Hkv, sh.N, D)) != S2ATTN_OK) return s;
-  if ((s = encode_pair(mv, v, sh.B, sh.Hkv, sh.N, D)) != S2ATTN_OK) return s;
-  if ((s = encode_pair(mo, dO, sh.B, sh.Hq, sh.N, D)) != S2ATTN_OK) return s;
+  if ((s = encode_pair(mq, q, sh.B, sh.Hq, sh.N, D, sh.sb[T_Q], sh.st[T_Q])) != S2ATTN_OK) return s;
+  if ((s = encode_pair(mk, k, sh.B, sh.Hkv, sh.N, D, sh.sb[T_K], sh.st[T_K])) != S2ATTN_OK) return s;
+  if ((s = encode_pair(mv, v, sh.B, sh.Hkv, sh.N, D, sh.sb[T_V], sh.st[T_V])) != S2ATTN_OK) return s;
+  if ((s = encode_pair(mo, dO, sh.B, sh.Hq, sh.N, D, sh.sb[T_DO], sh.st[T_DO])) != S2ATTN_OK) return s;
   s2::BwdParams p = bwd_params(sh, scale, workspace, dq, dk, dv, err);
   if (ds_kvh_begin >= 0) set_ds_pass(p, sh, workspace, ds_kvh_begin, ds_kvh_count);
   const unsigned tiles = (sh.N + 127) / 128;
   if (kDkdv) {
     MapPair mdk, mdv;
-    if ((s = encode_pair(mdk, dk, sh.B, sh.Hkv, sh.N, D)) != S2ATTN_OK) return s;
-    if ((s = encode_pair(mdv, dv, sh.B, sh.Hkv, sh.N, D)) != S2ATTN_OK) return s;
+    if ((s = encode_pair(mdk, dk, sh.B, sh.Hkv, sh.N, D, sh.sb[T_DK], sh.st[T_DK])) != S2ATTN_OK)
+      return s;
+    if ((s = encode_pair(mdv, dv, sh.B, sh.Hkv, sh.N, D, sh.sb[T_DV], sh.st[T_DV])) != S2ATTN_OK)
+      return s;
     const unsigned units = static_cast<unsigned>(sh.B) * p.kvh_count * tiles;
     const unsigned grid = units < static_cast<unsigned>(num_sms) ? units : static_cast<unsigned>(num_sms);
     s2::s2_bwd_dkdv_kernel<D><<<grid, s2::DkdvLayout<D>::kThreads, s2::DkdvLayout<D>::kLaunchBytes, stream>>>(
@@ -302,7 +323,7 @@ s2attn_status launch_dq_ds(const Shape& sh, const void* k, void* dq, float scale
                            cudaStream_t stream, unsigned int* err, int num_sms) {
   MapPair mk;
   s2attn_status s;
-  if ((s = encode_pair(mk, k, sh.B, sh.Hkv, sh.N, D)) != S2ATTN_OK) return s;
+  if ((s = encode_pair(mk, k, sh.B, sh.Hkv, sh.N, D, sh.sb[T_K], sh.st[T_K])) != S2ATTN_OK) return s;
   s2::BwdParams p = bwd_params(sh, scale, workspace, dq, nullptr, nullptr, err);
   set_ds_pass(p, sh, workspace, kvh_begin, kvh_count);
   p.sched = ws_sched(workspace, sh) + 2;
@@ -355,6 +376,24 @@ s2attn_status pre_impl(const Shape& sh, const void* o, const float* lse, const v
                     : launch_pre<128>(sh, o, lse, dO, ws, stream);
 }
 
+// Caller-given strides for tensors ids[0..n): strides[2i] = batch, strides[2i+1] = token (in
+// elements). Each must be a multiple of 8 (16 bytes, the TMA rule), the token stride must span
+// the token's (H, d) block, and batches must not overlap.
+s2attn_status apply_strides(Shape& sh, const long long* strides, const int* ids, int n) {
+  if (!strides) return S2ATTN_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i) {
+    const long long sb = strides[2 * i], st = strides[2 * i + 1];
+    const int t = ids[i];
+    if (sb < 0 || st < static_cast<long long>(sh.heads(t)) * sh.d || sb % 8 != 0 || st % 8 != 0)
+      return S2ATTN_ERR_INVALID_ARG;
+    if (sh.B > 1 && sb < st * sh.N) return S2ATTN_ERR_INVALID_ARG;
+    if (st >= (1ll << 37) || sb >= (1ll << 38)) return S2ATTN_ERR_UNSUPPORTED;   // TMA stride range
+    sh.sb[t] = sb;
+    sh.st[t] = st;
+  }
+  return S2ATTN_OK;
+}
+
 // Self-test kernel: a bounded wait on a barrier that nothing arrives on.
 __global__ void selftest_wait_kernel(unsigned int* err, unsigned long long timeout_ns) {
   __shared__ __align__(8) uint64_t barrier;
@@ -393,15 +432,20 @@ void s2attn_set_wait_timeout_ns(unsigned long long ns) {
   g_timeout_ns.store(ns == 0 ? kDefaultTimeoutNs : ns);
 }
 
-s2attn_status s2attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse,
-                            int B, int Hq, int Hkv, int N, int d, int G, float scale,
-                            int shift_head_begin, int shift, void* stream) {
+s2attn_status s2attn_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse,
+                                 int B, int Hq, int Hkv, int N, int d, int G, float scale,
+                                 int shift_head_begin, int shift, const long long* strides,
+                                 void* stream) {
   if (!q || !k || !v || !o || !lse) return S2ATTN_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return S2ATTN_ERR_INVALID_ARG;
   Shape sh;
   s2attn_status s = check_shape(B, Hq, Hkv, N, d, G, scale, shift_head_begin, shift, sh);
   if (s != S2ATTN_OK) return s;
+  if (strides) {
+    static const int ids[4] = {T_Q, T_K, T_V, T_O};
+    if ((s = apply_strides(sh, strides, ids, 4)) != S2ATTN_OK) return s;
+  }
   if ((s = get_encoder()) != S2ATTN_OK) return s;
   unsigned int* err = nullptr;
   int num_sms = 0;
@@ -409,6 +453,14 @@ s2attn_status s2attn_fwd_ex(const void* q, const void* k, const void* v, void* o
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return d == 64 ? launch_fwd<64>(sh, q, k, v, o, lse, scale, st, err, num_sms)
                  : launch_fwd<128>(sh, q, k, v, o, lse, scale, st, err, num_sms);
+}
+
+s2attn_status s2attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse,
+                            int B, int Hq, int Hkv, int N, int d, int G, float scale,
+                            int shift_head_begin, int shift, void* stream) {
+  // null strides: contiguous tensors
+  return s2attn_fwd_strided(q, k, v, o, lse, B, Hq, Hkv, N, d, G, scale, shift_head_begin, shift,
+                            nullptr, stream);
 }
 
 s2attn_status s2attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -447,7 +499,8 @@ s2attn_status s2attn_bwd_preprocess(const void* o, const float* lse, const void*
   if (d != 64 && d != 128) return S2ATTN_ERR_UNSUPPORTED;
   if (N >= (1 << 30) || static_cast<long long>(B) * Hq * ((N + 127) / 128) >= (1ll << 31))
     return S2ATTN_ERR_UNSUPPORTED;
-  const Shape sh{B, Hq, Hq, N, d, N, Hq, 0};
+  Shape sh{B, Hq, Hq, N, d, N, Hq, 0, {}, {}};
+  sh.set_contiguous();
   s2attn_status s = check_workspace(sh, workspace, workspace_bytes);
   if (s != S2ATTN_OK) return s;
   return pre_impl(sh, o, lse, dO, workspace, static_cast<cudaStream_t>(stream));
@@ -538,11 +591,11 @@ s2attn_status s2attn_bwd_dq_ds(const void* k, void* dq, int B, int Hq, int Hkv, 
                     num_sms);
 }
 
-s2attn_status s2attn_bwd_ex(const void* q, const void* k, const void* v, const void* o,
-                            const float* lse, const void* dO, void* dq, void* dk, void* dv,
-                            int B, int Hq, int Hkv, int N, int d, int G, float scale,
-                            int shift_head_begin, int shift, void* workspace,
-                            size_t workspace_bytes, void* stream) {
+s2attn_status s2attn_bwd_strided(const void* q, const void* k, const void* v, const void* o,
+                                 const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                                 int B, int Hq, int Hkv, int N, int d, int G, float scale,
+                                 int shift_head_begin, int shift, const long long* strides,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
   if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return S2ATTN_ERR_INVALID_ARG;
   const void* ptrs[] = {q, k, v, o, lse, dO, dq, dk, dv};
   for (const void* ptr : ptrs)
@@ -550,6 +603,10 @@ s2attn_status s2attn_bwd_ex(const void* q, const void* k, const void* v, const v
   Shape sh;
   s2attn_status s = check_shape(B, Hq, Hkv, N, d, G, scale, shift_head_begin, shift, sh);
   if (s != S2ATTN_OK) return s;
+  if (strides) {
+    static const int ids[8] = {T_Q, T_K, T_V, T_O, T_DO, T_DQ, T_DK, T_DV};
+    if ((s = apply_strides(sh, strides, ids, 8)) != S2ATTN_OK) return s;
+  }
   if ((s = check_workspace(sh, workspace, workspace_bytes)) != S2ATTN_OK) return s;
   if ((s = get_encoder()) != S2ATTN_OK) return s;
   unsigned int* err = nullptr;
@@ -573,6 +630,16 @@ s2attn_status s2attn_bwd_ex(const void* q, const void* k, const void* v, const v
       return s;
   }
   return S2ATTN_OK;
+}
+
+s2attn_status s2attn_bwd_ex(const void* q, const void* k, const void* v, const void* o,
+                            const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                            int B, int Hq, int Hkv, int N, int d, int G, float scale,
+                            int shift_head_begin, int shift, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  // null strides: contiguous tensors
+  return s2attn_bwd_strided(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, N, d, G, scale,
+                            shift_head_begin, shift, nullptr, workspace, workspace_bytes, stream);
 }
 
 s2attn_status s2attn_bwd(const void* q, const void* k, const void* v, const void* o,

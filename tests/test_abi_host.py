@@ -375,3 +375,24 @@ def test_chunked_kv_tile_order_is_a_permutation(shim, B, Hq, Hkv, N, G, shb, sh,
         assert t0 % 128 == 0
         order.append((b, kvh, t0 // 128))
     assert set(order) == {(b, k, t) for b in range(B) for k in range(Hkv) for t in range(nt)}
+
+
+def test_strided_entries_reject(lib):
+    """Stride validation happens on the host, before anything is launched."""
+    f = ctypes.c_float(0.125)
+    LL = ctypes.c_longlong
+    good = [256 * 4 * 64 * 3, 4 * 64 * 3] * 4          # packed qkv-like strides, B = 2
+    ok_args = [A] * 5 + [2, 4, 4, 256, 64, 64, f, 2, 32]
+    bad_cases = [
+        [256 * 4 * 64 * 3, 4 * 64 - 8] + good[2:],      # token stride below H*d
+        [256 * 4 * 64 * 3, 4 * 64 * 3 + 4] + good[2:],  # not a multiple of 8 elements
+        [4 * 64 * 3, 4 * 64 * 3] + good[2:],            # batches overlap (B = 2)
+    ]
+    for st in bad_cases:
+        arr = (LL * 8)(*st)
+        assert lib.s2attn_fwd_strided(*ok_args, arr, None) == 1
+    ws = 0x100000
+    need = lib.s2attn_bwd_workspace_size(2, 4, 256)
+    arr = (LL * 16)(*([4 * 64 * 3, 4 * 64 - 8] * 8))
+    assert lib.s2attn_bwd_strided(*([A] * 9), 2, 4, 4, 256, 64, 64, f, 2, 32, arr, ws, need,
+                                  None) == 1
