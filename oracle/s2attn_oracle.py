@@ -32,6 +32,10 @@ Readings where the page is silent (each also listed in the design notes):
   * ``shift_head_begin`` (default Hq/2, the page's chunk(2)) and ``shift`` (default G/2)
     generalise the split point and the roll amount for the ablation patterns; the roll
     is always rolled[r] = x[(r + shift) mod N].
+  * ``wrap_own_group`` is the page's Variant 2 (Table 8, Figure 6): in the shifted heads the
+    tokens that the roll wrapped around (original tokens 0..shift-1, the last ``shift``
+    rolled rows) form their own group instead of sharing the last group with the last
+    G - shift tokens; that last group is split at the wrap point into two causal groups.
 
 Everything is float64; inputs are the bf16 values widened exactly.
 """
@@ -69,24 +73,30 @@ def expand_kv(x: np.ndarray, Hq: int) -> np.ndarray:
     return np.repeat(x, rep, axis=2)
 
 
-def _group_probs(q: np.ndarray, k: np.ndarray, scale: float):
+def _group_probs(q: np.ndarray, k: np.ndarray, scale: float, split: int | None = None):
     """Causal softmax of scale * q k^T for one group and head; q, k are [G, d].
 
+    With ``split``, rows [0, split) and [split, G) are two separate causal groups.
     Returns (P, lse) with P [G, G] (zero above the diagonal) and lse [G].
     """
     G = q.shape[0]
     s = scale * (q @ k.T)
-    s = np.where(np.tril(np.ones((G, G), dtype=bool)), s, -np.inf)
+    allowed = np.tril(np.ones((G, G), dtype=bool))
+    if split is not None:
+        side = np.arange(G) >= split
+        allowed &= side[:, None] == side[None, :]
+    s = np.where(allowed, s, -np.inf)
     m = s.max(axis=1, keepdims=True)
     e = np.exp(s - m)
     l = e.sum(axis=1, keepdims=True)
     return e / l, (m + np.log(l))[:, 0]
 
 
-def causal_self_attn(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float):
+def causal_self_attn(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float, splits=None):
     """Standard causal self-attention on every batch element: q, k, v [Bg, G, H, d].
 
     This is the ``self_attn(qkv)`` call of Algorithm 1 after the view into groups.
+    ``splits(bg, h)`` optionally names a row where group bg of head h splits in two.
     Returns o [Bg, G, H, d] and lse [Bg, G, H].
     """
     Bg, G, H, d = q.shape
@@ -94,12 +104,13 @@ def causal_self_attn(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float):
     lse = np.empty((Bg, G, H))
     for b in range(Bg):
         for h in range(H):
-            p, lse[b, :, h] = _group_probs(q[b, :, h], k[b, :, h], scale)
+            sp = splits(b, h) if splits else None
+            p, lse[b, :, h] = _group_probs(q[b, :, h], k[b, :, h], scale, sp)
             o[b, :, h] = p @ v[b, :, h]
     return o, lse
 
 
-def causal_self_attn_backward(q, k, v, do, scale):
+def causal_self_attn_backward(q, k, v, do, scale, splits=None):
     """Gradients of causal_self_attn for upstream do [Bg, G, H, d] (direct differentiation).
 
     Returns dq, dk, dv, each [Bg, G, H, d]; dk and dv are per query head (not yet summed
@@ -111,7 +122,8 @@ def causal_self_attn_backward(q, k, v, do, scale):
     dv = np.empty_like(v)
     for b in range(Bg):
         for h in range(H):
-            p, _ = _group_probs(q[b, :, h], k[b, :, h], scale)
+            sp = splits(b, h) if splits else None
+            p, _ = _group_probs(q[b, :, h], k[b, :, h], scale, sp)
             dp = do[b, :, h] @ v[b, :, h].T
             ds = p * (dp - (p * dp).sum(axis=1, keepdims=True))
             dq[b, :, h] = scale * (ds @ k[b, :, h])
@@ -128,7 +140,18 @@ def _defaults(Hq, G, shift_head_begin, shift):
     return shift_head_begin, shift
 
 
-def s2attn_forward(q, k, v, G, scale, shift_head_begin=None, shift=None):
+def _wrap_splits(B, N, G, shb, shift, wrap_own_group):
+    """Variant 2: the last group of every batch element, in heads >= shb, splits at the wrap
+    (in-group row G - shift: rolled rows N - shift .. N - 1 hold original tokens 0..shift-1)."""
+    if not wrap_own_group:
+        return None
+    if not 0 < shift < G:
+        raise ValueError("the wrap group exists for 0 < shift < G")
+    ng = N // G
+    return lambda bg, h: (G - shift) if (h >= shb and bg % ng == ng - 1) else None
+
+
+def s2attn_forward(q, k, v, G, scale, shift_head_begin=None, shift=None, wrap_own_group=False):
     """S²-Attn forward. q [B,N,Hq,d], k, v [B,N,Hkv,d] float64.
 
     Returns o [B,N,Hq,d] and lse [B,Hq,N], both in original token order.
@@ -137,19 +160,21 @@ def s2attn_forward(q, k, v, G, scale, shift_head_begin=None, shift=None):
     if N % G != 0:
         raise ValueError("the view into groups needs G to divide N")
     shb, shift = _defaults(Hq, G, shift_head_begin, shift)
+    splits = _wrap_splits(B, N, G, shb, shift, wrap_own_group)
     ke, ve = expand_kv(k, Hq), expand_kv(v, Hq)
     # Key line 1: roll the second chunk of heads by -shift, then view as groups.
     qr = chunk_roll(q, -shift, shb).reshape(B * N // G, G, Hq, d)
     kr = chunk_roll(ke, -shift, shb).reshape(B * N // G, G, Hq, d)
     vr = chunk_roll(ve, -shift, shb).reshape(B * N // G, G, Hq, v.shape[3])
-    o, lse = causal_self_attn(qr, kr, vr, scale)
+    o, lse = causal_self_attn(qr, kr, vr, scale, splits)
     # Key line 2: back to [B, N, H, d], roll the second chunk back by +shift.
     o = chunk_roll(o.reshape(B, N, Hq, v.shape[3]), shift, shb)
     lse = chunk_roll(lse.reshape(B, N, Hq), shift, shb)
     return o, np.ascontiguousarray(lse.transpose(0, 2, 1))
 
 
-def s2attn_backward(q, k, v, do, G, scale, shift_head_begin=None, shift=None):
+def s2attn_backward(q, k, v, do, G, scale, shift_head_begin=None, shift=None,
+                    wrap_own_group=False):
     """Gradients of s2attn_forward's o with respect to q, k, v for upstream do [B,N,Hq,d].
 
     Returns dq [B,N,Hq,d], dk [B,N,Hkv,d], dv [B,N,Hkv,d] in original token order.
@@ -157,12 +182,13 @@ def s2attn_backward(q, k, v, do, G, scale, shift_head_begin=None, shift=None):
     B, N, Hq, d = q.shape
     Hkv = k.shape[2]
     shb, shift = _defaults(Hq, G, shift_head_begin, shift)
+    splits = _wrap_splits(B, N, G, shb, shift, wrap_own_group)
     ke, ve = expand_kv(k, Hq), expand_kv(v, Hq)
     qr = chunk_roll(q, -shift, shb).reshape(B * N // G, G, Hq, d)
     kr = chunk_roll(ke, -shift, shb).reshape(B * N // G, G, Hq, d)
     vr = chunk_roll(ve, -shift, shb).reshape(B * N // G, G, Hq, d)
     dor = chunk_roll(do, -shift, shb).reshape(B * N // G, G, Hq, d)
-    dq, dk, dv = causal_self_attn_backward(qr, kr, vr, dor, scale)
+    dq, dk, dv = causal_self_attn_backward(qr, kr, vr, dor, scale, splits)
     # The derivative of a roll is the opposite roll ...
     dq = chunk_roll(dq.reshape(B, N, Hq, d), shift, shb)
     dk = chunk_roll(dk.reshape(B, N, Hq, d), shift, shb)

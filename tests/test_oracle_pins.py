@@ -11,6 +11,8 @@
 * direction invariance of the roll when G divides N (§3.4 "Why shifting direction doesn't
   matter", Table 8);
 * the worked roll example (§3.4 "Step 2: Shift one chunk"), from tests/golden;
+* Variant 2 of Table 8 (wrapped tokens in their own group): equal to the library version with
+  the wrap group split by an explicit mask, and identical to the default outside that group;
 * central finite differences of the forward against the backward;
 * closed-form sums implied by rows of P summing to one;
 * planted mistakes in the oracle must fail these pins.
@@ -40,7 +42,7 @@ def make(B, Hq, Hkv, N, d, seed=0):
 # --------------------------------------------------------------------------------------
 # Library implementation: torch.roll + SDPA per head and group, autograd for gradients.
 # --------------------------------------------------------------------------------------
-def torch_s2attn(q, k, v, G, scale, shb, shift):
+def torch_s2attn(q, k, v, G, scale, shb, shift, wrap_own_group=False):
     B, N, Hq, d = q.shape
     rep = Hq // k.shape[2]
     outs, lses = [], []
@@ -49,9 +51,13 @@ def torch_s2attn(q, k, v, G, scale, shb, shift):
         qh = torch.roll(q[:, :, h], -s, dims=1).reshape(B, N // G, G, d)
         kh = torch.roll(k[:, :, h // rep], -s, dims=1).reshape(B, N // G, G, d)
         vh = torch.roll(v[:, :, h // rep], -s, dims=1).reshape(B, N // G, G, -1)
-        oh = F.scaled_dot_product_attention(qh, kh, vh, is_causal=True, scale=scale)
+        mask = torch.ones(N // G, G, G, dtype=torch.bool).tril()
+        if wrap_own_group and s > 0:
+            side = torch.arange(G) >= G - s          # rows that hold wrapped tokens
+            mask[-1] &= side[:, None] == side[None, :]
+        oh = F.scaled_dot_product_attention(qh, kh, vh, attn_mask=mask, scale=scale)
         scores = scale * qh @ kh.transpose(-1, -2)
-        scores = scores.masked_fill(~torch.ones(G, G, dtype=torch.bool).tril(), float("-inf"))
+        scores = scores.masked_fill(~mask, float("-inf"))
         lh = torch.logsumexp(scores, dim=-1)
         outs.append(torch.roll(oh.reshape(B, N, -1), s, dims=1))
         lses.append(torch.roll(lh.reshape(B, N), s, dims=1))
@@ -90,6 +96,41 @@ def test_matches_library_patterns(shb, shift):
     # written as shift = N - G/2), a different roll amount, and a zero roll.
     errs = library_errors(1, 4, 2, 32, 16, 4, shb=shb, shift=shift)
     assert max(errs) < 1e-12, errs
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,G,d,shift", [(1, 4, 4, 64, 16, 8, 8), (2, 4, 2, 48, 16, 8, 4),
+                                                  (1, 2, 1, 32, 32, 4, 16)])
+def test_variant2_matches_library_with_split_mask(B, Hq, Hkv, N, G, d, shift):
+    q, k, v, do = make(B, Hq, Hkv, N, d, 11)
+    scale = 1.0 / np.sqrt(d)
+    o, lse = orc.s2attn_forward(q, k, v, G, scale, None, shift, wrap_own_group=True)
+    dq, dk, dv = orc.s2attn_backward(q, k, v, do, G, scale, None, shift, wrap_own_group=True)
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    to, tl = torch_s2attn(tq, tk, tv, G, scale, Hq // 2, shift, wrap_own_group=True)
+    to.backward(torch.tensor(do))
+    for a, b in ((o, to), (lse, tl), (dq, tq.grad), (dk, tk.grad), (dv, tv.grad)):
+        assert np.abs(a - b.detach().numpy()).max() < 1e-12
+
+
+def test_variant2_only_changes_the_wrap_group():
+    """Unshifted heads and every shifted-head token outside the last rolled group are
+    bit-identical to the default; the wrapped tokens (0..shift-1) see only each other."""
+    B, Hq, N, G, d, shift = 1, 4, 64, 16, 8, 8
+    q, k, v, do = make(B, Hq, Hq, N, d, 5)
+    a, la = orc.s2attn_forward(q, k, v, G, 0.3, None, shift)
+    b, lb = orc.s2attn_forward(q, k, v, G, 0.3, None, shift, wrap_own_group=True)
+    assert np.array_equal(a[:, :, :2], b[:, :, :2])
+    wrap_tokens = np.r_[N - (G - shift):N, 0:shift]
+    keep = np.setdiff1d(np.arange(N), wrap_tokens)
+    assert np.array_equal(a[:, keep, 2:], b[:, keep, 2:])
+    assert not np.allclose(a[:, wrap_tokens, 2:], b[:, wrap_tokens, 2:])
+    # tokens 0..shift-1 of a shifted head: plain causal attention over those tokens alone
+    h = 3
+    sq = 0.3 * q[0, :shift, h] @ k[0, :shift, h].T
+    sq = np.where(np.tril(np.ones((shift, shift), dtype=bool)), sq, -np.inf)
+    p = np.exp(sq - sq.max(1, keepdims=True))
+    p /= p.sum(1, keepdims=True)
+    np.testing.assert_allclose(b[0, :shift, h], p @ v[0, :shift, h], atol=1e-13)
 
 
 def test_one_group_no_shift_is_full_causal_attention():
@@ -254,7 +295,7 @@ def _tile_kv(x, Hq):
     return np.tile(x, (1, 1, Hq // x.shape[2], 1))
 
 
-def _leaky_probs(q, k, scale):
+def _leaky_probs(q, k, scale, split=None):
     G = q.shape[0]
     s = scale * (q @ k.T)
     s = np.where(np.tril(np.ones((G, G), dtype=bool), k=1), s, -np.inf)
@@ -264,7 +305,7 @@ def _leaky_probs(q, k, scale):
     return e / l, (m + np.log(l))[:, 0]
 
 
-def _backward_without_rowsum(q, k, v, do, scale):
+def _backward_without_rowsum(q, k, v, do, scale, splits=None):
     Bg, G, H, d = q.shape
     dq, dk, dv = np.empty_like(q), np.empty_like(k), np.empty_like(v)
     for b in range(Bg):
