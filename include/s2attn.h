@@ -95,21 +95,32 @@ S2ATTN_API s2attn_status s2attn_fwd_ex(const void* q, const void* k, const void*
                             int B, int Hq, int Hkv, int N, int d, int G, float scale,
                             int shift_head_begin, int shift, void* stream);
 
+/* Option flags of the _general entry points. */
+#define S2ATTN_FLAG_WRAP_OWN_GROUP 1
 /*
- * Strided forms. Each [B, N, H, d] tensor X is read or written at X + b*sb + t*st + h*d + c
+ * S2ATTN_FLAG_WRAP_OWN_GROUP is the pages' Variant 2 (summary page, §3.4 "Information
+ * leakage considerations", Table 8, Figure 6): in the rolled heads the tokens that the roll
+ * wrapped around (original tokens 0..shift-1) form their own group instead of sharing the
+ * last group with the last G - shift tokens, i.e. the last rolled group is split at the wrap
+ * into two causal groups. Requires a rolled head (shift_head_begin < Hq) and 0 < shift < G
+ * (after reduction mod N), else S2ATTN_ERR_INVALID_ARG.
+ *
+ * Strides. Each [B, N, H, d] tensor X is read or written at X + b*sb + t*st + h*d + c
  * (elements): the (H, d) block of a token is contiguous, tokens and batches may be spaced
  * freely. This takes q, k and v as views of one packed qkv [B, N, 3, H, d] buffer, the layout
  * LongLoRA's Algorithm 1 (summary page, §3.4) feeds its attention: q = qkv, k = qkv + H*d,
  * v = qkv + 2*H*d, st = 3*H*d, sb = N*st (and likewise dq, dk, dv into a packed dqkv).
  * `strides` holds {sb, st} pairs: q, k, v, o for the forward; q, k, v, o, dO, dq, dk, dv for
- * the backward; NULL means contiguous (the _ex forms). Every stride must be a multiple of 8
- * elements, st >= H*d and, when B > 1, sb >= N*st; otherwise S2ATTN_ERR_INVALID_ARG. lse stays
- * a contiguous [B, Hq, N] array. Outputs must not overlap each other or the inputs.
+ * the backward; NULL means contiguous. Every stride must be a multiple of 8 elements,
+ * st >= H*d and, when B > 1, sb >= N*st; otherwise S2ATTN_ERR_INVALID_ARG. lse stays a
+ * contiguous [B, Hq, N] array. Outputs must not overlap each other or the inputs.
+ *
+ * s2attn_fwd_general: s2attn_fwd_ex with option flags and strides.
  */
-S2ATTN_API s2attn_status s2attn_fwd_strided(const void* q, const void* k, const void* v, void* o,
+S2ATTN_API s2attn_status s2attn_fwd_general(const void* q, const void* k, const void* v, void* o,
                                             float* lse, int B, int Hq, int Hkv, int N, int d,
                                             int G, float scale, int shift_head_begin, int shift,
-                                            const long long* strides, void* stream);
+                                            int flags, const long long* strides, void* stream);
 
 /* Smallest device workspace s2attn_bwd accepts: two fp32 [B, Hq, N] arrays (D and LSE in
  * base 2), each rounded up to 256 bytes, and 256 bytes of work counters for the gradient
@@ -130,6 +141,10 @@ S2ATTN_API size_t s2attn_bwd_workspace_size(int B, int Hq, int N);
  */
 S2ATTN_API size_t s2attn_bwd_workspace_size_ex(int B, int Hq, int Hkv, int N, int d, int G,
                                                int shift_head_begin, int shift, size_t cap_bytes);
+/* The same for the option flags of s2attn_bwd_general (Variant 2 changes the dS tile count). */
+S2ATTN_API size_t s2attn_bwd_workspace_size_general(int B, int Hq, int Hkv, int N, int d, int G,
+                                                    int shift_head_begin, int shift, int flags,
+                                                    size_t cap_bytes);
 
 /*
  * Backward: dq, dk, dv from q, k, v, the forward's o and lse, and the upstream dO.
@@ -154,12 +169,13 @@ S2ATTN_API s2attn_status s2attn_bwd_ex(const void* q, const void* k, const void*
                             int shift_head_begin, int shift, void* workspace,
                             size_t workspace_bytes, void* stream);
 
-/* Backward with strided tensors (see s2attn_fwd_strided; 8 {sb, st} pairs). */
-S2ATTN_API s2attn_status s2attn_bwd_strided(const void* q, const void* k, const void* v,
+/* s2attn_bwd_ex with option flags and strides (see s2attn_fwd_general; 8 {sb, st} pairs).
+ * With flags, size the workspace with s2attn_bwd_workspace_size_general. */
+S2ATTN_API s2attn_status s2attn_bwd_general(const void* q, const void* k, const void* v,
                                             const void* o, const float* lse, const void* dO,
                                             void* dq, void* dk, void* dv, int B, int Hq, int Hkv,
                                             int N, int d, int G, float scale,
-                                            int shift_head_begin, int shift,
+                                            int shift_head_begin, int shift, int flags,
                                             const long long* strides, void* workspace,
                                             size_t workspace_bytes, void* stream);
 

@@ -11,6 +11,7 @@ from ._lib import (  # noqa: F401
     S2ATTN_ERR_UNSUPPORTED,
     S2ATTN_ERR_CUDA,
     S2ATTN_ERR_TIMEOUT,
+    S2ATTN_FLAG_WRAP_OWN_GROUP,
     SIGNATURES,
     LIB_PATH,
     lib,

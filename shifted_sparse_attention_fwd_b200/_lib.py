@@ -21,6 +21,9 @@ S2ATTN_ERR_UNSUPPORTED = 2
 S2ATTN_ERR_CUDA = 3
 S2ATTN_ERR_TIMEOUT = 4
 
+# option flags of the _general entry points (include/s2attn.h)
+S2ATTN_FLAG_WRAP_OWN_GROUP = 1
+
 _P = ctypes.c_void_p
 _I = ctypes.c_int
 _F = ctypes.c_float
@@ -41,8 +44,9 @@ SIGNATURES = {
     "s2attn_bwd_dq": (_I, [_P] * 5 + [_I] * 6 + [_F, _I, _I, _P, _Z, _P]),
     "s2attn_bwd_noalloc": (_I, [_P] * 9 + [_I] * 6 + [_F, _P]),
     "s2attn_bwd_workspace_size_ex": (_Z, [_I] * 8 + [_Z]),
-    "s2attn_fwd_strided": (_I, [_P] * 5 + [_I] * 6 + [_F, _I, _I, _P, _P]),
-    "s2attn_bwd_strided": (_I, [_P] * 9 + [_I] * 6 + [_F, _I, _I, _P, _P, _Z, _P]),
+    "s2attn_fwd_general": (_I, [_P] * 5 + [_I] * 6 + [_F, _I, _I, _I, _P, _P]),
+    "s2attn_bwd_general": (_I, [_P] * 9 + [_I] * 6 + [_F, _I, _I, _I, _P, _P, _Z, _P]),
+    "s2attn_bwd_workspace_size_general": (_Z, [_I] * 9 + [_Z]),
     "s2attn_bwd_dkdv_ds": (_I, [_P] * 6 + [_I] * 6 + [_F, _I, _I, _P, _Z, _P]),
     "s2attn_bwd_dq_ds": (_I, [_P] * 2 + [_I] * 6 + [_F, _I, _I, _P, _Z, _P]),
     "s2attn_get_device_error": (_I, [_P, ctypes.POINTER(ctypes.c_uint)]),
@@ -138,19 +142,21 @@ def _check_bf16(*ts):
             raise ValueError(f"expected bf16, got {t.dtype}")
 
 
-def s2attn_fwd(q, k, v, o, lse, G, scale=None, shift_head_begin=None, shift=None, stream=None):
+def s2attn_fwd(q, k, v, o, lse, G, scale=None, shift_head_begin=None, shift=None, stream=None,
+               flags=0):
     """O and LSE of S²-Attn. q [B,N,Hq,d], k/v [B,N,Hkv,d] bf16; o like q; lse fp32 [B,Hq,N]."""
     _check_bf16(q, k, v, o)
     B, Hq, Hkv, N, d, G = _dims(q, k, G)
     scale = d ** -0.5 if scale is None else scale
-    if not _all_contiguous(q, k, v, o):
-        # views (e.g. of a packed qkv buffer): the strided entry point
+    if flags or not _all_contiguous(q, k, v, o):
+        # option flags, or views (e.g. of a packed qkv buffer): the general entry point
         shb = Hq // 2 if shift_head_begin is None else shift_head_begin
         sh = G // 2 if shift is None else shift
-        _check(lib().s2attn_fwd_strided(_ptr(q, True), _ptr(k, True), _ptr(v, True), _ptr(o, True),
+        strides = None if _all_contiguous(q, k, v, o) else _strides_array(q, k, v, o)
+        _check(lib().s2attn_fwd_general(_ptr(q, True), _ptr(k, True), _ptr(v, True), _ptr(o, True),
                                         _ptr(lse), B, Hq, Hkv, N, d, G, scale, shb, sh,
-                                        _strides_array(q, k, v, o), _stream(stream)),
-               "s2attn_fwd_strided")
+                                        int(flags), strides, _stream(stream)),
+               "s2attn_fwd_general")
         return
     if shift_head_begin is None and shift is None:
         _check(lib().s2attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, N, d,
@@ -171,18 +177,19 @@ DEFAULT_WORKSPACE_CAP = 8 << 30
 
 
 def s2attn_bwd_workspace_size_ex(B, Hq, Hkv, N, d, G, shift_head_begin=None, shift=None,
-                                 cap_bytes=0) -> int:
+                                 cap_bytes=0, flags=0) -> int:
     """Workspace for the backward without dQ recomputation (see include/s2attn.h)."""
     shb = Hq // 2 if shift_head_begin is None else shift_head_begin
     sh = G // 2 if shift is None else shift
-    n = int(lib().s2attn_bwd_workspace_size_ex(B, Hq, Hkv, N, d, G, shb, sh, int(cap_bytes)))
+    n = int(lib().s2attn_bwd_workspace_size_general(B, Hq, Hkv, N, d, G, shb, sh, int(flags),
+                                                    int(cap_bytes)))
     if n == 0:
         raise S2AttnError(S2ATTN_ERR_INVALID_ARG, "s2attn_bwd_workspace_size_ex")
     return n
 
 
 def s2attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, G, scale=None, shift_head_begin=None,
-               shift=None, workspace=None, stream=None):
+               shift=None, workspace=None, stream=None, flags=0):
     """dQ, dK, dV of S²-Attn (overwritten). workspace: a uint8 CUDA tensor, or None to let
     torch allocate s2attn_bwd_workspace_size_ex(..., DEFAULT_WORKSPACE_CAP) bytes."""
     _check_bf16(q, k, v, o, dO, dq, dk, dv)
@@ -190,16 +197,18 @@ def s2attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, G, scale=None, shift_head_begin=
     scale = d ** -0.5 if scale is None else scale
     if workspace is None:
         ws_bytes = s2attn_bwd_workspace_size_ex(B, Hq, Hkv, N, d, G, shift_head_begin, shift,
-                                                DEFAULT_WORKSPACE_CAP)
+                                                DEFAULT_WORKSPACE_CAP, flags)
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
-    if not _all_contiguous(q, k, v, o, dO, dq, dk, dv):
+    if flags or not _all_contiguous(q, k, v, o, dO, dq, dk, dv):
         shb = Hq // 2 if shift_head_begin is None else shift_head_begin
         sh = G // 2 if shift is None else shift
-        _check(lib().s2attn_bwd_strided(
+        ts = (q, k, v, o, dO, dq, dk, dv)
+        strides = None if _all_contiguous(*ts) else _strides_array(*ts)
+        _check(lib().s2attn_bwd_general(
             _ptr(q, True), _ptr(k, True), _ptr(v, True), _ptr(o, True), _ptr(lse),
             _ptr(dO, True), _ptr(dq, True), _ptr(dk, True), _ptr(dv, True), B, Hq, Hkv, N, d, G,
-            scale, shb, sh, _strides_array(q, k, v, o, dO, dq, dk, dv), _ptr(workspace),
-            workspace.numel(), _stream(stream)), "s2attn_bwd_strided")
+            scale, shb, sh, int(flags), strides, _ptr(workspace), workspace.numel(),
+            _stream(stream)), "s2attn_bwd_general")
         return
     if shift_head_begin is None and shift is None:
         _check(lib().s2attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dO),
@@ -298,14 +307,16 @@ def s2attn_selftest_wait_timeout(timeout_ns: int, stream=None):
 # ------------------------------------------------------------------------------------------
 # Allocating conveniences (torch provides the memory; the library does the work).
 # ------------------------------------------------------------------------------------------
-def fwd(q, k, v, G, scale=None, shift_head_begin=None, shift=None, stream=None):
+def fwd(q, k, v, G, scale=None, shift_head_begin=None, shift=None, stream=None, flags=0):
     o = torch.empty_like(q)
     lse = torch.empty((q.shape[0], q.shape[2], q.shape[1]), dtype=torch.float32, device=q.device)
-    s2attn_fwd(q, k, v, o, lse, G, scale, shift_head_begin, shift, stream)
+    s2attn_fwd(q, k, v, o, lse, G, scale, shift_head_begin, shift, stream, flags)
     return o, lse
 
 
-def bwd(q, k, v, o, lse, dO, G, scale=None, shift_head_begin=None, shift=None, stream=None):
+def bwd(q, k, v, o, lse, dO, G, scale=None, shift_head_begin=None, shift=None, stream=None,
+        flags=0):
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    s2attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, G, scale, shift_head_begin, shift, None, stream)
+    s2attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, G, scale, shift_head_begin, shift, None, stream,
+               flags)
     return dq, dk, dv

@@ -44,6 +44,7 @@ struct BwdParams {
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
   int B, Hq, Hkv, N, G, shift_head_begin, shift;
+  int wrap;           // wrap split of the shifted heads' last group (kNoWrapSplit: none)
   float scale_log2;   // scale * log2(e)
   float scale;
   unsigned int* err;
@@ -132,10 +133,11 @@ __global__ void __launch_bounds__(32 * (kDkdvEwWarps + 3), 1)
   const int T = (p.N + kTileRows - 1) / kTileRows;
   const int n_tiles = p.B * p.kvh_count * T;
   auto head_shift = [&](int hq) { return hq >= p.shift_head_begin ? p.shift : 0; };
+  auto head_wrap = [&](int hq) { return hq >= p.shift_head_begin ? p.wrap : kNoWrapSplit; };
   auto pairs_of = [&](int kvh, int t0) {
     int total = 0;
     for (int hq = kvh * rep; hq < (kvh + 1) * rep; ++hq)
-      total += kv_tile_qtiles(t0, head_shift(hq), p.N, p.G).count();
+      total += kv_tile_qtiles(t0, head_shift(hq), p.N, p.G, head_wrap(hq)).count();
     return total;
   };
 
@@ -212,7 +214,7 @@ __global__ void __launch_bounds__(32 * (kDkdvEwWarps + 3), 1)
         }
         for (int hq = kvh * rep; ok && hq < (kvh + 1) * rep; ++hq) {
           const int sh = head_shift(hq);
-          const QTileRanges qr = kv_tile_qtiles(t0, sh, p.N, p.G);
+          const QTileRanges qr = kv_tile_qtiles(t0, sh, p.N, p.G, head_wrap(hq));
           const float* lse_row = p.lse2 + (static_cast<size_t>(b) * p.Hq + hq) * p.N;
           const float* d_row = p.dvec + (static_cast<size_t>(b) * p.Hq + hq) * p.N;
           for (int i = 0; i < qr.count(); ++i, ++n) {
@@ -310,10 +312,10 @@ __global__ void __launch_bounds__(32 * (kDkdvEwWarps + 3), 1)
         if (p.ds) {
           for (int hq = kvh * rep; ok && hq < (kvh + 1) * rep; ++hq) {
             const int sh = head_shift(hq);
-            const QTileRanges qr = kv_tile_qtiles(t0, sh, p.N, p.G);
+            const QTileRanges qr = kv_tile_qtiles(t0, sh, p.N, p.G, head_wrap(hq));
             for (int i = 0; ok && i < qr.count(); ++i) {
               const int qt = qr.at(i);
-              const KvSpan sp = qtile_kv_span(qt, sh, p.N, p.G);
+              const KvSpan sp = qtile_kv_span(qt, sh, p.N, p.G, head_wrap(hq));
               int idx = t0 / kTileRows - sp.first;
               if (idx < 0) idx += T;
               ok = hand_over([&] {
@@ -366,9 +368,9 @@ __global__ void __launch_bounds__(32 * (kDkdvEwWarps + 3), 1)
       const bool kv_valid = t < p.N;
       for (int hq = kvh * rep; ok && hq < (kvh + 1) * rep; ++hq) {
         const int sh = head_shift(hq);
-        const QTileRanges qr = kv_tile_qtiles(t0, sh, p.N, p.G);
+        const QTileRanges qr = kv_tile_qtiles(t0, sh, p.N, p.G, head_wrap(hq));
         const int r_k = kv_valid ? (t - sh < 0 ? t - sh + p.N : t - sh) : 0;
-        const int ge_k = group_end(r_k, p.G);
+        const int ge_k = group_end(r_k, p.G, head_wrap(hq));
         for (int i = 0; i < qr.count(); ++i, ++n) {
           const int st = n & 1;
           const int q0 = qr.at(i) * kTileRows + W * grp;

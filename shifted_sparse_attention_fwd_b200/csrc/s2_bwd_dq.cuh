@@ -67,8 +67,9 @@ __global__ void __launch_bounds__(320, 1)
   query_tile_coords(blockIdx.x, p.B, p.Hq, p.N, p.G, b, h, qt);
   const int R0 = qt * kTileRows;
   const int shift_h = h >= p.shift_head_begin ? p.shift : 0;
+  const int wrap_h = h >= p.shift_head_begin ? p.wrap : kNoWrapSplit;
   const int kvh = h / (p.Hq / p.Hkv);
-  const int kt_begin = group_begin(R0, p.G) / kTileRows;
+  const int kt_begin = group_begin(R0, p.G, wrap_h) / kTileRows;
   const int n_kv = qt - kt_begin + 1;
 
   if (warp == 8 && lane == 0) {
@@ -186,7 +187,7 @@ __global__ void __launch_bounds__(320, 1)
     const int row = (warp % 4) * 32 + lane;
     const int r = R0 + row;
     const bool row_valid = r < p.N;
-    const int lo = row_valid ? group_begin(r, p.G) : kt_begin * kTileRows;
+    const int lo = row_valid ? group_begin(r, p.G, wrap_h) : kt_begin * kTileRows;
     const int hi = row_valid ? r : kt_begin * kTileRows;
     const long long tt = static_cast<long long>(r) + shift_h;
     const int t = row_valid ? static_cast<int>(tt >= p.N ? tt - p.N : tt) : 0;

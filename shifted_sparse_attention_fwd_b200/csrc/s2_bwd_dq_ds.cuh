@@ -69,6 +69,7 @@ __global__ void __launch_bounds__(192, 1)
   const int T = (p.N + kTileRows - 1) / kTileRows;
   const int units = p.B * p.kvh_count * rep * T;
   auto head_shift = [&](int hq) { return hq >= p.shift_head_begin ? p.shift : 0; };
+  auto head_wrap = [&](int hq) { return hq >= p.shift_head_begin ? p.wrap : kNoWrapSplit; };
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < L::kStages; ++s) {
@@ -109,7 +110,7 @@ __global__ void __launch_bounds__(192, 1)
         if (u < 0) break;
         int b, hq, qt;
         dq_ds_tile(p, u, b, hq, qt);
-        const KvSpan sp = qtile_kv_span(qt, head_shift(hq), p.N, p.G);
+        const KvSpan sp = qtile_kv_span(qt, head_shift(hq), p.N, p.G, head_wrap(hq));
         const __nv_bfloat16* ds0 = ds_slot_ptr(p, b, hq, p.slots.base(qt));
         const int kvh = hq / rep;
         for (int i = 0; i < sp.count; ++i, ++it) {
@@ -147,7 +148,7 @@ __global__ void __launch_bounds__(192, 1)
         if (u < 0) break;
         int b, hq, qt;
         dq_ds_tile(p, u, b, hq, qt);
-        const int count = qtile_kv_span(qt, head_shift(hq), p.N, p.G).count;
+        const int count = qtile_kv_span(qt, head_shift(hq), p.N, p.G, head_wrap(hq)).count;
         const int a = n & 1;
         if (n >= 2 && !wait_bar(bar(L::B_ACCE + a), ((n >> 1) - 1) & 1, ctx, 2)) { ok = false; break; }
         tc_fence_after();

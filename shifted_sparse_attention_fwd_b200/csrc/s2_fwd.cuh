@@ -41,6 +41,7 @@ struct FwdParams {
   long long o_sb, o_st;   // element strides of O's batch and token axes
   float* lse;
   int B, Hq, Hkv, N, G, shift_head_begin, shift;
+  int wrap;           // wrap split of the shifted heads' last group (kNoWrapSplit: none)
   float scale_log2;   // scale * log2(e)
   unsigned int* err;
   unsigned long long timeout_ns;
@@ -89,7 +90,7 @@ __device__ __forceinline__ float max_tree128(const float (&s)[128]) {
 
 // One work unit: query tiles 2*pair and 2*pair + 1 of (b, h) and the key tiles they see.
 struct FwdUnit {
-  int b, h, kvh, shift_h;
+  int b, h, kvh, shift_h, wrap_h;
   int qt[2], kb[2], ke[2];
   bool tv[2];
   int kv_lo, n_kv;
@@ -104,13 +105,14 @@ __device__ __forceinline__ FwdUnit fwd_unit(const FwdParams& p, int unit) {
   query_pair_coords_chunked(unit, p.B, p.Hq, p.N, p.G, kL2Chunk, u.b, u.h, pair);
   const int nqt = (p.N + kTileRows - 1) / kTileRows;
   u.shift_h = u.h >= p.shift_head_begin ? p.shift : 0;
+  u.wrap_h = u.h >= p.shift_head_begin ? p.wrap : kNoWrapSplit;
   u.kvh = u.h / (p.Hq / p.Hkv);
   // Tile t = 2*pair + t sees key tiles [kb[t], ke[t]]; tile 0 always exists, tile 1 may not.
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
     u.qt[t] = 2 * pair + t;
     u.tv[t] = u.qt[t] < nqt;
-    u.kb[t] = u.tv[t] ? group_begin(u.qt[t] * kTileRows, p.G) / kTileRows : 0;
+    u.kb[t] = u.tv[t] ? group_begin(u.qt[t] * kTileRows, p.G, u.wrap_h) / kTileRows : 0;
     u.ke[t] = u.qt[t];
   }
   u.kv_lo = u.kb[0];
@@ -306,7 +308,7 @@ __global__ void __launch_bounds__(320, 1)
       if (!u.tv[wg]) continue;
       const int r = u.qt[wg] * kTileRows + row;
       const bool row_valid = r < p.N;
-      const int lo = row_valid ? group_begin(r, p.G) : u.kb[wg] * kTileRows;
+      const int lo = row_valid ? group_begin(r, p.G, u.wrap_h) : u.kb[wg] * kTileRows;
       const int hi = row_valid ? r : u.kb[wg] * kTileRows;
       float m_run = -INFINITY, l_run = 0.f;
       for (int kt = u.kb[wg], cnt = 0; kt <= u.ke[wg]; ++kt, ++cnt, ++s_cnt) {

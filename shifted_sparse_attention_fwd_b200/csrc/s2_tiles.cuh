@@ -53,9 +53,20 @@ __host__ __device__ inline TileRuns original_tile_runs(int t0, int shift, int N)
   return rolled_tile_runs(t0, inv, N);
 }
 
-// First rolled row of the group containing rolled row r, and one past its last row.
-__host__ __device__ inline int group_begin(int r, int G) { return (r / G) * G; }
-__host__ __device__ inline int group_end(int r, int G) { return (r / G + 1) * G; }
+// No split of the wrap group (see group_begin).
+constexpr int kNoWrapSplit = 0x7fffffff;
+
+// First rolled row of the group containing rolled row r, and one past its last row. With a
+// wrap split W < N (the pages' Variant 2, Table 8: in the shifted heads the tokens the roll
+// wrapped around, rolled rows [W, N) with W = N - shift, form their own group), the last
+// group [N - G, N) is two groups, [N - G, W) and [W, N).
+__host__ __device__ inline int group_begin(int r, int G, int W = kNoWrapSplit) {
+  return r >= W ? W : (r / G) * G;
+}
+__host__ __device__ inline int group_end(int r, int G, int W = kNoWrapSplit) {
+  const int e = (r / G + 1) * G;
+  return (r < W && e > W) ? W : e;
+}
 
 // Query tiles (rolled, 128 rows) of a query head with roll `sh` that can see the original
 // kv rows [t0, t0 + 128): up to two disjoint index ranges, [r0a, r0b] then [r1a, r1b].
@@ -71,15 +82,16 @@ struct QTileRanges {
   }
 };
 
-__host__ __device__ inline QTileRanges kv_tile_qtiles(int t0, int sh, int N, int G) {
+__host__ __device__ inline QTileRanges kv_tile_qtiles(int t0, int sh, int N, int G,
+                                                      int W = kNoWrapSplit) {
   const TileRuns tr = original_tile_runs(t0, sh, N);
   // Run A: rolled rows [start, start + first) -> query rows [start, end of group).
   const int a0 = tr.start / kTileRows;
-  const int a1 = (group_end(tr.start + tr.first - 1, G) - 1) / kTileRows;
+  const int a1 = (group_end(tr.start + tr.first - 1, G, W) - 1) / kTileRows;
   QTileRanges q;
   if (tr.valid > tr.first) {
     // Run B: rolled rows [0, valid - first) -> query rows [0, end of that group).
-    const int b1 = (group_end(tr.valid - tr.first - 1, G) - 1) / kTileRows;
+    const int b1 = (group_end(tr.valid - tr.first - 1, G, W) - 1) / kTileRows;
     if (b1 + 1 >= a0) {
       q.r0a = 0; q.r0b = a1 > b1 ? a1 : b1; q.r1a = 1; q.r1b = 0;
     } else {
@@ -98,11 +110,12 @@ __host__ __device__ inline QTileRanges kv_tile_qtiles(int t0, int sh, int N, int
 struct KvSpan {
   int first, count;
 };
-__host__ __device__ inline KvSpan qtile_kv_span(int qt, int sh, int N, int G) {
+__host__ __device__ inline KvSpan qtile_kv_span(int qt, int sh, int N, int G,
+                                               int W = kNoWrapSplit) {
   const int T = (N + kTileRows - 1) / kTileRows;
   const int r0 = qt * kTileRows;
   const int last = r0 + kTileRows - 1 < N - 1 ? r0 + kTileRows - 1 : N - 1;
-  const int gb = group_begin(r0, G);
+  const int gb = group_begin(r0, G, W);
   const int len = last - gb + 1;
   const long long o = static_cast<long long>(gb) + sh;
   const int o0 = static_cast<int>(o >= N ? o - N : o);
@@ -135,11 +148,12 @@ struct DsSlots {
     return static_cast<long long>(qt) * stride;
   }
 };
-inline DsSlots ds_slots(int N, int G, int shifted_heads, int shift) {
+inline DsSlots ds_slots(int N, int G, int shifted_heads, int shift, int W = kNoWrapSplit) {
   DsSlots d;
   const int T = (N + kTileRows - 1) / kTileRows;
   const int sh = shifted_heads ? shift : 0;
-  d.aligned = (G % kTileRows == 0 && sh % kTileRows == 0) ? 1 : 0;
+  const int w = shifted_heads ? W : kNoWrapSplit;
+  d.aligned = (G % kTileRows == 0 && sh % kTileRows == 0 && w >= N) ? 1 : 0;
   d.gt = G / kTileRows;
   d.stride = 0;
   if (d.aligned) {
@@ -147,7 +161,7 @@ inline DsSlots ds_slots(int N, int G, int shifted_heads, int shift) {
   } else {
     for (int qt = 0; qt < T; ++qt) {
       const int c0 = qtile_kv_span(qt, 0, N, G).count;
-      const int c1 = qtile_kv_span(qt, sh, N, G).count;
+      const int c1 = qtile_kv_span(qt, sh, N, G, w).count;
       const int c = c0 > c1 ? c0 : c1;
       d.stride = c > d.stride ? c : d.stride;
     }

@@ -151,6 +151,7 @@ enum TensorId { T_Q = 0, T_K, T_V, T_O, T_DO, T_DQ, T_DK, T_DV, T_COUNT };
 
 struct Shape {
   int B, Hq, Hkv, N, d, G, shb, shift;
+  int wrap;   // the shifted heads' wrap split (Variant 2), or s2::kNoWrapSplit
   long long sb[T_COUNT], st[T_COUNT];
   int heads(int t) const { return (t == T_K || t == T_V || t == T_DK || t == T_DV) ? Hkv : Hq; }
   void set_contiguous() {
@@ -170,7 +171,9 @@ unsigned int* ws_sched(const void* workspace, const Shape& sh) {
                                          2 * ws_half(sh.B, sh.Hq, sh.N));
 }
 
-s2::DsSlots ds_layout(const Shape& sh) { return s2::ds_slots(sh.N, sh.G, sh.shb < sh.Hq, sh.shift); }
+s2::DsSlots ds_layout(const Shape& sh) {
+  return s2::ds_slots(sh.N, sh.G, sh.shb < sh.Hq, sh.shift, sh.wrap);
+}
 size_t ds_bytes_per_kv_head(const Shape& sh) {
   const s2::DsSlots sl = ds_layout(sh);
   return static_cast<size_t>(sh.B) * (sh.Hq / sh.Hkv) * static_cast<size_t>(sl.per_head) *
@@ -187,7 +190,7 @@ int ds_heads_per_pass(const Shape& sh, size_t bytes) {
 
 // Validation shared by every attention entry point (see s2attn.h, "Errors").
 s2attn_status check_shape(int B, int Hq, int Hkv, int N, int d, int G, float scale,
-                          int shift_head_begin, long long shift, Shape& out) {
+                          int shift_head_begin, long long shift, Shape& out, int flags = 0) {
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || N <= 0 || d <= 0 || G <= 0) return S2ATTN_ERR_INVALID_ARG;
   if (Hq % Hkv != 0 || N % G != 0 || G % 2 != 0) return S2ATTN_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !std::isfinite(scale)) return S2ATTN_ERR_INVALID_ARG;
@@ -201,7 +204,14 @@ s2attn_status check_shape(int B, int Hq, int Hkv, int N, int d, int G, float sca
   if (s % 8 != 0) return S2ATTN_ERR_UNSUPPORTED;
   const long long rows = static_cast<long long>(B) * (Hq > Hkv ? Hq : Hkv) * ((N + 127) / 128);
   if (rows >= (1ll << 31)) return S2ATTN_ERR_UNSUPPORTED;
-  out = Shape{B, Hq, Hkv, N, d, G, shift_head_begin, static_cast<int>(s), {}, {}};
+  if (flags & ~S2ATTN_FLAG_WRAP_OWN_GROUP) return S2ATTN_ERR_INVALID_ARG;
+  int wrap = s2::kNoWrapSplit;
+  if (flags & S2ATTN_FLAG_WRAP_OWN_GROUP) {
+    // the wrap group exists when some head is rolled by 0 < shift < G
+    if (shift_head_begin >= Hq || s <= 0 || s >= G) return S2ATTN_ERR_INVALID_ARG;
+    wrap = N - static_cast<int>(s);
+  }
+  out = Shape{B, Hq, Hkv, N, d, G, shift_head_begin, static_cast<int>(s), wrap, {}, {}};
   out.set_contiguous();
   return S2ATTN_OK;
 }
@@ -222,6 +232,7 @@ s2attn_status launch_fwd(const Shape& sh, const void* q, const void* k, const vo
   p.lse = lse;
   p.B = sh.B; p.Hq = sh.Hq; p.Hkv = sh.Hkv; p.N = sh.N; p.G = sh.G;
   p.shift_head_begin = sh.shb; p.shift = sh.shift;
+  p.wrap = sh.wrap;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.err = err;
   p.timeout_ns = g_timeout_ns.load();
@@ -244,6 +255,7 @@ s2::BwdParams bwd_params(const Shape& sh, float scale, const void* workspace, vo
   p.dv = static_cast<__nv_bfloat16*>(dv);
   p.B = sh.B; p.Hq = sh.Hq; p.Hkv = sh.Hkv; p.N = sh.N; p.G = sh.G;
   p.shift_head_begin = sh.shb; p.shift = sh.shift;
+  p.wrap = sh.wrap;
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.err = err;
@@ -432,15 +444,15 @@ void s2attn_set_wait_timeout_ns(unsigned long long ns) {
   g_timeout_ns.store(ns == 0 ? kDefaultTimeoutNs : ns);
 }
 
-s2attn_status s2attn_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse,
+s2attn_status s2attn_fwd_general(const void* q, const void* k, const void* v, void* o, float* lse,
                                  int B, int Hq, int Hkv, int N, int d, int G, float scale,
-                                 int shift_head_begin, int shift, const long long* strides,
-                                 void* stream) {
+                                 int shift_head_begin, int shift, int flags,
+                                 const long long* strides, void* stream) {
   if (!q || !k || !v || !o || !lse) return S2ATTN_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return S2ATTN_ERR_INVALID_ARG;
   Shape sh;
-  s2attn_status s = check_shape(B, Hq, Hkv, N, d, G, scale, shift_head_begin, shift, sh);
+  s2attn_status s = check_shape(B, Hq, Hkv, N, d, G, scale, shift_head_begin, shift, sh, flags);
   if (s != S2ATTN_OK) return s;
   if (strides) {
     static const int ids[4] = {T_Q, T_K, T_V, T_O};
@@ -459,8 +471,8 @@ s2attn_status s2attn_fwd_ex(const void* q, const void* k, const void* v, void* o
                             int B, int Hq, int Hkv, int N, int d, int G, float scale,
                             int shift_head_begin, int shift, void* stream) {
   // null strides: contiguous tensors
-  return s2attn_fwd_strided(q, k, v, o, lse, B, Hq, Hkv, N, d, G, scale, shift_head_begin, shift,
-                            nullptr, stream);
+  return s2attn_fwd_general(q, k, v, o, lse, B, Hq, Hkv, N, d, G, scale, shift_head_begin, shift,
+                            0, nullptr, stream);
 }
 
 s2attn_status s2attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -475,10 +487,12 @@ size_t s2attn_bwd_workspace_size(int B, int Hq, int N) {
   return ws_min_bytes(B, Hq, N);
 }
 
-size_t s2attn_bwd_workspace_size_ex(int B, int Hq, int Hkv, int N, int d, int G,
-                                    int shift_head_begin, int shift, size_t cap_bytes) {
+size_t s2attn_bwd_workspace_size_general(int B, int Hq, int Hkv, int N, int d, int G,
+                                         int shift_head_begin, int shift, int flags,
+                                         size_t cap_bytes) {
   Shape sh;
-  if (check_shape(B, Hq, Hkv, N, d, G, 1.0f, shift_head_begin, shift, sh) != S2ATTN_OK) return 0;
+  if (check_shape(B, Hq, Hkv, N, d, G, 1.0f, shift_head_begin, shift, sh, flags) != S2ATTN_OK)
+    return 0;
   const size_t base = ws_min_bytes(B, Hq, N);
   const size_t per = ds_bytes_per_kv_head(sh);
   size_t k = static_cast<size_t>(Hkv);
@@ -490,6 +504,12 @@ size_t s2attn_bwd_workspace_size_ex(int B, int Hq, int Hkv, int N, int d, int G,
   return base + k * per;
 }
 
+size_t s2attn_bwd_workspace_size_ex(int B, int Hq, int Hkv, int N, int d, int G,
+                                    int shift_head_begin, int shift, size_t cap_bytes) {
+  return s2attn_bwd_workspace_size_general(B, Hq, Hkv, N, d, G, shift_head_begin, shift, 0,
+                                           cap_bytes);
+}
+
 s2attn_status s2attn_bwd_preprocess(const void* o, const float* lse, const void* dO, int B,
                                     int Hq, int N, int d, void* workspace,
                                     size_t workspace_bytes, void* stream) {
@@ -499,7 +519,7 @@ s2attn_status s2attn_bwd_preprocess(const void* o, const float* lse, const void*
   if (d != 64 && d != 128) return S2ATTN_ERR_UNSUPPORTED;
   if (N >= (1 << 30) || static_cast<long long>(B) * Hq * ((N + 127) / 128) >= (1ll << 31))
     return S2ATTN_ERR_UNSUPPORTED;
-  Shape sh{B, Hq, Hq, N, d, N, Hq, 0, {}, {}};
+  Shape sh{B, Hq, Hq, N, d, N, Hq, 0, s2::kNoWrapSplit, {}, {}};
   sh.set_contiguous();
   s2attn_status s = check_workspace(sh, workspace, workspace_bytes);
   if (s != S2ATTN_OK) return s;
@@ -591,17 +611,18 @@ s2attn_status s2attn_bwd_dq_ds(const void* k, void* dq, int B, int Hq, int Hkv, 
                     num_sms);
 }
 
-s2attn_status s2attn_bwd_strided(const void* q, const void* k, const void* v, const void* o,
+s2attn_status s2attn_bwd_general(const void* q, const void* k, const void* v, const void* o,
                                  const float* lse, const void* dO, void* dq, void* dk, void* dv,
                                  int B, int Hq, int Hkv, int N, int d, int G, float scale,
-                                 int shift_head_begin, int shift, const long long* strides,
-                                 void* workspace, size_t workspace_bytes, void* stream) {
+                                 int shift_head_begin, int shift, int flags,
+                                 const long long* strides, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
   if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv) return S2ATTN_ERR_INVALID_ARG;
   const void* ptrs[] = {q, k, v, o, lse, dO, dq, dk, dv};
   for (const void* ptr : ptrs)
     if (!aligned16(ptr)) return S2ATTN_ERR_INVALID_ARG;
   Shape sh;
-  s2attn_status s = check_shape(B, Hq, Hkv, N, d, G, scale, shift_head_begin, shift, sh);
+  s2attn_status s = check_shape(B, Hq, Hkv, N, d, G, scale, shift_head_begin, shift, sh, flags);
   if (s != S2ATTN_OK) return s;
   if (strides) {
     static const int ids[8] = {T_Q, T_K, T_V, T_O, T_DO, T_DQ, T_DK, T_DV};
@@ -638,8 +659,8 @@ s2attn_status s2attn_bwd_ex(const void* q, const void* k, const void* v, const v
                             int shift_head_begin, int shift, void* workspace,
                             size_t workspace_bytes, void* stream) {
   // null strides: contiguous tensors
-  return s2attn_bwd_strided(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, N, d, G, scale,
-                            shift_head_begin, shift, nullptr, workspace, workspace_bytes, stream);
+  return s2attn_bwd_general(q, k, v, o, lse, dO, dq, dk, dv, B, Hq, Hkv, N, d, G, scale,
+                            shift_head_begin, shift, 0, nullptr, workspace, workspace_bytes, stream);
 }
 
 s2attn_status s2attn_bwd(const void* q, const void* k, const void* v, const void* o,

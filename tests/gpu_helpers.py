@@ -23,7 +23,7 @@ BF16_MEAN_ABS = 2e-3
 LSE_MAX_ABS = 1e-4
 
 
-def _bwd(qd, kd, vd, o, lse, dod, G, scale, shb, shift, mode):
+def _bwd(qd, kd, vd, o, lse, dod, G, scale, shb, shift, mode, flags=0):
     """Backward through one of the library's paths:
     auto        the allocating convenience (dS hand-off, all kv heads in one pass when the
                 default cap allows);
@@ -31,7 +31,7 @@ def _bwd(qd, kd, vd, o, lse, dod, G, scale, shb, shift, mode):
     per_kv_head room for one kv head's dS tiles: one dK/dV + dQ pass per kv head;
     phases      preprocess, s2attn_bwd_dkdv_ds and s2attn_bwd_dq_ds called one by one."""
     if mode == "auto":
-        return s2.bwd(qd, kd, vd, o, lse, dod, G, scale, shb, shift)
+        return s2.bwd(qd, kd, vd, o, lse, dod, G, scale, shb, shift, flags=flags)
     B, N, Hq, d = qd.shape
     Hkv = kd.shape[2]
     shb_ = Hq // 2 if shb is None else shb
@@ -40,26 +40,27 @@ def _bwd(qd, kd, vd, o, lse, dod, G, scale, shb, shift, mode):
         n = s2.s2attn_bwd_workspace_size(B, Hq, N)
     else:
         n = s2.s2attn_bwd_workspace_size_ex(B, Hq, Hkv, N, d, G, shb_, sh_,
-                                            1 if mode == "per_kv_head" else 0)
+                                            1 if mode == "per_kv_head" else 0, flags)
     ws = torch.empty(n, dtype=torch.uint8, device=qd.device)
     dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
     if mode == "phases":
+        assert flags == 0, "the phase entry points compute the default variant"
         s2.s2attn_bwd_preprocess(o, lse, dod, ws)
         s2.s2attn_bwd_dkdv_ds(qd, kd, vd, dod, dk, dv, G, ws, scale, shb_, sh_)
         s2.s2attn_bwd_dq_ds(kd, dq, G, ws, scale, shb_, sh_)
     else:
-        s2.s2attn_bwd(qd, kd, vd, o, lse, dod, dq, dk, dv, G, scale, shb_, sh_, ws)
+        s2.s2attn_bwd(qd, kd, vd, o, lse, dod, dq, dk, dv, G, scale, shb_, sh_, ws, flags=flags)
     return dq, dk, dv
 
 
-def gpu_run(q, k, v, do, G, scale, shb=None, shift=None, backward=True, mode="auto"):
+def gpu_run(q, k, v, do, G, scale, shb=None, shift=None, backward=True, mode="auto", flags=0):
     """Forward (+ backward) of the CUDA path on bf16 CPU inputs; returns CPU tensors."""
     dev = torch.device("cuda")
     qd, kd, vd, dod = (x.to(dev) for x in (q, k, v, do))
-    o, lse = s2.fwd(qd, kd, vd, G, scale, shb, shift)
+    o, lse = s2.fwd(qd, kd, vd, G, scale, shb, shift, flags=flags)
     out = {"o": o, "lse": lse}
     if backward:
-        dq, dk, dv = _bwd(qd, kd, vd, o, lse, dod, G, scale, shb, shift, mode)
+        dq, dk, dv = _bwd(qd, kd, vd, o, lse, dod, G, scale, shb, shift, mode, flags)
         out.update(dq=dq, dk=dk, dv=dv)
     torch.cuda.synchronize()
     st, code = s2.s2attn_get_device_error()
@@ -67,12 +68,14 @@ def gpu_run(q, k, v, do, G, scale, shb=None, shift=None, backward=True, mode="au
     return {k_: v_.cpu() for k_, v_ in out.items()}
 
 
-def oracle_run(q, k, v, do, G, scale, shb=None, shift=None, backward=True):
+def oracle_run(q, k, v, do, G, scale, shb=None, shift=None, backward=True, flags=0):
     qf, kf, vf, dof = (to_f64(x) for x in (q, k, v, do))
-    o, lse = orc.s2attn_forward(qf, kf, vf, G, scale, shb, shift)
+    wrap = bool(flags & s2.S2ATTN_FLAG_WRAP_OWN_GROUP)
+    o, lse = orc.s2attn_forward(qf, kf, vf, G, scale, shb, shift, wrap_own_group=wrap)
     out = {"o": o, "lse": lse}
     if backward:
-        dq, dk, dv = orc.s2attn_backward(qf, kf, vf, dof, G, scale, shb, shift)
+        dq, dk, dv = orc.s2attn_backward(qf, kf, vf, dof, G, scale, shb, shift,
+                                         wrap_own_group=wrap)
         out.update(dq=dq, dk=dk, dv=dv)
     return out
 
@@ -103,11 +106,11 @@ def assert_close(name, gpu, ref):
 
 
 def check_case(B, Hq, Hkv, N, G, d, seed, shb=None, shift=None, q_gain=1.0, scale=None,
-               backward=True, mode="auto"):
+               backward=True, mode="auto", flags=0):
     q, k, v, do = make_inputs(B, Hq, Hkv, N, d, seed, q_gain)
     scale = d ** -0.5 if scale is None else scale
-    g = gpu_run(q, k, v, do, G, scale, shb, shift, backward, mode)
-    r = oracle_run(q, k, v, do, G, scale, shb, shift, backward)
+    g = gpu_run(q, k, v, do, G, scale, shb, shift, backward, mode, flags)
+    r = oracle_run(q, k, v, do, G, scale, shb, shift, backward, flags)
     report = {}
     for name in g:
         gg, rr = g[name], r[name]

@@ -129,8 +129,8 @@ void rolled_runs(int r0, int shift, int N, int* o) {
   s2::TileRuns t = s2::rolled_tile_runs(r0, shift, N); o[0]=t.valid; o[1]=t.first; o[2]=t.start; }
 void original_runs(int t0, int shift, int N, int* o) {
   s2::TileRuns t = s2::original_tile_runs(t0, shift, N); o[0]=t.valid; o[1]=t.first; o[2]=t.start; }
-int qtiles(int t0, int sh, int N, int G, int* o) {
-  s2::QTileRanges q = s2::kv_tile_qtiles(t0, sh, N, G);
+int qtiles(int t0, int sh, int N, int G, int W, int* o) {
+  s2::QTileRanges q = s2::kv_tile_qtiles(t0, sh, N, G, W);
   int n = q.count(); for (int i = 0; i < n; ++i) o[i] = q.at(i); return n; }
 void qcoords(int bid, int B, int Hq, int N, int G, int* o) {
   s2::query_tile_coords(bid, B, Hq, N, G, o[0], o[1], o[2]); }
@@ -145,10 +145,10 @@ void paircoords_chunked(int bid, int B, int Hq, int N, int G, int chunk, int* o)
 void kvcoords_chunked(int bid, int B, int Hq, int Hkv, int N, int G, int shb, int sh, int chunk,
                       int* o) {
   s2::kv_tile_coords_chunked(bid, B, Hq, Hkv, N, G, shb, sh, chunk, o[0], o[1], o[2]); }
-void kvspan(int qt, int sh, int N, int G, int* o) {
-  s2::KvSpan s = s2::qtile_kv_span(qt, sh, N, G); o[0] = s.first; o[1] = s.count; }
-long long dsslots(int N, int G, int shifted, int shift, int qt) {
-  s2::DsSlots d = s2::ds_slots(N, G, shifted, shift);
+void kvspan(int qt, int sh, int N, int G, int W, int* o) {
+  s2::KvSpan s = s2::qtile_kv_span(qt, sh, N, G, W); o[0] = s.first; o[1] = s.count; }
+long long dsslots(int N, int G, int shifted, int shift, int W, int qt) {
+  s2::DsSlots d = s2::ds_slots(N, G, shifted, shift, W);
   return qt < 0 ? d.per_head : d.base(qt); }
 }
 """
@@ -163,6 +163,9 @@ def shim(tmp_path_factory):
     subprocess.run(["g++", "-O1", "-shared", "-fPIC", "-std=c++17", "-I", CSRC, str(src), "-o",
                     str(so)], check=True)
     return ctypes.CDLL(str(so))
+
+
+NOWRAP = 0x7FFFFFFF   # no wrap split (the default variant)
 
 
 def call4(fn, *args):
@@ -207,7 +210,7 @@ def test_kv_tile_query_tiles_exact(shim, N, G, shift):
     rolled_of[tok] = np.arange(N)
     out = (ctypes.c_int * 4096)()
     for t0 in range(0, N, 128):
-        n = shim.qtiles(t0, shift, N, G, out)
+        n = shim.qtiles(t0, shift, N, G, NOWRAP, out)
         got = list(out[:n])
         assert len(set(got)) == len(got)
         want = set()
@@ -271,7 +274,7 @@ def test_qtile_kv_span_exact(shim, N, G, shift):
     nt = (N + 127) // 128
     for sh in {0, shift}:
         for qt in range(nt) if N <= 8192 else list(range(0, nt, 37)) + [nt - 1]:
-            first, count = call4(shim.kvspan, qt, sh, N, G)[:2]
+            first, count = call4(shim.kvspan, qt, sh, N, G, NOWRAP)[:2]
             got = [(first + i) % nt for i in range(count)]
             assert len(set(got)) == count
             r0, last = qt * 128, min(qt * 128 + 127, N - 1)
@@ -286,25 +289,80 @@ def test_ds_slots_match_the_dkdv_pairs(shim, N, G, shift):
     the slots of one head are distinct and inside per_head."""
     nt = (N + 127) // 128
     shim.dsslots.restype = ctypes.c_longlong
-    per_head = shim.dsslots(N, G, 1, shift, -1)
+    per_head = shim.dsslots(N, G, 1, shift, NOWRAP, -1)
     out = (ctypes.c_int * 4096)()
     for sh in {0, shift}:
         visited = set()
         for t in range(nt):
-            n = shim.qtiles(t * 128, sh, N, G, out)
+            n = shim.qtiles(t * 128, sh, N, G, NOWRAP, out)
             visited.update((qt, t) for qt in out[:n])
         slots = set()
         for qt in range(nt):
-            first, count = call4(shim.kvspan, qt, sh, N, G)[:2]
-            base = shim.dsslots(N, G, 1, shift, qt)
+            first, count = call4(shim.kvspan, qt, sh, N, G, NOWRAP)[:2]
+            base = shim.dsslots(N, G, 1, shift, NOWRAP, qt)
             for i in range(count):
                 assert (qt, (first + i) % nt) in visited
                 slots.add(base + i)
             assert base + count <= per_head
-        assert len(slots) == sum(call4(shim.kvspan, qt, sh, N, G)[1] for qt in range(nt))
+        assert len(slots) == sum(call4(shim.kvspan, qt, sh, N, G, NOWRAP)[1] for qt in range(nt))
     if G % 128 == 0 and shift % 128 == 0:
         gt = G // 128
         assert per_head == (N // G) * gt * (gt + 1) // 2
+
+
+V2_CASES = [(256, 64, 32), (8192, 2048, 1024), (320, 64, 32), (384, 192, 96), (96, 32, 16),
+            (640, 128, 64), (2048, 512, 256), (448, 64, 8), (96, 96, 88), (1024, 256, 128),
+            (512, 128, 40)]
+
+
+def _v2_group(r, N, G, W):
+    """Rolled rows of the causal group holding rolled row r when the wrapped tokens (rolled
+    rows [W, N), W = N - shift) form their own group (Table 8, Variant 2)."""
+    if r >= W:
+        return W, N
+    return (r // G) * G, min((r // G + 1) * G, W)
+
+
+@pytest.mark.parametrize("N,G,shift", V2_CASES)
+def test_variant2_tile_sets_exact(shim, N, G, shift):
+    """Brute force with the wrap split: the query tiles each kv tile visits, the kv tiles each
+    query tile reads, and that the two agree in both directions (every dS tile the dK/dV kernel
+    hands off lands inside the reading tile's span, and every span entry is written)."""
+    W = N - shift
+    nt = (N + 127) // 128
+    tok = orc.rolled_token_index(N, G, shift).reshape(-1)
+    rolled_of = np.empty(N, dtype=np.int64)
+    rolled_of[tok] = np.arange(N)
+    out = (ctypes.c_int * 4096)()
+    visited = set()
+    for t in range(nt):
+        n = shim.qtiles(t * 128, shift, N, G, W, out)
+        got = set(out[:n])
+        assert len(got) == n
+        want = set()
+        for tk in range(t * 128, min(t * 128 + 128, N)):
+            rk = rolled_of[tk]
+            want.update(range(rk // 128, (_v2_group(rk, N, G, W)[1] - 1) // 128 + 1))
+        assert got == want
+        visited.update((qt, t) for qt in got)
+    shim.dsslots.restype = ctypes.c_longlong
+    per_head = shim.dsslots(N, G, 1, shift, W, -1)
+    read, slots = set(), set()
+    for qt in range(nt):
+        first, count = call4(shim.kvspan, qt, shift, N, G, W)[:2]
+        got = [(first + i) % nt for i in range(count)]
+        assert len(set(got)) == count
+        r0, last = qt * 128, min(qt * 128 + 127, N - 1)
+        gb = _v2_group(r0, N, G, W)[0]
+        assert set(got) == {((r + shift) % N) // 128 for r in range(gb, last + 1)}
+        read.update((qt, t) for t in got)
+        base = shim.dsslots(N, G, 1, shift, W, qt)
+        assert base + count <= per_head
+        slots.update(base + i for i in range(count))
+    assert read == visited
+    assert len(slots) == len(read)
+    # the default variant's slot layout holds at least as many tiles per head
+    assert per_head >= shim.dsslots(N, G, 1, shift, NOWRAP, -1) or G % 128 or shift % 128
 
 
 def test_workspace_size_ex(lib):
@@ -377,7 +435,7 @@ def test_chunked_kv_tile_order_is_a_permutation(shim, B, Hq, Hkv, N, G, shb, sh,
     assert set(order) == {(b, k, t) for b in range(B) for k in range(Hkv) for t in range(nt)}
 
 
-def test_strided_entries_reject(lib):
+def test_general_entries_reject(lib):
     """Stride validation happens on the host, before anything is launched."""
     f = ctypes.c_float(0.125)
     LL = ctypes.c_longlong
@@ -390,9 +448,15 @@ def test_strided_entries_reject(lib):
     ]
     for st in bad_cases:
         arr = (LL * 8)(*st)
-        assert lib.s2attn_fwd_strided(*ok_args, arr, None) == 1
+        assert lib.s2attn_fwd_general(*ok_args, 0, arr, None) == 1
     ws = 0x100000
     need = lib.s2attn_bwd_workspace_size(2, 4, 256)
     arr = (LL * 16)(*([4 * 64 * 3, 4 * 64 - 8] * 8))
-    assert lib.s2attn_bwd_strided(*([A] * 9), 2, 4, 4, 256, 64, 64, f, 2, 32, arr, ws, need,
+    assert lib.s2attn_bwd_general(*([A] * 9), 2, 4, 4, 256, 64, 64, f, 2, 32, 0, arr, ws, need,
                                   None) == 1
+    # option flags: unknown bits, and Variant 2 without a rolled head or with shift 0
+    assert lib.s2attn_fwd_general(*ok_args, 2, None, None) == 1
+    no_roll = [A] * 5 + [2, 4, 4, 256, 64, 64, f, 4, 32]
+    assert lib.s2attn_fwd_general(*no_roll, 1, None, None) == 1
+    zero_shift = [A] * 5 + [2, 4, 4, 256, 64, 64, f, 2, 0]
+    assert lib.s2attn_fwd_general(*zero_shift, 1, None, None) == 1
