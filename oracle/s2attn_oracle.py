@@ -36,6 +36,10 @@ Readings where the page is silent (each also listed in the design notes):
     tokens that the roll wrapped around (original tokens 0..shift-1, the last ``shift``
     rolled rows) form their own group instead of sharing the last group with the last
     G - shift tokens; that last group is split at the wrap point into two causal groups.
+  * ``wrap_front_first`` is the page's Variant 3 (Table 8, Figure 6): in the shifted heads
+    the wrapped tokens swap places with the front of the last group, i.e. that group lists
+    original tokens 0..shift-1 first and the last G - shift tokens after them, so its causal
+    order is the original token order; every other group is unchanged.
 
 Everything is float64; inputs are the bf16 values widened exactly.
 """
@@ -151,7 +155,25 @@ def _wrap_splits(B, N, G, shb, shift, wrap_own_group):
     return lambda bg, h: (G - shift) if (h >= shb and bg % ng == ng - 1) else None
 
 
-def s2attn_forward(q, k, v, G, scale, shift_head_begin=None, shift=None, wrap_own_group=False):
+def _swap_wrap_front(x: np.ndarray, N: int, G: int, shb: int, shift: int, enabled: bool,
+                     inverse: bool = False) -> np.ndarray:
+    """Variant 3 on the grouped view x [B*N/G, G, H, ...]: in heads >= shb, the last group of
+    every batch element (rolled rows N-G..N-1: tokens N-G+shift..N-1, then the wrapped tokens
+    0..shift-1) is reordered so the wrapped tokens come first (np.roll by +shift within the
+    group); ``inverse`` puts them back."""
+    if not enabled:
+        return x
+    if not 0 < shift < G:
+        raise ValueError("the wrap group exists for 0 < shift < G")
+    out = x.copy()
+    ng = N // G
+    last = slice(ng - 1, None, ng)
+    out[last, :, shb:] = np.roll(x[last, :, shb:], -shift if inverse else shift, axis=1)
+    return out
+
+
+def s2attn_forward(q, k, v, G, scale, shift_head_begin=None, shift=None, wrap_own_group=False,
+                   wrap_front_first=False):
     """S²-Attn forward. q [B,N,Hq,d], k, v [B,N,Hkv,d] float64.
 
     Returns o [B,N,Hq,d] and lse [B,Hq,N], both in original token order.
@@ -159,14 +181,19 @@ def s2attn_forward(q, k, v, G, scale, shift_head_begin=None, shift=None, wrap_ow
     B, N, Hq, d = q.shape
     if N % G != 0:
         raise ValueError("the view into groups needs G to divide N")
+    if wrap_own_group and wrap_front_first:
+        raise ValueError("Variant 2 and Variant 3 are alternatives")
     shb, shift = _defaults(Hq, G, shift_head_begin, shift)
     splits = _wrap_splits(B, N, G, shb, shift, wrap_own_group)
     ke, ve = expand_kv(k, Hq), expand_kv(v, Hq)
     # Key line 1: roll the second chunk of heads by -shift, then view as groups.
-    qr = chunk_roll(q, -shift, shb).reshape(B * N // G, G, Hq, d)
-    kr = chunk_roll(ke, -shift, shb).reshape(B * N // G, G, Hq, d)
-    vr = chunk_roll(ve, -shift, shb).reshape(B * N // G, G, Hq, v.shape[3])
+    sw = lambda x: _swap_wrap_front(x, N, G, shb, shift, wrap_front_first)
+    qr = sw(chunk_roll(q, -shift, shb).reshape(B * N // G, G, Hq, d))
+    kr = sw(chunk_roll(ke, -shift, shb).reshape(B * N // G, G, Hq, d))
+    vr = sw(chunk_roll(ve, -shift, shb).reshape(B * N // G, G, Hq, v.shape[3]))
     o, lse = causal_self_attn(qr, kr, vr, scale, splits)
+    o = _swap_wrap_front(o, N, G, shb, shift, wrap_front_first, inverse=True)
+    lse = _swap_wrap_front(lse, N, G, shb, shift, wrap_front_first, inverse=True)
     # Key line 2: back to [B, N, H, d], roll the second chunk back by +shift.
     o = chunk_roll(o.reshape(B, N, Hq, v.shape[3]), shift, shb)
     lse = chunk_roll(lse.reshape(B, N, Hq), shift, shb)
@@ -174,22 +201,28 @@ def s2attn_forward(q, k, v, G, scale, shift_head_begin=None, shift=None, wrap_ow
 
 
 def s2attn_backward(q, k, v, do, G, scale, shift_head_begin=None, shift=None,
-                    wrap_own_group=False):
+                    wrap_own_group=False, wrap_front_first=False):
     """Gradients of s2attn_forward's o with respect to q, k, v for upstream do [B,N,Hq,d].
 
     Returns dq [B,N,Hq,d], dk [B,N,Hkv,d], dv [B,N,Hkv,d] in original token order.
     """
     B, N, Hq, d = q.shape
     Hkv = k.shape[2]
+    if wrap_own_group and wrap_front_first:
+        raise ValueError("Variant 2 and Variant 3 are alternatives")
     shb, shift = _defaults(Hq, G, shift_head_begin, shift)
     splits = _wrap_splits(B, N, G, shb, shift, wrap_own_group)
     ke, ve = expand_kv(k, Hq), expand_kv(v, Hq)
-    qr = chunk_roll(q, -shift, shb).reshape(B * N // G, G, Hq, d)
-    kr = chunk_roll(ke, -shift, shb).reshape(B * N // G, G, Hq, d)
-    vr = chunk_roll(ve, -shift, shb).reshape(B * N // G, G, Hq, d)
-    dor = chunk_roll(do, -shift, shb).reshape(B * N // G, G, Hq, d)
+    sw = lambda x: _swap_wrap_front(x, N, G, shb, shift, wrap_front_first)
+    qr = sw(chunk_roll(q, -shift, shb).reshape(B * N // G, G, Hq, d))
+    kr = sw(chunk_roll(ke, -shift, shb).reshape(B * N // G, G, Hq, d))
+    vr = sw(chunk_roll(ve, -shift, shb).reshape(B * N // G, G, Hq, d))
+    dor = sw(chunk_roll(do, -shift, shb).reshape(B * N // G, G, Hq, d))
     dq, dk, dv = causal_self_attn_backward(qr, kr, vr, dor, scale, splits)
-    # The derivative of a roll is the opposite roll ...
+    # The derivative of a reordering is the inverse reordering ...
+    dq, dk, dv = (_swap_wrap_front(x, N, G, shb, shift, wrap_front_first, inverse=True)
+                  for x in (dq, dk, dv))
+    # ... and that of a roll is the opposite roll ...
     dq = chunk_roll(dq.reshape(B, N, Hq, d), shift, shb)
     dk = chunk_roll(dk.reshape(B, N, Hq, d), shift, shb)
     dv = chunk_roll(dv.reshape(B, N, Hq, d), shift, shb)

@@ -13,6 +13,8 @@
 * the worked roll example (§3.4 "Step 2: Shift one chunk"), from tests/golden;
 * Variant 2 of Table 8 (wrapped tokens in their own group): equal to the library version with
   the wrap group split by an explicit mask, and identical to the default outside that group;
+* Variant 3 of Table 8 (wrapped tokens moved to the front of the last group): equal to causal
+  attention in original token order under a same-shifted-group mask, written without any roll;
 * central finite differences of the forward against the backward;
 * closed-form sums implied by rows of P summing to one;
 * planted mistakes in the oracle must fail these pins.
@@ -131,6 +133,78 @@ def test_variant2_only_changes_the_wrap_group():
     p = np.exp(sq - sq.max(1, keepdims=True))
     p /= p.sum(1, keepdims=True)
     np.testing.assert_allclose(b[0, :shift, h], p @ v[0, :shift, h], atol=1e-13)
+
+
+def original_order_s2attn(q, k, v, G, scale, shb, shift):
+    """Variant 3 written without any roll: in original token order, a shifted head attends
+    causally (key not after query) within its shifted group, the group of token t being
+    ((t - shift) mod N) // G; an unshifted head within t // G. torch SDPA with that mask."""
+    B, N, Hq, d = q.shape
+    rep = Hq // k.shape[2]
+    t = torch.arange(N)
+    outs, lses = [], []
+    for h in range(Hq):
+        s = shift if h >= shb else 0
+        gid = ((t - s) % N) // G
+        mask = (gid[:, None] == gid[None, :]) & (t[None, :] <= t[:, None])
+        qh, kh, vh = q[:, :, h], k[:, :, h // rep], v[:, :, h // rep]
+        outs.append(F.scaled_dot_product_attention(qh, kh, vh, attn_mask=mask, scale=scale))
+        scores = (scale * qh @ kh.transpose(-1, -2)).masked_fill(~mask, float("-inf"))
+        lses.append(torch.logsumexp(scores, dim=-1))
+    return torch.stack(outs, dim=2), torch.stack(lses, dim=1)
+
+
+def variant3_errors(B, Hq, Hkv, N, G, d, shift, seed=13):
+    q, k, v, do = make(B, Hq, Hkv, N, d, seed)
+    scale = 1.0 / np.sqrt(d)
+    o, lse = orc.s2attn_forward(q, k, v, G, scale, None, shift, wrap_front_first=True)
+    dq, dk, dv = orc.s2attn_backward(q, k, v, do, G, scale, None, shift, wrap_front_first=True)
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    to, tl = original_order_s2attn(tq, tk, tv, G, scale, Hq // 2, shift)
+    to.backward(torch.tensor(do))
+    return [float(np.abs(a - b.detach().numpy()).max()) for a, b in
+            ((o, to), (lse, tl), (dq, tq.grad), (dk, tk.grad), (dv, tv.grad))]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,G,d,shift", [
+    (1, 4, 4, 64, 16, 8, 8),     # half-group roll
+    (2, 4, 2, 48, 16, 8, 4),     # GQA, batch 2, quarter-group roll
+    (1, 8, 1, 32, 8, 4, 6),      # MQA, most of the group wrapped
+])
+def test_variant3_is_causal_in_original_order_within_shifted_groups(B, Hq, Hkv, N, G, d, shift):
+    """Variant 3 (Table 8, Figure 6): with the wrapped tokens moved to the front of the last
+    group, every group's causal order is the original token order, so the oracle's roll,
+    group, swap, attend, unswap, unroll sequence must equal causal attention in original
+    order under a same-shifted-group mask (no roll anywhere), forward, LSE and autograd."""
+    assert max(variant3_errors(B, Hq, Hkv, N, G, d, shift)) < 1e-12
+
+
+def test_variant3_against_default_and_variant2():
+    """Outside the last rolled group Variant 3 is bit-identical to the default; the wrapped
+    tokens see only each other (as in Variant 2); the other tokens of that group now also
+    see the wrapped ones, which changes their outputs."""
+    B, Hq, N, G, d, shift = 1, 4, 64, 16, 8, 8
+    q, k, v, do = make(B, Hq, Hq, N, d, 5)
+    a, _ = orc.s2attn_forward(q, k, v, G, 0.3, None, shift)
+    b, _ = orc.s2attn_forward(q, k, v, G, 0.3, None, shift, wrap_own_group=True)
+    c, _ = orc.s2attn_forward(q, k, v, G, 0.3, None, shift, wrap_front_first=True)
+    assert np.array_equal(a[:, :, :2], c[:, :, :2])
+    last = np.r_[N - (G - shift):N, 0:shift]
+    keep = np.setdiff1d(np.arange(N), last)
+    assert np.array_equal(a[:, keep, 2:], c[:, keep, 2:])
+    np.testing.assert_allclose(c[:, :shift, 2:], b[:, :shift, 2:], atol=1e-13)
+    back = np.arange(N - (G - shift), N)
+    assert not np.allclose(c[:, back, 2:], a[:, back, 2:])
+
+
+def _swap_never_undone(x, N, G, shb, shift, enabled, inverse=False):
+    return _SWAP(x, N, G, shb, shift, enabled, inverse=False)
+
+
+def test_planted_variant3_mistake_is_caught(monkeypatch):
+    monkeypatch.setattr(orc, "_swap_wrap_front", _swap_never_undone)
+    # (with shift = G/2 a second forward swap would undo the first: use shift != G/2)
+    assert max(variant3_errors(1, 4, 2, 32, 8, 4, 2, seed=3)) > 1e-3
 
 
 def test_one_group_no_shift_is_full_causal_attention():
@@ -293,6 +367,9 @@ def test_head_group_rows_matches_full():
 # --------------------------------------------------------------------------------------
 def _tile_kv(x, Hq):
     return np.tile(x, (1, 1, Hq // x.shape[2], 1))
+
+
+_SWAP = orc._swap_wrap_front
 
 
 def _leaky_probs(q, k, scale, split=None):
