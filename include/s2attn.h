@@ -95,8 +95,9 @@ S2ATTN_API s2attn_status s2attn_fwd_ex(const void* q, const void* k, const void*
                             int B, int Hq, int Hkv, int N, int d, int G, float scale,
                             int shift_head_begin, int shift, void* stream);
 
-/* Option flags of the _general entry points. */
+/* Option flags of the _general entry points (at most one of the two). */
 #define S2ATTN_FLAG_WRAP_OWN_GROUP 1
+#define S2ATTN_FLAG_WRAP_FRONT_FIRST 2
 /*
  * S2ATTN_FLAG_WRAP_OWN_GROUP is the pages' Variant 2 (summary page, §3.4 "Information
  * leakage considerations", Table 8, Figure 6): in the rolled heads the tokens that the roll
@@ -104,6 +105,13 @@ S2ATTN_API s2attn_status s2attn_fwd_ex(const void* q, const void* k, const void*
  * last group with the last G - shift tokens, i.e. the last rolled group is split at the wrap
  * into two causal groups. Requires a rolled head (shift_head_begin < Hq) and 0 < shift < G
  * (after reduction mod N), else S2ATTN_ERR_INVALID_ARG.
+ *
+ * S2ATTN_FLAG_WRAP_FRONT_FIRST is the pages' Variant 3 (same passage: the shifted tokens swap
+ * places with the original front tokens): in the rolled heads the last rolled group lists the
+ * wrapped tokens 0..shift-1 first and the last G - shift tokens after them, so the causal
+ * order inside it is the original token order (the wrapped tokens no longer see the end of the
+ * sequence; the end of the sequence sees them). Same requirements as Variant 2; combining the
+ * two flags is S2ATTN_ERR_INVALID_ARG.
  *
  * Strides. Each [B, N, H, d] tensor X is read or written at X + b*sb + t*st + h*d + c
  * (elements): the (H, d) block of a token is contiguous, tokens and batches may be spaced

@@ -12,6 +12,7 @@ from ._lib import (  # noqa: F401
     S2ATTN_ERR_CUDA,
     S2ATTN_ERR_TIMEOUT,
     S2ATTN_FLAG_WRAP_OWN_GROUP,
+    S2ATTN_FLAG_WRAP_FRONT_FIRST,
     SIGNATURES,
     LIB_PATH,
     lib,

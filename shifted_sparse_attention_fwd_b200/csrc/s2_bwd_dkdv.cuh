@@ -45,6 +45,7 @@ struct BwdParams {
   __nv_bfloat16* dv;
   int B, Hq, Hkv, N, G, shift_head_begin, shift;
   int wrap;           // wrap split of the shifted heads' last group (kNoWrapSplit: none)
+  int front;          // Variant 3: the shifted heads' last group lists the wrapped tokens first
   float scale_log2;   // scale * log2(e)
   float scale;
   unsigned int* err;
@@ -107,7 +108,8 @@ __device__ __forceinline__ void dkdv_tile(const BwdParams& p, int u, int& b, int
   kvh += p.kvh_begin;
 }
 
-template <int D>
+// kFront: built for the Variant 3 reordering (otherwise p.front is ignored).
+template <int D, bool kFront>
 __global__ void __launch_bounds__(32 * (kDkdvEwWarps + 3), 1)
     s2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQ8,
                        const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmK8,
@@ -132,12 +134,15 @@ __global__ void __launch_bounds__(32 * (kDkdvEwWarps + 3), 1)
   const int rep = p.Hq / p.Hkv;
   const int T = (p.N + kTileRows - 1) / kTileRows;
   const int n_tiles = p.B * p.kvh_count * T;
-  auto head_shift = [&](int hq) { return hq >= p.shift_head_begin ? p.shift : 0; };
+  auto head_map = [&](int hq) {
+    const bool shifted = hq >= p.shift_head_begin;
+    return head_remap(p.N, p.G, shifted ? p.shift : 0, (kFront && shifted) ? p.front : 0);
+  };
   auto head_wrap = [&](int hq) { return hq >= p.shift_head_begin ? p.wrap : kNoWrapSplit; };
   auto pairs_of = [&](int kvh, int t0) {
     int total = 0;
     for (int hq = kvh * rep; hq < (kvh + 1) * rep; ++hq)
-      total += kv_tile_qtiles(t0, head_shift(hq), p.N, p.G, head_wrap(hq)).count();
+      total += kv_tile_qtiles(head_map(hq), t0, head_wrap(hq)).count();
     return total;
   };
 
@@ -204,7 +209,7 @@ __global__ void __launch_bounds__(32 * (kDkdvEwWarps + 3), 1)
         // K and V of the previous tile are free once its last S and dP MMAs are done.
         if (tc > 0 && !wait_bar(bar(L::B_KVE), (tc - 1) & 1, ctx, 11)) { ok = false; break; }
         mbar_expect_tx(bar(L::B_KV), 2 * L::kTile);
-        const TileRuns kv_runs = rolled_tile_runs(t0, 0, p.N);
+        const Runs kv_runs = identity_runs(t0, p.N);
         load_tile<D>(sbase + L::kK, &tmK, &tmK8, bar(L::B_KV), b, kvh, kv_runs, p.N);
         load_tile<D>(sbase + L::kV, &tmV, &tmV8, bar(L::B_KV), b, kvh, kv_runs, p.N);
         ++kv_loads;
@@ -213,24 +218,27 @@ __global__ void __launch_bounds__(32 * (kDkdvEwWarps + 3), 1)
           break;
         }
         for (int hq = kvh * rep; ok && hq < (kvh + 1) * rep; ++hq) {
-          const int sh = head_shift(hq);
-          const QTileRanges qr = kv_tile_qtiles(t0, sh, p.N, p.G, head_wrap(hq));
+          const HeadRemap hm = head_map(hq);
+          const QTileRanges qr = kv_tile_qtiles(hm, t0, head_wrap(hq));
           const float* lse_row = p.lse2 + (static_cast<size_t>(b) * p.Hq + hq) * p.N;
           const float* d_row = p.dvec + (static_cast<size_t>(b) * p.Hq + hq) * p.N;
           for (int i = 0; i < qr.count(); ++i, ++n) {
             const int st = n & 1;
             if (n >= 2 && !wait_bar(bar(L::B_QE + st), ((n >> 1) - 1) & 1, ctx, 1)) { ok = false; break; }
-            const TileRuns tr = rolled_tile_runs(qr.at(i) * kTileRows, sh, p.N);
+            const Runs tr = rolled_runs(hm, qr.at(i) * kTileRows);
             const uint32_t fb = bar(L::B_QF + st);
             mbar_expect_tx(fb, 2 * L::kTile + 8u * tr.valid);
             load_tile<D>(sbase + L::kQ + st * L::kTile, &tmQ, &tmQ8, fb, b, hq, tr, p.N);
             load_tile<D>(sbase + L::kDO + st * L::kTile, &tmO, &tmO8, fb, b, hq, tr, p.N);
             const uint32_t sl = sbase + L::kLse + st * 512, sd = sbase + L::kDv + st * 512;
-            bulk_load(sl, lse_row + tr.start, 4u * tr.first, fb);
-            bulk_load(sd, d_row + tr.start, 4u * tr.first, fb);
-            if (tr.valid > tr.first) {
-              bulk_load(sl + 4u * tr.first, lse_row, 4u * (tr.valid - tr.first), fb);
-              bulk_load(sd + 4u * tr.first, d_row, 4u * (tr.valid - tr.first), fb);
+            int base = 0;
+#pragma unroll
+            for (int r = 0; r < 3; ++r) {
+              if (r < tr.n) {
+                bulk_load(sl + 4u * base, lse_row + tr.src[r], 4u * tr.len[r], fb);
+                bulk_load(sd + 4u * base, d_row + tr.src[r], 4u * tr.len[r], fb);
+                base += tr.len[r];
+              }
             }
             last_parity[st] = (n >> 1) & 1;
           }
@@ -311,15 +319,13 @@ __global__ void __launch_bounds__(32 * (kDkdvEwWarps + 3), 1)
         dkdv_tile(p, u, b, kvh, t0);
         if (p.ds) {
           for (int hq = kvh * rep; ok && hq < (kvh + 1) * rep; ++hq) {
-            const int sh = head_shift(hq);
-            const QTileRanges qr = kv_tile_qtiles(t0, sh, p.N, p.G, head_wrap(hq));
+            const HeadRemap hm = head_map(hq);
+            const QTileRanges qr = kv_tile_qtiles(hm, t0, head_wrap(hq));
             for (int i = 0; ok && i < qr.count(); ++i) {
               const int qt = qr.at(i);
-              const KvSpan sp = qtile_kv_span(qt, sh, p.N, p.G, head_wrap(hq));
-              int idx = t0 / kTileRows - sp.first;
-              if (idx < 0) idx += T;
+              const int idx = qtile_kv_span(hm, qt, head_wrap(hq)).index_of(t0 / kTileRows);
               ok = hand_over([&] {
-                if (idx < sp.count)
+                if (idx >= 0)
                   bulk_store(ds_slot_ptr(p, b, hq, p.slots.base(qt) + idx), sbase + L::kStage,
                              kDsTileBytes);
               });
@@ -367,9 +373,9 @@ __global__ void __launch_bounds__(32 * (kDkdvEwWarps + 3), 1)
       const int t = t0 + row;
       const bool kv_valid = t < p.N;
       for (int hq = kvh * rep; ok && hq < (kvh + 1) * rep; ++hq) {
-        const int sh = head_shift(hq);
-        const QTileRanges qr = kv_tile_qtiles(t0, sh, p.N, p.G, head_wrap(hq));
-        const int r_k = kv_valid ? (t - sh < 0 ? t - sh + p.N : t - sh) : 0;
+        const HeadRemap hm = head_map(hq);
+        const QTileRanges qr = kv_tile_qtiles(hm, t0, head_wrap(hq));
+        const int r_k = kv_valid ? hm.rolled(t) : 0;
         const int ge_k = group_end(r_k, p.G, head_wrap(hq));
         for (int i = 0; i < qr.count(); ++i, ++n) {
           const int st = n & 1;
@@ -383,20 +389,22 @@ __global__ void __launch_bounds__(32 * (kDkdvEwWarps + 3), 1)
           const float* lse_t = s_lse + st * 128 + W * grp;
           const float* d_t = s_dv + st * 128 + W * grp;
           // P^T phase: W columns of S^T -> P^T (bf16), kept in registers for the dS phase.
+          // The columns are read in two halves of 16 to keep fewer values in flight.
           uint32_t pk[W / 2];
-          {
-            uint32_t raw[W];
-            tmem_ld32(t_lane + W * grp, raw);
 #pragma unroll
-            for (int e = 0; e < W / 2; ++e) {
-              const int col = 2 * e;
-              float x0 = fast_exp2(fmaf(__uint_as_float(raw[col]), c, -lse_t[col]));
-              float x1 = fast_exp2(fmaf(__uint_as_float(raw[col + 1]), c, -lse_t[col + 1]));
+          for (int h = 0; h < 2; ++h) {
+            uint32_t raw[16];
+            tmem_ld16(t_lane + W * grp + 16 * h, raw);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int col = 16 * h + 2 * e;
+              float x0 = fast_exp2(fmaf(__uint_as_float(raw[2 * e]), c, -lse_t[col]));
+              float x1 = fast_exp2(fmaf(__uint_as_float(raw[2 * e + 1]), c, -lse_t[col + 1]));
               if (mask) {
                 x0 = (col >= cl && col <= ch) ? x0 : 0.f;
                 x1 = (col + 1 >= cl && col + 1 <= ch) ? x1 : 0.f;
               }
-              pk[e] = pack_bf16(x0, x1);
+              pk[8 * h + e] = pack_bf16(x0, x1);
             }
           }
           tmem_st16(t_lane + W * grp, pk);
@@ -407,23 +415,24 @@ __global__ void __launch_bounds__(32 * (kDkdvEwWarps + 3), 1)
           if (!warp_wait(bar(L::B_DP), n & 1, ctx, 9)) { ok = false; break; }
           tc_fence_after();
           uint32_t ds[W / 2];
-          {
-            uint32_t raw[W];
-            tmem_ld32(t_lane + 128 + W * grp, raw);
 #pragma unroll
-            for (int e = 0; e < W / 2; ++e) {
-              const int col = 2 * e;
-              const float2 pf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[e]));
-              float y0 = pf.x * (__uint_as_float(raw[col]) - d_t[col]);
-              float y1 = pf.y * (__uint_as_float(raw[col + 1]) - d_t[col + 1]);
+          for (int h = 0; h < 2; ++h) {
+            uint32_t raw[16];
+            tmem_ld16(t_lane + 128 + W * grp + 16 * h, raw);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int col = 16 * h + 2 * e;
+              const float2 pf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[8 * h + e]));
+              float y0 = pf.x * (__uint_as_float(raw[2 * e]) - d_t[col]);
+              float y1 = pf.y * (__uint_as_float(raw[2 * e + 1]) - d_t[col + 1]);
               if (mask) {   // exact zeros where P is masked, whatever D holds for padding rows
                 y0 = (col >= cl && col <= ch) ? y0 : 0.f;
                 y1 = (col + 1 >= cl && col + 1 <= ch) ? y1 : 0.f;
               }
-              ds[e] = pack_bf16(y0, y1);
+              ds[8 * h + e] = pack_bf16(y0, y1);
             }
-            tmem_st16(t_lane + 128 + W * grp, ds);
           }
+          tmem_st16(t_lane + 128 + W * grp, ds);
           tmem_st_wait();
           tc_fence_before();
           mbar_arrive(bar(L::B_DS));

@@ -46,7 +46,8 @@ struct DqLayout {
   static constexpr int kThreads = 320;
 };
 
-template <int D>
+// kFront: built for the Variant 3 reordering (otherwise p.front is ignored).
+template <int D, bool kFront>
 __global__ void __launch_bounds__(320, 1)
     s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQ8,
                      const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmK8,
@@ -66,8 +67,9 @@ __global__ void __launch_bounds__(320, 1)
   int b, h, qt;
   query_tile_coords(blockIdx.x, p.B, p.Hq, p.N, p.G, b, h, qt);
   const int R0 = qt * kTileRows;
-  const int shift_h = h >= p.shift_head_begin ? p.shift : 0;
-  const int wrap_h = h >= p.shift_head_begin ? p.wrap : kNoWrapSplit;
+  const bool shifted = h >= p.shift_head_begin;
+  const HeadRemap hm = head_remap(p.N, p.G, shifted ? p.shift : 0, (kFront && shifted) ? p.front : 0);
+  const int wrap_h = shifted ? p.wrap : kNoWrapSplit;
   const int kvh = h / (p.Hq / p.Hkv);
   const int kt_begin = group_begin(R0, p.G, wrap_h) / kTileRows;
   const int n_kv = qt - kt_begin + 1;
@@ -107,7 +109,7 @@ __global__ void __launch_bounds__(320, 1)
   if (warp == 8) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
-      const TileRuns q_runs = rolled_tile_runs(R0, shift_h, p.N);
+      const Runs q_runs = rolled_runs(hm, R0);
       mbar_expect_tx(bar(L::B_QDO), 2 * L::kTile);
       load_tile<D>(sbase + L::kQ, &tmQ, &tmQ8, bar(L::B_QDO), b, h, q_runs, p.N);
       load_tile<D>(sbase + L::kDO, &tmO, &tmO8, bar(L::B_QDO), b, h, q_runs, p.N);
@@ -119,7 +121,7 @@ __global__ void __launch_bounds__(320, 1)
           return false;
         mbar_expect_tx(bar(L::B_K + st), L::kTile);
         load_tile<D>(sbase + L::kK + st * L::kTile, &tmK, &tmK8, bar(L::B_K + st), b, kvh,
-                     rolled_tile_runs((kt_begin + i) * kTileRows, shift_h, p.N), p.N);
+                     rolled_runs(hm, (kt_begin + i) * kTileRows), p.N);
         ++k_issued;
         return true;
       };
@@ -130,7 +132,7 @@ __global__ void __launch_bounds__(320, 1)
           return false;
         mbar_expect_tx(bar(L::B_V + st), L::kTile);
         load_tile<D>(sbase + L::kV + st * L::kTile, &tmV, &tmV8, bar(L::B_V + st), b, kvh,
-                     rolled_tile_runs((kt_begin + i) * kTileRows, shift_h, p.N), p.N);
+                     rolled_runs(hm, (kt_begin + i) * kTileRows), p.N);
         ++v_issued;
         return true;
       };
@@ -189,8 +191,7 @@ __global__ void __launch_bounds__(320, 1)
     const bool row_valid = r < p.N;
     const int lo = row_valid ? group_begin(r, p.G, wrap_h) : kt_begin * kTileRows;
     const int hi = row_valid ? r : kt_begin * kTileRows;
-    const long long tt = static_cast<long long>(r) + shift_h;
-    const int t = row_valid ? static_cast<int>(tt >= p.N ? tt - p.N : tt) : 0;
+    const int t = row_valid ? hm.token(r) : 0;
     const size_t lrow = (static_cast<size_t>(b) * p.Hq + h) * p.N + t;
     const float lse2 = row_valid ? p.lse2[lrow] : 0.f;
     const float dd = row_valid ? p.dvec[lrow] : 0.f;

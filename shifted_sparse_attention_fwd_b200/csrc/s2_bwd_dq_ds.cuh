@@ -51,7 +51,8 @@ __device__ __forceinline__ void dq_ds_tile(const BwdParams& p, int u, int& b, in
   hq = p.kvh_begin * rep + hl;
 }
 
-template <int D>
+// kFront: built for the Variant 3 reordering (otherwise p.front is ignored).
+template <int D, bool kFront>
 __global__ void __launch_bounds__(192, 1)
     s2_bwd_dq_ds_kernel(const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmK8, const BwdParams p) {
@@ -68,7 +69,10 @@ __global__ void __launch_bounds__(192, 1)
   const int rep = p.Hq / p.Hkv;
   const int T = (p.N + kTileRows - 1) / kTileRows;
   const int units = p.B * p.kvh_count * rep * T;
-  auto head_shift = [&](int hq) { return hq >= p.shift_head_begin ? p.shift : 0; };
+  auto head_map = [&](int hq) {
+    const bool shifted = hq >= p.shift_head_begin;
+    return head_remap(p.N, p.G, shifted ? p.shift : 0, (kFront && shifted) ? p.front : 0);
+  };
   auto head_wrap = [&](int hq) { return hq >= p.shift_head_begin ? p.wrap : kNoWrapSplit; };
 
   if (warp == 0 && lane == 0) {
@@ -110,10 +114,11 @@ __global__ void __launch_bounds__(192, 1)
         if (u < 0) break;
         int b, hq, qt;
         dq_ds_tile(p, u, b, hq, qt);
-        const KvSpan sp = qtile_kv_span(qt, head_shift(hq), p.N, p.G, head_wrap(hq));
+        const KvSpan sp = qtile_kv_span(head_map(hq), qt, head_wrap(hq));
         const __nv_bfloat16* ds0 = ds_slot_ptr(p, b, hq, p.slots.base(qt));
         const int kvh = hq / rep;
-        for (int i = 0; i < sp.count; ++i, ++it) {
+        const int count = sp.count();
+        for (int i = 0; i < count; ++i, ++it) {
           const int s = it % L::kStages;
           if (it >= L::kStages &&
               !wait_bar(bar(L::B_EMPTY + s), ((it / L::kStages) - 1) & 1, ctx, 1)) {
@@ -124,10 +129,8 @@ __global__ void __launch_bounds__(192, 1)
           const uint32_t dst = sbase + s * L::kStageBytes;
           mbar_expect_tx(fb, L::kStageBytes);
           bulk_load(dst, ds0 + static_cast<size_t>(i) * (kDsTileBytes / 2), kDsTileBytes, fb);
-          int t = sp.first + i;
-          if (t >= T) t -= T;
           load_tile<D>(dst + kDsTileBytes, &tmK, &tmK8, fb, b, kvh,
-                       rolled_tile_runs(t * kTileRows, 0, p.N), p.N);
+                       identity_runs(sp.at(i) * kTileRows, p.N), p.N);
         }
       }
       // Wait (bounded) for the copies still in flight before the CTA may exit.
@@ -148,7 +151,7 @@ __global__ void __launch_bounds__(192, 1)
         if (u < 0) break;
         int b, hq, qt;
         dq_ds_tile(p, u, b, hq, qt);
-        const int count = qtile_kv_span(qt, head_shift(hq), p.N, p.G, head_wrap(hq)).count;
+        const int count = qtile_kv_span(head_map(hq), qt, head_wrap(hq)).count();
         const int a = n & 1;
         if (n >= 2 && !wait_bar(bar(L::B_ACCE + a), ((n >> 1) - 1) & 1, ctx, 2)) { ok = false; break; }
         tc_fence_after();
@@ -189,10 +192,9 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_after();
       const int r = qt * kTileRows + row;
       const bool valid = r < p.N;
-      int t = r + head_shift(hq);
-      if (t >= p.N) t -= p.N;
+      const int t = valid ? head_map(hq).token(r) : 0;
       __nv_bfloat16* dst_row =
-          p.dq + b * p.dq_sb + (valid ? t : 0) * p.dq_st + static_cast<long long>(hq) * D;
+          p.dq + b * p.dq_sb + t * p.dq_st + static_cast<long long>(hq) * D;
 #pragma unroll
       for (int j = 0; j < D / 32; ++j) {
         uint32_t rr[32];

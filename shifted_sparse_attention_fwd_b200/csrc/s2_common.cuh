@@ -17,20 +17,25 @@ struct Tile {
 };
 
 // Issue the TMA loads of one 128-row tile of a [B, N, H, D] tensor whose rows are given by
-// `tr`. Runs of 128 rows use the 128-row box; anything else is moved in 8-row boxes (one
-// swizzle atom each), with rows past the sequence read out of bounds so TMA writes zeros.
-// Always delivers Tile<D>::kBytes on `bar`.
+// `tr`. A single run of 128 rows uses the 128-row box; anything else is moved in 8-row boxes
+// (one swizzle atom each; every run starts and ends on an 8-row boundary), with rows past the
+// sequence read out of bounds so TMA writes zeros. Always delivers Tile<D>::kBytes on `bar`.
 template <int D>
 __device__ __forceinline__ void load_tile(uint32_t dst, const CUtensorMap* m128,
                                           const CUtensorMap* m8, uint32_t bar, int b, int h,
-                                          const TileRuns& tr, int N) {
-  if (tr.first == kTileRows) {
+                                          const Runs& tr, int N) {
+  if (tr.n == 1 && tr.len[0] == kTileRows) {
 #pragma unroll
     for (int half = 0; half < Tile<D>::kHalves; ++half)
-      tma_load_4d(dst + half * Tile<D>::kHalfBytes, m128, bar, half * 64, h, tr.start, b);
+      tma_load_4d(dst + half * Tile<D>::kHalfBytes, m128, bar, half * 64, h, tr.src[0], b);
   } else {
     for (int row = 0; row < kTileRows; row += 8) {
-      const int src = row < tr.first ? tr.start + row : (row < tr.valid ? row - tr.first : N);
+      int src = N, base = 0;
+#pragma unroll
+      for (int k = 0; k < 3; ++k) {
+        if (k < tr.n && row >= base && row < base + tr.len[k]) src = tr.src[k] + (row - base);
+        base += k < tr.n ? tr.len[k] : 0;
+      }
 #pragma unroll
       for (int half = 0; half < Tile<D>::kHalves; ++half)
         tma_load_4d(dst + half * Tile<D>::kHalfBytes + row * 128, m8, bar, half * 64, h, src, b);

@@ -42,6 +42,7 @@ struct FwdParams {
   float* lse;
   int B, Hq, Hkv, N, G, shift_head_begin, shift;
   int wrap;           // wrap split of the shifted heads' last group (kNoWrapSplit: none)
+  int front;          // Variant 3: the shifted heads' last group lists the wrapped tokens first
   float scale_log2;   // scale * log2(e)
   unsigned int* err;
   unsigned long long timeout_ns;
@@ -90,7 +91,8 @@ __device__ __forceinline__ float max_tree128(const float (&s)[128]) {
 
 // One work unit: query tiles 2*pair and 2*pair + 1 of (b, h) and the key tiles they see.
 struct FwdUnit {
-  int b, h, kvh, shift_h, wrap_h;
+  int b, h, kvh, wrap_h;
+  int shift_h, front_h;   // the head's remap: head_remap(N, G, shift_h, front_h)
   int qt[2], kb[2], ke[2];
   bool tv[2];
   int kv_lo, n_kv;
@@ -99,13 +101,18 @@ struct FwdUnit {
   }
 };
 
+// kFront: the kernel is built for the Variant 3 reordering (otherwise p.front is ignored and
+// the plain-roll index code is all that is compiled in).
+template <bool kFront>
 __device__ __forceinline__ FwdUnit fwd_unit(const FwdParams& p, int unit) {
   FwdUnit u;
   int pair;
   query_pair_coords_chunked(unit, p.B, p.Hq, p.N, p.G, kL2Chunk, u.b, u.h, pair);
   const int nqt = (p.N + kTileRows - 1) / kTileRows;
-  u.shift_h = u.h >= p.shift_head_begin ? p.shift : 0;
-  u.wrap_h = u.h >= p.shift_head_begin ? p.wrap : kNoWrapSplit;
+  const bool shifted = u.h >= p.shift_head_begin;
+  u.shift_h = shifted ? p.shift : 0;
+  u.front_h = (kFront && shifted) ? p.front : 0;
+  u.wrap_h = shifted ? p.wrap : kNoWrapSplit;
   u.kvh = u.h / (p.Hq / p.Hkv);
   // Tile t = 2*pair + t sees key tiles [kb[t], ke[t]]; tile 0 always exists, tile 1 may not.
 #pragma unroll
@@ -120,7 +127,7 @@ __device__ __forceinline__ FwdUnit fwd_unit(const FwdParams& p, int unit) {
   return u;
 }
 
-template <int D>
+template <int D, bool kFront>
 __global__ void __launch_bounds__(320, 1)
     s2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQ8,
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmK8,
@@ -182,7 +189,7 @@ __global__ void __launch_bounds__(320, 1)
           return false;
         mbar_expect_tx(bar(L::B_K + st), L::kTile);
         load_tile<D>(sbase + L::kK + st * L::kTile, &tmK, &tmK8, bar(L::B_K + st), u.b, u.kvh,
-                     rolled_tile_runs((u.kv_lo + j) * kTileRows, u.shift_h, p.N), p.N);
+                     rolled_runs(head_remap(p.N, p.G, u.shift_h, kFront ? u.front_h : 0), (u.kv_lo + j) * kTileRows), p.N);
         ++k_issued;
         return true;
       };
@@ -193,12 +200,12 @@ __global__ void __launch_bounds__(320, 1)
           return false;
         mbar_expect_tx(bar(L::B_V + st), L::kTile);
         load_tile<D>(sbase + L::kV + st * L::kTile, &tmV, &tmV8, bar(L::B_V + st), u.b, u.kvh,
-                     rolled_tile_runs((u.kv_lo + j) * kTileRows, u.shift_h, p.N), p.N);
+                     rolled_runs(head_remap(p.N, p.G, u.shift_h, kFront ? u.front_h : 0), (u.kv_lo + j) * kTileRows), p.N);
         ++v_issued;
         return true;
       };
       for (int unit = blockIdx.x; ok && unit < n_units; unit += gridDim.x) {
-        const FwdUnit u = fwd_unit(p, unit);
+        const FwdUnit u = fwd_unit<kFront>(p, unit);
         ok = issue_k(u, 0);   // the first key tile can stream while the last unit finishes
         for (int t = 0; ok && t < 2; ++t) {
           if (!u.tv[t]) continue;
@@ -208,7 +215,7 @@ __global__ void __launch_bounds__(320, 1)
           }
           mbar_expect_tx(bar(L::B_Q + t), L::kTile);
           load_tile<D>(sbase + L::kQ + t * L::kTile, &tmQ, &tmQ8, bar(L::B_Q + t), u.b, u.h,
-                       rolled_tile_runs(u.qt[t] * kTileRows, u.shift_h, p.N), p.N);
+                       rolled_runs(head_remap(p.N, p.G, u.shift_h, kFront ? u.front_h : 0), u.qt[t] * kTileRows), p.N);
           ++q_loads[t];
         }
         for (int j = 0; ok && j < u.n_kv; ++j) {
@@ -235,7 +242,7 @@ __global__ void __launch_bounds__(320, 1)
         return wait_bar(bar(L::B_K + i % L::kKStages), (i / L::kKStages) & 1, ctx, 3);
       };
       for (int unit = blockIdx.x; ok && unit < n_units; unit += gridDim.x) {
-        const FwdUnit u = fwd_unit(p, unit);
+        const FwdUnit u = fwd_unit<kFront>(p, unit);
         bool q_ready[2] = {false, false}, first_pv[2] = {true, true};
         // S_t(j) = Q_t K(j)^T into TMEM columns [128 t, 128 t + 128).
         auto issue_s = [&](int t, int kidx) -> bool {
@@ -304,7 +311,7 @@ __global__ void __launch_bounds__(320, 1)
     int s_cnt = 0, o_cnt = 0;
     bool ok = true;
     for (int unit = blockIdx.x; ok && unit < n_units; unit += gridDim.x) {
-      const FwdUnit u = fwd_unit(p, unit);
+      const FwdUnit u = fwd_unit<kFront>(p, unit);
       if (!u.tv[wg]) continue;
       const int r = u.qt[wg] * kTileRows + row;
       const bool row_valid = r < p.N;
@@ -329,7 +336,9 @@ __global__ void __launch_bounds__(320, 1)
         const float m_cand = fmaxf(m_run, max_tree128(s) * c);
         const bool need = m_cand > m_run + kRescaleThreshold;
         if (__any_sync(0xffffffffu, need)) {
-          const float alpha = fast_exp2(m_run - m_cand);   // 0 when m_run = -inf
+          // 0 when m_run = -inf; 1 for a row that has seen no allowed key yet (its O and l
+          // are still zero) while others in the warp rescale: -inf - -inf would be NaN
+          const float alpha = m_cand == -INFINITY ? 1.f : fast_exp2(m_run - m_cand);
           if (cnt > 0) {
 #pragma unroll 1
             for (int j = 0; j < D / 32; ++j) {
@@ -399,8 +408,7 @@ __global__ void __launch_bounds__(320, 1)
           const uint4 w4 = *reinterpret_cast<const uint4*>(stage + rr * 128 + ((chunk ^ (rr & 7)) * 16));
           const int rq = r_warp + rr;
           if (rq < p.N) {
-            const long long tq = static_cast<long long>(rq) + u.shift_h;
-            const int tok = static_cast<int>(tq >= p.N ? tq - p.N : tq);
+            const int tok = head_remap(p.N, p.G, u.shift_h, kFront ? u.front_h : 0).token(rq);
             __nv_bfloat16* dst = p.o + u.b * p.o_sb + tok * p.o_st + static_cast<long long>(u.h) * D +
                                  64 * half + 8 * chunk;
             *reinterpret_cast<uint4*>(dst) = w4;
@@ -409,8 +417,7 @@ __global__ void __launch_bounds__(320, 1)
         __syncwarp();
       }
       if (row_valid) {
-        const long long tq = static_cast<long long>(r) + u.shift_h;
-        const int tok = static_cast<int>(tq >= p.N ? tq - p.N : tq);
+        const int tok = head_remap(p.N, p.G, u.shift_h, kFront ? u.front_h : 0).token(r);
         p.lse[(static_cast<size_t>(u.b) * p.Hq + u.h) * p.N + tok] =
             (m_run + __log2f(l_run)) * 0.6931471805599453f;
       }

@@ -8,7 +8,8 @@
 // where s_h is the head's roll (G/2 for the shifted heads, 0 otherwise); group of rolled
 // row r is floor(r / G). Tiles are 128 consecutive rolled rows; such a tile maps onto at
 // most two contiguous runs of original rows (the run that reaches token N-1 and the run
-// that wraps to token 0), plus zero rows past the end of the sequence.
+// that wraps to token 0; three with the Variant 3 reordering), plus zero rows past the end
+// of the sequence.
 #pragma once
 
 #ifndef __CUDACC__
@@ -25,36 +26,118 @@ constexpr int kTileRows = 128;
 // Q/dO) tiles of about this many groups stay resident in L2 while their work runs.
 constexpr int kL2Chunk = 10;
 
-struct TileRuns {
-  int valid;   // rows of the tile inside the sequence (rows [valid, 128) are padding)
-  int first;   // rows [0, first) come from original rows [start, start + first)
-  int start;   // original row of tile row 0
-  // rows [first, valid) come from original rows [0, valid - first)
-};
-
-// Rolled tile starting at rolled row r0, head roll `shift` (0 <= shift < N).
-__host__ __device__ inline TileRuns rolled_tile_runs(int r0, int shift, int N) {
-  TileRuns t;
-  t.valid = N - r0 < kTileRows ? N - r0 : kTileRows;
-  long long s = static_cast<long long>(r0) + shift;
-  t.start = static_cast<int>(s >= N ? s - N : s);
-  const int to_end = N - t.start;
-  t.first = t.valid < to_end ? t.valid : to_end;
-  return t;
-}
-
-// Tile of original rows [t0, t0 + 128): the rolled rows they occupy in a head with roll
-// `shift` are (t - shift) mod N, i.e. the tile is the rolled tile starting at
-// (t0 - shift) mod N read with the inverse roll. Returns the same run structure in rolled
-// coordinates: rows [0, first) are rolled rows [start, start + first), rows [first, valid)
-// are rolled rows [0, valid - first).
-__host__ __device__ inline TileRuns original_tile_runs(int t0, int shift, int N) {
-  const int inv = shift == 0 ? 0 : N - shift;
-  return rolled_tile_runs(t0, inv, N);
-}
-
 // No split of the wrap group (see group_begin).
 constexpr int kNoWrapSplit = 0x7fffffff;
+
+// The remap of one head. Rolled row r holds original token
+//     t = (r + shift) mod N                                   (Algorithm 1's roll)
+// and, with `front` (the pages' Variant 3, Table 8: the wrapped tokens swap places with the
+// front of the last group), the last rolled group [N - G, N) lists tokens 0..shift-1 first
+// and N - G + shift..N - 1 after them:
+//     t = r + shift        for r < N - G
+//     t = r - (N - G)      for N - G <= r < N - G + shift
+//     t = r                for r >= N - G + shift.
+// Both are piecewise t = r + const over at most three ranges of r, and so is the inverse.
+struct HeadRemap {
+  int N, G, shift, front;
+  __host__ __device__ __forceinline__ int token(int r) const {
+    if (front) return r < N - G ? r + shift : (r < N - G + shift ? r - (N - G) : r);
+    const int t = r + shift;
+    return t >= N ? t - N : t;
+  }
+  __host__ __device__ __forceinline__ int rolled(int t) const {
+    if (front) return t < shift ? t + (N - G) : (t < N - G + shift ? t - shift : t);
+    const int r = t - shift;
+    return r < 0 ? r + N : r;
+  }
+  // Rows where token(r) (rolled(t) when `inverse`) stops being r + const.
+  __host__ __device__ __forceinline__ int breaks(bool inverse, int (&br)[2]) const {
+    if (shift == 0) return 0;
+    if (!front) {
+      br[0] = inverse ? shift : N - shift;
+      return 1;
+    }
+    br[0] = inverse ? shift : N - G;
+    br[1] = N - G + shift;
+    return 2;
+  }
+};
+
+__host__ __device__ __forceinline__ HeadRemap head_remap(int N, int G, int shift, int front) {
+  HeadRemap m;
+  m.N = N;
+  m.G = G;
+  m.shift = shift;
+  m.front = shift > 0 ? front : 0;
+  return m;
+}
+
+// Rows [x0, x0 + len) (clipped to the sequence) of one side of the remap as at most three
+// runs, each contiguous on the other side: row x0 + base_k + i maps to src[k] + i for
+// i < len[k], base_k = len[0] + ... + len[k-1]. Rows [valid, len) of the range are past the
+// end of the sequence.
+struct Runs {
+  int n, valid;
+  int len[3], src[3];
+};
+// (Loops over the three slots are unrolled with constant indices so the arrays stay in
+// registers.)
+__host__ __device__ inline Runs remap_runs(const HeadRemap& m, bool inverse, int x0, int len) {
+  Runs t;
+  t.n = 0;
+  t.valid = m.N - x0 < len ? m.N - x0 : len;
+  if (!m.front) {
+    // the plain roll: the run that reaches the end of the sequence, then the one that wraps
+    const int sh = inverse ? (m.shift == 0 ? 0 : m.N - m.shift) : m.shift;
+    const int s0 = x0 + sh >= m.N ? x0 + sh - m.N : x0 + sh;
+    const int first = t.valid < m.N - s0 ? t.valid : m.N - s0;
+    t.n = first < t.valid ? 2 : 1;
+    t.len[0] = first;
+    t.src[0] = s0;
+    t.len[1] = t.valid - first;
+    t.src[1] = 0;
+    t.len[2] = 0;
+    t.src[2] = 0;
+    return t;
+  }
+  int br[2] = {0, 0};
+  const int nb = m.breaks(inverse, br);
+  const int end = x0 + t.valid;
+  int pos = x0;
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {
+    t.len[k] = 0;
+    t.src[k] = 0;
+    if (pos < end) {
+      int nxt = end;
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+        if (i < nb && br[i] > pos && br[i] < nxt) nxt = br[i];
+      t.len[k] = nxt - pos;
+      t.src[k] = inverse ? m.rolled(pos) : m.token(pos);
+      t.n = k + 1;
+      pos = nxt;
+    }
+  }
+  return t;
+}
+// The 128-row rolled tile at r0 as runs of original tokens (tile loads, output rows).
+__host__ __device__ inline Runs rolled_runs(const HeadRemap& m, int r0) {
+  return remap_runs(m, false, r0, kTileRows);
+}
+// The original tile [t0, t0 + 128) as runs of rolled rows.
+__host__ __device__ inline Runs token_runs(const HeadRemap& m, int t0) {
+  return remap_runs(m, true, t0, kTileRows);
+}
+// The original tile [t0, t0 + 128) itself (a single run).
+__host__ __device__ inline Runs identity_runs(int t0, int N) {
+  Runs t;
+  t.n = 1;
+  t.valid = N - t0 < kTileRows ? N - t0 : kTileRows;
+  t.len[0] = t.valid;
+  t.src[0] = t0;
+  return t;
+}
 
 // First rolled row of the group containing rolled row r, and one past its last row. With a
 // wrap split W < N (the pages' Variant 2, Table 8: in the shifted heads the tokens the roll
@@ -68,73 +151,195 @@ __host__ __device__ inline int group_end(int r, int G, int W = kNoWrapSplit) {
   return (r < W && e > W) ? W : e;
 }
 
-// Query tiles (rolled, 128 rows) of a query head with roll `sh` that can see the original
-// kv rows [t0, t0 + 128): up to two disjoint index ranges, [r0a, r0b] then [r1a, r1b].
-// A kv row at rolled position r is seen by the query rows [r, end of r's group).
-struct QTileRanges {
-  int r0a, r0b, r1a, r1b;
+// Up to three ranges of tile indices [a[i], b[i]], listed in order, no index twice.
+struct TileList {
+  int n;
+  int a[3], b[3];
   __host__ __device__ __forceinline__ int count() const {
-    return (r0b - r0a + 1) + (r1b >= r1a ? r1b - r1a + 1 : 0);
+    int c = 0;
+#pragma unroll
+    for (int i = 0; i < 3; ++i)
+      if (i < n) c += b[i] - a[i] + 1;
+    return c;
   }
-  __host__ __device__ __forceinline__ int at(int i) const {
-    const int n0 = r0b - r0a + 1;
-    return i < n0 ? r0a + i : r1a + (i - n0);
+  __host__ __device__ __forceinline__ int at(int k) const {
+    int r = -1;
+#pragma unroll
+    for (int i = 0; i < 3; ++i) {
+      const int c = b[i] - a[i] + 1;
+      if (i < n && r < 0) {
+        if (k < c) r = a[i] + k;
+        else k -= c;
+      }
+    }
+    return r;
+  }
+  // Position of tile `t` in the list, or -1.
+  __host__ __device__ __forceinline__ int index_of(int t) const {
+    int k = 0, r = -1;
+#pragma unroll
+    for (int i = 0; i < 3; ++i) {
+      if (i < n && r < 0) {
+        if (t >= a[i] && t <= b[i]) r = k + (t - a[i]);
+        k += b[i] - a[i] + 1;
+      }
+    }
+    return r;
+  }
+  __host__ __device__ __forceinline__ bool has(int t) const { return index_of(t) >= 0; }
+  // Append [lo, hi] minus the tiles already listed. Ranges built from disjoint contiguous
+  // runs of rows overlap earlier ranges only in their end tiles, so trimming the ends is
+  // enough (a range that would still overlap inside is not added; the index tests check
+  // that this never happens).
+  __host__ __device__ __forceinline__ void append(int lo, int hi) {
+#pragma unroll
+    for (int pass = 0; pass < 3; ++pass)
+#pragma unroll
+      for (int i = 0; i < 3; ++i)
+        if (i < n) {
+          if (lo >= a[i] && lo <= b[i]) lo = b[i] + 1;
+          if (hi >= a[i] && hi <= b[i]) hi = a[i] - 1;
+        }
+    if (lo > hi) return;
+#pragma unroll
+    for (int i = 0; i < 3; ++i)
+      if (i < n && a[i] <= hi && b[i] >= lo) return;
+    bool done = false;
+#pragma unroll
+    for (int i = 0; i < 3; ++i)
+      if (i + 1 == n && b[i] + 1 == lo) {
+        b[i] = hi;
+        done = true;
+      }
+    if (done) return;
+#pragma unroll
+    for (int i = 0; i < 3; ++i)
+      if (i == n) {
+        a[i] = lo;
+        b[i] = hi;
+      }
+    if (n < 3) ++n;
   }
 };
 
-__host__ __device__ inline QTileRanges kv_tile_qtiles(int t0, int sh, int N, int G,
+// Query tiles (rolled, 128 rows) of a query head that can see the original kv rows
+// [t0, t0 + 128), in increasing order. A kv row at rolled position r is seen by the query rows
+// [r, end of r's group), so a run [r0, r1] of rolled kv rows is seen by the query tiles
+// r0 / 128 .. (group_end(r1) - 1) / 128.
+using QTileRanges = TileList;
+__host__ __device__ inline QTileRanges kv_tile_qtiles(const HeadRemap& m, int t0,
                                                       int W = kNoWrapSplit) {
-  const TileRuns tr = original_tile_runs(t0, sh, N);
-  // Run A: rolled rows [start, start + first) -> query rows [start, end of group).
-  const int a0 = tr.start / kTileRows;
-  const int a1 = (group_end(tr.start + tr.first - 1, G, W) - 1) / kTileRows;
-  QTileRanges q;
-  if (tr.valid > tr.first) {
-    // Run B: rolled rows [0, valid - first) -> query rows [0, end of that group).
-    const int b1 = (group_end(tr.valid - tr.first - 1, G, W) - 1) / kTileRows;
-    if (b1 + 1 >= a0) {
-      q.r0a = 0; q.r0b = a1 > b1 ? a1 : b1; q.r1a = 1; q.r1b = 0;
+  const Runs tr = token_runs(m, t0);
+  if (!m.front) {
+    // run A: rolled rows [src0, src0 + len0); run B (after the wrap): rolled rows from 0
+    QTileRanges q;
+    const int a0 = tr.src[0] / kTileRows;
+    const int a1 = (group_end(tr.src[0] + tr.len[0] - 1, m.G, W) - 1) / kTileRows;
+    q.a[1] = 0; q.b[1] = -1; q.a[2] = 0; q.b[2] = -1;
+    if (tr.n == 2) {
+      const int b1 = (group_end(tr.len[1] - 1, m.G, W) - 1) / kTileRows;
+      if (b1 + 1 >= a0) {
+        q.n = 1; q.a[0] = 0; q.b[0] = a1 > b1 ? a1 : b1;
+      } else {
+        q.n = 2; q.a[0] = 0; q.b[0] = b1; q.a[1] = a0; q.b[1] = a1;
+      }
     } else {
-      q.r0a = 0; q.r0b = b1; q.r1a = a0; q.r1b = a1;
+      q.n = 1; q.a[0] = a0; q.b[0] = a1;
     }
-  } else {
-    q.r0a = a0; q.r0b = a1; q.r1a = 1; q.r1b = 0;
+    return q;
+  }
+  constexpr int kNone = 0x7fffffff;   // sorts after every real range
+  int lo[3], hi[3];
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {
+    lo[k] = k < tr.n ? tr.src[k] / kTileRows : kNone;
+    hi[k] = k < tr.n ? (group_end(tr.src[k] + tr.len[k] - 1, m.G, W) - 1) / kTileRows : kNone;
+  }
+  // sort the (at most three) ranges by start, then merge overlapping or adjacent ones
+#pragma unroll
+  for (int i = 0; i < 3; ++i)
+#pragma unroll
+    for (int j = i + 1; j < 3; ++j)
+      if (lo[j] < lo[i]) {
+        const int x = lo[i], y = hi[i];
+        lo[i] = lo[j]; hi[i] = hi[j];
+        lo[j] = x; hi[j] = y;
+      }
+  QTileRanges q;
+  q.n = 0;
+#pragma unroll
+  for (int i = 0; i < 3; ++i) {
+    q.a[i] = 0;
+    q.b[i] = -1;
+  }
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {
+    if (lo[k] == kNone) continue;
+    bool merged = false;
+#pragma unroll
+    for (int i = 0; i < 3; ++i)
+      if (i + 1 == q.n && lo[k] <= q.b[i] + 1) {
+        if (hi[k] > q.b[i]) q.b[i] = hi[k];
+        merged = true;
+      }
+    if (merged) continue;
+#pragma unroll
+    for (int i = 0; i < 3; ++i)
+      if (i == q.n) {
+        q.a[i] = lo[k];
+        q.b[i] = hi[k];
+      }
+    ++q.n;
   }
   return q;
 }
 
-// Original kv tiles that rolled query tile qt (head roll sh) reads. Its rows see the rolled
-// kv rows [start of the group of its first row, its last row]; under the roll these are a
-// contiguous range of original rows modulo N, covered by `count` consecutive original tiles
-// (indices taken modulo the tile count T) starting at `first`.
-struct KvSpan {
-  int first, count;
-};
-__host__ __device__ inline KvSpan qtile_kv_span(int qt, int sh, int N, int G,
+// Original kv tiles that rolled query tile qt reads: its rows see the rolled kv rows
+// [start of the group of its first row, its last row]; these map to at most three runs of
+// original rows, listed in rolled order, each run's tiles once.
+using KvSpan = TileList;
+__host__ __device__ inline KvSpan qtile_kv_span(const HeadRemap& m, int qt,
                                                int W = kNoWrapSplit) {
-  const int T = (N + kTileRows - 1) / kTileRows;
   const int r0 = qt * kTileRows;
-  const int last = r0 + kTileRows - 1 < N - 1 ? r0 + kTileRows - 1 : N - 1;
-  const int gb = group_begin(r0, G, W);
-  const int len = last - gb + 1;
-  const long long o = static_cast<long long>(gb) + sh;
-  const int o0 = static_cast<int>(o >= N ? o - N : o);
-  int count;
-  if (o0 + len <= N)
-    count = (o0 + len - 1) / kTileRows - o0 / kTileRows + 1;
-  else
-    count = (T - o0 / kTileRows) + (o0 + len - N - 1) / kTileRows + 1;
+  const int last = r0 + kTileRows - 1 < m.N - 1 ? r0 + kTileRows - 1 : m.N - 1;
+  const int gb = group_begin(r0, m.G, W);
   KvSpan s;
-  s.first = o0 / kTileRows;
-  s.count = count < T ? count : T;
+  if (!m.front) {
+    // under the plain roll the rows map to one cyclic range of original rows
+    const int T = (m.N + kTileRows - 1) / kTileRows;
+    const int len = last - gb + 1;
+    const int o0 = gb + m.shift >= m.N ? gb + m.shift - m.N : gb + m.shift;
+    int count = o0 + len <= m.N ? (o0 + len - 1) / kTileRows - o0 / kTileRows + 1
+                                : (T - o0 / kTileRows) + (o0 + len - m.N - 1) / kTileRows + 1;
+    count = count < T ? count : T;
+    const int first = o0 / kTileRows;
+    s.a[0] = first;
+    s.b[0] = first + count - 1 < T - 1 ? first + count - 1 : T - 1;
+    s.a[1] = 0;
+    s.b[1] = first + count - 1 - T;   // -1 (empty) when the range does not wrap
+    s.a[2] = 0;
+    s.b[2] = -1;
+    s.n = s.b[1] >= 0 ? 2 : 1;
+    return s;
+  }
+  const Runs tr = remap_runs(m, false, gb, last - gb + 1);
+  s.n = 0;
+#pragma unroll
+  for (int i = 0; i < 3; ++i) {
+    s.a[i] = 0;
+    s.b[i] = -1;
+  }
+#pragma unroll
+  for (int k = 0; k < 3; ++k)
+    if (k < tr.n) s.append(tr.src[k] / kTileRows, (tr.src[k] + tr.len[k] - 1) / kTileRows);
   return s;
 }
 
 // Slots of the bf16 dS tiles that the dK/dV kernel hands to the dQ pass: one 128 x 128 tile
-// (32 KB) per (query tile qt, original kv tile first + i), i < count, at slot base(qt) + i of
-// its (batch, query head). When groups and roll are tile-aligned, count = qt mod (G/128) + 1
-// and the slots are packed (a triangle per group); otherwise every query tile gets `stride`
-// slots, the largest count of any query tile.
+// (32 KB) per (query tile qt, kv tile span.at(i)), i < span.count(), at slot base(qt) + i of
+// its (batch, query head). When groups and roll are tile-aligned (and the last group is not
+// split or reordered), count = qt mod (G/128) + 1 and the slots are packed (a triangle per
+// group); otherwise every query tile gets `stride` slots, the largest count of any query tile.
 struct DsSlots {
   int aligned;          // G and every head's roll are multiples of the tile
   int gt;               // G / 128 (aligned case)
@@ -148,20 +353,23 @@ struct DsSlots {
     return static_cast<long long>(qt) * stride;
   }
 };
-inline DsSlots ds_slots(int N, int G, int shifted_heads, int shift, int W = kNoWrapSplit) {
+inline DsSlots ds_slots(int N, int G, int shifted_heads, int shift, int W = kNoWrapSplit,
+                        int front = 0) {
   DsSlots d;
   const int T = (N + kTileRows - 1) / kTileRows;
   const int sh = shifted_heads ? shift : 0;
   const int w = shifted_heads ? W : kNoWrapSplit;
-  d.aligned = (G % kTileRows == 0 && sh % kTileRows == 0 && w >= N) ? 1 : 0;
+  const int fr = shifted_heads ? front : 0;
+  d.aligned = (G % kTileRows == 0 && sh % kTileRows == 0 && w >= N && !fr) ? 1 : 0;
   d.gt = G / kTileRows;
   d.stride = 0;
   if (d.aligned) {
     d.per_head = static_cast<long long>(N / G) * d.gt * (d.gt + 1) / 2;
   } else {
+    const HeadRemap m0 = head_remap(N, G, 0, 0), m1 = head_remap(N, G, sh, fr);
     for (int qt = 0; qt < T; ++qt) {
-      const int c0 = qtile_kv_span(qt, 0, N, G).count;
-      const int c1 = qtile_kv_span(qt, sh, N, G, w).count;
+      const int c0 = qtile_kv_span(m0, qt).count();
+      const int c1 = qtile_kv_span(m1, qt, w).count();
       const int c = c0 > c1 ? c0 : c1;
       d.stride = c > d.stride ? c : d.stride;
     }

@@ -44,21 +44,29 @@ DeviceState g_dev[kMaxDevices];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
 
-template <int D>
-cudaError_t set_smem_attrs() {
+template <int D, bool kFront>
+cudaError_t set_smem_attrs_variant() {
   cudaError_t e;
-  e = cudaFuncSetAttribute(s2::s2_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           s2::FwdLayout<D>::kLaunchBytes);
+  e = cudaFuncSetAttribute(s2::s2_fwd_kernel<D, kFront>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, s2::FwdLayout<D>::kLaunchBytes);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(s2::s2_bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           s2::DkdvLayout<D>::kLaunchBytes);
+  e = cudaFuncSetAttribute(s2::s2_bwd_dkdv_kernel<D, kFront>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, s2::DkdvLayout<D>::kLaunchBytes);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(s2::s2_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           s2::DqLayout<D>::kLaunchBytes);
+  e = cudaFuncSetAttribute(s2::s2_bwd_dq_kernel<D, kFront>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, s2::DqLayout<D>::kLaunchBytes);
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(s2::s2_bwd_dq_ds_kernel<D>,
+  return cudaFuncSetAttribute(s2::s2_bwd_dq_ds_kernel<D, kFront>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize,
                               s2::DqDsLayout<D>::kLaunchBytes);
+}
+// Every kernel exists twice: with the plain-roll index code only, and with the Variant 3
+// reordering compiled in (S2ATTN_FLAG_WRAP_FRONT_FIRST), so the common case pays nothing
+// for the general remap.
+template <int D>
+cudaError_t set_smem_attrs() {
+  const cudaError_t e = set_smem_attrs_variant<D, false>();
+  return e != cudaSuccess ? e : set_smem_attrs_variant<D, true>();
 }
 
 // Per-device one-time set-up (with that device current): the device address of the error
@@ -152,6 +160,7 @@ enum TensorId { T_Q = 0, T_K, T_V, T_O, T_DO, T_DQ, T_DK, T_DV, T_COUNT };
 struct Shape {
   int B, Hq, Hkv, N, d, G, shb, shift;
   int wrap;   // the shifted heads' wrap split (Variant 2), or s2::kNoWrapSplit
+  int front;  // Variant 3: the shifted heads' last group lists the wrapped tokens first
   long long sb[T_COUNT], st[T_COUNT];
   int heads(int t) const { return (t == T_K || t == T_V || t == T_DK || t == T_DV) ? Hkv : Hq; }
   void set_contiguous() {
@@ -172,7 +181,7 @@ unsigned int* ws_sched(const void* workspace, const Shape& sh) {
 }
 
 s2::DsSlots ds_layout(const Shape& sh) {
-  return s2::ds_slots(sh.N, sh.G, sh.shb < sh.Hq, sh.shift, sh.wrap);
+  return s2::ds_slots(sh.N, sh.G, sh.shb < sh.Hq, sh.shift, sh.wrap, sh.front);
 }
 size_t ds_bytes_per_kv_head(const Shape& sh) {
   const s2::DsSlots sl = ds_layout(sh);
@@ -204,14 +213,15 @@ s2attn_status check_shape(int B, int Hq, int Hkv, int N, int d, int G, float sca
   if (s % 8 != 0) return S2ATTN_ERR_UNSUPPORTED;
   const long long rows = static_cast<long long>(B) * (Hq > Hkv ? Hq : Hkv) * ((N + 127) / 128);
   if (rows >= (1ll << 31)) return S2ATTN_ERR_UNSUPPORTED;
-  if (flags & ~S2ATTN_FLAG_WRAP_OWN_GROUP) return S2ATTN_ERR_INVALID_ARG;
-  int wrap = s2::kNoWrapSplit;
-  if (flags & S2ATTN_FLAG_WRAP_OWN_GROUP) {
-    // the wrap group exists when some head is rolled by 0 < shift < G
-    if (shift_head_begin >= Hq || s <= 0 || s >= G) return S2ATTN_ERR_INVALID_ARG;
-    wrap = N - static_cast<int>(s);
-  }
-  out = Shape{B, Hq, Hkv, N, d, G, shift_head_begin, static_cast<int>(s), wrap, {}, {}};
+  constexpr int kVariants = S2ATTN_FLAG_WRAP_OWN_GROUP | S2ATTN_FLAG_WRAP_FRONT_FIRST;
+  if (flags & ~kVariants) return S2ATTN_ERR_INVALID_ARG;
+  if ((flags & kVariants) == kVariants) return S2ATTN_ERR_INVALID_ARG;   // alternatives
+  // the wrap group exists when some head is rolled by 0 < shift < G
+  if ((flags & kVariants) && (shift_head_begin >= Hq || s <= 0 || s >= G))
+    return S2ATTN_ERR_INVALID_ARG;
+  const int wrap = (flags & S2ATTN_FLAG_WRAP_OWN_GROUP) ? N - static_cast<int>(s) : s2::kNoWrapSplit;
+  const int front = (flags & S2ATTN_FLAG_WRAP_FRONT_FIRST) ? 1 : 0;
+  out = Shape{B, Hq, Hkv, N, d, G, shift_head_begin, static_cast<int>(s), wrap, front, {}, {}};
   out.set_contiguous();
   return S2ATTN_OK;
 }
@@ -233,13 +243,18 @@ s2attn_status launch_fwd(const Shape& sh, const void* q, const void* k, const vo
   p.B = sh.B; p.Hq = sh.Hq; p.Hkv = sh.Hkv; p.N = sh.N; p.G = sh.G;
   p.shift_head_begin = sh.shb; p.shift = sh.shift;
   p.wrap = sh.wrap;
+  p.front = sh.front;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.err = err;
   p.timeout_ns = g_timeout_ns.load();
   const unsigned units = static_cast<unsigned>(sh.B) * sh.Hq * s2::query_pairs_per_head(sh.N);
   const unsigned grid = units < static_cast<unsigned>(num_sms) ? units : static_cast<unsigned>(num_sms);
-  s2::s2_fwd_kernel<D><<<grid, s2::FwdLayout<D>::kThreads, s2::FwdLayout<D>::kLaunchBytes, stream>>>(
-      mq.m128, mq.m8, mk.m128, mk.m8, mv.m128, mv.m8, p);
+  if (sh.front)
+    s2::s2_fwd_kernel<D, true><<<grid, s2::FwdLayout<D>::kThreads, s2::FwdLayout<D>::kLaunchBytes,
+                                 stream>>>(mq.m128, mq.m8, mk.m128, mk.m8, mv.m128, mv.m8, p);
+  else
+    s2::s2_fwd_kernel<D, false><<<grid, s2::FwdLayout<D>::kThreads, s2::FwdLayout<D>::kLaunchBytes,
+                                  stream>>>(mq.m128, mq.m8, mk.m128, mk.m8, mv.m128, mv.m8, p);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? S2ATTN_OK : cuda_fail(e, "s2_fwd_kernel launch");
 }
@@ -256,6 +271,7 @@ s2::BwdParams bwd_params(const Shape& sh, float scale, const void* workspace, vo
   p.B = sh.B; p.Hq = sh.Hq; p.Hkv = sh.Hkv; p.N = sh.N; p.G = sh.G;
   p.shift_head_begin = sh.shb; p.shift = sh.shift;
   p.wrap = sh.wrap;
+  p.front = sh.front;
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.err = err;
@@ -317,12 +333,24 @@ s2attn_status launch_grad(const Shape& sh, const void* q, const void* k, const v
       return s;
     const unsigned units = static_cast<unsigned>(sh.B) * p.kvh_count * tiles;
     const unsigned grid = units < static_cast<unsigned>(num_sms) ? units : static_cast<unsigned>(num_sms);
-    s2::s2_bwd_dkdv_kernel<D><<<grid, s2::DkdvLayout<D>::kThreads, s2::DkdvLayout<D>::kLaunchBytes, stream>>>(
-        mq.m128, mq.m8, mk.m128, mk.m8, mv.m128, mv.m8, mo.m128, mo.m8, mdk.m128, mdv.m128, p);
+    if (sh.front)
+      s2::s2_bwd_dkdv_kernel<D, true><<<grid, s2::DkdvLayout<D>::kThreads,
+                                        s2::DkdvLayout<D>::kLaunchBytes, stream>>>(
+          mq.m128, mq.m8, mk.m128, mk.m8, mv.m128, mv.m8, mo.m128, mo.m8, mdk.m128, mdv.m128, p);
+    else
+      s2::s2_bwd_dkdv_kernel<D, false><<<grid, s2::DkdvLayout<D>::kThreads,
+                                         s2::DkdvLayout<D>::kLaunchBytes, stream>>>(
+          mq.m128, mq.m8, mk.m128, mk.m8, mv.m128, mv.m8, mo.m128, mo.m8, mdk.m128, mdv.m128, p);
   } else {
     const unsigned grid = static_cast<unsigned>(sh.B) * sh.Hq * tiles;
-    s2::s2_bwd_dq_kernel<D><<<grid, s2::DqLayout<D>::kThreads, s2::DqLayout<D>::kLaunchBytes, stream>>>(
-        mq.m128, mq.m8, mk.m128, mk.m8, mv.m128, mv.m8, mo.m128, mo.m8, p);
+    if (sh.front)
+      s2::s2_bwd_dq_kernel<D, true><<<grid, s2::DqLayout<D>::kThreads, s2::DqLayout<D>::kLaunchBytes,
+                                      stream>>>(mq.m128, mq.m8, mk.m128, mk.m8, mv.m128, mv.m8,
+                                                mo.m128, mo.m8, p);
+    else
+      s2::s2_bwd_dq_kernel<D, false><<<grid, s2::DqLayout<D>::kThreads, s2::DqLayout<D>::kLaunchBytes,
+                                       stream>>>(mq.m128, mq.m8, mk.m128, mk.m8, mv.m128, mv.m8,
+                                                 mo.m128, mo.m8, p);
   }
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? S2ATTN_OK
@@ -342,8 +370,12 @@ s2attn_status launch_dq_ds(const Shape& sh, const void* k, void* dq, float scale
   const unsigned units = static_cast<unsigned>(sh.B) * kvh_count * (sh.Hq / sh.Hkv) *
                          ((sh.N + 127) / 128);
   const unsigned grid = units < static_cast<unsigned>(num_sms) ? units : static_cast<unsigned>(num_sms);
-  s2::s2_bwd_dq_ds_kernel<D><<<grid, s2::DqDsLayout<D>::kThreads, s2::DqDsLayout<D>::kLaunchBytes,
-                               stream>>>(mk.m128, mk.m8, p);
+  if (sh.front)
+    s2::s2_bwd_dq_ds_kernel<D, true><<<grid, s2::DqDsLayout<D>::kThreads,
+                                       s2::DqDsLayout<D>::kLaunchBytes, stream>>>(mk.m128, mk.m8, p);
+  else
+    s2::s2_bwd_dq_ds_kernel<D, false><<<grid, s2::DqDsLayout<D>::kThreads,
+                                        s2::DqDsLayout<D>::kLaunchBytes, stream>>>(mk.m128, mk.m8, p);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? S2ATTN_OK : cuda_fail(e, "s2_bwd_dq_ds_kernel launch");
 }

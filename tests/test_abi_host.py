@@ -125,13 +125,24 @@ def test_bwd_rejects(lib):
 SHIM = r"""
 #include "s2_tiles.cuh"
 extern "C" {
-void rolled_runs(int r0, int shift, int N, int* o) {
-  s2::TileRuns t = s2::rolled_tile_runs(r0, shift, N); o[0]=t.valid; o[1]=t.first; o[2]=t.start; }
-void original_runs(int t0, int shift, int N, int* o) {
-  s2::TileRuns t = s2::original_tile_runs(t0, shift, N); o[0]=t.valid; o[1]=t.first; o[2]=t.start; }
-int qtiles(int t0, int sh, int N, int G, int W, int* o) {
-  s2::QTileRanges q = s2::kv_tile_qtiles(t0, sh, N, G, W);
+static void put_runs(const s2::Runs& t, int* o) {
+  o[0] = t.n; o[1] = t.valid;
+  for (int k = 0; k < t.n; ++k) { o[2 + 2 * k] = t.len[k]; o[3 + 2 * k] = t.src[k]; } }
+void rolled_runs(int r0, int shift, int N, int G, int front, int* o) {
+  put_runs(s2::rolled_runs(s2::head_remap(N, G, shift, front), r0), o); }
+void token_runs(int t0, int shift, int N, int G, int front, int* o) {
+  put_runs(s2::token_runs(s2::head_remap(N, G, shift, front), t0), o); }
+int qtiles(int t0, int sh, int N, int G, int W, int front, int* o) {
+  s2::QTileRanges q = s2::kv_tile_qtiles(s2::head_remap(N, G, sh, front), t0, W);
   int n = q.count(); for (int i = 0; i < n; ++i) o[i] = q.at(i); return n; }
+int kvspan(int qt, int sh, int N, int G, int W, int front, int* o) {
+  s2::KvSpan s = s2::qtile_kv_span(s2::head_remap(N, G, sh, front), qt, W);
+  int n = s.count(); for (int i = 0; i < n; ++i) o[i] = s.at(i);
+  for (int i = 0; i < n; ++i) if (s.index_of(o[i]) != i) return -1;
+  return n; }
+long long dsslots(int N, int G, int shifted, int shift, int W, int front, int qt) {
+  s2::DsSlots d = s2::ds_slots(N, G, shifted, shift, W, front);
+  return qt < 0 ? d.per_head : d.base(qt); }
 void qcoords(int bid, int B, int Hq, int N, int G, int* o) {
   s2::query_tile_coords(bid, B, Hq, N, G, o[0], o[1], o[2]); }
 void paircoords(int bid, int B, int Hq, int N, int G, int* o) {
@@ -145,11 +156,6 @@ void paircoords_chunked(int bid, int B, int Hq, int N, int G, int chunk, int* o)
 void kvcoords_chunked(int bid, int B, int Hq, int Hkv, int N, int G, int shb, int sh, int chunk,
                       int* o) {
   s2::kv_tile_coords_chunked(bid, B, Hq, Hkv, N, G, shb, sh, chunk, o[0], o[1], o[2]); }
-void kvspan(int qt, int sh, int N, int G, int W, int* o) {
-  s2::KvSpan s = s2::qtile_kv_span(qt, sh, N, G, W); o[0] = s.first; o[1] = s.count; }
-long long dsslots(int N, int G, int shifted, int shift, int W, int qt) {
-  s2::DsSlots d = s2::ds_slots(N, G, shifted, shift, W);
-  return qt < 0 ? d.per_head : d.base(qt); }
 }
 """
 
@@ -162,7 +168,9 @@ def shim(tmp_path_factory):
     so = d / "shim.so"
     subprocess.run(["g++", "-O1", "-shared", "-fPIC", "-std=c++17", "-I", CSRC, str(src), "-o",
                     str(so)], check=True)
-    return ctypes.CDLL(str(so))
+    lib_ = ctypes.CDLL(str(so))
+    lib_.dsslots.restype = ctypes.c_longlong
+    return lib_
 
 
 NOWRAP = 0x7FFFFFFF   # no wrap split (the default variant)
@@ -174,51 +182,144 @@ def call4(fn, *args):
     return list(out)
 
 
+def runs_of(fn, *args):
+    """[(len, src), ...] and the valid row count of a Runs result."""
+    out = (ctypes.c_int * 8)()
+    fn(*args, out)
+    n, valid = out[0], out[1]
+    return [(out[2 + 2 * k], out[3 + 2 * k]) for k in range(n)], valid
+
+
+def listed(fn, *args):
+    out = (ctypes.c_int * 4096)()
+    n = fn(*args, out)
+    assert n >= 0, "index_of disagrees with at"
+    return list(out[:n])
+
+
 CASES = [(256, 64, 32), (8192, 2048, 1024), (320, 64, 32), (384, 192, 96), (200, 200, 0),
          (96, 32, 16), (1024, 1024, 512), (640, 128, 64), (2048, 512, 256), (448, 64, 8),
          (96, 96, 88), (768, 256, 640)]
+# (N, G, shift) with 0 < shift < G: the cases where Variants 2 and 3 exist
+SPLIT_CASES = [(256, 64, 32), (8192, 2048, 1024), (320, 64, 32), (384, 192, 96), (96, 32, 16),
+               (640, 128, 64), (2048, 512, 256), (448, 64, 8), (96, 96, 88), (1024, 256, 128),
+               (512, 128, 40), (1024, 1024, 512), (256, 256, 200), (136, 136, 8)]
+VARIANT_CASES = ([(n, g, s, "default") for n, g, s in CASES] +
+                 [(n, g, s, v) for n, g, s in SPLIT_CASES for v in ("v2", "v3")])
 
 
-@pytest.mark.parametrize("N,G,shift", CASES)
-def test_rolled_runs_match_literal_roll(shim, N, G, shift):
-    tok = orc.rolled_token_index(N, G, shift).reshape(-1)   # rolled row -> original token
-    for r0 in range(0, N, 128):
-        valid, first, start = call4(shim.rolled_runs, r0, shift, N)[:3]
-        assert valid == min(128, N - r0)
-        got = [start + i for i in range(first)] + [i - first for i in range(first, valid)]
-        assert got == list(tok[r0:r0 + valid])
-        assert first % 8 == 0 and valid % 8 == 0 and start % 8 == 0
+def rolled_tokens(N, G, shift, variant):
+    """Original token of every rolled row of a shifted head, from the oracle's own steps:
+    the roll of key line 1, then (Variant 3) the oracle's reordering of the last group."""
+    tok = orc.rolled_token_index(N, G, shift)
+    if variant == "v3":
+        tok = orc._swap_wrap_front(tok[:, :, None], N, G, 0, shift, True)[:, :, 0]
+    return tok.reshape(-1)
 
 
-@pytest.mark.parametrize("N,G,shift", CASES)
-def test_original_runs_invert_the_roll(shim, N, G, shift):
-    tok = orc.rolled_token_index(N, G, shift).reshape(-1)
+def groups(N, G, shift, variant):
+    """group id of every rolled row (Variant 2 splits the last group at N - shift)."""
+    gid = np.arange(N) // G
+    if variant == "v2":
+        gid = np.where(np.arange(N) >= N - shift, N // G, gid)
+    return gid
+
+
+def variant_args(N, shift, variant):
+    return (N - shift if variant == "v2" else NOWRAP), (1 if variant == "v3" else 0)
+
+
+@pytest.mark.parametrize("N,G,shift,variant", VARIANT_CASES)
+def test_rolled_runs_match_the_oracle(shim, N, G, shift, variant):
+    """Runs of a rolled tile give exactly the oracle's token of every row; runs of an
+    original tile give the inverse; every run starts and ends on an 8-row boundary."""
+    tok = rolled_tokens(N, G, shift, variant)
     rolled_of = np.empty(N, dtype=np.int64)
     rolled_of[tok] = np.arange(N)
-    for t0 in range(0, N, 128):
-        valid, first, start = call4(shim.original_runs, t0, shift, N)[:3]
-        got = [start + i for i in range(first)] + [i - first for i in range(first, valid)]
-        assert got == list(rolled_of[t0:t0 + valid])
+    front = 1 if variant == "v3" else 0
+    for x0 in range(0, N, 128):
+        for fn, ref in ((shim.rolled_runs, tok), (shim.token_runs, rolled_of)):
+            runs, valid = runs_of(fn, x0, shift, N, G, front)
+            assert valid == min(128, N - x0)
+            got = [src + i for ln, src in runs for i in range(ln)]
+            assert got == list(ref[x0:x0 + valid])
+            assert all(ln % 8 == 0 and src % 8 == 0 for ln, src in runs)
+            assert 1 <= len(runs) <= 3
 
 
-@pytest.mark.parametrize("N,G,shift", CASES)
-def test_kv_tile_query_tiles_exact(shim, N, G, shift):
-    """Brute force: q tile Qt is visited for kv tile t0 iff some rolled query row in Qt attends
-    some kv row of the tile (same rolled group, query not before key)."""
-    tok = orc.rolled_token_index(N, G, shift).reshape(-1)
+@pytest.mark.parametrize("N,G,shift,variant", VARIANT_CASES)
+def test_tile_sets_exact(shim, N, G, shift, variant):
+    """Brute force over rows: the query tiles each kv tile visits (increasing, each once) and
+    the kv tiles each query tile reads (each once) are exactly the tiles holding a (query,
+    key) pair of the same group with the key not after the query in rolled order."""
+    nt = (N + 127) // 128
+    W, front = variant_args(N, shift, variant)
+    tok = rolled_tokens(N, G, shift, variant)
     rolled_of = np.empty(N, dtype=np.int64)
     rolled_of[tok] = np.arange(N)
-    out = (ctypes.c_int * 4096)()
-    for t0 in range(0, N, 128):
-        n = shim.qtiles(t0, shift, N, G, NOWRAP, out)
-        got = list(out[:n])
-        assert len(set(got)) == len(got)
+    gid = groups(N, G, shift, variant)
+    gend = np.empty(N, dtype=np.int64)      # one past the last rolled row of each row's group
+    for g in np.unique(gid):
+        rows = np.nonzero(gid == g)[0]
+        gend[rows] = rows.max() + 1
+    pairs = set()
+    for t in range(nt):
+        got = listed(shim.qtiles, t * 128, shift, N, G, W, front)
+        assert got == sorted(set(got))
         want = set()
-        for t in range(t0, min(t0 + 128, N)):
-            rk = rolled_of[t]
-            ge = (rk // G + 1) * G
-            want.update(range(rk // 128, (ge - 1) // 128 + 1))
+        for tk in range(t * 128, min(t * 128 + 128, N)):
+            rk = rolled_of[tk]
+            want.update(range(rk // 128, (gend[rk] - 1) // 128 + 1))
         assert set(got) == want
+        pairs.update((qt, t) for qt in got)
+    for qt in range(nt):
+        got = listed(shim.kvspan, qt, shift, N, G, W, front)
+        assert len(set(got)) == len(got)
+        r0, last = qt * 128, min(qt * 128 + 127, N - 1)
+        gb = np.nonzero(gid == gid[r0])[0].min()
+        assert set(got) == {tok[r] // 128 for r in range(gb, last + 1)}
+        for t in got:
+            assert (qt, t) in pairs
+
+
+@pytest.mark.parametrize("N,G,shift,variant", VARIANT_CASES)
+def test_ds_slots_match_the_dkdv_pairs(shim, N, G, shift, variant):
+    """Every (query tile, kv tile) pair the dQ pass reads is one the dK/dV kernel visits and
+    vice versa, for both head kinds, and the slots of one head are distinct and inside
+    per_head."""
+    nt = (N + 127) // 128
+    W, front = variant_args(N, shift, variant)
+    per_head = shim.dsslots(N, G, 1, shift, W, front, -1)
+    for sh, w, fr in {(0, NOWRAP, 0), (shift, W if shift else NOWRAP, front if shift else 0)}:
+        visited = set()
+        for t in range(nt):
+            visited.update((qt, t) for qt in listed(shim.qtiles, t * 128, sh, N, G, w, fr))
+        read, slots = set(), set()
+        for qt in range(nt):
+            span = listed(shim.kvspan, qt, sh, N, G, w, fr)
+            base = shim.dsslots(N, G, 1, shift, W, front, qt)
+            assert base + len(span) <= per_head
+            read.update((qt, t) for t in span)
+            slots.update(base + i for i in range(len(span)))
+        assert read == visited
+        assert len(slots) == len(read)
+    if G % 128 == 0 and shift % 128 == 0 and variant == "default":
+        gt = G // 128
+        assert per_head == (N // G) * gt * (gt + 1) // 2
+
+
+@pytest.mark.parametrize("N,G,shift", [(102400, 25600, 12800), (32768, 8192, 4096)])
+def test_qtile_kv_span_large(shim, N, G, shift):
+    """The long-sequence workloads, sampled: spans are the kv tiles of the group start up to
+    the query tile, under the roll."""
+    nt = (N + 127) // 128
+    for sh in (0, shift):
+        for qt in list(range(0, nt, 37)) + [nt - 1]:
+            got = listed(shim.kvspan, qt, sh, N, G, NOWRAP, 0)
+            r0, last = qt * 128, min(qt * 128 + 127, N - 1)
+            gb = (r0 // G) * G
+            assert len(set(got)) == len(got)
+            assert set(got) == {((r + sh) % N) // 128 for r in range(gb, last + 1)}
 
 
 @pytest.mark.parametrize("B,Hq,N,G", [(1, 4, 256, 64), (2, 3, 8192, 2048), (1, 2, 384, 192),
@@ -264,105 +365,6 @@ def test_query_pair_order_is_a_permutation(shim, B, Hq, N, G):
     if G % 256 == 0 and G > 256:
         b, h, p = call4(shim.paircoords, 0, B, Hq, N, G)[:3]
         assert p % (G // 256) == G // 256 - 1
-
-
-@pytest.mark.parametrize("N,G,shift", CASES + [(102400, 25600, 12800), (32768, 8192, 4096)])
-def test_qtile_kv_span_exact(shim, N, G, shift):
-    """Brute force: the original kv tiles a rolled query tile reads are exactly the tiles
-    holding some kv row that one of its rows attends (same rolled group, key not after query),
-    listed once each from `first` on (indices modulo the tile count)."""
-    nt = (N + 127) // 128
-    for sh in {0, shift}:
-        for qt in range(nt) if N <= 8192 else list(range(0, nt, 37)) + [nt - 1]:
-            first, count = call4(shim.kvspan, qt, sh, N, G, NOWRAP)[:2]
-            got = [(first + i) % nt for i in range(count)]
-            assert len(set(got)) == count
-            r0, last = qt * 128, min(qt * 128 + 127, N - 1)
-            gb = (r0 // G) * G
-            want = {((r + sh) % N) // 128 for r in range(gb, last + 1)}
-            assert set(got) == want
-
-
-@pytest.mark.parametrize("N,G,shift", CASES)
-def test_ds_slots_match_the_dkdv_pairs(shim, N, G, shift):
-    """Every (query tile, kv tile) pair the dQ pass reads is one the dK/dV kernel visits, and
-    the slots of one head are distinct and inside per_head."""
-    nt = (N + 127) // 128
-    shim.dsslots.restype = ctypes.c_longlong
-    per_head = shim.dsslots(N, G, 1, shift, NOWRAP, -1)
-    out = (ctypes.c_int * 4096)()
-    for sh in {0, shift}:
-        visited = set()
-        for t in range(nt):
-            n = shim.qtiles(t * 128, sh, N, G, NOWRAP, out)
-            visited.update((qt, t) for qt in out[:n])
-        slots = set()
-        for qt in range(nt):
-            first, count = call4(shim.kvspan, qt, sh, N, G, NOWRAP)[:2]
-            base = shim.dsslots(N, G, 1, shift, NOWRAP, qt)
-            for i in range(count):
-                assert (qt, (first + i) % nt) in visited
-                slots.add(base + i)
-            assert base + count <= per_head
-        assert len(slots) == sum(call4(shim.kvspan, qt, sh, N, G, NOWRAP)[1] for qt in range(nt))
-    if G % 128 == 0 and shift % 128 == 0:
-        gt = G // 128
-        assert per_head == (N // G) * gt * (gt + 1) // 2
-
-
-V2_CASES = [(256, 64, 32), (8192, 2048, 1024), (320, 64, 32), (384, 192, 96), (96, 32, 16),
-            (640, 128, 64), (2048, 512, 256), (448, 64, 8), (96, 96, 88), (1024, 256, 128),
-            (512, 128, 40)]
-
-
-def _v2_group(r, N, G, W):
-    """Rolled rows of the causal group holding rolled row r when the wrapped tokens (rolled
-    rows [W, N), W = N - shift) form their own group (Table 8, Variant 2)."""
-    if r >= W:
-        return W, N
-    return (r // G) * G, min((r // G + 1) * G, W)
-
-
-@pytest.mark.parametrize("N,G,shift", V2_CASES)
-def test_variant2_tile_sets_exact(shim, N, G, shift):
-    """Brute force with the wrap split: the query tiles each kv tile visits, the kv tiles each
-    query tile reads, and that the two agree in both directions (every dS tile the dK/dV kernel
-    hands off lands inside the reading tile's span, and every span entry is written)."""
-    W = N - shift
-    nt = (N + 127) // 128
-    tok = orc.rolled_token_index(N, G, shift).reshape(-1)
-    rolled_of = np.empty(N, dtype=np.int64)
-    rolled_of[tok] = np.arange(N)
-    out = (ctypes.c_int * 4096)()
-    visited = set()
-    for t in range(nt):
-        n = shim.qtiles(t * 128, shift, N, G, W, out)
-        got = set(out[:n])
-        assert len(got) == n
-        want = set()
-        for tk in range(t * 128, min(t * 128 + 128, N)):
-            rk = rolled_of[tk]
-            want.update(range(rk // 128, (_v2_group(rk, N, G, W)[1] - 1) // 128 + 1))
-        assert got == want
-        visited.update((qt, t) for qt in got)
-    shim.dsslots.restype = ctypes.c_longlong
-    per_head = shim.dsslots(N, G, 1, shift, W, -1)
-    read, slots = set(), set()
-    for qt in range(nt):
-        first, count = call4(shim.kvspan, qt, shift, N, G, W)[:2]
-        got = [(first + i) % nt for i in range(count)]
-        assert len(set(got)) == count
-        r0, last = qt * 128, min(qt * 128 + 127, N - 1)
-        gb = _v2_group(r0, N, G, W)[0]
-        assert set(got) == {((r + shift) % N) // 128 for r in range(gb, last + 1)}
-        read.update((qt, t) for t in got)
-        base = shim.dsslots(N, G, 1, shift, W, qt)
-        assert base + count <= per_head
-        slots.update(base + i for i in range(count))
-    assert read == visited
-    assert len(slots) == len(read)
-    # the default variant's slot layout holds at least as many tiles per head
-    assert per_head >= shim.dsslots(N, G, 1, shift, NOWRAP, -1) or G % 128 or shift % 128
 
 
 def test_workspace_size_ex(lib):
@@ -455,8 +457,13 @@ def test_general_entries_reject(lib):
     assert lib.s2attn_bwd_general(*([A] * 9), 2, 4, 4, 256, 64, 64, f, 2, 32, 0, arr, ws, need,
                                   None) == 1
     # option flags: unknown bits, and Variant 2 without a rolled head or with shift 0
-    assert lib.s2attn_fwd_general(*ok_args, 2, None, None) == 1
+    assert lib.s2attn_fwd_general(*ok_args, 4, None, None) == 1      # unknown bit
+    assert lib.s2attn_fwd_general(*ok_args, 3, None, None) == 1      # Variants 2 and 3 together
     no_roll = [A] * 5 + [2, 4, 4, 256, 64, 64, f, 4, 32]
     assert lib.s2attn_fwd_general(*no_roll, 1, None, None) == 1
     zero_shift = [A] * 5 + [2, 4, 4, 256, 64, 64, f, 2, 0]
     assert lib.s2attn_fwd_general(*zero_shift, 1, None, None) == 1
+    assert lib.s2attn_fwd_general(*no_roll, 2, None, None) == 1      # Variant 3, same rules
+    assert lib.s2attn_fwd_general(*zero_shift, 2, None, None) == 1
+    big_shift = [A] * 5 + [2, 4, 4, 256, 64, 64, f, 2, 64]             # shift = G
+    assert lib.s2attn_fwd_general(*big_shift, 2, None, None) == 1

@@ -48,6 +48,9 @@ def test_small_workload():
     ("one_tile", 1, 2, 2, 16, 16, 128, None, None, 1.0),
     # several full tiles per group, rolled by a whole number of tiles
     ("aligned", 1, 2, 2, 2048, 512, 128, None, None, 1.0),
+    # a group boundary inside a warp's 32 rows of a query tile whose first key tile lies
+    # before that group: some rows of the warp see no key in their first step
+    ("midwarp_groups", 1, 4, 2, 544, 136, 64, None, 64, 1.0),
 ])
 def test_edge_cases(name, B, Hq, Hkv, N, G, d, shb, shift, q_gain):
     check_case(B, Hq, Hkv, N, G, d, seed=zlib.crc32(name.encode()) % 10000, shb=shb, shift=shift, q_gain=q_gain)

@@ -1,0 +1,82 @@
+"""Variants 2 and 3 of the S²-Attn ablation (LongLoRA summary page, §3.4 "Information leakage
+considerations", Table 8 and Figure 6). Variant 2: in the rolled heads the tokens that the roll
+wrapped around form their own causal group (S2ATTN_FLAG_WRAP_OWN_GROUP, oracle
+wrap_own_group=True). Variant 3: they move to the front of the last group, so its causal order
+is the original token order (S2ATTN_FLAG_WRAP_FRONT_FIRST, oracle wrap_front_first=True).
+CUDA path against the oracle, element by element.
+"""
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import shifted_sparse_attention_fwd_b200 as s2
+from shifted_sparse_attention_fwd_b200.inputs import make_inputs
+
+from gpu_helpers import check_case, gpu_run
+
+pytestmark = pytest.mark.gpu
+V2 = s2.S2ATTN_FLAG_WRAP_OWN_GROUP
+V3 = s2.S2ATTN_FLAG_WRAP_FRONT_FIRST
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    s2.lib()
+
+
+SHAPES = [
+    # the default half-group roll
+    ("half", 1, 4, 4, 512, 128, 128, None, None),
+    # the split falls inside a 128-row tile (shift 32), GQA, ragged tail, batch 2
+    ("ragged_gqa", 2, 4, 2, 320, 64, 64, None, None),
+    # groups straddle tiles, split mid-tile
+    ("straddle", 1, 4, 4, 384, 192, 128, None, 96),
+    # several tiles per group, split on a tile edge (triangular dS packing is off)
+    ("aligned", 1, 8, 4, 2048, 512, 128, None, None),
+    # every head rolled, MQA
+    ("pattern2_mqa", 1, 8, 1, 512, 128, 128, 0, 40),
+    # a small wrap remainder (shift 8) and a large one (G - 8)
+    ("shift8", 1, 2, 2, 256, 128, 64, None, 8),
+    ("shift_g_minus_8", 1, 2, 2, 256, 128, 64, None, 120),
+    # Variant 3: a rolled tile made of three runs of tokens (rows 128..191 -> 144..207,
+    # 192..207 -> 0..15, 208..255 -> 208..255)
+    ("three_runs", 1, 2, 2, 256, 64, 64, None, 16),
+    # one group: Variant 3 reorders the whole sequence back into plain causal order
+    ("one_group", 1, 2, 2, 384, 384, 64, None, 136),
+]
+
+
+@pytest.mark.parametrize("flags", [V2, V3], ids=["variant2", "variant3"])
+@pytest.mark.parametrize("name,B,Hq,Hkv,N,G,d,shb,shift", SHAPES)
+def test_variant_matches_oracle(flags, name, B, Hq, Hkv, N, G, d, shb, shift):
+    variant = 2 if flags == V2 else 3
+    check_case(B, Hq, Hkv, N, G, d, seed=zlib.crc32(("v%d" % variant + name).encode()) % 10000,
+               shb=shb, shift=shift, flags=flags)
+
+
+@pytest.mark.parametrize("flags", [V2, V3], ids=["variant2", "variant3"])
+@pytest.mark.parametrize("mode", ["recompute", "per_kv_head"])
+def test_variant_backward_paths(flags, mode):
+    check_case(1, 8, 4, 1024, 256, 128, seed=77 + flags, flags=flags, mode=mode)
+
+
+@pytest.mark.parametrize("flags", [V2, V3], ids=["variant2", "variant3"])
+def test_variant_touches_only_the_last_rolled_group(flags):
+    """Outside the last group of the rolled heads the variants compute the same rows as the
+    default, so the kernels must agree bit for bit there (same tiles, same order)."""
+    B, Hq, Hkv, N, G, d = 1, 4, 4, 512, 128, 64
+    q, k, v, do = make_inputs(B, Hq, Hkv, N, d, 5, 1.0)
+    scale = d ** -0.5
+    a = gpu_run(q, k, v, do, G, scale, backward=False)
+    b = gpu_run(q, k, v, do, G, scale, backward=False, flags=flags)
+    shb, sh = Hq // 2, G // 2
+    # rolled row r holds original token (r + sh) mod N; the last rolled group is rows N-G..N-1
+    last = (np.arange(N - G, N) + sh) % N
+    keep = np.setdiff1d(np.arange(N), last)
+    assert torch.equal(a["o"][:, :, :shb], b["o"][:, :, :shb])
+    assert torch.equal(a["o"][:, keep, shb:], b["o"][:, keep, shb:])
+    assert not torch.equal(a["o"][:, last, shb:], b["o"][:, last, shb:])
