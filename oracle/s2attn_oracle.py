@@ -40,6 +40,12 @@ Readings where the page is silent (each also listed in the design notes):
     the wrapped tokens swap places with the front of the last group, i.e. that group lists
     original tokens 0..shift-1 first and the last G - shift tokens after them, so its causal
     order is the original token order; every other group is unchanged.
+  * ``partial_last_group`` admits N not divisible by G (Table 7 uses a group of 1/6 of the
+    context): the rolled sequence is cut into groups of G rows with the last one shorter
+    (N mod G rows). Done literally by padding: the rolled tensors are extended with zero rows to
+    a multiple of G before the view into groups, and the pad rows' outputs are dropped. Pad rows
+    come last in their group, so the causal mask keeps every real query away from them, and in
+    the backward their upstream gradient is zero, so they contribute nothing.
 
 Everything is float64; inputs are the bf16 values widened exactly.
 """
@@ -172,60 +178,74 @@ def _swap_wrap_front(x: np.ndarray, N: int, G: int, shb: int, shift: int, enable
     return out
 
 
+def _pad_rows(x: np.ndarray, N: int, Np: int) -> np.ndarray:
+    """x [B, N, ...] extended with zero rows to [B, Np, ...] (Np >= N)."""
+    if Np == N:
+        return x
+    pad = np.zeros((x.shape[0], Np - N) + x.shape[2:])
+    return np.concatenate([x, pad], axis=1)
+
+
+def _check_groups(N, G, partial_last_group, wrap_own_group, wrap_front_first):
+    if wrap_own_group and wrap_front_first:
+        raise ValueError("Variant 2 and Variant 3 are alternatives")
+    if N % G != 0:
+        if not partial_last_group:
+            raise ValueError("the view into groups needs G to divide N")
+        if wrap_own_group or wrap_front_first:
+            raise ValueError("the variants are defined for G dividing N")
+    return -(-N // G) * G
+
+
 def s2attn_forward(q, k, v, G, scale, shift_head_begin=None, shift=None, wrap_own_group=False,
-                   wrap_front_first=False):
+                   wrap_front_first=False, partial_last_group=False):
     """S²-Attn forward. q [B,N,Hq,d], k, v [B,N,Hkv,d] float64.
 
     Returns o [B,N,Hq,d] and lse [B,Hq,N], both in original token order.
     """
     B, N, Hq, d = q.shape
-    if N % G != 0:
-        raise ValueError("the view into groups needs G to divide N")
-    if wrap_own_group and wrap_front_first:
-        raise ValueError("Variant 2 and Variant 3 are alternatives")
+    Np = _check_groups(N, G, partial_last_group, wrap_own_group, wrap_front_first)
     shb, shift = _defaults(Hq, G, shift_head_begin, shift)
     splits = _wrap_splits(B, N, G, shb, shift, wrap_own_group)
     ke, ve = expand_kv(k, Hq), expand_kv(v, Hq)
     # Key line 1: roll the second chunk of heads by -shift, then view as groups.
+    # (with a partial last group: pad the rolled sequence to Np rows, drop them afterwards)
     sw = lambda x: _swap_wrap_front(x, N, G, shb, shift, wrap_front_first)
-    qr = sw(chunk_roll(q, -shift, shb).reshape(B * N // G, G, Hq, d))
-    kr = sw(chunk_roll(ke, -shift, shb).reshape(B * N // G, G, Hq, d))
-    vr = sw(chunk_roll(ve, -shift, shb).reshape(B * N // G, G, Hq, v.shape[3]))
+    grp = lambda x: sw(_pad_rows(chunk_roll(x, -shift, shb), N, Np).reshape(B * Np // G, G, Hq, -1))
+    qr, kr, vr = grp(q), grp(ke), grp(ve)
     o, lse = causal_self_attn(qr, kr, vr, scale, splits)
     o = _swap_wrap_front(o, N, G, shb, shift, wrap_front_first, inverse=True)
     lse = _swap_wrap_front(lse, N, G, shb, shift, wrap_front_first, inverse=True)
     # Key line 2: back to [B, N, H, d], roll the second chunk back by +shift.
-    o = chunk_roll(o.reshape(B, N, Hq, v.shape[3]), shift, shb)
-    lse = chunk_roll(lse.reshape(B, N, Hq), shift, shb)
+    o = chunk_roll(o.reshape(B, Np, Hq, v.shape[3])[:, :N], shift, shb)
+    lse = chunk_roll(lse.reshape(B, Np, Hq)[:, :N], shift, shb)
     return o, np.ascontiguousarray(lse.transpose(0, 2, 1))
 
 
 def s2attn_backward(q, k, v, do, G, scale, shift_head_begin=None, shift=None,
-                    wrap_own_group=False, wrap_front_first=False):
+                    wrap_own_group=False, wrap_front_first=False, partial_last_group=False):
     """Gradients of s2attn_forward's o with respect to q, k, v for upstream do [B,N,Hq,d].
 
     Returns dq [B,N,Hq,d], dk [B,N,Hkv,d], dv [B,N,Hkv,d] in original token order.
     """
     B, N, Hq, d = q.shape
     Hkv = k.shape[2]
-    if wrap_own_group and wrap_front_first:
-        raise ValueError("Variant 2 and Variant 3 are alternatives")
+    Np = _check_groups(N, G, partial_last_group, wrap_own_group, wrap_front_first)
     shb, shift = _defaults(Hq, G, shift_head_begin, shift)
     splits = _wrap_splits(B, N, G, shb, shift, wrap_own_group)
     ke, ve = expand_kv(k, Hq), expand_kv(v, Hq)
     sw = lambda x: _swap_wrap_front(x, N, G, shb, shift, wrap_front_first)
-    qr = sw(chunk_roll(q, -shift, shb).reshape(B * N // G, G, Hq, d))
-    kr = sw(chunk_roll(ke, -shift, shb).reshape(B * N // G, G, Hq, d))
-    vr = sw(chunk_roll(ve, -shift, shb).reshape(B * N // G, G, Hq, d))
-    dor = sw(chunk_roll(do, -shift, shb).reshape(B * N // G, G, Hq, d))
+    grp = lambda x: sw(_pad_rows(chunk_roll(x, -shift, shb), N, Np).reshape(B * Np // G, G, Hq, -1))
+    qr, kr, vr, dor = grp(q), grp(ke), grp(ve), grp(do)
     dq, dk, dv = causal_self_attn_backward(qr, kr, vr, dor, scale, splits)
-    # The derivative of a reordering is the inverse reordering ...
+    # The derivative of a reordering is the inverse reordering, that of the padding is
+    # dropping the pad rows ...
     dq, dk, dv = (_swap_wrap_front(x, N, G, shb, shift, wrap_front_first, inverse=True)
-                  for x in (dq, dk, dv))
+                  .reshape(B, Np, Hq, d)[:, :N] for x in (dq, dk, dv))
     # ... and that of a roll is the opposite roll ...
-    dq = chunk_roll(dq.reshape(B, N, Hq, d), shift, shb)
-    dk = chunk_roll(dk.reshape(B, N, Hq, d), shift, shb)
-    dv = chunk_roll(dv.reshape(B, N, Hq, d), shift, shb)
+    dq = chunk_roll(dq, shift, shb)
+    dk = chunk_roll(dk, shift, shb)
+    dv = chunk_roll(dv, shift, shb)
     # ... and that of the shared K/V view is the sum over the query heads sharing it.
     rep = Hq // Hkv
     dk = dk.reshape(B, N, Hkv, rep, d).sum(axis=3)

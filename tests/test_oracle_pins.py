@@ -15,6 +15,8 @@
   the wrap group split by an explicit mask, and identical to the default outside that group;
 * Variant 3 of Table 8 (wrapped tokens moved to the front of the last group): equal to causal
   attention in original token order under a same-shifted-group mask, written without any roll;
+* G not dividing N (Table 7): the padded view equals a block-diagonal causal mask on the
+  rolled sequence;
 * central finite differences of the forward against the backward;
 * closed-form sums implied by rows of P summing to one;
 * planted mistakes in the oracle must fail these pins.
@@ -205,6 +207,57 @@ def test_planted_variant3_mistake_is_caught(monkeypatch):
     monkeypatch.setattr(orc, "_swap_wrap_front", _swap_never_undone)
     # (with shift = G/2 a second forward swap would undo the first: use shift != G/2)
     assert max(variant3_errors(1, 4, 2, 32, 8, 4, 2, seed=3)) > 1e-3
+
+
+def block_mask_s2attn(q, k, v, G, scale, shb, shift):
+    """G not dividing N, written without the view into groups: per head, torch.roll, then
+    SDPA over the whole rolled sequence with the mask 'same block of G rows (the last block
+    shorter), key not after query', then the roll back."""
+    B, N, Hq, d = q.shape
+    rep = Hq // k.shape[2]
+    r = torch.arange(N)
+    mask = ((r[:, None] // G) == (r[None, :] // G)) & (r[None, :] <= r[:, None])
+    outs, lses = [], []
+    for h in range(Hq):
+        s = shift if h >= shb else 0
+        qh = torch.roll(q[:, :, h], -s, dims=1)
+        kh = torch.roll(k[:, :, h // rep], -s, dims=1)
+        vh = torch.roll(v[:, :, h // rep], -s, dims=1)
+        oh = F.scaled_dot_product_attention(qh, kh, vh, attn_mask=mask, scale=scale)
+        scores = (scale * qh @ kh.transpose(-1, -2)).masked_fill(~mask, float("-inf"))
+        outs.append(torch.roll(oh, s, dims=1))
+        lses.append(torch.roll(torch.logsumexp(scores, dim=-1), s, dims=1))
+    return torch.stack(outs, dim=2), torch.stack(lses, dim=1)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,G,d,shift", [
+    (1, 4, 4, 40, 16, 8, 8),     # two full groups and one of 8
+    (2, 4, 2, 52, 24, 4, 12),    # GQA, batch 2, last group of 4
+    (1, 2, 1, 20, 32, 4, 16),    # G > N: a single, partial group
+])
+def test_partial_last_group_matches_block_mask(B, Hq, Hkv, N, G, d, shift):
+    """G not dividing N (Table 7's 1/6 group): the oracle's padding to a multiple of G equals
+    attention under a block-diagonal causal mask on the rolled sequence, forward, LSE and
+    autograd."""
+    q, k, v, do = make(B, Hq, Hkv, N, d, 17)
+    scale = 1.0 / np.sqrt(d)
+    kw = dict(partial_last_group=True)
+    o, lse = orc.s2attn_forward(q, k, v, G, scale, None, shift, **kw)
+    dq, dk, dv = orc.s2attn_backward(q, k, v, do, G, scale, None, shift, **kw)
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    to, tl = block_mask_s2attn(tq, tk, tv, G, scale, Hq // 2, shift)
+    to.backward(torch.tensor(do))
+    for a, b in ((o, to), (lse, tl), (dq, tq.grad), (dk, tk.grad), (dv, tv.grad)):
+        assert np.abs(a - b.detach().numpy()).max() < 1e-12
+
+
+def test_partial_last_group_option_is_inert_when_g_divides_n():
+    q, k, v, do = make(1, 4, 2, 48, 4, 19)
+    a = orc.s2attn_forward(q, k, v, 16, 0.5, None, 8)
+    b = orc.s2attn_forward(q, k, v, 16, 0.5, None, 8, partial_last_group=True)
+    assert all(np.array_equal(x, y) for x, y in zip(a, b))
+    with pytest.raises(ValueError):
+        orc.s2attn_forward(q[:, :40], k[:, :40], v[:, :40], 16, 0.5, None, 8)
 
 
 def test_one_group_no_shift_is_full_causal_attention():
