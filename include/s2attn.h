@@ -95,9 +95,10 @@ S2ATTN_API s2attn_status s2attn_fwd_ex(const void* q, const void* k, const void*
                             int B, int Hq, int Hkv, int N, int d, int G, float scale,
                             int shift_head_begin, int shift, void* stream);
 
-/* Option flags of the _general entry points (at most one of the two). */
+/* Option flags of the _general entry points (at most one of the first two). */
 #define S2ATTN_FLAG_WRAP_OWN_GROUP 1
 #define S2ATTN_FLAG_WRAP_FRONT_FIRST 2
+#define S2ATTN_FLAG_PARTIAL_LAST_GROUP 4
 /*
  * S2ATTN_FLAG_WRAP_OWN_GROUP is the pages' Variant 2 (summary page, §3.4 "Information
  * leakage considerations", Table 8, Figure 6): in the rolled heads the tokens that the roll
@@ -112,6 +113,13 @@ S2ATTN_API s2attn_status s2attn_fwd_ex(const void* q, const void* k, const void*
  * order inside it is the original token order (the wrapped tokens no longer see the end of the
  * sequence; the end of the sequence sees them). Same requirements as Variant 2; combining the
  * two flags is S2ATTN_ERR_INVALID_ARG.
+ *
+ * S2ATTN_FLAG_PARTIAL_LAST_GROUP admits N not divisible by G (summary page, Table 7, groups of
+ * 1/6 of the context): the rolled sequence is cut into groups of G rows and the last group is
+ * shorter (N mod G rows), which is what padding the grouped view to a multiple of G with rows
+ * that no query sees amounts to. G may then exceed N (one partial group). Without the flag
+ * N % G != 0 is S2ATTN_ERR_INVALID_ARG; with it and G | N it changes nothing. It cannot be
+ * combined with Variant 2 or 3 when G does not divide N (S2ATTN_ERR_INVALID_ARG).
  *
  * Strides. Each [B, N, H, d] tensor X is read or written at X + b*sb + t*st + h*d + c
  * (elements): the (H, d) block of a token is contiguous, tokens and batches may be spaced

@@ -13,6 +13,7 @@ from ._lib import (  # noqa: F401
     S2ATTN_ERR_TIMEOUT,
     S2ATTN_FLAG_WRAP_OWN_GROUP,
     S2ATTN_FLAG_WRAP_FRONT_FIRST,
+    S2ATTN_FLAG_PARTIAL_LAST_GROUP,
     SIGNATURES,
     LIB_PATH,
     lib,

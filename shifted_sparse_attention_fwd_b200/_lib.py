@@ -24,6 +24,7 @@ S2ATTN_ERR_TIMEOUT = 4
 # option flags of the _general entry points (include/s2attn.h)
 S2ATTN_FLAG_WRAP_OWN_GROUP = 1
 S2ATTN_FLAG_WRAP_FRONT_FIRST = 2
+S2ATTN_FLAG_PARTIAL_LAST_GROUP = 4
 
 _P = ctypes.c_void_p
 _I = ctypes.c_int

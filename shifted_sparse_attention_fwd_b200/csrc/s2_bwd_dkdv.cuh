@@ -376,7 +376,7 @@ __global__ void __launch_bounds__(32 * (kDkdvEwWarps + 3), 1)
         const HeadRemap hm = head_map(hq);
         const QTileRanges qr = kv_tile_qtiles(hm, t0, head_wrap(hq));
         const int r_k = kv_valid ? hm.rolled(t) : 0;
-        const int ge_k = group_end(r_k, p.G, head_wrap(hq));
+        const int ge_k = min_i(group_end(r_k, p.G, head_wrap(hq)), p.N);
         for (int i = 0; i < qr.count(); ++i, ++n) {
           const int st = n & 1;
           const int q0 = qr.at(i) * kTileRows + W * grp;

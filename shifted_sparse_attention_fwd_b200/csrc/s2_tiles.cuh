@@ -142,7 +142,9 @@ __host__ __device__ inline Runs identity_runs(int t0, int N) {
 // First rolled row of the group containing rolled row r, and one past its last row. With a
 // wrap split W < N (the pages' Variant 2, Table 8: in the shifted heads the tokens the roll
 // wrapped around, rolled rows [W, N) with W = N - shift, form their own group), the last
-// group [N - G, N) is two groups, [N - G, W) and [W, N).
+// group [N - G, N) is two groups, [N - G, W) and [W, N). When G does not divide N the last
+// group is shorter: callers clip group_end at N.
+__host__ __device__ __forceinline__ int min_i(int a, int b) { return a < b ? a : b; }
 __host__ __device__ inline int group_begin(int r, int G, int W = kNoWrapSplit) {
   return r >= W ? W : (r / G) * G;
 }
@@ -234,10 +236,10 @@ __host__ __device__ inline QTileRanges kv_tile_qtiles(const HeadRemap& m, int t0
     // run A: rolled rows [src0, src0 + len0); run B (after the wrap): rolled rows from 0
     QTileRanges q;
     const int a0 = tr.src[0] / kTileRows;
-    const int a1 = (group_end(tr.src[0] + tr.len[0] - 1, m.G, W) - 1) / kTileRows;
+    const int a1 = (min_i(group_end(tr.src[0] + tr.len[0] - 1, m.G, W), m.N) - 1) / kTileRows;
     q.a[1] = 0; q.b[1] = -1; q.a[2] = 0; q.b[2] = -1;
     if (tr.n == 2) {
-      const int b1 = (group_end(tr.len[1] - 1, m.G, W) - 1) / kTileRows;
+      const int b1 = (min_i(group_end(tr.len[1] - 1, m.G, W), m.N) - 1) / kTileRows;
       if (b1 + 1 >= a0) {
         q.n = 1; q.a[0] = 0; q.b[0] = a1 > b1 ? a1 : b1;
       } else {
@@ -253,7 +255,8 @@ __host__ __device__ inline QTileRanges kv_tile_qtiles(const HeadRemap& m, int t0
 #pragma unroll
   for (int k = 0; k < 3; ++k) {
     lo[k] = k < tr.n ? tr.src[k] / kTileRows : kNone;
-    hi[k] = k < tr.n ? (group_end(tr.src[k] + tr.len[k] - 1, m.G, W) - 1) / kTileRows : kNone;
+    hi[k] = k < tr.n ? (min_i(group_end(tr.src[k] + tr.len[k] - 1, m.G, W), m.N) - 1) / kTileRows
+                     : kNone;
   }
   // sort the (at most three) ranges by start, then merge overlapping or adjacent ones
 #pragma unroll
@@ -360,7 +363,7 @@ inline DsSlots ds_slots(int N, int G, int shifted_heads, int shift, int W = kNoW
   const int sh = shifted_heads ? shift : 0;
   const int w = shifted_heads ? W : kNoWrapSplit;
   const int fr = shifted_heads ? front : 0;
-  d.aligned = (G % kTileRows == 0 && sh % kTileRows == 0 && w >= N && !fr) ? 1 : 0;
+  d.aligned = (N % G == 0 && G % kTileRows == 0 && sh % kTileRows == 0 && w >= N && !fr) ? 1 : 0;
   d.gt = G / kTileRows;
   d.stride = 0;
   if (d.aligned) {
@@ -382,7 +385,7 @@ inline DsSlots ds_slots(int N, int G, int shifted_heads, int shift, int W = kNoW
 // multiple of the tile, tiles late in their group (more key tiles to visit) come first.
 __host__ __device__ inline void query_tile_coords(int bid, int B, int Hq, int N, int G, int& b,
                                                   int& h, int& qt) {
-  if (G % kTileRows == 0) {
+  if (N % G == 0 && G % kTileRows == 0) {
     const int tpg = G / kTileRows, ng = N / G;
     const int per = B * Hq * ng;
     const int il = tpg - 1 - bid / per;
@@ -406,7 +409,7 @@ __host__ __device__ inline void query_tile_coords(int bid, int B, int Hq, int N,
 // groups. Falls back to query_tile_coords when G is not a multiple of the tile.
 __host__ __device__ inline void query_tile_coords_chunked(int bid, int B, int Hq, int N, int G,
                                                           int chunk, int& b, int& h, int& qt) {
-  if (G % kTileRows != 0) {
+  if (N % G != 0 || G % kTileRows != 0) {
     query_tile_coords(bid, B, Hq, N, G, b, h, qt);
     return;
   }
@@ -432,7 +435,7 @@ __host__ __device__ inline int query_pairs_per_head(int N) {
 }
 __host__ __device__ inline void query_pair_coords(int bid, int B, int Hq, int N, int G, int& b,
                                                   int& h, int& pair) {
-  if (G % (2 * kTileRows) == 0) {
+  if (N % G == 0 && G % (2 * kTileRows) == 0) {
     const int ppg = G / (2 * kTileRows), ng = N / G;
     const int per = B * Hq * ng;
     const int pl = ppg - 1 - bid / per;
@@ -455,7 +458,7 @@ __host__ __device__ inline void query_pair_coords(int bid, int B, int Hq, int N,
 // chunk. Falls back to query_pair_coords when G is not a multiple of two tiles.
 __host__ __device__ inline void query_pair_coords_chunked(int bid, int B, int Hq, int N, int G,
                                                           int chunk, int& b, int& h, int& pair) {
-  if (G % (2 * kTileRows) != 0) {
+  if (N % G != 0 || G % (2 * kTileRows) != 0) {
     query_pair_coords(bid, B, Hq, N, G, b, h, pair);
     return;
   }
@@ -480,7 +483,7 @@ __host__ __device__ inline void kv_tile_coords(int bid, int B, int Hq, int Hkv, 
                                                int shift_head_begin, int shift, int& b,
                                                int& kvh, int& t0) {
   const int rep = Hq / Hkv;
-  if (G % kTileRows == 0 && shift % kTileRows == 0) {
+  if (N % G == 0 && G % kTileRows == 0 && shift % kTileRows == 0) {
     const int ng = N / G;
     const int per = B * Hkv * ng;
     const int jl = bid / per;
@@ -507,7 +510,7 @@ __host__ __device__ inline void kv_tile_coords(int bid, int B, int Hq, int Hkv, 
 __host__ __device__ inline void kv_tile_coords_chunked(int bid, int B, int Hq, int Hkv, int N,
                                                        int G, int shift_head_begin, int shift,
                                                        int chunk, int& b, int& kvh, int& t0) {
-  if (!(G % kTileRows == 0 && shift % kTileRows == 0)) {
+  if (!(N % G == 0 && G % kTileRows == 0 && shift % kTileRows == 0)) {
     kv_tile_coords(bid, B, Hq, Hkv, N, G, shift_head_begin, shift, b, kvh, t0);
     return;
   }

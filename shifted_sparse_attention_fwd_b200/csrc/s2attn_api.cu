@@ -201,12 +201,15 @@ int ds_heads_per_pass(const Shape& sh, size_t bytes) {
 s2attn_status check_shape(int B, int Hq, int Hkv, int N, int d, int G, float scale,
                           int shift_head_begin, long long shift, Shape& out, int flags = 0) {
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || N <= 0 || d <= 0 || G <= 0) return S2ATTN_ERR_INVALID_ARG;
-  if (Hq % Hkv != 0 || N % G != 0 || G % 2 != 0) return S2ATTN_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0 || G % 2 != 0) return S2ATTN_ERR_INVALID_ARG;
+  // G must divide N unless the caller asks for a shorter last group
+  if (N % G != 0 && !(flags & S2ATTN_FLAG_PARTIAL_LAST_GROUP)) return S2ATTN_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !std::isfinite(scale)) return S2ATTN_ERR_INVALID_ARG;
   if (shift_head_begin < 0 || shift_head_begin > Hq) return S2ATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return S2ATTN_ERR_UNSUPPORTED;
   if (N >= (1 << 30)) return S2ATTN_ERR_UNSUPPORTED;
   if (G % 8 != 0) return S2ATTN_ERR_UNSUPPORTED;
+  if (N % 8 != 0) return S2ATTN_ERR_UNSUPPORTED;   // (implied by G | N; tiles are 8-row runs)
   long long s = shift % N;
   if (s < 0) s += N;
   if (shift_head_begin == Hq) s = 0;   // no head is rolled: the roll amount is irrelevant
@@ -214,7 +217,8 @@ s2attn_status check_shape(int B, int Hq, int Hkv, int N, int d, int G, float sca
   const long long rows = static_cast<long long>(B) * (Hq > Hkv ? Hq : Hkv) * ((N + 127) / 128);
   if (rows >= (1ll << 31)) return S2ATTN_ERR_UNSUPPORTED;
   constexpr int kVariants = S2ATTN_FLAG_WRAP_OWN_GROUP | S2ATTN_FLAG_WRAP_FRONT_FIRST;
-  if (flags & ~kVariants) return S2ATTN_ERR_INVALID_ARG;
+  if (flags & ~(kVariants | S2ATTN_FLAG_PARTIAL_LAST_GROUP)) return S2ATTN_ERR_INVALID_ARG;
+  if ((flags & kVariants) && N % G != 0) return S2ATTN_ERR_INVALID_ARG;   // defined for G | N
   if ((flags & kVariants) == kVariants) return S2ATTN_ERR_INVALID_ARG;   // alternatives
   // the wrap group exists when some head is rolled by 0 < shift < G
   if ((flags & kVariants) && (shift_head_begin >= Hq || s <= 0 || s >= G))

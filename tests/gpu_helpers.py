@@ -72,12 +72,12 @@ def oracle_run(q, k, v, do, G, scale, shb=None, shift=None, backward=True, flags
     qf, kf, vf, dof = (to_f64(x) for x in (q, k, v, do))
     wrap = bool(flags & s2.S2ATTN_FLAG_WRAP_OWN_GROUP)
     front = bool(flags & s2.S2ATTN_FLAG_WRAP_FRONT_FIRST)
-    o, lse = orc.s2attn_forward(qf, kf, vf, G, scale, shb, shift, wrap_own_group=wrap,
-                                wrap_front_first=front)
+    partial = bool(flags & s2.S2ATTN_FLAG_PARTIAL_LAST_GROUP)
+    kw = dict(wrap_own_group=wrap, wrap_front_first=front, partial_last_group=partial)
+    o, lse = orc.s2attn_forward(qf, kf, vf, G, scale, shb, shift, **kw)
     out = {"o": o, "lse": lse}
     if backward:
-        dq, dk, dv = orc.s2attn_backward(qf, kf, vf, dof, G, scale, shb, shift,
-                                         wrap_own_group=wrap, wrap_front_first=front)
+        dq, dk, dv = orc.s2attn_backward(qf, kf, vf, dof, G, scale, shb, shift, **kw)
         out.update(dq=dq, dk=dk, dv=dv)
     return out
 

@@ -204,16 +204,20 @@ CASES = [(256, 64, 32), (8192, 2048, 1024), (320, 64, 32), (384, 192, 96), (200,
 SPLIT_CASES = [(256, 64, 32), (8192, 2048, 1024), (320, 64, 32), (384, 192, 96), (96, 32, 16),
                (640, 128, 64), (2048, 512, 256), (448, 64, 8), (96, 96, 88), (1024, 256, 128),
                (512, 128, 40), (1024, 1024, 512), (256, 256, 200), (136, 136, 8)]
-VARIANT_CASES = ([(n, g, s, "default") for n, g, s in CASES] +
+# (N, G, shift) with G not dividing N: the last rolled group is shorter
+PARTIAL_CASES = [(320, 128, 64), (200, 64, 32), (136, 64, 32), (264, 256, 128), (72, 128, 64),
+                 (8832, 2048, 1024), (1000, 96, 48), (384, 256, 0)]
+VARIANT_CASES = ([(n, g, s, "default") for n, g, s in CASES + PARTIAL_CASES] +
                  [(n, g, s, v) for n, g, s in SPLIT_CASES for v in ("v2", "v3")])
 
 
 def rolled_tokens(N, G, shift, variant):
     """Original token of every rolled row of a shifted head, from the oracle's own steps:
     the roll of key line 1, then (Variant 3) the oracle's reordering of the last group."""
+    if variant != "v3":
+        return np.roll(np.arange(N), -shift)
     tok = orc.rolled_token_index(N, G, shift)
-    if variant == "v3":
-        tok = orc._swap_wrap_front(tok[:, :, None], N, G, 0, shift, True)[:, :, 0]
+    tok = orc._swap_wrap_front(tok[:, :, None], N, G, 0, shift, True)[:, :, 0]
     return tok.reshape(-1)
 
 
@@ -303,7 +307,7 @@ def test_ds_slots_match_the_dkdv_pairs(shim, N, G, shift, variant):
             slots.update(base + i for i in range(len(span)))
         assert read == visited
         assert len(slots) == len(read)
-    if G % 128 == 0 and shift % 128 == 0 and variant == "default":
+    if N % G == 0 and G % 128 == 0 and shift % 128 == 0 and variant == "default":
         gt = G // 128
         assert per_head == (N // G) * gt * (gt + 1) // 2
 
@@ -323,14 +327,15 @@ def test_qtile_kv_span_large(shim, N, G, shift):
 
 
 @pytest.mark.parametrize("B,Hq,N,G", [(1, 4, 256, 64), (2, 3, 8192, 2048), (1, 2, 384, 192),
-                                      (3, 2, 320, 64), (1, 1, 1024, 1024)])
+                                      (3, 2, 320, 64), (1, 1, 1024, 1024), (1, 4, 320, 128),
+                                      (2, 2, 8832, 2048)])
 def test_query_tile_order_is_a_permutation(shim, B, Hq, N, G):
     nt = (N + 127) // 128
     seen = set()
     for bid in range(B * Hq * nt):
         seen.add(tuple(call4(shim.qcoords, bid, B, Hq, N, G)[:3]))
     assert seen == {(b, h, q) for b in range(B) for h in range(Hq) for q in range(nt)}
-    if G % 128 == 0 and G > 128:
+    if N % G == 0 and G % 128 == 0 and G > 128:
         # the first wave holds the tiles with the most key tiles (last tile of each group)
         b, h, qt = call4(shim.qcoords, 0, B, Hq, N, G)[:3]
         assert qt % (G // 128) == G // 128 - 1
@@ -340,7 +345,9 @@ def test_query_tile_order_is_a_permutation(shim, B, Hq, N, G):
                                                   (2, 8, 2, 8192, 2048, 4, 1024),
                                                   (1, 8, 1, 1024, 256, 4, 128),
                                                   (1, 4, 2, 384, 192, 2, 96),
-                                                  (1, 64, 8, 32768, 8192, 32, 4096)])
+                                                  (1, 64, 8, 32768, 8192, 32, 4096),
+                                                  (1, 4, 4, 320, 128, 2, 64),
+                                                  (2, 4, 2, 8832, 2048, 2, 1024)])
 def test_kv_tile_order_is_a_permutation(shim, B, Hq, Hkv, N, G, shb, sh):
     nt = (N + 127) // 128
     seen = set()
@@ -457,7 +464,7 @@ def test_general_entries_reject(lib):
     assert lib.s2attn_bwd_general(*([A] * 9), 2, 4, 4, 256, 64, 64, f, 2, 32, 0, arr, ws, need,
                                   None) == 1
     # option flags: unknown bits, and Variant 2 without a rolled head or with shift 0
-    assert lib.s2attn_fwd_general(*ok_args, 4, None, None) == 1      # unknown bit
+    assert lib.s2attn_fwd_general(*ok_args, 8, None, None) == 1      # unknown bit
     assert lib.s2attn_fwd_general(*ok_args, 3, None, None) == 1      # Variants 2 and 3 together
     no_roll = [A] * 5 + [2, 4, 4, 256, 64, 64, f, 4, 32]
     assert lib.s2attn_fwd_general(*no_roll, 1, None, None) == 1
@@ -467,3 +474,10 @@ def test_general_entries_reject(lib):
     assert lib.s2attn_fwd_general(*zero_shift, 2, None, None) == 1
     big_shift = [A] * 5 + [2, 4, 4, 256, 64, 64, f, 2, 64]             # shift = G
     assert lib.s2attn_fwd_general(*big_shift, 2, None, None) == 1
+    # G not dividing N: only with the partial-last-group flag, never with a variant, N % 8 == 0
+    ragged = [A] * 5 + [2, 4, 4, 320, 64, 128, f, 2, 64]
+    assert lib.s2attn_fwd_general(*ragged, 0, None, None) == 1
+    assert lib.s2attn_fwd_general(*ragged, 4 | 1, None, None) == 1
+    assert lib.s2attn_fwd_general(*ragged, 4 | 2, None, None) == 1
+    odd_n = [A] * 5 + [2, 4, 4, 324, 64, 128, f, 2, 64]
+    assert lib.s2attn_fwd_general(*odd_n, 4, None, None) == 2

@@ -1,8 +1,10 @@
-"""Variants 2 and 3 of the S²-Attn ablation (LongLoRA summary page, §3.4 "Information leakage
+"""Variants 2 and 3 of the S²-Attn ablation, and groups that do not divide the sequence (LongLoRA summary page, §3.4 "Information leakage
 considerations", Table 8 and Figure 6). Variant 2: in the rolled heads the tokens that the roll
 wrapped around form their own causal group (S2ATTN_FLAG_WRAP_OWN_GROUP, oracle
 wrap_own_group=True). Variant 3: they move to the front of the last group, so its causal order
 is the original token order (S2ATTN_FLAG_WRAP_FRONT_FIRST, oracle wrap_front_first=True).
+G not dividing N (Table 7's 1/6 group): S2ATTN_FLAG_PARTIAL_LAST_GROUP, the last rolled group
+shorter (oracle partial_last_group=True).
 CUDA path against the oracle, element by element.
 """
 import zlib
@@ -19,6 +21,7 @@ from gpu_helpers import check_case, gpu_run
 pytestmark = pytest.mark.gpu
 V2 = s2.S2ATTN_FLAG_WRAP_OWN_GROUP
 V3 = s2.S2ATTN_FLAG_WRAP_FRONT_FIRST
+PARTIAL = s2.S2ATTN_FLAG_PARTIAL_LAST_GROUP
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -80,3 +83,23 @@ def test_variant_touches_only_the_last_rolled_group(flags):
     assert torch.equal(a["o"][:, :, :shb], b["o"][:, :, :shb])
     assert torch.equal(a["o"][:, keep, shb:], b["o"][:, keep, shb:])
     assert not torch.equal(a["o"][:, last, shb:], b["o"][:, last, shb:])
+
+
+@pytest.mark.parametrize("name,B,Hq,Hkv,N,G,d,shb,shift", [
+    # two full groups of one tile and a half-tile group; GQA
+    ("tail_half_tile", 1, 4, 2, 320, 128, 64, None, None),
+    # G > N: one partial group, rolled
+    ("g_exceeds_n", 1, 2, 2, 72, 128, 64, None, None),
+    # groups that straddle tiles, a ragged sequence, batch 2
+    ("straddle_ragged", 2, 4, 4, 1000, 96, 128, None, None),
+    # the metric shape's group with a sequence of 4.3 groups
+    ("long_tail", 1, 2, 2, 8832, 2048, 128, None, None),
+])
+def test_partial_last_group_matches_oracle(name, B, Hq, Hkv, N, G, d, shb, shift):
+    check_case(B, Hq, Hkv, N, G, d, seed=zlib.crc32(("partial" + name).encode()) % 10000,
+               shb=shb, shift=shift, flags=PARTIAL)
+
+
+@pytest.mark.parametrize("mode", ["recompute", "per_kv_head"])
+def test_partial_last_group_backward_paths(mode):
+    check_case(1, 4, 2, 704, 256, 128, seed=91, flags=PARTIAL, mode=mode)
