@@ -62,6 +62,7 @@ __all__ = [
     "s2attn_backward",
     "rolled_token_index",
     "head_group_rows",
+    "rope_pi",
 ]
 
 
@@ -311,3 +312,29 @@ def head_group_rows(qh, kh, vh, doh, G, scale, shift, g, q_rows, kv_rows=None):
         out["dv"] = p2[:, kv_rows].T @ do_g[rows]
         out["dk"] = scale * (ds2[:, kv_rows].T @ q_g[rows])
     return out
+
+
+def rope_pi(x: np.ndarray, base: float = 10000.0, pi_scale: float = 1.0,
+            inverse: bool = False) -> np.ndarray:
+    """Rotary position embedding with Position Interpolation, the step just before the
+    attention (summary page, §3 Phase 1 step 2 "Position Embedding Modification" and §4
+    "Model setup": RoPE with positions rescaled by Position Interpolation).
+
+    The pages give no formula; this is the textbook rotary embedding in the half-split pairing
+    that Llama uses: for token t (original order) and i < d/2, the pair (x[i], x[i + d/2]) is
+    rotated by the angle (t * pi_scale) * base^(-2i/d). Position Interpolation multiplies the
+    positions by pi_scale = (pre-trained context) / (extended context), e.g. 4096 / 8192.
+    ``inverse`` rotates by the opposite angle: the transpose of the rotation, which maps the
+    gradient with respect to the rotated tensor back to the input.
+
+    x [B, N, H, d] float64; returns a new array.
+    """
+    B, N, H, d = x.shape
+    half = d // 2
+    theta = base ** (-2.0 * np.arange(half) / d)                 # [d/2]
+    ang = (np.arange(N) * pi_scale)[:, None] * theta[None, :]    # [N, d/2]
+    c, s = np.cos(ang)[None, :, None, :], np.sin(ang)[None, :, None, :]
+    if inverse:
+        s = -s
+    x1, x2 = x[..., :half], x[..., half:]
+    return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)

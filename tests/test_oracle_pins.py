@@ -17,6 +17,8 @@
   attention in original token order under a same-shifted-group mask, written without any roll;
 * G not dividing N (Table 7): the padded view equals a block-diagonal causal mask on the
   rolled sequence;
+* RoPE with Position Interpolation: pair norms preserved, scores depend only on the position
+  difference, the inverse undoes it, PI scale 1 is plain RoPE, and a hand-worked d = 4 case;
 * central finite differences of the forward against the backward;
 * closed-form sums implied by rows of P summing to one;
 * planted mistakes in the oracle must fail these pins.
@@ -465,3 +467,49 @@ def test_planted_mistakes_are_caught(monkeypatch, name, target, mutant):
     monkeypatch.setattr(orc, target, mutant)
     errs = library_errors(1, 4, 2, 32, 8, 4, seed=3)
     assert max(errs) > 1e-3, (name, errs)
+
+
+# --------------------------------------------------------------------------------------
+# RoPE with Position Interpolation (the step before the attention)
+# --------------------------------------------------------------------------------------
+def test_rope_preserves_pair_norms_and_inverts():
+    x = rand((2, 9, 3, 8), 41)
+    y = orc.rope_pi(x, pi_scale=0.5)
+    n = lambda a: a[..., :4] ** 2 + a[..., 4:] ** 2
+    np.testing.assert_allclose(n(y), n(x), rtol=1e-13)
+    np.testing.assert_allclose(orc.rope_pi(y, pi_scale=0.5, inverse=True), x, atol=1e-13)
+    assert np.array_equal(orc.rope_pi(x[:, :1]), x[:, :1])          # token 0: no rotation
+
+
+def test_rope_scores_depend_only_on_the_offset():
+    """The defining property of rotary embeddings: <R(m) q, R(n) k> = <R(m + c) q, R(n + c) k>.
+    Checked by placing the same q and k at positions shifted by c."""
+    d, N, c = 16, 12, 5
+    q, k = rand((d,), 1), rand((d,), 2)
+    x = np.zeros((1, N + c, 2, d))
+    x[0, 3, 0], x[0, 7, 1] = q, k              # q at 3, k at 7
+    x[0, 3 + c, 0], x[0, 7 + c, 1] = q, k      # the same pair shifted by c
+    y = orc.rope_pi(x, base=100.0, pi_scale=0.75)
+    a = y[0, 3, 0] @ y[0, 7, 1]
+    b = y[0, 3 + c, 0] @ y[0, 7 + c, 1]
+    assert abs(a - b) < 1e-12
+
+
+def test_rope_position_interpolation_is_a_position_rescale():
+    """Position Interpolation with scale 1/2: token t turns as far as token t/2 would without
+    it. Checked by placing token t at position 2t and rotating with scale 1/2."""
+    x = rand((1, 16, 2, 8), 43)
+    w = np.zeros((1, 32, 2, 8))
+    w[:, ::2] = x
+    np.testing.assert_allclose(orc.rope_pi(w, pi_scale=0.5)[:, ::2], orc.rope_pi(x), atol=1e-13)
+
+
+def test_rope_hand_worked_case():
+    """d = 4, base 100: theta = (1, 1/10). Token 2 with PI scale 1/2 sits at position 1:
+    pair 0 (x0, x2) turns by 1 rad, pair 1 (x1, x3) by 0.1 rad."""
+    x = np.zeros((1, 3, 1, 4))
+    x[0, 2, 0] = [1.0, 2.0, 3.0, 4.0]
+    y = orc.rope_pi(x, base=100.0, pi_scale=0.5)[0, 2, 0]
+    c1, s1, c2, s2 = np.cos(1.0), np.sin(1.0), np.cos(0.1), np.sin(0.1)
+    want = [1 * c1 - 3 * s1, 2 * c2 - 4 * s2, 3 * c1 + 1 * s1, 4 * c2 + 2 * s2]
+    np.testing.assert_allclose(y, want, atol=1e-15)
