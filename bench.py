@@ -233,6 +233,21 @@ def run_gpu(args, rank, world, local_rank):
     step_ms = [e[0].elapsed_time(e[4]) for e in evs]
     total_ms = sum(step_ms)
 
+    # The next-row kernel measured beside the step (not part of it): RoPE with Position
+    # Interpolation (4k -> 8k, scale 0.5) of this workload's Q and K, out of place, L2 flushed.
+    rq, rk = torch.empty_like(qd), torch.empty_like(kd)
+    rope_reps = 20
+    rope_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(rope_reps)]
+    for i in range(rope_reps + 2):
+        flush.fill_(i & 0xFF)
+        if i >= 2: rope_ev[i - 2][0].record(stream)
+        s2.s2attn_rope_pi(qd, rq, pi_scale=0.5)
+        s2.s2attn_rope_pi(kd, rk, pi_scale=0.5)
+        if i >= 2: rope_ev[i - 2][1].record(stream)
+    torch.cuda.synchronize()
+    rope_ms = sum(e[0].elapsed_time(e[1]) for e in rope_ev) / rope_reps
+    rope_bytes = 2 * (qd.numel() + kd.numel()) * 2
+
     # End to end through the public API with host buffers: pinned H2D of the step's inputs,
     # fwd + bwd, D2H of the step's results, all inside the timed region.
     hq_, hk_, hv_, hdo_ = (x.pin_memory() for x in (q, k, v, do))
@@ -323,6 +338,12 @@ def run_gpu(args, rank, world, local_rank):
                 "steps": e2e_steps, "ms_per_step": round(e2e_ms / e2e_steps, 4)},
         "clocks": sampler.summary(),
         "gpu_launches": 4 * args.steps,
+        "next_rows": {"rope_pi": {
+            "what": "s2attn_rope_pi on Q and K of the workload (PI scale 0.5), outside the step",
+            "ms": round(rope_ms, 4), "bytes": rope_bytes,
+            "gbs": round(rope_bytes / (rope_ms * 1e-3) / 1e9, 1),
+            "frac_of_hbm": round(rope_bytes / (rope_ms * 1e-3) / 1e9 /
+                                 float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])), 4)}},
     }
     return line
 

@@ -277,6 +277,27 @@ S2ATTN_API void s2attn_set_wait_timeout_ns(unsigned long long ns);
  */
 S2ATTN_API s2attn_status s2attn_selftest_wait_timeout(unsigned long long timeout_ns, void* stream);
 
+/*
+ * Rotary position embedding with Position Interpolation: the step just before the attention
+ * (summary page, §3 "Phase 1" step 2, and §4 "Model setup": RoPE with positions rescaled by
+ * Position Interpolation). x and y are bf16 [B, N, H, d] (d = 64 or 128); for token t and
+ * i < d/2 the pair (x[.., i], x[.., i + d/2]) is turned by the angle (t * pi_scale) *
+ * base^(-2i/d) (the Llama half-split pairing; t in original order) and written to y.
+ * pi_scale is the Position Interpolation factor (pre-trained context / extended context, e.g.
+ * 4096/8192 = 0.5; 1 for plain RoPE); base is the frequency base (10000 for Llama 2).
+ * inverse = 1 turns by the opposite angle: the transpose of the rotation, which maps dq, dk
+ * with respect to the rotated q, k back to the unrotated ones.
+ * y == x (in place) is allowed; other overlaps are not. `strides` = NULL (contiguous) or
+ * {x_sb, x_st, y_sb, y_st} in elements, with the rules of s2attn_fwd_general (so q and k can
+ * be rotated inside a packed qkv buffer). Errors: null or misaligned pointers, B, N, H <= 0,
+ * base <= 1, pi_scale <= 0, inverse not 0/1, bad strides -> S2ATTN_ERR_INVALID_ARG;
+ * d not in {64, 128}, N >= 2^24 -> S2ATTN_ERR_UNSUPPORTED; launch failure -> S2ATTN_ERR_CUDA.
+ * Asynchronous on `stream`; allocates nothing.
+ */
+S2ATTN_API s2attn_status s2attn_rope_pi(const void* x, void* y, int B, int N, int H, int d,
+                                        float base, float pi_scale, int inverse,
+                                        const long long* strides, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

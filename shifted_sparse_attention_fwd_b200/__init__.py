@@ -32,6 +32,8 @@ from ._lib import (  # noqa: F401
     s2attn_get_device_error,
     s2attn_set_wait_timeout_ns,
     s2attn_selftest_wait_timeout,
+    s2attn_rope_pi,
+    rope_pi,
     fwd,
     bwd,
 )

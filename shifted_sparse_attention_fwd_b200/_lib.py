@@ -49,6 +49,7 @@ SIGNATURES = {
     "s2attn_fwd_general": (_I, [_P] * 5 + [_I] * 6 + [_F, _I, _I, _I, _P, _P]),
     "s2attn_bwd_general": (_I, [_P] * 9 + [_I] * 6 + [_F, _I, _I, _I, _P, _P, _Z, _P]),
     "s2attn_bwd_workspace_size_general": (_Z, [_I] * 9 + [_Z]),
+    "s2attn_rope_pi": (_I, [_P, _P, _I, _I, _I, _I, _F, _F, _I, _P, _P]),
     "s2attn_bwd_dkdv_ds": (_I, [_P] * 6 + [_I] * 6 + [_F, _I, _I, _P, _Z, _P]),
     "s2attn_bwd_dq_ds": (_I, [_P] * 2 + [_I] * 6 + [_F, _I, _I, _P, _Z, _P]),
     "s2attn_get_device_error": (_I, [_P, ctypes.POINTER(ctypes.c_uint)]),
@@ -309,6 +310,26 @@ def s2attn_selftest_wait_timeout(timeout_ns: int, stream=None):
 # ------------------------------------------------------------------------------------------
 # Allocating conveniences (torch provides the memory; the library does the work).
 # ------------------------------------------------------------------------------------------
+def s2attn_rope_pi(x, y, base=10000.0, pi_scale=1.0, inverse=False, stream=None):
+    """Rotary position embedding with Position Interpolation of x [B,N,H,d] bf16 into y (y may
+    be x). Views with contiguous (H, d) blocks, e.g. q or k of a packed qkv, are accepted."""
+    _check_bf16(x, y)
+    B, N, H, d = x.shape
+    if tuple(y.shape) != tuple(x.shape):
+        raise ValueError("x and y must have the same shape")
+    strides = None if _all_contiguous(x, y) else _strides_array(x, y)
+    _check(lib().s2attn_rope_pi(_ptr(x, True), _ptr(y, True), B, N, H, d, float(base),
+                                float(pi_scale), 1 if inverse else 0, strides, _stream(stream)),
+           "s2attn_rope_pi")
+
+
+def rope_pi(x, base=10000.0, pi_scale=1.0, inverse=False, stream=None, out=None):
+    """Convenience form of s2attn_rope_pi: returns the rotated tensor (a new one unless `out`)."""
+    y = torch.empty_like(x) if out is None else out
+    s2attn_rope_pi(x, y, base, pi_scale, inverse, stream)
+    return y
+
+
 def fwd(q, k, v, G, scale=None, shift_head_begin=None, shift=None, stream=None, flags=0):
     o = torch.empty_like(q)
     lse = torch.empty((q.shape[0], q.shape[2], q.shape[1]), dtype=torch.float32, device=q.device)

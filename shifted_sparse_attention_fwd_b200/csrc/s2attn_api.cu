@@ -15,6 +15,7 @@
 #include "s2_bwd_dq.cuh"
 #include "s2_bwd_dq_ds.cuh"
 #include "s2_bwd_pre.cuh"
+#include "s2_rope.cuh"
 #include "s2_fwd.cuh"
 
 namespace {
@@ -735,6 +736,45 @@ s2attn_status s2attn_selftest_wait_timeout(unsigned long long timeout_ns, void* 
   selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(err, timeout_ns);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? S2ATTN_OK : cuda_fail(e, "selftest_wait_kernel launch");
+}
+
+s2attn_status s2attn_rope_pi(const void* x, void* y, int B, int N, int H, int d, float base,
+                             float pi_scale, int inverse, const long long* strides,
+                             void* stream) {
+  if (!x || !y || !aligned16(x) || !aligned16(y)) return S2ATTN_ERR_INVALID_ARG;
+  if (B <= 0 || N <= 0 || H <= 0 || d <= 0) return S2ATTN_ERR_INVALID_ARG;
+  if (!(base > 1.f) || !std::isfinite(base) || !(pi_scale > 0.f) || !std::isfinite(pi_scale))
+    return S2ATTN_ERR_INVALID_ARG;
+  if (inverse != 0 && inverse != 1) return S2ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return S2ATTN_ERR_UNSUPPORTED;
+  if (N >= (1 << 24) || static_cast<long long>(H) * d >= (1ll << 31)) return S2ATTN_ERR_UNSUPPORTED;
+  long long st[4] = {static_cast<long long>(N) * H * d, static_cast<long long>(H) * d,
+                     static_cast<long long>(N) * H * d, static_cast<long long>(H) * d};
+  if (strides) {
+    for (int i = 0; i < 2; ++i) {
+      const long long sb = strides[2 * i], stt = strides[2 * i + 1];
+      if (sb < 0 || stt < static_cast<long long>(H) * d || sb % 8 != 0 || stt % 8 != 0)
+        return S2ATTN_ERR_INVALID_ARG;
+      if (B > 1 && sb < stt * N) return S2ATTN_ERR_INVALID_ARG;
+      st[2 * i] = sb;
+      st[2 * i + 1] = stt;
+    }
+  }
+  const long long blocks = static_cast<long long>(B) * ((N + s2::kRopeTokens - 1) / s2::kRopeTokens);
+  if (blocks >= (1ll << 31)) return S2ATTN_ERR_UNSUPPORTED;
+  const float log2_base = std::log2(base);
+  const float sign = inverse ? -1.f : 1.f;
+  cudaStream_t sm = static_cast<cudaStream_t>(stream);
+  const auto* xb = static_cast<const __nv_bfloat16*>(x);
+  auto* yb = static_cast<__nv_bfloat16*>(y);
+  if (d == 64)
+    s2::s2_rope_kernel<64><<<static_cast<unsigned>(blocks), s2::kRopeThreads, 0, sm>>>(
+        xb, yb, N, H, st[0], st[1], st[2], st[3], log2_base, pi_scale, sign);
+  else
+    s2::s2_rope_kernel<128><<<static_cast<unsigned>(blocks), s2::kRopeThreads, 0, sm>>>(
+        xb, yb, N, H, st[0], st[1], st[2], st[3], log2_base, pi_scale, sign);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? S2ATTN_OK : cuda_fail(e, "s2_rope_kernel launch");
 }
 
 }  // extern "C"

@@ -374,6 +374,20 @@ def test_query_pair_order_is_a_permutation(shim, B, Hq, N, G):
         assert p % (G // 256) == G // 256 - 1
 
 
+def test_rope_rejects(lib):
+    """Argument checks of s2attn_rope_pi, before any launch."""
+    f = ctypes.c_float
+    ok = [A, A, 1, 64, 4, 128]
+    assert lib.s2attn_rope_pi(None, A, 1, 64, 4, 128, f(1e4), f(0.5), 0, None, None) == 1
+    assert lib.s2attn_rope_pi(A + 8, A, 1, 64, 4, 128, f(1e4), f(0.5), 0, None, None) == 1
+    assert lib.s2attn_rope_pi(*ok, f(1.0), f(0.5), 0, None, None) == 1      # base <= 1
+    assert lib.s2attn_rope_pi(*ok, f(1e4), f(0.0), 0, None, None) == 1      # pi_scale <= 0
+    assert lib.s2attn_rope_pi(*ok, f(1e4), f(0.5), 2, None, None) == 1      # inverse not 0/1
+    assert lib.s2attn_rope_pi(A, A, 1, 64, 4, 96, f(1e4), f(0.5), 0, None, None) == 2
+    bad = (ctypes.c_longlong * 4)(*[4 * 128 * 64, 4 * 128 - 8] * 2)      # token stride < H*d
+    assert lib.s2attn_rope_pi(*ok, f(1e4), f(0.5), 0, bad, None) == 1
+
+
 def test_workspace_size_ex(lib):
     base = lib.s2attn_bwd_workspace_size(1, 32, 8192)
     full = lib.s2attn_bwd_workspace_size_ex(1, 32, 32, 8192, 128, 2048, 16, 1024, 0)
