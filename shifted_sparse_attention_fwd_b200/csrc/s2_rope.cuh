@@ -45,32 +45,48 @@ __global__ void __launch_bounds__(kRopeThreads) s2_rope_kernel(
   }
   __syncthreads();
   // work item = (token, head, chunk): chunk c covers pairs 8c .. 8c + 7, i.e. the 16 bytes at
-  // column 8c of the first half and those at column D/2 + 8c
+  // column 8c of the first half and those at column D/2 + 8c. Each thread loads kRopeUnroll
+  // items before computing, to keep more bytes in flight.
+  constexpr int kRopeUnroll = 4;
   const int items = nt * H * kChunks;
-  for (int w = threadIdx.x; w < items; w += blockDim.x) {
-    const int c = w % kChunks, th = w / kChunks;
-    const int h = th % H, tt = th / H;
-    const long long t = t0 + tt;
-    const __nv_bfloat16* src = x + b * x_sb + t * x_st + static_cast<long long>(h) * D + 8 * c;
-    __nv_bfloat16* dst = y + b * y_sb + t * y_st + static_cast<long long>(h) * D + 8 * c;
-    const uint4 lo = *reinterpret_cast<const uint4*>(src);
-    const uint4 hi = *reinterpret_cast<const uint4*>(src + kHalf);
-    const __nv_bfloat162* l2 = reinterpret_cast<const __nv_bfloat162*>(&lo);
-    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&hi);
-    uint4 olo, ohi;
-    __nv_bfloat162* ol = reinterpret_cast<__nv_bfloat162*>(&olo);
-    __nv_bfloat162* oh = reinterpret_cast<__nv_bfloat162*>(&ohi);
+  for (int w0 = threadIdx.x; w0 < items; w0 += kRopeUnroll * blockDim.x) {
+    uint4 lo[kRopeUnroll], hi[kRopeUnroll];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float2 a = __bfloat1622float2(l2[j]), bb = __bfloat1622float2(h2[j]);
-      const int i = 8 * c + 2 * j;
-      const float c0 = s_cos[tt][i], c1 = s_cos[tt][i + 1];
-      const float s0 = s_sin[tt][i], s1 = s_sin[tt][i + 1];
-      ol[j] = __floats2bfloat162_rn(a.x * c0 - bb.x * s0, a.y * c1 - bb.y * s1);
-      oh[j] = __floats2bfloat162_rn(bb.x * c0 + a.x * s0, bb.y * c1 + a.y * s1);
+    for (int u = 0; u < kRopeUnroll; ++u) {
+      const int w = w0 + u * blockDim.x;
+      if (w < items) {
+        const int c = w % kChunks, th = w / kChunks;
+        const int h = th % H, tt = th / H;
+        const __nv_bfloat16* src =
+            x + b * x_sb + (t0 + tt) * x_st + static_cast<long long>(h) * D + 8 * c;
+        lo[u] = *reinterpret_cast<const uint4*>(src);
+        hi[u] = *reinterpret_cast<const uint4*>(src + kHalf);
+      }
     }
-    *reinterpret_cast<uint4*>(dst) = olo;
-    *reinterpret_cast<uint4*>(dst + kHalf) = ohi;
+#pragma unroll
+    for (int u = 0; u < kRopeUnroll; ++u) {
+      const int w = w0 + u * blockDim.x;
+      if (w >= items) break;
+      const int c = w % kChunks, th = w / kChunks;
+      const int h = th % H, tt = th / H;
+      __nv_bfloat16* dst = y + b * y_sb + (t0 + tt) * y_st + static_cast<long long>(h) * D + 8 * c;
+      const __nv_bfloat162* l2 = reinterpret_cast<const __nv_bfloat162*>(&lo[u]);
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&hi[u]);
+      uint4 olo, ohi;
+      __nv_bfloat162* ol = reinterpret_cast<__nv_bfloat162*>(&olo);
+      __nv_bfloat162* oh = reinterpret_cast<__nv_bfloat162*>(&ohi);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 a = __bfloat1622float2(l2[j]), bb = __bfloat1622float2(h2[j]);
+        const int i = 8 * c + 2 * j;
+        const float c0 = s_cos[tt][i], c1 = s_cos[tt][i + 1];
+        const float s0 = s_sin[tt][i], s1 = s_sin[tt][i + 1];
+        ol[j] = __floats2bfloat162_rn(a.x * c0 - bb.x * s0, a.y * c1 - bb.y * s1);
+        oh[j] = __floats2bfloat162_rn(bb.x * c0 + a.x * s0, bb.y * c1 + a.y * s1);
+      }
+      *reinterpret_cast<uint4*>(dst) = olo;
+      *reinterpret_cast<uint4*>(dst + kHalf) = ohi;
+    }
   }
 }
 
