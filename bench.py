@@ -317,6 +317,12 @@ def run_gpu(args, rank, world, local_rank):
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4),
+        "step_ms_spread": {
+            "min": round(min(step_ms), 4), "median": round(sorted(step_ms)[len(step_ms) // 2], 4),
+            "max": round(max(step_ms), 4),
+            "first_half": round(sum(step_ms[:len(step_ms) // 2]) / max(1, len(step_ms) // 2), 4),
+            "second_half": round(sum(step_ms[len(step_ms) // 2:]) /
+                                 max(1, len(step_ms) - len(step_ms) // 2), 4)},
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16 Q/K/V/dO, Llama2-7B attention layer shape)",
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "G": w.G,
