@@ -248,35 +248,60 @@ def run_gpu(args, rank, world, local_rank):
     rope_ms = sum(e[0].elapsed_time(e[1]) for e in rope_ev) / rope_reps
     rope_bytes = 2 * (qd.numel() + kd.numel()) * 2
 
-    # End to end through the public API with host buffers: pinned H2D of the step's inputs,
-    # fwd + bwd, D2H of the step's results, all inside the timed region.
+    # End to end through the public API with host buffers: every step copies its inputs from
+    # pinned host memory, runs fwd + bwd and copies its results back, all inside the timed
+    # region. Steps are pipelined the way a training loop with a prefetching loader would run
+    # them: two sets of device buffers, host-to-device copies on one stream, kernels on another,
+    # device-to-host copies on a third, so step i+1's inputs and step i-1's results move over
+    # PCIe (both directions at once) while step i computes.
     hq_, hk_, hv_, hdo_ = (x.pin_memory() for x in (q, k, v, do))
-    ho, hdq = torch.empty_like(hq_).pin_memory(), torch.empty_like(hq_).pin_memory()
-    hdk, hdv = torch.empty_like(hk_).pin_memory(), torch.empty_like(hv_).pin_memory()
-    hlse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32).pin_memory()
+    dbuf = [dict(q=qd, k=kd, v=vd, do=dod, o=o, lse=lse, dq=dq, dk=dk, dv=dv)]
+    dbuf.append({n: torch.empty_like(t) for n, t in dbuf[0].items()})
+    hout = [{n: torch.empty(t.shape, dtype=t.dtype).pin_memory() for n, t in dbuf[0].items()
+             if n in ("o", "lse", "dq", "dk", "dv")} for _ in range(2)]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in, ev_comp, ev_out = ([torch.cuda.Event() for _ in range(2)] for _ in range(3))
 
-    def e2e_step():
-        for dst, src in ((qd, hq_), (kd, hk_), (vd, hv_), (dod, hdo_)):
-            dst.copy_(src, non_blocking=True)
-        s2.s2attn_fwd(qd, kd, vd, o, lse, w.G, w.scale)
-        s2.s2attn_bwd(qd, kd, vd, o, lse, dod, dq, dk, dv, w.G, w.scale, workspace=ws)
-        for dst, src in ((ho, o), (hlse, lse), (hdq, dq), (hdk, dk), (hdv, dv)):
-            dst.copy_(src, non_blocking=True)
+    def e2e_step(i):
+        b = i % 2
+        db, hb = dbuf[b], hout[b]
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(ev_comp[b])        # step i-2 no longer reads these inputs
+            for n, src in (("q", hq_), ("k", hk_), ("v", hv_), ("do", hdo_)):
+                db[n].copy_(src, non_blocking=True)
+            ev_in[b].record(s_in)
+        stream.wait_event(ev_in[b])
+        if i >= 2:
+            stream.wait_event(ev_out[b])           # step i-2's results have been copied out
+        s2.s2attn_fwd(db["q"], db["k"], db["v"], db["o"], db["lse"], w.G, w.scale, stream=stream)
+        s2.s2attn_bwd(db["q"], db["k"], db["v"], db["o"], db["lse"], db["do"], db["dq"], db["dk"],
+                      db["dv"], w.G, w.scale, workspace=ws, stream=stream)
+        ev_comp[b].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_comp[b])
+            for n in ("o", "lse", "dq", "dk", "dv"):
+                hb[n].copy_(db[n], non_blocking=True)
+            ev_out[b].record(s_out)
 
     e2e_steps = max(3, min(args.steps, 20))
-    for _ in range(2):
-        e2e_step()
+    for i in range(2):
+        e2e_step(i)
     torch.cuda.synchronize()
     if dist: dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record(stream)
+    e0.record(s_in)
+    for i in range(2, 2 + e2e_steps):
+        e2e_step(i)
+    e1.record(s_out)                               # after the last step's results are out
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
+    # same inputs every step and deterministic kernels: both buffer sets must hold equal results
+    for n in ("o", "dq", "dk"):
+        if not torch.equal(hout[0][n], hout[1][n]):
+            raise RuntimeError(f"pipelined end-to-end steps disagree on {n}")
     h2d = sum(x.numel() * x.element_size() for x in (hq_, hk_, hv_, hdo_))
-    d2h = sum(x.numel() * x.element_size() for x in (ho, hlse, hdq, hdk, hdv))
+    d2h = sum(x.numel() * x.element_size() for x in hout[0].values())
 
     total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dist, dev)
     if rank != 0:
@@ -341,7 +366,8 @@ def run_gpu(args, rank, world, local_rank):
         "roofline": roof,
         "e2e": {"value": round(weak_scaling_value(world, flops_step, e2e_steps, e2e_ms), 2),
                 "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "steps": e2e_steps, "ms_per_step": round(e2e_ms / e2e_steps, 4)},
+                "steps": e2e_steps, "ms_per_step": round(e2e_ms / e2e_steps, 4),
+                "pipelining": "double-buffered: H2D, kernels and D2H on three streams"},
         "clocks": sampler.summary(),
         "gpu_launches": 4 * args.steps,
         "next_rows": {"rope_pi": {
