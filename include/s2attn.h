@@ -6,11 +6,11 @@
  * Attention as a Training-Time Proxy for Full Attention", Algorithm 1):
  *   1. split the Hq query heads into two chunks; in the second chunk (heads
  *      [Hq/2, Hq)) roll every sequence by -G/2 along the token axis, with wrap-around
- *      (key line 1, torch.roll semantics: rolled[r] = x[(r + G/2) mod N]);
+ *      (torch.roll semantics: rolled[r] = x[(r + G/2) mod N]);
  *   2. view the N tokens as N/G independent groups of G consecutive (rolled) tokens;
  *   3. inside each group apply standard causal self-attention
  *      o = softmax(scale * q k^T) v, the causal mask taken in rolled order;
- *   4. roll the second chunk's output back by +G/2 (key line 2).
+ *   4. roll the second chunk's output back by +G/2.
  * The backward is the gradient of those steps (the page uses S²-Attn only during
  * fine-tuning, §3.2, so gradients flow through it).
  * Grouped-query heads: query head h reads key/value head h / (Hq / Hkv); its roll is
@@ -75,7 +75,7 @@ S2ATTN_API const char* s2attn_status_string(int status);
 S2ATTN_API const char* s2attn_last_error(void);
 
 /*
- * Forward: o and lse from q, k, v (Algorithm 1, key line 1 -> self_attn -> key line 2).
+ * Forward: o and lse from q, k, v (Algorithm 1: roll -> self_attn -> roll back).
  * Heads [Hq/2, Hq) are rolled by G/2. scale multiplies q k^T (1/sqrt(d) for Llama2).
  */
 S2ATTN_API s2attn_status s2attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,

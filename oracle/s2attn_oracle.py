@@ -6,7 +6,7 @@ never calls it and has no CPU fallback.
 
 Source: "LongLoRA: Efficient Fine-tuning of Long-Context Large Language Models",
 paper-graph summary page, §3.4 "S2-Attn: Shifted Sparse Attention as a Training-Time
-Proxy for Full Attention", Algorithm 1 (key line 1, standard self-attention, key line 2)
+Proxy for Full Attention", Algorithm 1 (the roll, standard self-attention, the roll back)
 and the three-step description (split heads, shift one chunk, recombine).
 
 The forward is the algorithm written out literally, in the pages' notation:
@@ -69,8 +69,8 @@ __all__ = [
 def chunk_roll(x: np.ndarray, amount: int, shift_head_begin: int) -> np.ndarray:
     """Roll heads [shift_head_begin, H) of x [B, N, H, ...] by ``amount`` along N.
 
-    Key line 1 of Algorithm 1 is chunk_roll(qkv, -G/2, H/2); key line 2 is
-    chunk_roll(out, +G/2, H/2). np.roll has torch.roll's semantics:
+    Algorithm 1 rolls with chunk_roll(qkv, -G/2, H/2) before the attention and back with
+    chunk_roll(out, +G/2, H/2) after it. np.roll has torch.roll's semantics:
     np.roll(x, a)[r] = x[(r - a) mod N].
     """
     out = x.copy()
@@ -209,7 +209,7 @@ def s2attn_forward(q, k, v, G, scale, shift_head_begin=None, shift=None, wrap_ow
     shb, shift = _defaults(Hq, G, shift_head_begin, shift)
     splits = _wrap_splits(B, N, G, shb, shift, wrap_own_group)
     ke, ve = expand_kv(k, Hq), expand_kv(v, Hq)
-    # Key line 1: roll the second chunk of heads by -shift, then view as groups.
+    # Algorithm 1's roll: the second chunk of heads by -shift, then the view as groups.
     # (with a partial last group: pad the rolled sequence to Np rows, drop them afterwards)
     sw = lambda x: _swap_wrap_front(x, N, G, shb, shift, wrap_front_first)
     grp = lambda x: sw(_pad_rows(chunk_roll(x, -shift, shb), N, Np).reshape(B * Np // G, G, Hq, -1))
@@ -217,7 +217,7 @@ def s2attn_forward(q, k, v, G, scale, shift_head_begin=None, shift=None, wrap_ow
     o, lse = causal_self_attn(qr, kr, vr, scale, splits)
     o = _swap_wrap_front(o, N, G, shb, shift, wrap_front_first, inverse=True)
     lse = _swap_wrap_front(lse, N, G, shb, shift, wrap_front_first, inverse=True)
-    # Key line 2: back to [B, N, H, d], roll the second chunk back by +shift.
+    # Algorithm 1's roll back: to [B, N, H, d], the second chunk rolled back by +shift.
     o = chunk_roll(o.reshape(B, Np, Hq, v.shape[3])[:, :N], shift, shb)
     lse = chunk_roll(lse.reshape(B, Np, Hq)[:, :N], shift, shb)
     return o, np.ascontiguousarray(lse.transpose(0, 2, 1))
@@ -257,7 +257,7 @@ def s2attn_backward(q, k, v, do, G, scale, shift_head_begin=None, shift=None,
 def rolled_token_index(N: int, G: int, shift: int) -> np.ndarray:
     """Original token of every (group, in-group row) of a shifted head, as [N/G, G].
 
-    Obtained by applying key line 1 to the token index itself: np.roll(arange(N), -shift).
+    Obtained by applying Algorithm 1's roll to the token index itself: np.roll(arange(N), -shift).
     """
     return np.roll(np.arange(N), -shift).reshape(N // G, G)
 

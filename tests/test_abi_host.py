@@ -3,7 +3,7 @@
 * libs2attn.so loads and exports every function include/s2attn.h declares;
 * argument validation rejects bad calls before any CUDA call (fake device addresses);
 * the remap and tile-order functions the kernels use (s2_tiles.cuh), compiled here with g++,
-  agree with the oracle's literal roll (LongLoRA summary page, §3.4 Algorithm 1 key line 1)
+  agree with the oracle's literal roll (LongLoRA summary page, §3.4 Algorithm 1, the roll before the attention)
   and with a brute-force enumeration of which query rows see which key rows.
 """
 import ctypes
@@ -213,7 +213,7 @@ VARIANT_CASES = ([(n, g, s, "default") for n, g, s in CASES + PARTIAL_CASES] +
 
 def rolled_tokens(N, G, shift, variant):
     """Original token of every rolled row of a shifted head, from the oracle's own steps:
-    the roll of key line 1, then (Variant 3) the oracle's reordering of the last group."""
+    Algorithm 1's roll, then (Variant 3) the oracle's reordering of the last group."""
     if variant != "v3":
         return np.roll(np.arange(N), -shift)
     tok = orc.rolled_token_index(N, G, shift)
