@@ -1,8 +1,8 @@
 // The per-head shift-and-group remap, applied to 128-row tiles.
 //
 // LongLoRA summary page, §3.4 Algorithm 1: the second chunk of heads is rolled by -G/2
-// along N (the roll before the attention), viewed as groups of G (".view(B*N/G, G, ...)"), attended causally
-// per group, and rolled back (the roll after it). Instead of materialising the roll, every kernel
+// along N before the attention, viewed as groups of G (".view(B*N/G, G, ...)"), attended
+// causally per group, and rolled back after it. Instead of materialising the roll, every kernel
 // addresses the original tensors through
 //     t = (r + s_h) mod N          (rolled row r -> original token t)
 // where s_h is the head's roll (G/2 for the shifted heads, 0 otherwise); group of rolled
