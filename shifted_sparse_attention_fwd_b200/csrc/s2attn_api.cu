@@ -556,7 +556,7 @@ s2attn_status s2attn_bwd_preprocess(const void* o, const float* lse, const void*
   if (d != 64 && d != 128) return S2ATTN_ERR_UNSUPPORTED;
   if (N >= (1 << 30) || static_cast<long long>(B) * Hq * ((N + 127) / 128) >= (1ll << 31))
     return S2ATTN_ERR_UNSUPPORTED;
-  Shape sh{B, Hq, Hq, N, d, N, Hq, 0, s2::kNoWrapSplit, {}, {}};
+  Shape sh{B, Hq, Hq, N, d, N, Hq, 0, s2::kNoWrapSplit, 0, {}, {}};
   sh.set_contiguous();
   s2attn_status s = check_workspace(sh, workspace, workspace_bytes);
   if (s != S2ATTN_OK) return s;
