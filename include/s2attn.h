@@ -31,7 +31,8 @@
  *
  * Errors: arguments are validated on the host before any launch;
  *   S2ATTN_ERR_INVALID_ARG  null / misaligned pointer, a size <= 0, Hq % Hkv != 0,
- *                           N % G != 0, odd G, odd Hq (default split), scale not a
+ *                           N % G != 0 (unless S2ATTN_FLAG_PARTIAL_LAST_GROUP), odd G,
+ *                           odd Hq (default split), unknown option flags, scale not a
  *                           positive finite number, shift_head_begin outside [0, Hq],
  *                           workspace too small;
  *   S2ATTN_ERR_UNSUPPORTED  d not in {64, 128}; G or the roll not a multiple of 8 tokens
@@ -65,7 +66,8 @@ typedef enum {
 } s2attn_status;
 
 /* Version of this ABI (bumped on any signature change or workspace-size change); 2 adds the
- * dS hand-off entries and the work counters in the backward workspace. */
+ * dS hand-off entries and the work counters in the backward workspace; 3 adds the option flags
+ * (_general entries, which replace the strided-only entries) and s2attn_rope_pi. */
 S2ATTN_API int s2attn_abi_version(void);
 
 /* Static description of a status code. */

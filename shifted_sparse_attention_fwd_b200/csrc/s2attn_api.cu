@@ -22,7 +22,7 @@ namespace {
 
 __device__ unsigned int g_err_word;   // first pipeline-wait failure since the last read
 
-constexpr int kAbiVersion = 2;
+constexpr int kAbiVersion = 3;
 constexpr int kMaxDevices = 64;
 constexpr unsigned long long kDefaultTimeoutNs = 1000000000ull;
 

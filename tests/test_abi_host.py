@@ -50,7 +50,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.s2attn_abi_version() == 2
+    assert lib.s2attn_abi_version() == 3
     for st in range(5):
         assert s2.status_string(st)
     assert s2.status_string(99) == "unknown status"
