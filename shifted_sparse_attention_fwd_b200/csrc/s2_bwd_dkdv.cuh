@@ -11,7 +11,8 @@
 //   dK  += scale * dS^T Q
 // A work tile is 128 ORIGINAL key/value rows of one (batch, kv head), so the tile is shared
 // by all its query heads whatever their roll, and dK/dV are written once, without atomics.
-// For each query head the rows map to at most two runs of rolled rows; the query tiles
+// For each query head the rows map to at most two runs of rolled rows (three with the
+// Variant 3 reordering); the query tiles
 // visited are those covering [rolled row, end of its group) for every row of the tile.
 // The kernel is persistent: each CTA claims work tiles from a global counter (heaviest first,
 // grouped for L2 reuse), so one tile's epilogue overlaps the next tile's loads and first MMAs
@@ -21,10 +22,9 @@
 // four warps i/32 + 4 g, g = 0..3, warp group g taking query columns [32 g, 32 g + 32), so
 // four warps per SM sub-partition hide each other's TMEM and special-function latency;
 // warp 16 TMA producer (K, V per tile; Q, dO, LSE2, D per query tile, 2 stages); warp 17
-// TMEM allocator + MMA issuer; warp 18 store issuer: the
-// elementwise warps leave each dS tile (for the dQ pass) and the finished dV and dK tiles in
-// a shared-memory staging buffer, and warp 10 hands them to the TMA unit, so no elementwise
-// warp waits on global stores.
+// TMEM allocator + MMA issuer; warp 18 store issuer: the elementwise warps leave each dS
+// tile (for the dQ pass) and the finished dV and dK tiles in a shared-memory staging buffer,
+// and warp 18 hands them to the TMA unit, so no elementwise warp waits on global stores.
 // TMEM: S^T [0,128) and dP^T [128,256); each column group packs its bf16 P^T (dS^T) into the
 // first 16 of its own 32 fp32 input columns, so the warps of a row never overwrite each
 // other's unread data, and the dV (dK) MMA reads the A operand group by group
