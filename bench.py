@@ -6,6 +6,11 @@ dQ kernel (dQ = scale * dS K over those tiles), all through the C ABI. FLOPs are
 7 * B * Hq * N * G * d per fwd+bwd (causal half of each G x G group; fwd 2, bwd 5).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--workload NAME]
+                  [--bwd-path handoff|recompute] [--workspace-cap BYTES]
+
+--bwd-path recompute times the minimum-workspace backward (the dQ kernel recomputes S and dP);
+--workspace-cap bounds the dS hand-off workspace, so long sequences run the dK/dV + dQ kernels
+once per group of kv heads that fits (the whole backward is then timed as one span).
 
 N > 1 runs under torchrun, one process per GPU, each on its own batch of the same workload
 (weak scaling, no data-path collective); timing is the max over ranks of device time.
@@ -54,9 +59,11 @@ def weak_scaling_value(world, flops_per_step, steps, total_ms):
     return world * flops_per_step * steps / (total_ms * 1e-3) / 1e12
 
 
-def kernel_flops(w):
-    unit = float(w.B) * w.Hq * w.N * w.G * w.d   # one causal in-group GEMM over all heads
-    return {"s2_fwd": 2 * unit, "s2_bwd_dkdv": 4 * unit, "s2_bwd_dq_ds": 1 * unit}
+def kernel_flops(w, G=None):
+    """Algorithmic FLOPs per launch (causal half of each in-group G x G block)."""
+    unit = float(w.B) * w.Hq * w.N * (w.G if G is None else G) * w.d
+    return {"s2_fwd": 2 * unit, "s2_bwd_dkdv": 4 * unit, "s2_bwd_dq_ds": 1 * unit,
+            "s2_bwd_dq": 1 * unit, "s2_bwd": 5 * unit}
 
 
 def dq_ds_bytes(w, ds_tiles) -> float:
@@ -67,6 +74,14 @@ def dq_ds_bytes(w, ds_tiles) -> float:
 def pre_bytes(w) -> float:
     # O and dO read once (bf16), LSE read, D and LSE*log2(e) written (fp32)
     return 2.0 * (2 * w.B * w.N * w.Hq * w.d) + 3.0 * 4 * w.B * w.Hq * w.N
+
+
+def bench_config(w, world=1):
+    """The workload description both arms print (identical dicts, so the two lines compare)."""
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "G": w.G,
+            "d": w.d, "shift_heads": f"{w.Hq // 2}-{w.Hq - 1}", "batch_per_gpu": w.B,
+            "l2": f"flushed before every GPU step ({L2_FLUSH_BYTES >> 20} MiB write, untimed)",
+            "parallelism": f"{world} independent replicas (weak scaling)"}
 
 
 def load_peaks():
@@ -89,7 +104,7 @@ REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_pow
 
 
 class ClockSampler:
-    def __init__(self, device_index: int, period_s: float = 0.02):
+    def __init__(self, device_index: int, period_s: float = 0.001):
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self.period = period_s
         self._stop = threading.Event()
@@ -167,7 +182,9 @@ def oracle_sample(w, target_s: float = 12.0):
         if elapsed >= target_s:
             break
     flops = 7.0 * w.B * done * w.N * w.G * w.d
-    return {"value": flops / elapsed / 1e12, "unit": UNIT, "cores": int(cores), "kind": "oracle",
+    return {"value": flops / elapsed / 1e12, "unit": UNIT, "cores": int(cores),
+            "nproc": os.cpu_count(), "cores_note": "cores = BLAS threads numpy used; nproc = host CPUs",
+            "kind": "oracle",
             "sample": f"{done} of {w.Hq} heads (all {w.N // w.G} groups, B={w.B}) fwd+bwd, "
                       f"{elapsed:.1f} s, numpy fp64", "seconds": round(elapsed, 2)}
 
@@ -190,20 +207,44 @@ def run_gpu(args, rank, world, local_rank):
     lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=dev)
     dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
     ws_min = s2.s2attn_bwd_workspace_size(w.B, w.Hq, w.N)
-    ws_bytes = s2.s2attn_bwd_workspace_size_ex(w.B, w.Hq, w.Hkv, w.N, w.d, w.G)
-    ds_tiles = (ws_bytes - ws_min) // 32768
+    ws_all = s2.s2attn_bwd_workspace_size_ex(w.B, w.Hq, w.Hkv, w.N, w.d, w.G)
+    if args.bwd_path == "recompute":
+        ws_bytes, passes = ws_min, 0
+    else:
+        ws_bytes = s2.s2attn_bwd_workspace_size_ex(w.B, w.Hq, w.Hkv, w.N, w.d, w.G,
+                                                   cap_bytes=args.workspace_cap)
+        per_head = (ws_all - ws_min) // w.Hkv
+        passes = -(-w.Hkv // ((ws_bytes - ws_min) // per_head))
+    ds_tiles = (ws_all - ws_min) // 32768
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    # One step = forward + the whole backward; events between the stages that are timed apart.
+    if args.bwd_path == "recompute":
+        names = ["s2_fwd", "s2_bwd_pre", "s2_bwd_dkdv", "s2_bwd_dq"]
+    elif passes == 1:
+        names = ["s2_fwd", "s2_bwd_pre", "s2_bwd_dkdv", "s2_bwd_dq_ds"]
+    else:
+        names = ["s2_fwd", "s2_bwd"]      # `passes` dK/dV + dQ passes inside one span
 
     def step(ev=None):
         if ev: ev[0].record(stream)
         s2.s2attn_fwd(qd, kd, vd, o, lse, w.G, w.scale)
         if ev: ev[1].record(stream)
+        if len(names) == 2:
+            s2.s2attn_bwd(qd, kd, vd, o, lse, dod, dq, dk, dv, w.G, w.scale, workspace=ws)
+            if ev: ev[2].record(stream)
+            return
         s2.s2attn_bwd_preprocess(o, lse, dod, ws)
         if ev: ev[2].record(stream)
-        s2.s2attn_bwd_dkdv_ds(qd, kd, vd, dod, dk, dv, w.G, ws, w.scale)
-        if ev: ev[3].record(stream)
-        s2.s2attn_bwd_dq_ds(kd, dq, w.G, ws, w.scale)
+        if args.bwd_path == "recompute":
+            s2.s2attn_bwd_dkdv(qd, kd, vd, dod, dk, dv, w.G, ws, w.scale)
+            if ev: ev[3].record(stream)
+            s2.s2attn_bwd_dq(qd, kd, vd, dod, dq, w.G, ws, w.scale)
+        else:
+            s2.s2attn_bwd_dkdv_ds(qd, kd, vd, dod, dk, dv, w.G, ws, w.scale)
+            if ev: ev[3].record(stream)
+            s2.s2attn_bwd_dq_ds(kd, dq, w.G, ws, w.scale)
         if ev: ev[4].record(stream)
 
     for _ in range(args.warmup):
@@ -214,8 +255,9 @@ def run_gpu(args, rank, world, local_rank):
     if st != s2.S2ATTN_OK:
         raise RuntimeError(f"device error {st} code {code:#x} during warm-up")
 
-    # Timed region: K steps, L2 flushed (untimed) before each, per-kernel CUDA events.
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    # Timed region: K steps, L2 flushed (untimed) before each, per-stage CUDA events.
+    nev = len(names) + 1
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(args.steps)]
     if dist: dist.barrier()
     torch.cuda.synchronize()
     sampler = ClockSampler(dev.index)
@@ -228,10 +270,15 @@ def run_gpu(args, rank, world, local_rank):
     st, code = s2.s2attn_get_device_error()
     if st != s2.S2ATTN_OK:
         raise RuntimeError(f"device error {st} code {code:#x} in the timed region")
-    names = ["s2_fwd", "s2_bwd_pre", "s2_bwd_dkdv", "s2_bwd_dq_ds"]
     per_k = {n: [e[j].elapsed_time(e[j + 1]) for e in evs] for j, n in enumerate(names)}
-    step_ms = [e[0].elapsed_time(e[4]) for e in evs]
+    step_ms = [e[0].elapsed_time(e[nev - 1]) for e in evs]
     total_ms = sum(step_ms)
+    if args.bwd_path == "recompute":
+        launches_per_step = 4
+    elif passes == 1:
+        launches_per_step = 4
+    else:
+        launches_per_step = 2 + 2 * passes
 
     # The next-row kernel measured beside the step (not part of it): RoPE with Position
     # Interpolation (4k -> 8k, scale 0.5) of this workload's Q and K, out of place, L2 flushed.
@@ -247,6 +294,32 @@ def run_gpu(args, rank, world, local_rank):
     torch.cuda.synchronize()
     rope_ms = sum(e[0].elapsed_time(e[1]) for e in rope_ev) / rope_reps
     rope_bytes = 2 * (qd.numel() + kd.numel()) * 2
+
+    # Full causal attention (the pages' Phase 2, standard attention after fine-tuning) through
+    # the same kernels: one group of N rows and no roll (G = N, no rolled head), on the metric
+    # workload's tensors, beside the step (not part of it), L2 flushed.
+    full_causal = None
+    if args.workload == METRIC_WORKLOAD:
+        fc_ws = torch.empty(s2.s2attn_bwd_workspace_size_ex(w.B, w.Hq, w.Hkv, w.N, w.d, w.N, w.Hq, 0),
+                            dtype=torch.uint8, device=dev)
+        fc_reps = 10
+        fc_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(fc_reps)]
+        for i in range(fc_reps + 3):
+            flush.fill_(i & 0xFF)
+            if i >= 3: fc_ev[i - 3][0].record(stream)
+            s2.s2attn_fwd(qd, kd, vd, o, lse, w.N, w.scale, shift_head_begin=w.Hq, shift=0)
+            if i >= 3: fc_ev[i - 3][1].record(stream)
+            s2.s2attn_bwd(qd, kd, vd, o, lse, dod, dq, dk, dv, w.N, w.scale, shift_head_begin=w.Hq,
+                          shift=0, workspace=fc_ws)
+            if i >= 3: fc_ev[i - 3][2].record(stream)
+        torch.cuda.synchronize()
+        st, code = s2.s2attn_get_device_error()
+        if st != s2.S2ATTN_OK:
+            raise RuntimeError(f"device error {st} code {code:#x} in the full-causal run")
+        full_causal = {"fwd_ms": sum(e[0].elapsed_time(e[1]) for e in fc_ev) / fc_reps,
+                       "bwd_ms": sum(e[1].elapsed_time(e[2]) for e in fc_ev) / fc_reps,
+                       "workspace_bytes": fc_ws.numel()}
+        del fc_ws
 
     # End to end through the public API with host buffers: every step copies its inputs from
     # pinned host memory, runs fwd + bwd and copies its results back, all inside the timed
@@ -338,7 +411,32 @@ def run_gpu(args, rank, world, local_rank):
         if n == "s2_bwd_dq_ds":
             entry.update(gbs=round(dq_ds_bytes(w, ds_tiles) / (avg[n] * 1e-3) / 1e9, 1),
                          ds_tiles=int(ds_tiles))
+        if n == "s2_bwd_dq":
+            entry.update(executed_units=3, note="recomputes S and dP: 3 GEMMs for 1 algorithmic")
+        if n == "s2_bwd":
+            entry.update(passes=passes, note="preprocess + one dK/dV and one dQ launch per pass")
         kern[n] = entry
+    bwd_ms = sum(avg[n] for n in names if n != "s2_fwd")
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    next_rows = {"rope_pi": {
+        "what": "s2attn_rope_pi on Q and K of the workload (PI scale 0.5), outside the step",
+        "ms": round(rope_ms, 4), "bytes": rope_bytes,
+        "gbs": round(rope_bytes / (rope_ms * 1e-3) / 1e9, 1),
+        "frac_of_hbm": round(rope_bytes / (rope_ms * 1e-3) / 1e9 / hbm, 4)}}
+    if full_causal is not None:
+        fc_flops = 7.0 * w.B * w.Hq * w.N * w.N * w.d
+        fc_ms = full_causal["fwd_ms"] + full_causal["bwd_ms"]
+        fc_tf = fc_flops / (fc_ms * 1e-3) / 1e12
+        fwd_fc_tf = kernel_flops(w, G=w.N)["s2_fwd"] / (full_causal["fwd_ms"] * 1e-3) / 1e12
+        next_rows["full_causal"] = {
+            "what": f"full causal attention (G = N = {w.N}, no rolled head), fwd + bwd through "
+                    "the same kernels, outside the step",
+            "ms": round(fc_ms, 4), "fwd_ms": round(full_causal["fwd_ms"], 4),
+            "bwd_ms": round(full_causal["bwd_ms"], 4), "flops": fc_flops,
+            "tflops": round(fc_tf, 1), "workspace_bytes": full_causal["workspace_bytes"],
+            "roofline": {"bound": "tensor", "achieved": round(fc_tf, 1), "peak": peak_tf,
+                         "unit": "TFLOP/s", "frac": round(fc_tf / peak_tf, 4),
+                         "fwd_frac": round(fwd_fc_tf / peak_tf, 4)}}
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4),
@@ -349,18 +447,17 @@ def run_gpu(args, rank, world, local_rank):
             "second_half": round(sum(step_ms[len(step_ms) // 2:]) /
                                  max(1, len(step_ms) - len(step_ms) // 2), 4)},
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded N(0,1) bf16 Q/K/V/dO, Llama2-7B attention layer shape)",
-        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "G": w.G,
-                   "d": w.d, "shift_heads": f"{w.Hq // 2}-{w.Hq - 1}", "batch_per_gpu": w.B,
-                   "l2": f"flushed before every step ({L2_FLUSH_BYTES >> 20} MiB write, untimed)",
-                   "parallelism": f"{world} independent replicas (weak scaling)"},
+        "data": "synthetic (seeded N(0,1) bf16 Q/K/V/dO, Llama2 attention layer shape)",
+        "config": bench_config(w, world),
         "pct_of_peak": round(100 * value / peak_tf, 2),
         "fwd": {"ms": round(avg["s2_fwd"], 4),
                 "tflops": round(kflops["s2_fwd"] / (avg["s2_fwd"] * 1e-3) / 1e12, 1)},
-        "bwd": {"ms": round(avg["s2_bwd_pre"] + avg["s2_bwd_dkdv"] + avg["s2_bwd_dq_ds"], 4),
-                "tflops": round(5.0 * float(w.B) * w.Hq * w.N * w.G * w.d /
-                                ((avg["s2_bwd_pre"] + avg["s2_bwd_dkdv"] + avg["s2_bwd_dq_ds"]) * 1e-3)
-                                / 1e12, 1)},
+        "bwd": {"ms": round(bwd_ms, 4),
+                "tflops": round(kflops["s2_bwd"] / (bwd_ms * 1e-3) / 1e12, 1),
+                "path": ("dQ recomputed (minimum workspace)" if args.bwd_path == "recompute"
+                         else "dS hand-off"),
+                "passes": passes, "workspace_bytes": int(ws_bytes),
+                "workspace_bytes_one_pass": int(ws_all)},
         "peak": {"bf16_tflops": peak_tf, "source": peak_src},
         "kernels": kern,
         "roofline": roof,
@@ -369,13 +466,8 @@ def run_gpu(args, rank, world, local_rank):
                 "steps": e2e_steps, "ms_per_step": round(e2e_ms / e2e_steps, 4),
                 "pipelining": "double-buffered: H2D, kernels and D2H on three streams"},
         "clocks": sampler.summary(),
-        "gpu_launches": 4 * args.steps,
-        "next_rows": {"rope_pi": {
-            "what": "s2attn_rope_pi on Q and K of the workload (PI scale 0.5), outside the step",
-            "ms": round(rope_ms, 4), "bytes": rope_bytes,
-            "gbs": round(rope_bytes / (rope_ms * 1e-3) / 1e9, 1),
-            "frac_of_hbm": round(rope_bytes / (rope_ms * 1e-3) / 1e9 /
-                                 float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])), 4)}},
+        "gpu_launches": launches_per_step * args.steps,
+        "next_rows": next_rows,
     }
     return line
 
@@ -463,15 +555,15 @@ def run_reference(args, rank):
         vals.append(tf)
         secs += dt
     value = statistics.mean(vals)
-    cb = {"value": round(value, 6), "unit": UNIT, "cores": int(cores), "kind": "oracle",
+    cb = {"value": round(value, 6), "unit": UNIT, "cores": int(cores), "nproc": os.cpu_count(),
+          "cores_note": "cores = BLAS threads numpy used; nproc = host CPUs", "kind": "oracle",
           "sample": f"each step: one (batch, head, group) unit of G={w.G} rows, fwd+bwd, all "
                     f"rows; heads alternate unrolled/rolled; {secs:.1f} s over {args.steps} steps"}
     return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT,
             "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "ms_per_step": round(1e3 * secs / max(1, args.steps), 3),
-            "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N,
-                       "G": w.G, "d": w.d},
+            "config": bench_config(w, 1),
             "cpu_baseline": cb,
             "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
@@ -485,6 +577,9 @@ def main():
     ap.add_argument("--impl", default="s2attn", choices=["s2attn", "reference"])
     ap.add_argument("--workload", default=METRIC_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--bwd-path", default="handoff", choices=["handoff", "recompute"])
+    ap.add_argument("--workspace-cap", type=int, default=0,
+                    help="bytes for the dS hand-off workspace (0: all kv heads in one pass)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

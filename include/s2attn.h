@@ -31,12 +31,11 @@
  *
  * Errors: arguments are validated on the host before any launch;
  *   S2ATTN_ERR_INVALID_ARG  null / misaligned pointer, a size <= 0, Hq % Hkv != 0,
- *                           N % G != 0 (unless S2ATTN_FLAG_PARTIAL_LAST_GROUP), odd G,
+ *                           N % G != 0 (unless S2ATTN_FLAG_PARTIAL_LAST_GROUP),
  *                           odd Hq (default split), unknown option flags, scale not a
  *                           positive finite number, shift_head_begin outside [0, Hq],
  *                           workspace too small;
- *   S2ATTN_ERR_UNSUPPORTED  d not in {64, 128}; G or the roll not a multiple of 8 tokens
- *                           (for the default roll G/2: G % 16 != 0); N >= 2^30;
+ *   S2ATTN_ERR_UNSUPPORTED  d not in {64, 128}; N >= 2^30;
  *   S2ATTN_ERR_CUDA         a CUDA call or a launch failed (see s2attn_last_error);
  *   S2ATTN_ERR_TIMEOUT      reported by s2attn_get_device_error: a kernel's pipeline wait
  *                           exceeded its limit; the kernel stopped early and returned
@@ -67,7 +66,8 @@ typedef enum {
 
 /* Version of this ABI (bumped on any signature change or workspace-size change); 2 adds the
  * dS hand-off entries and the work counters in the backward workspace; 3 adds the option flags
- * (_general entries, which replace the strided-only entries) and s2attn_rope_pi. */
+ * (_general entries, which replace the strided-only entries) and s2attn_rope_pi; 4 adds the
+ * _general forms of the two dS hand-off stages. */
 S2ATTN_API int s2attn_abi_version(void);
 
 /* Static description of a status code. */
@@ -78,7 +78,9 @@ S2ATTN_API const char* s2attn_last_error(void);
 
 /*
  * Forward: o and lse from q, k, v (Algorithm 1: roll -> self_attn -> roll back).
- * Heads [Hq/2, Hq) are rolled by G/2. scale multiplies q k^T (1/sqrt(d) for Llama2).
+ * Heads [Hq/2, Hq) are rolled by G/2 (rounded down when G is odd: the page's group of
+ * 1/6 of 8192 tokens, Table 7, is G = 1365 rolled by 682). Any G >= 1 and any roll are
+ * supported. scale multiplies q k^T (1/sqrt(d) for Llama2).
  */
 S2ATTN_API s2attn_status s2attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
                          int B, int Hq, int Hkv, int N, int d, int G, float scale,
@@ -91,7 +93,7 @@ S2ATTN_API s2attn_status s2attn_fwd(const void* q, const void* k, const void* v,
  * grouped causal attention (the page's "short attention", Pattern 1 only); 0 rolls every
  * head (Pattern 2 only); shift = N - G/2 is the page's "shift up" variant (Table 8);
  * G = N with shift_head_begin = Hq is full causal attention. shift may be any integer; it
- * is taken mod N and must then be a multiple of 8.
+ * is taken mod N.
  */
 S2ATTN_API s2attn_status s2attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse,
                             int B, int Hq, int Hkv, int N, int d, int G, float scale,
@@ -218,9 +220,10 @@ S2ATTN_API s2attn_status s2attn_bwd_dq(const void* q, const void* k, const void*
                             size_t workspace_bytes, void* stream);
 
 /*
- * The two gradient stages of the dS hand-off, one kv-head group covering all kv heads: the
- * workspace must be at least s2attn_bwd_workspace_size_ex(..., cap_bytes = 0) bytes, else
- * S2ATTN_ERR_INVALID_ARG. Run s2attn_bwd_preprocess, then, on the same stream and with the
+ * The two gradient stages of the dS hand-off, one kv-head group covering all kv heads, for the
+ * default variant and contiguous tensors (the _general forms below take option flags and
+ * strides): the workspace must be at least s2attn_bwd_workspace_size_ex(..., cap_bytes = 0)
+ * bytes, else S2ATTN_ERR_INVALID_ARG. Run s2attn_bwd_preprocess, then, on the same stream and with the
  * same workspace:
  *   s2attn_bwd_dkdv_ds  dk, dv and the dS tiles <- from q, k, v, dO and D, LSE2
  *   s2attn_bwd_dq_ds    dq                      <- from k and the dS tiles
@@ -234,6 +237,31 @@ S2ATTN_API s2attn_status s2attn_bwd_dq_ds(const void* k, void* dq, int B, int Hq
                                           int d, int G, float scale, int shift_head_begin,
                                           int shift, const void* workspace,
                                           size_t workspace_bytes, void* stream);
+
+/*
+ * The two dS hand-off stages with option flags and strides, so that a caller driving the
+ * backward stage by stage keeps every variant of s2attn_bwd_general (Variants 2 and 3 of the
+ * pages' Table 8, a shorter last group) and packed dqkv outputs. Arguments as in
+ * s2attn_bwd_general: `strides` is NULL or its 8 {sb, st} pairs (q, k, v, o, dO, dq, dk, dv;
+ * the pairs of tensors a stage does not touch are validated but unused). The workspace must be
+ * at least s2attn_bwd_workspace_size_general(..., flags, cap_bytes = 0) bytes and carry the
+ * preprocess results (s2attn_bwd_preprocess) of the same o, lse, dO; errors as in
+ * s2attn_bwd_general, and S2ATTN_ERR_INVALID_ARG if the workspace holds the dS tiles of fewer
+ * than all kv heads. Run s2attn_bwd_dkdv_ds_general, then s2attn_bwd_dq_ds_general, on the
+ * same stream with the same flags.
+ */
+S2ATTN_API s2attn_status s2attn_bwd_dkdv_ds_general(const void* q, const void* k, const void* v,
+                                                    const void* dO, void* dk, void* dv, int B,
+                                                    int Hq, int Hkv, int N, int d, int G,
+                                                    float scale, int shift_head_begin, int shift,
+                                                    int flags, const long long* strides,
+                                                    void* workspace, size_t workspace_bytes,
+                                                    void* stream);
+S2ATTN_API s2attn_status s2attn_bwd_dq_ds_general(const void* k, void* dq, int B, int Hq, int Hkv,
+                                                  int N, int d, int G, float scale,
+                                                  int shift_head_begin, int shift, int flags,
+                                                  const long long* strides, const void* workspace,
+                                                  size_t workspace_bytes, void* stream);
 
 /*
  * Backward without a caller-provided workspace, for callers that cannot allocate device

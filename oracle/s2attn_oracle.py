@@ -20,7 +20,7 @@ dP = dO V^T, dS = P o (dP - rowsum(P o dP)), dQ = scale dS K, dK = scale dS^T Q,
 dV = P^T dO; the derivative of a roll is the opposite roll and the derivative of the
 shared K/V view (grouped-query heads) is a sum over the query heads that share it.
 
-Readings where the page is silent (each also listed in the design notes):
+Readings where the page is silent:
   * scale: the page writes softmax(q k^T); the caller's ``scale`` multiplies q k^T.
   * causal mask: applied in rolled order within each group, so in the shifted heads the
     wrap group (last G/2 tokens followed by the first G/2) lets the first G/2 tokens see

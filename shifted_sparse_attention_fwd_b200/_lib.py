@@ -52,6 +52,8 @@ SIGNATURES = {
     "s2attn_rope_pi": (_I, [_P, _P, _I, _I, _I, _I, _F, _F, _I, _P, _P]),
     "s2attn_bwd_dkdv_ds": (_I, [_P] * 6 + [_I] * 6 + [_F, _I, _I, _P, _Z, _P]),
     "s2attn_bwd_dq_ds": (_I, [_P] * 2 + [_I] * 6 + [_F, _I, _I, _P, _Z, _P]),
+    "s2attn_bwd_dkdv_ds_general": (_I, [_P] * 6 + [_I] * 6 + [_F, _I, _I, _I, _P, _P, _Z, _P]),
+    "s2attn_bwd_dq_ds_general": (_I, [_P] * 2 + [_I] * 6 + [_F, _I, _I, _I, _P, _P, _Z, _P]),
     "s2attn_get_device_error": (_I, [_P, ctypes.POINTER(ctypes.c_uint)]),
     "s2attn_set_wait_timeout_ns": (None, [ctypes.c_ulonglong]),
     "s2attn_selftest_wait_timeout": (_I, [ctypes.c_ulonglong, _P]),
@@ -257,23 +259,44 @@ def s2attn_bwd_dq(q, k, v, dO, dq, G, workspace, scale=None, shift_head_begin=No
 
 
 def s2attn_bwd_dkdv_ds(q, k, v, dO, dk, dv, G, workspace, scale=None, shift_head_begin=None,
-                       shift=None, stream=None):
+                       shift=None, stream=None, flags=0, dq=None):
+    """dK, dV and the dS tiles (first of the two dS hand-off stages). With option flags, or views
+    with contiguous (H, d) blocks, the _general entry is used (`dq` then supplies dQ's strides;
+    it is not written here)."""
     B, Hq, Hkv, N, d, G = _dims(q, k, G)
     scale = d ** -0.5 if scale is None else scale
     shb = Hq // 2 if shift_head_begin is None else shift_head_begin
     sh = G // 2 if shift is None else shift
+    if flags or not _all_contiguous(q, k, v, dO, dk, dv, dq):
+        ts = (q, k, v, dO, dO, dq if dq is not None else q, dk, dv)
+        strides = None if _all_contiguous(*ts) else _strides_array(*ts)
+        _check(lib().s2attn_bwd_dkdv_ds_general(
+            _ptr(q, True), _ptr(k, True), _ptr(v, True), _ptr(dO, True), _ptr(dk, True),
+            _ptr(dv, True), B, Hq, Hkv, N, d, G, scale, shb, sh, int(flags), strides,
+            _ptr(workspace), workspace.numel(), _stream(stream)), "s2attn_bwd_dkdv_ds_general")
+        return
     _check(lib().s2attn_bwd_dkdv_ds(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(dk), _ptr(dv), B,
                                     Hq, Hkv, N, d, G, scale, shb, sh, _ptr(workspace),
                                     workspace.numel(), _stream(stream)), "s2attn_bwd_dkdv_ds")
 
 
 def s2attn_bwd_dq_ds(k, dq, G, workspace, scale=None, shift_head_begin=None, shift=None,
-                     stream=None):
+                     stream=None, flags=0):
+    """dQ from the dS tiles (second of the two dS hand-off stages); flags or a strided k / dq
+    go through the _general entry."""
     B, N, Hq, d = dq.shape
     Hkv = k.shape[2]
     scale = d ** -0.5 if scale is None else scale
     shb = Hq // 2 if shift_head_begin is None else shift_head_begin
     sh = G // 2 if shift is None else shift
+    if flags or not _all_contiguous(k, dq):
+        ts = (dq, k, k, dq, dq, dq, k, k)
+        strides = None if _all_contiguous(k, dq) else _strides_array(*ts)
+        _check(lib().s2attn_bwd_dq_ds_general(
+            _ptr(k, True), _ptr(dq, True), B, Hq, Hkv, N, d, G, scale, shb, sh, int(flags),
+            strides, _ptr(workspace), workspace.numel(), _stream(stream)),
+            "s2attn_bwd_dq_ds_general")
+        return
     _check(lib().s2attn_bwd_dq_ds(_ptr(k), _ptr(dq), B, Hq, Hkv, N, d, G, scale, shb, sh,
                                   _ptr(workspace), workspace.numel(), _stream(stream)),
            "s2attn_bwd_dq_ds")

@@ -75,7 +75,7 @@ __global__ void __launch_bounds__(320, 1)
   const int n_kv = qt - kt_begin + 1;
 
   if (warp == 8 && lane == 0) {
-    mbar_init(bar(L::B_QDO), 1);
+    mbar_init(bar(L::B_QDO), 2);   // the Q tile and the dO tile
     for (int s = 0; s < L::kKStages; ++s) {
       mbar_init(bar(L::B_K + s), 1);
       mbar_init(bar(L::B_KE + s), 1);
@@ -108,31 +108,30 @@ __global__ void __launch_bounds__(320, 1)
 
   if (warp == 8) {
     // ---------------- TMA producer ----------------
-    if (lane == 0) {
+    // The whole warp runs the loop (see produce_tile): lane 0 waits on the ring barriers and
+    // issues the TMA copies, all lanes fill the tile rows TMA cannot move.
+    {
       const Runs q_runs = rolled_runs(hm, R0);
-      mbar_expect_tx(bar(L::B_QDO), 2 * L::kTile);
-      load_tile<D>(sbase + L::kQ, &tmQ, &tmQ8, bar(L::B_QDO), b, h, q_runs, p.N);
-      load_tile<D>(sbase + L::kDO, &tmO, &tmO8, bar(L::B_QDO), b, h, q_runs, p.N);
+      produce_tile<D>(sbase + L::kQ, &tmQ, &tmQ8, bar(L::B_QDO), p.q, b, h, q_runs, p.N);
+      produce_tile<D>(sbase + L::kDO, &tmO, &tmO8, bar(L::B_QDO), p.dO, b, h, q_runs, p.N);
       int k_issued = 0, v_issued = 0;
       auto issue_k = [&]() -> bool {
         const int i = k_issued, st = i % L::kKStages;
         if (i >= L::kKStages &&
-            !wait_bar(bar(L::B_KE + st), ((i / L::kKStages) - 1) & 1, ctx, 1))
+            !lead_wait(bar(L::B_KE + st), ((i / L::kKStages) - 1) & 1, ctx, 1))
           return false;
-        mbar_expect_tx(bar(L::B_K + st), L::kTile);
-        load_tile<D>(sbase + L::kK + st * L::kTile, &tmK, &tmK8, bar(L::B_K + st), b, kvh,
-                     rolled_runs(hm, (kt_begin + i) * kTileRows), p.N);
+        produce_tile<D>(sbase + L::kK + st * L::kTile, &tmK, &tmK8, bar(L::B_K + st), p.k, b, kvh,
+                        rolled_runs(hm, (kt_begin + i) * kTileRows), p.N);
         ++k_issued;
         return true;
       };
       auto issue_v = [&]() -> bool {
         const int i = v_issued, st = i % L::kVStages;
         if (i >= L::kVStages &&
-            !wait_bar(bar(L::B_VE + st), ((i / L::kVStages) - 1) & 1, ctx, 10))
+            !lead_wait(bar(L::B_VE + st), ((i / L::kVStages) - 1) & 1, ctx, 10))
           return false;
-        mbar_expect_tx(bar(L::B_V + st), L::kTile);
-        load_tile<D>(sbase + L::kV + st * L::kTile, &tmV, &tmV8, bar(L::B_V + st), b, kvh,
-                     rolled_runs(hm, (kt_begin + i) * kTileRows), p.N);
+        produce_tile<D>(sbase + L::kV + st * L::kTile, &tmV, &tmV8, bar(L::B_V + st), p.v, b, kvh,
+                        rolled_runs(hm, (kt_begin + i) * kTileRows), p.N);
         ++v_issued;
         return true;
       };
@@ -141,11 +140,13 @@ __global__ void __launch_bounds__(320, 1)
         if (j + 1 < n_kv) ok = issue_k();
         if (ok) ok = issue_v();
       }
-      drain_wait(bar(L::B_QDO), 0, p.timeout_ns);
-      for (int i = k_issued - L::kKStages; i < k_issued; ++i)
-        if (i >= 0) drain_wait(bar(L::B_K + i % L::kKStages), (i / L::kKStages) & 1, p.timeout_ns);
-      for (int i = v_issued - L::kVStages; i < v_issued; ++i)
-        if (i >= 0) drain_wait(bar(L::B_V + i % L::kVStages), (i / L::kVStages) & 1, p.timeout_ns);
+      if (lane == 0) {
+        drain_wait(bar(L::B_QDO), 0, p.timeout_ns);
+        for (int i = k_issued - L::kKStages; i < k_issued; ++i)
+          if (i >= 0) drain_wait(bar(L::B_K + i % L::kKStages), (i / L::kKStages) & 1, p.timeout_ns);
+        for (int i = v_issued - L::kVStages; i < v_issued; ++i)
+          if (i >= 0) drain_wait(bar(L::B_V + i % L::kVStages), (i / L::kVStages) & 1, p.timeout_ns);
+      }
     }
   } else if (warp == 9) {
     // ---------------- MMA issuer ----------------

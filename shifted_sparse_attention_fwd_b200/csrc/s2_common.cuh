@@ -16,20 +16,68 @@ struct Tile {
   static constexpr int kHalves = D / 64;
 };
 
+// A [B, N, H, D] bf16 tensor by address and element strides (batch, token), for the rows that
+// are loaded with plain loads instead of TMA.
+struct TensorRef {
+  const __nv_bfloat16* p;
+  long long sb, st;
+};
+
+// Bytes the TMA unit delivers for a tile whose atoms in `skip` are filled by plain loads.
+template <int D>
+__device__ __forceinline__ uint32_t tma_tile_bytes(uint32_t skip) {
+  return Tile<D>::kBytes - static_cast<uint32_t>(__popc(skip)) * (8u * 128u) * Tile<D>::kHalves;
+}
+
+// Whole warp: the rows of the atoms in `skip` (see straddled_atoms), read with 16-byte loads
+// from the tensor and written in the 128-byte-swizzled tile layout the TMA boxes produce
+// (16-byte chunk c of a row's 64-column half at chunk c XOR (row mod 8)); rows past the end of
+// the sequence become zeros. Ends with a proxy fence (the tensor core reads the tile) and a
+// warp barrier, after which one lane may signal the tile's barrier.
+template <int D>
+__device__ __noinline__ void fill_atoms(uint32_t dst, uint32_t skip, const Runs tr,
+                                        const TensorRef t, int b, int h) {
+  constexpr int kChunks = D / 8;   // 16-byte chunks per row
+  const int lane = threadIdx.x & 31;
+  for (uint32_t m = skip; m != 0; m &= m - 1) {
+    const int a = __ffs(m) - 1;
+    for (int i = lane; i < 8 * kChunks; i += 32) {
+      const int row = 8 * a + i / kChunks, c = i % kChunks;
+      int src = -1, base = 0;
+#pragma unroll
+      for (int k = 0; k < 3; ++k) {
+        if (k < tr.n && row >= base && row < base + tr.len[k]) src = tr.src[k] + (row - base);
+        base += k < tr.n ? tr.len[k] : 0;
+      }
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (src >= 0)
+        v = __ldg(reinterpret_cast<const uint4*>(t.p + b * t.sb + src * t.st +
+                                                 static_cast<long long>(h) * D + 8 * c));
+      const uint32_t off = (c / 8) * Tile<D>::kHalfBytes + row * 128 + (((c % 8) ^ (row & 7)) * 16);
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + off), "r"(v.x), "r"(v.y),
+                   "r"(v.z), "r"(v.w)
+                   : "memory");
+    }
+  }
+  fence_async_smem();
+  __syncwarp();
+}
+
 // Issue the TMA loads of one 128-row tile of a [B, N, H, D] tensor whose rows are given by
-// `tr`. A single run of 128 rows uses the 128-row box; anything else is moved in 8-row boxes
-// (one swizzle atom each; every run starts and ends on an 8-row boundary), with rows past the
-// sequence read out of bounds so TMA writes zeros. Always delivers Tile<D>::kBytes on `bar`.
+// `tr`, except the atoms in `skip`. A single run of 128 rows uses the 128-row box; anything
+// else is moved in 8-row boxes (one swizzle atom each), with rows past the sequence read out
+// of bounds so TMA writes zeros. Delivers tma_tile_bytes<D>(skip) on `bar`.
 template <int D>
 __device__ __forceinline__ void load_tile(uint32_t dst, const CUtensorMap* m128,
                                           const CUtensorMap* m8, uint32_t bar, int b, int h,
-                                          const Runs& tr, int N) {
+                                          const Runs& tr, int N, uint32_t skip = 0) {
   if (tr.n == 1 && tr.len[0] == kTileRows) {
 #pragma unroll
     for (int half = 0; half < Tile<D>::kHalves; ++half)
       tma_load_4d(dst + half * Tile<D>::kHalfBytes, m128, bar, half * 64, h, tr.src[0], b);
   } else {
     for (int row = 0; row < kTileRows; row += 8) {
+      if ((skip >> (row >> 3)) & 1u) continue;
       int src = N, base = 0;
 #pragma unroll
       for (int k = 0; k < 3; ++k) {
@@ -40,6 +88,22 @@ __device__ __forceinline__ void load_tile(uint32_t dst, const CUtensorMap* m128,
       for (int half = 0; half < Tile<D>::kHalves; ++half)
         tma_load_4d(dst + half * Tile<D>::kHalfBytes + row * 128, m8, bar, half * 64, h, src, b);
     }
+  }
+}
+
+// Producer warp: one tile through the remap. Atoms TMA cannot move are filled by the whole
+// warp first; then lane 0 arms `bar` with the bytes TMA will deliver (plus `extra_tx`, for
+// copies the caller issues on the same barrier) and issues the boxes. Warp-uniform arguments.
+template <int D>
+__device__ __forceinline__ void produce_tile(uint32_t dst, const CUtensorMap* m128,
+                                             const CUtensorMap* m8, uint32_t bar,
+                                             const TensorRef& t, int b, int h, const Runs& tr,
+                                             int N) {
+  const uint32_t skip = straddled_atoms(tr);
+  if (skip) fill_atoms<D>(dst, skip, tr, t, b, h);
+  if ((threadIdx.x & 31) == 0) {
+    mbar_expect_tx(bar, tma_tile_bytes<D>(skip));
+    load_tile<D>(dst, m128, m8, bar, b, h, tr, N, skip);
   }
 }
 
@@ -67,6 +131,19 @@ __device__ __forceinline__ void gemm_ts_mn(uint32_t d_tmem, uint32_t a_tmem, uin
   for (int kk = 0; kk < kTileRows / 16; ++kk)
     mma_ts(d_tmem, a_tmem + kk * 8, b0 + static_cast<uint64_t>((kk * 2048) >> 4), idesc,
            (accumulate || kk > 0) ? 1u : 0u);
+}
+
+// Steps [kk0, kk1) of gemm_ts_mn (16 keys each): the PV product in parts, so a part can start
+// before the whole bf16 A operand is in TMEM.
+template <int D>
+__device__ __forceinline__ void gemm_ts_mn_part(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_base,
+                                                uint32_t idesc, bool accumulate, int kk0, int kk1) {
+  const uint64_t b0 = sdesc_sw128(b_base, Tile<D>::kHalfBytes, 1024);
+#pragma unroll
+  for (int kk = 0; kk < kTileRows / 16; ++kk)
+    if (kk >= kk0 && kk < kk1)
+      mma_ts(d_tmem, a_tmem + kk * 8, b0 + static_cast<uint64_t>((kk * 2048) >> 4), idesc,
+             (accumulate || kk > 0) ? 1u : 0u);
 }
 
 // Dynamic work distribution for the persistent kernels. One thread of the CTA claims units
@@ -133,6 +210,18 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity,
   while (!mbar_try_wait(bar, parity)) {
     if (global_timer_ns() - t0 > timeout_ns) return;
   }
+}
+
+// Producer-warp wait: lane 0 alone polls the barrier (the other lanes park at the warp
+// barrier instead of issuing probes) and the verdict is shared. The lanes' later writes to the
+// freed slot (fill_atoms) execute after lane 0 saw the phase complete, i.e. after the tensor
+// core's reads of it.
+__device__ __forceinline__ bool lead_wait(uint32_t bar, uint32_t parity, const WaitCtx& ctx,
+                                          uint32_t site) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) ok = wait_bar(bar, parity, ctx, site) ? 1 : 0;
+  __syncwarp();
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
 // Warp-uniform wait: every lane waits (each needs the acquire), and the warp proceeds only

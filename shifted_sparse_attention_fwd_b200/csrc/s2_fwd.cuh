@@ -8,9 +8,10 @@
 // moves data: TMA reads the original rows (s2_tiles.cuh) and the epilogue stores O and LSE at
 // the original rows.
 //
-// The kernel is persistent: one CTA per SM sets up its barriers and TMEM once and takes work
-// units blockIdx.x, blockIdx.x + gridDim.x, ... (units are numbered heaviest first), so one
-// unit's epilogue and the next unit's loads overlap the tensor-core work.
+// The kernel is persistent: one CTA per SM sets up its barriers and TMEM once and takes the
+// work units a host-side longest-first schedule gives it (FwdSchedule; units are numbered
+// heaviest first within L2-sized groups), so one unit's epilogue and the next unit's loads
+// overlap the tensor-core work and the CTAs finish together.
 //
 // Warp roles (320 threads):
 //   warps 0-3, 4-7  softmax warpgroup of query tile 0 / 1: thread i owns query row i (TMEM
@@ -37,6 +38,7 @@
 namespace s2 {
 
 struct FwdParams {
+  TensorRef q, k, v;      // the inputs again, for rows the TMA boxes cannot move
   __nv_bfloat16* o;
   long long o_sb, o_st;   // element strides of O's batch and token axes
   float* lse;
@@ -47,6 +49,28 @@ struct FwdParams {
   unsigned int* err;
   unsigned long long timeout_ns;
 };
+
+// Which work units each CTA takes, computed on the host (longest-processing-time-first: the
+// units, in their heaviest-first L2-grouped order, each go to the CTA with the least work so
+// far, by a cost model of (query tile, key tile) steps plus a per-unit overhead) and passed by
+// value with the launch. count = 0: units blockIdx.x, blockIdx.x + gridDim.x, ... instead.
+constexpr int kFwdSchedMaxCtas = 160;
+constexpr int kFwdSchedMaxUnits = 6144;
+struct FwdSchedule {
+  int count;                                  // units in the list (0: round robin)
+  unsigned short start[kFwdSchedMaxCtas + 1];   // CTA c takes unit[start[c] .. start[c + 1])
+  unsigned short unit[kFwdSchedMaxUnits];
+};
+
+// The k-th unit of this CTA, or -1 when it has no more.
+__device__ __forceinline__ int fwd_unit_index(const FwdSchedule& s, int n_units, int k) {
+  if (s.count == 0) {
+    const long long u = blockIdx.x + static_cast<long long>(k) * gridDim.x;
+    return u < n_units ? static_cast<int>(u) : -1;
+  }
+  const int i = s.start[blockIdx.x] + k;
+  return i < s.start[blockIdx.x + 1] ? s.unit[i] : -1;
+}
 
 // Rescale O only when the running max (log2 units) grows by more than this: until then
 // exp2(s - stale max) <= 2^8, harmless in fp32 and bf16, and the final 1/l uses the same max.
@@ -63,7 +87,8 @@ struct FwdLayout {
   static constexpr uint32_t kStage = kV + kVStages * kTile; // ... for each softmax warp
   static constexpr uint32_t kBar = kStage + 8 * kStageWarp;
   enum { B_Q = 0, B_QE = 2, B_K = 4, B_KE = B_K + kKStages, B_V = B_KE + kKStages,
-         B_VE = B_V + kVStages, B_S = B_VE + kVStages, B_P = B_S + 2, B_ODONE = B_P + 2,
+         B_VE = B_V + kVStages, B_S = B_VE + kVStages, B_P = B_S + 2, B_PH = B_P + 2,
+         B_ODONE = B_PH + 2,
          B_DRAIN = B_ODONE + 2, B_COUNT = B_DRAIN + 1 };
   static constexpr uint32_t kTmemSlot = kBar + B_COUNT * 8;
   static constexpr uint32_t kAbort = kTmemSlot + 4;
@@ -132,7 +157,7 @@ __global__ void __launch_bounds__(320, 1)
     s2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQ8,
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmK8,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmV8,
-                  const FwdParams p) {
+                  const FwdParams p, const __grid_constant__ FwdSchedule sched) {
   using L = FwdLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = aligned_smem(smem_raw);
@@ -152,6 +177,7 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(bar(L::B_VE + s), 1);
       mbar_init(bar(L::B_S + s), 1);
       mbar_init(bar(L::B_P + s), 128);
+      mbar_init(bar(L::B_PH + s), 128);
       mbar_init(bar(L::B_ODONE + s), 1);
     }
     for (int s = 0; s < L::kKStages; ++s) {
@@ -176,46 +202,50 @@ __global__ void __launch_bounds__(320, 1)
 
   if (warp == 8) {
     // ---------------- TMA producer ----------------
-    // K(i) (i counts every key tile this CTA loads) goes to slot i % 3 once K(i - 3) has been
-    // released, V(i) to slot i % 2 once V(i - 2) has; within a unit K runs one tile ahead of
-    // V. Q tile t of a unit is loaded once the previous unit's last S MMA on it is done.
-    if (lane == 0) {
+    // The whole warp runs the loop: lane 0 waits on the ring barriers and issues the TMA
+    // copies, and all lanes fill the few tile rows TMA cannot move (produce_tile).
+    // K(i) (i counts every key tile this CTA loads) goes to slot i % 2 once K(i - 2) has been
+    // released, V(i) likewise; within a unit K runs one tile ahead of V. Q tile t of a unit is
+    // loaded once the previous unit's last S MMA on it is done.
+    {
       int k_issued = 0, v_issued = 0, q_loads[2] = {0, 0};
       bool ok = true;
       auto issue_k = [&](const FwdUnit& u, int j) -> bool {
         const int i = k_issued, st = i % L::kKStages;
         if (i >= L::kKStages &&
-            !wait_bar(bar(L::B_KE + st), ((i / L::kKStages) - 1) & 1, ctx, 1))
+            !lead_wait(bar(L::B_KE + st), ((i / L::kKStages) - 1) & 1, ctx, 1))
           return false;
-        mbar_expect_tx(bar(L::B_K + st), L::kTile);
-        load_tile<D>(sbase + L::kK + st * L::kTile, &tmK, &tmK8, bar(L::B_K + st), u.b, u.kvh,
-                     rolled_runs(head_remap(p.N, p.G, u.shift_h, kFront ? u.front_h : 0), (u.kv_lo + j) * kTileRows), p.N);
+        produce_tile<D>(sbase + L::kK + st * L::kTile, &tmK, &tmK8, bar(L::B_K + st), p.k, u.b,
+                        u.kvh, rolled_runs(head_remap(p.N, p.G, u.shift_h, kFront ? u.front_h : 0),
+                                           (u.kv_lo + j) * kTileRows), p.N);
         ++k_issued;
         return true;
       };
       auto issue_v = [&](const FwdUnit& u, int j) -> bool {
         const int i = v_issued, st = i % L::kVStages;
         if (i >= L::kVStages &&
-            !wait_bar(bar(L::B_VE + st), ((i / L::kVStages) - 1) & 1, ctx, 9))
+            !lead_wait(bar(L::B_VE + st), ((i / L::kVStages) - 1) & 1, ctx, 9))
           return false;
-        mbar_expect_tx(bar(L::B_V + st), L::kTile);
-        load_tile<D>(sbase + L::kV + st * L::kTile, &tmV, &tmV8, bar(L::B_V + st), u.b, u.kvh,
-                     rolled_runs(head_remap(p.N, p.G, u.shift_h, kFront ? u.front_h : 0), (u.kv_lo + j) * kTileRows), p.N);
+        produce_tile<D>(sbase + L::kV + st * L::kTile, &tmV, &tmV8, bar(L::B_V + st), p.v, u.b,
+                        u.kvh, rolled_runs(head_remap(p.N, p.G, u.shift_h, kFront ? u.front_h : 0),
+                                           (u.kv_lo + j) * kTileRows), p.N);
         ++v_issued;
         return true;
       };
-      for (int unit = blockIdx.x; ok && unit < n_units; unit += gridDim.x) {
+      for (int ku = 0; ok; ++ku) {
+        const int unit = fwd_unit_index(sched, n_units, ku);
+        if (unit < 0) break;
         const FwdUnit u = fwd_unit<kFront>(p, unit);
         ok = issue_k(u, 0);   // the first key tile can stream while the last unit finishes
         for (int t = 0; ok && t < 2; ++t) {
           if (!u.tv[t]) continue;
-          if (q_loads[t] > 0 && !wait_bar(bar(L::B_QE + t), (q_loads[t] - 1) & 1, ctx, 10)) {
+          if (q_loads[t] > 0 && !lead_wait(bar(L::B_QE + t), (q_loads[t] - 1) & 1, ctx, 10)) {
             ok = false;
             break;
           }
-          mbar_expect_tx(bar(L::B_Q + t), L::kTile);
-          load_tile<D>(sbase + L::kQ + t * L::kTile, &tmQ, &tmQ8, bar(L::B_Q + t), u.b, u.h,
-                       rolled_runs(head_remap(p.N, p.G, u.shift_h, kFront ? u.front_h : 0), u.qt[t] * kTileRows), p.N);
+          produce_tile<D>(sbase + L::kQ + t * L::kTile, &tmQ, &tmQ8, bar(L::B_Q + t), p.q, u.b,
+                          u.h, rolled_runs(head_remap(p.N, p.G, u.shift_h, kFront ? u.front_h : 0),
+                                           u.qt[t] * kTileRows), p.N);
           ++q_loads[t];
         }
         for (int j = 0; ok && j < u.n_kv; ++j) {
@@ -224,12 +254,14 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
       // Every issued copy lands before the CTA can exit.
-      for (int t = 0; t < 2; ++t)
-        if (q_loads[t] > 0) drain_wait(bar(L::B_Q + t), (q_loads[t] - 1) & 1, p.timeout_ns);
-      for (int i = k_issued - L::kKStages; i < k_issued; ++i)
-        if (i >= 0) drain_wait(bar(L::B_K + i % L::kKStages), (i / L::kKStages) & 1, p.timeout_ns);
-      for (int i = v_issued - L::kVStages; i < v_issued; ++i)
-        if (i >= 0) drain_wait(bar(L::B_V + i % L::kVStages), (i / L::kVStages) & 1, p.timeout_ns);
+      if (lane == 0) {
+        for (int t = 0; t < 2; ++t)
+          if (q_loads[t] > 0) drain_wait(bar(L::B_Q + t), (q_loads[t] - 1) & 1, p.timeout_ns);
+        for (int i = k_issued - L::kKStages; i < k_issued; ++i)
+          if (i >= 0) drain_wait(bar(L::B_K + i % L::kKStages), (i / L::kKStages) & 1, p.timeout_ns);
+        for (int i = v_issued - L::kVStages; i < v_issued; ++i)
+          if (i >= 0) drain_wait(bar(L::B_V + i % L::kVStages), (i / L::kVStages) & 1, p.timeout_ns);
+      }
     }
   } else if (warp == 9) {
     // ---------------- MMA issuer ----------------
@@ -241,7 +273,9 @@ __global__ void __launch_bounds__(320, 1)
       auto wait_k = [&](int i) {
         return wait_bar(bar(L::B_K + i % L::kKStages), (i / L::kKStages) & 1, ctx, 3);
       };
-      for (int unit = blockIdx.x; ok && unit < n_units; unit += gridDim.x) {
+      for (int ku = 0; ok; ++ku) {
+        const int unit = fwd_unit_index(sched, n_units, ku);
+        if (unit < 0) break;
         const FwdUnit u = fwd_unit<kFront>(p, unit);
         bool q_ready[2] = {false, false}, first_pv[2] = {true, true};
         // S_t(j) = Q_t K(j)^T into TMEM columns [128 t, 128 t + 128).
@@ -272,14 +306,20 @@ __global__ void __launch_bounds__(320, 1)
           bool v_ready = false, k_next_ready = false;
           for (int t = 0; ok && t < 2; ++t) {
             if (u.part(t, kt)) {
-              if (!wait_bar(bar(L::B_P + t), pcount[t] & 1, ctx, 4)) { ok = false; break; }
+              // O_t += P_t V in two halves of 64 keys: the first starts as soon as the
+              // softmax warpgroup has stored that half of P_t.
+              if (!wait_bar(bar(L::B_PH + t), pcount[t] & 1, ctx, 11)) { ok = false; break; }
               if (!v_ready) {
                 if (!wait_bar(bar(L::B_V + vst), (vi / L::kVStages) & 1, ctx, 5)) { ok = false; break; }
                 v_ready = true;
               }
               tc_fence_after();
-              gemm_ts_mn<D>(tmem + 256 + t * D, tmem + t * 128, sbase + L::kV + vst * L::kTile,
-                            idesc_pv, !first_pv[t]);
+              gemm_ts_mn_part<D>(tmem + 256 + t * D, tmem + t * 128, sbase + L::kV + vst * L::kTile,
+                                 idesc_pv, !first_pv[t], 0, 4);
+              if (!wait_bar(bar(L::B_P + t), pcount[t] & 1, ctx, 4)) { ok = false; break; }
+              tc_fence_after();
+              gemm_ts_mn_part<D>(tmem + 256 + t * D, tmem + t * 128, sbase + L::kV + vst * L::kTile,
+                                 idesc_pv, true, 4, 8);
               first_pv[t] = false;
               ++pcount[t];
               if (kt == u.ke[t]) mma_commit(bar(L::B_ODONE + t));
@@ -310,7 +350,9 @@ __global__ void __launch_bounds__(320, 1)
     const float c = p.scale_log2;
     int s_cnt = 0, o_cnt = 0;
     bool ok = true;
-    for (int unit = blockIdx.x; ok && unit < n_units; unit += gridDim.x) {
+    for (int ku = 0; ok; ++ku) {
+      const int unit = fwd_unit_index(sched, n_units, ku);
+      if (unit < 0) break;
       const FwdUnit u = fwd_unit<kFront>(p, unit);
       if (!u.tv[wg]) continue;
       const int r = u.qt[wg] * kTileRows + row;
@@ -367,6 +409,11 @@ __global__ void __launch_bounds__(320, 1)
             pk[i] = pack_bf16(e0, e1);
           }
           tmem_st16(s_col + 16 * j, pk);
+          if (j == 1) {   // keys 0-63 of P are in TMEM: the first half of the PV MMA may start
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(bar(L::B_PH + wg));
+          }
         }
         acc[0] = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
         l_run += f2_lo(acc[0]) + f2_hi(acc[0]);

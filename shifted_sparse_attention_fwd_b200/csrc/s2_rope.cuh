@@ -22,7 +22,7 @@ constexpr int kRopeThreads = 256;
 
 template <int D>
 __global__ void __launch_bounds__(kRopeThreads) s2_rope_kernel(
-    const __nv_bfloat16* __restrict__ x, __nv_bfloat16* __restrict__ y, int N, int H,
+    const __nv_bfloat16* x, __nv_bfloat16* y, int N, int H,
     long long x_sb, long long x_st, long long y_sb, long long y_st, float log2_base,
     float pi_scale, float sin_sign) {
   constexpr int kHalf = D / 2;

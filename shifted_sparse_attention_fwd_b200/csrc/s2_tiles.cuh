@@ -1,8 +1,8 @@
 // The per-head shift-and-group remap, applied to 128-row tiles.
 //
 // LongLoRA summary page, §3.4 Algorithm 1: the second chunk of heads is rolled by -G/2
-// along N before the attention, viewed as groups of G (".view(B*N/G, G, ...)"), attended
-// causally per group, and rolled back after it. Instead of materialising the roll, every kernel
+// along N before the attention, cut into independent groups of G consecutive rolled rows,
+// attended causally per group, and rolled back after it. Instead of materialising the roll, every kernel
 // addresses the original tensors through
 //     t = (r + s_h) mod N          (rolled row r -> original token t)
 // where s_h is the head's roll (G/2 for the shifted heads, 0 otherwise); group of rolled
@@ -137,6 +137,21 @@ __host__ __device__ inline Runs identity_runs(int t0, int N) {
   t.len[0] = t.valid;
   t.src[0] = t0;
   return t;
+}
+
+// TMA moves whole 8-row atoms (one 128-byte swizzle period). An atom that holds rows of two
+// different runs (a run boundary that is not a multiple of 8 rows into the tile, which happens
+// when G or the roll is not a multiple of 8) cannot be one box: bit a of the result marks such an
+// atom a. The kernels load the rows of these atoms with plain loads instead.
+__host__ __device__ inline unsigned int straddled_atoms(const Runs& tr) {
+  unsigned int m = 0;
+  int end = 0;
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    end += tr.len[k];
+    if (k + 1 < tr.n && (end & 7)) m |= 1u << (end >> 3);
+  }
+  return m;
 }
 
 // First rolled row of the group containing rolled row r, and one past its last row. With a

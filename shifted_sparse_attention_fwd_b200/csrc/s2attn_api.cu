@@ -3,8 +3,13 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
+#include <functional>
+#include <queue>
+#include <utility>
+#include <vector>
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
@@ -22,7 +27,7 @@ namespace {
 
 __device__ unsigned int g_err_word;   // first pipeline-wait failure since the last read
 
-constexpr int kAbiVersion = 3;
+constexpr int kAbiVersion = 4;
 constexpr int kMaxDevices = 64;
 constexpr unsigned long long kDefaultTimeoutNs = 1000000000ull;
 
@@ -64,10 +69,17 @@ cudaError_t set_smem_attrs_variant() {
 // Every kernel exists twice: with the plain-roll index code only, and with the Variant 3
 // reordering compiled in (S2ATTN_FLAG_WRAP_FRONT_FIRST), so the common case pays nothing
 // for the general remap.
+// Largest dynamic shared memory the streaming preprocess may request.
+constexpr uint32_t kPreSmemMax = 220 * 1024;
+
 template <int D>
 cudaError_t set_smem_attrs() {
-  const cudaError_t e = set_smem_attrs_variant<D, false>();
-  return e != cudaSuccess ? e : set_smem_attrs_variant<D, true>();
+  cudaError_t e = set_smem_attrs_variant<D, false>();
+  if (e != cudaSuccess) return e;
+  e = set_smem_attrs_variant<D, true>();
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(s2::s2_bwd_pre_stream_kernel<D>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, kPreSmemMax);
 }
 
 // Per-device one-time set-up (with that device current): the device address of the error
@@ -202,19 +214,18 @@ int ds_heads_per_pass(const Shape& sh, size_t bytes) {
 s2attn_status check_shape(int B, int Hq, int Hkv, int N, int d, int G, float scale,
                           int shift_head_begin, long long shift, Shape& out, int flags = 0) {
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || N <= 0 || d <= 0 || G <= 0) return S2ATTN_ERR_INVALID_ARG;
-  if (Hq % Hkv != 0 || G % 2 != 0) return S2ATTN_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return S2ATTN_ERR_INVALID_ARG;
   // G must divide N unless the caller asks for a shorter last group
   if (N % G != 0 && !(flags & S2ATTN_FLAG_PARTIAL_LAST_GROUP)) return S2ATTN_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !std::isfinite(scale)) return S2ATTN_ERR_INVALID_ARG;
   if (shift_head_begin < 0 || shift_head_begin > Hq) return S2ATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return S2ATTN_ERR_UNSUPPORTED;
   if (N >= (1 << 30)) return S2ATTN_ERR_UNSUPPORTED;
-  if (G % 8 != 0) return S2ATTN_ERR_UNSUPPORTED;
-  if (N % 8 != 0) return S2ATTN_ERR_UNSUPPORTED;   // (implied by G | N; tiles are 8-row runs)
+  // Any G and roll: tile rows that the 8-row TMA boxes cannot move (a run of the remap that
+  // starts or ends inside an 8-row atom) are loaded with plain loads by the producer warps.
   long long s = shift % N;
   if (s < 0) s += N;
   if (shift_head_begin == Hq) s = 0;   // no head is rolled: the roll amount is irrelevant
-  if (s % 8 != 0) return S2ATTN_ERR_UNSUPPORTED;
   const long long rows = static_cast<long long>(B) * (Hq > Hkv ? Hq : Hkv) * ((N + 127) / 128);
   if (rows >= (1ll << 31)) return S2ATTN_ERR_UNSUPPORTED;
   constexpr int kVariants = S2ATTN_FLAG_WRAP_OWN_GROUP | S2ATTN_FLAG_WRAP_FRONT_FIRST;
@@ -231,6 +242,67 @@ s2attn_status check_shape(int B, int Hq, int Hkv, int N, int d, int G, float sca
   return S2ATTN_OK;
 }
 
+// The forward's per-CTA unit lists (s2::FwdSchedule): longest-processing-time-first over the
+// units in their kernel order, by a cost of (query tile, key tile) steps plus 2 for the unit's
+// own loads and epilogue. Round robin (count = 0) when the lists would not fit the launch.
+void fwd_schedule(const Shape& sh, int grid, s2::FwdSchedule& out) {
+  out.count = 0;
+  const int nqt = (sh.N + s2::kTileRows - 1) / s2::kTileRows;
+  const long long n_units = static_cast<long long>(sh.B) * sh.Hq * s2::query_pairs_per_head(sh.N);
+  if (n_units > s2::kFwdSchedMaxUnits || grid > s2::kFwdSchedMaxCtas || n_units <= grid) return;
+  std::priority_queue<std::pair<double, int>, std::vector<std::pair<double, int>>,
+                      std::greater<std::pair<double, int>>> load;
+  for (int c = 0; c < grid; ++c) load.push({0.0, c});
+  std::vector<int> owner(n_units), count(grid, 0);
+  for (int u = 0; u < n_units; ++u) {
+    int b, h, pair;
+    s2::query_pair_coords_chunked(u, sh.B, sh.Hq, sh.N, sh.G, s2::kL2Chunk, b, h, pair);
+    const int wrap_h = h >= sh.shb ? sh.wrap : s2::kNoWrapSplit;
+    double cost = 2.0;
+    for (int t = 0; t < 2; ++t) {
+      const int qt = 2 * pair + t;
+      if (qt < nqt) cost += qt - s2::group_begin(qt * s2::kTileRows, sh.G, wrap_h) / s2::kTileRows + 1;
+    }
+    const auto least = load.top();
+    load.pop();
+    owner[u] = least.second;
+    ++count[least.second];
+    load.push({least.first + cost, least.second});
+  }
+  out.start[0] = 0;
+  for (int c = 0; c < grid; ++c) out.start[c + 1] = static_cast<unsigned short>(out.start[c] + count[c]);
+  std::vector<int> fill(out.start, out.start + grid);
+  for (int u = 0; u < n_units; ++u) out.unit[fill[owner[u]]++] = static_cast<unsigned short>(u);
+  out.count = static_cast<int>(n_units);
+}
+
+// Recently used schedules (the same shapes recur call after call).
+struct FwdScheduleCache {
+  std::mutex mu;
+  struct Entry {
+    long long key[9];
+    s2::FwdSchedule sched;
+  };
+  std::vector<Entry> entries;   // most recent last, at most 4
+};
+FwdScheduleCache g_fwd_sched;
+
+void fwd_schedule_cached(const Shape& sh, int grid, s2::FwdSchedule& out) {
+  const long long key[9] = {sh.B, sh.Hq, sh.N, sh.G, sh.shb, sh.shift, sh.wrap, sh.front, grid};
+  std::lock_guard<std::mutex> lock(g_fwd_sched.mu);
+  auto& es = g_fwd_sched.entries;
+  for (size_t i = 0; i < es.size(); ++i)
+    if (std::equal(key, key + 9, es[i].key)) {
+      out = es[i].sched;
+      return;
+    }
+  fwd_schedule(sh, grid, out);
+  if (es.size() == 4) es.erase(es.begin());
+  es.emplace_back();
+  std::copy(key, key + 9, es.back().key);
+  es.back().sched = out;
+}
+
 template <int D>
 s2attn_status launch_fwd(const Shape& sh, const void* q, const void* k, const void* v, void* o,
                          float* lse, float scale, cudaStream_t stream, unsigned int* err,
@@ -241,6 +313,9 @@ s2attn_status launch_fwd(const Shape& sh, const void* q, const void* k, const vo
   if ((s = encode_pair(mk, k, sh.B, sh.Hkv, sh.N, D, sh.sb[T_K], sh.st[T_K])) != S2ATTN_OK) return s;
   if ((s = encode_pair(mv, v, sh.B, sh.Hkv, sh.N, D, sh.sb[T_V], sh.st[T_V])) != S2ATTN_OK) return s;
   s2::FwdParams p{};
+  p.q = s2::TensorRef{static_cast<const __nv_bfloat16*>(q), sh.sb[T_Q], sh.st[T_Q]};
+  p.k = s2::TensorRef{static_cast<const __nv_bfloat16*>(k), sh.sb[T_K], sh.st[T_K]};
+  p.v = s2::TensorRef{static_cast<const __nv_bfloat16*>(v), sh.sb[T_V], sh.st[T_V]};
   p.o = static_cast<__nv_bfloat16*>(o);
   p.o_sb = sh.sb[T_O];
   p.o_st = sh.st[T_O];
@@ -254,12 +329,14 @@ s2attn_status launch_fwd(const Shape& sh, const void* q, const void* k, const vo
   p.timeout_ns = g_timeout_ns.load();
   const unsigned units = static_cast<unsigned>(sh.B) * sh.Hq * s2::query_pairs_per_head(sh.N);
   const unsigned grid = units < static_cast<unsigned>(num_sms) ? units : static_cast<unsigned>(num_sms);
+  static thread_local s2::FwdSchedule sched;
+  fwd_schedule_cached(sh, static_cast<int>(grid), sched);
   if (sh.front)
     s2::s2_fwd_kernel<D, true><<<grid, s2::FwdLayout<D>::kThreads, s2::FwdLayout<D>::kLaunchBytes,
-                                 stream>>>(mq.m128, mq.m8, mk.m128, mk.m8, mv.m128, mv.m8, p);
+                                 stream>>>(mq.m128, mq.m8, mk.m128, mk.m8, mv.m128, mv.m8, p, sched);
   else
     s2::s2_fwd_kernel<D, false><<<grid, s2::FwdLayout<D>::kThreads, s2::FwdLayout<D>::kLaunchBytes,
-                                  stream>>>(mq.m128, mq.m8, mk.m128, mk.m8, mv.m128, mv.m8, p);
+                                  stream>>>(mq.m128, mq.m8, mk.m128, mk.m8, mv.m128, mv.m8, p, sched);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? S2ATTN_OK : cuda_fail(e, "s2_fwd_kernel launch");
 }
@@ -301,17 +378,44 @@ void set_ds_pass(s2::BwdParams& p, const Shape& sh, const void* workspace, int k
                                           ws_min_bytes(sh.B, sh.Hq, sh.N));
 }
 
+// Tokens per stage of the streaming preprocess: about 32 KB of each tensor per stage, at least
+// one token; 0 when one token's heads do not fit the ring (the plain-load kernel runs then).
+int pre_tokens_per_stage(int Hq, int d) {
+  const long long row = static_cast<long long>(Hq) * d * 2;
+  const long long tps = row >= s2::kPreStageMax ? 1 : s2::kPreStageMax / row;
+  return s2::pre_smem_bytes(static_cast<int>(tps), Hq, d) <= kPreSmemMax ? static_cast<int>(tps) : 0;
+}
+
 template <int D>
 s2attn_status launch_pre(const Shape& sh, const void* o, const float* lse, const void* dO,
-                         void* workspace, cudaStream_t stream) {
+                         void* workspace, cudaStream_t stream, unsigned int* err, int num_sms) {
   const size_t half = ws_half(sh.B, sh.Hq, sh.N);
   float* dvec = static_cast<float*>(workspace);
   float* lse2 = reinterpret_cast<float*>(static_cast<char*>(workspace) + half);
-  const unsigned grid = static_cast<unsigned>(sh.B) * ((sh.N + s2::kPreTokens - 1) / s2::kPreTokens);
-  s2::s2_bwd_pre_kernel<D><<<grid, 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, dvec,
-      lse2, ws_sched(workspace, sh), kSchedWords, sh.Hq, sh.N, sh.sb[T_O], sh.st[T_O],
-      sh.sb[T_DO], sh.st[T_DO]);
+  const int tps = pre_tokens_per_stage(sh.Hq, D);
+  if (tps > 0) {
+    s2::PreParams p{};
+    p.o = static_cast<const __nv_bfloat16*>(o);
+    p.dO = static_cast<const __nv_bfloat16*>(dO);
+    p.o_sb = sh.sb[T_O]; p.o_st = sh.st[T_O];
+    p.do_sb = sh.sb[T_DO]; p.do_st = sh.st[T_DO];
+    p.lse = lse; p.dvec = dvec; p.lse2 = lse2;
+    p.sched = ws_sched(workspace, sh);
+    p.sched_words = kSchedWords;
+    p.B = sh.B; p.Hq = sh.Hq; p.N = sh.N; p.tps = tps;
+    p.err = err;
+    p.timeout_ns = g_timeout_ns.load();
+    const long long stages = (static_cast<long long>(sh.B) * sh.N + tps - 1) / tps;
+    const unsigned grid = static_cast<unsigned>(stages < num_sms ? stages : num_sms);
+    s2::s2_bwd_pre_stream_kernel<D><<<grid, s2::kPreThreads, s2::pre_smem_bytes(tps, sh.Hq, D),
+                                      stream>>>(p);
+  } else {
+    const unsigned grid = static_cast<unsigned>(sh.B) * ((sh.N + s2::kPreTokens - 1) / s2::kPreTokens);
+    s2::s2_bwd_pre_kernel<D><<<grid, 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, dvec,
+        lse2, ws_sched(workspace, sh), kSchedWords, sh.Hq, sh.N, sh.sb[T_O], sh.st[T_O],
+        sh.sb[T_DO], sh.st[T_DO]);
+  }
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? S2ATTN_OK : cuda_fail(e, "s2_bwd_pre_kernel launch");
 }
@@ -328,6 +432,10 @@ s2attn_status launch_grad(const Shape& sh, const void* q, const void* k, const v
   if ((s = encode_pair(mv, v, sh.B, sh.Hkv, sh.N, D, sh.sb[T_V], sh.st[T_V])) != S2ATTN_OK) return s;
   if ((s = encode_pair(mo, dO, sh.B, sh.Hq, sh.N, D, sh.sb[T_DO], sh.st[T_DO])) != S2ATTN_OK) return s;
   s2::BwdParams p = bwd_params(sh, scale, workspace, dq, dk, dv, err);
+  p.q = s2::TensorRef{static_cast<const __nv_bfloat16*>(q), sh.sb[T_Q], sh.st[T_Q]};
+  p.k = s2::TensorRef{static_cast<const __nv_bfloat16*>(k), sh.sb[T_K], sh.st[T_K]};
+  p.v = s2::TensorRef{static_cast<const __nv_bfloat16*>(v), sh.sb[T_V], sh.st[T_V]};
+  p.dO = s2::TensorRef{static_cast<const __nv_bfloat16*>(dO), sh.sb[T_DO], sh.st[T_DO]};
   if (ds_kvh_begin >= 0) set_ds_pass(p, sh, workspace, ds_kvh_begin, ds_kvh_count);
   const unsigned tiles = (sh.N + 127) / 128;
   if (kDkdv) {
@@ -420,9 +528,9 @@ s2attn_status dq_ds_impl(const Shape& sh, const void* k, void* dq, float scale, 
                     : launch_dq_ds<128>(sh, k, dq, scale, ws, kvh_begin, kvh_count, stream, err, num_sms);
 }
 s2attn_status pre_impl(const Shape& sh, const void* o, const float* lse, const void* dO, void* ws,
-                       cudaStream_t stream) {
-  return sh.d == 64 ? launch_pre<64>(sh, o, lse, dO, ws, stream)
-                    : launch_pre<128>(sh, o, lse, dO, ws, stream);
+                       cudaStream_t stream, unsigned int* err, int num_sms) {
+  return sh.d == 64 ? launch_pre<64>(sh, o, lse, dO, ws, stream, err, num_sms)
+                    : launch_pre<128>(sh, o, lse, dO, ws, stream, err, num_sms);
 }
 
 // Caller-given strides for tensors ids[0..n): strides[2i] = batch, strides[2i+1] = token (in
@@ -560,7 +668,10 @@ s2attn_status s2attn_bwd_preprocess(const void* o, const float* lse, const void*
   sh.set_contiguous();
   s2attn_status s = check_workspace(sh, workspace, workspace_bytes);
   if (s != S2ATTN_OK) return s;
-  return pre_impl(sh, o, lse, dO, workspace, static_cast<cudaStream_t>(stream));
+  unsigned int* err = nullptr;
+  int num_sms = 0;
+  if ((s = device_state(&err, &num_sms)) != S2ATTN_OK) return s;
+  return pre_impl(sh, o, lse, dO, workspace, static_cast<cudaStream_t>(stream), err, num_sms);
 }
 
 s2attn_status s2attn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO,
@@ -648,6 +759,74 @@ s2attn_status s2attn_bwd_dq_ds(const void* k, void* dq, int B, int Hq, int Hkv, 
                     num_sms);
 }
 
+// Shape, option flags and strides of the phase entry points (strides: the 8 {sb, st} pairs of
+// s2attn_bwd_general; the pairs of tensors a phase does not touch are validated all the same).
+s2attn_status phase_shape(int B, int Hq, int Hkv, int N, int d, int G, float scale,
+                          int shift_head_begin, int shift, int flags, const long long* strides,
+                          Shape& sh) {
+  s2attn_status s = check_shape(B, Hq, Hkv, N, d, G, scale, shift_head_begin, shift, sh, flags);
+  if (s != S2ATTN_OK) return s;
+  if (strides) {
+    static const int ids[8] = {T_Q, T_K, T_V, T_O, T_DO, T_DQ, T_DK, T_DV};
+    if ((s = apply_strides(sh, strides, ids, 8)) != S2ATTN_OK) return s;
+  }
+  return S2ATTN_OK;
+}
+
+s2attn_status s2attn_bwd_dkdv_ds_general(const void* q, const void* k, const void* v,
+                                         const void* dO, void* dk, void* dv, int B, int Hq,
+                                         int Hkv, int N, int d, int G, float scale,
+                                         int shift_head_begin, int shift, int flags,
+                                         const long long* strides, void* workspace,
+                                         size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !dO || !dk || !dv) return S2ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dO) || !aligned16(dk) ||
+      !aligned16(dv))
+    return S2ATTN_ERR_INVALID_ARG;
+  Shape sh;
+  s2attn_status s = phase_shape(B, Hq, Hkv, N, d, G, scale, shift_head_begin, shift, flags,
+                                strides, sh);
+  if (s != S2ATTN_OK) return s;
+  if ((s = check_workspace(sh, workspace, workspace_bytes)) != S2ATTN_OK) return s;
+  if (ds_heads_per_pass(sh, workspace_bytes) < Hkv) {
+    std::snprintf(g_last_error, sizeof(g_last_error),
+                  "s2attn_bwd_dkdv_ds_general: workspace of %zu bytes holds the dS tiles of fewer "
+                  "than all %d kv heads", workspace_bytes, Hkv);
+    return S2ATTN_ERR_INVALID_ARG;
+  }
+  if ((s = get_encoder()) != S2ATTN_OK) return s;
+  unsigned int* err = nullptr;
+  int num_sms = 0;
+  if ((s = device_state(&err, &num_sms)) != S2ATTN_OK) return s;
+  return dkdv_ds_impl(sh, q, k, v, dO, dk, dv, scale, workspace, 0, Hkv,
+                      static_cast<cudaStream_t>(stream), err, num_sms);
+}
+
+s2attn_status s2attn_bwd_dq_ds_general(const void* k, void* dq, int B, int Hq, int Hkv, int N,
+                                       int d, int G, float scale, int shift_head_begin,
+                                       int shift, int flags, const long long* strides,
+                                       const void* workspace, size_t workspace_bytes,
+                                       void* stream) {
+  if (!k || !dq || !aligned16(k) || !aligned16(dq)) return S2ATTN_ERR_INVALID_ARG;
+  Shape sh;
+  s2attn_status s = phase_shape(B, Hq, Hkv, N, d, G, scale, shift_head_begin, shift, flags,
+                                strides, sh);
+  if (s != S2ATTN_OK) return s;
+  if ((s = check_workspace(sh, workspace, workspace_bytes)) != S2ATTN_OK) return s;
+  if (ds_heads_per_pass(sh, workspace_bytes) < Hkv) {
+    std::snprintf(g_last_error, sizeof(g_last_error),
+                  "s2attn_bwd_dq_ds_general: workspace of %zu bytes holds the dS tiles of fewer "
+                  "than all %d kv heads", workspace_bytes, Hkv);
+    return S2ATTN_ERR_INVALID_ARG;
+  }
+  if ((s = get_encoder()) != S2ATTN_OK) return s;
+  unsigned int* err = nullptr;
+  int num_sms = 0;
+  if ((s = device_state(&err, &num_sms)) != S2ATTN_OK) return s;
+  return dq_ds_impl(sh, k, dq, scale, workspace, 0, Hkv, static_cast<cudaStream_t>(stream), err,
+                    num_sms);
+}
+
 s2attn_status s2attn_bwd_general(const void* q, const void* k, const void* v, const void* o,
                                  const float* lse, const void* dO, void* dq, void* dk, void* dv,
                                  int B, int Hq, int Hkv, int N, int d, int G, float scale,
@@ -671,7 +850,7 @@ s2attn_status s2attn_bwd_general(const void* q, const void* k, const void* v, co
   int num_sms = 0;
   if ((s = device_state(&err, &num_sms)) != S2ATTN_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if ((s = pre_impl(sh, o, lse, dO, workspace, st)) != S2ATTN_OK) return s;
+  if ((s = pre_impl(sh, o, lse, dO, workspace, st, err, num_sms)) != S2ATTN_OK) return s;
   const int per_pass = ds_heads_per_pass(sh, workspace_bytes);
   if (per_pass == 0) {
     // Workspace too small for one kv head's dS tiles: the dQ kernel recomputes S and dP.

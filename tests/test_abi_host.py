@@ -50,7 +50,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.s2attn_abi_version() == 3
+    assert lib.s2attn_abi_version() == 4
     for st in range(5):
         assert s2.status_string(st)
     assert s2.status_string(99) == "unknown status"
@@ -80,19 +80,16 @@ def fwd_ex_call(lib, shb, shift, **kw):
 @pytest.mark.parametrize("kw,status", [
     (dict(q=None), 1), (dict(lse=None), 1), (dict(k=A + 8), 1), (dict(o=A + 2), 1),
     (dict(B=0), 1), (dict(N=-8), 1), (dict(Hq=3, Hkv=3), 1), (dict(Hkv=3), 1),
-    (dict(N=200), 1), (dict(G=63, N=63 * 4), 1), (dict(scale=0.0), 1),
+    (dict(N=200), 1), (dict(scale=0.0), 1),
     (dict(scale=float("nan")), 1), (dict(scale=float("inf")), 1), (dict(scale=-1.0), 1),
-    (dict(d=96), 2), (dict(d=256), 2), (dict(G=24, N=240), 2), (dict(G=8, N=64), 2),
-    (dict(N=1 << 30, G=1 << 29), 2),
+    (dict(d=96), 2), (dict(d=256), 2), (dict(N=1 << 30, G=1 << 29), 2),
 ])
 def test_fwd_rejects(lib, kw, status):
     assert fwd_call(lib, **kw) == status
 
 
 @pytest.mark.parametrize("shb,shift,kw,status", [
-    (-1, 32, {}, 1), (5, 32, {}, 1), (2, 4, {}, 2), (2, 36, {}, 2),
-    # G=24: G/2 = 12 is not a multiple of 8, but a roll of 8 (or none) is fine -> reaches
-    # CUDA set-up, which is not available here; we only check it is not rejected as bad shape
+    (-1, 32, {}, 1), (5, 32, {}, 1), (5, 4, {}, 1),
 ])
 def test_fwd_ex_rejects(lib, shb, shift, kw, status):
     assert fwd_ex_call(lib, shb, shift, **kw) == status
@@ -115,8 +112,23 @@ def test_bwd_rejects(lib):
     assert lib.s2attn_bwd_preprocess(A, A, A, 1, 4, 256, 80, ws, need, None) == 2
     assert lib.s2attn_bwd_dq(A, A, A, A, None, 1, 4, 4, 256, 64, 64, ctypes.c_float(0.1), 2,
                              32, ws, need, None) == 1
-    assert lib.s2attn_bwd_dkdv(A, A, A, A, A, A, 1, 4, 4, 256, 64, 64, ctypes.c_float(0.1), 2,
+    assert lib.s2attn_bwd_dkdv(A, A, A, A, A, A, 1, 4, 4, 256, 96, 64, ctypes.c_float(0.1), 2,
                                36, ws, need, None) == 2
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,d,G,shb,shift,flags", [
+    (1, 32, 32, 8192, 128, 1365, 16, 682, 4),   # the page's 1/6 group (Table 7), rolled by 682
+    (1, 4, 4, 300, 64, 75, 2, 37, 0),           # odd G, odd roll
+    (1, 4, 2, 1000, 64, 333, 2, 166, 4),        # odd G, shorter last group
+    (1, 4, 4, 693, 64, 231, 2, 115, 1),         # odd G, Variant 2
+    (1, 4, 4, 512, 128, 128, 2, 37, 2),         # a roll of 37, Variant 3
+    (2, 2, 2, 129, 64, 43, 1, 21, 0),           # N, G, roll all odd
+    (1, 2, 2, 250, 64, 24, 1, 12, 4),           # G/2 not a multiple of 8
+])
+def test_any_group_and_roll_accepted(lib, B, Hq, Hkv, N, d, G, shb, shift, flags):
+    """G and the roll need not be multiples of 8 (nor G even): validation accepts them (the
+    workspace query runs the same checks without touching a device)."""
+    assert lib.s2attn_bwd_workspace_size_general(B, Hq, Hkv, N, d, G, shb, shift, flags, 0) > 0
 
 
 # --------------------------------------------------------------------------------------
@@ -130,6 +142,8 @@ static void put_runs(const s2::Runs& t, int* o) {
   for (int k = 0; k < t.n; ++k) { o[2 + 2 * k] = t.len[k]; o[3 + 2 * k] = t.src[k]; } }
 void rolled_runs(int r0, int shift, int N, int G, int front, int* o) {
   put_runs(s2::rolled_runs(s2::head_remap(N, G, shift, front), r0), o); }
+unsigned straddled(int r0, int shift, int N, int G, int front) {
+  return s2::straddled_atoms(s2::rolled_runs(s2::head_remap(N, G, shift, front), r0)); }
 void token_runs(int t0, int shift, int N, int G, int front, int* o) {
   put_runs(s2::token_runs(s2::head_remap(N, G, shift, front), t0), o); }
 int qtiles(int t0, int sh, int N, int G, int W, int front, int* o) {
@@ -199,14 +213,19 @@ def listed(fn, *args):
 
 CASES = [(256, 64, 32), (8192, 2048, 1024), (320, 64, 32), (384, 192, 96), (200, 200, 0),
          (96, 32, 16), (1024, 1024, 512), (640, 128, 64), (2048, 512, 256), (448, 64, 8),
-         (96, 96, 88), (768, 256, 640)]
+         (96, 96, 88), (768, 256, 640),
+         # G or the roll not a multiple of 8 (runs that start or end inside an 8-row atom)
+         (300, 75, 37), (129, 43, 21), (512, 128, 37), (250, 50, 25), (693, 231, 115)]
 # (N, G, shift) with 0 < shift < G: the cases where Variants 2 and 3 exist
 SPLIT_CASES = [(256, 64, 32), (8192, 2048, 1024), (320, 64, 32), (384, 192, 96), (96, 32, 16),
                (640, 128, 64), (2048, 512, 256), (448, 64, 8), (96, 96, 88), (1024, 256, 128),
-               (512, 128, 40), (1024, 1024, 512), (256, 256, 200), (136, 136, 8)]
+               (512, 128, 40), (1024, 1024, 512), (256, 256, 200), (136, 136, 8),
+               (300, 75, 37), (693, 231, 115), (512, 128, 37), (129, 129, 5), (384, 192, 101)]
 # (N, G, shift) with G not dividing N: the last rolled group is shorter
 PARTIAL_CASES = [(320, 128, 64), (200, 64, 32), (136, 64, 32), (264, 256, 128), (72, 128, 64),
-                 (8832, 2048, 1024), (1000, 96, 48), (384, 256, 0)]
+                 (8832, 2048, 1024), (1000, 96, 48), (384, 256, 0),
+                 # the page's 1/6 group of 8192 tokens (Table 7) and other odd shapes
+                 (8192, 1365, 682), (1000, 333, 166), (8191, 1365, 682), (77, 100, 50)]
 VARIANT_CASES = ([(n, g, s, "default") for n, g, s in CASES + PARTIAL_CASES] +
                  [(n, g, s, v) for n, g, s in SPLIT_CASES for v in ("v2", "v3")])
 
@@ -236,7 +255,8 @@ def variant_args(N, shift, variant):
 @pytest.mark.parametrize("N,G,shift,variant", VARIANT_CASES)
 def test_rolled_runs_match_the_oracle(shim, N, G, shift, variant):
     """Runs of a rolled tile give exactly the oracle's token of every row; runs of an
-    original tile give the inverse; every run starts and ends on an 8-row boundary."""
+    original tile give the inverse; the 8-row atoms that straddle two runs (loaded with plain
+    loads, not TMA boxes) are exactly the ones marked."""
     tok = rolled_tokens(N, G, shift, variant)
     rolled_of = np.empty(N, dtype=np.int64)
     rolled_of[tok] = np.arange(N)
@@ -247,8 +267,15 @@ def test_rolled_runs_match_the_oracle(shim, N, G, shift, variant):
             assert valid == min(128, N - x0)
             got = [src + i for ln, src in runs for i in range(ln)]
             assert got == list(ref[x0:x0 + valid])
-            assert all(ln % 8 == 0 and src % 8 == 0 for ln, src in runs)
             assert 1 <= len(runs) <= 3
+        # atoms (8 rows) that hold rows of two runs are exactly those marked for plain loads
+        runs, valid = runs_of(shim.rolled_runs, x0, shift, N, G, front)
+        run_of_row = [k for k, (ln, _) in enumerate(runs) for _ in range(ln)]
+        want = 0
+        for a in range(16):
+            if len({run_of_row[r] for r in range(8 * a, min(8 * a + 8, valid))}) > 1:
+                want |= 1 << a
+        assert shim.straddled(x0, shift, N, G, front) == want
 
 
 @pytest.mark.parametrize("N,G,shift,variant", VARIANT_CASES)
@@ -414,6 +441,20 @@ def test_ds_entries_reject(lib):
                                 None) == 1
     assert lib.s2attn_bwd_dq_ds(A, None, 1, 4, 4, 256, 64, 64, f, 2, 32, ws, full, None) == 1
     assert lib.s2attn_bwd_dq_ds(A, A, 1, 4, 4, 256, 96, 64, f, 2, 32, ws, full, None) == 2
+    # the _general forms: flags and strides are validated before the workspace size
+    full2 = lib.s2attn_bwd_workspace_size_general(1, 4, 4, 256, 64, 64, 2, 32, 1, 0)
+    assert full2 > 0
+    assert lib.s2attn_bwd_dkdv_ds_general(A, A, A, A, A, A, 1, 4, 4, 256, 64, 64, f, 2, 32, 8,
+                                          None, ws, full2, None) == 1   # unknown flag bit
+    assert lib.s2attn_bwd_dkdv_ds_general(A, A, A, A, A, A, 1, 4, 4, 256, 64, 64, f, 4, 32, 1,
+                                          None, ws, full2, None) == 1   # Variant 2, no rolled head
+    assert lib.s2attn_bwd_dkdv_ds_general(A, A, A, A, A, A, 1, 4, 4, 256, 64, 64, f, 2, 32, 1,
+                                          None, ws, small, None) == 1   # no room for dS
+    assert lib.s2attn_bwd_dq_ds_general(A, A, 1, 4, 4, 256, 64, 64, f, 2, 32, 2, None, ws,
+                                        full2 - 16, None) == 1
+    bad = (ctypes.c_longlong * 16)(*([4 * 64 * 3, 4 * 64 - 8] * 8))  # token stride below H*d
+    assert lib.s2attn_bwd_dq_ds_general(A, A, 1, 4, 4, 256, 64, 64, f, 2, 32, 0, bad, ws, full2,
+                                        None) == 1
 
 
 @pytest.mark.parametrize("B,Hq,N,G,chunk", [(1, 32, 8192, 2048, 10), (2, 3, 8192, 2048, 4),
@@ -488,10 +529,8 @@ def test_general_entries_reject(lib):
     assert lib.s2attn_fwd_general(*zero_shift, 2, None, None) == 1
     big_shift = [A] * 5 + [2, 4, 4, 256, 64, 64, f, 2, 64]             # shift = G
     assert lib.s2attn_fwd_general(*big_shift, 2, None, None) == 1
-    # G not dividing N: only with the partial-last-group flag, never with a variant, N % 8 == 0
+    # G not dividing N: only with the partial-last-group flag, never with a variant
     ragged = [A] * 5 + [2, 4, 4, 320, 64, 128, f, 2, 64]
     assert lib.s2attn_fwd_general(*ragged, 0, None, None) == 1
     assert lib.s2attn_fwd_general(*ragged, 4 | 1, None, None) == 1
     assert lib.s2attn_fwd_general(*ragged, 4 | 2, None, None) == 1
-    odd_n = [A] * 5 + [2, 4, 4, 324, 64, 128, f, 2, 64]
-    assert lib.s2attn_fwd_general(*odd_n, 4, None, None) == 2

@@ -62,7 +62,7 @@ def test_variant_matches_oracle(flags, name, B, Hq, Hkv, N, G, d, shb, shift):
 
 
 @pytest.mark.parametrize("flags", [V2, V3], ids=["variant2", "variant3"])
-@pytest.mark.parametrize("mode", ["recompute", "per_kv_head"])
+@pytest.mark.parametrize("mode", ["recompute", "per_kv_head", "phases"])
 def test_variant_backward_paths(flags, mode):
     check_case(1, 8, 4, 1024, 256, 128, seed=77 + flags, flags=flags, mode=mode)
 
@@ -100,6 +100,43 @@ def test_partial_last_group_matches_oracle(name, B, Hq, Hkv, N, G, d, shb, shift
                shb=shb, shift=shift, flags=PARTIAL)
 
 
-@pytest.mark.parametrize("mode", ["recompute", "per_kv_head"])
+@pytest.mark.parametrize("mode", ["recompute", "per_kv_head", "phases"])
 def test_partial_last_group_backward_paths(mode):
     check_case(1, 4, 2, 704, 256, 128, seed=91, flags=PARTIAL, mode=mode)
+
+
+# Groups and rolls that are not multiples of 8 rows: the remap's runs then start or end inside
+# the 8-row atoms that TMA moves, and the kernels load those rows with plain loads.
+ODD_SHAPES = [
+    # the pages' group of 1/6 of the context (Table 7, "Group size ablation") at the metric
+    # length: G = 1365, rolled by 682; the last rolled group has the 2 leftover rows
+    ("table7_one_sixth", 1, 8, 4, 8192, 1365, 128, 682, PARTIAL),
+    # odd G and roll, G | N
+    ("odd_g", 1, 4, 4, 300, 75, 64, 37, 0),
+    # odd G, shorter last group, two query heads per kv head
+    ("odd_g_partial", 1, 4, 2, 1000, 333, 64, 166, PARTIAL),
+    # N, G and roll all odd, batch 2
+    ("all_odd", 2, 2, 2, 129, 43, 64, 21, 0),
+    # Variants 2 and 3 with odd G and roll
+    ("odd_g_variant2", 1, 4, 4, 693, 231, 64, 115, V2),
+    ("odd_g_variant3", 1, 4, 4, 693, 231, 64, 115, V3),
+    # a roll of 37 with Variant 3: the last group's three runs all end inside atoms
+    ("roll37_variant3", 1, 4, 2, 512, 128, 128, 37, V3),
+]
+
+
+@pytest.mark.parametrize("name,B,Hq,Hkv,N,G,d,shift,flags", ODD_SHAPES)
+def test_any_group_and_roll_matches_oracle(name, B, Hq, Hkv, N, G, d, shift, flags):
+    check_case(B, Hq, Hkv, N, G, d, seed=zlib.crc32(("odd" + name).encode()) % 10000,
+               shift=shift, flags=flags)
+
+
+@pytest.mark.parametrize("mode", ["recompute", "per_kv_head", "phases"])
+def test_any_group_and_roll_backward_paths(mode):
+    check_case(1, 4, 2, 1000, 333, 64, seed=123, shift=166, flags=PARTIAL, mode=mode)
+
+
+def test_odd_group_default_roll():
+    """The default entry points with an odd G roll the second half of the heads by
+    floor(G / 2), as the oracle does."""
+    check_case(1, 4, 4, 450, 75, 128, seed=9)
