@@ -109,6 +109,45 @@ __device__ __forceinline__ void dkdv_tile(const BwdParams& p, int u, int& b, int
   kvh += p.kvh_begin;
 }
 
+// The Q and dO tiles and the LSE2 / D values of one query tile when TMA boxes and bulk copies
+// cannot move all of it (a remap run starting or ending inside an 8-row atom, or LSE2 / D runs
+// that are not 16-byte aligned, which happens when G or the roll is not a multiple of 8): the
+// odd parts are copied by this thread first, then `fb` is armed with the bytes the copy engines
+// still deliver. Kept out of line so the common path stays as small as it is.
+template <int D>
+__device__ __noinline__ void dkdv_load_query_tile_slow(
+    uint32_t q_dst, uint32_t do_dst, uint32_t sl, uint32_t sd, const CUtensorMap* tmQ,
+    const CUtensorMap* tmQ8, const CUtensorMap* tmO, const CUtensorMap* tmO8, uint32_t fb,
+    const TensorRef q, const TensorRef dO, const float* lse_row, const float* d_row, int N, int b,
+    int hq, const Runs tr, uint32_t skip, bool aligned) {
+  if (skip) {
+    fill_atoms<D>(q_dst, skip, tr, q, b, hq);
+    fill_atoms<D>(do_dst, skip, tr, dO, b, hq);
+  }
+  if (!aligned) {
+    int base = 0;
+    for (int r = 0; r < tr.n; ++r) {
+      for (int j = 0; j < tr.len[r]; ++j) {
+        cp_async4(sl + 4u * (base + j), lse_row + tr.src[r] + j);
+        cp_async4(sd + 4u * (base + j), d_row + tr.src[r] + j);
+      }
+      base += tr.len[r];
+    }
+    cp_async_wait_all();
+  }
+  mbar_expect_tx(fb, 2 * tma_tile_bytes<D>(skip) + (aligned ? 8u * tr.valid : 0u));
+  load_tile<D>(q_dst, tmQ, tmQ8, fb, b, hq, tr, N, skip);
+  load_tile<D>(do_dst, tmO, tmO8, fb, b, hq, tr, N, skip);
+  if (aligned) {
+    int base = 0;
+    for (int r = 0; r < tr.n; ++r) {
+      bulk_load(sl + 4u * base, lse_row + tr.src[r], 4u * tr.len[r], fb);
+      bulk_load(sd + 4u * base, d_row + tr.src[r], 4u * tr.len[r], fb);
+      base += tr.len[r];
+    }
+  }
+}
+
 // kFront: built for the Variant 3 reordering (otherwise p.front is ignored).
 template <int D, bool kFront>
 __global__ void __launch_bounds__(32 * (kDkdvEwWarps + 3), 1)
@@ -149,10 +188,10 @@ __global__ void __launch_bounds__(32 * (kDkdvEwWarps + 3), 1)
 
   constexpr int kProducer = kDkdvEwWarps, kMma = kDkdvEwWarps + 1, kStore = kDkdvEwWarps + 2;
   if (warp == kProducer && lane == 0) {
-    mbar_init(bar(L::B_KV), 2);        // the K tile and the V tile
+    mbar_init(bar(L::B_KV), 1);
     mbar_init(bar(L::B_KVE), 1);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(bar(L::B_QF + s), 3);  // the Q tile, the dO tile, the rows' LSE2 and D
+      mbar_init(bar(L::B_QF + s), 1);
       mbar_init(bar(L::B_QE + s), 1);
     }
     mbar_init(bar(L::B_S), 1);
@@ -193,38 +232,28 @@ __global__ void __launch_bounds__(32 * (kDkdvEwWarps + 3), 1)
 
   if (warp == kProducer) {
     // ---------------- TMA producer ----------------
-    // The whole warp runs the loop: lane 0 claims the work tiles, waits on the ring barriers
-    // and issues the TMA copies; every lane helps with the rows TMA cannot move
-    // (produce_tile, and LSE2 / D of rows whose runs are not 16-byte aligned).
-    {
+    if (lane == 0) {
       int last_parity[2] = {-1, -1};
       int n = 0, tc = 0, kv_loads = 0;
       bool ok = true;
-      auto claim = [&](int k, int& u) -> bool {
-        int good = 1, got = -1;
-        if (lane == 0)
-          good = publish_unit(k, got, p.sched, n_tiles, ring, bar(L::B_UF), bar(L::B_UE), ctx, 15);
-        good = __shfl_sync(0xffffffffu, good, 0);
-        u = __shfl_sync(0xffffffffu, got, 0);
-        return good != 0;
-      };
       // Units are claimed one ahead: unit k + 1 is published as soon as unit k's K and V
       // loads are issued, so the other roles never wait for the producer to finish issuing
       // unit k's query tiles before they can start on the next unit.
       int u_next;
-      ok = claim(0, u_next);
+      ok = publish_unit(0, u_next, p.sched, n_tiles, ring, bar(L::B_UF), bar(L::B_UE), ctx, 15);
       for (int k = 0; ok; ++k, ++tc) {
         const int u = u_next;
         if (u < 0) break;
         int b, kvh, t0;
         dkdv_tile(p, u, b, kvh, t0);
         // K and V of the previous tile are free once its last S and dP MMAs are done.
-        if (tc > 0 && !lead_wait(bar(L::B_KVE), (tc - 1) & 1, ctx, 11)) { ok = false; break; }
+        if (tc > 0 && !wait_bar(bar(L::B_KVE), (tc - 1) & 1, ctx, 11)) { ok = false; break; }
+        mbar_expect_tx(bar(L::B_KV), 2 * L::kTile);
         const Runs kv_runs = identity_runs(t0, p.N);
-        produce_tile<D>(sbase + L::kK, &tmK, &tmK8, bar(L::B_KV), p.k, b, kvh, kv_runs, p.N);
-        produce_tile<D>(sbase + L::kV, &tmV, &tmV8, bar(L::B_KV), p.v, b, kvh, kv_runs, p.N);
+        load_tile<D>(sbase + L::kK, &tmK, &tmK8, bar(L::B_KV), b, kvh, kv_runs, p.N);
+        load_tile<D>(sbase + L::kV, &tmV, &tmV8, bar(L::B_KV), b, kvh, kv_runs, p.N);
         ++kv_loads;
-        if (!claim(k + 1, u_next)) {
+        if (!publish_unit(k + 1, u_next, p.sched, n_tiles, ring, bar(L::B_UF), bar(L::B_UE), ctx, 15)) {
           ok = false;
           break;
         }
@@ -232,67 +261,52 @@ __global__ void __launch_bounds__(32 * (kDkdvEwWarps + 3), 1)
           const HeadRemap hm = head_map(hq);
           const QTileRanges qr = kv_tile_qtiles(hm, t0, head_wrap(hq));
           const size_t row0 = (static_cast<size_t>(b) * p.Hq + hq) * p.N;
+          const float* lse_row = p.lse2 + row0;
+          const float* d_row = p.dvec + row0;
           for (int i = 0; i < qr.count(); ++i, ++n) {
             const int st = n & 1;
-            if (n >= 2 && !lead_wait(bar(L::B_QE + st), ((n >> 1) - 1) & 1, ctx, 1)) { ok = false; break; }
+            if (n >= 2 && !wait_bar(bar(L::B_QE + st), ((n >> 1) - 1) & 1, ctx, 1)) { ok = false; break; }
             const Runs tr = rolled_runs(hm, qr.at(i) * kTileRows);
             const uint32_t fb = bar(L::B_QF + st);
-            produce_tile<D>(sbase + L::kQ + st * L::kTile, &tmQ, &tmQ8, fb, p.q, b, hq, tr, p.N);
-            produce_tile<D>(sbase + L::kDO + st * L::kTile, &tmO, &tmO8, fb, p.dO, b, hq, tr, p.N);
-            // LSE2 and D of the tile's rows: one bulk copy per run when every run is 16-byte
-            // aligned (offsets and lengths multiples of 4 floats), else plain loads.
             const uint32_t sl = sbase + L::kLse + st * 512, sd = sbase + L::kDv + st * 512;
+            // TMA boxes need runs of whole 8-row atoms, bulk copies 16-byte aligned runs.
+            const uint32_t skip = straddled_atoms(tr);
             bool aligned = true;
             {
               int base = 0;
 #pragma unroll
+              for (int r = 0; r < 3; ++r)
+                if (r < tr.n) {
+                  aligned = aligned && ((base | tr.len[r]) & 3) == 0 && ((row0 + tr.src[r]) & 3) == 0;
+                  base += tr.len[r];
+                }
+            }
+            if (skip != 0 || !aligned) {
+              dkdv_load_query_tile_slow<D>(sbase + L::kQ + st * L::kTile,
+                                           sbase + L::kDO + st * L::kTile, sl, sd, &tmQ, &tmQ8,
+                                           &tmO, &tmO8, fb, p.q, p.dO, lse_row, d_row, p.N, b,
+                                           hq, tr, skip, aligned);
+            } else {
+              mbar_expect_tx(fb, 2 * L::kTile + 8u * tr.valid);
+              load_tile<D>(sbase + L::kQ + st * L::kTile, &tmQ, &tmQ8, fb, b, hq, tr, p.N);
+              load_tile<D>(sbase + L::kDO + st * L::kTile, &tmO, &tmO8, fb, b, hq, tr, p.N);
+              int base = 0;
+#pragma unroll
               for (int r = 0; r < 3; ++r) {
                 if (r < tr.n) {
-                  aligned = aligned && (base & 3) == 0 && (tr.len[r] & 3) == 0 &&
-                            ((row0 + tr.src[r]) & 3) == 0;
+                  bulk_load(sl + 4u * base, lse_row + tr.src[r], 4u * tr.len[r], fb);
+                  bulk_load(sd + 4u * base, d_row + tr.src[r], 4u * tr.len[r], fb);
                   base += tr.len[r];
                 }
               }
-            }
-            if (aligned) {
-              if (lane == 0) {
-                mbar_expect_tx(fb, 8u * tr.valid);
-                int base = 0;
-#pragma unroll
-                for (int r = 0; r < 3; ++r) {
-                  if (r < tr.n) {
-                    bulk_load(sl + 4u * base, p.lse2 + row0 + tr.src[r], 4u * tr.len[r], fb);
-                    bulk_load(sd + 4u * base, p.dvec + row0 + tr.src[r], 4u * tr.len[r], fb);
-                    base += tr.len[r];
-                  }
-                }
-              }
-            } else {
-              float* s_l = reinterpret_cast<float*>(smem + L::kLse + st * 512);
-              float* s_d = reinterpret_cast<float*>(smem + L::kDv + st * 512);
-              for (int row = lane; row < tr.valid; row += 32) {
-                int src = 0, base = 0;
-#pragma unroll
-                for (int r = 0; r < 3; ++r) {
-                  if (r < tr.n && row >= base && row < base + tr.len[r]) src = tr.src[r] + (row - base);
-                  base += r < tr.n ? tr.len[r] : 0;
-                }
-                s_l[row] = p.lse2[row0 + src];
-                s_d[row] = p.dvec[row0 + src];
-              }
-              __threadfence_block();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(fb);
             }
             last_parity[st] = (n >> 1) & 1;
           }
         }
       }
-      if (lane == 0) {
-        if (kv_loads > 0) drain_wait(bar(L::B_KV), (kv_loads - 1) & 1, p.timeout_ns);
-        for (int s = 0; s < 2; ++s)
-          if (last_parity[s] >= 0) drain_wait(bar(L::B_QF + s), last_parity[s], p.timeout_ns);
-      }
+      if (kv_loads > 0) drain_wait(bar(L::B_KV), (kv_loads - 1) & 1, p.timeout_ns);
+      for (int s = 0; s < 2; ++s)
+        if (last_parity[s] >= 0) drain_wait(bar(L::B_QF + s), last_parity[s], p.timeout_ns);
     }
   } else if (warp == kMma) {
     // ---------------- MMA issuer ----------------

@@ -108,9 +108,8 @@ __global__ void __launch_bounds__(320, 1)
 
   if (warp == 8) {
     // ---------------- TMA producer ----------------
-    // The whole warp runs the loop (see produce_tile): lane 0 waits on the ring barriers and
-    // issues the TMA copies, all lanes fill the tile rows TMA cannot move.
-    {
+    // Tile rows TMA cannot move are copied by this thread first (produce_tile).
+    if (lane == 0) {
       const Runs q_runs = rolled_runs(hm, R0);
       produce_tile<D>(sbase + L::kQ, &tmQ, &tmQ8, bar(L::B_QDO), p.q, b, h, q_runs, p.N);
       produce_tile<D>(sbase + L::kDO, &tmO, &tmO8, bar(L::B_QDO), p.dO, b, h, q_runs, p.N);
@@ -118,7 +117,7 @@ __global__ void __launch_bounds__(320, 1)
       auto issue_k = [&]() -> bool {
         const int i = k_issued, st = i % L::kKStages;
         if (i >= L::kKStages &&
-            !lead_wait(bar(L::B_KE + st), ((i / L::kKStages) - 1) & 1, ctx, 1))
+            !wait_bar(bar(L::B_KE + st), ((i / L::kKStages) - 1) & 1, ctx, 1))
           return false;
         produce_tile<D>(sbase + L::kK + st * L::kTile, &tmK, &tmK8, bar(L::B_K + st), p.k, b, kvh,
                         rolled_runs(hm, (kt_begin + i) * kTileRows), p.N);
@@ -128,7 +127,7 @@ __global__ void __launch_bounds__(320, 1)
       auto issue_v = [&]() -> bool {
         const int i = v_issued, st = i % L::kVStages;
         if (i >= L::kVStages &&
-            !lead_wait(bar(L::B_VE + st), ((i / L::kVStages) - 1) & 1, ctx, 10))
+            !wait_bar(bar(L::B_VE + st), ((i / L::kVStages) - 1) & 1, ctx, 10))
           return false;
         produce_tile<D>(sbase + L::kV + st * L::kTile, &tmV, &tmV8, bar(L::B_V + st), p.v, b, kvh,
                         rolled_runs(hm, (kt_begin + i) * kTileRows), p.N);
@@ -140,13 +139,11 @@ __global__ void __launch_bounds__(320, 1)
         if (j + 1 < n_kv) ok = issue_k();
         if (ok) ok = issue_v();
       }
-      if (lane == 0) {
-        drain_wait(bar(L::B_QDO), 0, p.timeout_ns);
-        for (int i = k_issued - L::kKStages; i < k_issued; ++i)
-          if (i >= 0) drain_wait(bar(L::B_K + i % L::kKStages), (i / L::kKStages) & 1, p.timeout_ns);
-        for (int i = v_issued - L::kVStages; i < v_issued; ++i)
-          if (i >= 0) drain_wait(bar(L::B_V + i % L::kVStages), (i / L::kVStages) & 1, p.timeout_ns);
-      }
+      drain_wait(bar(L::B_QDO), 0, p.timeout_ns);
+      for (int i = k_issued - L::kKStages; i < k_issued; ++i)
+        if (i >= 0) drain_wait(bar(L::B_K + i % L::kKStages), (i / L::kKStages) & 1, p.timeout_ns);
+      for (int i = v_issued - L::kVStages; i < v_issued; ++i)
+        if (i >= 0) drain_wait(bar(L::B_V + i % L::kVStages), (i / L::kVStages) & 1, p.timeout_ns);
     }
   } else if (warp == 9) {
     // ---------------- MMA issuer ----------------

@@ -29,38 +29,49 @@ __device__ __forceinline__ uint32_t tma_tile_bytes(uint32_t skip) {
   return Tile<D>::kBytes - static_cast<uint32_t>(__popc(skip)) * (8u * 128u) * Tile<D>::kHalves;
 }
 
-// Whole warp: the rows of the atoms in `skip` (see straddled_atoms), read with 16-byte loads
-// from the tensor and written in the 128-byte-swizzled tile layout the TMA boxes produce
-// (16-byte chunk c of a row's 64-column half at chunk c XOR (row mod 8)); rows past the end of
-// the sequence become zeros. Ends with a proxy fence (the tensor core reads the tile) and a
-// warp barrier, after which one lane may signal the tile's barrier.
+// 16-byte (or 4-byte) asynchronous copy global -> shared by one thread; with src_bytes = 0 the
+// destination is filled with zeros. Completed by cp_async_wait_all.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst),
+               "l"(reinterpret_cast<uint64_t>(src))
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+// One thread: the rows of the atoms in `skip` (see straddled_atoms), copied with 16-byte
+// asynchronous copies from the tensor into the 128-byte-swizzled tile layout the TMA boxes
+// produce (16-byte chunk c of a row's 64-column half at chunk c XOR (row mod 8)); rows past the
+// end of the sequence become zeros. Returns when the copies have landed and are visible to the
+// tensor core (proxy fence), so the caller may signal the tile's barrier.
 template <int D>
-__device__ __noinline__ void fill_atoms(uint32_t dst, uint32_t skip, const Runs tr,
-                                        const TensorRef t, int b, int h) {
+__device__ __forceinline__ void fill_atoms(uint32_t dst, uint32_t skip, const Runs& tr,
+                                           const TensorRef& t, int b, int h) {
   constexpr int kChunks = D / 8;   // 16-byte chunks per row
-  const int lane = threadIdx.x & 31;
   for (uint32_t m = skip; m != 0; m &= m - 1) {
     const int a = __ffs(m) - 1;
-    for (int i = lane; i < 8 * kChunks; i += 32) {
-      const int row = 8 * a + i / kChunks, c = i % kChunks;
+    for (int row = 8 * a; row < 8 * a + 8; ++row) {
       int src = -1, base = 0;
 #pragma unroll
       for (int k = 0; k < 3; ++k) {
         if (k < tr.n && row >= base && row < base + tr.len[k]) src = tr.src[k] + (row - base);
         base += k < tr.n ? tr.len[k] : 0;
       }
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (src >= 0)
-        v = __ldg(reinterpret_cast<const uint4*>(t.p + b * t.sb + src * t.st +
-                                                 static_cast<long long>(h) * D + 8 * c));
-      const uint32_t off = (c / 8) * Tile<D>::kHalfBytes + row * 128 + (((c % 8) ^ (row & 7)) * 16);
-      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + off), "r"(v.x), "r"(v.y),
-                   "r"(v.z), "r"(v.w)
-                   : "memory");
+      const __nv_bfloat16* g = t.p + b * t.sb + (src < 0 ? 0 : src) * t.st + static_cast<long long>(h) * D;
+#pragma unroll
+      for (int c = 0; c < kChunks; ++c)
+        cp_async16(dst + (c / 8) * Tile<D>::kHalfBytes + row * 128 + (((c % 8) ^ (row & 7)) * 16),
+                   g + 8 * c, src < 0 ? 0u : 16u);
     }
   }
+  cp_async_wait_all();
   fence_async_smem();
-  __syncwarp();
 }
 
 // Issue the TMA loads of one 128-row tile of a [B, N, H, D] tensor whose rows are given by
@@ -91,20 +102,31 @@ __device__ __forceinline__ void load_tile(uint32_t dst, const CUtensorMap* m128,
   }
 }
 
-// Producer warp: one tile through the remap. Atoms TMA cannot move are filled by the whole
-// warp first; then lane 0 arms `bar` with the bytes TMA will deliver (plus `extra_tx`, for
-// copies the caller issues on the same barrier) and issues the boxes. Warp-uniform arguments.
+// A tile with atoms TMA cannot move: those are copied by this thread first, then `bar` is
+// armed with the bytes TMA still delivers (one arrival) and the other boxes are issued. Kept out
+// of line so the common path stays as small as it is.
+template <int D>
+__device__ __noinline__ void load_tile_slow(uint32_t dst, const CUtensorMap* m128,
+                                            const CUtensorMap* m8, uint32_t bar, const TensorRef t,
+                                            int b, int h, const Runs tr, int N, uint32_t skip) {
+  fill_atoms<D>(dst, skip, tr, t, b, h);
+  mbar_expect_tx(bar, tma_tile_bytes<D>(skip));
+  load_tile<D>(dst, m128, m8, bar, b, h, tr, N, skip);
+}
+
+// Producer thread: one tile through the remap, one arrival on `bar` with its bytes.
 template <int D>
 __device__ __forceinline__ void produce_tile(uint32_t dst, const CUtensorMap* m128,
                                              const CUtensorMap* m8, uint32_t bar,
                                              const TensorRef& t, int b, int h, const Runs& tr,
                                              int N) {
   const uint32_t skip = straddled_atoms(tr);
-  if (skip) fill_atoms<D>(dst, skip, tr, t, b, h);
-  if ((threadIdx.x & 31) == 0) {
-    mbar_expect_tx(bar, tma_tile_bytes<D>(skip));
-    load_tile<D>(dst, m128, m8, bar, b, h, tr, N, skip);
+  if (skip) {
+    load_tile_slow<D>(dst, m128, m8, bar, t, b, h, tr, N, skip);
+    return;
   }
+  mbar_expect_tx(bar, Tile<D>::kBytes);
+  load_tile<D>(dst, m128, m8, bar, b, h, tr, N);
 }
 
 // Whole-tile GEMMs issued by the MMA thread. Operand descriptors are built once per call and
@@ -131,19 +153,6 @@ __device__ __forceinline__ void gemm_ts_mn(uint32_t d_tmem, uint32_t a_tmem, uin
   for (int kk = 0; kk < kTileRows / 16; ++kk)
     mma_ts(d_tmem, a_tmem + kk * 8, b0 + static_cast<uint64_t>((kk * 2048) >> 4), idesc,
            (accumulate || kk > 0) ? 1u : 0u);
-}
-
-// Steps [kk0, kk1) of gemm_ts_mn (16 keys each): the PV product in parts, so a part can start
-// before the whole bf16 A operand is in TMEM.
-template <int D>
-__device__ __forceinline__ void gemm_ts_mn_part(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_base,
-                                                uint32_t idesc, bool accumulate, int kk0, int kk1) {
-  const uint64_t b0 = sdesc_sw128(b_base, Tile<D>::kHalfBytes, 1024);
-#pragma unroll
-  for (int kk = 0; kk < kTileRows / 16; ++kk)
-    if (kk >= kk0 && kk < kk1)
-      mma_ts(d_tmem, a_tmem + kk * 8, b0 + static_cast<uint64_t>((kk * 2048) >> 4), idesc,
-             (accumulate || kk > 0) ? 1u : 0u);
 }
 
 // Dynamic work distribution for the persistent kernels. One thread of the CTA claims units
@@ -210,18 +219,6 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity,
   while (!mbar_try_wait(bar, parity)) {
     if (global_timer_ns() - t0 > timeout_ns) return;
   }
-}
-
-// Producer-warp wait: lane 0 alone polls the barrier (the other lanes park at the warp
-// barrier instead of issuing probes) and the verdict is shared. The lanes' later writes to the
-// freed slot (fill_atoms) execute after lane 0 saw the phase complete, i.e. after the tensor
-// core's reads of it.
-__device__ __forceinline__ bool lead_wait(uint32_t bar, uint32_t parity, const WaitCtx& ctx,
-                                          uint32_t site) {
-  int ok = 1;
-  if ((threadIdx.x & 31) == 0) ok = wait_bar(bar, parity, ctx, site) ? 1 : 0;
-  __syncwarp();
-  return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
 // Warp-uniform wait: every lane waits (each needs the acquire), and the warp proceeds only

@@ -13,8 +13,7 @@ namespace s2 {
 // Error reporting shared by every kernel (read back by s2attn_get_device_error).
 // code = (kernel id << 8) | wait site; the first failing wait wins.
 // ----------------------------------------------------------------------------------------
-enum KernelId : uint32_t { KID_FWD = 1, KID_DKDV = 2, KID_DQ = 3, KID_SELFTEST = 4, KID_DQDS = 5,
-                           KID_PRE = 6 };
+enum KernelId : uint32_t { KID_FWD = 1, KID_DKDV = 2, KID_DQ = 3, KID_SELFTEST = 4, KID_DQDS = 5 };
 
 struct WaitCtx {
   volatile int* abort_flag;   // CTA-shared; set by the first waiter that gives up

@@ -87,8 +87,7 @@ struct FwdLayout {
   static constexpr uint32_t kStage = kV + kVStages * kTile; // ... for each softmax warp
   static constexpr uint32_t kBar = kStage + 8 * kStageWarp;
   enum { B_Q = 0, B_QE = 2, B_K = 4, B_KE = B_K + kKStages, B_V = B_KE + kKStages,
-         B_VE = B_V + kVStages, B_S = B_VE + kVStages, B_P = B_S + 2, B_PH = B_P + 2,
-         B_ODONE = B_PH + 2,
+         B_VE = B_V + kVStages, B_S = B_VE + kVStages, B_P = B_S + 2, B_ODONE = B_P + 2,
          B_DRAIN = B_ODONE + 2, B_COUNT = B_DRAIN + 1 };
   static constexpr uint32_t kTmemSlot = kBar + B_COUNT * 8;
   static constexpr uint32_t kAbort = kTmemSlot + 4;
@@ -177,7 +176,6 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(bar(L::B_VE + s), 1);
       mbar_init(bar(L::B_S + s), 1);
       mbar_init(bar(L::B_P + s), 128);
-      mbar_init(bar(L::B_PH + s), 128);
       mbar_init(bar(L::B_ODONE + s), 1);
     }
     for (int s = 0; s < L::kKStages; ++s) {
@@ -202,18 +200,17 @@ __global__ void __launch_bounds__(320, 1)
 
   if (warp == 8) {
     // ---------------- TMA producer ----------------
-    // The whole warp runs the loop: lane 0 waits on the ring barriers and issues the TMA
-    // copies, and all lanes fill the few tile rows TMA cannot move (produce_tile).
     // K(i) (i counts every key tile this CTA loads) goes to slot i % 2 once K(i - 2) has been
     // released, V(i) likewise; within a unit K runs one tile ahead of V. Q tile t of a unit is
-    // loaded once the previous unit's last S MMA on it is done.
-    {
+    // loaded once the previous unit's last S MMA on it is done. Tile rows TMA cannot move are
+    // copied by this thread first (produce_tile).
+    if (lane == 0) {
       int k_issued = 0, v_issued = 0, q_loads[2] = {0, 0};
       bool ok = true;
       auto issue_k = [&](const FwdUnit& u, int j) -> bool {
         const int i = k_issued, st = i % L::kKStages;
         if (i >= L::kKStages &&
-            !lead_wait(bar(L::B_KE + st), ((i / L::kKStages) - 1) & 1, ctx, 1))
+            !wait_bar(bar(L::B_KE + st), ((i / L::kKStages) - 1) & 1, ctx, 1))
           return false;
         produce_tile<D>(sbase + L::kK + st * L::kTile, &tmK, &tmK8, bar(L::B_K + st), p.k, u.b,
                         u.kvh, rolled_runs(head_remap(p.N, p.G, u.shift_h, kFront ? u.front_h : 0),
@@ -224,7 +221,7 @@ __global__ void __launch_bounds__(320, 1)
       auto issue_v = [&](const FwdUnit& u, int j) -> bool {
         const int i = v_issued, st = i % L::kVStages;
         if (i >= L::kVStages &&
-            !lead_wait(bar(L::B_VE + st), ((i / L::kVStages) - 1) & 1, ctx, 9))
+            !wait_bar(bar(L::B_VE + st), ((i / L::kVStages) - 1) & 1, ctx, 9))
           return false;
         produce_tile<D>(sbase + L::kV + st * L::kTile, &tmV, &tmV8, bar(L::B_V + st), p.v, u.b,
                         u.kvh, rolled_runs(head_remap(p.N, p.G, u.shift_h, kFront ? u.front_h : 0),
@@ -239,7 +236,7 @@ __global__ void __launch_bounds__(320, 1)
         ok = issue_k(u, 0);   // the first key tile can stream while the last unit finishes
         for (int t = 0; ok && t < 2; ++t) {
           if (!u.tv[t]) continue;
-          if (q_loads[t] > 0 && !lead_wait(bar(L::B_QE + t), (q_loads[t] - 1) & 1, ctx, 10)) {
+          if (q_loads[t] > 0 && !wait_bar(bar(L::B_QE + t), (q_loads[t] - 1) & 1, ctx, 10)) {
             ok = false;
             break;
           }
@@ -254,14 +251,12 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
       // Every issued copy lands before the CTA can exit.
-      if (lane == 0) {
-        for (int t = 0; t < 2; ++t)
-          if (q_loads[t] > 0) drain_wait(bar(L::B_Q + t), (q_loads[t] - 1) & 1, p.timeout_ns);
-        for (int i = k_issued - L::kKStages; i < k_issued; ++i)
-          if (i >= 0) drain_wait(bar(L::B_K + i % L::kKStages), (i / L::kKStages) & 1, p.timeout_ns);
-        for (int i = v_issued - L::kVStages; i < v_issued; ++i)
-          if (i >= 0) drain_wait(bar(L::B_V + i % L::kVStages), (i / L::kVStages) & 1, p.timeout_ns);
-      }
+      for (int t = 0; t < 2; ++t)
+        if (q_loads[t] > 0) drain_wait(bar(L::B_Q + t), (q_loads[t] - 1) & 1, p.timeout_ns);
+      for (int i = k_issued - L::kKStages; i < k_issued; ++i)
+        if (i >= 0) drain_wait(bar(L::B_K + i % L::kKStages), (i / L::kKStages) & 1, p.timeout_ns);
+      for (int i = v_issued - L::kVStages; i < v_issued; ++i)
+        if (i >= 0) drain_wait(bar(L::B_V + i % L::kVStages), (i / L::kVStages) & 1, p.timeout_ns);
     }
   } else if (warp == 9) {
     // ---------------- MMA issuer ----------------
@@ -306,20 +301,14 @@ __global__ void __launch_bounds__(320, 1)
           bool v_ready = false, k_next_ready = false;
           for (int t = 0; ok && t < 2; ++t) {
             if (u.part(t, kt)) {
-              // O_t += P_t V in two halves of 64 keys: the first starts as soon as the
-              // softmax warpgroup has stored that half of P_t.
-              if (!wait_bar(bar(L::B_PH + t), pcount[t] & 1, ctx, 11)) { ok = false; break; }
+              if (!wait_bar(bar(L::B_P + t), pcount[t] & 1, ctx, 4)) { ok = false; break; }
               if (!v_ready) {
                 if (!wait_bar(bar(L::B_V + vst), (vi / L::kVStages) & 1, ctx, 5)) { ok = false; break; }
                 v_ready = true;
               }
               tc_fence_after();
-              gemm_ts_mn_part<D>(tmem + 256 + t * D, tmem + t * 128, sbase + L::kV + vst * L::kTile,
-                                 idesc_pv, !first_pv[t], 0, 4);
-              if (!wait_bar(bar(L::B_P + t), pcount[t] & 1, ctx, 4)) { ok = false; break; }
-              tc_fence_after();
-              gemm_ts_mn_part<D>(tmem + 256 + t * D, tmem + t * 128, sbase + L::kV + vst * L::kTile,
-                                 idesc_pv, true, 4, 8);
+              gemm_ts_mn<D>(tmem + 256 + t * D, tmem + t * 128, sbase + L::kV + vst * L::kTile,
+                            idesc_pv, !first_pv[t]);
               first_pv[t] = false;
               ++pcount[t];
               if (kt == u.ke[t]) mma_commit(bar(L::B_ODONE + t));
@@ -409,11 +398,6 @@ __global__ void __launch_bounds__(320, 1)
             pk[i] = pack_bf16(e0, e1);
           }
           tmem_st16(s_col + 16 * j, pk);
-          if (j == 1) {   // keys 0-63 of P are in TMEM: the first half of the PV MMA may start
-            tmem_st_wait();
-            tc_fence_before();
-            mbar_arrive(bar(L::B_PH + wg));
-          }
         }
         acc[0] = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
         l_run += f2_lo(acc[0]) + f2_hi(acc[0]);

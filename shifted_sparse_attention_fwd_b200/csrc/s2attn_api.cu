@@ -69,17 +69,10 @@ cudaError_t set_smem_attrs_variant() {
 // Every kernel exists twice: with the plain-roll index code only, and with the Variant 3
 // reordering compiled in (S2ATTN_FLAG_WRAP_FRONT_FIRST), so the common case pays nothing
 // for the general remap.
-// Largest dynamic shared memory the streaming preprocess may request.
-constexpr uint32_t kPreSmemMax = 220 * 1024;
-
 template <int D>
 cudaError_t set_smem_attrs() {
-  cudaError_t e = set_smem_attrs_variant<D, false>();
-  if (e != cudaSuccess) return e;
-  e = set_smem_attrs_variant<D, true>();
-  if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(s2::s2_bwd_pre_stream_kernel<D>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize, kPreSmemMax);
+  const cudaError_t e = set_smem_attrs_variant<D, false>();
+  return e != cudaSuccess ? e : set_smem_attrs_variant<D, true>();
 }
 
 // Per-device one-time set-up (with that device current): the device address of the error
@@ -378,44 +371,17 @@ void set_ds_pass(s2::BwdParams& p, const Shape& sh, const void* workspace, int k
                                           ws_min_bytes(sh.B, sh.Hq, sh.N));
 }
 
-// Tokens per stage of the streaming preprocess: about 32 KB of each tensor per stage, at least
-// one token; 0 when one token's heads do not fit the ring (the plain-load kernel runs then).
-int pre_tokens_per_stage(int Hq, int d) {
-  const long long row = static_cast<long long>(Hq) * d * 2;
-  const long long tps = row >= s2::kPreStageMax ? 1 : s2::kPreStageMax / row;
-  return s2::pre_smem_bytes(static_cast<int>(tps), Hq, d) <= kPreSmemMax ? static_cast<int>(tps) : 0;
-}
-
 template <int D>
 s2attn_status launch_pre(const Shape& sh, const void* o, const float* lse, const void* dO,
-                         void* workspace, cudaStream_t stream, unsigned int* err, int num_sms) {
+                         void* workspace, cudaStream_t stream) {
   const size_t half = ws_half(sh.B, sh.Hq, sh.N);
   float* dvec = static_cast<float*>(workspace);
   float* lse2 = reinterpret_cast<float*>(static_cast<char*>(workspace) + half);
-  const int tps = pre_tokens_per_stage(sh.Hq, D);
-  if (tps > 0) {
-    s2::PreParams p{};
-    p.o = static_cast<const __nv_bfloat16*>(o);
-    p.dO = static_cast<const __nv_bfloat16*>(dO);
-    p.o_sb = sh.sb[T_O]; p.o_st = sh.st[T_O];
-    p.do_sb = sh.sb[T_DO]; p.do_st = sh.st[T_DO];
-    p.lse = lse; p.dvec = dvec; p.lse2 = lse2;
-    p.sched = ws_sched(workspace, sh);
-    p.sched_words = kSchedWords;
-    p.B = sh.B; p.Hq = sh.Hq; p.N = sh.N; p.tps = tps;
-    p.err = err;
-    p.timeout_ns = g_timeout_ns.load();
-    const long long stages = (static_cast<long long>(sh.B) * sh.N + tps - 1) / tps;
-    const unsigned grid = static_cast<unsigned>(stages < num_sms ? stages : num_sms);
-    s2::s2_bwd_pre_stream_kernel<D><<<grid, s2::kPreThreads, s2::pre_smem_bytes(tps, sh.Hq, D),
-                                      stream>>>(p);
-  } else {
-    const unsigned grid = static_cast<unsigned>(sh.B) * ((sh.N + s2::kPreTokens - 1) / s2::kPreTokens);
-    s2::s2_bwd_pre_kernel<D><<<grid, 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, dvec,
-        lse2, ws_sched(workspace, sh), kSchedWords, sh.Hq, sh.N, sh.sb[T_O], sh.st[T_O],
-        sh.sb[T_DO], sh.st[T_DO]);
-  }
+  const unsigned grid = static_cast<unsigned>(sh.B) * ((sh.N + s2::kPreTokens - 1) / s2::kPreTokens);
+  s2::s2_bwd_pre_kernel<D><<<grid, 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), lse, dvec,
+      lse2, ws_sched(workspace, sh), kSchedWords, sh.Hq, sh.N, sh.sb[T_O], sh.st[T_O],
+      sh.sb[T_DO], sh.st[T_DO]);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? S2ATTN_OK : cuda_fail(e, "s2_bwd_pre_kernel launch");
 }
@@ -528,9 +494,9 @@ s2attn_status dq_ds_impl(const Shape& sh, const void* k, void* dq, float scale, 
                     : launch_dq_ds<128>(sh, k, dq, scale, ws, kvh_begin, kvh_count, stream, err, num_sms);
 }
 s2attn_status pre_impl(const Shape& sh, const void* o, const float* lse, const void* dO, void* ws,
-                       cudaStream_t stream, unsigned int* err, int num_sms) {
-  return sh.d == 64 ? launch_pre<64>(sh, o, lse, dO, ws, stream, err, num_sms)
-                    : launch_pre<128>(sh, o, lse, dO, ws, stream, err, num_sms);
+                       cudaStream_t stream) {
+  return sh.d == 64 ? launch_pre<64>(sh, o, lse, dO, ws, stream)
+                    : launch_pre<128>(sh, o, lse, dO, ws, stream);
 }
 
 // Caller-given strides for tensors ids[0..n): strides[2i] = batch, strides[2i+1] = token (in
@@ -668,10 +634,7 @@ s2attn_status s2attn_bwd_preprocess(const void* o, const float* lse, const void*
   sh.set_contiguous();
   s2attn_status s = check_workspace(sh, workspace, workspace_bytes);
   if (s != S2ATTN_OK) return s;
-  unsigned int* err = nullptr;
-  int num_sms = 0;
-  if ((s = device_state(&err, &num_sms)) != S2ATTN_OK) return s;
-  return pre_impl(sh, o, lse, dO, workspace, static_cast<cudaStream_t>(stream), err, num_sms);
+  return pre_impl(sh, o, lse, dO, workspace, static_cast<cudaStream_t>(stream));
 }
 
 s2attn_status s2attn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO,
@@ -850,7 +813,7 @@ s2attn_status s2attn_bwd_general(const void* q, const void* k, const void* v, co
   int num_sms = 0;
   if ((s = device_state(&err, &num_sms)) != S2ATTN_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if ((s = pre_impl(sh, o, lse, dO, workspace, st, err, num_sms)) != S2ATTN_OK) return s;
+  if ((s = pre_impl(sh, o, lse, dO, workspace, st)) != S2ATTN_OK) return s;
   const int per_pass = ds_heads_per_pass(sh, workspace_bytes);
   if (per_pass == 0) {
     // Workspace too small for one kv head's dS tiles: the dQ kernel recomputes S and dP.
