@@ -295,6 +295,59 @@ def run_gpu(args, rank, world, local_rank):
     rope_ms = sum(e[0].elapsed_time(e[1]) for e in rope_ev) / rope_reps
     rope_bytes = 2 * (qd.numel() + kd.numel()) * 2
 
+    # The preprocess alone, after an L2 flush whose dirty lines were then evicted by a read-only
+    # pass (so the kernel pays no one else's write-backs): its own streaming rate.
+    pre_alone = None
+    if args.bwd_path == "handoff" and passes == 1:
+        clean = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+        pts = []
+        for i in range(12):
+            flush.fill_(i & 0xFF)
+            clean.sum()
+            a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            s2.s2attn_bwd_preprocess(o, lse, dod, ws)
+            b_.record(stream)
+            torch.cuda.synchronize()
+            if i >= 2:
+                pts.append(a.elapsed_time(b_))
+        pre_alone = statistics.median(pts)
+        del clean
+
+    # RoPE with PI of the queries fused into the forward's query-tile path (s2attn_fwd_rope_q)
+    # against the separate passes, alternating on this GPU, L2 flushed before each:
+    #   separate: rope(Q), rope(K), forward;   fused: rope(K), forward with Q rotated inside.
+    rope_ab = None
+    if args.workload == METRIC_WORKLOAD:
+        qrot = torch.empty_like(qd)
+        times = {"separate": [], "fused": [], "fwd": [], "fwd_rope_q": []}
+        for i in range(12):
+            for mode in ("separate", "fused"):
+                flush.fill_(i & 0xFF)
+                ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+                ev[0].record(stream)
+                if mode == "separate":
+                    s2.s2attn_rope_pi(qd, rq, pi_scale=0.5)
+                    s2.s2attn_rope_pi(kd, rk, pi_scale=0.5)
+                    ev[1].record(stream)
+                    s2.s2attn_fwd(rq, rk, vd, o, lse, w.G, w.scale)
+                else:
+                    s2.s2attn_rope_pi(kd, rk, pi_scale=0.5)
+                    ev[1].record(stream)
+                    s2.s2attn_fwd_rope_q(qd, rk, vd, o, lse, qrot, w.G, w.scale, pi_scale=0.5)
+                ev[2].record(stream)
+                torch.cuda.synchronize()
+                if i >= 2:
+                    times[mode].append(ev[0].elapsed_time(ev[2]))
+                    times["fwd" if mode == "separate" else "fwd_rope_q"].append(ev[1].elapsed_time(ev[2]))
+        # the two rotations differ slightly (angle addition vs per-row fp32 angles)
+        rope_diff = float((qrot.float() - rq.float()).abs().max())
+        rope_ab = {k_: round(statistics.median(v_), 4) for k_, v_ in times.items()}
+        rope_ab["max_abs_q_rot_difference"] = round(rope_diff, 5)
+        st, code = s2.s2attn_get_device_error()
+        if st != s2.S2ATTN_OK:
+            raise RuntimeError(f"device error {st} code {code:#x} in the RoPE comparison")
+
     # Full causal attention (the pages' Phase 2, standard attention after fine-tuning) through
     # the same kernels: one group of N rows and no roll (G = N, no rolled head), on the metric
     # workload's tensors, beside the step (not part of it), L2 flushed.
@@ -408,6 +461,9 @@ def run_gpu(args, rank, world, local_rank):
             entry.update(tflops_algorithmic=round(tf, 1), frac=round(tf / peak_tf, 4))
         if n == "s2_bwd_pre":
             entry.update(gbs=round(pre_bytes(w) / (avg[n] * 1e-3) / 1e9, 1))
+            if pre_alone is not None:
+                entry.update(alone_after_clean_l2_ms=round(pre_alone, 4),
+                             alone_gbs=round(pre_bytes(w) / (pre_alone * 1e-3) / 1e9, 1))
         if n == "s2_bwd_dq_ds":
             entry.update(gbs=round(dq_ds_bytes(w, ds_tiles) / (avg[n] * 1e-3) / 1e9, 1),
                          ds_tiles=int(ds_tiles))
@@ -423,6 +479,13 @@ def run_gpu(args, rank, world, local_rank):
         "ms": round(rope_ms, 4), "bytes": rope_bytes,
         "gbs": round(rope_bytes / (rope_ms * 1e-3) / 1e9, 1),
         "frac_of_hbm": round(rope_bytes / (rope_ms * 1e-3) / 1e9 / hbm, 4)}}
+    if rope_ab is not None:
+        next_rows["rope_pi_fused_q"] = {
+            "what": "RoPE-PI of Q fused into the forward (s2attn_fwd_rope_q) vs separate passes, "
+                    "median ms, alternating, L2 flushed: separate = rope(Q) + rope(K) + forward, "
+                    "fused = rope(K) + forward rotating Q itself",
+            **rope_ab,
+            "fused_minus_separate_ms": round(rope_ab["fused"] - rope_ab["separate"], 4)}
     if full_causal is not None:
         fc_flops = 7.0 * w.B * w.Hq * w.N * w.N * w.d
         fc_ms = full_causal["fwd_ms"] + full_causal["bwd_ms"]

@@ -67,7 +67,7 @@ typedef enum {
 /* Version of this ABI (bumped on any signature change or workspace-size change); 2 adds the
  * dS hand-off entries and the work counters in the backward workspace; 3 adds the option flags
  * (_general entries, which replace the strided-only entries) and s2attn_rope_pi; 4 adds the
- * _general forms of the two dS hand-off stages. */
+ * _general forms of the two dS hand-off stages; 5 adds s2attn_fwd_rope_q. */
 S2ATTN_API int s2attn_abi_version(void);
 
 /* Static description of a status code. */
@@ -141,6 +141,25 @@ S2ATTN_API s2attn_status s2attn_fwd_general(const void* q, const void* k, const 
                                             float* lse, int B, int Hq, int Hkv, int N, int d,
                                             int G, float scale, int shift_head_begin, int shift,
                                             int flags, const long long* strides, void* stream);
+
+/*
+ * Forward with the rotary position embedding of the queries fused into the kernel's query-tile
+ * path (summary page, §3 "Phase 1" step 2 and §4 "Model setup": RoPE with positions rescaled by
+ * Position Interpolation, the step just before the attention). q holds the UN-rotated queries;
+ * k must already be rotated (s2attn_rope_pi); each 128-row query tile is rotated in shared
+ * memory after it lands, exactly the rotation s2attn_rope_pi applies (pair (x[i], x[i + d/2]) of
+ * token t turned by (t * pi_scale) * base^(-2i/d)), before the tensor cores read it, and the
+ * rotated rows are also written to q_rot (contiguous bf16 [B, N, Hq, d]), which the backward
+ * needs. Otherwise as s2attn_fwd_general with contiguous tensors (no strides). q_rot may be q
+ * itself (rotation in place: every query row is read and rewritten by the same tile); no other
+ * overlap is allowed. Errors as s2attn_fwd_general, plus: q_rot NULL or misaligned, base <= 1 or
+ * pi_scale <= 0 -> S2ATTN_ERR_INVALID_ARG; N >= 2^24 -> S2ATTN_ERR_UNSUPPORTED.
+ */
+S2ATTN_API s2attn_status s2attn_fwd_rope_q(const void* q, const void* k, const void* v, void* o,
+                                           float* lse, void* q_rot, int B, int Hq, int Hkv,
+                                           int N, int d, int G, float scale,
+                                           int shift_head_begin, int shift, int flags,
+                                           float base, float pi_scale, void* stream);
 
 /* Smallest device workspace s2attn_bwd accepts: two fp32 [B, Hq, N] arrays (D and LSE in
  * base 2), each rounded up to 256 bytes, and 256 bytes of work counters for the gradient

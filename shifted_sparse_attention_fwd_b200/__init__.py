@@ -19,6 +19,7 @@ from ._lib import (  # noqa: F401
     lib,
     status_string,
     s2attn_fwd,
+    s2attn_fwd_rope_q,
     s2attn_bwd,
     s2attn_bwd_workspace_size,
     s2attn_bwd_workspace_size_ex,

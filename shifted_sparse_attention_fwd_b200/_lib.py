@@ -47,6 +47,7 @@ SIGNATURES = {
     "s2attn_bwd_noalloc": (_I, [_P] * 9 + [_I] * 6 + [_F, _P]),
     "s2attn_bwd_workspace_size_ex": (_Z, [_I] * 8 + [_Z]),
     "s2attn_fwd_general": (_I, [_P] * 5 + [_I] * 6 + [_F, _I, _I, _I, _P, _P]),
+    "s2attn_fwd_rope_q": (_I, [_P] * 6 + [_I] * 6 + [_F, _I, _I, _I, _F, _F, _P]),
     "s2attn_bwd_general": (_I, [_P] * 9 + [_I] * 6 + [_F, _I, _I, _I, _P, _P, _Z, _P]),
     "s2attn_bwd_workspace_size_general": (_Z, [_I] * 9 + [_Z]),
     "s2attn_rope_pi": (_I, [_P, _P, _I, _I, _I, _I, _F, _F, _I, _P, _P]),
@@ -171,6 +172,20 @@ def s2attn_fwd(q, k, v, o, lse, G, scale=None, shift_head_begin=None, shift=None
     sh = G // 2 if shift is None else shift
     _check(lib().s2attn_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, N, d,
                                G, scale, shb, sh, _stream(stream)), "s2attn_fwd_ex")
+
+
+def s2attn_fwd_rope_q(q, k, v, o, lse, q_rot, G, scale=None, shift_head_begin=None, shift=None,
+                      flags=0, base=10000.0, pi_scale=1.0, stream=None):
+    """Forward with the RoPE-PI rotation of the queries fused in: q un-rotated, k already rotated
+    (s2attn_rope_pi); also writes the rotated queries to q_rot (may be q itself)."""
+    _check_bf16(q, k, v, o, q_rot)
+    B, Hq, Hkv, N, d, G = _dims(q, k, G)
+    scale = d ** -0.5 if scale is None else scale
+    shb = Hq // 2 if shift_head_begin is None else shift_head_begin
+    sh = G // 2 if shift is None else shift
+    _check(lib().s2attn_fwd_rope_q(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(q_rot), B,
+                                   Hq, Hkv, N, d, G, scale, shb, sh, int(flags), float(base),
+                                   float(pi_scale), _stream(stream)), "s2attn_fwd_rope_q")
 
 
 def s2attn_bwd_workspace_size(B, Hq, N) -> int:

@@ -13,7 +13,7 @@
 // heaviest first within L2-sized groups), so one unit's epilogue and the next unit's loads
 // overlap the tensor-core work and the CTAs finish together.
 //
-// Warp roles (320 threads):
+// Warp roles (320 threads; 352 with the fused RoPE of the queries):
 //   warps 0-3, 4-7  softmax warpgroup of query tile 0 / 1: thread i owns query row i (TMEM
 //                   lane i); online softmax in fp32, P written back to TMEM as bf16 over S,
 //                   O rescaled in TMEM when the running max grows, epilogue.
@@ -21,6 +21,8 @@
 //                   V tiles (2-slot rings); each ring slot is released by a commit right
 //                   after the last MMA that reads it.
 //   warp 9          TMEM allocator and MMA issuer (one lane).
+//   warp 10         (fused RoPE only) rotates each query tile in shared memory once it has
+//                   landed and writes the rotated rows out; the MMAs wait for it.
 // TMEM columns: S0/P0 [0,128), S1/P1 [128,256), O0 [256,256+D), O1 [256+D, 256+2D).
 //
 // MMA issue order S0(0) S1(0) PV0(0) S0(1) PV1(0) S1(1) PV0(1) ... lets each warpgroup's
@@ -48,6 +50,11 @@ struct FwdParams {
   float scale_log2;   // scale * log2(e)
   unsigned int* err;
   unsigned long long timeout_ns;
+  // Fused rotary position embedding of the queries (kernel built with kRope): q holds the
+  // un-rotated queries, each query tile is rotated in shared memory before its first MMA and
+  // the rotated rows are written to q_rot (contiguous [B, N, Hq, D]).
+  __nv_bfloat16* q_rot;
+  float rope_log2_base, rope_pi_scale;
 };
 
 // Which work units each CTA takes, computed on the host (longest-processing-time-first: the
@@ -88,7 +95,7 @@ struct FwdLayout {
   static constexpr uint32_t kBar = kStage + 8 * kStageWarp;
   enum { B_Q = 0, B_QE = 2, B_K = 4, B_KE = B_K + kKStages, B_V = B_KE + kKStages,
          B_VE = B_V + kVStages, B_S = B_VE + kVStages, B_P = B_S + 2, B_ODONE = B_P + 2,
-         B_DRAIN = B_ODONE + 2, B_COUNT = B_DRAIN + 1 };
+         B_DRAIN = B_ODONE + 2, B_QR = B_DRAIN + 1, B_COUNT = B_QR + 2 };
   static constexpr uint32_t kTmemSlot = kBar + B_COUNT * 8;
   static constexpr uint32_t kAbort = kTmemSlot + 4;
   static constexpr uint32_t kBytes = kAbort + 4;
@@ -97,7 +104,72 @@ struct FwdLayout {
   static constexpr uint32_t kLaunchBytes =
       (kBytes + 1024 > 116 * 1024) ? kBytes + 1024 : 116 * 1024;
   static constexpr int kThreads = 320;
+  static constexpr int kRopeThreads = 352;   // + the rotation warp (warp 10) of the fused RoPE
 };
+
+// Fused RoPE with Position Interpolation of one 128-row query tile in shared memory (the
+// 128-byte-swizzled TMA layout), by one warp: the same rotation as s2_rope_kernel — the pair
+// (x[i], x[i + D/2]) of token t turns by (t * pi_scale) * base^(-2i/D) — written back in place
+// for the MMAs and to q_rot at the tile's original rows. Lane w of a row owns the 4-byte word of
+// columns 2w, 2w + 1 and its partner D/2 columns on. The angle of a run's first row is computed
+// as there (fp32 product, accurate sincosf); each following row of the run is reached by turning
+// by one token's angle (angle addition in fp32, relative drift about 1e-6 over a tile, far below
+// the bf16 rounding of the result).
+template <int D>
+__device__ __forceinline__ uint32_t swz_word(uint32_t tile, int row, int col) {
+  const int half = col / 64, cc = col % 64;
+  return tile + half * Tile<D>::kHalfBytes + row * 128 + ((((cc / 8) ^ (row & 7))) << 4) + (cc % 8) * 2;
+}
+template <int D>
+__device__ __noinline__ void rope_query_tile(uint32_t tile, const Runs tr, __nv_bfloat16* q_rot,
+                                             int N, int Hq, float log2_base, float pi_scale,
+                                             int b, int h) {
+  constexpr int kLanesPerRow = D / 4;
+  constexpr int kRowsPerStep = 32 / kLanesPerRow;
+  const int lane = threadIdx.x & 31;
+  const int w = lane % kLanesPerRow, r_off = lane / kLanesPerRow;
+  float th[2], cd[2], sd[2];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    th[k] = exp2f(-(2.0f * (2 * w + k) / D) * log2_base);
+    sincosf((kRowsPerStep * pi_scale) * th[k], &sd[k], &cd[k]);
+  }
+  __nv_bfloat16* out = q_rot + static_cast<long long>(b) * N * Hq * D + static_cast<long long>(h) * D;
+  int base = 0;
+  for (int r = 0; r < tr.n; ++r) {
+    const int len = tr.len[r], src = tr.src[r];
+    float c[2], sn[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k)
+      sincosf((static_cast<float>(src + r_off) * pi_scale) * th[k], &sn[k], &c[k]);
+    for (int i = r_off; i < len; i += kRowsPerStep) {
+      const int row = base + i;
+      const uint32_t a_lo = swz_word<D>(tile, row, 2 * w), a_hi = swz_word<D>(tile, row, 2 * w + D / 2);
+      uint32_t lo, hi;
+      asm volatile("ld.shared.b32 %0, [%1];" : "=r"(lo) : "r"(a_lo));
+      asm volatile("ld.shared.b32 %0, [%1];" : "=r"(hi) : "r"(a_hi));
+      const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&lo));
+      const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hi));
+      __nv_bfloat162 nx = __floats2bfloat162_rn(x.x * c[0] - y.x * sn[0], x.y * c[1] - y.y * sn[1]);
+      __nv_bfloat162 ny = __floats2bfloat162_rn(y.x * c[0] + x.x * sn[0], y.y * c[1] + x.y * sn[1]);
+      const uint32_t nlo = *reinterpret_cast<uint32_t*>(&nx), nhi = *reinterpret_cast<uint32_t*>(&ny);
+      asm volatile("st.shared.b32 [%0], %1;" ::"r"(a_lo), "r"(nlo) : "memory");
+      asm volatile("st.shared.b32 [%0], %1;" ::"r"(a_hi), "r"(nhi) : "memory");
+      __nv_bfloat16* dst = out + static_cast<long long>(src + i) * Hq * D + 2 * w;
+      *reinterpret_cast<uint32_t*>(dst) = nlo;
+      *reinterpret_cast<uint32_t*>(dst + D / 2) = nhi;
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const float cn = c[k] * cd[k] - sn[k] * sd[k];
+        sn[k] = sn[k] * cd[k] + c[k] * sd[k];
+        c[k] = cn;
+      }
+    }
+    base += len;
+  }
+  fence_async_smem();   // the MMAs read the rotated tile through the async proxy
+  __syncwarp();
+}
 
 // Row maximum of 128 values: eight independent chains of three-input max instructions.
 __device__ __forceinline__ float max_tree128(const float (&s)[128]) {
@@ -151,8 +223,8 @@ __device__ __forceinline__ FwdUnit fwd_unit(const FwdParams& p, int unit) {
   return u;
 }
 
-template <int D, bool kFront>
-__global__ void __launch_bounds__(320, 1)
+template <int D, bool kFront, bool kRope>
+__global__ void __launch_bounds__(kRope ? 352 : 320, 1)
     s2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQ8,
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmK8,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmV8,
@@ -177,6 +249,7 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(bar(L::B_S + s), 1);
       mbar_init(bar(L::B_P + s), 128);
       mbar_init(bar(L::B_ODONE + s), 1);
+      mbar_init(bar(L::B_QR + s), 1);
     }
     for (int s = 0; s < L::kKStages; ++s) {
       mbar_init(bar(L::B_K + s), 1);
@@ -276,7 +349,8 @@ __global__ void __launch_bounds__(320, 1)
         // S_t(j) = Q_t K(j)^T into TMEM columns [128 t, 128 t + 128).
         auto issue_s = [&](int t, int kidx) -> bool {
           if (!q_ready[t]) {
-            if (!wait_bar(bar(L::B_Q + t), q_used[t] & 1, ctx, 2)) return false;
+            // (with the fused RoPE: once the rotation warp has turned the tile)
+            if (!wait_bar(bar((kRope ? L::B_QR : L::B_Q) + t), q_used[t] & 1, ctx, 2)) return false;
             q_ready[t] = true;
             ++q_used[t];
           }
@@ -327,6 +401,27 @@ __global__ void __launch_bounds__(320, 1)
         }
         k_used = k0 + u.n_kv;
         v_used = v0 + u.n_kv;
+      }
+    }
+  } else if (warp == 10) {
+    // ---------------- rotation warp (fused RoPE of the queries) ----------------
+    if (kRope) {
+      int q_loads[2] = {0, 0};
+      bool ok = true;
+      for (int ku = 0; ok; ++ku) {
+        const int unit = fwd_unit_index(sched, n_units, ku);
+        if (unit < 0) break;
+        const FwdUnit u = fwd_unit<kFront>(p, unit);
+        for (int t = 0; t < 2; ++t) {
+          if (!u.tv[t]) continue;
+          if (!warp_wait(bar(L::B_Q + t), q_loads[t] & 1, ctx, 11)) { ok = false; break; }
+          ++q_loads[t];
+          rope_query_tile<D>(sbase + L::kQ + t * L::kTile,
+                             rolled_runs(head_remap(p.N, p.G, u.shift_h, kFront ? u.front_h : 0),
+                                         u.qt[t] * kTileRows),
+                             p.q_rot, p.N, p.Hq, p.rope_log2_base, p.rope_pi_scale, u.b, u.h);
+          if (lane == 0) mbar_arrive(bar(L::B_QR + t));
+        }
       }
     }
   } else {

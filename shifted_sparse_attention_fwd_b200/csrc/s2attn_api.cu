@@ -27,7 +27,7 @@ namespace {
 
 __device__ unsigned int g_err_word;   // first pipeline-wait failure since the last read
 
-constexpr int kAbiVersion = 4;
+constexpr int kAbiVersion = 5;
 constexpr int kMaxDevices = 64;
 constexpr unsigned long long kDefaultTimeoutNs = 1000000000ull;
 
@@ -53,7 +53,10 @@ std::once_flag g_encode_once;
 template <int D, bool kFront>
 cudaError_t set_smem_attrs_variant() {
   cudaError_t e;
-  e = cudaFuncSetAttribute(s2::s2_fwd_kernel<D, kFront>,
+  e = cudaFuncSetAttribute(s2::s2_fwd_kernel<D, kFront, false>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, s2::FwdLayout<D>::kLaunchBytes);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(s2::s2_fwd_kernel<D, kFront, true>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, s2::FwdLayout<D>::kLaunchBytes);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(s2::s2_bwd_dkdv_kernel<D, kFront>,
@@ -296,10 +299,16 @@ void fwd_schedule_cached(const Shape& sh, int grid, s2::FwdSchedule& out) {
   es.back().sched = out;
 }
 
+// Fused RoPE of the queries (s2attn_fwd_rope_q): where the rotated queries go and the rotation.
+struct RopeArgs {
+  void* q_rot = nullptr;
+  float log2_base = 0.f, pi_scale = 0.f;
+};
+
 template <int D>
 s2attn_status launch_fwd(const Shape& sh, const void* q, const void* k, const void* v, void* o,
                          float* lse, float scale, cudaStream_t stream, unsigned int* err,
-                         int num_sms) {
+                         int num_sms, const RopeArgs& rope = RopeArgs{}) {
   MapPair mq, mk, mv;
   s2attn_status s;
   if ((s = encode_pair(mq, q, sh.B, sh.Hq, sh.N, D, sh.sb[T_Q], sh.st[T_Q])) != S2ATTN_OK) return s;
@@ -322,14 +331,25 @@ s2attn_status launch_fwd(const Shape& sh, const void* q, const void* k, const vo
   p.timeout_ns = g_timeout_ns.load();
   const unsigned units = static_cast<unsigned>(sh.B) * sh.Hq * s2::query_pairs_per_head(sh.N);
   const unsigned grid = units < static_cast<unsigned>(num_sms) ? units : static_cast<unsigned>(num_sms);
+  p.q_rot = static_cast<__nv_bfloat16*>(rope.q_rot);
+  p.rope_log2_base = rope.log2_base;
+  p.rope_pi_scale = rope.pi_scale;
   static thread_local s2::FwdSchedule sched;
   fwd_schedule_cached(sh, static_cast<int>(grid), sched);
-  if (sh.front)
-    s2::s2_fwd_kernel<D, true><<<grid, s2::FwdLayout<D>::kThreads, s2::FwdLayout<D>::kLaunchBytes,
-                                 stream>>>(mq.m128, mq.m8, mk.m128, mk.m8, mv.m128, mv.m8, p, sched);
+  constexpr uint32_t kSmem = s2::FwdLayout<D>::kLaunchBytes;
+  constexpr int kT = s2::FwdLayout<D>::kThreads, kTR = s2::FwdLayout<D>::kRopeThreads;
+  if (rope.q_rot && sh.front)
+    s2::s2_fwd_kernel<D, true, true><<<grid, kTR, kSmem, stream>>>(mq.m128, mq.m8, mk.m128, mk.m8,
+                                                                   mv.m128, mv.m8, p, sched);
+  else if (rope.q_rot)
+    s2::s2_fwd_kernel<D, false, true><<<grid, kTR, kSmem, stream>>>(mq.m128, mq.m8, mk.m128, mk.m8,
+                                                                    mv.m128, mv.m8, p, sched);
+  else if (sh.front)
+    s2::s2_fwd_kernel<D, true, false><<<grid, kT, kSmem, stream>>>(mq.m128, mq.m8, mk.m128, mk.m8,
+                                                                   mv.m128, mv.m8, p, sched);
   else
-    s2::s2_fwd_kernel<D, false><<<grid, s2::FwdLayout<D>::kThreads, s2::FwdLayout<D>::kLaunchBytes,
-                                  stream>>>(mq.m128, mq.m8, mk.m128, mk.m8, mv.m128, mv.m8, p, sched);
+    s2::s2_fwd_kernel<D, false, false><<<grid, kT, kSmem, stream>>>(mq.m128, mq.m8, mk.m128, mk.m8,
+                                                                    mv.m128, mv.m8, p, sched);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? S2ATTN_OK : cuda_fail(e, "s2_fwd_kernel launch");
 }
@@ -576,6 +596,33 @@ s2attn_status s2attn_fwd_general(const void* q, const void* k, const void* v, vo
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return d == 64 ? launch_fwd<64>(sh, q, k, v, o, lse, scale, st, err, num_sms)
                  : launch_fwd<128>(sh, q, k, v, o, lse, scale, st, err, num_sms);
+}
+
+s2attn_status s2attn_fwd_rope_q(const void* q, const void* k, const void* v, void* o, float* lse,
+                                void* q_rot, int B, int Hq, int Hkv, int N, int d, int G,
+                                float scale, int shift_head_begin, int shift, int flags,
+                                float base, float pi_scale, void* stream) {
+  if (!q || !k || !v || !o || !lse || !q_rot) return S2ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+      !aligned16(q_rot))
+    return S2ATTN_ERR_INVALID_ARG;
+  if (!(base > 1.f) || !std::isfinite(base) || !(pi_scale > 0.f) || !std::isfinite(pi_scale))
+    return S2ATTN_ERR_INVALID_ARG;
+  Shape sh;
+  s2attn_status s = check_shape(B, Hq, Hkv, N, d, G, scale, shift_head_begin, shift, sh, flags);
+  if (s != S2ATTN_OK) return s;
+  if (N >= (1 << 24)) return S2ATTN_ERR_UNSUPPORTED;   // positions exact in fp32, as s2attn_rope_pi
+  if ((s = get_encoder()) != S2ATTN_OK) return s;
+  unsigned int* err = nullptr;
+  int num_sms = 0;
+  if ((s = device_state(&err, &num_sms)) != S2ATTN_OK) return s;
+  RopeArgs rope;
+  rope.q_rot = q_rot;
+  rope.log2_base = std::log2(base);
+  rope.pi_scale = pi_scale;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return d == 64 ? launch_fwd<64>(sh, q, k, v, o, lse, scale, st, err, num_sms, rope)
+                 : launch_fwd<128>(sh, q, k, v, o, lse, scale, st, err, num_sms, rope);
 }
 
 s2attn_status s2attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse,

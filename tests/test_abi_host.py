@@ -50,7 +50,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.s2attn_abi_version() == 4
+    assert lib.s2attn_abi_version() == 5
     for st in range(5):
         assert s2.status_string(st)
     assert s2.status_string(99) == "unknown status"
@@ -399,6 +399,19 @@ def test_query_pair_order_is_a_permutation(shim, B, Hq, N, G):
     if G % 256 == 0 and G > 256:
         b, h, p = call4(shim.paircoords, 0, B, Hq, N, G)[:3]
         assert p % (G // 256) == G // 256 - 1
+
+
+def test_fwd_rope_q_rejects(lib):
+    f = ctypes.c_float(0.125)
+    ok = [A] * 6 + [1, 4, 4, 256, 64, 64, f, 2, 32, 0]
+    assert lib.s2attn_fwd_rope_q(*([A] * 5), None, *ok[6:], ctypes.c_float(10000.0),
+                                 ctypes.c_float(1.0), None) == 1                  # no q_rot
+    assert lib.s2attn_fwd_rope_q(*([A] * 5), A + 8, *ok[6:], ctypes.c_float(10000.0),
+                                 ctypes.c_float(1.0), None) == 1                  # misaligned
+    assert lib.s2attn_fwd_rope_q(*ok, ctypes.c_float(1.0), ctypes.c_float(1.0), None) == 1  # base
+    assert lib.s2attn_fwd_rope_q(*ok, ctypes.c_float(10000.0), ctypes.c_float(0.0), None) == 1
+    bad_d = [A] * 6 + [1, 4, 4, 256, 96, 64, f, 2, 32, 0]
+    assert lib.s2attn_fwd_rope_q(*bad_d, ctypes.c_float(10000.0), ctypes.c_float(1.0), None) == 2
 
 
 def test_rope_rejects(lib):

@@ -15,7 +15,7 @@ import pytest
 import torch
 
 from oracle import s2attn_oracle as orc
-from shifted_sparse_attention_fwd_b200.inputs import WORKLOADS, make_workload_inputs, to_f64
+from shifted_sparse_attention_fwd_b200.inputs import WORKLOADS, make_inputs, make_workload_inputs, to_f64
 
 from gpu_helpers import assert_close, check_case, gpu_run
 
@@ -75,3 +75,28 @@ def test_full_size_sampled(name):
             dv_ref = np.stack([acc[t][1] for t in toks])
             assert_close("dk", g["dk"][b, toks, kvh], dk_ref)
             assert_close("dv", g["dv"][b, toks, kvh], dv_ref)
+
+
+def test_full_causal_n8192_sampled():
+    """Full causal attention (the pages' Phase 2: standard attention after fine-tuning) at the
+    metric length through the same kernels: one group of G = N = 8192 rows and no rolled head.
+    Every head on sampled rows against the oracle's row-restricted evaluation: query rows at
+    the start, the end and random places of the sequence; kv rows at the start (seen by all
+    8192 query rows) and at the end."""
+    B, Hq, Hkv, N, d = 1, 8, 8, 8192, 128
+    q, k, v, do = make_inputs(B, Hq, Hkv, N, d, 1006)
+    scale = d ** -0.5
+    g = gpu_run(q, k, v, do, N, scale, shb=Hq, shift=0)
+    rng = np.random.default_rng(1006)
+    q_rows = np.unique(np.concatenate([np.arange(64), np.arange(N - 64, N), rng.integers(0, N, 64)]))
+    kv_rows = np.concatenate([np.arange(8), np.arange(N - 128, N)])
+    for h in range(Hq):
+        r = orc.head_group_rows(to_f64(q[0, :, h]), to_f64(k[0, :, h]), to_f64(v[0, :, h]),
+                                to_f64(do[0, :, h]), N, scale, 0, 0, q_rows, kv_rows)
+        t = r["q_tok"]
+        assert_close("o", g["o"][0, t, h], r["o"])
+        assert_close("lse", g["lse"][0, h, t], r["lse"])
+        assert_close("dq", g["dq"][0, t, h], r["dq"])
+        tk = r["kv_tok"]
+        assert_close("dk", g["dk"][0, tk, h], r["dk"])
+        assert_close("dv", g["dv"][0, tk, h], r["dv"])

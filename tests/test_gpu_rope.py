@@ -90,3 +90,43 @@ def test_rope_then_s2attn_forward_and_backward():
     for name, g, r in (("o", o, o_ref), ("lse", lse, lse_ref), ("dq", dq, dq_ref),
                        ("dk", dk, dk_ref), ("dv", dv, dv_ref)):
         assert_close(name, g.cpu(), r)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,G,d,shift,flags,pi", [
+    (1, 8, 8, 2048, 512, 128, None, 0, 0.5),     # Llama-like heads, PI 4k -> 8k
+    (2, 4, 2, 640, 128, 64, None, 0, 1.0),       # d = 64 (two rows per lane step), GQA, batch 2
+    (1, 4, 2, 512, 128, 128, 37, 2, 0.25),       # a roll of 37 under Variant 3: tiles of 3 runs
+])
+def test_fused_rope_q_forward(B, Hq, Hkv, N, G, d, shift, flags, pi):
+    """s2attn_fwd_rope_q: the queries' RoPE-PI fused into the forward's query-tile path. The
+    rotated queries it writes match the oracle's rope_pi as closely as the standalone kernel's
+    do (run starts are computed as there, later rows by angle addition, which avoids the fp32
+    rounding of large angles); O and LSE match the oracle's attention over those rotated values;
+    rotating in place gives the same bits."""
+    q, k, v, _ = make_inputs(B, Hq, Hkv, N, d, 77 + N, 1.0)
+    scale = d ** -0.5
+    dev = torch.device("cuda")
+    qd, kd, vd = (t.to(dev) for t in (q, k, v))
+    kr = s2.rope_pi(kd, pi_scale=pi)
+    o, lse = torch.empty_like(qd), torch.empty((B, Hq, N), dtype=torch.float32, device=dev)
+    qr = torch.empty_like(qd)
+    s2.s2attn_fwd_rope_q(qd, kr, vd, o, lse, qr, G, scale, shift=shift, flags=flags, pi_scale=pi)
+    torch.cuda.synchronize()
+    st, code = s2.s2attn_get_device_error()
+    assert st == s2.S2ATTN_OK, (st, code)
+    # the rotated queries: as close to the exact rotation as the standalone kernel's
+    q_ref = orc.rope_pi(to_f64(q), pi_scale=pi)
+    fused_err = assert_close("q_rot", qr.cpu(), q_ref)["max_abs"]
+    alone_err = assert_close("q_rot", s2.rope_pi(qd, pi_scale=pi).cpu(), q_ref)["max_abs"]
+    assert fused_err <= alone_err * 1.25 + 1e-3, (fused_err, alone_err)
+    wrap = bool(flags & s2.S2ATTN_FLAG_WRAP_OWN_GROUP)
+    front = bool(flags & s2.S2ATTN_FLAG_WRAP_FRONT_FIRST)
+    o_ref, lse_ref = orc.s2attn_forward(to_f64(qr.cpu()), to_f64(kr.cpu()), to_f64(v), G, scale,
+                                        shift=shift, wrap_own_group=wrap, wrap_front_first=front)
+    assert_close("o", o.cpu(), o_ref)
+    assert_close("lse", lse.cpu(), lse_ref)
+    # in place: q_rot = q
+    o2, lse2 = torch.empty_like(o), torch.empty_like(lse)
+    s2.s2attn_fwd_rope_q(qd, kr, vd, o2, lse2, qd, G, scale, shift=shift, flags=flags, pi_scale=pi)
+    torch.cuda.synchronize()
+    assert torch.equal(qd, qr) and torch.equal(o2, o) and torch.equal(lse2, lse)
