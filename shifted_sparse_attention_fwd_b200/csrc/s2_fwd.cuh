@@ -83,6 +83,15 @@ __device__ __forceinline__ int fwd_unit_index(const FwdSchedule& s, int n_units,
 // exp2(s - stale max) <= 2^8, harmless in fp32 and bf16, and the final 1/l uses the same max.
 constexpr float kRescaleThreshold = 8.0f;
 
+// The integer divisions of a unit's decoding: (b, h, pair), the kv head and each tile's first
+// key tile. About 2000 cycles on one thread, so a CTA decodes its first kLocalUnits units
+// once, at the start, into shared memory (b = -1: no such unit), and every role reads them
+// from there at its unit boundaries.
+struct FwdUnitRec {
+  int b, h, pair, kvh, kb[2];
+};
+constexpr int kLocalUnits = 64;
+
 template <int D>
 struct FwdLayout {
   static constexpr uint32_t kTile = Tile<D>::kBytes;
@@ -92,7 +101,8 @@ struct FwdLayout {
   static constexpr uint32_t kV = kK + kKStages * kTile;     // V ring
   static constexpr uint32_t kStageWarp = 32 * 128;          // O staging: 32 rows x 64 columns
   static constexpr uint32_t kStage = kV + kVStages * kTile; // ... for each softmax warp
-  static constexpr uint32_t kBar = kStage + 8 * kStageWarp;
+  static constexpr uint32_t kRecs = kStage + 8 * kStageWarp;   // kLocalUnits FwdUnitRec
+  static constexpr uint32_t kBar = kRecs + kLocalUnits * sizeof(FwdUnitRec);
   enum { B_Q = 0, B_QE = 2, B_K = 4, B_KE = B_K + kKStages, B_V = B_KE + kKStages,
          B_VE = B_V + kVStages, B_S = B_VE + kVStages, B_P = B_S + 2, B_ODONE = B_P + 2,
          B_DRAIN = B_ODONE + 2, B_QR = B_DRAIN + 1, B_COUNT = B_QR + 2 };
@@ -105,6 +115,7 @@ struct FwdLayout {
       (kBytes + 1024 > 116 * 1024) ? kBytes + 1024 : 116 * 1024;
   static constexpr int kThreads = 320;
   static constexpr int kRopeThreads = 352;   // + the rotation warp (warp 10) of the fused RoPE
+  static_assert(kLaunchBytes <= 227 * 1024, "shared memory of one CTA");
 };
 
 // Fused RoPE with Position Interpolation of one 128-row query tile in shared memory (the
@@ -197,25 +208,40 @@ struct FwdUnit {
   }
 };
 
+template <bool kFront>
+__device__ __forceinline__ FwdUnitRec fwd_unit_rec(const FwdParams& p, int unit) {
+  FwdUnitRec r;
+  query_pair_coords_chunked(unit, p.B, p.Hq, p.N, p.G, kL2Chunk, r.b, r.h, r.pair);
+  r.kvh = r.h / (p.Hq / p.Hkv);
+  const int nqt = (p.N + kTileRows - 1) / kTileRows;
+  const int wrap_h = r.h >= p.shift_head_begin ? p.wrap : kNoWrapSplit;
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int qt = 2 * r.pair + t;
+    r.kb[t] = qt < nqt ? group_begin(qt * kTileRows, p.G, wrap_h) / kTileRows : 0;
+  }
+  return r;
+}
+
 // kFront: the kernel is built for the Variant 3 reordering (otherwise p.front is ignored and
 // the plain-roll index code is all that is compiled in).
 template <bool kFront>
-__device__ __forceinline__ FwdUnit fwd_unit(const FwdParams& p, int unit) {
+__device__ __forceinline__ FwdUnit fwd_unit_from(const FwdParams& p, const FwdUnitRec& r) {
   FwdUnit u;
-  int pair;
-  query_pair_coords_chunked(unit, p.B, p.Hq, p.N, p.G, kL2Chunk, u.b, u.h, pair);
+  u.b = r.b;
+  u.h = r.h;
+  u.kvh = r.kvh;
   const int nqt = (p.N + kTileRows - 1) / kTileRows;
   const bool shifted = u.h >= p.shift_head_begin;
   u.shift_h = shifted ? p.shift : 0;
   u.front_h = (kFront && shifted) ? p.front : 0;
   u.wrap_h = shifted ? p.wrap : kNoWrapSplit;
-  u.kvh = u.h / (p.Hq / p.Hkv);
   // Tile t = 2*pair + t sees key tiles [kb[t], ke[t]]; tile 0 always exists, tile 1 may not.
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
-    u.qt[t] = 2 * pair + t;
+    u.qt[t] = 2 * r.pair + t;
     u.tv[t] = u.qt[t] < nqt;
-    u.kb[t] = u.tv[t] ? group_begin(u.qt[t] * kTileRows, p.G, u.wrap_h) / kTileRows : 0;
+    u.kb[t] = r.kb[t];
     u.ke[t] = u.qt[t];
   }
   u.kv_lo = u.kb[0];
@@ -223,12 +249,30 @@ __device__ __forceinline__ FwdUnit fwd_unit(const FwdParams& p, int unit) {
   return u;
 }
 
+// The k-th unit of this CTA into u; false when it has no more.
+template <bool kFront>
+__device__ __forceinline__ bool fwd_unit_k(const FwdParams& p, const FwdSchedule& sched,
+                                           int n_units, const FwdUnitRec* recs, int k, FwdUnit& u) {
+  FwdUnitRec r;
+  if (k < kLocalUnits) {
+    r = recs[k];
+    if (r.b < 0) return false;
+  } else {
+    const int unit = fwd_unit_index(sched, n_units, k);
+    if (unit < 0) return false;
+    r = fwd_unit_rec<kFront>(p, unit);
+  }
+  u = fwd_unit_from<kFront>(p, r);
+  return true;
+}
+
 template <int D, bool kFront, bool kRope>
 __global__ void __launch_bounds__(kRope ? 352 : 320, 1)
     s2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQ8,
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmK8,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmV8,
-                  const FwdParams p, const __grid_constant__ FwdSchedule sched) {
+                  const __grid_constant__ CUtensorMap tmO8, const FwdParams p,
+                  const __grid_constant__ FwdSchedule sched) {
   using L = FwdLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = aligned_smem(smem_raw);
@@ -239,6 +283,7 @@ __global__ void __launch_bounds__(kRope ? 352 : 320, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kTmemSlot);
   const WaitCtx ctx{abort_flag, p.err, p.timeout_ns, KID_FWD};
   const int n_units = p.B * p.Hq * query_pairs_per_head(p.N);
+  FwdUnitRec* recs = reinterpret_cast<FwdUnitRec*>(smem + L::kRecs);
 
   if (warp == 8 && lane == 0) {
     for (int s = 0; s < 2; ++s) {
@@ -261,6 +306,15 @@ __global__ void __launch_bounds__(kRope ? 352 : 320, 1)
     tma_prefetch_map(&tmQ);
     tma_prefetch_map(&tmK);
     tma_prefetch_map(&tmV);
+    tma_prefetch_map(&tmO8);
+  }
+  if (warp == 8) {
+    for (int i = lane; i < kLocalUnits; i += 32) {
+      const int unit = fwd_unit_index(sched, n_units, i);
+      FwdUnitRec r{-1, 0, 0, 0, {0, 0}};
+      if (unit >= 0) r = fwd_unit_rec<kFront>(p, unit);
+      recs[i] = r;
+    }
   }
   if (warp == 9) {
     tmem_alloc(smem_u32(tmem_slot), 512);
@@ -303,9 +357,8 @@ __global__ void __launch_bounds__(kRope ? 352 : 320, 1)
         return true;
       };
       for (int ku = 0; ok; ++ku) {
-        const int unit = fwd_unit_index(sched, n_units, ku);
-        if (unit < 0) break;
-        const FwdUnit u = fwd_unit<kFront>(p, unit);
+        FwdUnit u;
+        if (!fwd_unit_k<kFront>(p, sched, n_units, recs, ku, u)) break;
         ok = issue_k(u, 0);   // the first key tile can stream while the last unit finishes
         for (int t = 0; ok && t < 2; ++t) {
           if (!u.tv[t]) continue;
@@ -341,11 +394,11 @@ __global__ void __launch_bounds__(kRope ? 352 : 320, 1)
       auto wait_k = [&](int i) {
         return wait_bar(bar(L::B_K + i % L::kKStages), (i / L::kKStages) & 1, ctx, 3);
       };
+      bool s0_early = false;   // this unit's first S on tile 0 went out during the last unit
       for (int ku = 0; ok; ++ku) {
-        const int unit = fwd_unit_index(sched, n_units, ku);
-        if (unit < 0) break;
-        const FwdUnit u = fwd_unit<kFront>(p, unit);
-        bool q_ready[2] = {false, false}, first_pv[2] = {true, true};
+        FwdUnit u;
+        if (!fwd_unit_k<kFront>(p, sched, n_units, recs, ku, u)) break;
+        bool q_ready[2] = {s0_early, false}, first_pv[2] = {true, true};
         // S_t(j) = Q_t K(j)^T into TMEM columns [128 t, 128 t + 128).
         auto issue_s = [&](int t, int kidx) -> bool {
           if (!q_ready[t]) {
@@ -364,15 +417,37 @@ __global__ void __launch_bounds__(kRope ? 352 : 320, 1)
         if (!wait_k(k0)) { ok = false; break; }
         for (int t = 0; ok && t < 2; ++t) {
           if (!u.part(t, u.kv_lo)) continue;
-          ok = issue_s(t, k0);
+          if (t != 0 || !s0_early) ok = issue_s(t, k0);
           if (ok && u.kv_lo == u.ke[t]) mma_commit(bar(L::B_QE + t));   // last S on Q_t
         }
+        s0_early = false;
         if (!ok) break;
         mma_commit(bar(L::B_KE + k0 % L::kKStages));
         for (int j = 0; ok && j < u.n_kv; ++j) {
           const int kt = u.kv_lo + j, vi = v0 + j, vst = vi % L::kVStages;
           const bool next = j + 1 < u.n_kv;
           bool v_ready = false, k_next_ready = false;
+          // Tile 1's last step has no tile-0 work: the next unit's first S on tile 0 goes out
+          // before it, so tile 0's softmax finds that S ready when its epilogue ends instead
+          // of one softmax pass later. Its key tile and query tile were loaded after this
+          // unit's S MMAs released their buffers, which all precede this step.
+          if (!next && !u.part(0, kt)) {
+            FwdUnit un;
+            if (fwd_unit_k<kFront>(p, sched, n_units, recs, ku + 1, un) && un.part(0, un.kv_lo)) {
+              const int kn = k0 + u.n_kv;
+              if (!wait_bar(bar((kRope ? L::B_QR : L::B_Q) + 0), q_used[0] & 1, ctx, 2) ||
+                  !wait_k(kn)) {
+                ok = false;
+                break;
+              }
+              ++q_used[0];
+              tc_fence_after();
+              gemm_ss_k<D>(tmem, sbase + L::kQ, sbase + L::kK + (kn % L::kKStages) * L::kTile,
+                           idesc_qk);
+              mma_commit(bar(L::B_S + 0));
+              s0_early = true;
+            }
+          }
           for (int t = 0; ok && t < 2; ++t) {
             if (u.part(t, kt)) {
               if (!wait_bar(bar(L::B_P + t), pcount[t] & 1, ctx, 4)) { ok = false; break; }
@@ -409,9 +484,8 @@ __global__ void __launch_bounds__(kRope ? 352 : 320, 1)
       int q_loads[2] = {0, 0};
       bool ok = true;
       for (int ku = 0; ok; ++ku) {
-        const int unit = fwd_unit_index(sched, n_units, ku);
-        if (unit < 0) break;
-        const FwdUnit u = fwd_unit<kFront>(p, unit);
+        FwdUnit u;
+        if (!fwd_unit_k<kFront>(p, sched, n_units, recs, ku, u)) break;
         for (int t = 0; t < 2; ++t) {
           if (!u.tv[t]) continue;
           if (!warp_wait(bar(L::B_Q + t), q_loads[t] & 1, ctx, 11)) { ok = false; break; }
@@ -435,9 +509,8 @@ __global__ void __launch_bounds__(kRope ? 352 : 320, 1)
     int s_cnt = 0, o_cnt = 0;
     bool ok = true;
     for (int ku = 0; ok; ++ku) {
-      const int unit = fwd_unit_index(sched, n_units, ku);
-      if (unit < 0) break;
-      const FwdUnit u = fwd_unit<kFront>(p, unit);
+      FwdUnit u;
+      if (!fwd_unit_k<kFront>(p, sched, n_units, recs, ku, u)) break;
       if (!u.tv[wg]) continue;
       const int r = u.qt[wg] * kTileRows + row;
       const bool row_valid = r < p.N;
@@ -504,14 +577,30 @@ __global__ void __launch_bounds__(kRope ? 352 : 320, 1)
       ++o_cnt;
       tc_fence_after();
       // Epilogue: O / l in bf16 through this warp's staging area (row `lane` of the warp at
-      // 128 bytes per 64 columns, 16-byte chunks XOR-swizzled by row), then stored four rows
-      // at a time: lane l writes chunk l % 8 of row 4 i + l / 8 — whole 128-byte segments
-      // instead of 16-byte pieces of 32 different rows.
+      // 128 bytes per 64 columns, 16-byte chunks XOR-swizzled by row: four 8-row atoms in the
+      // 128-byte-swizzled layout of an 8-row TMA box). An atom whose 8 rows are all in the
+      // sequence and land on 8 consecutive tokens goes out as one TMA box per 64 columns; the
+      // rows of other atoms (a run boundary of the roll inside the atom, or the end of the
+      // sequence) are stored by the warp, four whole 128-byte rows per instruction. Bulk stores
+      // keep the 32 KB of a tile off the SM's load/store path, which the next unit's barrier
+      // waits and shared-memory reads share (row stores held them up by ~2700 cycles).
       const float inv_l = 1.f / l_run;
       uint8_t* stage = smem + L::kStage + warp * L::kStageWarp;
+      const uint32_t stage_s = sbase + L::kStage + warp * L::kStageWarp;
       const int r_warp = u.qt[wg] * kTileRows + (warp % 4) * 32;
+      const HeadRemap hm = head_remap(p.N, p.G, u.shift_h, kFront ? u.front_h : 0);
+      const int tok_l = r_warp + lane < p.N ? hm.token(r_warp + lane) : -1;
+      const int tok_7 = __shfl_down_sync(0xffffffffu, tok_l, 7);
+      const unsigned boxed = __ballot_sync(
+          0xffffffffu, (lane & 7) == 0 && r_warp + lane + 7 < p.N && tok_7 - tok_l == 7);
+      int tok_atom[4];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) tok_atom[a] = __shfl_sync(0xffffffffu, tok_l, 8 * a);
 #pragma unroll 1
       for (int half = 0; half < D / 64; ++half) {
+        // the staging area is free once the TMA unit has read the boxes sent from it
+        if (lane == 0) bulk_wait_read_all();
+        __syncwarp();
 #pragma unroll
         for (int q2 = 0; q2 < 2; ++q2) {
           uint32_t ov[32];
@@ -527,17 +616,26 @@ __global__ void __launch_bounds__(kRope ? 352 : 320, 1)
             *reinterpret_cast<uint4*>(stage + lane * 128 + ((chunk ^ (lane & 7)) * 16)) = w4;
           }
         }
+        fence_async_smem();   // the TMA unit reads the staging area through the async proxy
         __syncwarp();
+        if (lane == 0) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int rr = 4 * i + (lane >> 3), chunk = lane & 7;
-          const uint4 w4 = *reinterpret_cast<const uint4*>(stage + rr * 128 + ((chunk ^ (rr & 7)) * 16));
-          const int rq = r_warp + rr;
-          if (rq < p.N) {
-            const int tok = head_remap(p.N, p.G, u.shift_h, kFront ? u.front_h : 0).token(rq);
-            __nv_bfloat16* dst = p.o + u.b * p.o_sb + tok * p.o_st + static_cast<long long>(u.h) * D +
-                                 64 * half + 8 * chunk;
-            *reinterpret_cast<uint4*>(dst) = w4;
+          for (int a = 0; a < 4; ++a)
+            if ((boxed >> (8 * a)) & 1u)
+              tma_store_4d(&tmO8, stage_s + a * 1024, 64 * half, u.h, tok_atom[a], u.b);
+          bulk_commit();
+        }
+        if (boxed != 0x01010101u) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int rr = 4 * i + (lane >> 3), chunk = lane & 7;
+            const int rq = r_warp + rr;
+            if (rq < p.N && !((boxed >> (rr & ~7)) & 1u)) {
+              const uint4 w4 = *reinterpret_cast<const uint4*>(stage + rr * 128 + ((chunk ^ (rr & 7)) * 16));
+              __nv_bfloat16* dst = p.o + u.b * p.o_sb + hm.token(rq) * p.o_st +
+                                   static_cast<long long>(u.h) * D + 64 * half + 8 * chunk;
+              *reinterpret_cast<uint4*>(dst) = w4;
+            }
           }
         }
         __syncwarp();
@@ -550,6 +648,9 @@ __global__ void __launch_bounds__(kRope ? 352 : 320, 1)
       // O_t is read: the next unit's first PV on it waits for this warpgroup's P anyway.
       tc_fence_before();
     }
+    // Every box has been written before the CTA's shared memory goes away.
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 
   // ---------------- teardown ----------------

@@ -314,6 +314,8 @@ s2attn_status launch_fwd(const Shape& sh, const void* q, const void* k, const vo
   if ((s = encode_pair(mq, q, sh.B, sh.Hq, sh.N, D, sh.sb[T_Q], sh.st[T_Q])) != S2ATTN_OK) return s;
   if ((s = encode_pair(mk, k, sh.B, sh.Hkv, sh.N, D, sh.sb[T_K], sh.st[T_K])) != S2ATTN_OK) return s;
   if ((s = encode_pair(mv, v, sh.B, sh.Hkv, sh.N, D, sh.sb[T_V], sh.st[T_V])) != S2ATTN_OK) return s;
+  CUtensorMap mo8;   // O, 8-row boxes: the epilogue's bulk stores
+  if ((s = encode_map(&mo8, o, sh.B, sh.Hq, sh.N, D, 8, sh.sb[T_O], sh.st[T_O])) != S2ATTN_OK) return s;
   s2::FwdParams p{};
   p.q = s2::TensorRef{static_cast<const __nv_bfloat16*>(q), sh.sb[T_Q], sh.st[T_Q]};
   p.k = s2::TensorRef{static_cast<const __nv_bfloat16*>(k), sh.sb[T_K], sh.st[T_K]};
@@ -340,16 +342,16 @@ s2attn_status launch_fwd(const Shape& sh, const void* q, const void* k, const vo
   constexpr int kT = s2::FwdLayout<D>::kThreads, kTR = s2::FwdLayout<D>::kRopeThreads;
   if (rope.q_rot && sh.front)
     s2::s2_fwd_kernel<D, true, true><<<grid, kTR, kSmem, stream>>>(mq.m128, mq.m8, mk.m128, mk.m8,
-                                                                   mv.m128, mv.m8, p, sched);
+                                                                   mv.m128, mv.m8, mo8, p, sched);
   else if (rope.q_rot)
     s2::s2_fwd_kernel<D, false, true><<<grid, kTR, kSmem, stream>>>(mq.m128, mq.m8, mk.m128, mk.m8,
-                                                                    mv.m128, mv.m8, p, sched);
+                                                                    mv.m128, mv.m8, mo8, p, sched);
   else if (sh.front)
     s2::s2_fwd_kernel<D, true, false><<<grid, kT, kSmem, stream>>>(mq.m128, mq.m8, mk.m128, mk.m8,
-                                                                   mv.m128, mv.m8, p, sched);
+                                                                   mv.m128, mv.m8, mo8, p, sched);
   else
     s2::s2_fwd_kernel<D, false, false><<<grid, kT, kSmem, stream>>>(mq.m128, mq.m8, mk.m128, mk.m8,
-                                                                    mv.m128, mv.m8, p, sched);
+                                                                    mv.m128, mv.m8, mo8, p, sched);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? S2ATTN_OK : cuda_fail(e, "s2_fwd_kernel launch");
 }
