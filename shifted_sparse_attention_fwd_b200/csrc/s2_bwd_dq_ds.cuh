@@ -17,8 +17,9 @@
 //
 // Warp roles (192 threads): warp 0 loader (dS tile by a plain bulk copy, K tile by TMA, a
 // 3-stage ring of 64 KB); warp 1 TMEM allocator and MMA issuer; warps 2-5 epilogue (warp w
-// reads TMEM lanes 32 (w mod 4) ...). TMEM: two dQ accumulators of D columns, so one query
-// tile's epilogue overlaps the next one's MMAs.
+// reads TMEM lanes 32 (w mod 4) ..., stages its 32 rows of bf16 dQ in shared memory and sends
+// them out as TMA boxes). TMEM: two dQ accumulators of D columns, so one query tile's
+// epilogue overlaps the next one's MMAs.
 #pragma once
 
 #include "s2_bwd_dkdv.cuh"
@@ -30,7 +31,11 @@ struct DqDsLayout {
   static constexpr uint32_t kKBytes = Tile<D>::kBytes;
   static constexpr int kStages = 3;
   static constexpr uint32_t kStageBytes = kDsTileBytes + kKBytes;
-  static constexpr uint32_t kRing = kStages * kStageBytes;   // claimed work units
+  // dQ staging of the epilogue warps: 32 rows x D columns of bf16 each, as D/64 column
+  // halves of four 8-row atoms in the 128-byte-swizzled layout of an 8-row TMA box.
+  static constexpr uint32_t kOut = kStages * kStageBytes;
+  static constexpr uint32_t kOutWarp = 32 * D * 2;
+  static constexpr uint32_t kRing = kOut + 4 * kOutWarp;   // claimed work units
   static constexpr uint32_t kBar = kRing + 4 * kUnitRing;
   enum { B_FULL = 0, B_EMPTY = kStages, B_ACC = 2 * kStages, B_ACCE = 2 * kStages + 2,
          B_DRAIN = 2 * kStages + 4, B_UF = 2 * kStages + 5, B_UE = B_UF + kUnitRing,
@@ -41,6 +46,7 @@ struct DqDsLayout {
   static constexpr uint32_t kLaunchBytes = kBytes + 1024;
   static constexpr int kThreads = 192;
   static constexpr uint32_t kTmemCols = 2 * D;
+  static_assert(kOut % 1024 == 0 && kLaunchBytes <= 227 * 1024, "shared memory of one CTA");
 };
 
 // Query tiles of this pass: (b, query head, rolled tile) for work index u, heaviest first.
@@ -55,7 +61,8 @@ __device__ __forceinline__ void dq_ds_tile(const BwdParams& p, int u, int& b, in
 template <int D, bool kFront>
 __global__ void __launch_bounds__(192, 1)
     s2_bwd_dq_ds_kernel(const __grid_constant__ CUtensorMap tmK,
-                        const __grid_constant__ CUtensorMap tmK8, const BwdParams p) {
+                        const __grid_constant__ CUtensorMap tmK8,
+                        const __grid_constant__ CUtensorMap tmDQ8, const BwdParams p) {
   using L = DqDsLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = aligned_smem(smem_raw);
@@ -92,6 +99,7 @@ __global__ void __launch_bounds__(192, 1)
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_map(&tmK);
+    tma_prefetch_map(&tmDQ8);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), L::kTmemCols);
@@ -178,8 +186,9 @@ __global__ void __launch_bounds__(192, 1)
   } else {
     // ---------------- epilogue warps 2-5 ----------------
     const int quad = warp % 4;
-    const int row = quad * 32 + lane;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+    uint8_t* stage = smem + L::kOut + quad * L::kOutWarp;
+    const uint32_t stage_s = sbase + L::kOut + quad * L::kOutWarp;
     int n = 0;
     for (int k = 0;; ++k, ++n) {
       int u;
@@ -190,11 +199,23 @@ __global__ void __launch_bounds__(192, 1)
       const int a = n & 1;
       if (!warp_wait(bar(L::B_ACC + a), (n >> 1) & 1, ctx, 4)) break;
       tc_fence_after();
-      const int r = qt * kTileRows + row;
-      const bool valid = r < p.N;
-      const int t = valid ? head_map(hq).token(r) : 0;
-      __nv_bfloat16* dst_row =
-          p.dq + b * p.dq_sb + t * p.dq_st + static_cast<long long>(hq) * D;
+      // dQ rows in bf16 through this warp's staging area; an 8-row atom whose rows are all in
+      // the sequence and land on 8 consecutive tokens goes out as one TMA box per 64 columns,
+      // the rows of other atoms (a run boundary of the roll inside the atom, or the end of the
+      // sequence) are stored by the warp. Bulk stores keep the 32 KB of a tile off the SM's
+      // load/store path, which the loader's barrier waits share.
+      const int r_warp = qt * kTileRows + quad * 32;
+      const HeadRemap hm = head_map(hq);
+      const int tok_l = r_warp + lane < p.N ? hm.token(r_warp + lane) : -1;
+      const int tok_7 = __shfl_down_sync(0xffffffffu, tok_l, 7);
+      const unsigned boxed = __ballot_sync(
+          0xffffffffu, (lane & 7) == 0 && r_warp + lane + 7 < p.N && tok_7 - tok_l == 7);
+      int tok_atom[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) tok_atom[i] = __shfl_sync(0xffffffffu, tok_l, 8 * i);
+      // the staging area is free once the TMA unit has read the last tile's boxes
+      if (lane == 0) bulk_wait_read_all();
+      __syncwarp();
 #pragma unroll
       for (int j = 0; j < D / 32; ++j) {
         uint32_t rr[32];
@@ -204,17 +225,47 @@ __global__ void __launch_bounds__(192, 1)
         for (int e = 0; e < 16; ++e)
           pk[e] = pack_bf16(__uint_as_float(rr[2 * e]) * p.scale,
                             __uint_as_float(rr[2 * e + 1]) * p.scale);
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(dst_row + 32 * j);
 #pragma unroll
-          for (int v = 0; v < 4; ++v)
-            dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        for (int v = 0; v < 4; ++v) {
+          const int chunk = (j % 2) * 4 + v;
+          *reinterpret_cast<uint4*>(stage + (j / 2) * 4096 + lane * 128 + ((chunk ^ (lane & 7)) * 16)) =
+              make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
         }
       }
       tc_fence_before();
+      fence_async_smem();   // the TMA unit reads the staging area through the async proxy
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(L::B_ACCE + a));
+      if (lane == 0) {
+        mbar_arrive(bar(L::B_ACCE + a));   // the accumulator is read: the MMA may reuse it
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h)
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            if ((boxed >> (8 * i)) & 1u)
+              tma_store_4d(&tmDQ8, stage_s + h * 4096 + i * 1024, 64 * h, hq, tok_atom[i], b);
+        bulk_commit();
+      }
+      if (boxed != 0x01010101u) {
+#pragma unroll 1
+        for (int h = 0; h < D / 64; ++h)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int rr = 4 * i + (lane >> 3), chunk = lane & 7;
+            const int rq = r_warp + rr;
+            if (rq < p.N && !((boxed >> (rr & ~7)) & 1u)) {
+              const uint4 w4 =
+                  *reinterpret_cast<const uint4*>(stage + h * 4096 + rr * 128 + ((chunk ^ (rr & 7)) * 16));
+              __nv_bfloat16* dst = p.dq + b * p.dq_sb + hm.token(rq) * p.dq_st +
+                                   static_cast<long long>(hq) * D + 64 * h + 8 * chunk;
+              *reinterpret_cast<uint4*>(dst) = w4;
+            }
+          }
+      }
+      __syncwarp();
     }
+    // Every box has been written before the CTA's shared memory goes away.
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 
   tc_fence_before();

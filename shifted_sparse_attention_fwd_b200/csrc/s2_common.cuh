@@ -129,6 +129,62 @@ __device__ __forceinline__ void produce_tile(uint32_t dst, const CUtensorMap* m1
   load_tile<D>(dst, m128, m8, bar, b, h, tr, N);
 }
 
+// The reverse of load_tile for one thread: TMA stores of a 128-row tile in shared memory (the
+// layout load_tile produces) to the rows `tr` gives, except the atoms in `skip`, which must
+// include every atom that straddles two runs or reaches past the end of the sequence
+// (straddled_atoms | past_end_atoms); committed as one bulk group.
+template <int D>
+__device__ __forceinline__ void store_tile(uint32_t src, const CUtensorMap* m128,
+                                           const CUtensorMap* m8, int b, int h, const Runs& tr,
+                                           uint32_t skip) {
+  if (tr.n == 1 && tr.len[0] == kTileRows && skip == 0) {
+#pragma unroll
+    for (int half = 0; half < Tile<D>::kHalves; ++half)
+      tma_store_4d(m128, src + half * Tile<D>::kHalfBytes, half * 64, h, tr.src[0], b);
+  } else {
+    for (int row = 0; row < kTileRows; row += 8) {
+      if ((skip >> (row >> 3)) & 1u) continue;
+      int dst = -1, base = 0;
+#pragma unroll
+      for (int k = 0; k < 3; ++k) {
+        if (k < tr.n && row >= base && row < base + tr.len[k]) dst = tr.src[k] + (row - base);
+        base += k < tr.n ? tr.len[k] : 0;
+      }
+      if (dst < 0) continue;
+#pragma unroll
+      for (int half = 0; half < Tile<D>::kHalves; ++half)
+        tma_store_4d(m8, src + half * Tile<D>::kHalfBytes + row * 128, half * 64, h, dst, b);
+    }
+  }
+  bulk_commit();
+}
+
+// The rows of the atoms in `skip` that are in the sequence, stored by a whole warp from a
+// 128-row tile in shared memory (load_tile's layout) to a contiguous [B, N, H, D] tensor.
+template <int D>
+__device__ __forceinline__ void store_atoms_warp(const uint8_t* tile, uint32_t skip,
+                                                 const Runs& tr, __nv_bfloat16* out, int N,
+                                                 int H, int b, int h) {
+  constexpr int kChunks = D / 8;   // 16-byte chunks per row
+  const int lane = threadIdx.x & 31;
+  for (uint32_t m = skip; m != 0; m &= m - 1) {
+    const int a = __ffs(m) - 1;
+    for (int i = lane; i < 8 * kChunks; i += 32) {
+      const int row = 8 * a + i / kChunks, c = i % kChunks;
+      int dst = -1, base = 0;
+#pragma unroll
+      for (int k = 0; k < 3; ++k) {
+        if (k < tr.n && row >= base && row < base + tr.len[k]) dst = tr.src[k] + (row - base);
+        base += k < tr.n ? tr.len[k] : 0;
+      }
+      if (dst < 0) continue;
+      const uint4 v = *reinterpret_cast<const uint4*>(
+          tile + (c / 8) * Tile<D>::kHalfBytes + row * 128 + (((c % 8) ^ (row & 7)) * 16));
+      *reinterpret_cast<uint4*>(out + ((static_cast<long long>(b) * N + dst) * H + h) * D + 8 * c) = v;
+    }
+  }
+}
+
 // Whole-tile GEMMs issued by the MMA thread. Operand descriptors are built once per call and
 // advanced by constant offsets: the tensor core's issue queue is only a few instructions
 // deep, so per-instruction scalar work in the issuing thread shows up as tensor-core idle time.

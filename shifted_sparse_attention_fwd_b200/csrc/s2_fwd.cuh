@@ -105,7 +105,7 @@ struct FwdLayout {
   static constexpr uint32_t kBar = kRecs + kLocalUnits * sizeof(FwdUnitRec);
   enum { B_Q = 0, B_QE = 2, B_K = 4, B_KE = B_K + kKStages, B_V = B_KE + kKStages,
          B_VE = B_V + kVStages, B_S = B_VE + kVStages, B_P = B_S + 2, B_ODONE = B_P + 2,
-         B_DRAIN = B_ODONE + 2, B_QR = B_DRAIN + 1, B_COUNT = B_QR + 2 };
+         B_DRAIN = B_ODONE + 2, B_QR = B_DRAIN + 1, B_QW = B_QR + 2, B_COUNT = B_QW + 2 };
   static constexpr uint32_t kTmemSlot = kBar + B_COUNT * 8;
   static constexpr uint32_t kAbort = kTmemSlot + 4;
   static constexpr uint32_t kBytes = kAbort + 4;
@@ -120,65 +120,70 @@ struct FwdLayout {
 
 // Fused RoPE with Position Interpolation of one 128-row query tile in shared memory (the
 // 128-byte-swizzled TMA layout), by one warp: the same rotation as s2_rope_kernel — the pair
-// (x[i], x[i + D/2]) of token t turns by (t * pi_scale) * base^(-2i/D) — written back in place
-// for the MMAs and to q_rot at the tile's original rows. Lane w of a row owns the 4-byte word of
-// columns 2w, 2w + 1 and its partner D/2 columns on. The angle of a run's first row is computed
-// as there (fp32 product, accurate sincosf); each following row of the run is reached by turning
-// by one token's angle (angle addition in fp32, relative drift about 1e-6 over a tile, far below
-// the bf16 rounding of the result).
+// (x[i], x[i + D/2]) of token t turns by (t * pi_scale) * base^(-2i/D) — written back in place,
+// for the MMAs and for the TMA stores of the rotated rows. A lane owns one 16-byte chunk of a
+// row's first half (8 columns) and its partner chunk D/2 columns on: D/16 lanes per row, 16-byte
+// shared-memory accesses. The angle of a run's first row is computed as there (fp32 product,
+// accurate sincosf); each following row of the run is reached by turning by the angle of the
+// rows in between (angle addition in fp32, relative drift about 1e-6 over a tile, far below the
+// bf16 rounding of the result).
 template <int D>
-__device__ __forceinline__ uint32_t swz_word(uint32_t tile, int row, int col) {
-  const int half = col / 64, cc = col % 64;
-  return tile + half * Tile<D>::kHalfBytes + row * 128 + ((((cc / 8) ^ (row & 7))) << 4) + (cc % 8) * 2;
+__device__ __forceinline__ uint32_t swz_chunk(uint32_t tile, int row, int col) {
+  const int half = col / 64, chunk = (col % 64) / 8;
+  return tile + half * Tile<D>::kHalfBytes + row * 128 + ((chunk ^ (row & 7)) << 4);
 }
 template <int D>
-__device__ __noinline__ void rope_query_tile(uint32_t tile, const Runs tr, __nv_bfloat16* q_rot,
-                                             int N, int Hq, float log2_base, float pi_scale,
-                                             int b, int h) {
-  constexpr int kLanesPerRow = D / 4;
+__device__ __noinline__ void rope_query_tile(uint32_t tile, const Runs tr, float log2_base,
+                                             float pi_scale) {
+  constexpr int kLanesPerRow = D / 16;
   constexpr int kRowsPerStep = 32 / kLanesPerRow;
   const int lane = threadIdx.x & 31;
-  const int w = lane % kLanesPerRow, r_off = lane / kLanesPerRow;
-  float th[2], cd[2], sd[2];
+  const int cl = lane % kLanesPerRow, r_off = lane / kLanesPerRow;
+  float th[8], cd[8], sd[8];
 #pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    th[k] = exp2f(-(2.0f * (2 * w + k) / D) * log2_base);
-    sincosf((kRowsPerStep * pi_scale) * th[k], &sd[k], &cd[k]);
+  for (int e = 0; e < 8; ++e) {
+    th[e] = exp2f(-(2.0f * (8 * cl + e) / D) * log2_base);
+    sincosf((kRowsPerStep * pi_scale) * th[e], &sd[e], &cd[e]);
   }
-  __nv_bfloat16* out = q_rot + static_cast<long long>(b) * N * Hq * D + static_cast<long long>(h) * D;
   int base = 0;
   for (int r = 0; r < tr.n; ++r) {
     const int len = tr.len[r], src = tr.src[r];
-    float c[2], sn[2];
+    float c[8], sn[8];
 #pragma unroll
-    for (int k = 0; k < 2; ++k)
-      sincosf((static_cast<float>(src + r_off) * pi_scale) * th[k], &sn[k], &c[k]);
+    for (int e = 0; e < 8; ++e)
+      sincosf((static_cast<float>(src + r_off) * pi_scale) * th[e], &sn[e], &c[e]);
     for (int i = r_off; i < len; i += kRowsPerStep) {
       const int row = base + i;
-      const uint32_t a_lo = swz_word<D>(tile, row, 2 * w), a_hi = swz_word<D>(tile, row, 2 * w + D / 2);
-      uint32_t lo, hi;
-      asm volatile("ld.shared.b32 %0, [%1];" : "=r"(lo) : "r"(a_lo));
-      asm volatile("ld.shared.b32 %0, [%1];" : "=r"(hi) : "r"(a_hi));
-      const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&lo));
-      const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hi));
-      __nv_bfloat162 nx = __floats2bfloat162_rn(x.x * c[0] - y.x * sn[0], x.y * c[1] - y.y * sn[1]);
-      __nv_bfloat162 ny = __floats2bfloat162_rn(y.x * c[0] + x.x * sn[0], y.y * c[1] + x.y * sn[1]);
-      const uint32_t nlo = *reinterpret_cast<uint32_t*>(&nx), nhi = *reinterpret_cast<uint32_t*>(&ny);
-      asm volatile("st.shared.b32 [%0], %1;" ::"r"(a_lo), "r"(nlo) : "memory");
-      asm volatile("st.shared.b32 [%0], %1;" ::"r"(a_hi), "r"(nhi) : "memory");
-      __nv_bfloat16* dst = out + static_cast<long long>(src + i) * Hq * D + 2 * w;
-      *reinterpret_cast<uint32_t*>(dst) = nlo;
-      *reinterpret_cast<uint32_t*>(dst + D / 2) = nhi;
+      const uint32_t a_lo = swz_chunk<D>(tile, row, 8 * cl);
+      const uint32_t a_hi = swz_chunk<D>(tile, row, 8 * cl + D / 2);
+      uint32_t x[4], y[4];
+      asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(x[0]), "=r"(x[1]), "=r"(x[2]), "=r"(x[3]) : "r"(a_lo));
+      asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(y[0]), "=r"(y[1]), "=r"(y[2]), "=r"(y[3]) : "r"(a_hi));
+      uint32_t nx[4], ny[4];
 #pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        const float cn = c[k] * cd[k] - sn[k] * sd[k];
-        sn[k] = sn[k] * cd[k] + c[k] * sd[k];
-        c[k] = cn;
+      for (int k = 0; k < 4; ++k) {
+        const float2 xf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&x[k]));
+        const float2 yf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&y[k]));
+        const int e0 = 2 * k, e1 = 2 * k + 1;
+        nx[k] = pack_bf16(xf.x * c[e0] - yf.x * sn[e0], xf.y * c[e1] - yf.y * sn[e1]);
+        ny[k] = pack_bf16(yf.x * c[e0] + xf.x * sn[e0], yf.y * c[e1] + xf.y * sn[e1]);
+      }
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a_lo), "r"(nx[0]), "r"(nx[1]),
+                   "r"(nx[2]), "r"(nx[3]) : "memory");
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a_hi), "r"(ny[0]), "r"(ny[1]),
+                   "r"(ny[2]), "r"(ny[3]) : "memory");
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float cn = c[e] * cd[e] - sn[e] * sd[e];
+        sn[e] = sn[e] * cd[e] + c[e] * sd[e];
+        c[e] = cn;
       }
     }
     base += len;
   }
-  fence_async_smem();   // the MMAs read the rotated tile through the async proxy
+  fence_async_smem();   // the MMAs and the TMA stores read the rotated tile (async proxy)
   __syncwarp();
 }
 
@@ -271,8 +276,9 @@ __global__ void __launch_bounds__(kRope ? 352 : 320, 1)
     s2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQ8,
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmK8,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmV8,
-                  const __grid_constant__ CUtensorMap tmO8, const FwdParams p,
-                  const __grid_constant__ FwdSchedule sched) {
+                  const __grid_constant__ CUtensorMap tmO8,
+                  const __grid_constant__ CUtensorMap tmQR, const __grid_constant__ CUtensorMap tmQR8,
+                  const FwdParams p, const __grid_constant__ FwdSchedule sched) {
   using L = FwdLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = aligned_smem(smem_raw);
@@ -295,6 +301,7 @@ __global__ void __launch_bounds__(kRope ? 352 : 320, 1)
       mbar_init(bar(L::B_P + s), 128);
       mbar_init(bar(L::B_ODONE + s), 1);
       mbar_init(bar(L::B_QR + s), 1);
+      mbar_init(bar(L::B_QW + s), 1);
     }
     for (int s = 0; s < L::kKStages; ++s) {
       mbar_init(bar(L::B_K + s), 1);
@@ -363,6 +370,11 @@ __global__ void __launch_bounds__(kRope ? 352 : 320, 1)
         for (int t = 0; ok && t < 2; ++t) {
           if (!u.tv[t]) continue;
           if (q_loads[t] > 0 && !wait_bar(bar(L::B_QE + t), (q_loads[t] - 1) & 1, ctx, 10)) {
+            ok = false;
+            break;
+          }
+          // (fused RoPE: and once the TMA unit has read the rotated rows out of the slot)
+          if (kRope && q_loads[t] > 0 && !wait_bar(bar(L::B_QW + t), (q_loads[t] - 1) & 1, ctx, 12)) {
             ok = false;
             break;
           }
@@ -490,13 +502,28 @@ __global__ void __launch_bounds__(kRope ? 352 : 320, 1)
           if (!u.tv[t]) continue;
           if (!warp_wait(bar(L::B_Q + t), q_loads[t] & 1, ctx, 11)) { ok = false; break; }
           ++q_loads[t];
-          rope_query_tile<D>(sbase + L::kQ + t * L::kTile,
-                             rolled_runs(head_remap(p.N, p.G, u.shift_h, kFront ? u.front_h : 0),
-                                         u.qt[t] * kTileRows),
-                             p.q_rot, p.N, p.Hq, p.rope_log2_base, p.rope_pi_scale, u.b, u.h);
-          if (lane == 0) mbar_arrive(bar(L::B_QR + t));
+          const Runs tr = rolled_runs(head_remap(p.N, p.G, u.shift_h, kFront ? u.front_h : 0),
+                                      u.qt[t] * kTileRows);
+          const uint32_t q_s = sbase + L::kQ + t * L::kTile;
+          rope_query_tile<D>(q_s, tr, p.rope_log2_base, p.rope_pi_scale);
+          // The rotated rows go to q_rot by TMA stores (whole atoms) and by this warp (atoms
+          // that straddle two runs or reach past the end); the slot is released for the next
+          // load once all of them have been read out.
+          const uint32_t plain = straddled_atoms(tr) | past_end_atoms(tr);
+          if (lane == 0) {
+            mbar_arrive(bar(L::B_QR + t));
+            store_tile<D>(q_s, &tmQR, &tmQR8, u.b, u.h, tr, plain);
+          }
+          store_atoms_warp<D>(smem + L::kQ + t * L::kTile, plain, tr, p.q_rot, p.N, p.Hq, u.b, u.h);
+          __syncwarp();
+          if (lane == 0) {
+            bulk_wait_read_all();
+            mbar_arrive(bar(L::B_QW + t));
+          }
         }
       }
+      if (lane == 0) bulk_wait_all();   // every rotated row written before the CTA exits
+      __syncwarp();
     }
   } else {
     // ---------------- softmax warpgroups ----------------

@@ -153,6 +153,10 @@ __host__ __device__ inline unsigned int straddled_atoms(const Runs& tr) {
   }
   return m;
 }
+// The atoms of a 128-row tile that hold a row past the end of the sequence (rows [valid, 128)).
+__host__ __device__ inline unsigned int past_end_atoms(const Runs& tr) {
+  return tr.valid >= 128 ? 0u : (0xFFFFu & ~((1u << (tr.valid >> 3)) - 1u));
+}
 
 // First rolled row of the group containing rolled row r, and one past its last row. With a
 // wrap split W < N (the pages' Variant 2, Table 8: in the shifted heads the tokens the roll

@@ -316,6 +316,11 @@ s2attn_status launch_fwd(const Shape& sh, const void* q, const void* k, const vo
   if ((s = encode_pair(mv, v, sh.B, sh.Hkv, sh.N, D, sh.sb[T_V], sh.st[T_V])) != S2ATTN_OK) return s;
   CUtensorMap mo8;   // O, 8-row boxes: the epilogue's bulk stores
   if ((s = encode_map(&mo8, o, sh.B, sh.Hq, sh.N, D, 8, sh.sb[T_O], sh.st[T_O])) != S2ATTN_OK) return s;
+  MapPair mqr = mq;   // the rotated queries (contiguous), stored by the fused RoPE
+  if (rope.q_rot) {
+    const long long st = static_cast<long long>(sh.Hq) * D;
+    if ((s = encode_pair(mqr, rope.q_rot, sh.B, sh.Hq, sh.N, D, st * sh.N, st)) != S2ATTN_OK) return s;
+  }
   s2::FwdParams p{};
   p.q = s2::TensorRef{static_cast<const __nv_bfloat16*>(q), sh.sb[T_Q], sh.st[T_Q]};
   p.k = s2::TensorRef{static_cast<const __nv_bfloat16*>(k), sh.sb[T_K], sh.st[T_K]};
@@ -342,16 +347,16 @@ s2attn_status launch_fwd(const Shape& sh, const void* q, const void* k, const vo
   constexpr int kT = s2::FwdLayout<D>::kThreads, kTR = s2::FwdLayout<D>::kRopeThreads;
   if (rope.q_rot && sh.front)
     s2::s2_fwd_kernel<D, true, true><<<grid, kTR, kSmem, stream>>>(mq.m128, mq.m8, mk.m128, mk.m8,
-                                                                   mv.m128, mv.m8, mo8, p, sched);
+                                                                   mv.m128, mv.m8, mo8, mqr.m128, mqr.m8, p, sched);
   else if (rope.q_rot)
     s2::s2_fwd_kernel<D, false, true><<<grid, kTR, kSmem, stream>>>(mq.m128, mq.m8, mk.m128, mk.m8,
-                                                                    mv.m128, mv.m8, mo8, p, sched);
+                                                                    mv.m128, mv.m8, mo8, mqr.m128, mqr.m8, p, sched);
   else if (sh.front)
     s2::s2_fwd_kernel<D, true, false><<<grid, kT, kSmem, stream>>>(mq.m128, mq.m8, mk.m128, mk.m8,
-                                                                   mv.m128, mv.m8, mo8, p, sched);
+                                                                   mv.m128, mv.m8, mo8, mqr.m128, mqr.m8, p, sched);
   else
     s2::s2_fwd_kernel<D, false, false><<<grid, kT, kSmem, stream>>>(mq.m128, mq.m8, mk.m128, mk.m8,
-                                                                    mv.m128, mv.m8, mo8, p, sched);
+                                                                    mv.m128, mv.m8, mo8, mqr.m128, mqr.m8, p, sched);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? S2ATTN_OK : cuda_fail(e, "s2_fwd_kernel launch");
 }
@@ -465,6 +470,9 @@ s2attn_status launch_dq_ds(const Shape& sh, const void* k, void* dq, float scale
   MapPair mk;
   s2attn_status s;
   if ((s = encode_pair(mk, k, sh.B, sh.Hkv, sh.N, D, sh.sb[T_K], sh.st[T_K])) != S2ATTN_OK) return s;
+  CUtensorMap mdq8;   // dQ, 8-row boxes: the epilogue's bulk stores
+  if ((s = encode_map(&mdq8, dq, sh.B, sh.Hq, sh.N, D, 8, sh.sb[T_DQ], sh.st[T_DQ])) != S2ATTN_OK)
+    return s;
   s2::BwdParams p = bwd_params(sh, scale, workspace, dq, nullptr, nullptr, err);
   set_ds_pass(p, sh, workspace, kvh_begin, kvh_count);
   p.sched = ws_sched(workspace, sh) + 2;
@@ -473,10 +481,10 @@ s2attn_status launch_dq_ds(const Shape& sh, const void* k, void* dq, float scale
   const unsigned grid = units < static_cast<unsigned>(num_sms) ? units : static_cast<unsigned>(num_sms);
   if (sh.front)
     s2::s2_bwd_dq_ds_kernel<D, true><<<grid, s2::DqDsLayout<D>::kThreads,
-                                       s2::DqDsLayout<D>::kLaunchBytes, stream>>>(mk.m128, mk.m8, p);
+                                       s2::DqDsLayout<D>::kLaunchBytes, stream>>>(mk.m128, mk.m8, mdq8, p);
   else
     s2::s2_bwd_dq_ds_kernel<D, false><<<grid, s2::DqDsLayout<D>::kThreads,
-                                        s2::DqDsLayout<D>::kLaunchBytes, stream>>>(mk.m128, mk.m8, p);
+                                        s2::DqDsLayout<D>::kLaunchBytes, stream>>>(mk.m128, mk.m8, mdq8, p);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? S2ATTN_OK : cuda_fail(e, "s2_bwd_dq_ds_kernel launch");
 }

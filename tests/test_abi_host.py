@@ -144,6 +144,8 @@ void rolled_runs(int r0, int shift, int N, int G, int front, int* o) {
   put_runs(s2::rolled_runs(s2::head_remap(N, G, shift, front), r0), o); }
 unsigned straddled(int r0, int shift, int N, int G, int front) {
   return s2::straddled_atoms(s2::rolled_runs(s2::head_remap(N, G, shift, front), r0)); }
+unsigned past_end(int r0, int shift, int N, int G, int front) {
+  return s2::past_end_atoms(s2::rolled_runs(s2::head_remap(N, G, shift, front), r0)); }
 void token_runs(int t0, int shift, int N, int G, int front, int* o) {
   put_runs(s2::token_runs(s2::head_remap(N, G, shift, front), t0), o); }
 int qtiles(int t0, int sh, int N, int G, int W, int front, int* o) {
@@ -276,6 +278,17 @@ def test_rolled_runs_match_the_oracle(shim, N, G, shift, variant):
             if len({run_of_row[r] for r in range(8 * a, min(8 * a + 8, valid))}) > 1:
                 want |= 1 << a
         assert shim.straddled(x0, shift, N, G, front) == want
+        # tile stores (rotated queries): an atom sent as one 8-row box must have its 8 rows in
+        # the sequence on 8 consecutive tokens; every atom reaching past the end, and every
+        # atom whose tokens are not consecutive, is left to row-by-row stores
+        past = shim.past_end(x0, shift, N, G, front)
+        skip = shim.straddled(x0, shift, N, G, front) | past
+        for a in range(16):
+            rows = list(range(x0 + 8 * a, x0 + 8 * a + 8))
+            boxable = rows[-1] < N and all(tok[r] == tok[rows[0]] + i for i, r in enumerate(rows))
+            assert bool((past >> a) & 1) == (rows[-1] >= N), (x0, a)
+            if not (skip >> a) & 1:
+                assert boxable, (x0, a)
 
 
 @pytest.mark.parametrize("N,G,shift,variant", VARIANT_CASES)

@@ -96,6 +96,7 @@ def test_rope_then_s2attn_forward_and_backward():
     (1, 8, 8, 2048, 512, 128, None, 0, 0.5),     # Llama-like heads, PI 4k -> 8k
     (2, 4, 2, 640, 128, 64, None, 0, 1.0),       # d = 64 (two rows per lane step), GQA, batch 2
     (1, 4, 2, 512, 128, 128, 37, 2, 0.25),       # a roll of 37 under Variant 3: tiles of 3 runs
+    (1, 4, 4, 300, 75, 64, None, 0, 0.5),        # odd G, roll 37, ragged end (rows past N)
 ])
 def test_fused_rope_q_forward(B, Hq, Hkv, N, G, d, shift, flags, pi):
     """s2attn_fwd_rope_q: the queries' RoPE-PI fused into the forward's query-tile path. The
