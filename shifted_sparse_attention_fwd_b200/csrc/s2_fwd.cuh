@@ -13,7 +13,7 @@
 // heaviest first within L2-sized groups), so one unit's epilogue and the next unit's loads
 // overlap the tensor-core work and the CTAs finish together.
 //
-// Warp roles (320 threads; 352 with the fused RoPE of the queries):
+// Warp roles (320 threads; 384 with the fused RoPE of the queries):
 //   warps 0-3, 4-7  softmax warpgroup of query tile 0 / 1: thread i owns query row i (TMEM
 //                   lane i); online softmax in fp32, P written back to TMEM as bf16 over S,
 //                   O rescaled in TMEM when the running max grows, epilogue.
@@ -105,7 +105,8 @@ struct FwdLayout {
   static constexpr uint32_t kBar = kRecs + kLocalUnits * sizeof(FwdUnitRec);
   enum { B_Q = 0, B_QE = 2, B_K = 4, B_KE = B_K + kKStages, B_V = B_KE + kKStages,
          B_VE = B_V + kVStages, B_S = B_VE + kVStages, B_P = B_S + 2, B_ODONE = B_P + 2,
-         B_DRAIN = B_ODONE + 2, B_QR = B_DRAIN + 1, B_QW = B_QR + 2, B_COUNT = B_QW + 2 };
+         B_DRAIN = B_ODONE + 2, B_QR = B_DRAIN + 1, B_QW = B_QR + 2, B_RR = B_QW + 2,
+         B_COUNT = B_RR + 2 };
   static constexpr uint32_t kTmemSlot = kBar + B_COUNT * 8;
   static constexpr uint32_t kAbort = kTmemSlot + 4;
   static constexpr uint32_t kBytes = kAbort + 4;
@@ -114,19 +115,21 @@ struct FwdLayout {
   static constexpr uint32_t kLaunchBytes =
       (kBytes + 1024 > 116 * 1024) ? kBytes + 1024 : 116 * 1024;
   static constexpr int kThreads = 320;
-  static constexpr int kRopeThreads = 352;   // + the rotation warp (warp 10) of the fused RoPE
+  static constexpr int kRopeThreads = 384;   // + the rotation warps (10, 11) of the fused RoPE
   static_assert(kLaunchBytes <= 227 * 1024, "shared memory of one CTA");
 };
 
 // Fused RoPE with Position Interpolation of one 128-row query tile in shared memory (the
-// 128-byte-swizzled TMA layout), by one warp: the same rotation as s2_rope_kernel — the pair
-// (x[i], x[i + D/2]) of token t turns by (t * pi_scale) * base^(-2i/D) — written back in place,
-// for the MMAs and for the TMA stores of the rotated rows. A lane owns one 16-byte chunk of a
-// row's first half (8 columns) and its partner chunk D/2 columns on: D/16 lanes per row, 16-byte
-// shared-memory accesses. The angle of a run's first row is computed as there (fp32 product,
-// accurate sincosf); each following row of the run is reached by turning by the angle of the
-// rows in between (angle addition in fp32, relative drift about 1e-6 over a tile, far below the
-// bf16 rounding of the result).
+// 128-byte-swizzled TMA layout), by the kRopeWarps rotation warps together (`part` = this
+// warp's index among them): the same rotation as s2_rope_kernel — the pair (x[i], x[i + D/2]) of
+// token t turns by (t * pi_scale) * base^(-2i/D) — written back in place, for the MMAs and for
+// the TMA stores of the rotated rows. A lane owns one 16-byte chunk of a row's first half (8
+// columns) and its partner chunk D/2 columns on: D/16 lanes per row, 16-byte shared-memory
+// accesses, packed f32x2 arithmetic on column pairs. The angle of a run's first row is computed
+// as there (fp32 product, accurate sincosf); each following row of the run is reached by turning
+// by the angle of the rows in between (angle addition in fp32, relative drift about 1e-6 over a
+// tile, far below the bf16 rounding of the result).
+constexpr int kRopeWarps = 2;
 template <int D>
 __device__ __forceinline__ uint32_t swz_chunk(uint32_t tile, int row, int col) {
   const int half = col / 64, chunk = (col % 64) / 8;
@@ -134,24 +137,38 @@ __device__ __forceinline__ uint32_t swz_chunk(uint32_t tile, int row, int col) {
 }
 template <int D>
 __device__ __noinline__ void rope_query_tile(uint32_t tile, const Runs tr, float log2_base,
-                                             float pi_scale) {
+                                             float pi_scale, int part) {
   constexpr int kLanesPerRow = D / 16;
-  constexpr int kRowsPerStep = 32 / kLanesPerRow;
+  constexpr int kRowsPerWarp = 32 / kLanesPerRow;
+  constexpr int kRowsPerStep = kRowsPerWarp * kRopeWarps;
   const int lane = threadIdx.x & 31;
-  const int cl = lane % kLanesPerRow, r_off = lane / kLanesPerRow;
-  float th[8], cd[8], sd[8];
+  const int cl = lane % kLanesPerRow, r_off = part * kRowsPerWarp + lane / kLanesPerRow;
+  // column pairs (8 cl + 2k, 8 cl + 2k + 1), k < 4, as packed fp32 pairs
+  float th[8];
+  uint64_t cd[4], sd[4], nsd[4];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    th[e] = exp2f(-(2.0f * (8 * cl + e) / D) * log2_base);
-    sincosf((kRowsPerStep * pi_scale) * th[e], &sd[e], &cd[e]);
+  for (int e = 0; e < 8; ++e) th[e] = exp2f(-(2.0f * (8 * cl + e) / D) * log2_base);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    float s0, c0, s1, c1;
+    sincosf((kRowsPerStep * pi_scale) * th[2 * k], &s0, &c0);
+    sincosf((kRowsPerStep * pi_scale) * th[2 * k + 1], &s1, &c1);
+    cd[k] = f2_pack(c0, c1);
+    sd[k] = f2_pack(s0, s1);
+    nsd[k] = f2_pack(-s0, -s1);
   }
   int base = 0;
   for (int r = 0; r < tr.n; ++r) {
     const int len = tr.len[r], src = tr.src[r];
-    float c[8], sn[8];
+    uint64_t c[4], sn[4];
 #pragma unroll
-    for (int e = 0; e < 8; ++e)
-      sincosf((static_cast<float>(src + r_off) * pi_scale) * th[e], &sn[e], &c[e]);
+    for (int k = 0; k < 4; ++k) {
+      float s0, c0, s1, c1;
+      sincosf((static_cast<float>(src + r_off) * pi_scale) * th[2 * k], &s0, &c0);
+      sincosf((static_cast<float>(src + r_off) * pi_scale) * th[2 * k + 1], &s1, &c1);
+      c[k] = f2_pack(c0, c1);
+      sn[k] = f2_pack(s0, s1);
+    }
     for (int i = r_off; i < len; i += kRowsPerStep) {
       const int row = base + i;
       const uint32_t a_lo = swz_chunk<D>(tile, row, 8 * cl);
@@ -164,21 +181,22 @@ __device__ __noinline__ void rope_query_tile(uint32_t tile, const Runs tr, float
       uint32_t nx[4], ny[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        const float2 xf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&x[k]));
-        const float2 yf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&y[k]));
-        const int e0 = 2 * k, e1 = 2 * k + 1;
-        nx[k] = pack_bf16(xf.x * c[e0] - yf.x * sn[e0], xf.y * c[e1] - yf.y * sn[e1]);
-        ny[k] = pack_bf16(yf.x * c[e0] + xf.x * sn[e0], yf.y * c[e1] + xf.y * sn[e1]);
+        const uint64_t xf = f2_from_bf16x2(x[k]), yf = f2_from_bf16x2(y[k]);
+        // x' = x c - y s, y' = y c + x s
+        const uint64_t xr = f2_fma(xf, c[k], f2_mul(yf, sn[k] ^ 0x8000000080000000ull));
+        const uint64_t yr = f2_fma(yf, c[k], f2_mul(xf, sn[k]));
+        nx[k] = pack_bf16(f2_lo(xr), f2_hi(xr));
+        ny[k] = pack_bf16(f2_lo(yr), f2_hi(yr));
       }
       asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a_lo), "r"(nx[0]), "r"(nx[1]),
                    "r"(nx[2]), "r"(nx[3]) : "memory");
       asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a_hi), "r"(ny[0]), "r"(ny[1]),
                    "r"(ny[2]), "r"(ny[3]) : "memory");
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float cn = c[e] * cd[e] - sn[e] * sd[e];
-        sn[e] = sn[e] * cd[e] + c[e] * sd[e];
-        c[e] = cn;
+      for (int k = 0; k < 4; ++k) {
+        const uint64_t cn = f2_fma(c[k], cd[k], f2_mul(sn[k], nsd[k]));
+        sn[k] = f2_fma(sn[k], cd[k], f2_mul(c[k], sd[k]));
+        c[k] = cn;
       }
     }
     base += len;
@@ -272,7 +290,7 @@ __device__ __forceinline__ bool fwd_unit_k(const FwdParams& p, const FwdSchedule
 }
 
 template <int D, bool kFront, bool kRope>
-__global__ void __launch_bounds__(kRope ? 352 : 320, 1)
+__global__ void __launch_bounds__(kRope ? 384 : 320, 1)
     s2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQ8,
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmK8,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmV8,
@@ -302,6 +320,7 @@ __global__ void __launch_bounds__(kRope ? 352 : 320, 1)
       mbar_init(bar(L::B_ODONE + s), 1);
       mbar_init(bar(L::B_QR + s), 1);
       mbar_init(bar(L::B_QW + s), 1);
+      mbar_init(bar(L::B_RR + s), kRopeWarps);
     }
     for (int s = 0; s < L::kKStages; ++s) {
       mbar_init(bar(L::B_K + s), 1);
@@ -441,17 +460,15 @@ __global__ void __launch_bounds__(kRope ? 352 : 320, 1)
           bool v_ready = false, k_next_ready = false;
           // Tile 1's last step has no tile-0 work: the next unit's first S on tile 0 goes out
           // before it, so tile 0's softmax finds that S ready when its epilogue ends instead
-          // of one softmax pass later. Its key tile and query tile were loaded after this
-          // unit's S MMAs released their buffers, which all precede this step.
+          // of one softmax pass later — if that unit's query tile (rotated, with the fused
+          // RoPE) and first key tile are already in place; this thread does not wait for them
+          // here, the unit's start issues the S otherwise.
           if (!next && !u.part(0, kt)) {
             FwdUnit un;
-            if (fwd_unit_k<kFront>(p, sched, n_units, recs, ku + 1, un) && un.part(0, un.kv_lo)) {
-              const int kn = k0 + u.n_kv;
-              if (!wait_bar(bar((kRope ? L::B_QR : L::B_Q) + 0), q_used[0] & 1, ctx, 2) ||
-                  !wait_k(kn)) {
-                ok = false;
-                break;
-              }
+            const int kn = k0 + u.n_kv;
+            if (fwd_unit_k<kFront>(p, sched, n_units, recs, ku + 1, un) && un.part(0, un.kv_lo) &&
+                mbar_test_wait(bar((kRope ? L::B_QR : L::B_Q) + 0), q_used[0] & 1) &&
+                mbar_test_wait(bar(L::B_K + kn % L::kKStages), (kn / L::kKStages) & 1)) {
               ++q_used[0];
               tc_fence_after();
               gemm_ss_k<D>(tmem, sbase + L::kQ, sbase + L::kK + (kn % L::kKStages) * L::kTile,
@@ -490,9 +507,14 @@ __global__ void __launch_bounds__(kRope ? 352 : 320, 1)
         v_used = v0 + u.n_kv;
       }
     }
-  } else if (warp == 10) {
-    // ---------------- rotation warp (fused RoPE of the queries) ----------------
+  } else if (warp >= 10) {
+    // ---------------- rotation warps (fused RoPE of the queries) ----------------
+    // Both rotate half of each query tile's rows as soon as it has landed; warp 10 then lets
+    // the MMAs at it, sends the rotated rows to q_rot (TMA stores for whole atoms, its own
+    // stores for atoms that straddle two runs or reach past the end) and releases the slot
+    // for the next load once they have been read out.
     if (kRope) {
+      const int part = warp - 10;
       int q_loads[2] = {0, 0};
       bool ok = true;
       for (int ku = 0; ok; ++ku) {
@@ -501,14 +523,14 @@ __global__ void __launch_bounds__(kRope ? 352 : 320, 1)
         for (int t = 0; t < 2; ++t) {
           if (!u.tv[t]) continue;
           if (!warp_wait(bar(L::B_Q + t), q_loads[t] & 1, ctx, 11)) { ok = false; break; }
-          ++q_loads[t];
+          const int k = q_loads[t]++;
           const Runs tr = rolled_runs(head_remap(p.N, p.G, u.shift_h, kFront ? u.front_h : 0),
                                       u.qt[t] * kTileRows);
           const uint32_t q_s = sbase + L::kQ + t * L::kTile;
-          rope_query_tile<D>(q_s, tr, p.rope_log2_base, p.rope_pi_scale);
-          // The rotated rows go to q_rot by TMA stores (whole atoms) and by this warp (atoms
-          // that straddle two runs or reach past the end); the slot is released for the next
-          // load once all of them have been read out.
+          rope_query_tile<D>(q_s, tr, p.rope_log2_base, p.rope_pi_scale, part);
+          if (lane == 0) mbar_arrive(bar(L::B_RR + t));
+          if (part != 0) continue;
+          if (!warp_wait(bar(L::B_RR + t), k & 1, ctx, 13)) { ok = false; break; }
           const uint32_t plain = straddled_atoms(tr) | past_end_atoms(tr);
           if (lane == 0) {
             mbar_arrive(bar(L::B_QR + t));
