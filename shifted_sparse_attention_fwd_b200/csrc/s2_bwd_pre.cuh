@@ -44,15 +44,29 @@ __global__ void __launch_bounds__(256) s2_bwd_pre_kernel(const __nv_bfloat16* __
   const int sub = lane / kLanesPerRow, li = lane % kLanesPerRow;
 
   constexpr int kUnroll = 4;                     // row pairs in flight per thread
-  for (int r0 = warp * kRowsPerWarp; r0 < rows; r0 += kUnroll * 8 * kRowsPerWarp) {
+  constexpr int kStride = 8 * kRowsPerWarp;      // rows between a thread's unrolled loads
+  // Row rr of the block is (token t0 + rr / Hq, head rr % Hq). Each thread's rows advance by
+  // fixed steps, so their (token, head) pairs are stepped instead of divided per load: the
+  // integer divisions had made this memory-bound kernel issue-bound.
+  int tk[kUnroll], hk[kUnroll];
+#pragma unroll
+  for (int k = 0; k < kUnroll; ++k) {
+    const int rr = warp * kRowsPerWarp + k * kStride + sub;
+    tk[k] = rr / Hq;
+    hk[k] = rr % Hq;
+  }
+  const int step_rows = kUnroll * kStride;       // rows from one iteration to the next
+  const int dt = step_rows / Hq, dh = step_rows % Hq;
+  const long long o_base = b * o_sb + t0 * o_st + li * 8, do_base = b * do_sb + t0 * do_st + li * 8;
+  for (int r0 = warp * kRowsPerWarp; r0 < rows; r0 += step_rows) {
     uint4 ov[kUnroll], gv[kUnroll];
 #pragma unroll
     for (int k = 0; k < kUnroll; ++k) {
-      const int rr = r0 + k * 8 * kRowsPerWarp + sub;
+      const int rr = r0 + k * kStride + sub;
       if (rr < rows) {
-        const long long t = t0 + rr / Hq, hd = static_cast<long long>(rr % Hq) * D + li * 8;
-        ov[k] = __ldg(reinterpret_cast<const uint4*>(o + b * o_sb + t * o_st + hd));
-        gv[k] = __ldg(reinterpret_cast<const uint4*>(dO + b * do_sb + t * do_st + hd));
+        const long long hd = static_cast<long long>(hk[k]) * D;
+        ov[k] = __ldg(reinterpret_cast<const uint4*>(o + o_base + tk[k] * o_st + hd));
+        gv[k] = __ldg(reinterpret_cast<const uint4*>(dO + do_base + tk[k] * do_st + hd));
       } else {
         ov[k] = make_uint4(0, 0, 0, 0);
         gv[k] = make_uint4(0, 0, 0, 0);
@@ -60,7 +74,7 @@ __global__ void __launch_bounds__(256) s2_bwd_pre_kernel(const __nv_bfloat16* __
     }
 #pragma unroll
     for (int k = 0; k < kUnroll; ++k) {
-      const int rr = r0 + k * 8 * kRowsPerWarp + sub;
+      const int rr = r0 + k * kStride + sub;
       const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&ov[k]);
       const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gv[k]);
       float acc = 0.f;
@@ -74,10 +88,16 @@ __global__ void __launch_bounds__(256) s2_bwd_pre_kernel(const __nv_bfloat16* __
 #pragma unroll
       for (int sh = kLanesPerRow / 2; sh > 0; sh >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, sh);
       if (li == 0 && rr < rows) {
-        const int h = rr % Hq, t = t0 + rr / Hq;
-        const size_t idx = (static_cast<size_t>(b) * Hq + h) * N + t;
+        const size_t idx = (static_cast<size_t>(b) * Hq + hk[k]) * N + t0 + tk[k];
         dvec[idx] = acc;
         lse2[idx] = lse[idx] * 1.4426950408889634f;
+      }
+      // this thread's next row of slot k
+      tk[k] += dt;
+      hk[k] += dh;
+      if (hk[k] >= Hq) {
+        hk[k] -= Hq;
+        ++tk[k];
       }
     }
   }
