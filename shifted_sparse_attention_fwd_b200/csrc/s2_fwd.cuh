@@ -8,10 +8,11 @@
 // moves data: TMA reads the original rows (s2_tiles.cuh) and the epilogue stores O and LSE at
 // the original rows.
 //
-// The kernel is persistent: one CTA per SM sets up its barriers and TMEM once and takes the
-// work units a host-side longest-first schedule gives it (FwdSchedule; units are numbered
-// heaviest first within L2-sized groups), so one unit's epilogue and the next unit's loads
-// overlap the tensor-core work and the CTAs finish together.
+// The kernel is persistent: one CTA per SM sets up its barriers and TMEM once, decodes its
+// first units into a shared-memory table and takes the work units a host-side schedule gives it
+// (FwdSchedule: least-loaded-CTA assignment in the L2-grouped unit order, the last units
+// heaviest first), so one unit's epilogue and the next unit's loads overlap the tensor-core
+// work and the CTAs finish together.
 //
 // Warp roles (320 threads; 384 with the fused RoPE of the queries):
 //   warps 0-3, 4-7  softmax warpgroup of query tile 0 / 1: thread i owns query row i (TMEM
@@ -21,17 +22,19 @@
 //                   V tiles (2-slot rings); each ring slot is released by a commit right
 //                   after the last MMA that reads it.
 //   warp 9          TMEM allocator and MMA issuer (one lane).
-//   warp 10         (fused RoPE only) rotates each query tile in shared memory once it has
-//                   landed and writes the rotated rows out; the MMAs wait for it.
+//   warps 10, 11    (fused RoPE only) rotate each query tile in shared memory once it has
+//                   landed and send the rotated rows out; the MMAs wait for the rotation.
 // TMEM columns: S0/P0 [0,128), S1/P1 [128,256), O0 [256,256+D), O1 [256+D, 256+2D).
 //
 // MMA issue order S0(0) S1(0) PV0(0) S0(1) PV1(0) S1(1) PV0(1) ... lets each warpgroup's
 // softmax run while the tensor core works on the other tile. tcgen05 MMAs from one thread
 // complete in issue order, so when S_t(j+1) is signalled, PV_t(j) — which read P_t(j) from
 // the same columns and accumulated into O_t — is complete: the softmax may rescale O_t at once.
+// Tile 1 of a unit has one more key tile than tile 0, so the next unit's first S on tile 0 is
+// issued before tile 1's last step when its tiles are already in place.
 //
 // The epilogue stages each warp's 32 rows of O (64 columns at a time) in shared memory and
-// writes whole 128-byte row segments, four rows per store instruction.
+// sends them out as 8-row TMA boxes (row stores only where the roll splits an 8-row atom).
 #pragma once
 
 #include "s2_common.cuh"
@@ -135,28 +138,42 @@ __device__ __forceinline__ uint32_t swz_chunk(uint32_t tile, int row, int col) {
   const int half = col / 64, chunk = (col % 64) / 8;
   return tile + half * Tile<D>::kHalfBytes + row * 128 + ((chunk ^ (row & 7)) << 4);
 }
+// A lane's frequencies and the turn of one row step, the same for every tile: worked out once.
+struct RopeLane {
+  float th[8];                  // base^(-2i/D) of the lane's 8 columns
+  uint64_t cd[4], sd[4], nsd[4];   // cos, sin and -sin of one step's angle, column pairs packed
+};
 template <int D>
-__device__ __noinline__ void rope_query_tile(uint32_t tile, const Runs tr, float log2_base,
-                                             float pi_scale, int part) {
+__device__ __forceinline__ RopeLane rope_lane(float log2_base, float pi_scale) {
+  constexpr int kLanesPerRow = D / 16;
+  constexpr int kRowsPerStep = (32 / kLanesPerRow) * kRopeWarps;
+  const int cl = (threadIdx.x & 31) % kLanesPerRow;
+  RopeLane rl;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) rl.th[e] = exp2f(-(2.0f * (8 * cl + e) / D) * log2_base);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    float s0, c0, s1, c1;
+    sincosf((kRowsPerStep * pi_scale) * rl.th[2 * k], &s0, &c0);
+    sincosf((kRowsPerStep * pi_scale) * rl.th[2 * k + 1], &s1, &c1);
+    rl.cd[k] = f2_pack(c0, c1);
+    rl.sd[k] = f2_pack(s0, s1);
+    rl.nsd[k] = f2_pack(-s0, -s1);
+  }
+  return rl;
+}
+template <int D>
+__device__ __forceinline__ void rope_query_tile(uint32_t tile, const Runs& tr, const RopeLane& rl,
+                                                float pi_scale, int part) {
   constexpr int kLanesPerRow = D / 16;
   constexpr int kRowsPerWarp = 32 / kLanesPerRow;
   constexpr int kRowsPerStep = kRowsPerWarp * kRopeWarps;
   const int lane = threadIdx.x & 31;
   const int cl = lane % kLanesPerRow, r_off = part * kRowsPerWarp + lane / kLanesPerRow;
-  // column pairs (8 cl + 2k, 8 cl + 2k + 1), k < 4, as packed fp32 pairs
-  float th[8];
-  uint64_t cd[4], sd[4], nsd[4];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) th[e] = exp2f(-(2.0f * (8 * cl + e) / D) * log2_base);
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    float s0, c0, s1, c1;
-    sincosf((kRowsPerStep * pi_scale) * th[2 * k], &s0, &c0);
-    sincosf((kRowsPerStep * pi_scale) * th[2 * k + 1], &s1, &c1);
-    cd[k] = f2_pack(c0, c1);
-    sd[k] = f2_pack(s0, s1);
-    nsd[k] = f2_pack(-s0, -s1);
-  }
+  const float* th = rl.th;
+  const uint64_t* cd = rl.cd;
+  const uint64_t* sd = rl.sd;
+  const uint64_t* nsd = rl.nsd;
   int base = 0;
   for (int r = 0; r < tr.n; ++r) {
     const int len = tr.len[r], src = tr.src[r];
@@ -515,6 +532,7 @@ __global__ void __launch_bounds__(kRope ? 384 : 320, 1)
     // for the next load once they have been read out.
     if (kRope) {
       const int part = warp - 10;
+      const RopeLane rl = rope_lane<D>(p.rope_log2_base, p.rope_pi_scale);
       int q_loads[2] = {0, 0};
       bool ok = true;
       for (int ku = 0; ok; ++ku) {
@@ -527,7 +545,7 @@ __global__ void __launch_bounds__(kRope ? 384 : 320, 1)
           const Runs tr = rolled_runs(head_remap(p.N, p.G, u.shift_h, kFront ? u.front_h : 0),
                                       u.qt[t] * kTileRows);
           const uint32_t q_s = sbase + L::kQ + t * L::kTile;
-          rope_query_tile<D>(q_s, tr, p.rope_log2_base, p.rope_pi_scale, part);
+          rope_query_tile<D>(q_s, tr, rl, p.rope_pi_scale, part);
           if (lane == 0) mbar_arrive(bar(L::B_RR + t));
           if (part != 0) continue;
           if (!warp_wait(bar(L::B_RR + t), k & 1, ctx, 13)) { ok = false; break; }
