@@ -132,6 +132,10 @@ class ClockSampler:
 
     def __enter__(self):
         if self.nv is not None:
+            # the timed loop holds the interpreter lock between launches: switch threads often
+            # enough that the sampler runs several times even in a ~15 ms timed region
+            self._switch = sys.getswitchinterval()
+            sys.setswitchinterval(1e-4)
             self._thread = threading.Thread(target=self._run, daemon=True)
             self._thread.start()
         return self
@@ -140,6 +144,7 @@ class ClockSampler:
         self._stop.set()
         if self._thread is not None:
             self._thread.join()
+            sys.setswitchinterval(self._switch)
 
     def summary(self):
         if self.nv is None:
