@@ -118,16 +118,27 @@ class ClockSampler:
         except Exception as e:  # no NVML: report that, never guess
             self.nv, self.err = None, str(e)
 
+    def sample(self):
+        try:
+            self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+            mask = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            for bit, name in REASON_BITS.items():
+                if mask & bit:
+                    self.reasons.add(name)
+        except Exception:
+            pass
+
     def _run(self):
         while not self._stop.is_set():
-            try:
-                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
-                mask = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                for bit, name in REASON_BITS.items():
-                    if mask & bit:
-                        self.reasons.add(name)
-            except Exception:
-                pass
+            self.sample()
+            time.sleep(self.period)
+
+    def wait(self, event):
+        """Sample from the calling thread until `event` has completed: the host enqueues the
+        timed steps long before the GPU finishes them, so this covers the rest of the region."""
+        while not event.query():
+            if self.nv is not None:
+                self.sample()
             time.sleep(self.period)
 
     def __enter__(self):
@@ -151,7 +162,8 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": self.err}
         med = statistics.median(self.samples) if self.samples else None
         return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons - {"gpu_idle"}),
-                "samples": len(self.samples)}
+                "samples": len(self.samples),
+                "sm_mhz_range": [min(self.samples), max(self.samples)] if self.samples else None}
 
 
 # ------------------------------------------------------------------------------------------
@@ -270,6 +282,7 @@ def run_gpu(args, rank, world, local_rank):
         for i in range(args.steps):
             flush.fill_(i & 0xFF)
             step(evs[i])
+        sampler.wait(evs[-1][nev - 1])
         torch.cuda.synchronize()
     if dist: dist.barrier()
     st, code = s2.s2attn_get_device_error()
