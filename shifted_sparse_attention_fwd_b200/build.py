@@ -25,7 +25,7 @@ def nvcc_path() -> str:
 
 def sources():
     csrc = os.path.join(PKG_DIR, "csrc")
-    out = [os.path.join(csrc, f) for f in sorted(os.listdir(csrc)) if f.endswith((".cu", ".cuh"))]
+    out = [os.path.join(csrc, f) for f in sorted(os.listdir(csrc)) if f.endswith((".cu", ".cuh", ".h"))]
     return out + [os.path.join(ROOT, "include", "s2attn.h")]
 
 

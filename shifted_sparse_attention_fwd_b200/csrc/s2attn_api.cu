@@ -6,8 +6,6 @@
 #include <algorithm>
 #include <atomic>
 #include <cmath>
-#include <functional>
-#include <queue>
 #include <utility>
 #include <vector>
 #include <cstdint>
@@ -22,6 +20,7 @@
 #include "s2_bwd_pre.cuh"
 #include "s2_rope.cuh"
 #include "s2_fwd.cuh"
+#include "s2_fwd_sched.h"
 
 namespace {
 
@@ -238,52 +237,16 @@ s2attn_status check_shape(int B, int Hq, int Hkv, int N, int d, int G, float sca
   return S2ATTN_OK;
 }
 
-// The forward's per-CTA unit lists (s2::FwdSchedule): each unit goes to the CTA with the least
-// work so far, by a cost of (query tile, key tile) steps plus 3 for the unit's own loads,
-// epilogue and boundary (per-role traces of the kernel put a unit's fixed cost at about 3.25
-// steps). The units are handed out in the kernel's L2-grouped order, which keeps the CTAs moving
-// through the heads and groups together, except the last 2 x grid, which go heaviest first
-// (longest-processing-time-first) so they even out what the earlier ones left: on the Llama2-7B
-// layer the busiest CTA ends 3 % above the mean instead of 11 % (all units heaviest first: 2.6 %,
-// but the lost L2 grouping costs more than that at B = 4). Each CTA takes its units in index
-// order. Round robin (count = 0) when the lists would not fit the launch.
+// The forward's per-CTA unit lists (s2::FwdSchedule), built by s2::fwd_unit_lists; round robin
+// (count = 0) when the lists would not fit the launch.
 void fwd_schedule(const Shape& sh, int grid, s2::FwdSchedule& out) {
   out.count = 0;
-  const int nqt = (sh.N + s2::kTileRows - 1) / s2::kTileRows;
   const long long n_units = static_cast<long long>(sh.B) * sh.Hq * s2::query_pairs_per_head(sh.N);
-  if (n_units > s2::kFwdSchedMaxUnits || grid > s2::kFwdSchedMaxCtas || n_units <= grid) return;
-  std::vector<double> cost(n_units);
-  for (int u = 0; u < n_units; ++u) {
-    int b, h, pair;
-    s2::query_pair_coords_chunked(u, sh.B, sh.Hq, sh.N, sh.G, s2::kL2Chunk, b, h, pair);
-    const int wrap_h = h >= sh.shb ? sh.wrap : s2::kNoWrapSplit;
-    double c = 3.0;
-    for (int t = 0; t < 2; ++t) {
-      const int qt = 2 * pair + t;
-      if (qt < nqt) c += qt - s2::group_begin(qt * s2::kTileRows, sh.G, wrap_h) / s2::kTileRows + 1;
-    }
-    cost[u] = c;
-  }
-  std::vector<int> order(n_units);
-  for (int u = 0; u < n_units; ++u) order[u] = u;
-  const long long tail = std::min<long long>(n_units, 2ll * grid);
-  std::stable_sort(order.begin() + (n_units - tail), order.end(),
-                   [&](int a, int b) { return cost[a] > cost[b]; });
-  std::priority_queue<std::pair<double, int>, std::vector<std::pair<double, int>>,
-                      std::greater<std::pair<double, int>>> load;
-  for (int c = 0; c < grid; ++c) load.push({0.0, c});
-  std::vector<int> owner(n_units), count(grid, 0);
-  for (const int u : order) {
-    const auto least = load.top();
-    load.pop();
-    owner[u] = least.second;
-    ++count[least.second];
-    load.push({least.first + cost[u], least.second});
-  }
-  out.start[0] = 0;
-  for (int c = 0; c < grid; ++c) out.start[c + 1] = static_cast<unsigned short>(out.start[c] + count[c]);
-  std::vector<int> fill(out.start, out.start + grid);
-  for (int u = 0; u < n_units; ++u) out.unit[fill[owner[u]]++] = static_cast<unsigned short>(u);
+  if (n_units > s2::kFwdSchedMaxUnits || grid > s2::kFwdSchedMaxCtas) return;
+  std::vector<int> start, unit;
+  if (!s2::fwd_unit_lists(sh.B, sh.Hq, sh.N, sh.G, sh.shb, sh.wrap, grid, start, unit)) return;
+  for (int c = 0; c <= grid; ++c) out.start[c] = static_cast<unsigned short>(start[c]);
+  for (size_t i = 0; i < unit.size(); ++i) out.unit[i] = static_cast<unsigned short>(unit[i]);
   out.count = static_cast<int>(n_units);
 }
 

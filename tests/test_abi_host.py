@@ -136,7 +136,14 @@ def test_any_group_and_roll_accepted(lib, B, Hq, Hkv, N, d, G, shb, shift, flags
 # --------------------------------------------------------------------------------------
 SHIM = r"""
 #include "s2_tiles.cuh"
+#include "s2_fwd_sched.h"
 extern "C" {
+int fwdlists(int B, int Hq, int N, int G, int shb, int wrap, int grid, int* start, int* unit) {
+  std::vector<int> s, u;
+  if (!s2::fwd_unit_lists(B, Hq, N, G, shb, wrap, grid, s, u)) return -1;
+  std::copy(s.begin(), s.end(), start);
+  std::copy(u.begin(), u.end(), unit);
+  return static_cast<int>(u.size()); }
 static void put_runs(const s2::Runs& t, int* o) {
   o[0] = t.n; o[1] = t.valid;
   for (int k = 0; k < t.n; ++k) { o[2 + 2 * k] = t.len[k]; o[3 + 2 * k] = t.src[k]; } }
@@ -508,6 +515,57 @@ def test_chunked_pair_order_is_a_permutation(shim, B, Hq, N, G, chunk):
     order = [tuple(call4(shim.paircoords_chunked, bid, B, Hq, N, G, chunk)[:3])
              for bid in range(B * Hq * npair)]
     assert set(order) == {(b, h, q) for b in range(B) for h in range(Hq) for q in range(npair)}
+
+
+def fwd_lists(shim, B, Hq, N, G, shb, grid):
+    npair = ((N + 127) // 128 + 1) // 2
+    start = (ctypes.c_int * (grid + 1))()
+    unit = (ctypes.c_int * (B * Hq * npair))()
+    n = shim.fwdlists(B, Hq, N, G, shb, NOWRAP, grid, start, unit)
+    return n, list(start), list(unit)
+
+
+def pair_cost(shim, u, B, Hq, N, G):
+    """The schedule's cost model restated: 3 per unit plus, for each of the pair's query tiles,
+    the key tiles it visits (its own and the earlier ones of its group; no wrap split)."""
+    _, _, pair = call4(shim.paircoords_chunked, u, B, Hq, N, G, 10)[:3]
+    nqt = (N + 127) // 128
+    c = 3
+    for qt in (2 * pair, 2 * pair + 1):
+        if qt < nqt:
+            c += qt - (qt * 128 // G) * G // 128 + 1
+    return c
+
+
+@pytest.mark.parametrize("B,Hq,N,G,shb,grid", [(1, 32, 8192, 2048, 16, 148),
+                                               (4, 32, 8192, 2048, 16, 148),
+                                               (1, 32, 8192, 1365, 16, 148),
+                                               (1, 4, 2048, 512, 2, 17),
+                                               (2, 3, 1000, 333, 1, 5),
+                                               (1, 8, 4096, 4096, 8, 64)])
+def test_fwd_schedule_lists(shim, B, Hq, N, G, shb, grid):
+    """The forward's per-CTA unit lists: every unit exactly once, each CTA's list ascending, and
+    the greedy bound of list scheduling — each unit went to the least-loaded CTA, so no CTA ends
+    more than one unit's cost above the mean."""
+    n, start, unit = fwd_lists(shim, B, Hq, N, G, shb, grid)
+    npair = ((N + 127) // 128 + 1) // 2
+    assert n == B * Hq * npair
+    assert start[0] == 0 and start[-1] == n and all(a <= b for a, b in zip(start, start[1:]))
+    assert sorted(unit) == list(range(n))
+    cost = [pair_cost(shim, u, B, Hq, N, G) for u in range(n)]
+    loads = []
+    for c in range(grid):
+        mine = unit[start[c]:start[c + 1]]
+        assert mine == sorted(mine)
+        loads.append(sum(cost[u] for u in mine))
+    mean = sum(cost) / grid
+    assert max(loads) <= mean + max(cost)
+    if (B, Hq, N, G, grid) == (1, 32, 8192, 2048, 148):
+        assert max(loads) <= 1.04 * mean      # the busiest CTA about 3 % above the mean
+
+
+def test_fwd_schedule_round_robin_when_units_do_not_outnumber_ctas(shim):
+    assert fwd_lists(shim, 1, 2, 512, 128, 1, 148)[0] == -1    # 4 units, 148 CTAs
 
 
 @pytest.mark.parametrize("B,Hq,Hkv,N,G,shb,sh,chunk", [(1, 32, 32, 8192, 2048, 16, 1024, 10),
