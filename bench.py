@@ -138,8 +138,9 @@ class ClockSampler:
         timed steps long before the GPU finishes them, so this covers the rest of the region."""
         while not event.query():
             if self.nv is not None:
-                self.sample()
-            time.sleep(self.period)
+                self.sample()              # paced by the NVML calls themselves
+            else:
+                time.sleep(self.period)
 
     def __enter__(self):
         if self.nv is not None:
